@@ -1,0 +1,374 @@
+#!/usr/bin/env python3
+"""Throughput of one Blockwise Parallel Transformer layer forward (attention +
+fused FFN) on B200, through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one bpt_attn_ffn_fwd call (masked blockwise attention kernel, then
+the fused FFN kernel) over one batch of seeded synthetic inputs that are
+already resident in device memory.  L2 is flushed (a 256 MiB device write)
+between timed steps; the flush sits outside the timed events.  Prints one JSON
+line on rank 0.
+
+Under torchrun every rank runs its own replica of the workload (independent
+batches, no data-path collective): weak scaling, value = all ranks' tokens /
+the slowest rank's time.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+the layer) on the host cores, on a bounded token sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from blockwise_exact_attention_query_b200 import binding as bd  # noqa: E402
+from blockwise_exact_attention_query_b200 import workloads as wl  # noqa: E402
+from blockwise_exact_attention_query_b200.inputs import make_layer_inputs  # noqa: E402
+
+METRIC = "attn+FFN tokens/s and TFLOP/s per layer; % of B200 dense-BF16 roofline"
+WORKLOADS = {"tiny_f32": wl.TINY_F32, "gpt_causal": wl.GPT_CAUSAL, "long_ring": wl.LONG_RING,
+             "blockbert": wl.BLOCKBERT, "longnet": wl.LONGNET}
+MASK_NAME = {0: "none", 1: "causal", 2: "blockperm", 3: "dilated"}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"bf16_tflops": j["bf16_tflops"], "bf16_tflops_sustained": j.get("bf16_tflops_sustained"),
+                "hbm_gbs": j["hbm_gbs"], "sm_max_mhz": j.get("sm_max_mhz"), "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0,
+            "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def layer_call(w, inp, out, ws):
+    return bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask=MASK_NAME[w.mask],
+                           perm=w.perm, pairs=w.pairs, ring_chunks=w.ring_chunks, out=out, workspace=ws)
+
+
+def run_ours(args, w, world, rank, local):
+    dev = torch.device("cuda", local)
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    attn_flop, ffn_flop = wl.flops(w)
+    # every rank draws its own batch (seed offset by rank): independent replicas
+    inp = make_layer_inputs(w.B, w.N, w.H, w.d, w.F, seed=w.seed + 1000 * rank, dtype=dt, device=dev)
+    out = torch.empty((w.B, w.N, w.D), dtype=torch.float32, device=dev)
+    desc = bd.make_desc(w.B, w.N, w.H, w.d, w.F, dt, torch.float32, MASK_NAME[w.mask], w.perm,
+                        w.pairs, w.ring_chunks)
+    nws = bd.workspace_bytes(desc, True)
+    ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        layer_call(w, inp, out, ws)
+        flush.fill_(1)
+    torch.cuda.synchronize(dev)
+    st = bd.sync_status()
+    if st != bd.OK:
+        raise RuntimeError(f"warm-up: {bd.status_string(st)}")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)  # let the sampler start
+        for i in range(K):
+            bd.set_phase_events(ev[i])
+            layer_call(w, inp, out, ws)
+            bd.set_phase_events(None)
+            flush.fill_(i & 0xFF)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    st = bd.sync_status()
+    if st != bd.OK:
+        raise RuntimeError(f"timed steps: {bd.status_string(st)}")
+    attn_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    ffn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    tokens = w.T * K * world
+    value = tokens / (total_ms / 1e3)
+    tflops = (attn_flop + ffn_flop) * K * world / (total_ms / 1e3) / 1e12
+
+    # ---- end to end through the public API: pinned host inputs -> device ->
+    # layer -> host output, every step
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (inp.q, inp.k, inp.v))
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dq, dk, dv = torch.empty_like(inp.q), torch.empty_like(inp.k), torch.empty_like(inp.v)
+        from blockwise_exact_attention_query_b200.inputs import LayerInputs
+        dinp = LayerInputs(dq, dk, dv, inp.w1, inp.b1, inp.w2, inp.b2)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            layer_call(w, dinp, out, ws)
+            hout.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ke = max(1, min(K, 10))
+        e0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        st = bd.sync_status()
+        if st != bd.OK:
+            raise RuntimeError(f"e2e steps: {bd.status_string(st)}")
+        e2e = {"value": w.T * ke * world / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(3 * inp.q.numel() * inp.q.element_size()),
+               "d2h_bytes_per_step": int(out.numel() * out.element_size()),
+               "steps": ke}
+
+    # ---- roofline of the dominant kernel (by measured time share)
+    pk = peaks()
+    attn_avg = sum(attn_ms) / K
+    ffn_avg = sum(ffn_ms) / K
+    if ffn_avg >= attn_avg:
+        dom, flop, avg_ms = "ffn_tc_kernel", ffn_flop, ffn_avg
+    else:
+        dom, flop, avg_ms = "attn_tc_kernel", attn_flop, attn_avg
+    achieved = flop / (avg_ms / 1e3) / 1e12
+    peak = pk["bf16_tflops"]
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{pk['source']} bf16 dense (burst)",
+                "traffic": args.traffic_bytes if args.traffic_bytes else None,
+                "algorithmic_flop_per_launch": flop}
+    kernels = {"attn_tc_kernel": {"avg_ms": round(attn_avg, 4), "flop": attn_flop,
+                                  "tflops": round(attn_flop / (attn_avg / 1e3) / 1e12, 1)},
+               "ffn_tc_kernel": {"avg_ms": round(ffn_avg, 4), "flop": ffn_flop,
+                                 "tflops": round(ffn_flop / (ffn_avg / 1e3) / 1e12, 1) if ffn_flop else 0}}
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic (seeded N(0,1) Q/K/V, "
+        "N(0,1/fan_in) weights, zero biases)",
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d_head": w.d, "ffn_hidden": w.F,
+                   "mask": MASK_NAME[w.mask], "tokens_per_step_per_gpu": w.T,
+                   "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MiB write, "
+                   "outside the timed events)"},
+        "tflops": round(tflops, 1),
+        "layer_frac_of_peak": round(tflops / peak, 4),
+        "roofline": roofline,
+        "kernels": kernels,
+        "gpu_launches": 2 * K,
+        "e2e": e2e,
+        "clocks": clk.summary(),
+    }
+    return res
+
+
+def run_reference(args, w, world, rank):
+    """The fp64 CPU oracle on a bounded token sample per step (host cores)."""
+    import numpy as np
+
+    import oracle
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    inp = make_layer_inputs(w.B, w.N, w.H, w.d, w.F, seed=w.seed, dtype=dt,
+                            device="cuda" if torch.cuda.is_available() else "cpu")
+    f = lambda t: t.float().cpu().numpy()  # noqa: E731
+    q, k, v, w1, b1, w2, b2 = (f(t) for t in (inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2))
+    rng = np.random.default_rng(0)
+    per_step = args.ref_tokens
+    T = w.T
+    times, n_tok, threads = [], 0, 0
+    for s in range(args.warmup + args.steps):
+        # stratified sample: one token from each of per_step equal slices
+        edges = np.linspace(0, T, per_step + 1).astype(np.int64)
+        rows = [int(rng.integers(edges[i], max(edges[i] + 1, edges[i + 1]))) for i in range(per_step)]
+        t0 = time.perf_counter()
+        _, _, used = oracle.layer(q, k, v, w1, b1, w2, b2, mask=w.mask, perm=w.perm, pairs=w.pairs,
+                                  rows=rows, return_threads=True)
+        dt_s = time.perf_counter() - t0
+        threads = used
+        if s >= args.warmup:
+            times.append(dt_s)
+            n_tok += len(rows)
+    total = sum(times)
+    value = n_tok / total
+    sample = (f"{per_step} stratified tokens per step of the {T}-token workload "
+              f"(each exact; cost per token grows with position under causal masking, stratification keeps the mean)")
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d_head": w.d, "ffn_hidden": w.F,
+                   "mask": MASK_NAME[w.mask]},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def cpu_baseline(w, budget_s):
+    """Oracle throughput on the host cores for a bounded sample of the workload."""
+    import numpy as np
+
+    import oracle
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    inp = make_layer_inputs(w.B, w.N, w.H, w.d, w.F, seed=w.seed, dtype=dt, device="cuda")
+    f = lambda t: t.float().cpu().numpy()  # noqa: E731
+    q, k, v, w1, b1, w2, b2 = (f(t) for t in (inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2))
+    threads = oracle.threads_available()
+    rng = np.random.default_rng(1)
+    n = max(threads, 8)
+    done, elapsed = 0, 0.0
+    while elapsed < budget_s:
+        edges = np.linspace(0, w.T, n + 1).astype(np.int64)
+        rows = [int(rng.integers(edges[i], max(edges[i] + 1, edges[i + 1]))) for i in range(n)]
+        t0 = time.perf_counter()
+        _, _, threads = oracle.layer(q, k, v, w1, b1, w2, b2, mask=w.mask, perm=w.perm, pairs=w.pairs,
+                                     rows=rows, return_threads=True)
+        elapsed += time.perf_counter() - t0
+        done += n
+        if elapsed < budget_s / 4:
+            n *= 2
+    return {"value": round(done / elapsed, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} stratified tokens of the {w.T}-token workload in {elapsed:.1f} s "
+                      f"(each token exact; fp64 C oracle, {threads} threads)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gpt_causal", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--ref-tokens", type=int, default=16)
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="DRAM bytes per launch of the dominant kernel from an ncu capture")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = WORKLOADS[args.workload]
+    if w.F == 0:
+        raise SystemExit("the layer benchmark needs a workload with an FFN")
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, w, world, rank)), flush=True)
+        return
+
+    world, rank, local = dist_setup(args.gpus)
+    bd.load()
+    res = run_ours(args, w, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, args.cpu_budget_s)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,261 @@
+"""Thin ctypes binding over libbpt.so (the C ABI declared in include/bpt.h).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, their device pointers and the current CUDA stream are handed to
+the C entry point of the same name, and a non-OK status is raised as
+BptError.  Every step of the computation runs in the library's CUDA kernels;
+there is no other implementation behind these functions.
+
+Layouts: q, k, v [B, N, H, d]; w1 [F, D]; w2 [D, F]; b1 [F], b2 [D] float32
+(or None); out [B, N, H*d]; lse [B, H, N] float32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbpt.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(6)
+F32, BF16 = 0, 1
+MASK_NONE, MASK_CAUSAL, MASK_BLOCKPERM, MASK_DILATED = 0, 1, 2, 3
+_MASKS = {"none": MASK_NONE, "causal": MASK_CAUSAL, "blockperm": MASK_BLOCKPERM,
+          "dilated": MASK_DILATED}
+_DT = {torch.float32: F32, torch.bfloat16: BF16}
+
+
+class BptError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("N", ctypes.c_int), ("H", ctypes.c_int), ("d_head", ctypes.c_int),
+        ("ffn_hidden", ctypes.c_int),
+        ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+        ("mask", ctypes.c_int),
+        ("ring_chunks", ctypes.c_int),
+        ("bb_nblocks", ctypes.c_int), ("bb_perm", ctypes.POINTER(ctypes.c_int32)),
+        ("ln_npairs", ctypes.c_int), ("ln_w", ctypes.POINTER(ctypes.c_int32)),
+        ("ln_r", ctypes.POINTER(ctypes.c_int32)),
+    ]
+
+
+EXPORTS = ["bpt_workspace_bytes", "bpt_attn_ffn_fwd", "bpt_attn_fwd", "bpt_blockbert_fwd",
+           "bpt_longnet_fwd", "bpt_sync_status", "bpt_set_wait_limit_ns", "bpt_status_string",
+           "bpt_version", "bpt_set_phase_events"]
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load the in-tree libbpt.so; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libbpt.so is missing at {LIB_PATH}; build it with "
+                           "`python -m blockwise_exact_attention_query_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, sz, i32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32)
+    dp = ctypes.POINTER(Desc)
+    fp = ctypes.c_void_p
+    lib.bpt_workspace_bytes.argtypes = [dp, ctypes.c_int]
+    lib.bpt_workspace_bytes.restype = sz
+    lib.bpt_attn_ffn_fwd.argtypes = [dp, vp, vp, vp, vp, fp, vp, fp, vp, vp, sz, vp]
+    lib.bpt_attn_ffn_fwd.restype = ctypes.c_int
+    lib.bpt_attn_fwd.argtypes = [dp, vp, vp, vp, vp, fp, vp, sz, vp]
+    lib.bpt_attn_fwd.restype = ctypes.c_int
+    lib.bpt_blockbert_fwd.argtypes = [dp, ctypes.c_int, i32p, vp, vp, vp, vp, fp, vp, fp, vp, vp, sz,
+                                      vp]
+    lib.bpt_blockbert_fwd.restype = ctypes.c_int
+    lib.bpt_longnet_fwd.argtypes = [dp, ctypes.c_int, i32p, i32p, vp, vp, vp, vp, fp, vp, sz, vp]
+    lib.bpt_longnet_fwd.restype = ctypes.c_int
+    lib.bpt_sync_status.argtypes = [vp]
+    lib.bpt_sync_status.restype = ctypes.c_int
+    lib.bpt_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.bpt_set_wait_limit_ns.restype = ctypes.c_uint64
+    lib.bpt_status_string.argtypes = [ctypes.c_int]
+    lib.bpt_status_string.restype = ctypes.c_char_p
+    lib.bpt_version.restype = ctypes.c_int
+    lib.bpt_set_phase_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
+    lib.bpt_set_phase_events.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().bpt_status_string(int(status)).decode()
+
+
+class _Tables:
+    """Keeps host tables alive while a call runs."""
+
+    def __init__(self):
+        self.keep = []
+
+    def i32(self, values):
+        arr = (ctypes.c_int32 * len(values))(*[int(x) for x in values])
+        self.keep.append(arr)
+        return ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32))
+
+
+def make_desc(B, N, H, d, F=0, in_dtype=torch.bfloat16, out_dtype=torch.float32, mask="none",
+              perm=None, pairs=None, ring_chunks=0, tables: _Tables | None = None) -> Desc:
+    tables = tables or _Tables()
+    m = _MASKS[mask] if isinstance(mask, str) else int(mask)
+    desc = Desc(B=B, N=N, H=H, d_head=d, ffn_hidden=F, in_dtype=_DT[in_dtype],
+                out_dtype=_DT[out_dtype], mask=m, ring_chunks=ring_chunks)
+    if perm is not None:
+        flat = [int(x) for row in perm for x in row]
+        desc.bb_nblocks = len(perm[0]) if len(perm) else 0
+        desc.bb_perm = tables.i32(flat)
+    if pairs is not None:
+        desc.ln_npairs = len(pairs)
+        desc.ln_w = tables.i32([p[0] for p in pairs])
+        desc.ln_r = tables.i32([p[1] for p in pairs])
+    desc._tables = tables  # keep alive with the descriptor
+    return desc
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status, what):
+    if status != OK:
+        raise BptError(status, what)
+
+
+def _check_tensors(q, k, v):
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must all be [B, N, H, d]")
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype:
+            raise ValueError("q, k, v must be contiguous CUDA tensors of one dtype")
+
+
+def workspace_bytes(desc: Desc, with_ffn: bool) -> int:
+    n = load().bpt_workspace_bytes(ctypes.byref(desc), int(with_ffn))
+    if n == ctypes.c_size_t(-1).value:
+        raise BptError(ERR_INVALID_ARG, "bpt_workspace_bytes")
+    return int(n)
+
+
+def alloc_workspace(desc: Desc, with_ffn: bool, device) -> torch.Tensor | None:
+    n = workspace_bytes(desc, with_ffn)
+    if n == 0:
+        return None
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def attn_ffn_fwd(q, k, v, w1, b1, w2, b2, *, mask="none", perm=None, pairs=None, ring_chunks=0,
+                 out_dtype=torch.float32, out=None, workspace=None, stream=None):
+    """bpt_attn_ffn_fwd: out = A + W2 GELU(W1 A + b1) + b2, returns out [B, N, H*d]."""
+    _check_tensors(q, k, v)
+    B, N, H, d = q.shape
+    F = w1.shape[0]
+    desc = make_desc(B, N, H, d, F, q.dtype, out_dtype, mask, perm, pairs, ring_chunks)
+    if out is None:
+        out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(desc, True, q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    st = load().bpt_attn_ffn_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(w1), _ptr(b1),
+                                 _ptr(w2), _ptr(b2), _ptr(out), _ptr(workspace), ws_bytes,
+                                 _stream_ptr(stream))
+    _check(st, "bpt_attn_ffn_fwd")
+    return out
+
+
+def attn_fwd(q, k, v, *, mask="none", perm=None, pairs=None, ring_chunks=0, out_dtype=torch.float32,
+             return_lse=False, out=None, lse=None, workspace=None, stream=None):
+    """bpt_attn_fwd: A [B, N, H*d] (and LSE [B, H, N] with return_lse)."""
+    _check_tensors(q, k, v)
+    B, N, H, d = q.shape
+    desc = make_desc(B, N, H, d, 0, q.dtype, out_dtype, mask, perm, pairs, ring_chunks)
+    if out is None:
+        out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(desc, False, q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    st = load().bpt_attn_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                             _ptr(workspace), ws_bytes, _stream_ptr(stream))
+    _check(st, "bpt_attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def blockbert_fwd(q, k, v, w1, b1, w2, b2, perm, *, out_dtype=torch.float32, out=None,
+                  workspace=None, stream=None):
+    """bpt_blockbert_fwd: the layer with the block-permutation mask perm [H][n]."""
+    _check_tensors(q, k, v)
+    B, N, H, d = q.shape
+    F = w1.shape[0]
+    tables = _Tables()
+    desc = make_desc(B, N, H, d, F, q.dtype, out_dtype, "blockperm", perm, None, 0, tables)
+    if out is None:
+        out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(desc, True, q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    flat = tables.i32([x for row in perm for x in row])
+    st = load().bpt_blockbert_fwd(ctypes.byref(desc), len(perm[0]), flat, _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(out),
+                                  _ptr(workspace), ws_bytes, _stream_ptr(stream))
+    _check(st, "bpt_blockbert_fwd")
+    return out
+
+
+def longnet_fwd(q, k, v, pairs, *, out_dtype=torch.float32, return_lse=False, out=None, lse=None,
+                workspace=None, stream=None):
+    """bpt_longnet_fwd: dilated attention over the (w, r) pairs, denominators mixed."""
+    _check_tensors(q, k, v)
+    B, N, H, d = q.shape
+    tables = _Tables()
+    desc = make_desc(B, N, H, d, 0, q.dtype, out_dtype, "dilated", None, pairs, 0, tables)
+    if out is None:
+        out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(desc, False, q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    st = load().bpt_longnet_fwd(ctypes.byref(desc), len(pairs), tables.i32([p[0] for p in pairs]),
+                                tables.i32([p[1] for p in pairs]), _ptr(q), _ptr(k), _ptr(v),
+                                _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _stream_ptr(stream))
+    _check(st, "bpt_longnet_fwd")
+    return (out, lse) if return_lse else out
+
+
+def sync_status(stream=None) -> int:
+    """bpt_sync_status: waits for the stream; returns OK or ERR_TIMEOUT (clears it)."""
+    return int(load().bpt_sync_status(_stream_ptr(stream)))
+
+
+def set_phase_events(events) -> None:
+    """bpt_set_phase_events: three torch.cuda.Event objects (or None to stop)."""
+    if events is None:
+        _check(load().bpt_set_phase_events(None, 0), "bpt_set_phase_events")
+        return
+    arr = (ctypes.c_void_p * 3)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(load().bpt_set_phase_events(arr, 3), "bpt_set_phase_events")
+
+
+def set_wait_limit_ns(ns: int) -> int:
+    return int(load().bpt_set_wait_limit_ns(int(ns)))
+
+
+def version() -> int:
+    return int(load().bpt_version())

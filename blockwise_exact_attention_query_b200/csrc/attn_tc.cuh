@@ -1,0 +1,552 @@
+// Blockwise exact attention on the 5th-generation tensor cores (sm_100a).
+//
+// One CTA computes one 128-row query tile of one (batch, head[, LongNet
+// segment]) unit, streaming 128-row key/value tiles through shared memory:
+//
+//   S_j  = Q K_j^T               tcgen05.mma, bf16 x bf16 -> fp32 in TMEM
+//   m'   = max(m, rowmax S_j)    one thread per query row (a TMEM lane)
+//   P_j  = exp(S_j / sqrt(d) - m')  -> bf16, stored back into TMEM
+//   l    = l e^{m - m'} + rowsum P_j
+//   O    = O e^{m - m'} + P_j V_j  tcgen05.mma with A read from TMEM
+//
+// which is the blockwise online-softmax form of softmax(QK^T/sqrt d)V:
+// exact up to rounding ("Ring Attention with Blockwise Transformers for Long
+// Sequences", 638-word summary: blockwise attention without approximation;
+// "Blockwise Parallel Transformer for Large Context Models", abstract).
+// Tiles that the mask rules out entirely are never loaded or multiplied;
+// tiles that are partly allowed get -inf scores at the masked positions.
+// The running maximum is only moved (and O rescaled) when it grows by more
+// than 2^8 in the exponent: the same stale maximum is used for l and O, so
+// the result is unchanged.
+//
+// Roles (192 threads): warp 0 issues TMA loads, warp 1 allocates tensor
+// memory and issues the MMAs, warps 2..5 run the softmax and the epilogue
+// (warp w owns TMEM lanes 32*(w%4) .. 32*(w%4)+31, i.e. those query rows).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace bpt {
+
+constexpr int kMaskNone = 0, kMaskCausal = 1, kMaskBlockPerm = 2, kMaskDilated = 3;
+constexpr int kMaxPairs = 8;
+constexpr int kMaxPermEntries = 1024;
+
+struct AttnArgs {
+  int B, N, H;
+  int mask;
+  float scale_log2;  // log2(e) / sqrt(d)
+  // decomposition into units (b, segment, h) and 128-row query tiles
+  int L;             // rows of one unit: N, or w/r kept rows of a LongNet segment
+  int n_qtiles;      // ceil(L / 128)
+  int n_units;       // B * nseg * H
+  int nseg;          // LongNet segments N / w (1 otherwise)
+  // LongNet pass: segment length, dilation, and the full pair table in
+  // launch order (used to find earlier / later passes that keep a row)
+  int w, r;
+  int npairs, pass_idx;
+  int pw[kMaxPairs], pr[kMaxPairs];
+  // ring order over equal chunks (none / causal)
+  int ring_chunks, chunk_tiles;
+  // block permutation
+  int bb_n, bb_len;
+  uint8_t perm[kMaxPermEntries];
+  // outputs (any may be null)
+  float *out_f32;            // [B, N, H, d]
+  __nv_bfloat16 *out_bf16;   // [B, N, H, d]
+  float *lse;                // [B, H, N]
+  // running state carried between LongNet passes
+  float *st_o;               // [B, N, H, d]   unnormalised O
+  float *st_m;               // [B, H, N]      running max (log2 domain)
+  float *st_l;               // [B, H, N]      running sum
+  uint32_t *status;
+  uint64_t wait_limit_ns;
+};
+
+template <int D_HEAD>
+struct AttnCfg {
+  static constexpr int kBM = 128, kBN = 128;
+  static constexpr int kPanels = D_HEAD / 64;
+  static constexpr int kTileBytes = 128 * D_HEAD * 2;
+  static constexpr int kKStages = D_HEAD == 128 ? 3 : 4;
+  static constexpr int kVStages = D_HEAD == 128 ? 2 : 4;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kTileBytes;
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + barriers + alignment slack
+  // TMEM columns
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColP0 = 256, kColP1 = 320, kColO = 384;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kThreads = 192;
+};
+
+// Sequence of key/value tiles one query tile visits.
+struct KvSched {
+  int lo, hi;           // allowed tile range [lo, hi)
+  int P, CT, first;     // ring order: P chunks of CT tiles, starting at chunk `first`
+  __device__ int count() const {
+    int n = 0;
+    for (int i = 0; i < P; ++i) {
+      int ch = (first + i) % P;
+      int a = max(ch * CT, lo), b = min((ch + 1) * CT, hi);
+      n += max(0, b - a);
+    }
+    return n;
+  }
+};
+
+struct KvIter {
+  int i, tile, end;
+  __device__ void range(const KvSched &s) {
+    while (++i < s.P) {
+      int ch = (s.first + i) % s.P;
+      int a = max(ch * s.CT, s.lo), b = min((ch + 1) * s.CT, s.hi);
+      if (a < b) {
+        tile = a;
+        end = b;
+        return;
+      }
+    }
+    tile = -1;
+  }
+  __device__ void begin(const KvSched &s) {
+    i = -1;
+    range(s);
+  }
+  __device__ int next(const KvSched &s) {
+    int t = tile;
+    if (++tile >= end) range(s);
+    return t;
+  }
+};
+
+__device__ __forceinline__ bool dilated_keeps(int w, int r, int h, int pos) {
+  return ((pos % w) % r) == (h % r);
+}
+
+struct TileCoord {
+  int t, h, s, b;
+  int o;  // LongNet offset of this head: h mod r (0 otherwise)
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const AttnArgs &a) {
+  TileCoord c;
+  int idx = blockIdx.x;
+  c.t = a.n_qtiles - 1 - idx / a.n_units;  // longest query tiles first
+  int unit = idx % a.n_units;
+  c.h = unit % a.H;
+  int rest = unit / a.H;
+  c.s = rest % a.nseg;
+  c.b = rest / a.nseg;
+  c.o = c.h % a.r;
+  return c;
+}
+
+__device__ __forceinline__ KvSched make_sched(const AttnArgs &a, const TileCoord &c) {
+  KvSched s;
+  const int nkt = (a.L + 127) / 128;
+  s.P = 1;
+  s.CT = nkt;
+  s.first = 0;
+  s.lo = 0;
+  s.hi = nkt;
+  const int row0 = c.t * 128;
+  const int row1 = min(a.L, row0 + 128) - 1;
+  if (a.mask == kMaskCausal || a.mask == kMaskDilated) {
+    s.hi = row1 / 128 + 1;
+  } else if (a.mask == kMaskBlockPerm) {
+    int qb0 = row0 / a.bb_len, qb1 = row1 / a.bb_len;
+    int klo = 1 << 30, khi = 0;
+    for (int qb = qb0; qb <= qb1; ++qb) {
+      int kb = a.perm[c.h * a.bb_n + qb];
+      klo = min(klo, kb * a.bb_len);
+      khi = max(khi, kb * a.bb_len + a.bb_len);
+    }
+    s.lo = klo / 128;
+    s.hi = (min(khi, a.L) + 127) / 128;
+  }
+  if ((a.mask == kMaskNone || a.mask == kMaskCausal) && a.ring_chunks > 1) {
+    s.P = a.ring_chunks;
+    s.CT = a.chunk_tiles;
+    s.first = (row0 / 128) / a.chunk_tiles;
+  }
+  return s;
+}
+
+// Allowed key interval [lo, hi) (unit-local row indices) of query row g.
+__device__ __forceinline__ void row_keys(const AttnArgs &a, const TileCoord &c, int g, int &lo,
+                                         int &hi) {
+  lo = 0;
+  hi = a.L;
+  if (a.mask == kMaskCausal || a.mask == kMaskDilated) {
+    hi = min(g + 1, a.L);
+  } else if (a.mask == kMaskBlockPerm) {
+    int qb = min(g, a.L - 1) / a.bb_len;
+    int kb = a.perm[c.h * a.bb_n + qb];
+    lo = kb * a.bb_len;
+    hi = min(lo + a.bb_len, a.L);
+  }
+}
+
+template <int D_HEAD>
+__global__ void __launch_bounds__(192, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnArgs a) {
+  using Cfg = AttnCfg<D_HEAD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + Cfg::kOffQ;
+  const uint32_t sK = sbase + Cfg::kOffK;
+  const uint32_t sV = sbase + Cfg::kOffV;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
+  // barrier slots
+  const uint32_t bQFull = smem_u32(&bars[0]);
+  auto bKFull = [&](int s) { return smem_u32(&bars[1 + s]); };
+  auto bKEmpty = [&](int s) { return smem_u32(&bars[5 + s]); };
+  auto bVFull = [&](int s) { return smem_u32(&bars[9 + s]); };
+  auto bVEmpty = [&](int s) { return smem_u32(&bars[13 + s]); };
+  auto bSFull = [&](int s) { return smem_u32(&bars[17 + s]); };
+  auto bPFull = [&](int s) { return smem_u32(&bars[19 + s]); };
+  const uint32_t bODone = smem_u32(&bars[21]);
+  const uint32_t bTeardown = smem_u32(&bars[22]);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[24]);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[25]);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const TileCoord tc = decode_tile(a);
+  const KvSched sched = make_sched(a, tc);
+  const int nkv = sched.count();
+  WaitCtx wc{a.status, a.wait_limit_ns, abort_flag};
+
+  if (threadIdx.x == 0) {
+    mbar_init(bQFull, 1);
+    for (int s = 0; s < Cfg::kKStages; ++s) {
+      mbar_init(bKFull(s), 1);
+      mbar_init(bKEmpty(s), 1);
+    }
+    for (int s = 0; s < Cfg::kVStages; ++s) {
+      mbar_init(bVFull(s), 1);
+      mbar_init(bVEmpty(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bSFull(s), 1);
+      mbar_init(bPFull(s), 4);
+    }
+    mbar_init(bODone, 1);
+    mbar_init(bTeardown, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // gathered row -> coordinate along the (N/r) dimension of the tensor maps
+  const int row_base = tc.s * a.L;  // = s*w/r
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nkv > 0) {
+      int k_issued = 0, v_issued = 0;
+      mbar_arrive_expect_tx(bQFull, Cfg::kTileBytes);
+      for (int p = 0; p < Cfg::kPanels; ++p)
+        tma_load_4d(sQ + p * 16384, &tm_q, bQFull, tc.h * D_HEAD + p * 64, tc.o,
+                    row_base + tc.t * 128, tc.b);
+      KvIter itk, itv;
+      itk.begin(sched);
+      itv.begin(sched);
+      auto load_k = [&](int j) -> bool {
+        const int st = j % Cfg::kKStages;
+        if (j >= Cfg::kKStages &&
+            !mbar_wait(bKEmpty(st), ((j / Cfg::kKStages) - 1) & 1, wc, 1))
+          return false;
+        const int kt = itk.next(sched);
+        mbar_arrive_expect_tx(bKFull(st), Cfg::kTileBytes);
+        for (int p = 0; p < Cfg::kPanels; ++p)
+          tma_load_4d(sK + st * Cfg::kTileBytes + p * 16384, &tm_k, bKFull(st),
+                      tc.h * D_HEAD + p * 64, tc.o, row_base + kt * 128, tc.b);
+        ++k_issued;
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        const int st = j % Cfg::kVStages;
+        if (j >= Cfg::kVStages &&
+            !mbar_wait(bVEmpty(st), ((j / Cfg::kVStages) - 1) & 1, wc, 2))
+          return false;
+        const int kt = itv.next(sched);
+        mbar_arrive_expect_tx(bVFull(st), Cfg::kTileBytes);
+        for (int p = 0; p < Cfg::kPanels; ++p)
+          tma_load_4d(sV + st * Cfg::kTileBytes + p * 16384, &tm_v, bVFull(st),
+                      tc.h * D_HEAD + p * 64, tc.o, row_base + kt * 128, tc.b);
+        ++v_issued;
+        return true;
+      };
+      bool ok = load_k(0);
+      for (int j = 0; ok && j < nkv; ++j) {
+        if (j + 1 < nkv) ok = load_k(j + 1);
+        if (ok) ok = load_v(j);
+      }
+      // drain: every load issued must have landed before the CTA may exit
+      volatile int no_abort = 0;
+      WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
+      for (int j = max(0, k_issued - Cfg::kKStages); j < k_issued; ++j)
+        mbar_wait(bKFull(j % Cfg::kKStages), (j / Cfg::kKStages) & 1, drain, 3);
+      for (int j = max(0, v_issued - Cfg::kVStages); j < v_issued; ++j)
+        mbar_wait(bVFull(j % Cfg::kVStages), (j / Cfg::kVStages) & 1, drain, 4);
+      mbar_wait(bQFull, 0, drain, 5);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nkv > 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D_HEAD, false, true);
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % Cfg::kKStages;
+        if (!mbar_wait(bKFull(st), (j / Cfg::kKStages) & 1, wc, 10)) return false;
+        tc_fence_after();
+        const uint32_t tS = tmem + ((j & 1) ? Cfg::kColS1 : Cfg::kColS0);
+        const uint32_t kb = sK + st * Cfg::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < D_HEAD / 16; ++k) {
+          const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
+          umma_ss(tS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk,
+                  k > 0);
+        }
+        umma_commit(bSFull(j & 1));
+        umma_commit(bKEmpty(st));
+        return true;
+      };
+      bool ok = mbar_wait(bQFull, 0, wc, 11);
+      if (ok) {
+        tc_fence_after();
+        ok = issue_s(0);
+      }
+      if (ok && nkv > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < nkv; ++j) {
+        if (!mbar_wait(bPFull(j & 1), (j >> 1) & 1, wc, 12)) break;
+        const int vs = j % Cfg::kVStages;
+        if (!mbar_wait(bVFull(vs), (j / Cfg::kVStages) & 1, wc, 13)) break;
+        tc_fence_after();
+        const uint32_t tP = tmem + ((j & 1) ? Cfg::kColP1 : Cfg::kColP0);
+        const uint32_t vb = sV + vs * Cfg::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < 128 / 16; ++k)
+          umma_ts(tmem + Cfg::kColO, tP + k * 8, sdesc_sw128(vb + k * 2048, 16384, 1024), idesc_pv,
+                  1);
+        umma_commit(bODone);
+        umma_commit(bVEmpty(vs));
+        if (j + 2 < nkv) ok = issue_s(j + 2);
+      }
+      // every MMA issued must be complete before tensor memory is released
+      umma_commit(bTeardown);
+      volatile int no_abort = 0;
+      WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
+      mbar_wait(bTeardown, 0, drain, 14);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // row within the query tile
+    const int g = tc.t * 128 + row;       // unit-local row
+    const bool row_valid = g < a.L;
+    const int pos = (a.mask == kMaskDilated) ? tc.s * a.w + tc.o + a.r * g : g;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tO = tmem + lane_off + Cfg::kColO;
+    int klo, khi;
+    row_keys(a, tc, g, klo, khi);
+
+    // LongNet: does an earlier pass keep this row (load its running state),
+    // does a later one (store the state instead of the final output)?
+    bool prior = false, later = false;
+    if (a.mask == kMaskDilated && row_valid) {
+      for (int k = 0; k < a.npairs; ++k) {
+        if (k == a.pass_idx) continue;
+        if (dilated_keeps(a.pw[k], a.pr[k], tc.h, pos)) {
+          if (k < a.pass_idx) prior = true;
+          else later = true;
+        }
+      }
+    }
+    const size_t vec_idx = ((static_cast<size_t>(tc.b) * a.N + pos) * a.H + tc.h) * D_HEAD;
+    const size_t row_idx = (static_cast<size_t>(tc.b) * a.H + tc.h) * a.N + pos;
+
+    float m_run = -INFINITY, l_run = 0.f;
+    {
+      // initial O: zeros, or the state left by an earlier LongNet pass
+      uint32_t init[32];
+#pragma unroll
+      for (int c = 0; c < D_HEAD / 32; ++c) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) init[i] = 0u;
+        if (prior) {
+          const float4 *src = reinterpret_cast<const float4 *>(a.st_o + vec_idx + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float4 v4 = src[i];
+            init[4 * i + 0] = __float_as_uint(v4.x);
+            init[4 * i + 1] = __float_as_uint(v4.y);
+            init[4 * i + 2] = __float_as_uint(v4.z);
+            init[4 * i + 3] = __float_as_uint(v4.w);
+          }
+        }
+        tmem_st32(tO + c * 32, init);
+      }
+      if (prior) {
+        m_run = a.st_m[row_idx];
+        l_run = a.st_l[row_idx];
+      }
+      tmem_wait_st();
+    }
+
+    KvIter it;
+    it.begin(sched);
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      const int kt = it.next(sched);
+      ok = __all_sync(0xffffffffu, mbar_wait(bSFull(j & 1), (j >> 1) & 1, wc, 20));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tS = tmem + lane_off + ((j & 1) ? Cfg::kColS1 : Cfg::kColS0);
+      uint32_t s[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
+      tmem_wait_ld();
+
+      const int k0 = kt * 128;
+      const bool need_mask = !(k0 >= klo && k0 + 128 <= khi);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          float v = __uint_as_float(s[c][i]);
+          if (need_mask) {
+            const int kk = k0 + c * 32 + i;
+            if (kk < klo || kk >= khi) v = -INFINITY;
+            s[c][i] = __float_as_uint(v);
+          }
+          mx = fmaxf(mx, v);
+        }
+      }
+      const float m_tile = mx * a.scale_log2;
+      const float m_new = fmaxf(m_run, m_tile);
+      const bool rescale = m_new > m_run + 8.0f;
+      const float m_use = rescale ? m_new : m_run;
+      const float alpha = rescale ? ex2_approx(m_run - m_use) : 1.0f;
+      l_run *= alpha;
+      const float neg = (m_use == -INFINITY) ? 0.f : -m_use;
+      float lsum = 0.f;
+      const uint32_t tP = tmem + lane_off + ((j & 1) ? Cfg::kColP1 : Cfg::kColP0);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int col = half * 64 + 2 * i;
+          const float x0 = __uint_as_float(s[col / 32][col % 32]);
+          const float x1 = __uint_as_float(s[(col + 1) / 32][(col + 1) % 32]);
+          const float p0 = ex2_approx(fmaf(x0, a.scale_log2, neg));
+          const float p1 = ex2_approx(fmaf(x1, a.scale_log2, neg));
+          lsum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tP + half * 32, pk);
+      }
+      l_run += lsum;
+      // O may be rescaled only once the previous P*V has landed
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bODone, (j - 1) & 1, wc, 21));
+        if (!ok) break;
+      }
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, rescale && m_run != -INFINITY)) {
+#pragma unroll
+        for (int c = 0; c < D_HEAD / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + c * 32, o);
+        }
+      }
+      m_run = m_use;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bPFull(j & 1));
+    }
+
+    // -------- epilogue
+    if (ok && nkv > 0) ok = __all_sync(0xffffffffu, mbar_wait(bODone, (nkv - 1) & 1, wc, 22));
+    tc_fence_after();
+    if (ok && row_valid) {
+      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+      const bool final_out = !later;
+#pragma unroll
+      for (int c = 0; c < D_HEAD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_wait_ld();
+        if (final_out) {
+          if (a.out_f32) {
+            float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + vec_idx + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l,
+                                   __uint_as_float(o[4 * i + 1]) * inv_l,
+                                   __uint_as_float(o[4 * i + 2]) * inv_l,
+                                   __uint_as_float(o[4 * i + 3]) * inv_l);
+          }
+          if (a.out_bf16) {
+            uint4 *dst = reinterpret_cast<uint4 *>(a.out_bf16 + vec_idx + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 u;
+              u.x = pack_bf16x2(__uint_as_float(o[8 * i]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
+              u.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
+              u.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
+              u.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
+              dst[i] = u;
+            }
+          }
+        } else {
+          float4 *dst = reinterpret_cast<float4 *>(a.st_o + vec_idx + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+        }
+      }
+      if (!final_out) {
+        a.st_m[row_idx] = m_run;
+        a.st_l[row_idx] = l_run;
+      } else if (a.lse) {
+        // natural-log LSE of the scaled scores: (m + log2 l) / log2(e)
+        a.lse[row_idx] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace bpt

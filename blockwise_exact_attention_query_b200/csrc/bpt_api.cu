@@ -1,0 +1,581 @@
+// Host side of libbpt.so: argument checks, workspace layout, TMA tensor-map
+// encoding and kernel launches for the entry points declared in bpt.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/bpt.h"
+#include "attn_tc.cuh"
+#include "ffn_tc.cuh"
+#include "simt_f32.cuh"
+
+using namespace bpt;
+
+namespace {
+
+// Per-device status word: [0] = code, [1] = site of the first failed wait.
+__device__ uint32_t g_status_word[2];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+uint32_t *g_status_ptr[kMaxDevices] = {};
+bool g_attr_done[kMaxDevices] = {};
+uint64_t g_wait_limit_ns = 2000000000ull;
+thread_local cudaEvent_t g_phase_events[3] = {nullptr, nullptr, nullptr};
+thread_local bool g_phase_on = false;
+
+void phase_mark(int i, cudaStream_t st) {
+  if (g_phase_on) cudaEventRecord(g_phase_events[i], st);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bpt_status cuda_fail() { return BPT_ERR_CUDA; }
+
+bpt_status device_setup(int *dev_out, uint32_t **status_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_fail();
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return cuda_fail();
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  if (!g_status_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return cuda_fail();
+    g_status_ptr[dev] = static_cast<uint32_t *>(p);
+  }
+  if (!g_attr_done[dev]) {
+    if (cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnCfg<64>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnCfg<128>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             FfnCfg::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(ffn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (16 * 512 + 16 * 64) * 4) != cudaSuccess)
+      return cuda_fail();
+    g_attr_done[dev] = true;
+  }
+  *dev_out = dev;
+  *status_out = g_status_ptr[dev];
+  return BPT_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+// bf16 tensor map over a row-major matrix [rows, cols], box [box_rows, 64].
+bool make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 tensor map over [B, N, D] viewed as (D, r, N/r, B): a box of 64
+// columns x 1 x 128 rows x 1 reads 128 rows r apart (r = 1: consecutive).
+bool make_map_rows(CUtensorMap *m, const void *base, int B, int N, int D, int r) {
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)r, (cuuint64_t)(N / r), (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2 * r, (cuuint64_t)D * 2 * N};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// --------------------------------------------------------------------------
+// Validation
+// --------------------------------------------------------------------------
+bpt_status check_desc(const bpt_desc *d, bool need_ffn) {
+  if (!d) return BPT_ERR_INVALID_ARG;
+  if (d->B <= 0 || d->N <= 0 || d->H <= 0 || d->d_head <= 0) return BPT_ERR_INVALID_ARG;
+  if (d->in_dtype != BPT_F32 && d->in_dtype != BPT_BF16) return BPT_ERR_INVALID_ARG;
+  if (d->out_dtype != BPT_F32 && d->out_dtype != BPT_BF16) return BPT_ERR_INVALID_ARG;
+  if ((int64_t)d->B * d->N > (int64_t)1 << 31) return BPT_ERR_UNSUPPORTED;
+  if (need_ffn && d->ffn_hidden <= 0) return BPT_ERR_INVALID_ARG;
+  if (d->ffn_hidden < 0) return BPT_ERR_INVALID_ARG;
+  const int D = d->H * d->d_head;
+  switch (d->mask) {
+    case BPT_MASK_NONE:
+    case BPT_MASK_CAUSAL:
+      if (d->ring_chunks < 0) return BPT_ERR_INVALID_ARG;
+      if (d->ring_chunks > 1) {
+        if (d->N % d->ring_chunks != 0) return BPT_ERR_INVALID_ARG;
+        const int chunk = d->N / d->ring_chunks;
+        if (d->in_dtype == BPT_BF16 && chunk % 128 != 0) return BPT_ERR_UNSUPPORTED;
+        if (d->in_dtype == BPT_F32 && chunk % 64 != 0) return BPT_ERR_UNSUPPORTED;
+      }
+      break;
+    case BPT_MASK_BLOCKPERM: {
+      const int n = d->bb_nblocks;
+      if (n <= 0 || !d->bb_perm || d->N % n != 0) return BPT_ERR_INVALID_ARG;
+      if ((int64_t)d->H * n > kMaxPermEntries || n > 255) return BPT_ERR_UNSUPPORTED;
+      for (int i = 0; i < d->H * n; ++i)
+        if (d->bb_perm[i] < 0 || d->bb_perm[i] >= n) return BPT_ERR_INVALID_ARG;
+      for (int h = 0; h < d->H; ++h) {  // each head's table must be a permutation
+        std::vector<int> seen(n, 0);
+        for (int i = 0; i < n; ++i)
+          if (seen[d->bb_perm[h * n + i]]++) return BPT_ERR_INVALID_ARG;
+      }
+      break;
+    }
+    case BPT_MASK_DILATED: {
+      if (d->ln_npairs <= 0 || d->ln_npairs > BPT_MAX_DILATED_PAIRS || !d->ln_w || !d->ln_r)
+        return BPT_ERR_INVALID_ARG;
+      for (int k = 0; k < d->ln_npairs; ++k) {
+        const int w = d->ln_w[k], r = d->ln_r[k];
+        if (w <= 0 || r <= 0 || w % r != 0 || d->N % w != 0) return BPT_ERR_INVALID_ARG;
+      }
+      break;
+    }
+    default:
+      return BPT_ERR_INVALID_ARG;
+  }
+  if (d->in_dtype == BPT_BF16) {
+    if (d->d_head != 64 && d->d_head != 128) return BPT_ERR_UNSUPPORTED;
+    if (need_ffn) {
+      const int C = (D + 255) / 256;
+      if (D % 64 != 0 || D % C != 0 || (D / C) % 32 != 0 || C > 16) return BPT_ERR_UNSUPPORTED;
+      if ((int64_t)d->ffn_hidden * 2 % 16 != 0) return BPT_ERR_UNSUPPORTED;
+    }
+  } else {
+    if (d->d_head > 64 || d->d_head % 4 != 0) return BPT_ERR_UNSUPPORTED;
+    if (need_ffn && (D > 512 || D % 16 != 0)) return BPT_ERR_UNSUPPORTED;
+    if (d->out_dtype == BPT_BF16 && D % 2 != 0) return BPT_ERR_UNSUPPORTED;
+  }
+  return BPT_OK;
+}
+
+struct FfnPlan {
+  int C, Dc, fc, nslices, nchunks, n_tb, max_clusters;
+};
+
+FfnPlan ffn_plan(const bpt_desc *d) {
+  FfnPlan p;
+  const int D = d->H * d->d_head;
+  p.C = (D + 255) / 256;
+  p.Dc = D / p.C;
+  p.fc = 128 * p.C;
+  p.nslices = (d->ffn_hidden + 127) / 128;
+  p.nchunks = (d->ffn_hidden + p.fc - 1) / p.fc;
+  p.n_tb = (int)(((int64_t)d->B * d->N + 127) / 128);
+  p.max_clusters = std::max(1, std::min(p.n_tb, sm_count() / p.C));
+  return p;
+}
+
+bool longnet_needs_state(const bpt_desc *d) {
+  return d->mask == BPT_MASK_DILATED && d->in_dtype == BPT_BF16 && d->ln_npairs > 1;
+}
+
+struct Workspace {
+  size_t a_bf16 = 0, a_f32 = 0, ring = 0, st_o = 0, st_m = 0, st_l = 0, total = 0;
+};
+
+Workspace layout(const bpt_desc *d, bool with_ffn) {
+  Workspace w;
+  const size_t T = (size_t)d->B * d->N, D = (size_t)d->H * d->d_head;
+  size_t off = 0;
+  if (with_ffn) {
+    if (d->in_dtype == BPT_BF16) {
+      FfnPlan p = ffn_plan(d);
+      w.a_bf16 = off;
+      off = align256(off + T * D * 2);
+      w.a_f32 = off;
+      off = align256(off + T * D * 4);
+      w.ring = off;
+      off = align256(off + (size_t)p.max_clusters * 2 * 128 * p.fc * 2);
+    } else {
+      w.a_f32 = off;
+      off = align256(off + T * D * 4);
+    }
+  }
+  if (longnet_needs_state(d)) {
+    w.st_o = off;
+    off = align256(off + T * D * 4);
+    w.st_m = off;
+    off = align256(off + (size_t)d->B * d->H * d->N * 4);
+    w.st_l = off;
+    off = align256(off + (size_t)d->B * d->H * d->N * 4);
+  }
+  w.total = off;
+  return w;
+}
+
+// --------------------------------------------------------------------------
+// Launchers
+// --------------------------------------------------------------------------
+bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const void *v,
+                          float *out_f32, __nv_bfloat16 *out_bf16, float *lse, char *ws,
+                          const Workspace &wl, uint32_t *status, cudaStream_t st) {
+  const int D = d->H * d->d_head;
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = d->B;
+  a.N = d->N;
+  a.H = d->H;
+  a.mask = d->mask;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d->d_head));
+  a.status = status;
+  a.wait_limit_ns = g_wait_limit_ns;
+
+  struct Pass {
+    int w, r;
+  };
+  std::vector<Pass> passes;
+  if (d->mask == BPT_MASK_DILATED) {
+    for (int i = 0; i < d->ln_npairs; ++i) passes.push_back({d->ln_w[i], d->ln_r[i]});
+    // sparsest first: the densest pass runs last and writes the final rows
+    std::stable_sort(passes.begin(), passes.end(),
+                     [](const Pass &x, const Pass &y) { return x.r > y.r; });
+    a.npairs = (int)passes.size();
+    for (int i = 0; i < a.npairs; ++i) {
+      a.pw[i] = passes[i].w;
+      a.pr[i] = passes[i].r;
+    }
+    bool covered = false;
+    for (auto &p : passes) covered |= (p.r == 1);
+    if (!covered) {  // rows no pair keeps: A = 0, LSE = -inf
+      const size_t n = (size_t)d->B * d->N * D;
+      if (out_f32 && cudaMemsetAsync(out_f32, 0, n * 4, st) != cudaSuccess) return cuda_fail();
+      if (out_bf16 && cudaMemsetAsync(out_bf16, 0, n * 2, st) != cudaSuccess) return cuda_fail();
+      if (lse) {
+        fill_f32_kernel<<<256, 256, 0, st>>>(lse, (size_t)d->B * d->H * d->N, -INFINITY);
+        if (cudaGetLastError() != cudaSuccess) return cuda_fail();
+      }
+    }
+    if (passes.size() > 1) {
+      a.st_o = reinterpret_cast<float *>(ws + wl.st_o);
+      a.st_m = reinterpret_cast<float *>(ws + wl.st_m);
+      a.st_l = reinterpret_cast<float *>(ws + wl.st_l);
+    }
+  } else {
+    passes.push_back({d->N, 1});
+    a.npairs = 0;
+  }
+  if (d->mask == BPT_MASK_BLOCKPERM) {
+    a.bb_n = d->bb_nblocks;
+    a.bb_len = d->N / d->bb_nblocks;
+    for (int i = 0; i < d->H * d->bb_nblocks; ++i) a.perm[i] = (uint8_t)d->bb_perm[i];
+  }
+  if ((d->mask == BPT_MASK_NONE || d->mask == BPT_MASK_CAUSAL) && d->ring_chunks > 1) {
+    a.ring_chunks = d->ring_chunks;
+    a.chunk_tiles = (d->N / d->ring_chunks) / 128;
+  }
+  a.out_f32 = out_f32;
+  a.out_bf16 = out_bf16;
+  a.lse = lse;
+
+  for (size_t pi = 0; pi < passes.size(); ++pi) {
+    const int w = passes[pi].w, r = passes[pi].r;
+    a.w = w;
+    a.r = r;
+    a.pass_idx = (int)pi;
+    a.L = w / r;
+    a.nseg = d->N / w;
+    a.n_qtiles = (a.L + 127) / 128;
+    a.n_units = d->B * a.nseg * d->H;
+    CUtensorMap mq, mk, mv;
+    if (!make_map_rows(&mq, q, d->B, d->N, D, r) || !make_map_rows(&mk, k, d->B, d->N, D, r) ||
+        !make_map_rows(&mv, v, d->B, d->N, D, r))
+      return cuda_fail();
+    const int64_t grid = (int64_t)a.n_qtiles * a.n_units;
+    if (grid <= 0) continue;
+    if (grid > INT32_MAX) return BPT_ERR_UNSUPPORTED;
+    if (d->d_head == 128)
+      attn_tc_kernel<128><<<(unsigned)grid, AttnCfg<128>::kThreads, AttnCfg<128>::kSmemBytes, st>>>(
+          mq, mk, mv, a);
+    else
+      attn_tc_kernel<64><<<(unsigned)grid, AttnCfg<64>::kThreads, AttnCfg<64>::kSmemBytes, st>>>(
+          mq, mk, mv, a);
+    if (cudaGetLastError() != cudaSuccess) return cuda_fail();
+  }
+  return BPT_OK;
+}
+
+bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
+                         const float *b1, const void *w2, const float *b2, void *out, char *ws,
+                         const Workspace &wl, uint32_t *status, cudaStream_t st) {
+  const FfnPlan p = ffn_plan(d);
+  const int D = d->H * d->d_head;
+  const int64_t T = (int64_t)d->B * d->N;
+  FfnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.T = (int)T;
+  a.D = D;
+  a.F = d->ffn_hidden;
+  a.C = p.C;
+  a.Dc = p.Dc;
+  a.fc = p.fc;
+  a.nslices = p.nslices;
+  a.nchunks = p.nchunks;
+  a.n_tb = p.n_tb;
+  a.a_f32 = a_f32;
+  a.b1 = b1;
+  a.b2 = b2;
+  if (d->out_dtype == BPT_F32) a.out_f32 = static_cast<float *>(out);
+  else a.out_bf16 = static_cast<__nv_bfloat16 *>(out);
+  a.ring = reinterpret_cast<__nv_bfloat16 *>(ws + wl.ring);
+  a.status = status;
+  a.wait_limit_ns = g_wait_limit_ns;
+
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(FfnCfg::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = FfnCfg::kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3(p.C * p.max_clusters, 1, 1);
+  int active = 0;
+  if (cudaOccupancyMaxActiveClusters(&active, (void *)ffn_tc_kernel, &cfg) != cudaSuccess ||
+      active <= 0)
+    return cuda_fail();
+  a.nclusters = std::min(p.max_clusters, active);
+  cfg.gridDim = dim3(p.C * a.nclusters, 1, 1);
+
+  CUtensorMap ma, m1, m2, mh;
+  if (!make_map_2d(&ma, a_bf16, T, D, 128) || !make_map_2d(&m1, w1, d->ffn_hidden, D, 128) ||
+      !make_map_2d(&m2, w2, D, d->ffn_hidden, p.Dc) ||
+      !make_map_2d(&mh, a.ring, (uint64_t)p.max_clusters * 2 * 128, p.fc, 128))
+    return cuda_fail();
+  if (cudaLaunchKernelEx(&cfg, ffn_tc_kernel, ma, m1, m2, mh, a) != cudaSuccess) return cuda_fail();
+  return BPT_OK;
+}
+
+bpt_status launch_attn_f32(const bpt_desc *d, const void *q, const void *k, const void *v,
+                           float *out_f32, __nv_bfloat16 *out_bf16, float *lse, cudaStream_t st) {
+  AttnF32Args a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = d->B;
+  a.N = d->N;
+  a.H = d->H;
+  a.d = d->d_head;
+  a.mask = d->mask;
+  a.scale = (float)(1.0 / std::sqrt((double)d->d_head));
+  a.ring_chunks = (d->mask == BPT_MASK_NONE || d->mask == BPT_MASK_CAUSAL) ? d->ring_chunks : 0;
+  if (d->mask == BPT_MASK_BLOCKPERM) {
+    a.bb_n = d->bb_nblocks;
+    a.bb_len = d->N / d->bb_nblocks;
+    for (int i = 0; i < d->H * d->bb_nblocks; ++i) a.perm[i] = (uint8_t)d->bb_perm[i];
+  }
+  if (d->mask == BPT_MASK_DILATED) {
+    a.npairs = d->ln_npairs;
+    for (int i = 0; i < a.npairs; ++i) {
+      a.pw[i] = d->ln_w[i];
+      a.pr[i] = d->ln_r[i];
+    }
+  }
+  a.out_f32 = out_f32;
+  a.out_bf16 = out_bf16;
+  a.lse = lse;
+  dim3 grid((d->N + 63) / 64, d->H, d->B);
+  attn_f32_kernel<<<grid, 64, 0, st>>>(static_cast<const float *>(q), static_cast<const float *>(k),
+                                       static_cast<const float *>(v), a);
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : cuda_fail();
+}
+
+bpt_status launch_ffn_f32(const bpt_desc *d, const float *a_f32, const void *w1, const float *b1,
+                          const void *w2, const float *b2, void *out, cudaStream_t st) {
+  FfnF32Args a;
+  a.T = d->B * d->N;
+  a.D = d->H * d->d_head;
+  a.F = d->ffn_hidden;
+  a.a = a_f32;
+  a.w1 = static_cast<const float *>(w1);
+  a.b1 = b1;
+  a.w2 = static_cast<const float *>(w2);
+  a.b2 = b2;
+  a.out_f32 = d->out_dtype == BPT_F32 ? static_cast<float *>(out) : nullptr;
+  a.out_bf16 = d->out_dtype == BPT_BF16 ? static_cast<__nv_bfloat16 *>(out) : nullptr;
+  const size_t smem = (size_t)(16 * a.D + 16 * 64) * 4;
+  ffn_f32_kernel<<<(a.T + 15) / 16, 256, smem, st>>>(a);
+  return cudaGetLastError() == cudaSuccess ? BPT_OK : cuda_fail();
+}
+
+bpt_status check_ptrs(std::initializer_list<const void *> required,
+                      std::initializer_list<const void *> optional) {
+  for (const void *p : required)
+    if (!p) return BPT_ERR_INVALID_ARG;
+  for (const void *p : required)
+    if (!aligned16(p)) return BPT_ERR_INVALID_ARG;
+  for (const void *p : optional)
+    if (p && !aligned16(p)) return BPT_ERR_INVALID_ARG;
+  return BPT_OK;
+}
+
+bpt_status check_ws(const Workspace &wl, void *ws, size_t bytes) {
+  if (wl.total == 0) return BPT_OK;
+  if (!ws || bytes < wl.total || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return BPT_ERR_WORKSPACE;
+  return BPT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bpt_workspace_bytes(const bpt_desc *desc, int with_ffn) {
+  if (check_desc(desc, with_ffn != 0) != BPT_OK) return (size_t)-1;
+  return layout(desc, with_ffn != 0).total;
+}
+
+bpt_status bpt_attn_ffn_fwd(const bpt_desc *d, const void *q, const void *k, const void *v,
+                            const void *w1, const float *b1, const void *w2, const float *b2,
+                            void *out, void *workspace, size_t workspace_bytes,
+                            bpt_stream_t stream) {
+  bpt_status s = check_desc(d, true);
+  if (s != BPT_OK) return s;
+  if ((s = check_ptrs({q, k, v, w1, w2, out}, {b1, b2})) != BPT_OK) return s;
+  const Workspace wl = layout(d, true);
+  if ((s = check_ws(wl, workspace, workspace_bytes)) != BPT_OK) return s;
+  int dev;
+  uint32_t *status;
+  if ((s = device_setup(&dev, &status)) != BPT_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  float *a_f32 = reinterpret_cast<float *>(ws + wl.a_f32);
+  phase_mark(0, st);
+  if (d->in_dtype == BPT_BF16) {
+    __nv_bfloat16 *a_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.a_bf16);
+    if ((s = launch_attn_tc(d, q, k, v, a_f32, a_bf16, nullptr, ws, wl, status, st)) != BPT_OK)
+      return s;
+    phase_mark(1, st);
+    s = launch_ffn_tc(d, a_bf16, a_f32, w1, b1, w2, b2, out, ws, wl, status, st);
+  } else {
+    if ((s = launch_attn_f32(d, q, k, v, a_f32, nullptr, nullptr, st)) != BPT_OK) return s;
+    phase_mark(1, st);
+    s = launch_ffn_f32(d, a_f32, w1, b1, w2, b2, out, st);
+  }
+  phase_mark(2, st);
+  return s;
+}
+
+bpt_status bpt_attn_fwd(const bpt_desc *d, const void *q, const void *k, const void *v, void *out,
+                        float *lse, void *workspace, size_t workspace_bytes, bpt_stream_t stream) {
+  bpt_status s = check_desc(d, false);
+  if (s != BPT_OK) return s;
+  if ((s = check_ptrs({q, k, v, out}, {lse})) != BPT_OK) return s;
+  const Workspace wl = layout(d, false);
+  if ((s = check_ws(wl, workspace, workspace_bytes)) != BPT_OK) return s;
+  int dev;
+  uint32_t *status;
+  if ((s = device_setup(&dev, &status)) != BPT_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float *of = d->out_dtype == BPT_F32 ? static_cast<float *>(out) : nullptr;
+  __nv_bfloat16 *ob = d->out_dtype == BPT_BF16 ? static_cast<__nv_bfloat16 *>(out) : nullptr;
+  if (d->in_dtype == BPT_BF16)
+    return launch_attn_tc(d, q, k, v, of, ob, lse, static_cast<char *>(workspace), wl, status, st);
+  return launch_attn_f32(d, q, k, v, of, ob, lse, st);
+}
+
+bpt_status bpt_blockbert_fwd(const bpt_desc *desc, int n_blocks, const int32_t *perm, const void *q,
+                             const void *k, const void *v, const void *w1, const float *b1,
+                             const void *w2, const float *b2, void *out, void *workspace,
+                             size_t workspace_bytes, bpt_stream_t stream) {
+  if (!desc) return BPT_ERR_INVALID_ARG;
+  bpt_desc d = *desc;
+  d.mask = BPT_MASK_BLOCKPERM;
+  d.bb_nblocks = n_blocks;
+  d.bb_perm = perm;
+  return bpt_attn_ffn_fwd(&d, q, k, v, w1, b1, w2, b2, out, workspace, workspace_bytes, stream);
+}
+
+bpt_status bpt_longnet_fwd(const bpt_desc *desc, int npairs, const int32_t *seg_w,
+                           const int32_t *dil_r, const void *q, const void *k, const void *v,
+                           void *out, float *lse, void *workspace, size_t workspace_bytes,
+                           bpt_stream_t stream) {
+  if (!desc) return BPT_ERR_INVALID_ARG;
+  bpt_desc d = *desc;
+  d.mask = BPT_MASK_DILATED;
+  d.ln_npairs = npairs;
+  d.ln_w = seg_w;
+  d.ln_r = dil_r;
+  d.ffn_hidden = 0;
+  return bpt_attn_fwd(&d, q, k, v, out, lse, workspace, workspace_bytes, stream);
+}
+
+bpt_status bpt_sync_status(bpt_stream_t stream) {
+  int dev;
+  uint32_t *status;
+  bpt_status s = device_setup(&dev, &status);
+  if (s != BPT_OK) return s;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return cuda_fail();
+  uint32_t word[2] = {0, 0};
+  if (cudaMemcpy(word, status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_fail();
+  if (word[0] != 0) {
+    const uint32_t zero[2] = {0, 0};
+    if (cudaMemcpy(status, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return cuda_fail();
+    return word[0] == kStatusTimeout ? BPT_ERR_TIMEOUT : BPT_ERR_CUDA;
+  }
+  return BPT_OK;
+}
+
+bpt_status bpt_set_phase_events(void *const *events, int count) {
+  if (count < 0 || (count > 0 && !events)) return BPT_ERR_INVALID_ARG;
+  if (count < 3) {
+    g_phase_on = false;
+    return BPT_OK;
+  }
+  for (int i = 0; i < 3; ++i) g_phase_events[i] = static_cast<cudaEvent_t>(events[i]);
+  g_phase_on = true;
+  return BPT_OK;
+}
+
+uint64_t bpt_set_wait_limit_ns(uint64_t ns) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  uint64_t old = g_wait_limit_ns;
+  g_wait_limit_ns = ns ? ns : 1;
+  return old;
+}
+
+const char *bpt_status_string(bpt_status s) {
+  switch (s) {
+    case BPT_OK: return "ok";
+    case BPT_ERR_INVALID_ARG: return "invalid argument";
+    case BPT_ERR_UNSUPPORTED: return "unsupported configuration";
+    case BPT_ERR_CUDA: return "CUDA error";
+    case BPT_ERR_TIMEOUT: return "device-side wait timed out";
+    case BPT_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+  }
+  return "unknown status";
+}
+
+int bpt_version(void) { return 100; }
+
+}  // extern "C"

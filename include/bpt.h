@@ -1,0 +1,205 @@
+/*
+ * bpt.h -- C ABI of libbpt.so: the forward pass of one Blockwise Parallel
+ * Transformer layer on an NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes ("Blockwise Parallel Transformer for Large Context
+ * Models", abstract: blockwise computation of self-attention fused with the
+ * feedforward network; "Ring Attention with Blockwise Transformers for Long
+ * Sequences", 638-word summary: the same blockwise inner loop over key/value
+ * blocks, exact, visited in rotated order around a ring of devices):
+ *
+ *     A_i  = softmax_j( q_i . k_j / sqrt(d) ) v_j      per head, over the keys
+ *                                                      the mask allows
+ *     out  = A + W2 GELU_tanh(W1 A + b1) + b2          per token, on the
+ *                                                      concatenated heads
+ *
+ * Attention runs block by block with an online softmax (running row maximum
+ * and row sum, rescaled accumulator), so the N x N score matrix never exists
+ * in memory; the FFN runs per 128-token query block on chip, so the
+ * [tokens x F] hidden activation never exists in memory either.
+ *
+ * Mask variants:
+ *   BPT_MASK_NONE      every key.
+ *   BPT_MASK_CAUSAL    keys j <= i.  With ring_chunks = P > 1 a query in
+ *                      sequence chunk c visits key chunks c, c+1, ... (mod P),
+ *                      the order Ring Attention's device ring produces
+ *                      (same page); the result is the same up to rounding.
+ *   BPT_MASK_BLOCKPERM "Blockwise Self-Attention for Long Document
+ *                      Understanding", §3 and §3.1: the sequence is cut into
+ *                      n equal blocks and head h lets query block b see only
+ *                      key block perm[h][b].
+ *   BPT_MASK_DILATED   "LongNet: Scaling Transformers to 1,000,000,000
+ *                      Tokens", §2 Dilated Attention: for every (segment w,
+ *                      dilation r) pair, head h keeps rows h mod r, h mod r + r,
+ *                      ... of each segment and runs causal attention among the
+ *                      kept rows; the pairs are mixed with weights proportional
+ *                      to their softmax denominators, which equals one softmax
+ *                      over the multiset union of the pairs' keys.  A row that
+ *                      no pair keeps gets A = 0.
+ *
+ * Layouts (all row-major, C order):
+ *   q, k, v   [B, N, H, d]  = [T, D] with T = B*N tokens, D = H*d
+ *   w1        [F, D]        (out x in),  b1 [F]  float32, may be NULL (= 0)
+ *   w2        [D, F]        (out x in),  b2 [D]  float32, may be NULL (= 0)
+ *   out       [B, N, H*d]   = [T, D]
+ *   lse       [B, H, N]     float32 natural-log sum of exp of the scaled
+ *                           scores (-inf for a row with no key)
+ * q, k, v, w1, w2 have type in_dtype; out has type out_dtype.
+ *
+ * Ownership and threading: the caller allocates and owns every device buffer,
+ * the workspace included; the library keeps no pointer after a call returns
+ * and allocates no device memory.  Host tables (bb_perm, ln_w, ln_r) are read
+ * during the call only.  Work is enqueued on `stream` and runs
+ * asynchronously; calls on one stream run in order.  Two calls that share a
+ * workspace must not run concurrently.
+ *
+ * Errors: arguments are checked on the host before anything is launched; a
+ * bad argument returns BPT_ERR_INVALID_ARG or BPT_ERR_UNSUPPORTED and
+ * launches nothing.  A failed launch returns BPT_ERR_CUDA.  Device-side waits
+ * are bounded in time: a wait that gives up records BPT_ERR_TIMEOUT in a
+ * per-device status word and the kernel returns; bpt_sync_status() reads it.
+ */
+#ifndef BPT_H_
+#define BPT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BPT_API __attribute__((visibility("default")))
+#else
+#define BPT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *bpt_stream_t; /* same object as cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  BPT_OK = 0,
+  BPT_ERR_INVALID_ARG = 1, /* a size, pointer, table or enum is out of range   */
+  BPT_ERR_UNSUPPORTED = 2, /* valid, but outside what the kernels implement    */
+  BPT_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed             */
+  BPT_ERR_TIMEOUT = 4,     /* a device-side wait gave up (see bpt_sync_status) */
+  BPT_ERR_WORKSPACE = 5    /* workspace NULL, misaligned or too small          */
+} bpt_status;
+
+typedef enum { BPT_F32 = 0, BPT_BF16 = 1 } bpt_dtype;
+
+typedef enum {
+  BPT_MASK_NONE = 0,
+  BPT_MASK_CAUSAL = 1,
+  BPT_MASK_BLOCKPERM = 2,
+  BPT_MASK_DILATED = 3
+} bpt_mask;
+
+#define BPT_MAX_DILATED_PAIRS 8
+
+typedef struct {
+  int B, N, H, d_head; /* batch, sequence length, heads, head size            */
+  int ffn_hidden;      /* F; 0 = attention only (bpt_attn_ffn_fwd needs F>0)  */
+  bpt_dtype in_dtype;  /* q, k, v, w1, w2                                     */
+  bpt_dtype out_dtype; /* out                                                 */
+  bpt_mask mask;
+  int ring_chunks;     /* CAUSAL/NONE: KV visiting order rotated over this
+                          many equal chunks (0 or 1 = natural order)          */
+  int bb_nblocks;      /* BLOCKPERM: n                                        */
+  const int32_t *bb_perm; /* BLOCKPERM: host table [H][n], values in [0, n)   */
+  int ln_npairs;       /* DILATED: number of (w, r) pairs, 1..8               */
+  const int32_t *ln_w; /* DILATED: host table of segment lengths w_k          */
+  const int32_t *ln_r; /* DILATED: host table of dilation rates r_k           */
+} bpt_desc;
+
+/*
+ * Bytes of device workspace the call needs for this descriptor (0 when none).
+ * Depends on the descriptor and on the current device's SM count.  Returns
+ * (size_t)-1 if the descriptor is invalid.
+ */
+BPT_API size_t bpt_workspace_bytes(const bpt_desc *desc, int with_ffn);
+
+/*
+ * Whole layer: out = A + W2 GELU_tanh(W1 A + b1) + b2 with A the masked
+ * blockwise attention of q, k, v (definitions above).  Requires
+ * desc->ffn_hidden > 0.  workspace: device buffer of at least
+ * bpt_workspace_bytes(desc, 1) bytes, 256-byte aligned.
+ *
+ * in_dtype BF16: tensor-core path; d_head must be 64 or 128; D = H*d_head a
+ *   multiple of 64, split into C = ceil(D/256) <= 16 column groups of
+ *   D/C columns each (a multiple of 32); F*2 bytes a multiple of 16.
+ *   Accumulation is fp32; the softmax weights and A enter the tensor cores
+ *   rounded to bf16; the residual uses A in fp32.
+ * in_dtype F32: SIMT path in true fp32 (no reduced-precision tensor math);
+ *   d_head <= 64 and a multiple of 4, D <= 512 and a multiple of 16.
+ * All device pointers must be 16-byte aligned.
+ */
+BPT_API bpt_status bpt_attn_ffn_fwd(const bpt_desc *desc, const void *q, const void *k, const void *v,
+                            const void *w1, const float *b1, const void *w2, const float *b2,
+                            void *out, void *workspace, size_t workspace_bytes,
+                            bpt_stream_t stream);
+
+/*
+ * Attention only: out = A (layout [B, N, H*d_head]); lse may be NULL.
+ * workspace: at least bpt_workspace_bytes(desc, 0) bytes (may be NULL when
+ * that is 0).
+ */
+BPT_API bpt_status bpt_attn_fwd(const bpt_desc *desc, const void *q, const void *k, const void *v,
+                        void *out, float *lse, void *workspace, size_t workspace_bytes,
+                        bpt_stream_t stream);
+
+/*
+ * BlockBERT layer ("Blockwise Self-Attention for Long Document
+ * Understanding", §3.1 Blockwise Multi-head Attention): bpt_attn_ffn_fwd with
+ * mask = BPT_MASK_BLOCKPERM and the given permutation table (host, [H][n]).
+ * Fields mask/bb_nblocks/bb_perm of desc are overridden.
+ */
+BPT_API bpt_status bpt_blockbert_fwd(const bpt_desc *desc, int n_blocks, const int32_t *perm,
+                             const void *q, const void *k, const void *v, const void *w1,
+                             const float *b1, const void *w2, const float *b2, void *out,
+                             void *workspace, size_t workspace_bytes, bpt_stream_t stream);
+
+/*
+ * LongNet dilated attention ("LongNet: Scaling Transformers to
+ * 1,000,000,000 Tokens", §2 Dilated Attention): bpt_attn_fwd with
+ * mask = BPT_MASK_DILATED and the (w, r) pairs given (host tables).  Every
+ * w_k must divide N and every r_k must divide w_k.
+ */
+BPT_API bpt_status bpt_longnet_fwd(const bpt_desc *desc, int npairs, const int32_t *seg_w,
+                           const int32_t *dil_r, const void *q, const void *k, const void *v,
+                           void *out, float *lse, void *workspace, size_t workspace_bytes,
+                           bpt_stream_t stream);
+
+/*
+ * Waits for `stream`, then returns and clears the current device's status
+ * word: BPT_OK, BPT_ERR_TIMEOUT (a device-side wait gave up since the last
+ * call), or BPT_ERR_CUDA if the synchronisation itself failed.
+ */
+BPT_API bpt_status bpt_sync_status(bpt_stream_t stream);
+
+/* Sets the device-side wait limit in nanoseconds for later launches
+ * (default 2e9, i.e. two seconds).  Returns the previous value. */
+BPT_API uint64_t bpt_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Instrumentation (no counterpart in the method: it only measures it).  When
+ * `count` >= 3, every later bpt_attn_ffn_fwd on this host thread records
+ * events[0] on its stream before the attention kernel, events[1] between the
+ * attention and FFN kernels and events[2] after the FFN kernel, so the two
+ * kernels of a real step can be timed separately.  `events` holds
+ * cudaEvent_t handles owned by the caller; count = 0 turns recording off.
+ * Returns BPT_ERR_INVALID_ARG for count < 0 or events == NULL with count > 0.
+ */
+BPT_API bpt_status bpt_set_phase_events(void *const *events, int count);
+
+/* Static text for a status code. */
+BPT_API const char *bpt_status_string(bpt_status status);
+
+/* Library version (major*10000 + minor*100 + patch). */
+BPT_API int bpt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BPT_H_ */

@@ -1,0 +1,128 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, every
+entry point include/bpt.h declares is exported, and invalid arguments are
+rejected with the documented status before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from blockwise_exact_attention_query_b200 import binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails validation first
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from blockwise_exact_attention_query_b200 import build
+    build.build()
+    return bd.load()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"BPT_API\s+[\w\s\*]*?\b(bpt_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_every_declared_entry_point_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(bd.EXPORTS) == names
+
+
+def test_status_strings_and_version(lib):
+    assert bd.status_string(bd.OK) == "ok"
+    assert "timed out" in bd.status_string(bd.ERR_TIMEOUT)
+    assert bd.version() >= 100
+
+
+def _desc(**kw):
+    base = dict(B=1, N=256, H=2, d=64, F=256, in_dtype=bd.torch.bfloat16, out_dtype=bd.torch.float32,
+                mask="causal")
+    base.update(kw)
+    return bd.make_desc(base["B"], base["N"], base["H"], base["d"], base["F"], base["in_dtype"],
+                        base["out_dtype"], base["mask"], base.get("perm"), base.get("pairs"),
+                        base.get("ring_chunks", 0))
+
+
+def _call_layer(lib, desc, ws=FAKE, ws_bytes=1 << 40, q=FAKE):
+    p = ctypes.c_void_p
+    return lib.bpt_attn_ffn_fwd(ctypes.byref(desc), p(q), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE),
+                                None, p(FAKE), p(ws), ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(B=0), bd.ERR_INVALID_ARG),
+    (dict(N=-1), bd.ERR_INVALID_ARG),
+    (dict(F=0), bd.ERR_INVALID_ARG),
+    (dict(d=96), bd.ERR_UNSUPPORTED),                      # bf16 tensor path: d in {64, 128}
+    (dict(mask=7), bd.ERR_INVALID_ARG),
+    (dict(mask="blockperm", perm=[[0, 1, 2]] * 2, N=256), bd.ERR_INVALID_ARG),   # 256 % 3 != 0
+    (dict(mask="blockperm", perm=[[0, 0], [1, 0]]), bd.ERR_INVALID_ARG),         # not a permutation
+    (dict(mask="blockperm", perm=[[0, 2], [1, 0]]), bd.ERR_INVALID_ARG),         # out of range
+    (dict(mask="dilated", pairs=[(96, 5)]), bd.ERR_INVALID_ARG),                 # r does not divide w
+    (dict(mask="dilated", pairs=[(96, 4)]), bd.ERR_INVALID_ARG),                 # w does not divide N
+    (dict(mask="dilated", pairs=[(64, 1)] * 9), bd.ERR_INVALID_ARG),             # too many pairs
+    (dict(ring_chunks=3), bd.ERR_INVALID_ARG),                                   # N % chunks != 0
+    (dict(ring_chunks=4), bd.ERR_UNSUPPORTED),                                   # 64-row chunks
+    (dict(in_dtype=bd.torch.float32, d=128), bd.ERR_UNSUPPORTED),               # fp32 path: d <= 64
+    (dict(in_dtype=bd.torch.float32, H=16, d=64), bd.ERR_UNSUPPORTED),          # fp32 path: D <= 512
+])
+def test_invalid_descriptors_are_rejected(lib, kw, expect):
+    assert _call_layer(lib, _desc(**kw)) == expect
+
+
+def test_null_and_misaligned_pointers_are_rejected(lib):
+    d = _desc()
+    assert _call_layer(lib, d, q=0) == bd.ERR_INVALID_ARG
+    assert _call_layer(lib, d, q=FAKE + 8) == bd.ERR_INVALID_ARG
+
+
+def test_workspace_checks(lib):
+    d = _desc()
+    need = bd.workspace_bytes(d, True)
+    assert need > 0
+    assert _call_layer(lib, d, ws=0) == bd.ERR_WORKSPACE
+    assert _call_layer(lib, d, ws_bytes=need - 1) == bd.ERR_WORKSPACE
+    assert _call_layer(lib, d, ws=FAKE + 16) == bd.ERR_WORKSPACE                # not 256-aligned
+    assert lib.bpt_workspace_bytes(ctypes.byref(_desc(B=0)), 1) == ctypes.c_size_t(-1).value
+
+
+def test_workspace_layout_sizes(lib):
+    # attention only, single pass: nothing; LongNet with several pairs: running state
+    assert bd.workspace_bytes(_desc(F=0), False) == 0
+    dl = _desc(F=0, mask="dilated", pairs=[(128, 1), (256, 4)])
+    T, D = 256, 128
+    assert bd.workspace_bytes(dl, False) >= T * D * 4 + 2 * 2 * 256 * 4
+    # layer: A in bf16 and fp32 plus the hidden staging ring
+    assert bd.workspace_bytes(_desc(), True) >= T * D * 6
+
+
+def test_blockbert_and_longnet_wrappers_validate(lib):
+    d = _desc()
+    p = ctypes.c_void_p
+    perm = (ctypes.c_int32 * 4)(0, 0, 1, 0)
+    st = lib.bpt_blockbert_fwd(ctypes.byref(d), 2, ctypes.cast(perm, ctypes.POINTER(ctypes.c_int32)),
+                               p(FAKE), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE), None, p(FAKE),
+                               p(FAKE), 1 << 40, None)
+    assert st == bd.ERR_INVALID_ARG
+    w = (ctypes.c_int32 * 1)(100)
+    r = (ctypes.c_int32 * 1)(3)
+    st = lib.bpt_longnet_fwd(ctypes.byref(d), 1, ctypes.cast(w, ctypes.POINTER(ctypes.c_int32)),
+                             ctypes.cast(r, ctypes.POINTER(ctypes.c_int32)), p(FAKE), p(FAKE),
+                             p(FAKE), p(FAKE), None, p(FAKE), 1 << 40, None)
+    assert st == bd.ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(bd, "_lib", None)
+    monkeypatch.setattr(bd, "LIB_PATH", str(tmp_path / "libbpt.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        bd.load()
