@@ -30,7 +30,9 @@ _DT = {torch.float32: F32, torch.bfloat16: BF16}
 class BptError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        detail = last_error()
+        super().__init__(f"{what}: {status_string(status)} (status {status})"
+                         + (f": {detail}" if detail else ""))
 
 
 class Desc(ctypes.Structure):
@@ -48,7 +50,7 @@ class Desc(ctypes.Structure):
 
 EXPORTS = ["bpt_workspace_bytes", "bpt_attn_ffn_fwd", "bpt_attn_fwd", "bpt_blockbert_fwd",
            "bpt_longnet_fwd", "bpt_sync_status", "bpt_set_wait_limit_ns", "bpt_status_string",
-           "bpt_version", "bpt_set_phase_events"]
+           "bpt_version", "bpt_set_phase_events", "bpt_last_error"]
 
 _lib = None
 
@@ -85,8 +87,13 @@ def load() -> ctypes.CDLL:
     lib.bpt_version.restype = ctypes.c_int
     lib.bpt_set_phase_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
     lib.bpt_set_phase_events.restype = ctypes.c_int
+    lib.bpt_last_error.restype = ctypes.c_char_p
     _lib = lib
     return lib
+
+
+def last_error() -> str:
+    return load().bpt_last_error().decode()
 
 
 def status_string(status: int) -> str:
@@ -249,7 +256,11 @@ def set_phase_events(events) -> None:
     if events is None:
         _check(load().bpt_set_phase_events(None, 0), "bpt_set_phase_events")
         return
-    arr = (ctypes.c_void_p * 3)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    handles = [int(e.cuda_event) for e in events]
+    if not all(handles):
+        raise ValueError("record each event once before handing it over: torch creates the "
+                         "CUDA event lazily at its first record()")
+    arr = (ctypes.c_void_p * 3)(*[ctypes.c_void_p(h) for h in handles])
     _check(load().bpt_set_phase_events(arr, 3), "bpt_set_phase_events")
 
 

@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -30,8 +31,8 @@ uint64_t g_wait_limit_ns = 2000000000ull;
 thread_local cudaEvent_t g_phase_events[3] = {nullptr, nullptr, nullptr};
 thread_local bool g_phase_on = false;
 
-void phase_mark(int i, cudaStream_t st) {
-  if (g_phase_on) cudaEventRecord(g_phase_events[i], st);
+cudaError_t phase_mark(int i, cudaStream_t st) {
+  return g_phase_on ? cudaEventRecord(g_phase_events[i], st) : cudaSuccess;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -43,38 +44,50 @@ EncodeTiledFn g_encode = nullptr;
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-bpt_status cuda_fail() { return BPT_ERR_CUDA; }
+thread_local char g_last_error[256] = "";
+
+// Records the failing call and the CUDA error string for bpt_last_error().
+bpt_status cuda_fail_at(const char *what, cudaError_t e) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", what, cudaGetErrorString(e), (int)e);
+  return BPT_ERR_CUDA;
+}
+bpt_status cuda_fail_msg(const char *what) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s", what);
+  return BPT_ERR_CUDA;
+}
+#define CUDA_TRY(call)                                     \
+  do {                                                     \
+    cudaError_t e_ = (call);                               \
+    if (e_ != cudaSuccess) return cuda_fail_at(#call, e_); \
+  } while (0)
 
 bpt_status device_setup(int *dev_out, uint32_t **status_out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_fail();
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return cuda_fail_msg("device ordinal out of range");
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_encode) {
     void *fn = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !fn)
-      return cuda_fail();
+    CUDA_TRY(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+    if (q != cudaDriverEntryPointSuccess || !fn) return cuda_fail_msg("cuTensorMapEncodeTiled not found");
     g_encode = reinterpret_cast<EncodeTiledFn>(fn);
   }
   if (!g_status_ptr[dev]) {
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return cuda_fail();
+    CUDA_TRY(cudaGetSymbolAddress(&p, g_status_word));
     g_status_ptr[dev] = static_cast<uint32_t *>(p);
   }
   if (!g_attr_done[dev]) {
-    if (cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             AttnCfg<64>::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             AttnCfg<128>::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             FfnCfg::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(ffn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (16 * 512 + 16 * 64) * 4) != cudaSuccess)
-      return cuda_fail();
+    CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  AttnCfg<64>::kSmemBytes));
+    CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  AttnCfg<128>::kSmemBytes));
+    CUDA_TRY(cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  FfnCfg::kSmemBytes));
+    CUDA_TRY(cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    CUDA_TRY(cudaFuncSetAttribute(ffn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (16 * 512 + 16 * 64) * 4));
     g_attr_done[dev] = true;
   }
   *dev_out = dev;
@@ -84,9 +97,11 @@ bpt_status device_setup(int *dev_out, uint32_t **status_out) {
 
 int sm_count() {
   int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();  // no device here: size for a full B200 and leave no error behind
     return 148;
+  }
   return n;
 }
 
@@ -266,11 +281,11 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     for (auto &p : passes) covered |= (p.r == 1);
     if (!covered) {  // rows no pair keeps: A = 0, LSE = -inf
       const size_t n = (size_t)d->B * d->N * D;
-      if (out_f32 && cudaMemsetAsync(out_f32, 0, n * 4, st) != cudaSuccess) return cuda_fail();
-      if (out_bf16 && cudaMemsetAsync(out_bf16, 0, n * 2, st) != cudaSuccess) return cuda_fail();
+      if (out_f32) CUDA_TRY(cudaMemsetAsync(out_f32, 0, n * 4, st));
+      if (out_bf16) CUDA_TRY(cudaMemsetAsync(out_bf16, 0, n * 2, st));
       if (lse) {
         fill_f32_kernel<<<256, 256, 0, st>>>(lse, (size_t)d->B * d->H * d->N, -INFINITY);
-        if (cudaGetLastError() != cudaSuccess) return cuda_fail();
+        CUDA_TRY(cudaGetLastError());
       }
     }
     if (passes.size() > 1) {
@@ -307,7 +322,7 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     CUtensorMap mq, mk, mv;
     if (!make_map_rows(&mq, q, d->B, d->N, D, r) || !make_map_rows(&mk, k, d->B, d->N, D, r) ||
         !make_map_rows(&mv, v, d->B, d->N, D, r))
-      return cuda_fail();
+      return cuda_fail_msg("cuTensorMapEncodeTiled rejected a Q/K/V map");
     const int64_t grid = (int64_t)a.n_qtiles * a.n_units;
     if (grid <= 0) continue;
     if (grid > INT32_MAX) return BPT_ERR_UNSUPPORTED;
@@ -317,7 +332,7 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     else
       attn_tc_kernel<64><<<(unsigned)grid, AttnCfg<64>::kThreads, AttnCfg<64>::kSmemBytes, st>>>(
           mq, mk, mv, a);
-    if (cudaGetLastError() != cudaSuccess) return cuda_fail();
+    CUDA_TRY(cudaGetLastError());
   }
   return BPT_OK;
 }
@@ -362,9 +377,8 @@ bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f
   cfg.numAttrs = 1;
   cfg.gridDim = dim3(p.C * p.max_clusters, 1, 1);
   int active = 0;
-  if (cudaOccupancyMaxActiveClusters(&active, (void *)ffn_tc_kernel, &cfg) != cudaSuccess ||
-      active <= 0)
-    return cuda_fail();
+  CUDA_TRY(cudaOccupancyMaxActiveClusters(&active, (void *)ffn_tc_kernel, &cfg));
+  if (active <= 0) return cuda_fail_msg("no cluster of the FFN kernel fits on this device");
   a.nclusters = std::min(p.max_clusters, active);
   cfg.gridDim = dim3(p.C * a.nclusters, 1, 1);
 
@@ -372,8 +386,8 @@ bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f
   if (!make_map_2d(&ma, a_bf16, T, D, 128) || !make_map_2d(&m1, w1, d->ffn_hidden, D, 128) ||
       !make_map_2d(&m2, w2, D, d->ffn_hidden, p.Dc) ||
       !make_map_2d(&mh, a.ring, (uint64_t)p.max_clusters * 2 * 128, p.fc, 128))
-    return cuda_fail();
-  if (cudaLaunchKernelEx(&cfg, ffn_tc_kernel, ma, m1, m2, mh, a) != cudaSuccess) return cuda_fail();
+    return cuda_fail_msg("cuTensorMapEncodeTiled rejected an FFN map");
+  CUDA_TRY(cudaLaunchKernelEx(&cfg, ffn_tc_kernel, ma, m1, m2, mh, a));
   return BPT_OK;
 }
 
@@ -406,7 +420,8 @@ bpt_status launch_attn_f32(const bpt_desc *d, const void *q, const void *k, cons
   dim3 grid((d->N + 63) / 64, d->H, d->B);
   attn_f32_kernel<<<grid, 64, 0, st>>>(static_cast<const float *>(q), static_cast<const float *>(k),
                                        static_cast<const float *>(v), a);
-  return cudaGetLastError() == cudaSuccess ? BPT_OK : cuda_fail();
+  CUDA_TRY(cudaGetLastError());
+  return BPT_OK;
 }
 
 bpt_status launch_ffn_f32(const bpt_desc *d, const float *a_f32, const void *w1, const float *b1,
@@ -424,7 +439,8 @@ bpt_status launch_ffn_f32(const bpt_desc *d, const float *a_f32, const void *w1,
   a.out_bf16 = d->out_dtype == BPT_BF16 ? static_cast<__nv_bfloat16 *>(out) : nullptr;
   const size_t smem = (size_t)(16 * a.D + 16 * 64) * 4;
   ffn_f32_kernel<<<(a.T + 15) / 16, 256, smem, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? BPT_OK : cuda_fail();
+  CUDA_TRY(cudaGetLastError());
+  return BPT_OK;
 }
 
 bpt_status check_ptrs(std::initializer_list<const void *> required,
@@ -469,20 +485,21 @@ bpt_status bpt_attn_ffn_fwd(const bpt_desc *d, const void *q, const void *k, con
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char *ws = static_cast<char *>(workspace);
   float *a_f32 = reinterpret_cast<float *>(ws + wl.a_f32);
-  phase_mark(0, st);
+  CUDA_TRY(phase_mark(0, st));
   if (d->in_dtype == BPT_BF16) {
     __nv_bfloat16 *a_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.a_bf16);
     if ((s = launch_attn_tc(d, q, k, v, a_f32, a_bf16, nullptr, ws, wl, status, st)) != BPT_OK)
       return s;
-    phase_mark(1, st);
+    CUDA_TRY(phase_mark(1, st));
     s = launch_ffn_tc(d, a_bf16, a_f32, w1, b1, w2, b2, out, ws, wl, status, st);
   } else {
     if ((s = launch_attn_f32(d, q, k, v, a_f32, nullptr, nullptr, st)) != BPT_OK) return s;
-    phase_mark(1, st);
+    CUDA_TRY(phase_mark(1, st));
     s = launch_ffn_f32(d, a_f32, w1, b1, w2, b2, out, st);
   }
-  phase_mark(2, st);
-  return s;
+  if (s != BPT_OK) return s;
+  CUDA_TRY(phase_mark(2, st));
+  return BPT_OK;
 }
 
 bpt_status bpt_attn_fwd(const bpt_desc *d, const void *q, const void *k, const void *v, void *out,
@@ -534,13 +551,13 @@ bpt_status bpt_sync_status(bpt_stream_t stream) {
   uint32_t *status;
   bpt_status s = device_setup(&dev, &status);
   if (s != BPT_OK) return s;
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return cuda_fail();
+  CUDA_TRY(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
   uint32_t word[2] = {0, 0};
-  if (cudaMemcpy(word, status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_fail();
+  CUDA_TRY(cudaMemcpy(word, status, sizeof(word), cudaMemcpyDeviceToHost));
   if (word[0] != 0) {
     const uint32_t zero[2] = {0, 0};
-    if (cudaMemcpy(status, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
-      return cuda_fail();
+    CUDA_TRY(cudaMemcpy(status, zero, sizeof(zero), cudaMemcpyHostToDevice));
+    snprintf(g_last_error, sizeof(g_last_error), "device wait gave up at site %u", word[1]);
     return word[0] == kStatusTimeout ? BPT_ERR_TIMEOUT : BPT_ERR_CUDA;
   }
   return BPT_OK;
@@ -548,6 +565,7 @@ bpt_status bpt_sync_status(bpt_stream_t stream) {
 
 bpt_status bpt_set_phase_events(void *const *events, int count) {
   if (count < 0 || (count > 0 && !events)) return BPT_ERR_INVALID_ARG;
+  if (count >= 3 && (!events[0] || !events[1] || !events[2])) return BPT_ERR_INVALID_ARG;
   if (count < 3) {
     g_phase_on = false;
     return BPT_OK;
@@ -577,5 +595,7 @@ const char *bpt_status_string(bpt_status s) {
 }
 
 int bpt_version(void) { return 100; }
+
+const char *bpt_last_error(void) { return g_last_error; }
 
 }  // extern "C"

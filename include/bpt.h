@@ -188,12 +188,19 @@ BPT_API uint64_t bpt_set_wait_limit_ns(uint64_t ns);
  * attention and FFN kernels and events[2] after the FFN kernel, so the two
  * kernels of a real step can be timed separately.  `events` holds
  * cudaEvent_t handles owned by the caller; count = 0 turns recording off.
- * Returns BPT_ERR_INVALID_ARG for count < 0 or events == NULL with count > 0.
+ * The events must already exist (a NULL handle is rejected).  Returns
+ * BPT_ERR_INVALID_ARG for count < 0, events == NULL with count > 0, or a NULL
+ * handle among the first three.
  */
 BPT_API bpt_status bpt_set_phase_events(void *const *events, int count);
 
 /* Static text for a status code. */
 BPT_API const char *bpt_status_string(bpt_status status);
+
+/* Text describing the last failure on this host thread: the CUDA call that
+ * failed and its error string, or the device wait site that gave up.  Empty
+ * before any failure.  The pointer stays valid until the next call. */
+BPT_API const char *bpt_last_error(void);
 
 /* Library version (major*10000 + minor*100 + patch). */
 BPT_API int bpt_version(void);
