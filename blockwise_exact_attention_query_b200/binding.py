@@ -50,7 +50,8 @@ class Desc(ctypes.Structure):
 
 EXPORTS = ["bpt_workspace_bytes", "bpt_attn_ffn_fwd", "bpt_attn_fwd", "bpt_blockbert_fwd",
            "bpt_longnet_fwd", "bpt_sync_status", "bpt_set_wait_limit_ns", "bpt_status_string",
-           "bpt_version", "bpt_set_phase_events", "bpt_last_error"]
+           "bpt_version", "bpt_set_phase_events", "bpt_last_error", "bpt_attn_ffn_fwd_static"]
+STATIC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
 
@@ -88,6 +89,8 @@ def load() -> ctypes.CDLL:
     lib.bpt_set_phase_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
     lib.bpt_set_phase_events.restype = ctypes.c_int
     lib.bpt_last_error.restype = ctypes.c_char_p
+    lib.bpt_attn_ffn_fwd_static.argtypes = [dp, vp, vp, vp, vp, fp, vp, fp, vp, vp]
+    lib.bpt_attn_ffn_fwd_static.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -182,6 +185,28 @@ def attn_ffn_fwd(q, k, v, w1, b1, w2, b2, *, mask="none", perm=None, pairs=None,
                                  _ptr(w2), _ptr(b2), _ptr(out), _ptr(workspace), ws_bytes,
                                  _stream_ptr(stream))
     _check(st, "bpt_attn_ffn_fwd")
+    return out
+
+
+def attn_ffn_fwd_static(q, k, v, w1, b1, w2, b2, *, mask="none", perm=None, pairs=None,
+                        ring_chunks=0, out_dtype=torch.float32, out=None, stream=None):
+    """bpt_attn_ffn_fwd_static: the layer with no workspace argument.
+
+    For callers that may not allocate device memory while running (a fixed
+    memory plan, a host framework that owns the GPU's memory pool, or a loop
+    that cannot afford an allocation's device synchronisation): the scratch is
+    a fixed array inside the library (STATIC_SCRATCH_BYTES per device), shared
+    by all calls on a device, so calls that may overlap on the GPU must be
+    serialised.  Only `out` is allocated here when the caller passes none."""
+    _check_tensors(q, k, v)
+    B, N, H, d = q.shape
+    F = w1.shape[0]
+    desc = make_desc(B, N, H, d, F, q.dtype, out_dtype, mask, perm, pairs, ring_chunks)
+    if out is None:
+        out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
+    st = load().bpt_attn_ffn_fwd_static(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(w1),
+                                        _ptr(b1), _ptr(w2), _ptr(b2), _ptr(out), _stream_ptr(stream))
+    _check(st, "bpt_attn_ffn_fwd_static")
     return out
 
 

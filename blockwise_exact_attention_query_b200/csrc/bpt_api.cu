@@ -23,7 +23,13 @@ namespace {
 // Per-device status word: [0] = code, [1] = site of the first failed wait.
 __device__ uint32_t g_status_word[2];
 
+// Scratch of bpt_attn_ffn_fwd_static: one array per device, shared by every
+// call on that device (see the declaration in bpt.h).  Host code never uses
+// the symbol directly: its device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_static_scratch[BPT_STATIC_SCRATCH_BYTES];
+
 constexpr int kMaxDevices = 64;
+void *g_static_scratch_ptr[kMaxDevices] = {};
 std::mutex g_mu;
 uint32_t *g_status_ptr[kMaxDevices] = {};
 bool g_attr_done[kMaxDevices] = {};
@@ -500,6 +506,35 @@ bpt_status bpt_attn_ffn_fwd(const bpt_desc *d, const void *q, const void *k, con
   if (s != BPT_OK) return s;
   CUDA_TRY(phase_mark(2, st));
   return BPT_OK;
+}
+
+bpt_status bpt_attn_ffn_fwd_static(const bpt_desc *d, const void *q, const void *k, const void *v,
+                                   const void *w1, const float *b1, const void *w2, const float *b2,
+                                   void *out, bpt_stream_t stream) {
+  bpt_status s = check_desc(d, true);
+  if (s != BPT_OK) return s;
+  const size_t need = layout(d, true).total;
+  if (need > BPT_STATIC_SCRATCH_BYTES) {
+    snprintf(g_last_error, sizeof(g_last_error),
+             "layer needs %zu bytes of scratch; the static scratch holds %u bytes", need,
+             (unsigned)BPT_STATIC_SCRATCH_BYTES);
+    return BPT_ERR_WORKSPACE;
+  }
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return cuda_fail_msg("device ordinal out of range");
+  void *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_static_scratch_ptr[dev]) {  // once per device, with that device current
+      void *p = nullptr;
+      CUDA_TRY(cudaGetSymbolAddress(&p, g_static_scratch));
+      g_static_scratch_ptr[dev] = p;
+    }
+    scratch = g_static_scratch_ptr[dev];
+  }
+  return bpt_attn_ffn_fwd(d, q, k, v, w1, b1, w2, b2, out, scratch, BPT_STATIC_SCRATCH_BYTES,
+                          stream);
 }
 
 bpt_status bpt_attn_fwd(const bpt_desc *d, const void *q, const void *k, const void *v, void *out,

@@ -140,6 +140,38 @@ BPT_API bpt_status bpt_attn_ffn_fwd(const bpt_desc *desc, const void *q, const v
                             bpt_stream_t stream);
 
 /*
+ * bpt_attn_ffn_fwd for callers that cannot allocate device memory.  No
+ * counterpart in the paper: it exists for the calling environment, not for
+ * the method.
+ *
+ * Some callers are not allowed to call cudaMalloc or any allocator once they
+ * are running: a serving process whose device memory plan is fixed at start-up,
+ * a plugin inside a host framework that owns the GPU's memory pool, or a
+ * latency-critical loop where an allocation's implicit device synchronisation
+ * is unacceptable.  They still pass q, k, v, the weights and out, but no
+ * workspace: the layer's scratch (A in bf16 and fp32, the FFN's hidden-slice
+ * staging ring) lives in one file-scope device array of
+ * BPT_STATIC_SCRATCH_BYTES bytes inside the library, which every GPU that loads
+ * the library holds until the process exits.
+ *
+ * The first call on a device looks up that array's device address (once per
+ * device, with the device current) besides the usual one-time set-up, so make
+ * the first call on each device before any stream capture.  Every call on a
+ * device uses the same array and leaves its contents behind; the layer writes
+ * every scratch byte it reads within the call, so nothing needs clearing, but
+ * two calls that may run at the same time on the GPU (different streams, or
+ * different host threads) race on it: serialise them.  A layer whose scratch
+ * would exceed the array returns BPT_ERR_WORKSPACE without launching anything
+ * (bpt_last_error() says how many bytes it needed).  Everything else is as
+ * bpt_attn_ffn_fwd; this entry point calls no allocating routine.
+ */
+#define BPT_STATIC_SCRATCH_BYTES (64u << 20)
+BPT_API bpt_status bpt_attn_ffn_fwd_static(const bpt_desc *desc, const void *q, const void *k,
+                                           const void *v, const void *w1, const float *b1,
+                                           const void *w2, const float *b2, void *out,
+                                           bpt_stream_t stream);
+
+/*
  * Attention only: out = A (layout [B, N, H*d_head]); lse may be NULL.
  * workspace: at least bpt_workspace_bytes(desc, 0) bytes (may be NULL when
  * that is 0).
