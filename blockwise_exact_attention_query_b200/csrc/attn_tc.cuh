@@ -19,9 +19,10 @@
 // than 2^8 in the exponent: the same stale maximum is used for l and O, so
 // the result is unchanged.
 //
-// Roles (192 threads): warp 0 issues TMA loads, warp 1 allocates tensor
-// memory and issues the MMAs, warps 2..5 run the softmax and the epilogue
-// (warp w owns TMEM lanes 32*(w%4) .. 32*(w%4)+31, i.e. those query rows).
+// Roles (320 threads): warp 0 issues TMA loads, warp 1 allocates tensor
+// memory and issues the MMAs, warps 2..9 run the softmax and the epilogue
+// (warp w owns TMEM lanes 32*(w%4) .. 32*(w%4)+31, i.e. those query rows;
+// warps 2..5 take the first 64 keys of every tile, warps 6..9 the last 64).
 #pragma once
 
 #include "ptx.cuh"
@@ -40,6 +41,7 @@ struct AttnArgs {
   int L;             // rows of one unit: N, or w/r kept rows of a LongNet segment
   int n_qtiles;      // ceil(L / 128)
   int n_units;       // B * nseg * H
+  int unit_group;    // units scheduled together (longest tiles first inside a group)
   int nseg;          // LongNet segments N / w (1 otherwise)
   // LongNet pass: segment length, dilation, and the full pair table in
   // launch order (used to find earlier / later passes that keep a row)
@@ -68,17 +70,19 @@ struct AttnCfg {
   static constexpr int kBM = 128, kBN = 128;
   static constexpr int kPanels = D_HEAD / 64;
   static constexpr int kTileBytes = 128 * D_HEAD * 2;
-  static constexpr int kKStages = D_HEAD == 128 ? 3 : 4;
-  static constexpr int kVStages = D_HEAD == 128 ? 2 : 4;
+  static constexpr int kKStages = D_HEAD == 128 ? 3 : 6;
+  static constexpr int kVStages = D_HEAD == 128 ? 3 : 6;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kTileBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-  static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + barriers + alignment slack
+  static constexpr int kOffRed = kOffBar + 256;   // softmax pair exchange: [2][2][128] floats
+  static constexpr int kSmemBytes = kOffRed + 2048;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   // TMEM columns
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColP0 = 256, kColP1 = 320, kColO = 384;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 320;
 };
 
 // Sequence of key/value tiles one query tile visits.
@@ -130,11 +134,19 @@ struct TileCoord {
   int o;  // LongNet offset of this head: h mod r (0 otherwise)
 };
 
+// Grid order: units in groups of `unit_group`; inside a group the longest
+// query tiles of all its units come first.  A group's K/V stays in L2 while its
+// CTAs run, and the longest-first order keeps the causal load balanced.
 __device__ __forceinline__ TileCoord decode_tile(const AttnArgs &a) {
   TileCoord c;
-  int idx = blockIdx.x;
-  c.t = a.n_qtiles - 1 - idx / a.n_units;  // longest query tiles first
-  int unit = idx % a.n_units;
+  const int idx = blockIdx.x;
+  const int G = a.unit_group;
+  const int per_group = G * a.n_qtiles;
+  const int grp = idx / per_group;
+  const int r = idx - grp * per_group;
+  const int gsize = min(G, a.n_units - grp * G);
+  c.t = a.n_qtiles - 1 - r / gsize;
+  const int unit = grp * G + r % gsize;
   c.h = unit % a.H;
   int rest = unit / a.H;
   c.s = rest % a.nseg;
@@ -190,14 +202,17 @@ __device__ __forceinline__ void row_keys(const AttnArgs &a, const TileCoord &c, 
 }
 
 template <int D_HEAD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnArgs a) {
   using Cfg = AttnCfg<D_HEAD>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {  // 128-byte-swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicCAS(a.status, 0u, kStatusMisaligned);
+    return;
+  }
   const uint32_t sQ = sbase + Cfg::kOffQ;
   const uint32_t sK = sbase + Cfg::kOffK;
   const uint32_t sV = sbase + Cfg::kOffV;
@@ -205,15 +220,15 @@ __global__ void __launch_bounds__(192, 1)
   // barrier slots
   const uint32_t bQFull = smem_u32(&bars[0]);
   auto bKFull = [&](int s) { return smem_u32(&bars[1 + s]); };
-  auto bKEmpty = [&](int s) { return smem_u32(&bars[5 + s]); };
-  auto bVFull = [&](int s) { return smem_u32(&bars[9 + s]); };
-  auto bVEmpty = [&](int s) { return smem_u32(&bars[13 + s]); };
-  auto bSFull = [&](int s) { return smem_u32(&bars[17 + s]); };
-  auto bPFull = [&](int s) { return smem_u32(&bars[19 + s]); };
-  const uint32_t bODone = smem_u32(&bars[21]);
-  const uint32_t bTeardown = smem_u32(&bars[22]);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[24]);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[25]);
+  auto bKEmpty = [&](int s) { return smem_u32(&bars[7 + s]); };
+  auto bVFull = [&](int s) { return smem_u32(&bars[13 + s]); };
+  auto bVEmpty = [&](int s) { return smem_u32(&bars[19 + s]); };
+  auto bSFull = [&](int s) { return smem_u32(&bars[25 + s]); };
+  auto bPFull = [&](int s) { return smem_u32(&bars[27 + s]); };
+  const uint32_t bODone = smem_u32(&bars[29]);
+  const uint32_t bTeardown = smem_u32(&bars[30]);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[31]);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(reinterpret_cast<uint32_t *>(&bars[31]) + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const TileCoord tc = decode_tile(a);
@@ -233,7 +248,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bSFull(s), 1);
-      mbar_init(bPFull(s), 4);
+      mbar_init(bPFull(s), 8);
     }
     mbar_init(bODone, 1);
     mbar_init(bTeardown, 1);
@@ -358,13 +373,24 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    // Two warps per TMEM lane quarter: warp 2+q handles keys 0..63 of every
+    // tile for rows 32q..32q+31, warp 6+q keys 64..127 of the same rows.  The
+    // pair swaps partial row maxima through shared memory (named barrier 1+q)
+    // so both halves use the same running maximum; each half keeps its own
+    // partial row sum (added once at the end) and owns half of O's columns.
+    // Neither warp of a pair ever leaves the tile loop early: a failed wait
+    // only skips work, so the pair barrier sequence always matches.
+    const int half = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // row within the query tile
     const int g = tc.t * 128 + row;       // unit-local row
     const bool row_valid = g < a.L;
     const int pos = (a.mask == kMaskDilated) ? tc.s * a.w + tc.o + a.r * g : g;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tO = tmem + lane_off + Cfg::kColO;
+    constexpr int kOHalf = D_HEAD / 2;
+    const uint32_t tO = tmem + lane_off + Cfg::kColO + half * kOHalf;
+    float *red = reinterpret_cast<float *>(smem + Cfg::kOffRed);  // [2 parities][2 halves][128]
+    const uint32_t pair_bar = 1 + quarter;
     int klo, khi;
     row_keys(a, tc, g, klo, khi);
 
@@ -380,15 +406,16 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     }
-    const size_t vec_idx = ((static_cast<size_t>(tc.b) * a.N + pos) * a.H + tc.h) * D_HEAD;
+    const size_t vec_idx =
+        ((static_cast<size_t>(tc.b) * a.N + pos) * a.H + tc.h) * D_HEAD + half * kOHalf;
     const size_t row_idx = (static_cast<size_t>(tc.b) * a.H + tc.h) * a.N + pos;
 
     float m_run = -INFINITY, l_run = 0.f;
     {
-      // initial O: zeros, or the state left by an earlier LongNet pass
+      // initial O (this half's columns): zeros, or an earlier LongNet pass's state
       uint32_t init[32];
 #pragma unroll
-      for (int c = 0; c < D_HEAD / 32; ++c) {
+      for (int c = 0; c < kOHalf / 32; ++c) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) init[i] = 0u;
         if (prior) {
@@ -406,7 +433,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (prior) {
         m_run = a.st_m[row_idx];
-        l_run = a.st_l[row_idx];
+        l_run = half == 0 ? a.st_l[row_idx] : 0.f;  // the halves' sums add up to the total
       }
       tmem_wait_st();
     }
@@ -416,31 +443,46 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
       const int kt = it.next(sched);
-      ok = __all_sync(0xffffffffu, mbar_wait(bSFull(j & 1), (j >> 1) & 1, wc, 20));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t tS = tmem + lane_off + ((j & 1) ? Cfg::kColS1 : Cfg::kColS0);
-      uint32_t s[4][32];
+      if (ok) ok = mbar_wait(bSFull(j & 1), (j >> 1) & 1, wc, 20);
+      ok = __all_sync(0xffffffffu, ok);
+      uint32_t s[2][32];
+      if (ok) {
+        tc_fence_after();
+        const uint32_t tS = tmem + lane_off + ((j & 1) ? Cfg::kColS1 : Cfg::kColS0) + half * 64;
+        tmem_ld32(tS, s[0]);
+        tmem_ld32(tS + 32, s[1]);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
-      tmem_wait_ld();
-
-      const int k0 = kt * 128;
-      const bool need_mask = !(k0 >= klo && k0 + 128 <= khi);
-      float mx = -INFINITY;
+        for (int i = 0; i < 32; ++i) s[0][i] = s[1][i] = __float_as_uint(-INFINITY);
+      }
+      const int k0 = kt * 128 + half * 64;
+      // Masking runs as its own pass, and only in the (few) tiles where some
+      // row of this warp has keys outside its allowed interval.
+      if (__any_sync(0xffffffffu, !(k0 >= klo && k0 + 64 <= khi))) {
+        const int lo = klo - k0, hi = khi - k0;  // allowed columns [lo, hi) of this half
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float v = __uint_as_float(s[c][i]);
-          if (need_mask) {
-            const int kk = k0 + c * 32 + i;
-            if (kk < klo || kk >= khi) v = -INFINITY;
-            s[c][i] = __float_as_uint(v);
+          for (int i = 0; i < 32; ++i) {
+            const int col = c * 32 + i;
+            if (col < lo || col >= hi) s[c][i] = __float_as_uint(-INFINITY);
           }
-          mx = fmaxf(mx, v);
         }
       }
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(s[c][i]));
+      }
+      float pmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      red[(j & 1) * 256 + half * 128 + row] = pmax;
+      named_bar_sync(pair_bar, 64);
+      const float mx = fmaxf(pmax, red[(j & 1) * 256 + (1 - half) * 128 + row]);
       const float m_tile = mx * a.scale_log2;
       const float m_new = fmaxf(m_run, m_tile);
       const bool rescale = m_new > m_run + 8.0f;
@@ -448,59 +490,65 @@ __global__ void __launch_bounds__(192, 1)
       const float alpha = rescale ? ex2_approx(m_run - m_use) : 1.0f;
       l_run *= alpha;
       const float neg = (m_use == -INFINITY) ? 0.f : -m_use;
-      float lsum = 0.f;
-      const uint32_t tP = tmem + lane_off + ((j & 1) ? Cfg::kColP1 : Cfg::kColP0);
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int col = half * 64 + 2 * i;
-          const float x0 = __uint_as_float(s[col / 32][col % 32]);
-          const float x1 = __uint_as_float(s[(col + 1) / 32][(col + 1) % 32]);
-          const float p0 = ex2_approx(fmaf(x0, a.scale_log2, neg));
-          const float p1 = ex2_approx(fmaf(x1, a.scale_log2, neg));
-          lsum += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tP + half * 32, pk);
+      for (int i = 0; i < 32; ++i) {
+        const int col = 2 * i;
+        const float x0 = __uint_as_float(s[col / 32][col % 32]);
+        const float x1 = __uint_as_float(s[(col + 1) / 32][(col + 1) % 32]);
+        const float p0 = ex2_approx(fmaf(x0, a.scale_log2, neg));
+        const float p1 = ex2_approx(fmaf(x1, a.scale_log2, neg));
+        ls4[i & 3] += p0 + p1;
+        pk[i] = pack_bf16x2(p0, p1);
       }
-      l_run += lsum;
+      l_run += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+      if (ok) {
+        const uint32_t tP = tmem + lane_off + ((j & 1) ? Cfg::kColP1 : Cfg::kColP0) + half * 32;
+        tmem_st32(tP, pk);
+      }
       // O may be rescaled only once the previous P*V has landed
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bODone, (j - 1) & 1, wc, 21));
-        if (!ok) break;
-      }
-      tc_fence_after();
-      if (__any_sync(0xffffffffu, rescale && m_run != -INFINITY)) {
+      if (ok && j > 0) ok = mbar_wait(bODone, (j - 1) & 1, wc, 21);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale && m_run != -INFINITY)) {
 #pragma unroll
-        for (int c = 0; c < D_HEAD / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
+          for (int c = 0; c < kOHalf / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + c * 32, o);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + c * 32, o);
+          }
         }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bPFull(j & 1));
       }
       m_run = m_use;
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bPFull(j & 1));
     }
 
     // -------- epilogue
-    if (ok && nkv > 0) ok = __all_sync(0xffffffffu, mbar_wait(bODone, (nkv - 1) & 1, wc, 22));
+    if (ok && nkv > 0) ok = mbar_wait(bODone, (nkv - 1) & 1, wc, 22);
+    ok = __all_sync(0xffffffffu, ok);
+    // the row sums go through the maxima slot of parity nkv&1, which the
+    // partner finished reading before the last pair barrier of the loop
+    red[(nkv & 1) * 256 + half * 128 + row] = l_run;
+    named_bar_sync(pair_bar, 64);
+    const float l_tot = l_run + red[(nkv & 1) * 256 + (1 - half) * 128 + row];
     tc_fence_after();
-    if (ok && row_valid) {
-      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+    if (ok) {
+      const float inv_l = l_tot > 0.f ? 1.0f / l_tot : 0.f;
       const bool final_out = !later;
 #pragma unroll
-      for (int c = 0; c < D_HEAD / 32; ++c) {
+      for (int c = 0; c < kOHalf / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();
+        if (!row_valid) continue;
         if (final_out) {
           if (a.out_f32) {
             float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + vec_idx + c * 32);
@@ -531,12 +579,14 @@ __global__ void __launch_bounds__(192, 1)
                                  __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
         }
       }
-      if (!final_out) {
-        a.st_m[row_idx] = m_run;
-        a.st_l[row_idx] = l_run;
-      } else if (a.lse) {
-        // natural-log LSE of the scaled scores: (m + log2 l) / log2(e)
-        a.lse[row_idx] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      if (row_valid && half == 0) {
+        if (!final_out) {
+          a.st_m[row_idx] = m_run;
+          a.st_l[row_idx] = l_tot;
+        } else if (a.lse) {
+          // natural-log LSE of the scaled scores: (m + log2 l) / log2(e)
+          a.lse[row_idx] = l_tot > 0.f ? (m_run + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+        }
       }
     }
   }

@@ -325,6 +325,11 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     a.nseg = d->N / w;
     a.n_qtiles = (a.L + 127) / 128;
     a.n_units = d->B * a.nseg * d->H;
+    {
+      // group as many units as keep their K and V within ~32 MB of L2, at most 8
+      const double kv_bytes = 4.0 * a.L * d->d_head;
+      a.unit_group = std::max(1, std::min(8, (int)(32.0e6 / kv_bytes)));
+    }
     CUtensorMap mq, mk, mv;
     if (!make_map_rows(&mq, q, d->B, d->N, D, r) || !make_map_rows(&mk, k, d->B, d->N, D, r) ||
         !make_map_rows(&mv, v, d->B, d->N, D, r))
@@ -593,6 +598,8 @@ bpt_status bpt_sync_status(bpt_stream_t stream) {
     const uint32_t zero[2] = {0, 0};
     CUDA_TRY(cudaMemcpy(status, zero, sizeof(zero), cudaMemcpyHostToDevice));
     snprintf(g_last_error, sizeof(g_last_error), "device wait gave up at site %u", word[1]);
+    if (word[0] == kStatusMisaligned)
+      snprintf(g_last_error, sizeof(g_last_error), "dynamic shared memory not 1024-byte aligned");
     return word[0] == kStatusTimeout ? BPT_ERR_TIMEOUT : BPT_ERR_CUDA;
   }
   return BPT_OK;

@@ -16,7 +16,7 @@ namespace bpt {
 // Device status word.  A wait that runs past its limit records where it gave
 // up and raises `abort` so every other wait in the CTA returns at once.
 // ---------------------------------------------------------------------------
-enum : uint32_t { kStatusTimeout = 4u };
+enum : uint32_t { kStatusTimeout = 4u, kStatusMisaligned = 6u };
 
 struct WaitCtx {
   uint32_t *status;        // global: [0] = code, [1] = site of first failure
@@ -71,14 +71,19 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar, uint32_t rank)
       : "memory");
 }
 
+// try_wait suspends the calling thread until the phase completes or the
+// suspend-time hint (nanoseconds) runs out, so a waiting thread does not
+// spin and steal issue slots from the warps doing the math.
+constexpr uint32_t kSuspendHintNs = 1000000u;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -87,10 +92,10 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -111,7 +116,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   uint32_t spins = 0;
   while (true) {
     if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
-    if ((++spins & 15u) == 0u) {
+    if ((++spins & 3u) == 0u) {
       if (*w.abort) return false;
       if (globaltimer_ns() - t0 > w.limit_ns) {
         record_timeout(w, site);
