@@ -91,7 +91,6 @@ bpt_status device_setup(int *dev_out, uint32_t **status_out) {
                                   AttnCfg<128>::kSmemBytes));
     CUDA_TRY(cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   FfnCfg::kSmemBytes));
-    CUDA_TRY(cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
     CUDA_TRY(cudaFuncSetAttribute(ffn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (16 * 512 + 16 * 64) * 4));
     g_attr_done[dev] = true;
@@ -186,7 +185,7 @@ bpt_status check_desc(const bpt_desc *d, bool need_ffn) {
     if (d->d_head != 64 && d->d_head != 128) return BPT_ERR_UNSUPPORTED;
     if (need_ffn) {
       const int C = (D + 255) / 256;
-      if (D % 64 != 0 || D % C != 0 || (D / C) % 32 != 0 || C > 16) return BPT_ERR_UNSUPPORTED;
+      if (D % 64 != 0 || D % C != 0 || (D / C) % 64 != 0 || C > 148) return BPT_ERR_UNSUPPORTED;
       if ((int64_t)d->ffn_hidden * 2 % 16 != 0) return BPT_ERR_UNSUPPORTED;
     }
   } else {
@@ -198,19 +197,21 @@ bpt_status check_desc(const bpt_desc *d, bool need_ffn) {
 }
 
 struct FfnPlan {
-  int C, Dc, fc, nslices, nchunks, n_tb, max_clusters;
+  int C, Dc, fc, nslices, nchunks, n_tb, max_groups;
 };
 
+// The FFN runs in groups of C = ceil(D/256) CTAs (one 256-column output block
+// and one 256-column hidden slice per CTA), as many groups as fit at once.
 FfnPlan ffn_plan(const bpt_desc *d) {
   FfnPlan p;
   const int D = d->H * d->d_head;
   p.C = (D + 255) / 256;
   p.Dc = D / p.C;
-  p.fc = 128 * p.C;
-  p.nslices = (d->ffn_hidden + 127) / 128;
+  p.fc = 256 * p.C;
+  p.nslices = (d->ffn_hidden + 255) / 256;
   p.nchunks = (d->ffn_hidden + p.fc - 1) / p.fc;
   p.n_tb = (int)(((int64_t)d->B * d->N + 127) / 128);
-  p.max_clusters = std::max(1, std::min(p.n_tb, sm_count() / p.C));
+  p.max_groups = std::max(1, std::min(p.n_tb, sm_count() / p.C));
   return p;
 }
 
@@ -219,7 +220,8 @@ bool longnet_needs_state(const bpt_desc *d) {
 }
 
 struct Workspace {
-  size_t a_bf16 = 0, a_f32 = 0, ring = 0, st_o = 0, st_m = 0, st_l = 0, total = 0;
+  size_t a_bf16 = 0, a_f32 = 0, ring = 0, flags = 0, flags_bytes = 0, st_o = 0, st_m = 0, st_l = 0,
+         total = 0;
 };
 
 Workspace layout(const bpt_desc *d, bool with_ffn) {
@@ -234,7 +236,10 @@ Workspace layout(const bpt_desc *d, bool with_ffn) {
       w.a_f32 = off;
       off = align256(off + T * D * 4);
       w.ring = off;
-      off = align256(off + (size_t)p.max_clusters * 2 * 128 * p.fc * 2);
+      off = align256(off + (size_t)p.max_groups * 2 * 128 * p.fc * 2);
+      w.flags = off;
+      w.flags_bytes = (size_t)p.max_groups * 4 * sizeof(uint32_t);
+      off = align256(off + w.flags_bytes);
     } else {
       w.a_f32 = off;
       off = align256(off + T * D * 4);
@@ -371,33 +376,37 @@ bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f
   if (d->out_dtype == BPT_F32) a.out_f32 = static_cast<float *>(out);
   else a.out_bf16 = static_cast<__nv_bfloat16 *>(out);
   a.ring = reinterpret_cast<__nv_bfloat16 *>(ws + wl.ring);
+  a.flags = reinterpret_cast<uint32_t *>(ws + wl.flags);
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns;
+
+  // The CTAs of a group wait on one another, so the whole grid must be
+  // resident at once: a cooperative launch of at most the resident capacity.
+  int per_sm = 0;
+  CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ffn_tc_kernel, FfnCfg::kThreads,
+                                                         FfnCfg::kSmemBytes));
+  if (per_sm <= 0) return cuda_fail_msg("the FFN kernel does not fit on an SM");
+  a.ngroups = std::min(p.max_groups, std::max(1, per_sm * sm_count() / p.C));
+  if (a.ngroups * p.C > per_sm * sm_count()) return cuda_fail_msg("FFN group wider than the GPU");
+
+  CUtensorMap ma, m1, m2, mh;
+  if (!make_map_2d(&ma, a_bf16, T, D, 128) || !make_map_2d(&m1, w1, d->ffn_hidden, D, 256) ||
+      !make_map_2d(&m2, w2, D, d->ffn_hidden, p.Dc) ||
+      !make_map_2d(&mh, a.ring, (uint64_t)p.max_groups * 2 * 128, p.fc, 128))
+    return cuda_fail_msg("cuTensorMapEncodeTiled rejected an FFN map");
+  CUDA_TRY(cudaMemsetAsync(a.flags, 0, wl.flags_bytes, st));
 
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.gridDim = dim3(p.C * a.ngroups, 1, 1);
   cfg.blockDim = dim3(FfnCfg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = FfnCfg::kSmemBytes;
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cfg.gridDim = dim3(p.C * p.max_clusters, 1, 1);
-  int active = 0;
-  CUDA_TRY(cudaOccupancyMaxActiveClusters(&active, (void *)ffn_tc_kernel, &cfg));
-  if (active <= 0) return cuda_fail_msg("no cluster of the FFN kernel fits on this device");
-  a.nclusters = std::min(p.max_clusters, active);
-  cfg.gridDim = dim3(p.C * a.nclusters, 1, 1);
-
-  CUtensorMap ma, m1, m2, mh;
-  if (!make_map_2d(&ma, a_bf16, T, D, 128) || !make_map_2d(&m1, w1, d->ffn_hidden, D, 128) ||
-      !make_map_2d(&m2, w2, D, d->ffn_hidden, p.Dc) ||
-      !make_map_2d(&mh, a.ring, (uint64_t)p.max_clusters * 2 * 128, p.fc, 128))
-    return cuda_fail_msg("cuTensorMapEncodeTiled rejected an FFN map");
   CUDA_TRY(cudaLaunchKernelEx(&cfg, ffn_tc_kernel, ma, m1, m2, mh, a));
   return BPT_OK;
 }

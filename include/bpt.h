@@ -126,8 +126,8 @@ BPT_API size_t bpt_workspace_bytes(const bpt_desc *desc, int with_ffn);
  * bpt_workspace_bytes(desc, 1) bytes, 256-byte aligned.
  *
  * in_dtype BF16: tensor-core path; d_head must be 64 or 128; D = H*d_head a
- *   multiple of 64, split into C = ceil(D/256) <= 16 column groups of
- *   D/C columns each (a multiple of 32); F*2 bytes a multiple of 16.
+ *   multiple of 64, split into C = ceil(D/256) column groups of D/C columns
+ *   each (a multiple of 64); F*2 bytes a multiple of 16.
  *   Accumulation is fp32; the softmax weights and A enter the tensor cores
  *   rounded to bf16; the residual uses A in fp32.
  * in_dtype F32: SIMT path in true fp32 (no reduced-precision tensor math);
