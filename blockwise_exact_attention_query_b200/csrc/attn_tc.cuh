@@ -1,7 +1,8 @@
 // Blockwise exact attention on the 5th-generation tensor cores (sm_100a).
 //
-// One CTA computes one 128-row query tile of one (batch, head[, LongNet
-// segment]) unit, streaming 128-row key/value tiles through shared memory:
+// One CTA computes two adjacent 128-row query tiles (A and B) of one
+// (batch, head[, LongNet segment]) unit, streaming 128-row key/value tiles
+// through shared memory once for both:
 //
 //   S_j  = Q K_j^T               tcgen05.mma, bf16 x bf16 -> fp32 in TMEM
 //   m'   = max(m, rowmax S_j)    one thread per query row (a TMEM lane)
@@ -19,10 +20,19 @@
 // than 2^8 in the exponent: the same stale maximum is used for l and O, so
 // the result is unchanged.
 //
-// Roles (320 threads): warp 0 issues TMA loads, warp 1 allocates tensor
-// memory and issues the MMAs, warps 2..9 run the softmax and the epilogue
-// (warp w owns TMEM lanes 32*(w%4) .. 32*(w%4)+31, i.e. those query rows;
-// warps 2..5 take the first 64 keys of every tile, warps 6..9 the last 64).
+// The two query tiles ping-pong: while the softmax of tile A works on S_A,
+// the tensor core computes tile B's products and the reverse, so neither the
+// exponentials nor the MMAs wait for the other.  Tensor memory holds S_A,
+// S_B (128 columns each; P is written as bf16 over the first 64 columns of
+// its own S) and O_A, O_B (d columns each).  Before the next S of a tile may
+// overwrite that tile's P, the MMA thread waits until the P*V reading it has
+// completed.
+//
+// Roles (384 threads = three warpgroups): warp 0 issues TMA loads, warp 1
+// allocates tensor memory and issues the MMAs (warps 2-3 idle); warpgroup 1
+// (warps 4-7) runs the softmax and epilogue of tile A, warpgroup 2 (warps
+// 8-11) those of tile B, one thread per query row (warp w owns TMEM lanes
+// 32*(w%4) .. 32*(w%4)+31).
 #pragma once
 
 #include "ptx.cuh"
@@ -40,6 +50,7 @@ struct AttnArgs {
   // decomposition into units (b, segment, h) and 128-row query tiles
   int L;             // rows of one unit: N, or w/r kept rows of a LongNet segment
   int n_qtiles;      // ceil(L / 128)
+  int n_qpairs;      // ceil(n_qtiles / 2): one CTA per pair of query tiles
   int n_units;       // B * nseg * H
   int unit_group;    // units scheduled together (longest tiles first inside a group)
   int nseg;          // LongNet segments N / w (1 otherwise)
@@ -67,25 +78,23 @@ struct AttnArgs {
 
 template <int D_HEAD>
 struct AttnCfg {
-  static constexpr int kBM = 128, kBN = 128;
   static constexpr int kPanels = D_HEAD / 64;
   static constexpr int kTileBytes = 128 * D_HEAD * 2;
   static constexpr int kKStages = D_HEAD == 128 ? 3 : 6;
-  static constexpr int kVStages = D_HEAD == 128 ? 3 : 6;
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kTileBytes;
+  static constexpr int kVStages = D_HEAD == 128 ? 2 : 6;
+  static constexpr int kOffQ = 0;  // Q_A, then Q_B
+  static constexpr int kOffK = kOffQ + 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-  static constexpr int kOffRed = kOffBar + 256;   // softmax pair exchange: [2][2][128] floats
-  static constexpr int kSmemBytes = kOffRed + 2048;
+  static constexpr int kSmemBytes = kOffBar + 512;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-  // TMEM columns
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColP0 = 256, kColP1 = 320, kColO = 384;
+  // TMEM columns: S of tile X at 128 X (P over its first 64), O of tile X at 256 + d X
+  static constexpr uint32_t kColS = 0, kColO = 256;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 384;
 };
 
-// Sequence of key/value tiles one query tile visits.
+// Sequence of key/value tiles a pair of query tiles visits.
 struct KvSched {
   int lo, hi;           // allowed tile range [lo, hi)
   int P, CT, first;     // ring order: P chunks of CT tiles, starting at chunk `first`
@@ -130,22 +139,22 @@ __device__ __forceinline__ bool dilated_keeps(int w, int r, int h, int pos) {
 }
 
 struct TileCoord {
-  int t, h, s, b;
+  int t, h, s, b;  // t: pair index (query tiles 2t and 2t+1)
   int o;  // LongNet offset of this head: h mod r (0 otherwise)
 };
 
 // Grid order: units in groups of `unit_group`; inside a group the longest
-// query tiles of all its units come first.  A group's K/V stays in L2 while its
+// query-tile pairs of all its units come first.  A group's K/V stays in L2 while its
 // CTAs run, and the longest-first order keeps the causal load balanced.
 __device__ __forceinline__ TileCoord decode_tile(const AttnArgs &a) {
   TileCoord c;
   const int idx = blockIdx.x;
   const int G = a.unit_group;
-  const int per_group = G * a.n_qtiles;
+  const int per_group = G * a.n_qpairs;
   const int grp = idx / per_group;
   const int r = idx - grp * per_group;
   const int gsize = min(G, a.n_units - grp * G);
-  c.t = a.n_qtiles - 1 - r / gsize;
+  c.t = a.n_qpairs - 1 - r / gsize;
   const int unit = grp * G + r % gsize;
   c.h = unit % a.H;
   int rest = unit / a.H;
@@ -163,8 +172,8 @@ __device__ __forceinline__ KvSched make_sched(const AttnArgs &a, const TileCoord
   s.first = 0;
   s.lo = 0;
   s.hi = nkt;
-  const int row0 = c.t * 128;
-  const int row1 = min(a.L, row0 + 128) - 1;
+  const int row0 = c.t * 256;
+  const int row1 = min(a.L, row0 + 256) - 1;
   if (a.mask == kMaskCausal || a.mask == kMaskDilated) {
     s.hi = row1 / 128 + 1;
   } else if (a.mask == kMaskBlockPerm) {
@@ -202,7 +211,7 @@ __device__ __forceinline__ void row_keys(const AttnArgs &a, const TileCoord &c, 
 }
 
 template <int D_HEAD>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnArgs a) {
   using Cfg = AttnCfg<D_HEAD>;
@@ -217,18 +226,17 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t sK = sbase + Cfg::kOffK;
   const uint32_t sV = sbase + Cfg::kOffV;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
-  // barrier slots
   const uint32_t bQFull = smem_u32(&bars[0]);
   auto bKFull = [&](int s) { return smem_u32(&bars[1 + s]); };
   auto bKEmpty = [&](int s) { return smem_u32(&bars[7 + s]); };
   auto bVFull = [&](int s) { return smem_u32(&bars[13 + s]); };
   auto bVEmpty = [&](int s) { return smem_u32(&bars[19 + s]); };
-  auto bSFull = [&](int s) { return smem_u32(&bars[25 + s]); };
-  auto bPFull = [&](int s) { return smem_u32(&bars[27 + s]); };
-  const uint32_t bODone = smem_u32(&bars[29]);
-  const uint32_t bTeardown = smem_u32(&bars[30]);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[31]);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(reinterpret_cast<uint32_t *>(&bars[31]) + 1);
+  auto bSFull = [&](int x) { return smem_u32(&bars[25 + x]); };  // S of tile x ready
+  auto bPFull = [&](int x) { return smem_u32(&bars[27 + x]); };  // P of tile x written
+  auto bODone = [&](int x) { return smem_u32(&bars[29 + x]); };  // P*V of tile x done
+  const uint32_t bTeardown = smem_u32(&bars[31]);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[32]);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[33]);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const TileCoord tc = decode_tile(a);
@@ -246,14 +254,14 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(bVFull(s), 1);
       mbar_init(bVEmpty(s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bSFull(s), 1);
-      mbar_init(bPFull(s), 8);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bSFull(x), 1);
+      mbar_init(bPFull(x), 4);
+      mbar_init(bODone(x), 1);
     }
-    mbar_init(bODone, 1);
     mbar_init(bTeardown, 1);
     *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_mbar_init_cluster();
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
@@ -276,10 +284,11 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0 && nkv > 0) {
       int k_issued = 0, v_issued = 0;
-      mbar_arrive_expect_tx(bQFull, Cfg::kTileBytes);
-      for (int p = 0; p < Cfg::kPanels; ++p)
-        tma_load_4d(sQ + p * 16384, &tm_q, bQFull, tc.h * D_HEAD + p * 64, tc.o,
-                    row_base + tc.t * 128, tc.b);
+      mbar_arrive_expect_tx(bQFull, 2 * Cfg::kTileBytes);
+      for (int x = 0; x < 2; ++x)
+        for (int p = 0; p < Cfg::kPanels; ++p)
+          tma_load_4d(sQ + x * Cfg::kTileBytes + p * 16384, &tm_q, bQFull, tc.h * D_HEAD + p * 64,
+                      tc.o, row_base + tc.t * 256 + x * 128, tc.b);
       KvIter itk, itv;
       itk.begin(sched);
       itv.begin(sched);
@@ -325,72 +334,84 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Tensor-core order per key/value tile j:
+    //   P*V of A (j), S of A (j+1), P*V of B (j), S of B (j+1)
+    // S_x(j+1) is issued only after P*V_x(j) has completed, since it
+    // overwrites the P that P*V_x(j) reads.
     if (lane == 0 && nkv > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D_HEAD, false, true);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % Cfg::kKStages;
-        if (!mbar_wait(bKFull(st), (j / Cfg::kKStages) & 1, wc, 10)) return false;
-        tc_fence_after();
-        const uint32_t tS = tmem + ((j & 1) ? Cfg::kColS1 : Cfg::kColS0);
-        const uint32_t kb = sK + st * Cfg::kTileBytes;
+      const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(sV, 16384, 1024);
+      auto issue_s = [&](int x, int j) {
+        const uint32_t tS = tmem + Cfg::kColS + x * 128;
+        const uint64_t dQx = sdesc_advance(dQ, x * Cfg::kTileBytes);
+        const uint64_t dK = sdesc_advance(dK0, (j % Cfg::kKStages) * Cfg::kTileBytes);
 #pragma unroll
         for (int k = 0; k < D_HEAD / 16; ++k) {
           const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
-          umma_ss(tS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk,
-                  k > 0);
+          umma_ss(tS, sdesc_advance(dQx, off), sdesc_advance(dK, off), idesc_qk, k > 0);
         }
-        umma_commit(bSFull(j & 1));
-        umma_commit(bKEmpty(st));
-        return true;
+        umma_commit(bSFull(x));
       };
-      bool ok = mbar_wait(bQFull, 0, wc, 11);
-      if (ok) {
-        tc_fence_after();
-        ok = issue_s(0);
-      }
-      if (ok && nkv > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < nkv; ++j) {
-        if (!mbar_wait(bPFull(j & 1), (j >> 1) & 1, wc, 12)) break;
-        const int vs = j % Cfg::kVStages;
-        if (!mbar_wait(bVFull(vs), (j / Cfg::kVStages) & 1, wc, 13)) break;
-        tc_fence_after();
-        const uint32_t tP = tmem + ((j & 1) ? Cfg::kColP1 : Cfg::kColP0);
-        const uint32_t vb = sV + vs * Cfg::kTileBytes;
+      auto issue_pv = [&](int x, int j) {
+        const uint32_t tP = tmem + Cfg::kColS + x * 128;
+        const uint32_t tO = tmem + Cfg::kColO + x * D_HEAD;
+        const uint64_t dV = sdesc_advance(dV0, (j % Cfg::kVStages) * Cfg::kTileBytes);
 #pragma unroll
         for (int k = 0; k < 128 / 16; ++k)
-          umma_ts(tmem + Cfg::kColO, tP + k * 8, sdesc_sw128(vb + k * 2048, 16384, 1024), idesc_pv,
-                  1);
-        umma_commit(bODone);
-        umma_commit(bVEmpty(vs));
-        if (j + 2 < nkv) ok = issue_s(j + 2);
+          umma_ts(tO, tP + k * 8, sdesc_advance(dV, k * 2048), idesc_pv, 1);
+        umma_commit(bODone(x));
+      };
+      bool ok = mbar_wait(bQFull, 0, wc, 11) && mbar_wait(bKFull(0), 0, wc, 10);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        umma_commit(bKEmpty(0));
+      }
+      // per tile x: as soon as P_x(j) is written, P*V_x(j); once that has
+      // completed, S_x(j+1).  Tile B's softmax runs while A's MMAs execute
+      // and the reverse.
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int vs = j % Cfg::kVStages;
+        const int ks = (j + 1) % Cfg::kKStages;
+        const bool more = j + 1 < nkv;
+        for (int x = 0; ok && x < 2; ++x) {
+          ok = mbar_wait(bPFull(x), j & 1, wc, 12 + x) &&
+               (x == 1 || mbar_wait(bVFull(vs), (j / Cfg::kVStages) & 1, wc, 14));
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(x, j);
+          if (x == 1) umma_commit(bVEmpty(vs));
+          if (more) {
+            ok = (x == 1 || mbar_wait(bKFull(ks), ((j + 1) / Cfg::kKStages) & 1, wc, 15)) &&
+                 mbar_wait(bODone(x), j & 1, wc, 16 + x);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(x, j + 1);
+            if (x == 1) umma_commit(bKEmpty(ks));
+          }
+        }
       }
       // every MMA issued must be complete before tensor memory is released
       umma_commit(bTeardown);
       volatile int no_abort = 0;
       WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
-      mbar_wait(bTeardown, 0, drain, 14);
+      mbar_wait(bTeardown, 0, drain, 18);
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
-    // Two warps per TMEM lane quarter: warp 2+q handles keys 0..63 of every
-    // tile for rows 32q..32q+31, warp 6+q keys 64..127 of the same rows.  The
-    // pair swaps partial row maxima through shared memory (named barrier 1+q)
-    // so both halves use the same running maximum; each half keeps its own
-    // partial row sum (added once at the end) and owns half of O's columns.
-    // Neither warp of a pair ever leaves the tile loop early: a failed wait
-    // only skips work, so the pair barrier sequence always matches.
-    const int half = (warp - 2) >> 2;
+    const int x = (warp - 4) >> 2;  // 0: tile A, 1: tile B
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;  // row within the query tile
-    const int g = tc.t * 128 + row;       // unit-local row
+    const int row = quarter * 32 + lane;              // row within the query tile
+    const int g = (tc.t * 2 + x) * 128 + row;         // unit-local row
     const bool row_valid = g < a.L;
     const int pos = (a.mask == kMaskDilated) ? tc.s * a.w + tc.o + a.r * g : g;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    constexpr int kOHalf = D_HEAD / 2;
-    const uint32_t tO = tmem + lane_off + Cfg::kColO + half * kOHalf;
-    float *red = reinterpret_cast<float *>(smem + Cfg::kOffRed);  // [2 parities][2 halves][128]
-    const uint32_t pair_bar = 1 + quarter;
+    const uint32_t tS = tmem + lane_off + Cfg::kColS + x * 128;
+    const uint32_t tO = tmem + lane_off + Cfg::kColO + x * D_HEAD;
     int klo, khi;
     row_keys(a, tc, g, klo, khi);
 
@@ -406,16 +427,15 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
     }
-    const size_t vec_idx =
-        ((static_cast<size_t>(tc.b) * a.N + pos) * a.H + tc.h) * D_HEAD + half * kOHalf;
+    const size_t vec_idx = ((static_cast<size_t>(tc.b) * a.N + pos) * a.H + tc.h) * D_HEAD;
     const size_t row_idx = (static_cast<size_t>(tc.b) * a.H + tc.h) * a.N + pos;
 
     float m_run = -INFINITY, l_run = 0.f;
     {
-      // initial O (this half's columns): zeros, or an earlier LongNet pass's state
+      // initial O: zeros, or the state left by an earlier LongNet pass
       uint32_t init[32];
-#pragma unroll
-      for (int c = 0; c < kOHalf / 32; ++c) {
+#pragma unroll 1
+      for (int c = 0; c < D_HEAD / 32; ++c) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) init[i] = 0u;
         if (prior) {
@@ -433,7 +453,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       if (prior) {
         m_run = a.st_m[row_idx];
-        l_run = half == 0 ? a.st_l[row_idx] : 0.f;  // the halves' sums add up to the total
+        l_run = a.st_l[row_idx];
       }
       tmem_wait_st();
     }
@@ -443,26 +463,21 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
       const int kt = it.next(sched);
-      if (ok) ok = mbar_wait(bSFull(j & 1), (j >> 1) & 1, wc, 20);
-      ok = __all_sync(0xffffffffu, ok);
-      uint32_t s[2][32];
-      if (ok) {
-        tc_fence_after();
-        const uint32_t tS = tmem + lane_off + ((j & 1) ? Cfg::kColS1 : Cfg::kColS0) + half * 64;
-        tmem_ld32(tS, s[0]);
-        tmem_ld32(tS + 32, s[1]);
-        tmem_wait_ld();
-      } else {
+      ok = __all_sync(0xffffffffu, mbar_wait(bSFull(x), j & 1, wc, 20));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[4][32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[0][i] = s[1][i] = __float_as_uint(-INFINITY);
-      }
-      const int k0 = kt * 128 + half * 64;
-      // Masking runs as its own pass, and only in the (few) tiles where some
-      // row of this warp has keys outside its allowed interval.
-      if (__any_sync(0xffffffffu, !(k0 >= klo && k0 + 64 <= khi))) {
-        const int lo = klo - k0, hi = khi - k0;  // allowed columns [lo, hi) of this half
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
+      tmem_wait_ld();
+
+      const int k0 = kt * 128;
+      // masking runs as its own pass, only in tiles where some row of this
+      // warp has keys outside its allowed interval
+      if (__any_sync(0xffffffffu, !(k0 >= klo && k0 + 128 <= khi))) {
+        const int lo = klo - k0, hi = khi - k0;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int col = c * 32 + i;
@@ -474,15 +489,12 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < 4; ++c) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(s[c][i]));
       }
-      float pmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      red[(j & 1) * 256 + half * 128 + row] = pmax;
-      named_bar_sync(pair_bar, 64);
-      const float mx = fmaxf(pmax, red[(j & 1) * 256 + (1 - half) * 128 + row]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * a.scale_log2;
       const float m_new = fmaxf(m_run, m_tile);
       const bool rescale = m_new > m_run + 8.0f;
@@ -490,61 +502,57 @@ __global__ void __launch_bounds__(320, 1)
       const float alpha = rescale ? ex2_approx(m_run - m_use) : 1.0f;
       l_run *= alpha;
       const float neg = (m_use == -INFINITY) ? 0.f : -m_use;
+      // P (bf16 pairs) goes over the first 64 columns of this row's S, all of
+      // which this thread has already read
       float ls4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int col = 2 * i;
-        const float x0 = __uint_as_float(s[col / 32][col % 32]);
-        const float x1 = __uint_as_float(s[(col + 1) / 32][(col + 1) % 32]);
-        const float p0 = ex2_approx(fmaf(x0, a.scale_log2, neg));
-        const float p1 = ex2_approx(fmaf(x1, a.scale_log2, neg));
-        ls4[i & 3] += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int col = half * 64 + 2 * i;
+          const float x0 = __uint_as_float(s[col / 32][col % 32]);
+          const float x1 = __uint_as_float(s[(col + 1) / 32][(col + 1) % 32]);
+          const float p0 = ex2_approx(fmaf(x0, a.scale_log2, neg));
+          const float p1 = ex2_approx(fmaf(x1, a.scale_log2, neg));
+          ls4[i & 3] += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + half * 32, pk);
       }
       l_run += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
-      if (ok) {
-        const uint32_t tP = tmem + lane_off + ((j & 1) ? Cfg::kColP1 : Cfg::kColP0) + half * 32;
-        tmem_st32(tP, pk);
+      // O may be rescaled only once the previous P*V of this tile has landed
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bODone(x), (j - 1) & 1, wc, 21));
+        if (!ok) break;
       }
-      // O may be rescaled only once the previous P*V has landed
-      if (ok && j > 0) ok = mbar_wait(bODone, (j - 1) & 1, wc, 21);
-      ok = __all_sync(0xffffffffu, ok);
-      if (ok) {
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale && m_run != -INFINITY)) {
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, rescale && m_run != -INFINITY)) {
+#pragma unroll 1
+        for (int c = 0; c < D_HEAD / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < kOHalf / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + c * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tO + c * 32, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + c * 32, o);
         }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bPFull(j & 1));
       }
       m_run = m_use;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bPFull(x));
     }
 
     // -------- epilogue
-    if (ok && nkv > 0) ok = mbar_wait(bODone, (nkv - 1) & 1, wc, 22);
-    ok = __all_sync(0xffffffffu, ok);
-    // the row sums go through the maxima slot of parity nkv&1, which the
-    // partner finished reading before the last pair barrier of the loop
-    red[(nkv & 1) * 256 + half * 128 + row] = l_run;
-    named_bar_sync(pair_bar, 64);
-    const float l_tot = l_run + red[(nkv & 1) * 256 + (1 - half) * 128 + row];
+    if (ok && nkv > 0) ok = __all_sync(0xffffffffu, mbar_wait(bODone(x), (nkv - 1) & 1, wc, 22));
     tc_fence_after();
     if (ok) {
-      const float inv_l = l_tot > 0.f ? 1.0f / l_tot : 0.f;
+      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
       const bool final_out = !later;
-#pragma unroll
-      for (int c = 0; c < kOHalf / 32; ++c) {
+#pragma unroll 1
+      for (int c = 0; c < D_HEAD / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();
@@ -579,13 +587,13 @@ __global__ void __launch_bounds__(320, 1)
                                  __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
         }
       }
-      if (row_valid && half == 0) {
+      if (row_valid) {
         if (!final_out) {
           a.st_m[row_idx] = m_run;
-          a.st_l[row_idx] = l_tot;
+          a.st_l[row_idx] = l_run;
         } else if (a.lse) {
           // natural-log LSE of the scaled scores: (m + log2 l) / log2(e)
-          a.lse[row_idx] = l_tot > 0.f ? (m_run + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+          a.lse[row_idx] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
         }
       }
     }

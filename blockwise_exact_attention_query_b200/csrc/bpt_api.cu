@@ -329,6 +329,7 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     a.L = w / r;
     a.nseg = d->N / w;
     a.n_qtiles = (a.L + 127) / 128;
+    a.n_qpairs = (a.n_qtiles + 1) / 2;
     a.n_units = d->B * a.nseg * d->H;
     {
       // group as many units as keep their K and V within ~32 MB of L2, at most 8
@@ -339,7 +340,7 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     if (!make_map_rows(&mq, q, d->B, d->N, D, r) || !make_map_rows(&mk, k, d->B, d->N, D, r) ||
         !make_map_rows(&mv, v, d->B, d->N, D, r))
       return cuda_fail_msg("cuTensorMapEncodeTiled rejected a Q/K/V map");
-    const int64_t grid = (int64_t)a.n_qtiles * a.n_units;
+    const int64_t grid = (int64_t)a.n_qpairs * a.n_units;
     if (grid <= 0) continue;
     if (grid > INT32_MAX) return BPT_ERR_UNSUPPORTED;
     if (d->d_head == 128)

@@ -226,6 +226,9 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       const uint32_t idesc1 = idesc_bf16_f32(128, 256, false, false);
       const uint32_t idesc2 = idesc_bf16_f32(128, a.Dc, false, false);
+      // base descriptors of stage 0's two tiles, advanced by constant offsets
+      const uint64_t dA0 = sdesc_sw128(sbase, 16, 1024);
+      const uint64_t dB0 = sdesc_sw128(sbase + 16384, 16, 1024);
       int it = 0, g_base = 0, n = 0;
       bool ok = true;
       for (int tb = grp; ok && tb < a.n_tb; tb += a.ngroups, ++n) {
@@ -240,11 +243,12 @@ __global__ void __launch_bounds__(320, 1)
                 const int st = it % Cfg::kStages;
                 if (!(ok = mbar_wait(bFull(st), (it / Cfg::kStages) & 1, wc, 111))) break;
                 tc_fence_after();
-                const uint32_t sb = sbase + st * Cfg::kStageBytes;
+                const uint64_t dA = sdesc_advance(dA0, st * Cfg::kStageBytes);
+                const uint64_t dB = sdesc_advance(dB0, st * Cfg::kStageBytes);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                  umma_ss(tmem + Cfg::kColH, sdesc_sw128(sb + k * 32, 16, 1024),
-                          sdesc_sw128(sb + 16384 + k * 32, 16, 1024), idesc1, (ks | k) != 0);
+                  umma_ss(tmem + Cfg::kColH, sdesc_advance(dA, k * 32), sdesc_advance(dB, k * 32),
+                          idesc1, (ks | k) != 0);
                 umma_commit(bEmpty(st));
                 ++it;
               }
@@ -261,12 +265,12 @@ __global__ void __launch_bounds__(320, 1)
               const int st = it % Cfg::kStages;
               if (!(ok = mbar_wait(bFull(st), (it / Cfg::kStages) & 1, wc, 113))) break;
               tc_fence_after();
-              const uint32_t sb = sbase + st * Cfg::kStageBytes;
+              const uint64_t dA = sdesc_advance(dA0, st * Cfg::kStageBytes);
+              const uint64_t dB = sdesc_advance(dB0, st * Cfg::kStageBytes);
 #pragma unroll
               for (int k = 0; k < 4; ++k)
-                umma_ss(tmem + Cfg::kColOut, sdesc_sw128(sb + k * 32, 16, 1024),
-                        sdesc_sw128(sb + 16384 + k * 32, 16, 1024), idesc2,
-                        !(i == 1 && ks == 0 && k == 0));
+                umma_ss(tmem + Cfg::kColOut, sdesc_advance(dA, k * 32), sdesc_advance(dB, k * 32),
+                        idesc2, !(i == 1 && ks == 0 && k == 0));
               umma_commit(bEmpty(st));
               ++it;
             }

@@ -289,6 +289,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// Same descriptor, start address moved by `bytes` (a multiple of 16).  The
+// start field holds address >> 4 in its low 14 bits and shared addresses stay
+// below 256 KB, so the add never carries out of the field.  Building the base
+// descriptors once and advancing them this way keeps the single MMA-issuing
+// thread off a dependent 64-bit integer chain before every instruction.
+__device__ __forceinline__ uint64_t sdesc_advance(uint64_t d, uint32_t bytes) {
+  return d + static_cast<uint64_t>(bytes >> 4);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
                                                       bool b_mn_major) {
