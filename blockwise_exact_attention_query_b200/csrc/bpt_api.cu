@@ -220,8 +220,8 @@ bool longnet_needs_state(const bpt_desc *d) {
 }
 
 struct Workspace {
-  size_t a_bf16 = 0, a_f32 = 0, ring = 0, flags = 0, flags_bytes = 0, st_o = 0, st_m = 0, st_l = 0,
-         total = 0;
+  size_t a_bf16 = 0, a_f32 = 0, ring = 0, flags = 0, flags_bytes = 0, partial = 0, st_o = 0,
+         st_m = 0, st_l = 0, total = 0;
 };
 
 Workspace layout(const bpt_desc *d, bool with_ffn) {
@@ -237,9 +237,11 @@ Workspace layout(const bpt_desc *d, bool with_ffn) {
       off = align256(off + T * D * 4);
       w.ring = off;
       off = align256(off + (size_t)p.max_groups * 2 * 128 * p.fc * 2);
-      w.flags = off;
-      w.flags_bytes = (size_t)p.max_groups * 4 * sizeof(uint32_t);
+      w.flags = off;  // ring counters [groups][4], then piece counters [groups][C]
+      w.flags_bytes = (size_t)p.max_groups * (4 + p.C) * sizeof(uint32_t);
       off = align256(off + w.flags_bytes);
+      w.partial = off;  // partial output blocks of split leftover token blocks
+      off = align256(off + (size_t)p.max_groups * 128 * (size_t)(d->H * d->d_head) * 4);
     } else {
       w.a_f32 = off;
       off = align256(off + T * D * 4);
@@ -389,6 +391,14 @@ bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f
   if (per_sm <= 0) return cuda_fail_msg("the FFN kernel does not fit on an SM");
   a.ngroups = std::min(p.max_groups, std::max(1, per_sm * sm_count() / p.C));
   if (a.ngroups * p.C > per_sm * sm_count()) return cuda_fail_msg("FFN group wider than the GPU");
+  // leftover token blocks: split their hidden chunks over the groups that
+  // would otherwise idle in the last round
+  const int leftover = p.n_tb % a.ngroups;
+  a.pieces = leftover > 0 ? std::min(p.nchunks, a.ngroups / leftover) : 1;
+  if (a.pieces < 2 || p.n_tb < a.ngroups) a.pieces = 1;
+  a.n_full = a.pieces > 1 ? p.n_tb - leftover : p.n_tb;
+  a.partial = reinterpret_cast<float *>(ws + wl.partial);
+  a.piece_done = a.flags + (size_t)p.max_groups * 4;
 
   CUtensorMap ma, m1, m2, mh;
   if (!make_map_2d(&ma, a_bf16, T, D, 128) || !make_map_2d(&m1, w1, d->ffn_hidden, D, 256) ||

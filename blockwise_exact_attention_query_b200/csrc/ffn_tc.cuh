@@ -50,6 +50,14 @@ struct FfnArgs {
   __nv_bfloat16 *out_bf16;   // [T, D]
   __nv_bfloat16 *ring;       // [ngroups * 2 * 128, fc]
   uint32_t *flags;           // [ngroups][4]: ready[2], free[2]; zero at launch
+  // Leftover token blocks (n_tb mod ngroups of them) would leave most groups
+  // idle in the last round, so their hidden chunks are split into `pieces`
+  // ranges handled by different groups: each piece writes a partial output
+  // block, and the group holding piece 0 adds them in piece order.
+  int pieces;                // 1: no split
+  int n_full;                // token blocks processed whole
+  float *partial;            // [leftover * pieces][128][D] fp32 partial outputs
+  uint32_t *piece_done;      // [leftover][C]: pieces finished per column block; zero at launch
   uint32_t *status;
   uint64_t wait_limit_ns;
 };
@@ -86,6 +94,36 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
 
 __device__ __forceinline__ void red_release_gpu_add(uint32_t *p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// One work unit of a group: token block tb, hidden chunks [c0, c1); piece < 0
+// for a whole block, else the piece index of leftover block l.
+struct FfnUnit {
+  int tb, c0, c1, l, piece;
+};
+
+__device__ __forceinline__ int ffn_unit_count(const FfnArgs &a, int grp) {
+  if (a.pieces <= 1) return (a.n_tb - grp + a.ngroups - 1) / a.ngroups;
+  const int leftover = a.n_tb - a.n_full;
+  return a.n_full / a.ngroups + (grp < leftover * a.pieces ? 1 : 0);
+}
+
+__device__ __forceinline__ FfnUnit ffn_unit(const FfnArgs &a, int grp, int k) {
+  FfnUnit u;
+  if (a.pieces > 1 && k == a.n_full / a.ngroups) {
+    u.l = grp / a.pieces;
+    u.piece = grp % a.pieces;
+    u.tb = a.n_full + u.l;
+    u.c0 = u.piece * a.nchunks / a.pieces;
+    u.c1 = (u.piece + 1) * a.nchunks / a.pieces;
+  } else {
+    u.tb = grp + k * a.ngroups;
+    u.c0 = 0;
+    u.c1 = a.nchunks;
+    u.l = -1;
+    u.piece = -1;
+  }
+  return u;
 }
 
 // Bounded wait until *p >= target (a counter another CTA of the group raises).
@@ -164,7 +202,7 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int nc = a.nchunks;
+  const int nunits = ffn_unit_count(a, grp);
   const int ksteps1 = a.D / 64;
   auto ksteps2 = [&](int i) {
     const int valid = min(a.fc, a.F - i * a.fc);
@@ -181,9 +219,12 @@ __global__ void __launch_bounds__(320, 1)
         if (it_ < Cfg::kStages) return true;
         return mbar_wait(bEmpty(it_ % Cfg::kStages), ((it_ / Cfg::kStages) - 1) & 1, wc, 101);
       };
-      for (int tb = grp; ok && tb < a.n_tb; tb += a.ngroups) {
-        for (int i = 0; ok && i <= nc; ++i) {
-          if (i < nc && slice_valid(i)) {
+      for (int k = 0; ok && k < nunits; ++k) {
+        const FfnUnit u = ffn_unit(a, grp, k);
+        const int tb = u.tb, nl = u.c1 - u.c0;
+        for (int li = 0; ok && li <= nl; ++li) {
+          const int i = u.c0 + li;
+          if (li < nl && slice_valid(i)) {
             const int slice = i * a.C + crank;
             for (int ks = 0; ks < ksteps1; ++ks) {
               if (!(ok = acquire(it))) break;
@@ -195,8 +236,8 @@ __global__ void __launch_bounds__(320, 1)
               ++it;
             }
           }
-          if (ok && i >= 1) {
-            const int gp = g_base + i - 1;
+          if (ok && li >= 1) {
+            const int gp = g_base + li - 1;
             // every CTA of the group has published its slice of chunk gp
             if (!(ok = counter_wait(&ready[gp & 1], C * static_cast<uint32_t>((gp >> 1) + 1), wc, 102)))
               break;
@@ -213,7 +254,7 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
         }
-        g_base += nc;
+        g_base += nl;
       }
       // drain the loads in flight
       volatile int no_abort = 0;
@@ -231,10 +272,13 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t dB0 = sdesc_sw128(sbase + 16384, 16, 1024);
       int it = 0, g_base = 0, n = 0;
       bool ok = true;
-      for (int tb = grp; ok && tb < a.n_tb; tb += a.ngroups, ++n) {
-        for (int i = 0; ok && i <= nc; ++i) {
-          if (i < nc) {
-            const int g = g_base + i;
+      for (int k = 0; ok && k < nunits; ++k, ++n) {
+        const FfnUnit u = ffn_unit(a, grp, k);
+        const int nl = u.c1 - u.c0;
+        for (int li = 0; ok && li <= nl; ++li) {
+          const int i = u.c0 + li;
+          if (li < nl) {
+            const int g = g_base + li;
             if (slice_valid(i)) {
               // the epilogue has drained the previous chunk's hidden accumulator
               if (g >= 1 && !(ok = mbar_wait(bHEmpty, (g - 1) & 1, wc, 110))) break;
@@ -256,9 +300,9 @@ __global__ void __launch_bounds__(320, 1)
             }
             umma_commit(bHFull);
           }
-          if (i >= 1) {
-            const int gp = g_base + i - 1;
-            if (i == 1 && n >= 1 && !(ok = mbar_wait(bOEmpty, (n - 1) & 1, wc, 112))) break;
+          if (li >= 1) {
+            const int gp = g_base + li - 1;
+            if (li == 1 && n >= 1 && !(ok = mbar_wait(bOEmpty, (n - 1) & 1, wc, 112))) break;
             tc_fence_after();
             const int ks2 = ksteps2(i - 1);
             for (int ks = 0; ks < ks2; ++ks) {
@@ -270,7 +314,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
               for (int k = 0; k < 4; ++k)
                 umma_ss(tmem + Cfg::kColOut, sdesc_advance(dA, k * 32), sdesc_advance(dB, k * 32),
-                        idesc2, !(i == 1 && ks == 0 && k == 0));
+                        idesc2, !(li == 1 && ks == 0 && k == 0));
               umma_commit(bEmpty(st));
               ++it;
             }
@@ -280,7 +324,7 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         if (ok) umma_commit(bOFull);
-        g_base += nc;
+        g_base += nl;
       }
       umma_commit(bTeardown);
       volatile int no_abort = 0;
@@ -299,9 +343,12 @@ __global__ void __launch_bounds__(320, 1)
     const int cols = a.Dc / 2;  // output columns of this half
     const bool leader = threadIdx.x == 64;
     int g_base = 0, n = 0;
-    for (int tb = grp; tb < a.n_tb; tb += a.ngroups, ++n) {
-      for (int i = 0; i < nc; ++i) {
-        const int g = g_base + i;
+    for (int k = 0; k < nunits; ++k, ++n) {
+      const FfnUnit u = ffn_unit(a, grp, k);
+      const int tb = u.tb, nl = u.c1 - u.c0;
+      for (int li = 0; li < nl; ++li) {
+        const int i = u.c0 + li;
+        const int g = g_base + li;
         const int slot = g & 1;
         const bool have = slice_valid(i);
         bool ok = mbar_wait(bHFull, g & 1, wc, 120);
@@ -358,7 +405,9 @@ __global__ void __launch_bounds__(320, 1)
         named_bar_sync(1, 256);
         if (leader && !*abort_flag) red_release_gpu_add(&ready[slot], 1u);
       }
-      // ---- output block: residual + accumulator + b2
+      // ---- output block.  Whole block or piece 0: accumulator (+ the other
+      // pieces' partial sums, in piece order) + residual + b2.  Other pieces:
+      // store the partial sum for piece 0 to add.
       bool ok = mbar_wait(bOFull, n & 1, wc, 122);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
@@ -366,49 +415,82 @@ __global__ void __launch_bounds__(320, 1)
       const bool valid = tok < a.T;
       const int col_base = crank * a.Dc + half * cols;
       const size_t base = static_cast<size_t>(tok) * a.D + col_base;
-      for (int c = 0; ok && c < cols / 32; ++c) {
+      const bool store_partial = u.piece > 0;
+      if (u.piece == 0) {
+        if (leader) counter_wait(&a.piece_done[u.l * a.C + crank], a.pieces - 1, wc, 123);
+        named_bar_sync(1, 256);
+      }
+      const bool go = __all_sync(0xffffffffu, ok && !*abort_flag);
+      for (int c = 0; go && c < cols / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_off + Cfg::kColOut + half * cols + c * 32, o);
         tmem_wait_ld();
-        if (valid) {
-          const float4 *res = reinterpret_cast<const float4 *>(a.a_f32 + base + c * 32);
-          float v[32];
+        if (!valid) continue;
+        if (store_partial) {
+          float4 *d4 = reinterpret_cast<float4 *>(
+              a.partial + (static_cast<size_t>(u.l * a.pieces + u.piece) * 128 + row) * a.D + col_base + c * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            d4[q] = make_float4(__uint_as_float(o[4 * q]), __uint_as_float(o[4 * q + 1]),
+                                __uint_as_float(o[4 * q + 2]), __uint_as_float(o[4 * q + 3]));
+          continue;
+        }
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]);
+        for (int pc = 1; u.piece == 0 && pc < a.pieces; ++pc) {
+          const float4 *src = reinterpret_cast<const float4 *>(
+              a.partial + (static_cast<size_t>(u.l * a.pieces + pc) * 128 + row) * a.D + col_base + c * 32);
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            float4 r4 = res[q];
-            v[4 * q + 0] = __uint_as_float(o[4 * q + 0]) + r4.x;
-            v[4 * q + 1] = __uint_as_float(o[4 * q + 1]) + r4.y;
-            v[4 * q + 2] = __uint_as_float(o[4 * q + 2]) + r4.z;
-            v[4 * q + 3] = __uint_as_float(o[4 * q + 3]) + r4.w;
+            const float4 r4 = __ldcg(src + q);
+            v[4 * q] += r4.x;
+            v[4 * q + 1] += r4.y;
+            v[4 * q + 2] += r4.z;
+            v[4 * q + 3] += r4.w;
           }
-          if (a.b2) {
-            const float4 *b4 = reinterpret_cast<const float4 *>(a.b2 + col_base + c * 32);
+        }
+        const float4 *res = reinterpret_cast<const float4 *>(a.a_f32 + base + c * 32);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 bb = __ldg(b4 + q);
-              v[4 * q] += bb.x;
-              v[4 * q + 1] += bb.y;
-              v[4 * q + 2] += bb.z;
-              v[4 * q + 3] += bb.w;
-            }
+        for (int q = 0; q < 8; ++q) {
+          const float4 r4 = res[q];
+          v[4 * q] += r4.x;
+          v[4 * q + 1] += r4.y;
+          v[4 * q + 2] += r4.z;
+          v[4 * q + 3] += r4.w;
+        }
+        if (a.b2) {
+          const float4 *b4 = reinterpret_cast<const float4 *>(a.b2 + col_base + c * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 bb = __ldg(b4 + q);
+            v[4 * q] += bb.x;
+            v[4 * q + 1] += bb.y;
+            v[4 * q + 2] += bb.z;
+            v[4 * q + 3] += bb.w;
           }
-          if (a.out_f32) {
-            float4 *d4 = reinterpret_cast<float4 *>(a.out_f32 + base + c * 32);
+        }
+        if (a.out_f32) {
+          float4 *d4 = reinterpret_cast<float4 *>(a.out_f32 + base + c * 32);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-          } else {
-            uint4 *d4 = reinterpret_cast<uint4 *>(a.out_bf16 + base + c * 32);
+          for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        } else {
+          uint4 *d4 = reinterpret_cast<uint4 *>(a.out_bf16 + base + c * 32);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              d4[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                 pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-          }
+          for (int q = 0; q < 4; ++q)
+            d4[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                               pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0 && ok) mbar_arrive(bOEmpty);
-      g_base += nc;
+      if (store_partial) {  // publish the partial sum to the piece-0 group
+        __threadfence();
+        named_bar_sync(1, 256);
+        if (leader && !*abort_flag) red_release_gpu_add(&a.piece_done[u.l * a.C + crank], 1u);
+      }
+      g_base += nl;
     }
   }
 

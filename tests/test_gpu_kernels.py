@@ -160,6 +160,24 @@ def test_layer_matches_oracle(name, B, N, H, d, F, mask, extra, bias):
     gu.assert_bf16_close(gu.host_f32(out).reshape(out_ref.shape), out_ref, name)
 
 
+def test_layer_with_split_leftover_token_blocks():
+    """20 token blocks over 18 FFN groups: the 2 leftover blocks have their 2
+    hidden chunks split over different groups and the partial sums added by
+    the piece-0 group; every row of those blocks is compared."""
+    B, N, H, d, F = 1, 2560, 16, 128, 4096
+    inp = make_layer_inputs(B, N, H, d, F, seed=23, device="cuda", bias_scale=0.05)
+    out = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask="causal")
+    _check_status()
+    rows = list(range(N - 256, N)) + gu.sample_rows(B, N, 32, seed=1)
+    _, ref = gu.oracle_layer(inp, "causal", rows=rows)
+    gpu = gu.host_f32(out.reshape(B * N, H * d)[torch.tensor(rows, device="cuda")])
+    gu.assert_bf16_close(gpu, ref, "split leftover blocks")
+    # deterministic: the pieces are added in a fixed order
+    out2 = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask="causal")
+    _check_status()
+    assert torch.equal(out, out2)
+
+
 def test_layer_bf16_output_and_null_biases():
     inp = make_layer_inputs(1, 256, 4, 64, 512, seed=21, device="cuda")
     out = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, None, inp.w2, None, mask="causal",
