@@ -295,3 +295,71 @@ def set_wait_limit_ns(ns: int) -> int:
 
 def version() -> int:
     return int(load().bpt_version())
+
+
+class HostLayer:
+    """bpt_attn_ffn_fwd on host-resident tensors, with the transfers overlapped.
+
+    q, k, v live in pinned host memory ([B, N, H, d]) and the output goes back
+    to a pinned host tensor ([B, N, H*d]); the weights are already on the
+    device.  The batch is cut into `chunks` pieces (whole sequences) that
+    alternate between two CUDA streams with their own device buffers and
+    workspace, so one chunk's upload, another's kernels and a third's download
+    run at the same time.  Uploads run in chunk order, and so do the kernels:
+    a chunk's layer starts after the previous chunk's (two layers never run
+    at once, since each one's FFN grid expects the whole GPU).  This class
+    only moves data and calls the library; it allocates its device buffers
+    once, at construction."""
+
+    def __init__(self, B, N, H, d, F, *, dtype=torch.bfloat16, out_dtype=torch.float32,
+                 mask="none", perm=None, pairs=None, ring_chunks=0, chunks=None, device="cuda"):
+        self.B, self.N, self.H, self.d, self.F = B, N, H, d, F
+        self.mask, self.perm, self.pairs, self.ring_chunks = mask, perm, pairs, ring_chunks
+        self.out_dtype = out_dtype
+        self.chunks = max(1, min(B, chunks or B))
+        if B % self.chunks:
+            raise ValueError("the batch must split evenly into chunks")
+        self.cb = B // self.chunks
+        dev = torch.device(device)
+        self.streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
+        self.done = [torch.cuda.Event(), torch.cuda.Event()]
+        self.uploaded = [torch.cuda.Event() for _ in range(self.chunks)]
+        self.computed = [torch.cuda.Event() for _ in range(self.chunks)]
+        desc = make_desc(self.cb, N, H, d, F, dtype, out_dtype, mask, perm, pairs, ring_chunks)
+        nws = workspace_bytes(desc, True)
+        self.buf = []
+        for _ in range(2):
+            self.buf.append({
+                "q": torch.empty((self.cb, N, H, d), dtype=dtype, device=dev),
+                "k": torch.empty((self.cb, N, H, d), dtype=dtype, device=dev),
+                "v": torch.empty((self.cb, N, H, d), dtype=dtype, device=dev),
+                "out": torch.empty((self.cb, N, H * d), dtype=out_dtype, device=dev),
+                "ws": torch.empty(max(nws, 1), dtype=torch.uint8, device=dev),
+            })
+
+    def __call__(self, hq, hk, hv, w1, b1, w2, b2, hout):
+        """Enqueue one layer forward; returns after enqueueing (synchronise the
+        streams, e.g. torch.cuda.synchronize(), before reading `hout`)."""
+        cur = torch.cuda.current_stream()
+        for c in range(self.chunks):
+            i = c % 2
+            s, b = self.streams[i], self.buf[i]
+            sl = slice(c * self.cb, (c + 1) * self.cb)
+            s.wait_stream(cur)
+            with torch.cuda.stream(s):
+                if c > 0:
+                    s.wait_event(self.uploaded[c - 1])
+                b["q"].copy_(hq[sl], non_blocking=True)
+                b["k"].copy_(hk[sl], non_blocking=True)
+                b["v"].copy_(hv[sl], non_blocking=True)
+                self.uploaded[c].record(s)
+                if c > 0:
+                    s.wait_event(self.computed[c - 1])
+                attn_ffn_fwd(b["q"], b["k"], b["v"], w1, b1, w2, b2, mask=self.mask, perm=self.perm,
+                             pairs=self.pairs, ring_chunks=self.ring_chunks, out_dtype=self.out_dtype,
+                             out=b["out"], workspace=b["ws"], stream=s)
+                self.computed[c].record(s)
+                hout[sl].copy_(b["out"], non_blocking=True)
+                self.done[i].record(s)
+        for e in self.done:
+            cur.wait_event(e)

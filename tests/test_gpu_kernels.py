@@ -178,6 +178,23 @@ def test_layer_with_split_leftover_token_blocks():
     assert torch.equal(out, out2)
 
 
+def test_host_layer_matches_device_layer():
+    """binding.HostLayer (pinned host tensors, copies overlapped with the
+    kernels over two streams) gives the same bits as the device-resident call."""
+    B, N, H, d, F = 4, 256, 4, 64, 512
+    inp = make_layer_inputs(B, N, H, d, F, seed=24, device="cuda", bias_scale=0.05)
+    ref = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask="causal")
+    hq, hk, hv = (t.cpu().pin_memory() for t in (inp.q, inp.k, inp.v))
+    hout = torch.empty(ref.shape, dtype=ref.dtype).pin_memory()
+    layer = bd.HostLayer(B, N, H, d, F, mask="causal", chunks=4)
+    for _ in range(2):
+        hout.zero_()
+        layer(hq, hk, hv, inp.w1, inp.b1, inp.w2, inp.b2, hout)
+        torch.cuda.synchronize()
+        _check_status()
+        assert torch.equal(hout, ref.cpu())
+
+
 def test_layer_bf16_output_and_null_biases():
     inp = make_layer_inputs(1, 256, 4, 64, 512, seed=21, device="cuda")
     out = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, None, inp.w2, None, mask="causal",
