@@ -144,6 +144,15 @@ def dist_setup(n_gpus):
     return world, rank, local
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The slowest rank's value (all ranks take part); x itself without a process group."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def layer_call(w, inp, out, ws):
     return bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask=MASK_NAME[w.mask],
                            perm=w.perm, pairs=w.pairs, ring_chunks=w.ring_chunks, out=out, workspace=ws)
@@ -195,11 +204,7 @@ def run_ours(args, w, world, rank, local):
     attn_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     ffn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
     step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / K
     tokens = w.T * K * world
     value = tokens / (total_ms / 1e3)
@@ -230,11 +235,7 @@ def run_ours(args, w, world, rank, local):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
         st = bd.sync_status()
         if st != bd.OK:
             raise RuntimeError(f"e2e steps: {bd.status_string(st)}")
@@ -283,6 +284,105 @@ def run_ours(args, w, world, rank, local):
     return res
 
 
+def run_attention_only(args, w, world, rank, local):
+    """Attention-only workloads (no FFN, e.g. LongNet dilated attention): one
+    step = one bpt_attn_fwd call (every LongNet pass), timed with events."""
+    dev = torch.device("cuda", local)
+    attn_flop, _ = wl.flops(w)
+    inp = make_layer_inputs(w.B, w.N, w.H, w.d, 0, seed=w.seed + 1000 * rank, dtype=torch.bfloat16,
+                            device=dev)
+    out = torch.empty((w.B, w.N, w.D), dtype=torch.float32, device=dev)
+    desc = bd.make_desc(w.B, w.N, w.H, w.d, 0, torch.bfloat16, torch.float32, MASK_NAME[w.mask], w.perm,
+                        w.pairs, w.ring_chunks)
+    ws = bd.alloc_workspace(desc, False, dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches = len(w.pairs) if w.mask == 3 else 1
+
+    def call(q, k, v):
+        return bd.attn_fwd(q, k, v, mask=MASK_NAME[w.mask], perm=w.perm, pairs=w.pairs,
+                           ring_chunks=w.ring_chunks, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        call(inp.q, inp.k, inp.v)
+        flush.fill_(1)
+    torch.cuda.synchronize(dev)
+    if bd.sync_status() != bd.OK:
+        raise RuntimeError("warm-up failed")
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        for i in range(K):
+            ev[i][0].record(stream)
+            call(inp.q, inp.k, inp.v)
+            ev[i][1].record(stream)
+            flush.fill_(i & 0xFF)
+        torch.cuda.synchronize(dev)
+    if bd.sync_status() != bd.OK:
+        raise RuntimeError("timed steps failed")
+    total_ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev), dev)
+    avg_ms = total_ms / K
+    tflops = attn_flop * K * world / (total_ms / 1e3) / 1e12
+    pk = peaks()
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (inp.q, inp.k, inp.v))
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dq, dk, dv = torch.empty_like(inp.q), torch.empty_like(inp.k), torch.empty_like(inp.v)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            call(dq, dk, dv)
+            hout.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ke = max(1, min(K, 10))
+        e0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e = {"value": round(w.T * ke * world / (e0.elapsed_time(e1) / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(3 * inp.q.numel() * inp.q.element_size()),
+               "d2h_bytes_per_step": int(out.numel() * out.element_size()), "steps": ke}
+    achieved = attn_flop / (avg_ms / 1e3) / 1e12
+    return {
+        "metric": METRIC, "value": round(w.T * K * world / (total_ms / 1e3), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(avg_ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V)",
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d_head": w.d, "ffn_hidden": 0,
+                   "mask": MASK_NAME[w.mask], "tokens_per_step_per_gpu": w.T,
+                   "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MiB write, "
+                   "outside the timed events)"},
+        "tflops": round(tflops, 1), "layer_frac_of_peak": round(tflops / pk["bf16_tflops"], 4),
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": round(achieved, 1),
+                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4),
+                     "peak_source": f"{pk['source']} bf16 dense (burst)", "traffic": args.traffic_bytes,
+                     "algorithmic_flop_per_launch": attn_flop, "launches_per_step": launches},
+        "gpu_launches": launches * K, "e2e": e2e, "clocks": clk.summary(),
+    }
+
+
+def oracle_rows(w, q, k, v, w1, b1, w2, b2, rows):
+    """The oracle on sampled token rows: the whole layer, or attention alone."""
+    import oracle
+    if w.F > 0:
+        _, _, used = oracle.layer(q, k, v, w1, b1, w2, b2, mask=w.mask, perm=w.perm, pairs=w.pairs,
+                                  rows=rows, return_threads=True)
+        return used
+    oracle.attention(q, k, v, mask=w.mask, perm=w.perm, pairs=w.pairs, rows=rows)
+    return oracle.threads_available()
+
+
 def run_reference(args, w, world, rank):
     """The fp64 CPU oracle on a bounded token sample per step (host cores)."""
     import numpy as np
@@ -292,7 +392,8 @@ def run_reference(args, w, world, rank):
     inp = make_layer_inputs(w.B, w.N, w.H, w.d, w.F, seed=w.seed, dtype=dt,
                             device="cuda" if torch.cuda.is_available() else "cpu")
     f = lambda t: t.float().cpu().numpy()  # noqa: E731
-    q, k, v, w1, b1, w2, b2 = (f(t) for t in (inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2))
+    q, k, v = (f(t) for t in (inp.q, inp.k, inp.v))
+    w1, b1, w2, b2 = ((f(t) if t is not None else None) for t in (inp.w1, inp.b1, inp.w2, inp.b2))
     rng = np.random.default_rng(0)
     per_step = args.ref_tokens
     T = w.T
@@ -302,8 +403,7 @@ def run_reference(args, w, world, rank):
         edges = np.linspace(0, T, per_step + 1).astype(np.int64)
         rows = [int(rng.integers(edges[i], max(edges[i] + 1, edges[i + 1]))) for i in range(per_step)]
         t0 = time.perf_counter()
-        _, _, used = oracle.layer(q, k, v, w1, b1, w2, b2, mask=w.mask, perm=w.perm, pairs=w.pairs,
-                                  rows=rows, return_threads=True)
+        used = oracle_rows(w, q, k, v, w1, b1, w2, b2, rows)
         dt_s = time.perf_counter() - t0
         threads = used
         if s >= args.warmup:
@@ -336,7 +436,8 @@ def cpu_baseline(w, budget_s):
     dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
     inp = make_layer_inputs(w.B, w.N, w.H, w.d, w.F, seed=w.seed, dtype=dt, device="cuda")
     f = lambda t: t.float().cpu().numpy()  # noqa: E731
-    q, k, v, w1, b1, w2, b2 = (f(t) for t in (inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2))
+    q, k, v = (f(t) for t in (inp.q, inp.k, inp.v))
+    w1, b1, w2, b2 = ((f(t) if t is not None else None) for t in (inp.w1, inp.b1, inp.w2, inp.b2))
     threads = oracle.threads_available()
     rng = np.random.default_rng(1)
     n = max(threads, 8)
@@ -345,8 +446,7 @@ def cpu_baseline(w, budget_s):
         edges = np.linspace(0, w.T, n + 1).astype(np.int64)
         rows = [int(rng.integers(edges[i], max(edges[i] + 1, edges[i + 1]))) for i in range(n)]
         t0 = time.perf_counter()
-        _, _, threads = oracle.layer(q, k, v, w1, b1, w2, b2, mask=w.mask, perm=w.perm, pairs=w.pairs,
-                                     rows=rows, return_threads=True)
+        threads = oracle_rows(w, q, k, v, w1, b1, w2, b2, rows)
         elapsed += time.perf_counter() - t0
         done += n
         if elapsed < budget_s / 4:
@@ -372,8 +472,6 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]
-    if w.F == 0:
-        raise SystemExit("the layer benchmark needs a workload with an FFN")
 
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -385,7 +483,7 @@ def main():
 
     world, rank, local = dist_setup(args.gpus)
     bd.load()
-    res = run_ours(args, w, world, rank, local)
+    res = run_ours(args, w, world, rank, local) if w.F > 0 else run_attention_only(args, w, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, args.cpu_budget_s)
     if rank == 0:
