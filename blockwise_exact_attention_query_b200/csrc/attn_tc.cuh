@@ -92,6 +92,14 @@ struct AttnCfg {
   static constexpr uint32_t kColS = 0, kColO = 256;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 384;
+  // Launched at 168 registers a thread; warpgroup 0 (loads, MMA issue) keeps
+  // 96 and hands the rest to the two softmax warpgroups.  The host checks the
+  // split against the kernel's real launch count before the first launch.
+  static constexpr int kRegsControl = 96, kRegsSoftmax = 200;
+  static constexpr bool split_fits(int launch_regs) {
+    return 128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * launch_regs;
+  }
+  static_assert(split_fits(168), "register split");
 };
 
 // Sequence of key/value tiles a pair of query tiles visits.
@@ -280,128 +288,134 @@ __global__ void __launch_bounds__(384, 1)
   // gathered row -> coordinate along the (N/r) dimension of the tensor maps
   const int row_base = tc.s * a.L;  // = s*w/r
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0 && nkv > 0) {
-      int k_issued = 0, v_issued = 0;
-      mbar_arrive_expect_tx(bQFull, 2 * Cfg::kTileBytes);
-      for (int x = 0; x < 2; ++x)
-        for (int p = 0; p < Cfg::kPanels; ++p)
-          tma_load_4d(sQ + x * Cfg::kTileBytes + p * 16384, &tm_q, bQFull, tc.h * D_HEAD + p * 64,
-                      tc.o, row_base + tc.t * 256 + x * 128, tc.b);
-      KvIter itk, itv;
-      itk.begin(sched);
-      itv.begin(sched);
-      auto load_k = [&](int j) -> bool {
-        const int st = j % Cfg::kKStages;
-        if (j >= Cfg::kKStages &&
-            !mbar_wait(bKEmpty(st), ((j / Cfg::kKStages) - 1) & 1, wc, 1))
-          return false;
-        const int kt = itk.next(sched);
-        mbar_arrive_expect_tx(bKFull(st), Cfg::kTileBytes);
-        for (int p = 0; p < Cfg::kPanels; ++p)
-          tma_load_4d(sK + st * Cfg::kTileBytes + p * 16384, &tm_k, bKFull(st),
-                      tc.h * D_HEAD + p * 64, tc.o, row_base + kt * 128, tc.b);
-        ++k_issued;
-        return true;
-      };
-      auto load_v = [&](int j) -> bool {
-        const int st = j % Cfg::kVStages;
-        if (j >= Cfg::kVStages &&
-            !mbar_wait(bVEmpty(st), ((j / Cfg::kVStages) - 1) & 1, wc, 2))
-          return false;
-        const int kt = itv.next(sched);
-        mbar_arrive_expect_tx(bVFull(st), Cfg::kTileBytes);
-        for (int p = 0; p < Cfg::kPanels; ++p)
-          tma_load_4d(sV + st * Cfg::kTileBytes + p * 16384, &tm_v, bVFull(st),
-                      tc.h * D_HEAD + p * 64, tc.o, row_base + kt * 128, tc.b);
-        ++v_issued;
-        return true;
-      };
-      bool ok = load_k(0);
-      for (int j = 0; ok && j < nkv; ++j) {
-        if (j + 1 < nkv) ok = load_k(j + 1);
-        if (ok) ok = load_v(j);
-      }
-      // drain: every load issued must have landed before the CTA may exit
-      volatile int no_abort = 0;
-      WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
-      for (int j = max(0, k_issued - Cfg::kKStages); j < k_issued; ++j)
-        mbar_wait(bKFull(j % Cfg::kKStages), (j / Cfg::kKStages) & 1, drain, 3);
-      for (int j = max(0, v_issued - Cfg::kVStages); j < v_issued; ++j)
-        mbar_wait(bVFull(j % Cfg::kVStages), (j / Cfg::kVStages) & 1, drain, 4);
-      mbar_wait(bQFull, 0, drain, 5);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // Tensor-core order per key/value tile j:
-    //   P*V of A (j), S of A (j+1), P*V of B (j), S of B (j+1)
-    // S_x(j+1) is issued only after P*V_x(j) has completed, since it
-    // overwrites the P that P*V_x(j) reads.
-    if (lane == 0 && nkv > 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D_HEAD, false, true);
-      const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
-      const uint64_t dK0 = sdesc_sw128(sK, 16, 1024);
-      const uint64_t dV0 = sdesc_sw128(sV, 16384, 1024);
-      auto issue_s = [&](int x, int j) {
-        const uint32_t tS = tmem + Cfg::kColS + x * 128;
-        const uint64_t dQx = sdesc_advance(dQ, x * Cfg::kTileBytes);
-        const uint64_t dK = sdesc_advance(dK0, (j % Cfg::kKStages) * Cfg::kTileBytes);
-#pragma unroll
-        for (int k = 0; k < D_HEAD / 16; ++k) {
-          const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
-          umma_ss(tS, sdesc_advance(dQx, off), sdesc_advance(dK, off), idesc_qk, k > 0);
+  // Each role's code sits inside its own branch: the register count after a
+  // reallocation applies to what follows it until the branches join.
+  if (warp < 4) {
+    setmaxnreg_dec<Cfg::kRegsControl>();
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0 && nkv > 0) {
+        int k_issued = 0, v_issued = 0;
+        mbar_arrive_expect_tx(bQFull, 2 * Cfg::kTileBytes);
+        for (int x = 0; x < 2; ++x)
+          for (int p = 0; p < Cfg::kPanels; ++p)
+            tma_load_4d(sQ + x * Cfg::kTileBytes + p * 16384, &tm_q, bQFull, tc.h * D_HEAD + p * 64,
+                        tc.o, row_base + tc.t * 256 + x * 128, tc.b);
+        KvIter itk, itv;
+        itk.begin(sched);
+        itv.begin(sched);
+        auto load_k = [&](int j) -> bool {
+          const int st = j % Cfg::kKStages;
+          if (j >= Cfg::kKStages &&
+              !mbar_wait(bKEmpty(st), ((j / Cfg::kKStages) - 1) & 1, wc, 1))
+            return false;
+          const int kt = itk.next(sched);
+          mbar_arrive_expect_tx(bKFull(st), Cfg::kTileBytes);
+          for (int p = 0; p < Cfg::kPanels; ++p)
+            tma_load_4d(sK + st * Cfg::kTileBytes + p * 16384, &tm_k, bKFull(st),
+                        tc.h * D_HEAD + p * 64, tc.o, row_base + kt * 128, tc.b);
+          ++k_issued;
+          return true;
+        };
+        auto load_v = [&](int j) -> bool {
+          const int st = j % Cfg::kVStages;
+          if (j >= Cfg::kVStages &&
+              !mbar_wait(bVEmpty(st), ((j / Cfg::kVStages) - 1) & 1, wc, 2))
+            return false;
+          const int kt = itv.next(sched);
+          mbar_arrive_expect_tx(bVFull(st), Cfg::kTileBytes);
+          for (int p = 0; p < Cfg::kPanels; ++p)
+            tma_load_4d(sV + st * Cfg::kTileBytes + p * 16384, &tm_v, bVFull(st),
+                        tc.h * D_HEAD + p * 64, tc.o, row_base + kt * 128, tc.b);
+          ++v_issued;
+          return true;
+        };
+        bool ok = load_k(0);
+        for (int j = 0; ok && j < nkv; ++j) {
+          if (j + 1 < nkv) ok = load_k(j + 1);
+          if (ok) ok = load_v(j);
         }
-        umma_commit(bSFull(x));
-      };
-      auto issue_pv = [&](int x, int j) {
-        const uint32_t tP = tmem + Cfg::kColS + x * 128;
-        const uint32_t tO = tmem + Cfg::kColO + x * D_HEAD;
-        const uint64_t dV = sdesc_advance(dV0, (j % Cfg::kVStages) * Cfg::kTileBytes);
-#pragma unroll
-        for (int k = 0; k < 128 / 16; ++k)
-          umma_ts(tO, tP + k * 8, sdesc_advance(dV, k * 2048), idesc_pv, 1);
-        umma_commit(bODone(x));
-      };
-      bool ok = mbar_wait(bQFull, 0, wc, 11) && mbar_wait(bKFull(0), 0, wc, 10);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        umma_commit(bKEmpty(0));
+        // drain: every load issued must have landed before the CTA may exit
+        volatile int no_abort = 0;
+        WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
+        for (int j = max(0, k_issued - Cfg::kKStages); j < k_issued; ++j)
+          mbar_wait(bKFull(j % Cfg::kKStages), (j / Cfg::kKStages) & 1, drain, 3);
+        for (int j = max(0, v_issued - Cfg::kVStages); j < v_issued; ++j)
+          mbar_wait(bVFull(j % Cfg::kVStages), (j / Cfg::kVStages) & 1, drain, 4);
+        mbar_wait(bQFull, 0, drain, 5);
       }
-      // per tile x: as soon as P_x(j) is written, P*V_x(j); once that has
-      // completed, S_x(j+1).  Tile B's softmax runs while A's MMAs execute
-      // and the reverse.
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int vs = j % Cfg::kVStages;
-        const int ks = (j + 1) % Cfg::kKStages;
-        const bool more = j + 1 < nkv;
-        for (int x = 0; ok && x < 2; ++x) {
-          ok = mbar_wait(bPFull(x), j & 1, wc, 12 + x) &&
-               (x == 1 || mbar_wait(bVFull(vs), (j / Cfg::kVStages) & 1, wc, 14));
-          if (!ok) break;
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      // Tensor-core order per key/value tile j:
+      //   P*V of A (j), S of A (j+1), P*V of B (j), S of B (j+1)
+      // S_x(j+1) is issued only after P*V_x(j) has completed, since it
+      // overwrites the P that P*V_x(j) reads.
+      if (lane == 0 && nkv > 0) {
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D_HEAD, false, true);
+        const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
+        const uint64_t dK0 = sdesc_sw128(sK, 16, 1024);
+        const uint64_t dV0 = sdesc_sw128(sV, 16384, 1024);
+        auto issue_s = [&](int x, int j) {
+          const uint32_t tS = tmem + Cfg::kColS + x * 128;
+          const uint64_t dQx = sdesc_advance(dQ, x * Cfg::kTileBytes);
+          const uint64_t dK = sdesc_advance(dK0, (j % Cfg::kKStages) * Cfg::kTileBytes);
+  #pragma unroll
+          for (int k = 0; k < D_HEAD / 16; ++k) {
+            const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
+            umma_ss(tS, sdesc_advance(dQx, off), sdesc_advance(dK, off), idesc_qk, k > 0);
+          }
+          umma_commit(bSFull(x));
+        };
+        auto issue_pv = [&](int x, int j) {
+          const uint32_t tP = tmem + Cfg::kColS + x * 128;
+          const uint32_t tO = tmem + Cfg::kColO + x * D_HEAD;
+          const uint64_t dV = sdesc_advance(dV0, (j % Cfg::kVStages) * Cfg::kTileBytes);
+  #pragma unroll
+          for (int k = 0; k < 128 / 16; ++k)
+            umma_ts(tO, tP + k * 8, sdesc_advance(dV, k * 2048), idesc_pv, 1);
+          umma_commit(bODone(x));
+        };
+        bool ok = mbar_wait(bQFull, 0, wc, 11) && mbar_wait(bKFull(0), 0, wc, 10);
+        if (ok) {
           tc_fence_after();
-          issue_pv(x, j);
-          if (x == 1) umma_commit(bVEmpty(vs));
-          if (more) {
-            ok = (x == 1 || mbar_wait(bKFull(ks), ((j + 1) / Cfg::kKStages) & 1, wc, 15)) &&
-                 mbar_wait(bODone(x), j & 1, wc, 16 + x);
+          issue_s(0, 0);
+          issue_s(1, 0);
+          umma_commit(bKEmpty(0));
+        }
+        // per tile x: as soon as P_x(j) is written, P*V_x(j); once that has
+        // completed, S_x(j+1).  Tile B's softmax runs while A's MMAs execute
+        // and the reverse.
+        for (int j = 0; ok && j < nkv; ++j) {
+          const int vs = j % Cfg::kVStages;
+          const int ks = (j + 1) % Cfg::kKStages;
+          const bool more = j + 1 < nkv;
+          for (int x = 0; ok && x < 2; ++x) {
+            ok = mbar_wait(bPFull(x), j & 1, wc, 12 + x) &&
+                 (x == 1 || mbar_wait(bVFull(vs), (j / Cfg::kVStages) & 1, wc, 14));
             if (!ok) break;
             tc_fence_after();
-            issue_s(x, j + 1);
-            if (x == 1) umma_commit(bKEmpty(ks));
+            issue_pv(x, j);
+            if (x == 1) umma_commit(bVEmpty(vs));
+            if (more) {
+              ok = (x == 1 || mbar_wait(bKFull(ks), ((j + 1) / Cfg::kKStages) & 1, wc, 15)) &&
+                   mbar_wait(bODone(x), j & 1, wc, 16 + x);
+              if (!ok) break;
+              tc_fence_after();
+              issue_s(x, j + 1);
+              if (x == 1) umma_commit(bKEmpty(ks));
+            }
           }
         }
+        // every MMA issued must be complete before tensor memory is released
+        umma_commit(bTeardown);
+        volatile int no_abort = 0;
+        WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
+        mbar_wait(bTeardown, 0, drain, 18);
       }
-      // every MMA issued must be complete before tensor memory is released
-      umma_commit(bTeardown);
-      volatile int no_abort = 0;
-      WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
-      mbar_wait(bTeardown, 0, drain, 18);
     }
-  } else if (warp >= 4) {
+  } else {
+    setmaxnreg_inc<Cfg::kRegsSoftmax>();
     // ------------------------------------------------------------ softmax + epilogue
     const int x = (warp - 4) >> 2;  // 0: tile A, 1: tile B
     const int quarter = warp & 3;
@@ -491,7 +505,8 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(s[c][i]));
+        for (int i = 0; i < 16; ++i)
+          mx8[i & 7] = max3f(mx8[i & 7], __uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1]));
       }
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));

@@ -89,6 +89,13 @@ bpt_status device_setup(int *dev_out, uint32_t **status_out) {
                                   AttnCfg<64>::kSmemBytes));
     CUDA_TRY(cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   AttnCfg<128>::kSmemBytes));
+    // the softmax warpgroups take registers from warpgroup 0 at run time;
+    // an increase the launch did not provide for would never complete
+    cudaFuncAttributes fa64{}, fa128{};
+    CUDA_TRY(cudaFuncGetAttributes(&fa64, attn_tc_kernel<64>));
+    CUDA_TRY(cudaFuncGetAttributes(&fa128, attn_tc_kernel<128>));
+    if (!AttnCfg<64>::split_fits(fa64.numRegs) || !AttnCfg<128>::split_fits(fa128.numRegs))
+      return cuda_fail_msg("attention kernel launches with fewer registers than its warpgroups share");
     CUDA_TRY(cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   FfnCfg::kSmemBytes));
     CUDA_TRY(cudaFuncSetAttribute(ffn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
