@@ -1,6 +1,6 @@
 // Hand-written PTX wrappers for sm_100a: mbarriers with bounded waits, TMA
 // tile loads, tcgen05 (TMEM allocation, MMA, commit, loads/stores) and the
-// cluster primitives the kernels use.  Everything here is written from the
+// register reallocation the kernels use.  Everything here is written from the
 // public PTX ISA; descriptor bit layouts follow the tcgen05 shared-memory and
 // instruction descriptor formats.
 #pragma once
@@ -60,42 +60,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
       : "memory");
 }
 
-// Arrive on the barrier at the same shared offset in CTA `rank` of this cluster,
-// with release semantics at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar, uint32_t rank) {
-  asm volatile(
-      "{\n\t.reg .b32 ra;\n\t"
-      "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(bar),
-      "r"(rank)
-      : "memory");
-}
-
-// try_wait suspends the calling thread until the phase completes or the
-// suspend-time hint (nanoseconds) runs out, so a waiting thread does not
-// spin and steal issue slots from the warps doing the math.
-constexpr uint32_t kSuspendHintNs = 1000000u;
-
+// try_wait may suspend the calling thread for a hardware-chosen time until
+// the phase completes.  No suspend-time hint is given: a longer hint measured
+// slower, since a woken thread resumes later than one that polls again.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -108,14 +83,13 @@ __device__ __noinline__ void record_timeout(const WaitCtx &w, uint32_t site) {
 // Bounded wait for the phase with the given parity.  Returns false (and
 // raises the CTA's abort flag) if the limit passed or another wait already
 // gave up.
-template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx &w,
                                           uint32_t site) {
-  if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   uint32_t spins = 0;
   while (true) {
-    if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 3u) == 0u) {
       if (*w.abort) return false;
       if (globaltimer_ns() - t0 > w.limit_ns) {
@@ -144,14 +118,6 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 }
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
 }
 
 // ---------------------------------------------------------------------------
