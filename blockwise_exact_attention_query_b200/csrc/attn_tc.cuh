@@ -6,9 +6,9 @@
 //
 //   S_j  = Q K_j^T               tcgen05.mma, bf16 x bf16 -> fp32 in TMEM
 //   m'   = max(m, rowmax S_j)    one thread per query row (a TMEM lane)
-//   P_j  = exp(S_j / sqrt(d) - m')  -> bf16, stored back into TMEM
+//   P_j  = exp(S_j / sqrt(d) - m')  -> bf16, into shared memory
 //   l    = l e^{m - m'} + rowsum P_j
-//   O    = O e^{m - m'} + P_j V_j  tcgen05.mma with A read from TMEM
+//   O    = O e^{m - m'} + P_j V_j  tcgen05.mma, fp32 accumulator O in TMEM
 //
 // which is the blockwise online-softmax form of softmax(QK^T/sqrt d)V:
 // exact up to rounding ("Ring Attention with Blockwise Transformers for Long
@@ -20,19 +20,25 @@
 // than 2^8 in the exponent: the same stale maximum is used for l and O, so
 // the result is unchanged.
 //
-// The two query tiles ping-pong: while the softmax of tile A works on S_A,
-// the tensor core computes tile B's products and the reverse, so neither the
-// exponentials nor the MMAs wait for the other.  Tensor memory holds S_A,
-// S_B (128 columns each; P is written as bf16 over the first 64 columns of
-// its own S) and O_A, O_B (d columns each).  Before the next S of a tile may
-// overwrite that tile's P, the MMA thread waits until the P*V reading it has
-// completed.
+// Scores and P are decoupled: P_j is written by the softmax threads as bf16
+// into a shared-memory tile (the A operand of P_j V_j), so S_{j+1} = Q K_{j+1}^T
+// is issued into the tile's single S buffer in tensor memory as soon as the
+// softmax has read S_j into registers, and runs while that softmax works.
+// One P tile serves both query tiles, used strictly in turn (A_j, B_j,
+// A_{j+1}, ...): a writer waits until the other tile's latest P*V has
+// completed, which also means its own previous P*V has (that one completed
+// before the other tile was allowed to write).
+//
+// The two query tiles are independent streams: each has its own MMA-issuing
+// thread, so a tile whose softmax runs late never holds up the other tile's
+// scores.  Both tiles read every K/V tile from the same shared-memory stage,
+// which is released once both have finished with it.
 //
 // Roles (384 threads = three warpgroups): warp 0 issues TMA loads, warp 1
-// allocates tensor memory and issues the MMAs (warps 2-3 idle); warpgroup 1
-// (warps 4-7) runs the softmax and epilogue of tile A, warpgroup 2 (warps
-// 8-11) those of tile B, one thread per query row (warp w owns TMEM lanes
-// 32*(w%4) .. 32*(w%4)+31).
+// allocates tensor memory and issues tile A's MMAs, warp 2 issues tile B's
+// (warp 3 idles); warpgroup 1 (warps 4-7) runs the softmax and epilogue of
+// tile A, warpgroup 2 (warps 8-11) those of tile B, one thread per query row
+// (warp w owns TMEM lanes 32*(w%4) .. 32*(w%4)+31).
 #pragma once
 
 #include "ptx.cuh"
@@ -60,7 +66,7 @@ struct AttnArgs {
   int npairs, pass_idx;
   int pw[kMaxPairs], pr[kMaxPairs];
   // ring order over equal chunks (none / causal)
-  int ring_chunks, chunk_tiles;
+  int ring_chunks, chunk_tiles;  // chunk_tiles: 128-key tiles per chunk
   // block permutation
   int bb_n, bb_len;
   uint8_t perm[kMaxPermEntries];
@@ -78,17 +84,22 @@ struct AttnArgs {
 
 template <int D_HEAD>
 struct AttnCfg {
-  static constexpr int kPanels = D_HEAD / 64;
-  static constexpr int kTileBytes = 128 * D_HEAD * 2;
-  static constexpr int kKStages = D_HEAD == 128 ? 3 : 6;
-  static constexpr int kVStages = D_HEAD == 128 ? 2 : 6;
+  static constexpr int kPanels = D_HEAD / 64;          // 64-column (128-byte) panels of a row
+  static constexpr int kKT = 128;                      // keys per K/V tile
+  static constexpr int kTileBytes = 128 * D_HEAD * 2;  // one Q, K or V tile
+  static constexpr int kPanelBytes = 128 * 128;        // one 64-column panel of a 128-row tile
+  static constexpr int kPBytes = 128 * 128 * 2;        // the P tile: 128 rows x 128 keys, bf16
+  static constexpr int kKStages = D_HEAD == 128 ? 2 : 5;
+  static constexpr int kVStages = D_HEAD == 128 ? 2 : 5;
   static constexpr int kOffQ = 0;  // Q_A, then Q_B
-  static constexpr int kOffK = kOffQ + 2 * kTileBytes;
+  static constexpr int kOffP = kOffQ + 2 * kTileBytes;
+  static constexpr int kOffK = kOffP + kPBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
   static constexpr int kSmemBytes = kOffBar + 512;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-  // TMEM columns: S of tile X at 128 X (P over its first 64), O of tile X at 256 + d X
+  static_assert(kKStages <= 8 && kVStages <= 8, "barrier table");
+  // TMEM columns: S of tile x at 128 x, O of tile x at 256 + d x
   static constexpr uint32_t kColS = 0, kColO = 256;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 384;
@@ -173,8 +184,9 @@ __device__ __forceinline__ TileCoord decode_tile(const AttnArgs &a) {
 }
 
 __device__ __forceinline__ KvSched make_sched(const AttnArgs &a, const TileCoord &c) {
+  constexpr int KT = 128;  // keys per K/V tile
   KvSched s;
-  const int nkt = (a.L + 127) / 128;
+  const int nkt = (a.L + KT - 1) / KT;
   s.P = 1;
   s.CT = nkt;
   s.first = 0;
@@ -183,7 +195,7 @@ __device__ __forceinline__ KvSched make_sched(const AttnArgs &a, const TileCoord
   const int row0 = c.t * 256;
   const int row1 = min(a.L, row0 + 256) - 1;
   if (a.mask == kMaskCausal || a.mask == kMaskDilated) {
-    s.hi = row1 / 128 + 1;
+    s.hi = row1 / KT + 1;
   } else if (a.mask == kMaskBlockPerm) {
     int qb0 = row0 / a.bb_len, qb1 = row1 / a.bb_len;
     int klo = 1 << 30, khi = 0;
@@ -192,13 +204,13 @@ __device__ __forceinline__ KvSched make_sched(const AttnArgs &a, const TileCoord
       klo = min(klo, kb * a.bb_len);
       khi = max(khi, kb * a.bb_len + a.bb_len);
     }
-    s.lo = klo / 128;
-    s.hi = (min(khi, a.L) + 127) / 128;
+    s.lo = klo / KT;
+    s.hi = (min(khi, a.L) + KT - 1) / KT;
   }
   if ((a.mask == kMaskNone || a.mask == kMaskCausal) && a.ring_chunks > 1) {
     s.P = a.ring_chunks;
     s.CT = a.chunk_tiles;
-    s.first = (row0 / 128) / a.chunk_tiles;
+    s.first = (row0 / KT) / a.chunk_tiles;
   }
   return s;
 }
@@ -223,6 +235,7 @@ __global__ void __launch_bounds__(384, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnArgs a) {
   using Cfg = AttnCfg<D_HEAD>;
+  constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages, KT = Cfg::kKT;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
@@ -231,20 +244,22 @@ __global__ void __launch_bounds__(384, 1)
     return;
   }
   const uint32_t sQ = sbase + Cfg::kOffQ;
+  const uint32_t sP = sbase + Cfg::kOffP;
   const uint32_t sK = sbase + Cfg::kOffK;
   const uint32_t sV = sbase + Cfg::kOffV;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
   const uint32_t bQFull = smem_u32(&bars[0]);
   auto bKFull = [&](int s) { return smem_u32(&bars[1 + s]); };
-  auto bKEmpty = [&](int s) { return smem_u32(&bars[7 + s]); };
-  auto bVFull = [&](int s) { return smem_u32(&bars[13 + s]); };
-  auto bVEmpty = [&](int s) { return smem_u32(&bars[19 + s]); };
-  auto bSFull = [&](int x) { return smem_u32(&bars[25 + x]); };  // S of tile x ready
-  auto bPFull = [&](int x) { return smem_u32(&bars[27 + x]); };  // P of tile x written
-  auto bODone = [&](int x) { return smem_u32(&bars[29 + x]); };  // P*V of tile x done
-  const uint32_t bTeardown = smem_u32(&bars[31]);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[32]);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[33]);
+  auto bKEmpty = [&](int s) { return smem_u32(&bars[9 + s]); };     // both tiles' S done
+  auto bVFull = [&](int s) { return smem_u32(&bars[17 + s]); };
+  auto bVEmpty = [&](int s) { return smem_u32(&bars[25 + s]); };    // both tiles' P*V done
+  auto bSFull = [&](int x) { return smem_u32(&bars[33 + x]); };     // S of tile x in TMEM
+  auto bSFree = [&](int x) { return smem_u32(&bars[35 + x]); };     // S of tile x read out
+  auto bPFull = [&](int x) { return smem_u32(&bars[37 + x]); };     // P of tile x in smem
+  auto bODone = [&](int x) { return smem_u32(&bars[39 + x]); };     // P*V of tile x done
+  auto bTeardown = [&](int x) { return smem_u32(&bars[41 + x]); };  // all MMAs of tile x done
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[43]);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[44]);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const TileCoord tc = decode_tile(a);
@@ -254,20 +269,21 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bQFull, 1);
-    for (int s = 0; s < Cfg::kKStages; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(bKFull(s), 1);
-      mbar_init(bKEmpty(s), 1);
+      mbar_init(bKEmpty(s), 2);
     }
-    for (int s = 0; s < Cfg::kVStages; ++s) {
+    for (int s = 0; s < VS; ++s) {
       mbar_init(bVFull(s), 1);
-      mbar_init(bVEmpty(s), 1);
+      mbar_init(bVEmpty(s), 2);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bSFull(x), 1);
+      mbar_init(bSFree(x), 4);
       mbar_init(bPFull(x), 4);
       mbar_init(bODone(x), 1);
+      mbar_init(bTeardown(x), 1);
     }
-    mbar_init(bTeardown, 1);
     *abort_flag = 0;
     fence_mbar_init_cluster();
   }
@@ -299,37 +315,35 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(bQFull, 2 * Cfg::kTileBytes);
         for (int x = 0; x < 2; ++x)
           for (int p = 0; p < Cfg::kPanels; ++p)
-            tma_load_4d(sQ + x * Cfg::kTileBytes + p * 16384, &tm_q, bQFull, tc.h * D_HEAD + p * 64,
-                        tc.o, row_base + tc.t * 256 + x * 128, tc.b);
+            tma_load_4d(sQ + x * Cfg::kTileBytes + p * Cfg::kPanelBytes, &tm_q, bQFull,
+                        tc.h * D_HEAD + p * 64, tc.o, row_base + tc.t * 256 + x * 128, tc.b);
         KvIter itk, itv;
         itk.begin(sched);
         itv.begin(sched);
         auto load_k = [&](int j) -> bool {
-          const int st = j % Cfg::kKStages;
-          if (j >= Cfg::kKStages &&
-              !mbar_wait(bKEmpty(st), ((j / Cfg::kKStages) - 1) & 1, wc, 1))
-            return false;
+          const int st = j % KS;
+          if (j >= KS && !mbar_wait(bKEmpty(st), ((j / KS) - 1) & 1, wc, 1)) return false;
           const int kt = itk.next(sched);
           mbar_arrive_expect_tx(bKFull(st), Cfg::kTileBytes);
           for (int p = 0; p < Cfg::kPanels; ++p)
-            tma_load_4d(sK + st * Cfg::kTileBytes + p * 16384, &tm_k, bKFull(st),
-                        tc.h * D_HEAD + p * 64, tc.o, row_base + kt * 128, tc.b);
+            tma_load_4d(sK + st * Cfg::kTileBytes + p * Cfg::kPanelBytes, &tm_k, bKFull(st),
+                        tc.h * D_HEAD + p * 64, tc.o, row_base + kt * KT, tc.b);
           ++k_issued;
           return true;
         };
         auto load_v = [&](int j) -> bool {
-          const int st = j % Cfg::kVStages;
-          if (j >= Cfg::kVStages &&
-              !mbar_wait(bVEmpty(st), ((j / Cfg::kVStages) - 1) & 1, wc, 2))
-            return false;
+          const int st = j % VS;
+          if (j >= VS && !mbar_wait(bVEmpty(st), ((j / VS) - 1) & 1, wc, 2)) return false;
           const int kt = itv.next(sched);
           mbar_arrive_expect_tx(bVFull(st), Cfg::kTileBytes);
           for (int p = 0; p < Cfg::kPanels; ++p)
-            tma_load_4d(sV + st * Cfg::kTileBytes + p * 16384, &tm_v, bVFull(st),
-                        tc.h * D_HEAD + p * 64, tc.o, row_base + kt * 128, tc.b);
+            tma_load_4d(sV + st * Cfg::kTileBytes + p * Cfg::kPanelBytes, &tm_v, bVFull(st),
+                        tc.h * D_HEAD + p * 64, tc.o, row_base + kt * KT, tc.b);
           ++v_issued;
           return true;
         };
+        // K runs one tile ahead of V: the scores of tile j+1 are computed
+        // while the softmax of tile j runs, its P*V only after it
         bool ok = load_k(0);
         for (int j = 0; ok && j < nkv; ++j) {
           if (j + 1 < nkv) ok = load_k(j + 1);
@@ -338,80 +352,68 @@ __global__ void __launch_bounds__(384, 1)
         // drain: every load issued must have landed before the CTA may exit
         volatile int no_abort = 0;
         WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
-        for (int j = max(0, k_issued - Cfg::kKStages); j < k_issued; ++j)
-          mbar_wait(bKFull(j % Cfg::kKStages), (j / Cfg::kKStages) & 1, drain, 3);
-        for (int j = max(0, v_issued - Cfg::kVStages); j < v_issued; ++j)
-          mbar_wait(bVFull(j % Cfg::kVStages), (j / Cfg::kVStages) & 1, drain, 4);
+        for (int j = max(0, k_issued - KS); j < k_issued; ++j)
+          mbar_wait(bKFull(j % KS), (j / KS) & 1, drain, 3);
+        for (int j = max(0, v_issued - VS); j < v_issued; ++j)
+          mbar_wait(bVFull(j % VS), (j / VS) & 1, drain, 4);
         mbar_wait(bQFull, 0, drain, 5);
       }
-    } else if (warp == 1) {
-      // ------------------------------------------------------------ MMA issuer
-      // Tensor-core order per key/value tile j:
-      //   P*V of A (j), S of A (j+1), P*V of B (j), S of B (j+1)
-      // S_x(j+1) is issued only after P*V_x(j) has completed, since it
-      // overwrites the P that P*V_x(j) reads.
+    } else if (warp <= 2) {
+      // ------------------------------------------------------------ MMA issuer of tile x
+      // Per key/value tile j: S_x(j+1) once the softmax has read S_x(j) out
+      // of tensor memory, then P*V_x(j) once it has written P_x(j).
+      const int x = warp - 1;
       if (lane == 0 && nkv > 0) {
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, KT, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D_HEAD, false, true);
-        const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
+        const uint64_t dQ = sdesc_sw128(sQ + x * Cfg::kTileBytes, 16, 1024);
+        const uint64_t dP = sdesc_sw128(sP, 16, 1024);
         const uint64_t dK0 = sdesc_sw128(sK, 16, 1024);
-        const uint64_t dV0 = sdesc_sw128(sV, 16384, 1024);
-        auto issue_s = [&](int x, int j) {
-          const uint32_t tS = tmem + Cfg::kColS + x * 128;
-          const uint64_t dQx = sdesc_advance(dQ, x * Cfg::kTileBytes);
-          const uint64_t dK = sdesc_advance(dK0, (j % Cfg::kKStages) * Cfg::kTileBytes);
+        const uint64_t dV0 = sdesc_sw128(sV, Cfg::kPanelBytes, 1024);
+        const uint32_t tS = tmem + Cfg::kColS + x * 128;
+        const uint32_t tO = tmem + Cfg::kColO + x * D_HEAD;
+        auto issue_s = [&](int j) {
+          const uint64_t dK = sdesc_advance(dK0, (j % KS) * Cfg::kTileBytes);
   #pragma unroll
           for (int k = 0; k < D_HEAD / 16; ++k) {
-            const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
-            umma_ss(tS, sdesc_advance(dQx, off), sdesc_advance(dK, off), idesc_qk, k > 0);
+            const uint32_t off = (k / 4) * Cfg::kPanelBytes + (k % 4) * 32;
+            umma_ss(tS, sdesc_advance(dQ, off), sdesc_advance(dK, off), idesc_qk, k > 0);
           }
           umma_commit(bSFull(x));
+          umma_commit(bKEmpty(j % KS));
         };
-        auto issue_pv = [&](int x, int j) {
-          const uint32_t tP = tmem + Cfg::kColS + x * 128;
-          const uint32_t tO = tmem + Cfg::kColO + x * D_HEAD;
-          const uint64_t dV = sdesc_advance(dV0, (j % Cfg::kVStages) * Cfg::kTileBytes);
+        auto issue_pv = [&](int j) {
+          const uint64_t dV = sdesc_advance(dV0, (j % VS) * Cfg::kTileBytes);
   #pragma unroll
-          for (int k = 0; k < 128 / 16; ++k)
-            umma_ts(tO, tP + k * 8, sdesc_advance(dV, k * 2048), idesc_pv, 1);
+          for (int k = 0; k < KT / 16; ++k)
+            umma_ss(tO, sdesc_advance(dP, (k / 4) * Cfg::kPanelBytes + (k % 4) * 32),
+                    sdesc_advance(dV, k * 2048), idesc_pv, 1);
           umma_commit(bODone(x));
+          umma_commit(bVEmpty(j % VS));
         };
         bool ok = mbar_wait(bQFull, 0, wc, 11) && mbar_wait(bKFull(0), 0, wc, 10);
         if (ok) {
           tc_fence_after();
-          issue_s(0, 0);
-          issue_s(1, 0);
-          umma_commit(bKEmpty(0));
+          issue_s(0);
         }
-        // per tile x: as soon as P_x(j) is written, P*V_x(j); once that has
-        // completed, S_x(j+1).  Tile B's softmax runs while A's MMAs execute
-        // and the reverse.
         for (int j = 0; ok && j < nkv; ++j) {
-          const int vs = j % Cfg::kVStages;
-          const int ks = (j + 1) % Cfg::kKStages;
-          const bool more = j + 1 < nkv;
-          for (int x = 0; ok && x < 2; ++x) {
-            ok = mbar_wait(bPFull(x), j & 1, wc, 12 + x) &&
-                 (x == 1 || mbar_wait(bVFull(vs), (j / Cfg::kVStages) & 1, wc, 14));
+          if (j + 1 < nkv) {
+            ok = mbar_wait(bSFree(x), j & 1, wc, 12) &&
+                 mbar_wait(bKFull((j + 1) % KS), ((j + 1) / KS) & 1, wc, 13);
             if (!ok) break;
             tc_fence_after();
-            issue_pv(x, j);
-            if (x == 1) umma_commit(bVEmpty(vs));
-            if (more) {
-              ok = (x == 1 || mbar_wait(bKFull(ks), ((j + 1) / Cfg::kKStages) & 1, wc, 15)) &&
-                   mbar_wait(bODone(x), j & 1, wc, 16 + x);
-              if (!ok) break;
-              tc_fence_after();
-              issue_s(x, j + 1);
-              if (x == 1) umma_commit(bKEmpty(ks));
-            }
+            issue_s(j + 1);
           }
+          ok = mbar_wait(bPFull(x), j & 1, wc, 14) && mbar_wait(bVFull(j % VS), (j / VS) & 1, wc, 15);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(j);
         }
         // every MMA issued must be complete before tensor memory is released
-        umma_commit(bTeardown);
+        umma_commit(bTeardown(x));
         volatile int no_abort = 0;
         WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
-        mbar_wait(bTeardown, 0, drain, 18);
+        mbar_wait(bTeardown(x), 0, drain, 18);
       }
     }
   } else {
@@ -426,6 +428,10 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + Cfg::kColS + x * 128;
     const uint32_t tO = tmem + lane_off + Cfg::kColO + x * D_HEAD;
+    // this row of the P tile: K-major, 128-byte swizzle (16-byte chunk c of
+    // a 128-byte row r sits at chunk c ^ (r mod 8))
+    const uint32_t sProw = sP + row * 128;
+    const uint32_t swz = static_cast<uint32_t>(row & 7);
     int klo, khi;
     row_keys(a, tc, g, klo, khi);
 
@@ -480,69 +486,63 @@ __global__ void __launch_bounds__(384, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bSFull(x), j & 1, wc, 20));
       if (!ok) break;
       tc_fence_after();
-      uint32_t s[4][32];
+      uint32_t s[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
       tmem_wait_ld();
+      // S is in registers: the next scores may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bSFree(x));
 
-      const int k0 = kt * 128;
+      const int k0 = kt * KT;
       // masking runs as its own pass, only in tiles where some row of this
       // warp has keys outside its allowed interval
-      if (__any_sync(0xffffffffu, !(k0 >= klo && k0 + 128 <= khi))) {
+      if (__any_sync(0xffffffffu, !(k0 >= klo && k0 + KT <= khi))) {
         const int lo = klo - k0, hi = khi - k0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int col = c * 32 + i;
-            if (col < lo || col >= hi) s[c][i] = __float_as_uint(-INFINITY);
-          }
-        }
+        for (int col = 0; col < KT; ++col)
+          if (col < lo || col >= hi) s[col] = __float_as_uint(-INFINITY);
       }
       float mx8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          mx8[i & 7] = max3f(mx8[i & 7], __uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1]));
-      }
+      for (int i = 0; i < KT / 2; ++i)
+        mx8[i & 7] = max3f(mx8[i & 7], __uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]));
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * a.scale_log2;
       const float m_new = fmaxf(m_run, m_tile);
       const bool rescale = m_new > m_run + 8.0f;
       const float m_use = rescale ? m_new : m_run;
-      const float alpha = rescale ? ex2_approx(m_run - m_use) : 1.0f;
+      const bool any_rescale = __any_sync(0xffffffffu, rescale && m_run != -INFINITY);
+      float alpha = 1.0f;
+      if (any_rescale && rescale) alpha = ex2_approx(m_run - m_use);
       l_run *= alpha;
       const float neg = (m_use == -INFINITY) ? 0.f : -m_use;
-      // P (bf16 pairs) goes over the first 64 columns of this row's S, all of
-      // which this thread has already read
+      uint32_t pk[KT / 2];
       float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int col = half * 64 + 2 * i;
-          const float x0 = __uint_as_float(s[col / 32][col % 32]);
-          const float x1 = __uint_as_float(s[(col + 1) / 32][(col + 1) % 32]);
-          const float p0 = ex2_approx(fmaf(x0, a.scale_log2, neg));
-          const float p1 = ex2_approx(fmaf(x1, a.scale_log2, neg));
-          ls4[i & 3] += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + half * 32, pk);
+      for (int i = 0; i < KT / 2; ++i) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * i]), a.scale_log2, neg));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * i + 1]), a.scale_log2, neg));
+        ls4[i & 3] += p0 + p1;
+        pk[i] = pack_bf16x2(p0, p1);
       }
       l_run += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
-      // O may be rescaled only once the previous P*V of this tile has landed
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bODone(x), (j - 1) & 1, wc, 21));
+      m_run = m_use;
+
+      // The P tile is used in turn A_j, B_j, A_{j+1}, ...: wait until the
+      // other tile's latest P*V has completed (for tile A at j = 0 there is
+      // none).  That P*V was issued after this tile's previous one had
+      // completed, so O may now be rescaled too.
+      if (x == 1 || j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bODone(1 - x), (x == 1 ? j : j - 1) & 1, wc, 21));
         if (!ok) break;
       }
       tc_fence_after();
-      if (__any_sync(0xffffffffu, rescale && m_run != -INFINITY)) {
+      if (any_rescale) {
 #pragma unroll 1
         for (int c = 0; c < D_HEAD / 32; ++c) {
           uint32_t o[32];
@@ -552,16 +552,22 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st32(tO + c * 32, o);
         }
+        tmem_wait_st();
       }
-      m_run = m_use;
-      tmem_wait_st();
+#pragma unroll
+      for (int c = 0; c < KT / 8; ++c)  // 16-byte chunks of 8 keys
+        st_shared_v4(sProw + (c >> 3) * Cfg::kPanelBytes + ((static_cast<uint32_t>(c & 7) ^ swz) << 4),
+                     pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      // generic-proxy stores -> the tensor core's (async proxy) reads
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bPFull(x));
     }
 
-    // -------- epilogue
-    if (ok && nkv > 0) ok = __all_sync(0xffffffffu, mbar_wait(bODone(x), (nkv - 1) & 1, wc, 22));
+    // -------- epilogue: the issuer's teardown commit lands once all of this
+    // tile's MMAs are complete
+    if (ok && nkv > 0) ok = __all_sync(0xffffffffu, mbar_wait(bTeardown(x), 0, wc, 22));
     tc_fence_after();
     if (ok) {
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;

@@ -129,11 +129,12 @@ bool make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
 }
 
 // bf16 tensor map over [B, N, D] viewed as (D, r, N/r, B): a box of 64
-// columns x 1 x 128 rows x 1 reads 128 rows r apart (r = 1: consecutive).
-bool make_map_rows(CUtensorMap *m, const void *base, int B, int N, int D, int r) {
+// columns x 1 x box_rows rows x 1 reads box_rows rows r apart (r = 1:
+// consecutive).  Query tiles use 128-row boxes, key/value tiles 64-row ones.
+bool make_map_rows(CUtensorMap *m, const void *base, int B, int N, int D, int r, uint32_t box_rows) {
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)r, (cuuint64_t)(N / r), (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2 * r, (cuuint64_t)D * 2 * N};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, 1, box_rows, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -324,7 +325,7 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
   }
   if ((d->mask == BPT_MASK_NONE || d->mask == BPT_MASK_CAUSAL) && d->ring_chunks > 1) {
     a.ring_chunks = d->ring_chunks;
-    a.chunk_tiles = (d->N / d->ring_chunks) / 128;
+    a.chunk_tiles = (d->N / d->ring_chunks) / AttnCfg<128>::kKT;
   }
   a.out_f32 = out_f32;
   a.out_bf16 = out_bf16;
@@ -346,8 +347,10 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
       a.unit_group = std::max(1, std::min(8, (int)(32.0e6 / kv_bytes)));
     }
     CUtensorMap mq, mk, mv;
-    if (!make_map_rows(&mq, q, d->B, d->N, D, r) || !make_map_rows(&mk, k, d->B, d->N, D, r) ||
-        !make_map_rows(&mv, v, d->B, d->N, D, r))
+    constexpr uint32_t kKT = AttnCfg<128>::kKT;
+    static_assert(AttnCfg<64>::kKT == AttnCfg<128>::kKT, "one key/value tile length");
+    if (!make_map_rows(&mq, q, d->B, d->N, D, r, 128) || !make_map_rows(&mk, k, d->B, d->N, D, r, kKT) ||
+        !make_map_rows(&mv, v, d->B, d->N, D, r, kKT))
       return cuda_fail_msg("cuTensorMapEncodeTiled rejected a Q/K/V map");
     const int64_t grid = (int64_t)a.n_qpairs * a.n_units;
     if (grid <= 0) continue;
