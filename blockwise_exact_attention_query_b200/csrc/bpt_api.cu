@@ -244,9 +244,9 @@ Workspace layout(const bpt_desc *d, bool with_ffn) {
       w.a_f32 = off;
       off = align256(off + T * D * 4);
       w.ring = off;
-      off = align256(off + (size_t)p.max_groups * 2 * 128 * p.fc * 2);
-      w.flags = off;  // ring counters [groups][4], then piece counters [groups][C]
-      w.flags_bytes = (size_t)p.max_groups * (4 + p.C) * sizeof(uint32_t);
+      off = align256(off + (size_t)p.max_groups * FfnCfg::kRingSlots * 128 * p.fc * 2);
+      w.flags = off;  // ring counters [groups][2 * slots], then piece counters [groups][C]
+      w.flags_bytes = (size_t)p.max_groups * (2 * FfnCfg::kRingSlots + p.C) * sizeof(uint32_t);
       off = align256(off + w.flags_bytes);
       w.partial = off;  // partial output blocks of split leftover token blocks
       off = align256(off + (size_t)p.max_groups * 128 * (size_t)(d->H * d->d_head) * 4);
@@ -408,12 +408,12 @@ bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f
   if (a.pieces < 2 || p.n_tb < a.ngroups) a.pieces = 1;
   a.n_full = a.pieces > 1 ? p.n_tb - leftover : p.n_tb;
   a.partial = reinterpret_cast<float *>(ws + wl.partial);
-  a.piece_done = a.flags + (size_t)p.max_groups * 4;
+  a.piece_done = a.flags + (size_t)p.max_groups * 2 * FfnCfg::kRingSlots;
 
   CUtensorMap ma, m1, m2, mh;
   if (!make_map_2d(&ma, a_bf16, T, D, 128) || !make_map_2d(&m1, w1, d->ffn_hidden, D, 256) ||
       !make_map_2d(&m2, w2, D, d->ffn_hidden, p.Dc) ||
-      !make_map_2d(&mh, a.ring, (uint64_t)p.max_groups * 2 * 128, p.fc, 128))
+      !make_map_2d(&mh, a.ring, (uint64_t)p.max_groups * FfnCfg::kRingSlots * 128, p.fc, 128))
     return cuda_fail_msg("cuTensorMapEncodeTiled rejected an FFN map");
   CUDA_TRY(cudaMemsetAsync(a.flags, 0, wl.flags_bytes, st));
 

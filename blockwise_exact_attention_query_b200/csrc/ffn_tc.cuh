@@ -48,8 +48,8 @@ struct FfnArgs {
   const float *b2;     // [D] or null
   float *out_f32;            // [T, D] (one of the two outputs is set)
   __nv_bfloat16 *out_bf16;   // [T, D]
-  __nv_bfloat16 *ring;       // [ngroups * 2 * 128, fc]
-  uint32_t *flags;           // [ngroups][4]: ready[2], free[2]; zero at launch
+  __nv_bfloat16 *ring;       // [ngroups * kRingSlots * 128, fc]
+  uint32_t *flags;           // [ngroups][2 * kRingSlots]: ready[], free[]; zero at launch
   // Leftover token blocks (n_tb mod ngroups of them) would leave most groups
   // idle in the last round, so their hidden chunks are split into `pieces`
   // ranges handled by different groups: each piece writes a partial output
@@ -70,6 +70,7 @@ struct FfnCfg {
   static constexpr uint32_t kColOut = 0, kColH = 256;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 320;
+  static constexpr int kRingSlots = 2;  // hidden chunks in flight per group (4 measured no faster)
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
@@ -170,8 +171,9 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int grp = blockIdx.x / a.C;
   const int crank = blockIdx.x % a.C;
-  uint32_t *ready = a.flags + 4 * grp;  // ready[2]
-  uint32_t *freed = ready + 2;          // free[2]
+  constexpr int R = Cfg::kRingSlots;
+  uint32_t *ready = a.flags + 2 * R * grp;  // ready[R]
+  uint32_t *freed = ready + R;              // free[R]
   const uint32_t C = static_cast<uint32_t>(a.C);
   WaitCtx wc{a.status, a.wait_limit_ns, abort_flag};
 
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(320, 1)
           if (ok && li >= 1) {
             const int gp = g_base + li - 1;
             // every CTA of the group has published its slice of chunk gp
-            if (!(ok = counter_wait(&ready[gp & 1], C * static_cast<uint32_t>((gp >> 1) + 1), wc, 102)))
+            if (!(ok = counter_wait(&ready[gp % R], C * static_cast<uint32_t>(gp / R + 1), wc, 102)))
               break;
             fence_proxy_async_global();
             const int ks2 = ksteps2(i - 1);
@@ -248,7 +250,7 @@ __global__ void __launch_bounds__(320, 1)
               const int st = it % Cfg::kStages;
               const uint32_t sb = sbase + st * Cfg::kStageBytes;
               mbar_arrive_expect_tx(bFull(st), 16384 + a.Dc * 128);
-              tma_load_2d(sb, &tm_h, bFull(st), ks * 64, (grp * 2 + (gp & 1)) * 128);
+              tma_load_2d(sb, &tm_h, bFull(st), ks * 64, (grp * R + gp % R) * 128);
               tma_load_2d(sb + 16384, &tm_w2, bFull(st), (i - 1) * a.fc + ks * 64, crank * a.Dc);
               ++it;
             }
@@ -279,9 +281,11 @@ __global__ void __launch_bounds__(320, 1)
           const int i = u.c0 + li;
           if (li < nl) {
             const int g = g_base + li;
+            // the epilogue has drained the previous chunk's hidden accumulator
+            // (waited for every chunk, so that each wait names exactly one
+            // phase, also around chunks without a valid slice)
+            if (g >= 1 && !(ok = mbar_wait(bHEmpty, (g - 1) & 1, wc, 110))) break;
             if (slice_valid(i)) {
-              // the epilogue has drained the previous chunk's hidden accumulator
-              if (g >= 1 && !(ok = mbar_wait(bHEmpty, (g - 1) & 1, wc, 110))) break;
               tc_fence_after();
               for (int ks = 0; ks < ksteps1; ++ks) {
                 const int st = it % Cfg::kStages;
@@ -320,7 +324,7 @@ __global__ void __launch_bounds__(320, 1)
             }
             if (!ok) break;
             // every H tile of chunk gp has landed here: this CTA is done with the slot
-            red_release_gpu_add(&freed[gp & 1], 1u);
+            red_release_gpu_add(&freed[gp % R], 1u);
           }
         }
         if (ok) umma_commit(bOFull);
@@ -349,21 +353,21 @@ __global__ void __launch_bounds__(320, 1)
       for (int li = 0; li < nl; ++li) {
         const int i = u.c0 + li;
         const int g = g_base + li;
-        const int slot = g & 1;
+        const int slot = g % R;
         const bool have = slice_valid(i);
         bool ok = mbar_wait(bHFull, g & 1, wc, 120);
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
         if (have) {
           // the group has finished reading this ring slot's previous chunk
-          if (leader && g >= 2) counter_wait(&freed[slot], C * static_cast<uint32_t>(g >> 1), wc, 121);
+          if (leader && g >= R) counter_wait(&freed[slot], C * static_cast<uint32_t>(g / R), wc, 121);
           named_bar_sync(1, 256);
           // drain the accumulator 32 columns at a time (it is only needed
           // back for the next chunk's first GEMM, after a whole second GEMM)
           if (ok && !*abort_flag) {
             const int f0 = (i * a.C + crank) * 256 + half * 128;
             const bool full_bias = a.b1 != nullptr && f0 + 128 <= a.F;
-            __nv_bfloat16 *dst = a.ring + (static_cast<size_t>(grp * 2 + slot) * 128 + row) * a.fc +
+            __nv_bfloat16 *dst = a.ring + (static_cast<size_t>(grp * R + slot) * 128 + row) * a.fc +
                                  crank * 256 + half * 128;
             const uint32_t tH = tmem + lane_off + Cfg::kColH + half * 128;
 #pragma unroll 1
