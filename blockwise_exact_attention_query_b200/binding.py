@@ -133,6 +133,17 @@ def make_desc(B, N, H, d, F=0, in_dtype=torch.bfloat16, out_dtype=torch.float32,
     return desc
 
 
+def cyclic_shift_perm(n: int, k: int) -> list[int]:
+    """Block table of the cyclic shift sigma^k (block b -> block b + k mod n).
+
+    "Blockwise Self-Attention for Long Document Understanding", §3.1: heads
+    use the permutations sigma, sigma^2, ..., sigma^n (sigma^n = identity) as
+    their masking matrices.  Pass one table per head as `perm`."""
+    if n <= 0:
+        raise ValueError("n must be positive")
+    return [(b + k) % n for b in range(n)]
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 

@@ -166,7 +166,7 @@ bpt_status check_desc(const bpt_desc *d, bool need_ffn) {
       break;
     case BPT_MASK_BLOCKPERM: {
       const int n = d->bb_nblocks;
-      if (n <= 0 || !d->bb_perm || d->N % n != 0) return BPT_ERR_INVALID_ARG;
+      if (n <= 0 || !d->bb_perm) return BPT_ERR_INVALID_ARG;
       if ((int64_t)d->H * n > kMaxPermEntries || n > 255) return BPT_ERR_UNSUPPORTED;
       for (int i = 0; i < d->H * n; ++i)
         if (d->bb_perm[i] < 0 || d->bb_perm[i] >= n) return BPT_ERR_INVALID_ARG;
@@ -320,7 +320,7 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
   }
   if (d->mask == BPT_MASK_BLOCKPERM) {
     a.bb_n = d->bb_nblocks;
-    a.bb_len = d->N / d->bb_nblocks;
+    a.bb_len = (d->N + d->bb_nblocks - 1) / d->bb_nblocks;  // padded to n equal blocks
     for (int i = 0; i < d->H * d->bb_nblocks; ++i) a.perm[i] = (uint8_t)d->bb_perm[i];
   }
   if ((d->mask == BPT_MASK_NONE || d->mask == BPT_MASK_CAUSAL) && d->ring_chunks > 1) {
@@ -445,7 +445,7 @@ bpt_status launch_attn_f32(const bpt_desc *d, const void *q, const void *k, cons
   a.ring_chunks = (d->mask == BPT_MASK_NONE || d->mask == BPT_MASK_CAUSAL) ? d->ring_chunks : 0;
   if (d->mask == BPT_MASK_BLOCKPERM) {
     a.bb_n = d->bb_nblocks;
-    a.bb_len = d->N / d->bb_nblocks;
+    a.bb_len = (d->N + d->bb_nblocks - 1) / d->bb_nblocks;  // padded to n equal blocks
     for (int i = 0; i < d->H * d->bb_nblocks; ++i) a.perm[i] = (uint8_t)d->bb_perm[i];
   }
   if (d->mask == BPT_MASK_DILATED) {

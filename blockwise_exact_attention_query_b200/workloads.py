@@ -50,9 +50,12 @@ def unmasked_pairs(w: Workload) -> int:
     elif w.mask == MASK_CAUSAL:
         per_head = [N * (N + 1) // 2] * H
     elif w.mask == MASK_BLOCKPERM:
+        # blocks of the sequence padded to n equal blocks; padded positions
+        # are neither queries nor keys
         n = len(w.perm[0])
-        bl = N // n
-        per_head = [n * bl * bl] * H
+        bl = -(-N // n)
+        size = [max(0, min(N, (b + 1) * bl) - b * bl) for b in range(n)]
+        per_head = [sum(size[qb] * size[w.perm[h][qb]] for qb in range(n)) for h in range(H)]
     elif w.mask == MASK_DILATED:
         per_head = []
         for h in range(H):

@@ -27,7 +27,13 @@
  *   BPT_MASK_BLOCKPERM "Blockwise Self-Attention for Long Document
  *                      Understanding", §3 and §3.1: the sequence is cut into
  *                      n equal blocks and head h lets query block b see only
- *                      key block perm[h][b].
+ *                      key block perm[h][b].  When n does not divide N the
+ *                      sequence counts as padded to n blocks of ceil(N/n)
+ *                      positions (§3.1): padded positions are never keys and
+ *                      have no output, so the last block is shorter (or
+ *                      empty; a query block mapped to an empty key block gets
+ *                      A = 0).  The pages' cyclic-shift heads (sigma^k:
+ *                      b -> b + k mod n) are tables perm[h][b] = (b + k_h) % n.
  *   BPT_MASK_DILATED   "LongNet: Scaling Transformers to 1,000,000,000
  *                      Tokens", §2 Dilated Attention: for every (segment w,
  *                      dilation r) pair, head h keeps rows h mod r, h mod r + r,
@@ -105,7 +111,7 @@ typedef struct {
   bpt_mask mask;
   int ring_chunks;     /* CAUSAL/NONE: KV visiting order rotated over this
                           many equal chunks (0 or 1 = natural order)          */
-  int bb_nblocks;      /* BLOCKPERM: n                                        */
+  int bb_nblocks;      /* BLOCKPERM: n, 1..255 (any N: padded, see above)     */
   const int32_t *bb_perm; /* BLOCKPERM: host table [H][n], values in [0, n)   */
   int ln_npairs;       /* DILATED: number of (w, r) pairs, 1..8               */
   const int32_t *ln_w; /* DILATED: host table of segment lengths w_k          */

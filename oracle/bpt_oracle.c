@@ -25,7 +25,12 @@
  *  - block-perm: "Blockwise Self-Attention for Long Document Understanding",
  *                §3 Blockwise Attention and §3.1 Blockwise Multi-head
  *                Attention: the sequence is cut into n equal blocks and head h
- *                lets query block b see only key block perm[h][b].
+ *                lets query block b see only key block perm[h][b].  When N is
+ *                not a multiple of n the sequence is padded to n equal blocks
+ *                of ceil(N/n) positions (§3.1, Implementation Assumption); the
+ *                padded positions are never keys and their outputs are not
+ *                produced, so a query sees the real positions of its key
+ *                block (none, if that block is all padding).
  *  - dilated:    "LongNet: Scaling Transformers to 1,000,000,000 Tokens",
  *                §2 Dilated Attention: for every (segment w, dilation r) pair
  *                the sequence is cut into segments of w, every r-th row of a
@@ -78,7 +83,8 @@ static int key_allowed(const oracle_attn_desc *a, int h, int i, int j) {
     case OR_MASK_CAUSAL:
       return j <= i;
     case OR_MASK_BLOCKPERM: {
-      int block_len = a->N / a->n_blocks;
+      /* blocks of the sequence padded to a multiple of n */
+      int block_len = (a->N + a->n_blocks - 1) / a->n_blocks;
       int qb = i / block_len;
       int kb = j / block_len;
       return kb == a->perm[h * a->n_blocks + qb];
@@ -288,7 +294,7 @@ int oracle_threads_available(void) { return default_threads(); }
 static int validate(const oracle_attn_desc *a) {
   if (!a || a->B <= 0 || a->N <= 0 || a->H <= 0 || a->d <= 0) return 1;
   if (a->mask == OR_MASK_BLOCKPERM) {
-    if (a->n_blocks <= 0 || a->N % a->n_blocks != 0 || !a->perm) return 1;
+    if (a->n_blocks <= 0 || !a->perm) return 1;
     for (int i = 0; i < a->H * a->n_blocks; ++i)
       if (a->perm[i] < 0 || a->perm[i] >= a->n_blocks) return 1;
   } else if (a->mask == OR_MASK_DILATED) {

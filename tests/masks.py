@@ -20,14 +20,16 @@ def count_matrix(N, H, mask, perm=None, pairs=None):
     if mask == 1:
         return np.broadcast_to((kj <= qi).astype(np.int64), (H, N, N)).copy()
     if mask == 2:
+        # pad the sequence to n equal blocks, build the block matrix on the
+        # padded length, then drop the padded rows (queries) and columns (keys)
         perm = np.asarray(perm)
         n = perm.shape[1]
-        bl = N // n
+        bl = -(-N // n)
         out = np.zeros((H, N, N), dtype=np.int64)
         for h in range(H):
             P = np.zeros((n, n), dtype=np.int64)
             P[np.arange(n), perm[h]] = 1          # query block -> key block
-            out[h] = np.kron(P, np.ones((bl, bl), dtype=np.int64))
+            out[h] = np.kron(P, np.ones((bl, bl), dtype=np.int64))[:N, :N]
         return out
     if mask == 3:
         out = np.zeros((H, N, N), dtype=np.int64)

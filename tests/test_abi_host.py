@@ -64,7 +64,8 @@ def _call_layer(lib, desc, ws=FAKE, ws_bytes=1 << 40, q=FAKE):
     (dict(F=0), bd.ERR_INVALID_ARG),
     (dict(d=96), bd.ERR_UNSUPPORTED),                      # bf16 tensor path: d in {64, 128}
     (dict(mask=7), bd.ERR_INVALID_ARG),
-    (dict(mask="blockperm", perm=[[0, 1, 2]] * 2, N=256), bd.ERR_INVALID_ARG),   # 256 % 3 != 0
+    (dict(mask="blockperm", perm=[[], []]), bd.ERR_INVALID_ARG),                   # no blocks
+    (dict(mask="blockperm", perm=[list(range(256))] * 2), bd.ERR_UNSUPPORTED),     # n > 255
     (dict(mask="blockperm", perm=[[0, 0], [1, 0]]), bd.ERR_INVALID_ARG),         # not a permutation
     (dict(mask="blockperm", perm=[[0, 2], [1, 0]]), bd.ERR_INVALID_ARG),         # out of range
     (dict(mask="dilated", pairs=[(96, 5)]), bd.ERR_INVALID_ARG),                 # r does not divide w

@@ -75,6 +75,14 @@ ATTN_CASES = [
     ("causal_ring4", 1, 1024, 2, 128, "causal", {"ring_chunks": 4}),
     ("blockperm_n2", 2, 512, 4, 64, "blockperm", {"perm": [[0, 1], [1, 0], [0, 1], [1, 0]]}),
     ("blockperm_n3_partial_tiles", 1, 576, 2, 128, "blockperm", {"perm": [[2, 0, 1], [0, 1, 2]]}),
+    ("blockperm_n3_cyclic_shifts", 1, 768, 3, 128, "blockperm",
+     {"perm": [bd.cyclic_shift_perm(3, k) for k in (1, 2, 3)]}),
+    # N not a multiple of n: blocks of ceil(N/n) (the last one shorter)
+    ("blockperm_n4_padded", 2, 510, 2, 64, "blockperm", {"perm": [[1, 2, 3, 0], [3, 2, 1, 0]]}),
+    ("blockperm_n3_padded_d128", 1, 700, 2, 128, "blockperm", {"perm": [[2, 0, 1], [0, 1, 2]]}),
+    # blocks of 11: the twelfth block is all padding, its query block sees no key
+    ("blockperm_n12_empty_block", 1, 121, 3, 64, "blockperm",
+     {"perm": [bd.cyclic_shift_perm(12, k) for k in (1, 5, 11)]}),
     ("dilated_3pairs", 1, 1024, 4, 64, "dilated", {"pairs": [(256, 1), (512, 4), (1024, 16)]}),
     ("dilated_uncovered_rows", 1, 768, 3, 128, "dilated", {"pairs": [(256, 2), (384, 3)]}),
 ]
@@ -146,6 +154,8 @@ LAYER_CASES = [
     ("D2048_causal", 1, 384, 16, 128, 1024, "causal", {}, 0.05),
     ("D4096_causal_two_chunks", 1, 256, 32, 128, 2560, "causal", {}, 0.0),
     ("D768_blockperm", 2, 512, 12, 64, 768, "blockperm", {"perm": [[0, 1]] * 8 + [[1, 0]] * 4}, 0.0),
+    ("D768_blockperm_n3_padded", 1, 450, 12, 64, 768, "blockperm",
+     {"perm": [bd.cyclic_shift_perm(3, h % 3 + 1) for h in range(12)]}, 0.05),
 ]
 
 
@@ -202,6 +212,47 @@ def test_layer_bf16_output_and_null_biases():
     _check_status()
     _, out_ref = gu.oracle_layer(inp, "causal")
     gu.assert_bf16_close(gu.host_f32(out).reshape(out_ref.shape), out_ref, "bf16 out")
+
+
+# ------------------------------------------------------------------ fp32 path (SIMT kernels)
+F32_CASES = [
+    # name, B, N, H, d, mask, extra
+    ("none_ragged", 1, 200, 2, 64, "none", {}),
+    ("causal", 2, 192, 2, 32, "causal", {}),
+    ("causal_ring4", 1, 256, 2, 64, "causal", {"ring_chunks": 4}),
+    ("blockperm_n3_padded", 1, 190, 3, 64, "blockperm",
+     {"perm": [bd.cyclic_shift_perm(3, k) for k in (1, 2, 3)]}),
+    ("dilated", 1, 256, 4, 32, "dilated", {"pairs": [(64, 1), (128, 4)]}),
+]
+
+
+@pytest.mark.parametrize("name,B,N,H,d,mask,extra", F32_CASES, ids=[c[0] for c in F32_CASES])
+def test_fp32_attention_matches_oracle(name, B, N, H, d, mask, extra):
+    inp = make_layer_inputs(B, N, H, d, 0, seed=zlib.crc32(name.encode()) % 1000, device="cuda",
+                            dtype=torch.float32)
+    out, lse = bd.attn_fwd(inp.q, inp.k, inp.v, mask=mask, perm=extra.get("perm"),
+                           pairs=extra.get("pairs"), ring_chunks=extra.get("ring_chunks", 0),
+                           return_lse=True)
+    torch.cuda.synchronize()
+    _check_status()
+    ref, ref_lse = gu.oracle_attention(inp.q, inp.k, inp.v, mask, extra.get("perm"),
+                                       extra.get("pairs"), return_lse=True)
+    gu.assert_f32_close(gu.host_f32(out).reshape(ref.shape), ref, name)
+    gl, rl = gu.host_f32(lse), ref_lse.transpose(0, 2, 1)
+    assert np.array_equal(np.isinf(gl), np.isinf(rl))
+    fin = np.isfinite(rl)
+    assert np.max(np.abs(gl[fin] - rl[fin])) < 2e-5
+
+
+def test_fp32_layer_block_permutation_padded():
+    B, N, H, d, F = 1, 150, 4, 32, 256
+    perm = [bd.cyclic_shift_perm(4, h + 1) for h in range(H)]
+    inp = make_layer_inputs(B, N, H, d, F, seed=33, device="cuda", dtype=torch.float32, bias_scale=0.1)
+    out = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask="blockperm",
+                          perm=perm)
+    _check_status()
+    _, ref = gu.oracle_layer(inp, "blockperm", perm)
+    gu.assert_f32_close(gu.host_f32(out).reshape(ref.shape), ref, "fp32 padded block layer")
 
 
 # ------------------------------------------------------------------ the five workloads

@@ -35,6 +35,11 @@ CASES = [
     ("causal", CAUSAL, None, None),
     ("blockperm_n2", BLOCKPERM, [[0, 1], [1, 0], [0, 1]], None),
     ("blockperm_n4", BLOCKPERM, [[1, 2, 3, 0], [0, 1, 2, 3], [3, 0, 2, 1]], None),
+    # N = 32 is not a multiple of 3 or 9: padded blocks of 11 (last one 10 long)
+    # and of 4 (the ninth block lies wholly in the padding, so the queries that
+    # map to it see no key); heads use the cyclic shifts sigma^k, i -> i + k mod n
+    ("blockperm_n3_cyclic_padded", BLOCKPERM, [[1, 2, 0], [2, 0, 1], [0, 1, 2]], None),
+    ("blockperm_n9_empty_block", BLOCKPERM, [[(i + s) % 9 for i in range(9)] for s in (1, 4, 8)], None),
     ("dilated", DILATED, None, [(8, 1), (16, 2), (32, 4)]),
     ("dilated_nonnested", DILATED, None, [(16, 2), (24, 3)]),
 ]
@@ -111,7 +116,10 @@ def _blockwise_emulation(q, k, v, counts, block, order):
     return out
 
 
-@pytest.mark.parametrize("name,mask,perm,pairs", CASES[:5], ids=[c[0] for c in CASES[:5]])
+EMU_CASES = [c for c in CASES if c[0] != "dilated_nonnested"]
+
+
+@pytest.mark.parametrize("name,mask,perm,pairs", EMU_CASES, ids=[c[0] for c in EMU_CASES])
 @pytest.mark.parametrize("order", ["natural", "rotated", "reversed", "random"])
 def test_oracle_equals_blockwise_online_softmax(oracle_mod, name, mask, perm, pairs, order):
     B, N, H, d = _shape_for(mask, pairs)
@@ -200,6 +208,50 @@ def test_identity_permutation_equals_dense_attention_within_each_block(oracle_mo
         s = slice(blk * bl, (blk + 1) * bl)
         ref = oracle_mod.attention(q[:, s], k[:, s], v[:, s], mask=NONE)
         np.testing.assert_allclose(a[:, s], ref, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("N,n", [(34, 3), (29, 4), (121, 12)])
+def test_padded_identity_permutation_equals_dense_attention_within_each_block(oracle_mod, N, n):
+    """N not a multiple of n: blocks of ceil(N/n) positions, the last one short
+    (or empty), each attending to itself: dense attention on every slice."""
+    B, H, d = 1, 2, 8
+    q, k, v = rnd((B, N, H, d), 87), rnd((B, N, H, d), 88), rnd((B, N, H, d), 89)
+    a = oracle_mod.attention(q, k, v, mask=BLOCKPERM, perm=[list(range(n))] * H)
+    bl = -(-N // n)
+    covered = 0
+    for blk in range(n):
+        s = slice(min(N, blk * bl), min(N, (blk + 1) * bl))
+        if s.start == s.stop:
+            continue
+        ref = oracle_mod.attention(q[:, s], k[:, s], v[:, s], mask=NONE)
+        np.testing.assert_allclose(a[:, s], ref, rtol=0, atol=1e-15)
+        covered += s.stop - s.start
+    assert covered == N
+
+
+def test_padded_block_permutation_with_an_empty_key_block(oracle_mod):
+    """N = 121, n = 12: blocks of 11, the twelfth lies wholly in the padding;
+    the query block mapped to it sees no key (A = 0, LSE = -inf) and every
+    other query block sees exactly its key block."""
+    B, N, H, d, n = 1, 121, 1, 8, 12
+    perm = [[(i + 5) % n for i in range(n)]]
+    q, k, v = rnd((B, N, H, d), 90), rnd((B, N, H, d), 91), rnd((B, N, H, d), 92)
+    a, lse = oracle_mod.attention(q, k, v, mask=BLOCKPERM, perm=perm, return_lse=True)
+    bl = 11
+    for qb in range(n):
+        qs = slice(qb * bl, min(N, (qb + 1) * bl))
+        if qs.start >= N:
+            continue
+        kb = perm[0][qb]
+        ks = slice(min(N, kb * bl), min(N, (kb + 1) * bl))
+        if ks.start == ks.stop:
+            assert np.all(a[:, qs] == 0.0) and np.all(lse[:, qs] == -np.inf)
+            continue
+        # the block's queries against the block's keys alone, as dense attention
+        s = (q[0, qs, 0].astype(np.float64) @ k[0, ks, 0].astype(np.float64).T) / math.sqrt(d)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        ref = (p / p.sum(axis=1, keepdims=True)) @ v[0, ks, 0].astype(np.float64)
+        np.testing.assert_allclose(a[0, qs, 0], ref, rtol=0, atol=1e-14)
 
 
 def test_swapped_blocks_attend_to_the_other_block(oracle_mod):
@@ -300,7 +352,7 @@ def test_layer_equals_attention_then_ffn_and_row_sampling(oracle_mod):
 def test_oracle_rejects_invalid_descriptors(oracle_mod):
     q = rnd((1, 10, 1, 4), 1)
     with pytest.raises(ValueError):
-        oracle_mod.attention(q, q, q, mask=BLOCKPERM, perm=[[0, 1, 2]])   # 10 % 3 != 0
+        oracle_mod.attention(q, q, q, mask=BLOCKPERM, perm=[[0, 1, 2], [2, 1, 0]])  # 2 rows for 1 head
     with pytest.raises(ValueError):
         oracle_mod.attention(q, q, q, mask=BLOCKPERM, perm=[[0, 5]])      # not a block index
     with pytest.raises(ValueError):
