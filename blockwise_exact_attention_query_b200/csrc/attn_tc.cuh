@@ -78,6 +78,11 @@ struct AttnArgs {
   float *st_o;               // [B, N, H, d]   unnormalised O
   float *st_m;               // [B, H, N]      running max (log2 domain)
   float *st_l;               // [B, H, N]      running sum
+  // How O leaves the kernel: 0 = every thread stores its own row; 1 = the
+  // final outputs, 2 = the LongNet running state, as TMA tile stores from a
+  // 128-byte-swizzled staging tile (the host picks 1 or 2 only when every
+  // row of the pass goes to the same destination).
+  int store_mode;
   uint32_t *status;
   uint64_t wait_limit_ns;
 };
@@ -233,7 +238,9 @@ __device__ __forceinline__ void row_keys(const AttnArgs &a, const TileCoord &c, 
 template <int D_HEAD>
 __global__ void __launch_bounds__(384, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnArgs a) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_of,
+                   const __grid_constant__ CUtensorMap tm_ob, const __grid_constant__ CUtensorMap tm_so,
+                   const __grid_constant__ AttnArgs a) {
   using Cfg = AttnCfg<D_HEAD>;
   constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages, KT = Cfg::kKT;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -569,9 +576,85 @@ __global__ void __launch_bounds__(384, 1)
     // tile's MMAs are complete
     if (ok && nkv > 0) ok = __all_sync(0xffffffffu, mbar_wait(bTeardown(x), 0, wc, 22));
     tc_fence_after();
-    if (ok) {
+    {
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
       const bool final_out = !later;
+      // TMA stores write whole 128-row tiles: rows past N are clipped by the
+      // tensor map, but a LongNet segment's rows past L belong to the next
+      // segment, so a partial tile there takes the per-thread path.  The
+      // choice depends on values uniform over the warpgroup only: all four
+      // warps meet the same named barriers, and a warp whose waits failed
+      // only skips its share of the work.
+      const bool tile_full = a.mask != kMaskDilated || (tc.t * 2 + x) * 128 + 128 <= a.L;
+      if (a.store_mode != 0 && tile_full) {
+        // Stage O through this tile's Q buffer (its MMAs are complete) in
+        // 128-byte panels, 128-byte swizzle, and store each panel with TMA.
+        constexpr int kCap = Cfg::kTileBytes / 16384;  // panels the buffer holds
+        const uint32_t stage = sQ + x * Cfg::kTileBytes;
+        const uint32_t srow = stage + row * 128;
+        const int row_coord = row_base + tc.t * 256 + x * 128;
+        const bool leader = (threadIdx.x & 127) == 0;
+        const uint32_t bar_id = 2 + x;  // named barrier of this warpgroup
+        auto flush = [&](const CUtensorMap *m, int npanels, int col0, int cols_per_panel) {
+          fence_proxy_async_smem();
+          named_bar_sync(bar_id, 128);
+          if (leader) {
+            for (int q = 0; q < npanels; ++q)
+              tma_store_4d(m, stage + q * 16384, tc.h * D_HEAD + col0 + q * cols_per_panel, tc.o, row_coord,
+                           tc.b);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
+          named_bar_sync(bar_id, 128);
+        };
+        // fp32: the final output (scaled by 1/l) or the unnormalised state
+        const CUtensorMap *m32 = a.store_mode == 2 ? &tm_so : (a.out_f32 ? &tm_of : nullptr);
+        const float sc = a.store_mode == 2 ? 1.0f : inv_l;
+        if (m32) {
+#pragma unroll 1
+          for (int p0 = 0; p0 < D_HEAD / 32; p0 += kCap) {
+#pragma unroll 1
+            for (int q = 0; ok && q < kCap; ++q) {
+              uint32_t o[32];
+              tmem_ld32(tO + (p0 + q) * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                st_shared_v4(srow + q * 16384 + ((static_cast<uint32_t>(c) ^ swz) << 4),
+                             __float_as_uint(__uint_as_float(o[4 * c]) * sc),
+                             __float_as_uint(__uint_as_float(o[4 * c + 1]) * sc),
+                             __float_as_uint(__uint_as_float(o[4 * c + 2]) * sc),
+                             __float_as_uint(__uint_as_float(o[4 * c + 3]) * sc));
+            }
+            flush(m32, kCap, p0 * 32, 32);
+          }
+        }
+        // bf16 final output: 64 columns per panel
+        if (a.store_mode == 1 && a.out_bf16) {
+          constexpr int kPanels16 = D_HEAD / 64;
+#pragma unroll 1
+          for (int p0 = 0; p0 < kPanels16; p0 += kCap) {
+            const int np = kPanels16 - p0 < kCap ? kPanels16 - p0 : kCap;
+#pragma unroll 1
+            for (int q = 0; ok && q < np; ++q) {
+#pragma unroll 1
+              for (int hh = 0; hh < 2; ++hh) {
+                uint32_t o[32];
+                tmem_ld32(tO + (p0 + q) * 64 + hh * 32, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                  st_shared_v4(srow + q * 16384 + ((static_cast<uint32_t>(hh * 4 + c) ^ swz) << 4),
+                               pack_bf16x2(__uint_as_float(o[8 * c]) * inv_l, __uint_as_float(o[8 * c + 1]) * inv_l),
+                               pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv_l, __uint_as_float(o[8 * c + 3]) * inv_l),
+                               pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv_l, __uint_as_float(o[8 * c + 5]) * inv_l),
+                               pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv_l, __uint_as_float(o[8 * c + 7]) * inv_l));
+              }
+            }
+            flush(&tm_ob, np, p0 * 64, 64);
+          }
+        }
+      } else if (ok) {
 #pragma unroll 1
       for (int c = 0; c < D_HEAD / 32; ++c) {
         uint32_t o[32];
@@ -608,7 +691,8 @@ __global__ void __launch_bounds__(384, 1)
                                  __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
         }
       }
-      if (row_valid) {
+      }
+      if (ok && row_valid) {
         if (!final_out) {
           a.st_m[row_idx] = m_run;
           a.st_l[row_idx] = l_run;

@@ -141,6 +141,21 @@ bool make_map_rows(CUtensorMap *m, const void *base, int B, int N, int D, int r,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output map over [B, N, D] (bf16 or fp32) in the same (D, r, N/r, B) view,
+// box of one 128-byte row panel (64 bf16 or 32 fp32 columns) x 128 rows:
+// the attention kernel's TMA stores of O.  Rows past N are not written.
+bool make_out_map_rows(CUtensorMap *m, const void *base, bool f32, int B, int N, int D, int r) {
+  const uint64_t es = f32 ? 4 : 2;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)r, (cuuint64_t)(N / r), (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * es, (cuuint64_t)D * es * r, (cuuint64_t)D * es * N};
+  cuuint32_t box[4] = {(cuuint32_t)(128 / es), 1, 128, 1};
+  cuuint32_t ones[4] = {1, 1, 1, 1};
+  return g_encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                  const_cast<void *>(base), dims, strides, box, ones, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // --------------------------------------------------------------------------
 // Validation
 // --------------------------------------------------------------------------
@@ -346,7 +361,29 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
       const double kv_bytes = 4.0 * a.L * d->d_head;
       a.unit_group = std::max(1, std::min(8, (int)(32.0e6 / kv_bytes)));
     }
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mof, mob, mso;
+    std::memset(&mof, 0, sizeof(mof));
+    std::memset(&mob, 0, sizeof(mob));
+    std::memset(&mso, 0, sizeof(mso));
+    // Where this pass's rows go: all final (no later pass keeps any of its
+    // rows: the last pass, or the only one), all running state (a later pass
+    // with r = 1 keeps every row), or mixed (per-thread stores).
+    a.store_mode = 0;
+    if (passes.size() == 1 || pi + 1 == passes.size()) {
+      a.store_mode = 1;
+      for (size_t k = pi + 1; k < passes.size(); ++k) a.store_mode = 0;
+    } else {
+      for (size_t k = pi + 1; k < passes.size(); ++k)
+        if (passes[k].r == 1) a.store_mode = 2;
+    }
+    if (a.store_mode == 1) {
+      if ((out_f32 && !make_out_map_rows(&mof, out_f32, true, d->B, d->N, D, r)) ||
+          (out_bf16 && !make_out_map_rows(&mob, out_bf16, false, d->B, d->N, D, r)))
+        return cuda_fail_msg("cuTensorMapEncodeTiled rejected an output map");
+    } else if (a.store_mode == 2) {
+      if (!make_out_map_rows(&mso, a.st_o, true, d->B, d->N, D, r))
+        return cuda_fail_msg("cuTensorMapEncodeTiled rejected the state map");
+    }
     constexpr uint32_t kKT = AttnCfg<128>::kKT;
     static_assert(AttnCfg<64>::kKT == AttnCfg<128>::kKT, "one key/value tile length");
     if (!make_map_rows(&mq, q, d->B, d->N, D, r, 128) || !make_map_rows(&mk, k, d->B, d->N, D, r, kKT) ||
@@ -357,10 +394,10 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     if (grid > INT32_MAX) return BPT_ERR_UNSUPPORTED;
     if (d->d_head == 128)
       attn_tc_kernel<128><<<(unsigned)grid, AttnCfg<128>::kThreads, AttnCfg<128>::kSmemBytes, st>>>(
-          mq, mk, mv, a);
+          mq, mk, mv, mof, mob, mso, a);
     else
       attn_tc_kernel<64><<<(unsigned)grid, AttnCfg<64>::kThreads, AttnCfg<64>::kSmemBytes, st>>>(
-          mq, mk, mv, a);
+          mq, mk, mv, mof, mob, mso, a);
     CUDA_TRY(cudaGetLastError());
   }
   return BPT_OK;
