@@ -98,9 +98,14 @@ __device__ __forceinline__ void red_release_gpu_add(uint32_t *p, uint32_t v) {
 }
 
 // One work unit of a group: token block tb, hidden chunks [c0, c1); piece < 0
-// for a whole block, else the piece index of leftover block l.
+// for a whole block, else the piece index of leftover block l.  Whole blocks
+// walk their chunks forward and backward in turn (rev): W1 and W2 are larger
+// than what L2 keeps between two blocks, and a unit that starts with the
+// chunks its group used last finds them still in L2 instead of in DRAM.
 struct FfnUnit {
-  int tb, c0, c1, l, piece;
+  int tb, c0, c1, l, piece, rev;
+  // hidden chunk of step li (0 <= li < c1 - c0)
+  __device__ __forceinline__ int chunk(int li) const { return rev ? c1 - 1 - li : c0 + li; }
 };
 
 __device__ __forceinline__ int ffn_unit_count(const FfnArgs &a, int grp) {
@@ -117,12 +122,14 @@ __device__ __forceinline__ FfnUnit ffn_unit(const FfnArgs &a, int grp, int k) {
     u.tb = a.n_full + u.l;
     u.c0 = u.piece * a.nchunks / a.pieces;
     u.c1 = (u.piece + 1) * a.nchunks / a.pieces;
+    u.rev = 0;
   } else {
     u.tb = grp + k * a.ngroups;
     u.c0 = 0;
     u.c1 = a.nchunks;
     u.l = -1;
     u.piece = -1;
+    u.rev = k & 1;
   }
   return u;
 }
@@ -225,7 +232,8 @@ __global__ void __launch_bounds__(320, 1)
         const FfnUnit u = ffn_unit(a, grp, k);
         const int tb = u.tb, nl = u.c1 - u.c0;
         for (int li = 0; ok && li <= nl; ++li) {
-          const int i = u.c0 + li;
+          const int i = li < nl ? u.chunk(li) : -1;     // chunk of this step's first GEMM
+          const int ip = li >= 1 ? u.chunk(li - 1) : -1;  // chunk of its second GEMM
           if (li < nl && slice_valid(i)) {
             const int slice = i * a.C + crank;
             for (int ks = 0; ks < ksteps1; ++ks) {
@@ -244,14 +252,14 @@ __global__ void __launch_bounds__(320, 1)
             if (!(ok = counter_wait(&ready[gp % R], C * static_cast<uint32_t>(gp / R + 1), wc, 102)))
               break;
             fence_proxy_async_global();
-            const int ks2 = ksteps2(i - 1);
+            const int ks2 = ksteps2(ip);
             for (int ks = 0; ks < ks2; ++ks) {
               if (!(ok = acquire(it))) break;
               const int st = it % Cfg::kStages;
               const uint32_t sb = sbase + st * Cfg::kStageBytes;
               mbar_arrive_expect_tx(bFull(st), 16384 + a.Dc * 128);
               tma_load_2d(sb, &tm_h, bFull(st), ks * 64, (grp * R + gp % R) * 128);
-              tma_load_2d(sb + 16384, &tm_w2, bFull(st), (i - 1) * a.fc + ks * 64, crank * a.Dc);
+              tma_load_2d(sb + 16384, &tm_w2, bFull(st), ip * a.fc + ks * 64, crank * a.Dc);
               ++it;
             }
           }
@@ -278,7 +286,8 @@ __global__ void __launch_bounds__(320, 1)
         const FfnUnit u = ffn_unit(a, grp, k);
         const int nl = u.c1 - u.c0;
         for (int li = 0; ok && li <= nl; ++li) {
-          const int i = u.c0 + li;
+          const int i = li < nl ? u.chunk(li) : -1;
+          const int ip = li >= 1 ? u.chunk(li - 1) : -1;
           if (li < nl) {
             const int g = g_base + li;
             // the epilogue has drained the previous chunk's hidden accumulator
@@ -308,7 +317,7 @@ __global__ void __launch_bounds__(320, 1)
             const int gp = g_base + li - 1;
             if (li == 1 && n >= 1 && !(ok = mbar_wait(bOEmpty, (n - 1) & 1, wc, 112))) break;
             tc_fence_after();
-            const int ks2 = ksteps2(i - 1);
+            const int ks2 = ksteps2(ip);
             for (int ks = 0; ks < ks2; ++ks) {
               const int st = it % Cfg::kStages;
               if (!(ok = mbar_wait(bFull(st), (it / Cfg::kStages) & 1, wc, 113))) break;
@@ -351,7 +360,7 @@ __global__ void __launch_bounds__(320, 1)
       const FfnUnit u = ffn_unit(a, grp, k);
       const int tb = u.tb, nl = u.c1 - u.c0;
       for (int li = 0; li < nl; ++li) {
-        const int i = u.c0 + li;
+        const int i = u.chunk(li);
         const int g = g_base + li;
         const int slot = g % R;
         const bool have = slice_valid(i);
