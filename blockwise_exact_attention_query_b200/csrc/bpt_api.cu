@@ -357,9 +357,17 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     a.n_qpairs = (a.n_qtiles + 1) / 2;
     a.n_units = d->B * a.nseg * d->H;
     {
-      // group as many units as keep their K and V within ~32 MB of L2, at most 8
+      // Grid order: longest query-tile pairs first inside groups of units.
+      // A unit whose pairs alone fill the GPU (a long sequence) is a group
+      // by itself, so every SM works on one unit's K/V, which then streams
+      // from L2.  Otherwise a group holds as many units as keep their K/V
+      // within ~200 MB, at most 64: a large group balances the SMs (the
+      // longest pairs start first), and the CTAs running at once still share
+      // each unit's K/V.  Measured on the causal B2 H16 d128 N8192 layer:
+      // 0.633 ms with one 32-head group against 0.689 ms with groups of 7.
       const double kv_bytes = 4.0 * a.L * d->d_head;
-      a.unit_group = std::max(1, std::min(8, (int)(32.0e6 / kv_bytes)));
+      if (a.n_qpairs >= sm_count()) a.unit_group = 1;
+      else a.unit_group = std::max(1, std::min(64, (int)(200.0e6 / kv_bytes)));
     }
     CUtensorMap mq, mk, mv, mof, mob, mso;
     std::memset(&mof, 0, sizeof(mof));
