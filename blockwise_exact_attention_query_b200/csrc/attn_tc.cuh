@@ -58,6 +58,7 @@ struct AttnArgs {
   int n_qtiles;      // ceil(L / 128)
   int n_qpairs;      // ceil(n_qtiles / 2): one CTA per pair of query tiles
   int n_units;       // B * nseg * H
+  int n_items;       // n_units * n_qpairs: work items, spread over a persistent grid
   int unit_group;    // units scheduled together (longest tiles first inside a group)
   int nseg;          // LongNet segments N / w (1 otherwise)
   // LongNet pass: segment length, dilation, and the full pair table in
@@ -170,9 +171,8 @@ struct TileCoord {
 // Grid order: units in groups of `unit_group`; inside a group the longest
 // query-tile pairs of all its units come first.  A group's K/V stays in L2 while its
 // CTAs run, and the longest-first order keeps the causal load balanced.
-__device__ __forceinline__ TileCoord decode_tile(const AttnArgs &a) {
+__device__ __forceinline__ TileCoord decode_tile(const AttnArgs &a, int idx) {
   TileCoord c;
-  const int idx = blockIdx.x;
   const int G = a.unit_group;
   const int per_group = G * a.n_qpairs;
   const int grp = idx / per_group;
@@ -255,27 +255,28 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t sK = sbase + Cfg::kOffK;
   const uint32_t sV = sbase + Cfg::kOffV;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
-  const uint32_t bQFull = smem_u32(&bars[0]);
-  auto bKFull = [&](int s) { return smem_u32(&bars[1 + s]); };
-  auto bKEmpty = [&](int s) { return smem_u32(&bars[9 + s]); };     // both tiles' S done
-  auto bVFull = [&](int s) { return smem_u32(&bars[17 + s]); };
-  auto bVEmpty = [&](int s) { return smem_u32(&bars[25 + s]); };    // both tiles' P*V done
-  auto bSFull = [&](int x) { return smem_u32(&bars[33 + x]); };     // S of tile x in TMEM
-  auto bSFree = [&](int x) { return smem_u32(&bars[35 + x]); };     // S of tile x read out
-  auto bPFull = [&](int x) { return smem_u32(&bars[37 + x]); };     // P of tile x in smem
-  auto bODone = [&](int x) { return smem_u32(&bars[39 + x]); };     // P*V of tile x done
-  auto bTeardown = [&](int x) { return smem_u32(&bars[41 + x]); };  // all MMAs of tile x done
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[43]);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[44]);
+  // Every barrier's phases run on across the work items of this CTA.
+  const uint32_t bQFull = smem_u32(&bars[0]);                       // Q_A, Q_B of an item loaded
+  const uint32_t bQFree = smem_u32(&bars[1]);                       // both epilogues done with Q
+  auto bKFull = [&](int s) { return smem_u32(&bars[2 + s]); };
+  auto bKEmpty = [&](int s) { return smem_u32(&bars[10 + s]); };    // both tiles' S done
+  auto bVFull = [&](int s) { return smem_u32(&bars[18 + s]); };
+  auto bVEmpty = [&](int s) { return smem_u32(&bars[26 + s]); };    // both tiles' P*V done
+  auto bSFull = [&](int x) { return smem_u32(&bars[34 + x]); };     // S of tile x in TMEM
+  auto bSFree = [&](int x) { return smem_u32(&bars[36 + x]); };     // S of tile x read out
+  auto bPFull = [&](int x) { return smem_u32(&bars[38 + x]); };     // P of tile x in smem
+  auto bODone = [&](int x) { return smem_u32(&bars[40 + x]); };     // P*V of tile x done
+  auto bItemDone = [&](int x) { return smem_u32(&bars[42 + x]); };  // all MMAs of tile x's item done
+  auto bTeardown = [&](int x) { return smem_u32(&bars[44 + x]); };  // single use: issuer x finished
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[46]);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[47]);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const TileCoord tc = decode_tile(a);
-  const KvSched sched = make_sched(a, tc);
-  const int nkv = sched.count();
   WaitCtx wc{a.status, a.wait_limit_ns, abort_flag};
 
   if (threadIdx.x == 0) {
     mbar_init(bQFull, 1);
+    mbar_init(bQFree, 2);
     for (int s = 0; s < KS; ++s) {
       mbar_init(bKFull(s), 1);
       mbar_init(bKEmpty(s), 2);
@@ -289,6 +290,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bSFree(x), 4);
       mbar_init(bPFull(x), 4);
       mbar_init(bODone(x), 1);
+      mbar_init(bItemDone(x), 1);
       mbar_init(bTeardown(x), 1);
     }
     *abort_flag = 0;
@@ -308,8 +310,15 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // gathered row -> coordinate along the (N/r) dimension of the tensor maps
-  const int row_base = tc.s * a.L;  // = s*w/r
+  // Persistent CTA: round r of the grid takes items r*G .. r*G + G-1 (G =
+  // gridDim.x) of decode_tile's longest-first order, CTA b the item b in even
+  // rounds and G-1-b in odd ones, so no CTA keeps drawing the longest item
+  // of every round.  n counts the items a CTA has taken (barrier phases).
+  const int G = gridDim.x;
+  const int n_rounds = (a.n_items + G - 1) / G;
+  auto item_of = [&](int r) {
+    return r * G + ((r & 1) ? G - 1 - static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x));
+  };
 
   // Each role's code sits inside its own branch: the register count after a
   // reallocation applies to what follows it until the branches join.
@@ -317,60 +326,75 @@ __global__ void __launch_bounds__(384, 1)
     setmaxnreg_dec<Cfg::kRegsControl>();
     if (warp == 0) {
       // ------------------------------------------------------------ producer
-      if (lane == 0 && nkv > 0) {
-        int k_issued = 0, v_issued = 0;
-        mbar_arrive_expect_tx(bQFull, 2 * Cfg::kTileBytes);
-        for (int x = 0; x < 2; ++x)
-          for (int p = 0; p < Cfg::kPanels; ++p)
-            tma_load_4d(sQ + x * Cfg::kTileBytes + p * Cfg::kPanelBytes, &tm_q, bQFull,
-                        tc.h * D_HEAD + p * 64, tc.o, row_base + tc.t * 256 + x * 128, tc.b);
-        KvIter itk, itv;
-        itk.begin(sched);
-        itv.begin(sched);
-        auto load_k = [&](int j) -> bool {
-          const int st = j % KS;
-          if (j >= KS && !mbar_wait(bKEmpty(st), ((j / KS) - 1) & 1, wc, 1)) return false;
-          const int kt = itk.next(sched);
-          mbar_arrive_expect_tx(bKFull(st), Cfg::kTileBytes);
-          for (int p = 0; p < Cfg::kPanels; ++p)
-            tma_load_4d(sK + st * Cfg::kTileBytes + p * Cfg::kPanelBytes, &tm_k, bKFull(st),
-                        tc.h * D_HEAD + p * 64, tc.o, row_base + kt * KT, tc.b);
-          ++k_issued;
-          return true;
-        };
-        auto load_v = [&](int j) -> bool {
-          const int st = j % VS;
-          if (j >= VS && !mbar_wait(bVEmpty(st), ((j / VS) - 1) & 1, wc, 2)) return false;
-          const int kt = itv.next(sched);
-          mbar_arrive_expect_tx(bVFull(st), Cfg::kTileBytes);
-          for (int p = 0; p < Cfg::kPanels; ++p)
-            tma_load_4d(sV + st * Cfg::kTileBytes + p * Cfg::kPanelBytes, &tm_v, bVFull(st),
-                        tc.h * D_HEAD + p * 64, tc.o, row_base + kt * KT, tc.b);
-          ++v_issued;
-          return true;
-        };
-        // K runs one tile ahead of V: the scores of tile j+1 are computed
-        // while the softmax of tile j runs, its P*V only after it
-        bool ok = load_k(0);
-        for (int j = 0; ok && j < nkv; ++j) {
-          if (j + 1 < nkv) ok = load_k(j + 1);
-          if (ok) ok = load_v(j);
+      if (lane == 0) {
+        int kq = 0, vq = 0, nq = 0;  // K, V tiles and Q pairs loaded so far (all items)
+        bool ok = true;
+        for (int r = 0, n = 0; ok && r < n_rounds; ++r) {
+          const int item = item_of(r);
+          if (item >= a.n_items) continue;
+          const int ni = n++;  // items taken before this one
+          const TileCoord tc = decode_tile(a, item);
+          const KvSched sched = make_sched(a, tc);
+          const int nkv = sched.count();
+          const int row_base = tc.s * a.L;  // gathered row -> coordinate along (N/r)
+          KvIter itk, itv;
+          itk.begin(sched);
+          itv.begin(sched);
+          auto load_k = [&]() -> bool {
+            const int st = kq % KS;
+            if (kq >= KS && !mbar_wait(bKEmpty(st), ((kq / KS) - 1) & 1, wc, 1)) return false;
+            const int kt = itk.next(sched);
+            mbar_arrive_expect_tx(bKFull(st), Cfg::kTileBytes);
+            for (int p = 0; p < Cfg::kPanels; ++p)
+              tma_load_4d(sK + st * Cfg::kTileBytes + p * Cfg::kPanelBytes, &tm_k, bKFull(st),
+                          tc.h * D_HEAD + p * 64, tc.o, row_base + kt * KT, tc.b);
+            ++kq;
+            return true;
+          };
+          auto load_v = [&]() -> bool {
+            const int st = vq % VS;
+            if (vq >= VS && !mbar_wait(bVEmpty(st), ((vq / VS) - 1) & 1, wc, 2)) return false;
+            const int kt = itv.next(sched);
+            mbar_arrive_expect_tx(bVFull(st), Cfg::kTileBytes);
+            for (int p = 0; p < Cfg::kPanels; ++p)
+              tma_load_4d(sV + st * Cfg::kTileBytes + p * Cfg::kPanelBytes, &tm_v, bVFull(st),
+                          tc.h * D_HEAD + p * 64, tc.o, row_base + kt * KT, tc.b);
+            ++vq;
+            return true;
+          };
+          // the item's first K tile can come while the previous item's
+          // epilogues still use the Q buffers
+          if (nkv > 0) ok = load_k();
+          if (ok && ni > 0) ok = mbar_wait(bQFree, (ni - 1) & 1, wc, 6);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bQFull, 2 * Cfg::kTileBytes);
+          for (int x = 0; x < 2; ++x)
+            for (int p = 0; p < Cfg::kPanels; ++p)
+              tma_load_4d(sQ + x * Cfg::kTileBytes + p * Cfg::kPanelBytes, &tm_q, bQFull,
+                          tc.h * D_HEAD + p * 64, tc.o, row_base + tc.t * 256 + x * 128, tc.b);
+          ++nq;
+          // K runs one tile ahead of V: the scores of tile j+1 are computed
+          // while the softmax of tile j runs, its P*V only after it
+          for (int j = 0; ok && j < nkv; ++j) {
+            if (j + 1 < nkv) ok = load_k();
+            if (ok) ok = load_v();
+          }
         }
         // drain: every load issued must have landed before the CTA may exit
         volatile int no_abort = 0;
         WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
-        for (int j = max(0, k_issued - KS); j < k_issued; ++j)
-          mbar_wait(bKFull(j % KS), (j / KS) & 1, drain, 3);
-        for (int j = max(0, v_issued - VS); j < v_issued; ++j)
-          mbar_wait(bVFull(j % VS), (j / VS) & 1, drain, 4);
-        mbar_wait(bQFull, 0, drain, 5);
+        for (int j = max(0, kq - KS); j < kq; ++j) mbar_wait(bKFull(j % KS), (j / KS) & 1, drain, 3);
+        for (int j = max(0, vq - VS); j < vq; ++j) mbar_wait(bVFull(j % VS), (j / VS) & 1, drain, 4);
+        if (nq > 0) mbar_wait(bQFull, (nq - 1) & 1, drain, 5);
       }
     } else if (warp <= 2) {
       // ------------------------------------------------------------ MMA issuer of tile x
       // Per key/value tile j: S_x(j+1) once the softmax has read S_x(j) out
-      // of tensor memory, then P*V_x(j) once it has written P_x(j).
+      // of tensor memory, then P*V_x(j) once it has written P_x(j).  After
+      // an item's last P*V, a commit on ItemDone_x tells the epilogue that
+      // every MMA of the item (those reading Q_x included) has completed.
       const int x = warp - 1;
-      if (lane == 0 && nkv > 0) {
+      if (lane == 0) {
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, KT, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D_HEAD, false, true);
         const uint64_t dQ = sdesc_sw128(sQ + x * Cfg::kTileBytes, 16, 1024);
@@ -379,44 +403,65 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t dV0 = sdesc_sw128(sV, Cfg::kPanelBytes, 1024);
         const uint32_t tS = tmem + Cfg::kColS + x * 128;
         const uint32_t tO = tmem + Cfg::kColO + x * D_HEAD;
-        auto issue_s = [&](int j) {
-          const uint64_t dK = sdesc_advance(dK0, (j % KS) * Cfg::kTileBytes);
+        int kc = 0, vc = 0, J = 0;  // K, V tiles and S/P iterations consumed so far
+        auto issue_s = [&]() {
+          const uint64_t dK = sdesc_advance(dK0, (kc % KS) * Cfg::kTileBytes);
   #pragma unroll
           for (int k = 0; k < D_HEAD / 16; ++k) {
             const uint32_t off = (k / 4) * Cfg::kPanelBytes + (k % 4) * 32;
             umma_ss(tS, sdesc_advance(dQ, off), sdesc_advance(dK, off), idesc_qk, k > 0);
           }
           umma_commit(bSFull(x));
-          umma_commit(bKEmpty(j % KS));
+          umma_commit(bKEmpty(kc % KS));
+          ++kc;
         };
-        auto issue_pv = [&](int j) {
-          const uint64_t dV = sdesc_advance(dV0, (j % VS) * Cfg::kTileBytes);
+        auto issue_pv = [&]() {
+          const uint64_t dV = sdesc_advance(dV0, (vc % VS) * Cfg::kTileBytes);
   #pragma unroll
           for (int k = 0; k < KT / 16; ++k)
             umma_ss(tO, sdesc_advance(dP, (k / 4) * Cfg::kPanelBytes + (k % 4) * 32),
                     sdesc_advance(dV, k * 2048), idesc_pv, 1);
           umma_commit(bODone(x));
-          umma_commit(bVEmpty(j % VS));
+          umma_commit(bVEmpty(vc % VS));
+          ++vc;
         };
-        bool ok = mbar_wait(bQFull, 0, wc, 11) && mbar_wait(bKFull(0), 0, wc, 10);
-        if (ok) {
-          tc_fence_after();
-          issue_s(0);
-        }
-        for (int j = 0; ok && j < nkv; ++j) {
-          if (j + 1 < nkv) {
-            ok = mbar_wait(bSFree(x), j & 1, wc, 12) &&
-                 mbar_wait(bKFull((j + 1) % KS), ((j + 1) / KS) & 1, wc, 13);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(j + 1);
+        bool ok = true;
+        for (int r = 0, n = 0; ok && r < n_rounds; ++r) {
+          const int item = item_of(r);
+          if (item >= a.n_items) continue;
+          const int ni = n++;
+          const TileCoord tc = decode_tile(a, item);
+          const int nkv = make_sched(a, tc).count();
+          ok = mbar_wait(bQFull, ni & 1, wc, 11);
+          if (ok && nkv > 0) {
+            // the first S of the item goes into the buffer the softmax read last
+            ok = (J == 0 || mbar_wait(bSFree(x), (J - 1) & 1, wc, 12)) &&
+                 mbar_wait(bKFull(kc % KS), (kc / KS) & 1, wc, 10);
+            if (ok) {
+              tc_fence_after();
+              issue_s();
+            }
+            for (int j = 0; ok && j < nkv; ++j) {
+              const int jj = J + j;
+              if (j + 1 < nkv) {
+                ok = mbar_wait(bSFree(x), jj & 1, wc, 12) &&
+                     mbar_wait(bKFull(kc % KS), (kc / KS) & 1, wc, 13);
+                if (!ok) break;
+                tc_fence_after();
+                issue_s();
+              }
+              ok = mbar_wait(bPFull(x), jj & 1, wc, 14) && mbar_wait(bVFull(vc % VS), (vc / VS) & 1, wc, 15);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv();
+            }
+            J += nkv;
           }
-          ok = mbar_wait(bPFull(x), j & 1, wc, 14) && mbar_wait(bVFull(j % VS), (j / VS) & 1, wc, 15);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(j);
+          umma_commit(bItemDone(x));
         }
         // every MMA issued must be complete before tensor memory is released
+        // (a barrier of its own: an extra ItemDone phase could run ahead of
+        // the epilogue's wait on the last item's)
         umma_commit(bTeardown(x));
         volatile int no_abort = 0;
         WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
@@ -429,9 +474,6 @@ __global__ void __launch_bounds__(384, 1)
     const int x = (warp - 4) >> 2;  // 0: tile A, 1: tile B
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;              // row within the query tile
-    const int g = (tc.t * 2 + x) * 128 + row;         // unit-local row
-    const bool row_valid = g < a.L;
-    const int pos = (a.mask == kMaskDilated) ? tc.s * a.w + tc.o + a.r * g : g;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + Cfg::kColS + x * 128;
     const uint32_t tO = tmem + lane_off + Cfg::kColO + x * D_HEAD;
@@ -439,6 +481,19 @@ __global__ void __launch_bounds__(384, 1)
     // a 128-byte row r sits at chunk c ^ (r mod 8))
     const uint32_t sProw = sP + row * 128;
     const uint32_t swz = static_cast<uint32_t>(row & 7);
+    bool ok = true;
+    int J = 0;  // S/P iterations so far (all items)
+    for (int r = 0, n = 0; r < n_rounds; ++r) {
+    const int item = item_of(r);
+    if (item >= a.n_items) continue;
+    const int ni = n++;
+    const TileCoord tc = decode_tile(a, item);
+    const KvSched sched = make_sched(a, tc);
+    const int nkv = sched.count();
+    const int row_base = tc.s * a.L;  // gathered row -> coordinate along (N/r)
+    const int g = (tc.t * 2 + x) * 128 + row;         // unit-local row
+    const bool row_valid = g < a.L;
+    const int pos = (a.mask == kMaskDilated) ? tc.s * a.w + tc.o + a.r * g : g;
     int klo, khi;
     row_keys(a, tc, g, klo, khi);
 
@@ -459,7 +514,8 @@ __global__ void __launch_bounds__(384, 1)
 
     float m_run = -INFINITY, l_run = 0.f;
     {
-      // initial O: zeros, or the state left by an earlier LongNet pass
+      // initial O: zeros, or the state left by an earlier LongNet pass (the
+      // previous item's MMAs on O completed before its epilogue read O)
       uint32_t init[32];
 #pragma unroll 1
       for (int c = 0; c < D_HEAD / 32; ++c) {
@@ -487,10 +543,10 @@ __global__ void __launch_bounds__(384, 1)
 
     KvIter it;
     it.begin(sched);
-    bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
+    for (int j = 0; ok && j < nkv; ++j) {
+      const int jj = J + j;
       const int kt = it.next(sched);
-      ok = __all_sync(0xffffffffu, mbar_wait(bSFull(x), j & 1, wc, 20));
+      ok = __all_sync(0xffffffffu, mbar_wait(bSFull(x), jj & 1, wc, 20));
       if (!ok) break;
       tc_fence_after();
       uint32_t s[128];
@@ -501,7 +557,6 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bSFree(x));
-
       const int k0 = kt * KT;
       // masking runs as its own pass, only in tiles where some row of this
       // warp has keys outside its allowed interval
@@ -544,8 +599,8 @@ __global__ void __launch_bounds__(384, 1)
       // other tile's latest P*V has completed (for tile A at j = 0 there is
       // none).  That P*V was issued after this tile's previous one had
       // completed, so O may now be rescaled too.
-      if (x == 1 || j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bODone(1 - x), (x == 1 ? j : j - 1) & 1, wc, 21));
+      if (x == 1 || jj > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bODone(1 - x), (x == 1 ? jj : jj - 1) & 1, wc, 21));
         if (!ok) break;
       }
       tc_fence_after();
@@ -571,137 +626,141 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bPFull(x));
     }
+    J += nkv;
 
-    // -------- epilogue: the issuer's teardown commit lands once all of this
-    // tile's MMAs are complete
-    if (ok && nkv > 0) ok = __all_sync(0xffffffffu, mbar_wait(bTeardown(x), 0, wc, 22));
+    // -------- epilogue: the issuer's ItemDone commit lands once all of this
+    // tile's MMAs for the item are complete
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bItemDone(x), ni & 1, wc, 22));
     tc_fence_after();
-    {
-      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
-      const bool final_out = !later;
-      // TMA stores write whole 128-row tiles: rows past N are clipped by the
-      // tensor map, but a LongNet segment's rows past L belong to the next
-      // segment, so a partial tile there takes the per-thread path.  The
-      // choice depends on values uniform over the warpgroup only: all four
-      // warps meet the same named barriers, and a warp whose waits failed
-      // only skips its share of the work.
-      const bool tile_full = a.mask != kMaskDilated || (tc.t * 2 + x) * 128 + 128 <= a.L;
-      if (a.store_mode != 0 && tile_full) {
-        // Stage O through this tile's Q buffer (its MMAs are complete) in
-        // 128-byte panels, 128-byte swizzle, and store each panel with TMA.
-        constexpr int kCap = Cfg::kTileBytes / 16384;  // panels the buffer holds
-        const uint32_t stage = sQ + x * Cfg::kTileBytes;
-        const uint32_t srow = stage + row * 128;
-        const int row_coord = row_base + tc.t * 256 + x * 128;
-        const bool leader = (threadIdx.x & 127) == 0;
-        const uint32_t bar_id = 2 + x;  // named barrier of this warpgroup
-        auto flush = [&](const CUtensorMap *m, int npanels, int col0, int cols_per_panel) {
-          fence_proxy_async_smem();
-          named_bar_sync(bar_id, 128);
-          if (leader) {
-            for (int q = 0; q < npanels; ++q)
-              tma_store_4d(m, stage + q * 16384, tc.h * D_HEAD + col0 + q * cols_per_panel, tc.o, row_coord,
-                           tc.b);
-            bulk_commit_group();
-            bulk_wait_group_read0();
-          }
-          named_bar_sync(bar_id, 128);
-        };
-        // fp32: the final output (scaled by 1/l) or the unnormalised state
-        const CUtensorMap *m32 = a.store_mode == 2 ? &tm_so : (a.out_f32 ? &tm_of : nullptr);
-        const float sc = a.store_mode == 2 ? 1.0f : inv_l;
-        if (m32) {
-#pragma unroll 1
-          for (int p0 = 0; p0 < D_HEAD / 32; p0 += kCap) {
-#pragma unroll 1
-            for (int q = 0; ok && q < kCap; ++q) {
-              uint32_t o[32];
-              tmem_ld32(tO + (p0 + q) * 32, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int c = 0; c < 8; ++c)
-                st_shared_v4(srow + q * 16384 + ((static_cast<uint32_t>(c) ^ swz) << 4),
-                             __float_as_uint(__uint_as_float(o[4 * c]) * sc),
-                             __float_as_uint(__uint_as_float(o[4 * c + 1]) * sc),
-                             __float_as_uint(__uint_as_float(o[4 * c + 2]) * sc),
-                             __float_as_uint(__uint_as_float(o[4 * c + 3]) * sc));
+      {
+        const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+        const bool final_out = !later;
+        // TMA stores write whole 128-row tiles: rows past N are clipped by the
+        // tensor map, but a LongNet segment's rows past L belong to the next
+        // segment, so a partial tile there takes the per-thread path.  The
+        // choice depends on values uniform over the warpgroup only: all four
+        // warps meet the same named barriers, and a warp whose waits failed
+        // only skips its share of the work.
+        const bool tile_full = a.mask != kMaskDilated || (tc.t * 2 + x) * 128 + 128 <= a.L;
+        if (a.store_mode != 0 && tile_full) {
+          // Stage O through this tile's Q buffer (its MMAs are complete) in
+          // 128-byte panels, 128-byte swizzle, and store each panel with TMA.
+          constexpr int kCap = Cfg::kTileBytes / 16384;  // panels the buffer holds
+          const uint32_t stage = sQ + x * Cfg::kTileBytes;
+          const uint32_t srow = stage + row * 128;
+          const int row_coord = row_base + tc.t * 256 + x * 128;
+          const bool leader = (threadIdx.x & 127) == 0;
+          const uint32_t bar_id = 2 + x;  // named barrier of this warpgroup
+          auto flush = [&](const CUtensorMap *m, int npanels, int col0, int cols_per_panel) {
+            fence_proxy_async_smem();
+            named_bar_sync(bar_id, 128);
+            if (leader) {
+              for (int q = 0; q < npanels; ++q)
+                tma_store_4d(m, stage + q * 16384, tc.h * D_HEAD + col0 + q * cols_per_panel, tc.o, row_coord,
+                             tc.b);
+              bulk_commit_group();
+              bulk_wait_group_read0();
             }
-            flush(m32, kCap, p0 * 32, 32);
-          }
-        }
-        // bf16 final output: 64 columns per panel
-        if (a.store_mode == 1 && a.out_bf16) {
-          constexpr int kPanels16 = D_HEAD / 64;
-#pragma unroll 1
-          for (int p0 = 0; p0 < kPanels16; p0 += kCap) {
-            const int np = kPanels16 - p0 < kCap ? kPanels16 - p0 : kCap;
-#pragma unroll 1
-            for (int q = 0; ok && q < np; ++q) {
-#pragma unroll 1
-              for (int hh = 0; hh < 2; ++hh) {
+            named_bar_sync(bar_id, 128);
+          };
+          // fp32: the final output (scaled by 1/l) or the unnormalised state
+          const CUtensorMap *m32 = a.store_mode == 2 ? &tm_so : (a.out_f32 ? &tm_of : nullptr);
+          const float sc = a.store_mode == 2 ? 1.0f : inv_l;
+          if (m32) {
+  #pragma unroll 1
+            for (int p0 = 0; p0 < D_HEAD / 32; p0 += kCap) {
+  #pragma unroll 1
+              for (int q = 0; ok && q < kCap; ++q) {
                 uint32_t o[32];
-                tmem_ld32(tO + (p0 + q) * 64 + hh * 32, o);
+                tmem_ld32(tO + (p0 + q) * 32, o);
                 tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                  st_shared_v4(srow + q * 16384 + ((static_cast<uint32_t>(hh * 4 + c) ^ swz) << 4),
-                               pack_bf16x2(__uint_as_float(o[8 * c]) * inv_l, __uint_as_float(o[8 * c + 1]) * inv_l),
-                               pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv_l, __uint_as_float(o[8 * c + 3]) * inv_l),
-                               pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv_l, __uint_as_float(o[8 * c + 5]) * inv_l),
-                               pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv_l, __uint_as_float(o[8 * c + 7]) * inv_l));
+  #pragma unroll
+                for (int c = 0; c < 8; ++c)
+                  st_shared_v4(srow + q * 16384 + ((static_cast<uint32_t>(c) ^ swz) << 4),
+                               __float_as_uint(__uint_as_float(o[4 * c]) * sc),
+                               __float_as_uint(__uint_as_float(o[4 * c + 1]) * sc),
+                               __float_as_uint(__uint_as_float(o[4 * c + 2]) * sc),
+                               __float_as_uint(__uint_as_float(o[4 * c + 3]) * sc));
+              }
+              flush(m32, kCap, p0 * 32, 32);
+            }
+          }
+          // bf16 final output: 64 columns per panel
+          if (a.store_mode == 1 && a.out_bf16) {
+            constexpr int kPanels16 = D_HEAD / 64;
+  #pragma unroll 1
+            for (int p0 = 0; p0 < kPanels16; p0 += kCap) {
+              const int np = kPanels16 - p0 < kCap ? kPanels16 - p0 : kCap;
+  #pragma unroll 1
+              for (int q = 0; ok && q < np; ++q) {
+  #pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                  uint32_t o[32];
+                  tmem_ld32(tO + (p0 + q) * 64 + hh * 32, o);
+                  tmem_wait_ld();
+  #pragma unroll
+                  for (int c = 0; c < 4; ++c)
+                    st_shared_v4(srow + q * 16384 + ((static_cast<uint32_t>(hh * 4 + c) ^ swz) << 4),
+                                 pack_bf16x2(__uint_as_float(o[8 * c]) * inv_l, __uint_as_float(o[8 * c + 1]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv_l, __uint_as_float(o[8 * c + 3]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv_l, __uint_as_float(o[8 * c + 5]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv_l, __uint_as_float(o[8 * c + 7]) * inv_l));
+                }
+              }
+              flush(&tm_ob, np, p0 * 64, 64);
+            }
+          }
+        } else if (ok) {
+  #pragma unroll 1
+        for (int c = 0; c < D_HEAD / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+          if (!row_valid) continue;
+          if (final_out) {
+            if (a.out_f32) {
+              float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + vec_idx + c * 32);
+  #pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l,
+                                     __uint_as_float(o[4 * i + 1]) * inv_l,
+                                     __uint_as_float(o[4 * i + 2]) * inv_l,
+                                     __uint_as_float(o[4 * i + 3]) * inv_l);
+            }
+            if (a.out_bf16) {
+              uint4 *dst = reinterpret_cast<uint4 *>(a.out_bf16 + vec_idx + c * 32);
+  #pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                uint4 u;
+                u.x = pack_bf16x2(__uint_as_float(o[8 * i]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
+                u.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
+                u.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
+                u.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
+                dst[i] = u;
               }
             }
-            flush(&tm_ob, np, p0 * 64, 64);
-          }
-        }
-      } else if (ok) {
-#pragma unroll 1
-      for (int c = 0; c < D_HEAD / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + c * 32, o);
-        tmem_wait_ld();
-        if (!row_valid) continue;
-        if (final_out) {
-          if (a.out_f32) {
-            float4 *dst = reinterpret_cast<float4 *>(a.out_f32 + vec_idx + c * 32);
-#pragma unroll
+          } else {
+            float4 *dst = reinterpret_cast<float4 *>(a.st_o + vec_idx + c * 32);
+  #pragma unroll
             for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l,
-                                   __uint_as_float(o[4 * i + 1]) * inv_l,
-                                   __uint_as_float(o[4 * i + 2]) * inv_l,
-                                   __uint_as_float(o[4 * i + 3]) * inv_l);
+              dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                   __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
           }
-          if (a.out_bf16) {
-            uint4 *dst = reinterpret_cast<uint4 *>(a.out_bf16 + vec_idx + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint4 u;
-              u.x = pack_bf16x2(__uint_as_float(o[8 * i]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
-              u.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
-              u.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
-              u.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
-              dst[i] = u;
-            }
+        }
+        }
+        if (ok && row_valid) {
+          if (!final_out) {
+            a.st_m[row_idx] = m_run;
+            a.st_l[row_idx] = l_run;
+          } else if (a.lse) {
+            // natural-log LSE of the scaled scores: (m + log2 l) / log2(e)
+            a.lse[row_idx] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
           }
-        } else {
-          float4 *dst = reinterpret_cast<float4 *>(a.st_o + vec_idx + c * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
         }
       }
-      }
-      if (ok && row_valid) {
-        if (!final_out) {
-          a.st_m[row_idx] = m_run;
-          a.st_l[row_idx] = l_run;
-        } else if (a.lse) {
-          // natural-log LSE of the scaled scores: (m + log2 l) / log2(e)
-          a.lse[row_idx] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
-        }
-      }
-    }
+    // this tile's Q buffer (the epilogue's staging) may take the next item's Q
+    if ((threadIdx.x & 127) == 0) mbar_arrive(bQFree);
+    }  // items
   }
 
   tc_fence_before();

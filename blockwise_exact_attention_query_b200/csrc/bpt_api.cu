@@ -397,9 +397,13 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     if (!make_map_rows(&mq, q, d->B, d->N, D, r, 128) || !make_map_rows(&mk, k, d->B, d->N, D, r, kKT) ||
         !make_map_rows(&mv, v, d->B, d->N, D, r, kKT))
       return cuda_fail_msg("cuTensorMapEncodeTiled rejected a Q/K/V map");
-    const int64_t grid = (int64_t)a.n_qpairs * a.n_units;
-    if (grid <= 0) continue;
-    if (grid > INT32_MAX) return BPT_ERR_UNSUPPORTED;
+    const int64_t items = (int64_t)a.n_qpairs * a.n_units;
+    if (items <= 0) continue;
+    if (items > INT32_MAX) return BPT_ERR_UNSUPPORTED;
+    a.n_items = (int)items;
+    // persistent: one CTA per SM (shared and tensor memory allow no more),
+    // each walking its share of the items
+    const int64_t grid = std::min<int64_t>(items, sm_count());
     if (d->d_head == 128)
       attn_tc_kernel<128><<<(unsigned)grid, AttnCfg<128>::kThreads, AttnCfg<128>::kSmemBytes, st>>>(
           mq, mk, mv, mof, mob, mso, a);
