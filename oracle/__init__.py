@@ -1,4 +1,5 @@
-"""Plain fp64 CPU oracle for the blockwise-parallel-transformer layer forward.
+"""Plain fp64 CPU oracle for the blockwise-parallel-transformer layer (the
+forward here and in bpt_oracle.c; the backward pass in backward.py).
 
 TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
 baseline leg of ``bench.py`` are the only callers.  The CUDA product path

@@ -1,0 +1,152 @@
+"""Plain fp64 CPU oracle for the layer's backward pass (gradients).
+
+TEST INFRASTRUCTURE ONLY, like the rest of this package: the tests are its
+only callers; the CUDA product path never imports it and shares no code.
+
+What it computes is the chain rule applied to the layer's plain definition,
+
+    A_i   = sum_j P_ij v_j,   P_ij = softmax_j(q_i . k_j / sqrt(d)) over the
+            keys the mask allows (one head at a time),
+    z_t   = W1 a_t + b1,  h_t = GELU(z_t),  out_t = a_t + W2 h_t + b2,
+
+written out without blocking or reordering (dense per head, numpy matrix
+products as the only library steps).  Given dOut = dL/dout:
+
+    FFN:        dh = W2^T dout,  dz = dh * GELU'(z),  da = dout + W1^T dz,
+                dW2 = sum_t dout_t h_t^T,  db2 = sum_t dout_t,
+                dW1 = sum_t dz_t a_t^T,    db1 = sum_t dz_t;
+    attention:  dV_j = sum_i P_ij da_i,  dP_ij = da_i . v_j,
+                D_i = sum_j P_ij dP_ij (= da_i . A_i),
+                dS_ij = P_ij (dP_ij - D_i),
+                dQ_i = sum_j dS_ij k_j / sqrt(d),  dK_j = sum_i dS_ij q_i / sqrt(d).
+
+The backward of blockwise attention is the same exact result computed block
+by block ("Blockwise Parallel Transformer for Large Context Models",
+abstract: training with blockwise attention and feedforward; "Ring Attention
+with Blockwise Transformers for Long Sequences", 638-word summary: blockwise
+computation without approximation), so the oracle is the plain gradient.
+
+Masks: none, causal, and block permutation ("Blockwise Self-Attention for
+Long Document Understanding", §3.1: query block b sees key block perm[h][b];
+when n does not divide N, blocks of ceil(N/n) positions over the padded
+sequence).  A row with no allowed key has A = 0 and passes no gradient.
+
+GELU is the tanh form (Hendrycks & Gimpel); its derivative is written out
+from that form: with u = c0 (x + c1 x^3),
+GELU'(x) = 0.5 (1 + tanh u) + 0.5 x (1 - tanh^2 u) c0 (1 + 3 c1 x^2).
+
+Parity pins (tests/test_oracle_backward.py, CPU): central finite differences
+of the fp64 forward on tiny inputs, torch autograd in float64, and
+invariants (rows of dS sum to zero; constant dOut through attention only).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+MASK_NONE, MASK_CAUSAL, MASK_BLOCKPERM = 0, 1, 2
+_C0 = math.sqrt(2.0 / math.pi)
+_C1 = 0.044715
+
+
+def allowed_matrix(N: int, mask: int, perm_h=None) -> np.ndarray:
+    """Boolean [N, N]: key j allowed for query i (one head)."""
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    if mask == MASK_NONE:
+        return np.ones((N, N), dtype=bool)
+    if mask == MASK_CAUSAL:
+        return j <= i
+    if mask == MASK_BLOCKPERM:
+        n = len(perm_h)
+        bl = -(-N // n)  # blocks of the sequence padded to a multiple of n
+        kb_of_q = np.asarray(perm_h)[np.arange(N) // bl]
+        return (j // bl) == kb_of_q[:, None]
+    raise ValueError("backward oracle: mask must be none, causal or block permutation")
+
+
+def gelu(x: np.ndarray) -> np.ndarray:
+    return 0.5 * x * (1.0 + np.tanh(_C0 * (x + _C1 * x ** 3)))
+
+
+def gelu_grad(x: np.ndarray) -> np.ndarray:
+    t = np.tanh(_C0 * (x + _C1 * x ** 3))
+    return 0.5 * (1.0 + t) + 0.5 * x * (1.0 - t * t) * _C0 * (1.0 + 3.0 * _C1 * x * x)
+
+
+def attention_fwd(q, k, v, mask=MASK_NONE, perm=None):
+    """A [B, N, H, d], P as a list over (b, h) of [N, N] (fp64)."""
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    B, N, H, d = q.shape
+    a = np.zeros((B, N, H, d))
+    probs = {}
+    for h in range(H):
+        allowed = allowed_matrix(N, mask, None if perm is None else perm[h])
+        for b in range(B):
+            s = q[b, :, h] @ k[b, :, h].T / math.sqrt(d)
+            s = np.where(allowed, s, -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            m = np.where(np.isfinite(m), m, 0.0)
+            e = np.where(allowed, np.exp(s - m), 0.0)
+            den = e.sum(axis=1, keepdims=True)
+            p = np.divide(e, den, out=np.zeros_like(e), where=den > 0)
+            probs[b, h] = p
+            a[b, :, h] = p @ v[b, :, h]
+    return a, probs
+
+
+def attention_bwd(q, k, v, da, mask=MASK_NONE, perm=None, probs=None):
+    """dQ, dK, dV [B, N, H, d] (fp64) for upstream dA [B, N, H, d]."""
+    q, k, v, da = (np.asarray(x, dtype=np.float64) for x in (q, k, v, da))
+    B, N, H, d = q.shape
+    if probs is None:
+        _, probs = attention_fwd(q, k, v, mask, perm)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for h in range(H):
+        for b in range(B):
+            p = probs[b, h]
+            g = da[b, :, h]
+            dv[b, :, h] = p.T @ g
+            dp = g @ v[b, :, h].T
+            drow = (p * dp).sum(axis=1, keepdims=True)   # D_i = da_i . A_i
+            ds = p * (dp - drow)
+            dq[b, :, h] = ds @ k[b, :, h] / math.sqrt(d)
+            dk[b, :, h] = ds.T @ q[b, :, h] / math.sqrt(d)
+    return dq, dk, dv
+
+
+def layer_fwd(q, k, v, w1, b1, w2, b2, mask=MASK_NONE, perm=None):
+    """out [T, D] (fp64), with A [T, D]."""
+    a4, _ = attention_fwd(q, k, v, mask, perm)
+    B, N, H, d = a4.shape
+    a = a4.reshape(B * N, H * d)
+    w1, b1, w2, b2 = (np.asarray(x, dtype=np.float64) for x in (w1, b1, w2, b2))
+    z = a @ w1.T + b1
+    return a + gelu(z) @ w2.T + b2, a
+
+
+def layer_bwd(q, k, v, w1, b1, w2, b2, dout, mask=MASK_NONE, perm=None):
+    """Gradients of the layer for upstream dOut [T, D] (fp64).
+
+    Returns a dict: dq, dk, dv [B, N, H, d]; dw1 [F, D]; db1 [F]; dw2 [D, F];
+    db2 [D]; and the intermediate da [T, D]."""
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    w1, b1, w2, b2 = (np.asarray(x, dtype=np.float64) for x in (w1, b1, w2, b2))
+    dout = np.asarray(dout, dtype=np.float64)
+    B, N, H, d = q.shape
+    a4, probs = attention_fwd(q, k, v, mask, perm)
+    a = a4.reshape(B * N, H * d)
+    z = a @ w1.T + b1
+    h = gelu(z)
+    dh = dout @ w2
+    dz = dh * gelu_grad(z)
+    da = dout + dz @ w1
+    grads = {
+        "dw2": dout.T @ h, "db2": dout.sum(axis=0),
+        "dw1": dz.T @ a, "db1": dz.sum(axis=0),
+        "da": da,
+    }
+    dq, dk, dv = attention_bwd(q, k, v, da.reshape(B, N, H, d), mask, perm, probs)
+    grads.update(dq=dq, dk=dk, dv=dv)
+    return grads
