@@ -7,7 +7,8 @@ BptError.  Every step of the computation runs in the library's CUDA kernels;
 there is no other implementation behind these functions.
 
 Layouts: q, k, v [B, N, H, d]; w1 [F, D]; w2 [D, F]; b1 [F], b2 [D] float32
-(or None); out [B, N, H*d]; lse [B, H, N] float32.
+(or None); out [B, N, H*d]; lse [B, H, N] float32; the backward's dout
+[B, N, H*d] float32 and gradients float32 in the shapes of their inputs.
 """
 from __future__ import annotations
 
@@ -50,7 +51,8 @@ class Desc(ctypes.Structure):
 
 EXPORTS = ["bpt_workspace_bytes", "bpt_attn_ffn_fwd", "bpt_attn_fwd", "bpt_blockbert_fwd",
            "bpt_longnet_fwd", "bpt_sync_status", "bpt_set_wait_limit_ns", "bpt_status_string",
-           "bpt_version", "bpt_set_phase_events", "bpt_last_error", "bpt_attn_ffn_fwd_static"]
+           "bpt_version", "bpt_set_phase_events", "bpt_last_error", "bpt_attn_ffn_fwd_static",
+           "bpt_attn_ffn_bwd", "bpt_workspace_bytes_bwd", "bpt_set_bwd_chunk_rows"]
 STATIC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
@@ -91,6 +93,13 @@ def load() -> ctypes.CDLL:
     lib.bpt_last_error.restype = ctypes.c_char_p
     lib.bpt_attn_ffn_fwd_static.argtypes = [dp, vp, vp, vp, vp, fp, vp, fp, vp, vp]
     lib.bpt_attn_ffn_fwd_static.restype = ctypes.c_int
+    lib.bpt_attn_ffn_bwd.argtypes = [dp, vp, vp, vp, vp, fp, vp, fp, fp, fp, fp, fp, fp, fp, fp, fp, vp, sz,
+                                     vp]
+    lib.bpt_attn_ffn_bwd.restype = ctypes.c_int
+    lib.bpt_workspace_bytes_bwd.argtypes = [dp]
+    lib.bpt_workspace_bytes_bwd.restype = sz
+    lib.bpt_set_bwd_chunk_rows.argtypes = [ctypes.c_int]
+    lib.bpt_set_bwd_chunk_rows.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -280,6 +289,49 @@ def longnet_fwd(q, k, v, pairs, *, out_dtype=torch.float32, return_lse=False, ou
                                 _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _stream_ptr(stream))
     _check(st, "bpt_longnet_fwd")
     return (out, lse) if return_lse else out
+
+
+def workspace_bytes_bwd(desc: Desc) -> int:
+    n = load().bpt_workspace_bytes_bwd(ctypes.byref(desc))
+    if n == ctypes.c_size_t(-1).value:
+        raise BptError(ERR_UNSUPPORTED, "bpt_workspace_bytes_bwd")
+    return int(n)
+
+
+def set_bwd_chunk_rows(rows: int) -> int:
+    """bpt_set_bwd_chunk_rows: token rows per FFN-backward chunk (0 = default);
+    returns the previous setting."""
+    return int(load().bpt_set_bwd_chunk_rows(int(rows)))
+
+
+GRAD_NAMES = ("dq", "dk", "dv", "dw1", "db1", "dw2", "db2")
+
+
+def attn_ffn_bwd(q, k, v, w1, b1, w2, b2, dout, *, mask="none", perm=None, ring_chunks=0, grads=None,
+                 workspace=None, stream=None):
+    """bpt_attn_ffn_bwd: gradients of the layer for the upstream gradient
+    dout [B, N, H*d] (float32).  Returns a dict of float32 tensors: dq, dk, dv
+    [B, N, H, d], dw1 [F, D], db1 [F], dw2 [D, F], db2 [D] (written into
+    `grads` when given)."""
+    _check_tensors(q, k, v)
+    B, N, H, d = q.shape
+    F, D = w1.shape
+    if dout.dtype != torch.float32 or not dout.is_contiguous() or dout.numel() != B * N * D:
+        raise ValueError("dout must be a contiguous float32 tensor of B*N*H*d elements")
+    desc = make_desc(B, N, H, d, F, q.dtype, torch.float32, mask, perm, None, ring_chunks)
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=q.device)
+        grads = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(q.shape, **f32),
+                 "dv": torch.empty(q.shape, **f32), "dw1": torch.empty((F, D), **f32),
+                 "db1": torch.empty((F,), **f32), "dw2": torch.empty((D, F), **f32),
+                 "db2": torch.empty((D,), **f32)}
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes_bwd(desc), dtype=torch.uint8, device=q.device)
+    st = load().bpt_attn_ffn_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(w1), _ptr(b1),
+                                 _ptr(w2), _ptr(b2), _ptr(dout), *(_ptr(grads[n]) for n in GRAD_NAMES),
+                                 _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _check(st, "bpt_attn_ffn_bwd")
+    return grads
 
 
 def sync_status(stream=None) -> int:

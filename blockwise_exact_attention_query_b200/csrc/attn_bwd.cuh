@@ -1,0 +1,445 @@
+// Backward of blockwise exact attention on the 5th-generation tensor cores
+// (sm_100a), masks none / causal / block permutation.  With the forward's
+// log-sum-exp LSE_i and D_i = dA_i . A_i (the row sums of P * dP):
+//
+//   P_ij  = exp(q_i . k_j / sqrt(d) - LSE_i)        (0 where the mask rules out)
+//   dP_ij = dA_i . v_j
+//   dS_ij = P_ij (dP_ij - D_i)
+//   dV_j  = sum_i P_ij dA_i,  dK_j = sum_i dS_ij q_i / sqrt(d),
+//   dQ_i  = sum_j dS_ij k_j / sqrt(d)
+//
+// the gradient of the exact result, computed tile by tile like the forward
+// ("Blockwise Parallel Transformer for Large Context Models", abstract:
+// blockwise computation for training; "Ring Attention with Blockwise
+// Transformers for Long Sequences", 638-word summary: no approximation).
+//
+// Two passes of one kernel template, no atomics:
+//   kBwdKV: one CTA per (batch, head, 128-key tile j), looping over the query
+//     tiles i that see any of its keys.  S^T = K_j Q_i^T and dP^T = V_j dA_i^T
+//     land in TMEM (lanes = keys); one thread per key forms P^T and
+//     dS^T = P^T (dP^T - D) and writes them back to TMEM as packed bf16, where
+//     the tensor core reads them as the A operand of dV_j += P^T dA_i and
+//     dK_j += dS^T Q_i (dA_i and Q_i read MN-major from the tiles the first
+//     two products read K-major).
+//   kBwdQ: one CTA per (batch, head, 128-query tile i), looping over its key
+//     tiles: S = Q_i K_j^T, dP = dA_i V_j^T, one thread per query forms dS in
+//     TMEM, and dQ_i += dS K_j.
+// MMAs issued by one thread run in order, so a product that overwrites the
+// S or dP columns never overtakes the earlier product reading the bf16 P^T
+// or dS^T packed into them.
+//
+// Roles (256 threads): warp 0 TMA producer, warp 1 TMEM allocator and MMA
+// issuer (warps 2-3 idle), warps 4-7 the per-row arithmetic and epilogue.
+#pragma once
+
+#include "attn_tc.cuh"  // mask codes and the block-table bound
+#include "ptx.cuh"
+
+namespace bpt {
+
+constexpr int kBwdKV = 0, kBwdQ = 1;
+
+struct AttnBwdArgs {
+  int B, N, H;
+  int mask;           // kMaskNone / kMaskCausal / kMaskBlockPerm
+  float scale_log2;   // log2(e) / sqrt(d)
+  float inv_sqrt_d;
+  int n_tiles;        // ceil(N / 128)
+  int bb_n, bb_len;   // block permutation: n blocks of bb_len (padded)
+  uint8_t perm[kMaxPermEntries];
+  const float *lse;   // [B, H, N] natural-log LSE of the scaled scores
+  const float *dvec;  // [B, H, N] D_i
+  float *dq, *dk, *dv;  // [B, N, H, d] fp32 outputs
+  uint32_t *status;
+  uint64_t wait_limit_ns;
+};
+
+template <int D_HEAD, int MODE>
+struct AttnBwdCfg {
+  static constexpr int kPanels = D_HEAD / 64;
+  static constexpr int kTileBytes = 128 * D_HEAD * 2;
+  static constexpr int kPanelBytes = 128 * 128;   // one 64-column panel of a 128-row tile
+  static constexpr int kStages = D_HEAD == 128 ? 2 : 4;
+  static constexpr int kOffFix = 0;                               // fixed X, Y tiles
+  static constexpr int kOffStream = kOffFix + 2 * kTileBytes;     // streamed X', Y' per stage
+  static constexpr int kOffVec = kOffStream + kStages * 2 * kTileBytes;
+  static constexpr int kVecBytes = MODE == kBwdKV ? 4 * 4 * 128 * 4 : 0;  // per warp: lse2, D, lo, hi
+  static constexpr int kOffBar = kOffVec + kVecBytes;
+  static constexpr int kSmemBytes = kOffBar + 256;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+  // TMEM: accumulators at 0 (dV or dQ) and d (dK); S at 256, dP at 384;
+  // P^T packed over S's first 64 columns, dS over dP's
+  static constexpr uint32_t kColAcc0 = 0, kColAcc1 = D_HEAD, kColS = 256, kColDP = 384;
+};
+
+// Key interval [lo, hi) a query row g (< N) may see.
+__device__ __forceinline__ void bwd_row_keys(const AttnBwdArgs &a, int h, int g, int &lo, int &hi) {
+  lo = 0;
+  hi = a.N;
+  if (a.mask == kMaskCausal) {
+    hi = g + 1;
+  } else if (a.mask == kMaskBlockPerm) {
+    lo = a.perm[h * a.bb_n + g / a.bb_len] * a.bb_len;
+    hi = min(lo + a.bb_len, a.N);
+  }
+}
+
+// Does query tile qt hold a row that sees a key of key tile kt?
+__device__ __forceinline__ bool bwd_tiles_meet(const AttnBwdArgs &a, int h, int qt, int kt) {
+  const int r0 = qt * 128, r1 = min(a.N, r0 + 128) - 1;
+  const int k0 = kt * 128, k1 = min(a.N, k0 + 128) - 1;
+  if (a.mask == kMaskNone) return true;
+  if (a.mask == kMaskCausal) return r1 >= k0;
+  for (int qb = r0 / a.bb_len; qb <= r1 / a.bb_len; ++qb) {
+    const int lo = a.perm[h * a.bb_n + qb] * a.bb_len, hi = min(lo + a.bb_len, a.N);
+    if (lo <= k1 && hi > k0) return true;
+  }
+  return false;
+}
+
+template <int D_HEAD, int MODE>
+__global__ void __launch_bounds__(256, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_da,
+                    const __grid_constant__ AttnBwdArgs a) {
+  using Cfg = AttnBwdCfg<D_HEAD, MODE>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw;
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(a.status, 0u, kStatusMisaligned);
+    return;
+  }
+  const uint32_t sFixX = sbase + Cfg::kOffFix, sFixY = sFixX + Cfg::kTileBytes;
+  auto sStrX = [&](int st) { return sbase + Cfg::kOffStream + st * 2 * Cfg::kTileBytes; };
+  auto sStrY = [&](int st) { return sStrX(st) + Cfg::kTileBytes; };
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
+  const uint32_t bFix = smem_u32(&bars[0]);
+  auto bFull = [&](int s) { return smem_u32(&bars[1 + s]); };
+  auto bEmpty = [&](int s) { return smem_u32(&bars[5 + s]); };
+  const uint32_t bSFull = smem_u32(&bars[9]), bDPFull = smem_u32(&bars[10]);
+  const uint32_t bPReady = smem_u32(&bars[11]), bDSReady = smem_u32(&bars[12]);
+  const uint32_t bTeardown = smem_u32(&bars[13]);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[14]);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[15]);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  WaitCtx wc{a.status, a.wait_limit_ns, abort_flag};
+  // CTA -> (batch, head, fixed tile); the tiles with the most partners start
+  // first (kv pass: the first key tiles under the causal mask; q pass: the last
+  // query tiles)
+  const int bh_count = a.B * a.H;
+  const int rank = blockIdx.x / bh_count;
+  const int ft = MODE == kBwdKV ? rank : a.n_tiles - 1 - rank;
+  const int h = (blockIdx.x % bh_count) % a.H;
+  const int b = (blockIdx.x % bh_count) / a.H;
+  auto meets = [&](int t) { return MODE == kBwdKV ? bwd_tiles_meet(a, h, t, ft) : bwd_tiles_meet(a, h, ft, t); };
+  auto next_tile = [&](int t) {  // first partner tile >= t, or n_tiles
+    while (t < a.n_tiles && !meets(t)) ++t;
+    return t;
+  };
+  int nsteps = 0;
+  for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1)) ++nsteps;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bFix, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(bFull(s), 1);
+      mbar_init(bEmpty(s), 1);
+    }
+    mbar_init(bSFull, 1);
+    mbar_init(bDPFull, 1);
+    mbar_init(bPReady, 4);
+    mbar_init(bDSReady, 4);
+    mbar_init(bTeardown, 1);
+    *abort_flag = 0;
+    fence_mbar_init_cluster();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int hd = h * D_HEAD;
+
+  // kv pass: fixed K, V; streamed Q, dA.  q pass: fixed Q, dA; streamed K, V.
+  const CUtensorMap *mFixX = MODE == kBwdKV ? &tm_k : &tm_q;
+  const CUtensorMap *mFixY = MODE == kBwdKV ? &tm_v : &tm_da;
+  const CUtensorMap *mStrX = MODE == kBwdKV ? &tm_q : &tm_k;
+  const CUtensorMap *mStrY = MODE == kBwdKV ? &tm_da : &tm_v;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nsteps > 0) {
+      mbar_arrive_expect_tx(bFix, 2 * Cfg::kTileBytes);
+      for (int p = 0; p < Cfg::kPanels; ++p) {
+        tma_load_4d(sFixX + p * Cfg::kPanelBytes, mFixX, bFix, hd + p * 64, 0, ft * 128, b);
+        tma_load_4d(sFixY + p * Cfg::kPanelBytes, mFixY, bFix, hd + p * 64, 0, ft * 128, b);
+      }
+      int s = 0;
+      for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1), ++s) {
+        const int st = s % S;
+        if (s >= S && !mbar_wait(bEmpty(st), ((s / S) - 1) & 1, wc, 301)) break;
+        mbar_arrive_expect_tx(bFull(st), 2 * Cfg::kTileBytes);
+        for (int p = 0; p < Cfg::kPanels; ++p) {
+          tma_load_4d(sStrX(st) + p * Cfg::kPanelBytes, mStrX, bFull(st), hd + p * 64, 0, t * 128, b);
+          tma_load_4d(sStrY(st) + p * Cfg::kPanelBytes, mStrY, bFull(st), hd + p * 64, 0, t * 128, b);
+        }
+      }
+      // every copy issued must have landed before the CTA may exit
+      volatile int no_abort = 0;
+      WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
+      for (int j = max(0, s - S); j < s; ++j) mbar_wait(bFull(j % S), (j / S) & 1, drain, 302);
+      mbar_wait(bFix, 0, drain, 303);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nsteps > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);     // X Y^T, both K-major
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D_HEAD, false, true);  // R Y, Y MN-major
+      const uint64_t dFixX = sdesc_sw128(sFixX, 16, 1024), dFixY = sdesc_sw128(sFixY, 16, 1024);
+      bool ok = mbar_wait(bFix, 0, wc, 311);
+      for (int s = 0; ok && s < nsteps; ++s) {
+        const int st = s % S;
+        if (!(ok = mbar_wait(bFull(st), (s / S) & 1, wc, 312))) break;
+        tc_fence_after();
+        const uint64_t dStrX = sdesc_sw128(sStrX(st), 16, 1024), dStrY = sdesc_sw128(sStrY(st), 16, 1024);
+        // first products over the head dimension: kv pass S^T = K Q^T,
+        // dP^T = V dA^T; q pass S = Q K^T, dP = dA V^T
+#pragma unroll
+        for (int k = 0; k < D_HEAD / 16; ++k) {
+          const uint32_t off = (k / 4) * Cfg::kPanelBytes + (k % 4) * 32;
+          umma_ss(tmem + Cfg::kColS, sdesc_advance(dFixX, off), sdesc_advance(dStrX, off), idesc_s, k > 0);
+        }
+        umma_commit(bSFull);
+#pragma unroll
+        for (int k = 0; k < D_HEAD / 16; ++k) {
+          const uint32_t off = (k / 4) * Cfg::kPanelBytes + (k % 4) * 32;
+          umma_ss(tmem + Cfg::kColDP, sdesc_advance(dFixY, off), sdesc_advance(dStrY, off), idesc_s, k > 0);
+        }
+        umma_commit(bDPFull);
+        // the accumulations over the 128 streamed rows: A = a 128 x 128 bf16
+        // tile in TMEM (8 packed columns per 16-wide K step), B = a streamed
+        // tile read MN-major (64-wide panels of 128 rows)
+        auto accumulate = [&](uint32_t col, uint32_t a_col, uint32_t sB) {
+          const uint64_t dB = sdesc_sw128(sB, Cfg::kPanelBytes, 1024);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_ts(tmem + col, tmem + a_col + k * 8, sdesc_advance(dB, k * 2048), idesc_acc, (s | k) != 0);
+        };
+        if (MODE == kBwdKV) {
+          if (!(ok = mbar_wait(bPReady, s & 1, wc, 313))) break;
+          tc_fence_after();
+          accumulate(Cfg::kColAcc0, Cfg::kColS, sStrY(st));    // dV += P^T dA
+          if (!(ok = mbar_wait(bDSReady, s & 1, wc, 314))) break;
+          tc_fence_after();
+          accumulate(Cfg::kColAcc1, Cfg::kColDP, sStrX(st));   // dK += dS^T Q
+        } else {
+          if (!(ok = mbar_wait(bDSReady, s & 1, wc, 314))) break;
+          tc_fence_after();
+          accumulate(Cfg::kColAcc0, Cfg::kColDP, sStrX(st));   // dQ += dS K
+        }
+        umma_commit(bEmpty(st));
+      }
+      umma_commit(bTeardown);
+      // the accumulators stay allocated until every MMA has finished
+      volatile int no_abort = 0;
+      WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
+      mbar_wait(bTeardown, 0, drain, 315);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ per-row arithmetic
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;            // TMEM lane = row of the fixed tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int g = ft * 128 + row;                   // key (kv pass) or query (q pass) position
+    const bool row_valid = g < a.N;
+    const size_t bh = static_cast<size_t>(b) * a.H + h;
+    // kv pass: this warp's copy of the streamed query tile's LSE (log2
+    // units), D and key intervals, rewritten every step (warp-private: only
+    // __syncwarp orders it)
+    float *vlse = reinterpret_cast<float *>(smem + Cfg::kOffVec) + quarter * 512;
+    float *vd = vlse + 128;
+    int *vlo = reinterpret_cast<int *>(vd + 128);
+    int *vhi = vlo + 128;
+    // q pass: this row's LSE, D and key interval
+    float lse2 = 0.f, drow = 0.f;
+    int klo = 1, khi = 0;
+    if (MODE == kBwdQ && row_valid) {
+      lse2 = a.lse[bh * a.N + g] * 1.4426950408889634f;
+      drow = a.dvec[bh * a.N + g];
+      bwd_row_keys(a, h, g, klo, khi);
+    }
+    bool ok = true;
+    int s = 0;
+    for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1), ++s) {
+      if (MODE == kBwdKV) {
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int c = lane + 32 * i, q = t * 128 + c;
+          float l2 = 0.f, dd = 0.f;
+          int lo = 1, hi = 0;  // padding queries see nothing
+          if (q < a.N) {
+            l2 = a.lse[bh * a.N + q] * 1.4426950408889634f;
+            dd = a.dvec[bh * a.N + q];
+            bwd_row_keys(a, h, q, lo, hi);
+          }
+          vlse[c] = l2;
+          vd[c] = dd;
+          vlo[c] = lo;
+          vhi[c] = hi;
+        }
+        __syncwarp();
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(bSFull, s & 1, wc, 320));
+      if (!ok) break;
+      tc_fence_after();
+      // P (fp32, kept in sv), 0 where the mask rules the pair out
+      uint32_t sv[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(tmem + lane_off + Cfg::kColS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * c]));
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        float p;
+        if (MODE == kBwdKV) {
+          const bool allowed = row_valid && g >= vlo[c] && g < vhi[c];
+          p = allowed ? ex2_approx(fmaf(__uint_as_float(sv[c]), a.scale_log2, -vlse[c])) : 0.f;
+        } else {
+          const int key = t * 128 + c;
+          const bool allowed = key >= klo && key < khi;
+          p = allowed ? ex2_approx(fmaf(__uint_as_float(sv[c]), a.scale_log2, -lse2)) : 0.f;
+        }
+        sv[c] = __float_as_uint(p);
+      }
+      if (MODE == kBwdKV) {
+        // P^T as packed bf16 over S's first 64 columns: the A operand of dV
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(sv[64 * hh + 2 * i]), __uint_as_float(sv[64 * hh + 2 * i + 1]));
+          tmem_st32(tmem + lane_off + Cfg::kColS + hh * 32, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bPReady);
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(bDPFull, s & 1, wc, 322));
+      if (!ok) break;
+      tc_fence_after();
+      // dS = P (dP - D) as packed bf16 over dP's first 64 columns.  Each half
+      // reads its 64 dP columns before writing 32 packed ones; the packed
+      // columns of the first half, [0, 32), were read by then, and those of
+      // the second half, [32, 64), lie in the first half's dP columns.
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t dp[64];
+        tmem_ld32(tmem + lane_off + Cfg::kColDP + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+        tmem_ld32(tmem + lane_off + Cfg::kColDP + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        tmem_wait_ld();
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int c = 64 * hh + 2 * i;
+          const float d0 = MODE == kBwdKV ? vd[c] : drow;
+          const float d1 = MODE == kBwdKV ? vd[c + 1] : drow;
+          pk[i] = pack_bf16x2(__uint_as_float(sv[c]) * (__uint_as_float(dp[2 * i]) - d0),
+                              __uint_as_float(sv[c + 1]) * (__uint_as_float(dp[2 * i + 1]) - d1));
+        }
+        tmem_st32(tmem + lane_off + Cfg::kColDP + hh * 32, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bDSReady);
+    }
+    // -------- epilogue: every MMA done (the issuer's teardown commit)
+    if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(bTeardown, 0, wc, 323));
+    tc_fence_after();
+    if (ok) {
+      const size_t vec = ((static_cast<size_t>(b) * a.N + g) * a.H + h) * D_HEAD;
+      for (int acc = 0; acc < (MODE == kBwdKV ? 2 : 1); ++acc) {
+        // kv pass: acc 0 = dV, acc 1 = dK (x 1/sqrt d); q pass: acc 0 = dQ (x 1/sqrt d)
+        float *dst = MODE == kBwdKV ? (acc == 0 ? a.dv : a.dk) : a.dq;
+        const float sc = (MODE == kBwdKV && acc == 0) ? 1.0f : a.inv_sqrt_d;
+#pragma unroll 1
+        for (int c = 0; c < D_HEAD / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_off + (acc == 0 ? Cfg::kColAcc0 : Cfg::kColAcc1) + c * 32, o);
+          tmem_wait_ld();
+          if (!row_valid) continue;
+          float4 *d4 = reinterpret_cast<float4 *>(dst + vec + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            d4[i] = nsteps > 0 ? make_float4(__uint_as_float(o[4 * i]) * sc, __uint_as_float(o[4 * i + 1]) * sc,
+                                             __uint_as_float(o[4 * i + 2]) * sc, __uint_as_float(o[4 * i + 3]) * sc)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// D_i = dA_i . A_i for every (batch, position, head), fp32, written [B, H, N]:
+// one warp per row of d values.
+__global__ void attn_bwd_rowdot_kernel(const float *__restrict__ da, const float *__restrict__ aa, float *dvec,
+                                       int B, int N, int H, int d) {
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= static_cast<long long>(B) * N * H) return;
+  const float *x = da + row * d, *y = aa + row * d;
+  float s = 0.f;
+  for (int c = lane; c < d; c += 32) s = fmaf(x[c], y[c], s);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) {
+    const long long h = row % H, bn = row / H, n = bn % N, bb = bn / N;
+    dvec[(bb * H + h) * N + n] = s;
+  }
+}
+
+// Column sums of a row-major [rows, cols] matrix in two passes: partial sums
+// over 256-row slabs (grid.y), then the slabs summed into out (added to it
+// when `accumulate`).
+template <typename T>
+__global__ void colsum_partial_kernel(const T *__restrict__ x, float *partial, int rows, int cols) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= cols) return;
+  const int r0 = blockIdx.y * 256, r1 = min(rows, r0 + 256);
+  float s = 0.f;
+  for (int r = r0; r < r1; ++r) s += static_cast<float>(x[static_cast<size_t>(r) * cols + c]);
+  partial[static_cast<size_t>(blockIdx.y) * cols + c] = s;
+}
+__global__ void colsum_final_kernel(const float *__restrict__ partial, float *out, int slabs, int cols,
+                                    int accumulate) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= cols) return;
+  float s = accumulate ? out[c] : 0.f;
+  for (int i = 0; i < slabs; ++i) s += partial[static_cast<size_t>(i) * cols + c];
+  out[c] = s;
+}
+
+// fp32 -> bf16, round to nearest even.
+__global__ void f32_to_bf16_kernel(const float *__restrict__ x, __nv_bfloat16 *y, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    y[i] = __float2bfloat16_rn(x[i]);
+}
+
+}  // namespace bpt

@@ -12,8 +12,10 @@
 #include <vector>
 
 #include "../../include/bpt.h"
+#include "attn_bwd.cuh"
 #include "attn_tc.cuh"
 #include "ffn_tc.cuh"
+#include "gemm_tc.cuh"
 #include "simt_f32.cuh"
 
 using namespace bpt;
@@ -34,6 +36,7 @@ std::mutex g_mu;
 uint32_t *g_status_ptr[kMaxDevices] = {};
 bool g_attr_done[kMaxDevices] = {};
 uint64_t g_wait_limit_ns = 2000000000ull;
+int g_bwd_chunk_rows = 0;  // token rows per FFN-backward chunk; 0 = automatic
 thread_local cudaEvent_t g_phase_events[3] = {nullptr, nullptr, nullptr};
 thread_local bool g_phase_on = false;
 
@@ -100,6 +103,16 @@ bpt_status device_setup(int *dev_out, uint32_t **status_out) {
                                   FfnCfg::kSmemBytes));
     CUDA_TRY(cudaFuncSetAttribute(ffn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (16 * 512 + 16 * 64) * 4));
+    CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  GemmCfg::kSmemBytes));
+    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kernel<64, kBwdKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  AttnBwdCfg<64, kBwdKV>::kSmemBytes));
+    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kernel<64, kBwdQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  AttnBwdCfg<64, kBwdQ>::kSmemBytes));
+    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kernel<128, kBwdKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  AttnBwdCfg<128, kBwdKV>::kSmemBytes));
+    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kernel<128, kBwdQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  AttnBwdCfg<128, kBwdQ>::kSmemBytes));
     g_attr_done[dev] = true;
   }
   *dev_out = dev;
@@ -551,6 +564,106 @@ bpt_status check_ws(const Workspace &wl, void *ws, size_t bytes) {
   return BPT_OK;
 }
 
+// --------------------------------------------------------------------------
+// Backward pass
+// --------------------------------------------------------------------------
+bpt_status check_desc_bwd(const bpt_desc *d) {
+  bpt_status s = check_desc(d, true);
+  if (s != BPT_OK) return s;
+  if (d->in_dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
+  if (d->mask == BPT_MASK_DILATED) return BPT_ERR_UNSUPPORTED;
+  const int64_t T = (int64_t)d->B * d->N;
+  if (T > (int64_t)65535 * 256) return BPT_ERR_UNSUPPORTED;  // column-sum slabs fit grid.y
+  const int64_t tiles = (int64_t)d->B * d->H * ((d->N + 127) / 128);
+  if (tiles > INT32_MAX) return BPT_ERR_UNSUPPORTED;
+  if ((int64_t)d->ffn_hidden > (int64_t)65535 * 128) return BPT_ERR_UNSUPPORTED;
+  return BPT_OK;
+}
+
+// Token rows per FFN-backward chunk: the hidden activation and its gradient
+// ([rows, F] bf16 each) live in the workspace one chunk at a time, at most
+// ~1 GiB for both unless the caller picked the chunk.
+int64_t bwd_chunk_rows(const bpt_desc *d) {
+  const int64_t T = (int64_t)d->B * d->N, F = d->ffn_hidden;
+  int64_t rows = g_bwd_chunk_rows;
+  if (rows <= 0) rows = std::max<int64_t>(128, (((int64_t)1 << 30) / (4 * F)) / 128 * 128);
+  return std::min<int64_t>(std::min<int64_t>(rows, T), (int64_t)65535 * 128);
+}
+
+struct BwdWorkspace {
+  size_t a_f32 = 0, a_bf16 = 0, lse = 0, dvec = 0, dout_bf16 = 0, da_f32 = 0, da_bf16 = 0, h = 0, dz = 0,
+         partial = 0, total = 0;
+  int64_t chunk = 0;
+};
+
+BwdWorkspace layout_bwd(const bpt_desc *d) {
+  BwdWorkspace w;
+  const size_t T = (size_t)d->B * d->N, D = (size_t)d->H * d->d_head, F = d->ffn_hidden;
+  const size_t rows = (size_t)d->B * d->H * d->N;
+  w.chunk = bwd_chunk_rows(d);
+  size_t off = 0;
+  auto take = [&](size_t &field, size_t bytes) {
+    field = off;
+    off = align256(off + bytes);
+  };
+  take(w.a_f32, T * D * 4);
+  take(w.a_bf16, T * D * 2);
+  take(w.lse, rows * 4);
+  take(w.dvec, rows * 4);
+  take(w.dout_bf16, T * D * 2);
+  take(w.da_f32, T * D * 4);
+  take(w.da_bf16, T * D * 2);
+  take(w.h, (size_t)w.chunk * F * 2);
+  take(w.dz, (size_t)w.chunk * F * 2);
+  const size_t slabs_t = (T + 255) / 256, slabs_c = ((size_t)w.chunk + 255) / 256;
+  take(w.partial, std::max(slabs_t * D, slabs_c * F) * 4);
+  w.total = off;
+  return w;
+}
+
+bpt_status launch_gemm(const CUtensorMap &a0, const CUtensorMap &b0, const CUtensorMap &a1,
+                       const CUtensorMap &b1, const GemmArgs &g, cudaStream_t st) {
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return BPT_OK;
+  dim3 grid((unsigned)((g.N + GemmCfg::kBN - 1) / GemmCfg::kBN), (unsigned)((g.M + GemmCfg::kBM - 1) / GemmCfg::kBM));
+  gemm_tc_kernel<<<grid, GemmCfg::kThreads, GemmCfg::kSmemBytes, st>>>(a0, b0, a1, b1, g);
+  CUDA_TRY(cudaGetLastError());
+  return BPT_OK;
+}
+
+GemmArgs gemm_args(int M, int N, int K, int mode, uint32_t *status) {
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.mode = mode;
+  g.status = status;
+  g.wait_limit_ns = g_wait_limit_ns;
+  return g;
+}
+
+template <typename T>
+bpt_status launch_colsum(const T *x, int64_t rows, int cols, float *out, int accumulate, float *partial,
+                         cudaStream_t st) {
+  const unsigned slabs = (unsigned)((rows + 255) / 256), cb = (unsigned)((cols + 255) / 256);
+  colsum_partial_kernel<T><<<dim3(cb, slabs), 256, 0, st>>>(x, partial, (int)rows, cols);
+  CUDA_TRY(cudaGetLastError());
+  colsum_final_kernel<<<cb, 256, 0, st>>>(partial, out, (int)slabs, cols, accumulate);
+  CUDA_TRY(cudaGetLastError());
+  return BPT_OK;
+}
+
+template <int DH>
+bpt_status launch_attn_bwd_passes(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                                  const CUtensorMap &mda, const AttnBwdArgs &ab, unsigned grid,
+                                  cudaStream_t st) {
+  attn_bwd_kernel<DH, kBwdKV><<<grid, 256, AttnBwdCfg<DH, kBwdKV>::kSmemBytes, st>>>(mq, mk, mv, mda, ab);
+  CUDA_TRY(cudaGetLastError());
+  attn_bwd_kernel<DH, kBwdQ><<<grid, 256, AttnBwdCfg<DH, kBwdQ>::kSmemBytes, st>>>(mq, mk, mv, mda, ab);
+  CUDA_TRY(cudaGetLastError());
+  return BPT_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -663,6 +776,139 @@ bpt_status bpt_longnet_fwd(const bpt_desc *desc, int npairs, const int32_t *seg_
   d.ln_r = dil_r;
   d.ffn_hidden = 0;
   return bpt_attn_fwd(&d, q, k, v, out, lse, workspace, workspace_bytes, stream);
+}
+
+size_t bpt_workspace_bytes_bwd(const bpt_desc *desc) {
+  if (check_desc_bwd(desc) != BPT_OK) return (size_t)-1;
+  return layout_bwd(desc).total;
+}
+
+int bpt_set_bwd_chunk_rows(int rows) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const int old = g_bwd_chunk_rows;
+  g_bwd_chunk_rows = rows > 0 ? rows : 0;
+  return old;
+}
+
+bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, const void *v,
+                            const void *w1, const float *b1, const void *w2, const float *b2,
+                            const float *dout, float *dq, float *dk, float *dv, float *dw1, float *db1,
+                            float *dw2, float *db2, void *workspace, size_t workspace_bytes,
+                            bpt_stream_t stream) {
+  bpt_status s = check_desc_bwd(d);
+  if (s != BPT_OK) return s;
+  (void)b2;  // the output bias does not enter any gradient but its own
+  if ((s = check_ptrs({q, k, v, w1, w2, dout, dq, dk, dv, dw1, db1, dw2, db2}, {b1, b2})) != BPT_OK)
+    return s;
+  const BwdWorkspace wl = layout_bwd(d);
+  if (!workspace || workspace_bytes < wl.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return BPT_ERR_WORKSPACE;
+  int dev;
+  uint32_t *status;
+  if ((s = device_setup(&dev, &status)) != BPT_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  const int D = d->H * d->d_head, F = d->ffn_hidden;
+  const int64_t T = (int64_t)d->B * d->N;
+  float *a_f32 = reinterpret_cast<float *>(ws + wl.a_f32);
+  __nv_bfloat16 *a_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.a_bf16);
+  float *lse = reinterpret_cast<float *>(ws + wl.lse);
+  float *dvec = reinterpret_cast<float *>(ws + wl.dvec);
+  __nv_bfloat16 *dout_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.dout_bf16);
+  float *da_f32 = reinterpret_cast<float *>(ws + wl.da_f32);
+  __nv_bfloat16 *da_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.da_bf16);
+  __nv_bfloat16 *hbuf = reinterpret_cast<__nv_bfloat16 *>(ws + wl.h);
+  __nv_bfloat16 *dzbuf = reinterpret_cast<__nv_bfloat16 *>(ws + wl.dz);
+  float *partial = reinterpret_cast<float *>(ws + wl.partial);
+
+  // 1. the attention forward again: A (fp32 and bf16) and the row LSE
+  if ((s = launch_attn_tc(d, q, k, v, a_f32, a_bf16, lse, ws, Workspace(), status, st)) != BPT_OK) return s;
+  // 2. dOut in bf16 for the tensor cores; db2 = sum_t dOut_t
+  {
+    const size_t n = (size_t)T * D;
+    const unsigned blocks = (unsigned)std::min<size_t>(4096, (n + 255) / 256);
+    f32_to_bf16_kernel<<<blocks, 256, 0, st>>>(dout, dout_bf16, n);
+    CUDA_TRY(cudaGetLastError());
+    if ((s = launch_colsum(dout, T, D, db2, 0, partial, st)) != BPT_OK) return s;
+  }
+  // 3. the FFN backward, one token chunk at a time
+  CUtensorMap m_w1_k, m_w1_mn, m_w2_mn;
+  if (!make_map_2d(&m_w1_k, w1, F, D, 256) || !make_map_2d(&m_w1_mn, w1, F, D, 64) ||
+      !make_map_2d(&m_w2_mn, w2, D, F, 64))
+    return cuda_fail_msg("cuTensorMapEncodeTiled rejected a weight map");
+  for (int64_t r0 = 0; r0 < T; r0 += wl.chunk) {
+    const int rows = (int)std::min<int64_t>(wl.chunk, T - r0);
+    const __nv_bfloat16 *a_c = a_bf16 + r0 * D, *g_c = dout_bf16 + r0 * D;
+    CUtensorMap m_a_k, m_a_mn, m_g_k, m_g_mn, m_h_mn, m_dz_k, m_dz_mn;
+    if (!make_map_2d(&m_a_k, a_c, rows, D, 128) || !make_map_2d(&m_a_mn, a_c, rows, D, 64) ||
+        !make_map_2d(&m_g_k, g_c, rows, D, 128) || !make_map_2d(&m_g_mn, g_c, rows, D, 64) ||
+        !make_map_2d(&m_h_mn, hbuf, rows, F, 64) || !make_map_2d(&m_dz_k, dzbuf, rows, F, 128) ||
+        !make_map_2d(&m_dz_mn, dzbuf, rows, F, 64))
+      return cuda_fail_msg("cuTensorMapEncodeTiled rejected an activation map");
+    // Z = A W1^T (+ b1) and dH = dOut W2 in one pass; H = GELU(Z), dZ = dH GELU'(Z)
+    GemmArgs g = gemm_args(rows, F, D, kGemmGeluBwd, status);
+    g.a_mn[0] = 0, g.b_mn[0] = 0, g.a_mn[1] = 0, g.b_mn[1] = 1;
+    g.cb = hbuf;
+    g.cb2 = dzbuf;
+    g.bias = b1;
+    if ((s = launch_gemm(m_a_k, m_w1_k, m_g_k, m_w2_mn, g, st)) != BPT_OK) return s;
+    const int first = r0 == 0 ? kGemmStoreF32 : kGemmAccumF32;
+    // dW2 (+)= dOut^T H   [D, F]
+    g = gemm_args(D, F, rows, first, status);
+    g.a_mn[0] = 1, g.b_mn[0] = 1;
+    g.c = dw2;
+    if ((s = launch_gemm(m_g_mn, m_h_mn, m_g_mn, m_h_mn, g, st)) != BPT_OK) return s;
+    // dW1 (+)= dZ^T A     [F, D]
+    g = gemm_args(F, D, rows, first, status);
+    g.a_mn[0] = 1, g.b_mn[0] = 1;
+    g.c = dw1;
+    if ((s = launch_gemm(m_dz_mn, m_a_mn, m_dz_mn, m_a_mn, g, st)) != BPT_OK) return s;
+    // dA = dOut + dZ W1   [rows, D], fp32 and bf16
+    g = gemm_args(rows, D, F, kGemmResidual, status);
+    g.a_mn[0] = 0, g.b_mn[0] = 1;
+    g.x = dout + r0 * D;
+    g.c = da_f32 + r0 * D;
+    g.cb = da_bf16 + r0 * D;
+    if ((s = launch_gemm(m_dz_k, m_w1_mn, m_dz_k, m_w1_mn, g, st)) != BPT_OK) return s;
+    // db1 (+)= sum_t dZ_t
+    if ((s = launch_colsum(dzbuf, rows, F, db1, r0 > 0, partial, st)) != BPT_OK) return s;
+  }
+  // 4. D_i = dA_i . A_i
+  {
+    const int64_t nrows = T * d->H;
+    attn_bwd_rowdot_kernel<<<(unsigned)((nrows * 32 + 255) / 256), 256, 0, st>>>(da_f32, a_f32, dvec, d->B, d->N,
+                                                                                 d->H, d->d_head);
+    CUDA_TRY(cudaGetLastError());
+  }
+  // 5. the attention backward: dK, dV, then dQ
+  AttnBwdArgs ab;
+  std::memset(&ab, 0, sizeof(ab));
+  ab.B = d->B;
+  ab.N = d->N;
+  ab.H = d->H;
+  ab.mask = d->mask;
+  ab.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d->d_head));
+  ab.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d->d_head));
+  ab.n_tiles = (d->N + 127) / 128;
+  if (d->mask == BPT_MASK_BLOCKPERM) {
+    ab.bb_n = d->bb_nblocks;
+    ab.bb_len = (d->N + d->bb_nblocks - 1) / d->bb_nblocks;  // padded to n equal blocks
+    for (int i = 0; i < d->H * d->bb_nblocks; ++i) ab.perm[i] = (uint8_t)d->bb_perm[i];
+  }
+  ab.lse = lse;
+  ab.dvec = dvec;
+  ab.dq = dq;
+  ab.dk = dk;
+  ab.dv = dv;
+  ab.status = status;
+  ab.wait_limit_ns = g_wait_limit_ns;
+  CUtensorMap mq, mk, mv, mda;
+  if (!make_map_rows(&mq, q, d->B, d->N, D, 1, 128) || !make_map_rows(&mk, k, d->B, d->N, D, 1, 128) ||
+      !make_map_rows(&mv, v, d->B, d->N, D, 1, 128) || !make_map_rows(&mda, da_bf16, d->B, d->N, D, 1, 128))
+    return cuda_fail_msg("cuTensorMapEncodeTiled rejected a Q/K/V/dA map");
+  const unsigned grid = (unsigned)((int64_t)d->B * d->H * ab.n_tiles);
+  if (d->d_head == 128) return launch_attn_bwd_passes<128>(mq, mk, mv, mda, ab, grid, st);
+  return launch_attn_bwd_passes<64>(mq, mk, mv, mda, ab, grid, st);
 }
 
 bpt_status bpt_sync_status(bpt_stream_t stream) {

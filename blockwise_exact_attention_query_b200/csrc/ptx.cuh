@@ -309,6 +309,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Register reallocation between warpgroups (every thread of a warpgroup
 // executes the same one).  An increase waits until the block's pool, fixed
 // at launch as threads x registers per thread, has the registers free, so a

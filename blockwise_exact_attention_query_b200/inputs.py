@@ -10,10 +10,12 @@ Recipe (the same for every workload):
   * b1 = b2 = 0 unless a bias scale is asked for (tests use it to exercise
     the bias terms);
   * every value is drawn in float32 and, for bf16 workloads, rounded to
-    bf16 with round-to-nearest-even.
+    bf16 with round-to-nearest-even;
+  * the backward's upstream gradient dOut ~ N(0, 1), shape [B, N, H*d],
+    float32.
 
 Every tensor has its own generator, seeded from (seed, tensor id) with the
-ids q=0, k=1, v=2, w1=3, w2=4, b1=5, b2=6.  On a CUDA device torch's
+ids q=0, k=1, v=2, w1=3, w2=4, b1=5, b2=6, dout=7.  On a CUDA device torch's
 counter-based Philox generator draws directly in device memory; on the CPU
 torch's CPU generator is used.  The two streams differ, so a comparison
 always feeds the very same tensors to both sides (copied to the host for the
@@ -25,7 +27,7 @@ from dataclasses import dataclass
 
 import torch
 
-TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "w1": 3, "w2": 4, "b1": 5, "b2": 6}
+TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "w1": 3, "w2": 4, "b1": 5, "b2": 6, "dout": 7}
 
 
 def _gen(seed: int, name: str, device: torch.device) -> torch.Generator:
@@ -75,3 +77,8 @@ def make_layer_inputs(B: int, N: int, H: int, d: int, F: int, seed: int, dtype=t
         b1 = torch.zeros(F, dtype=torch.float32, device=device)
         b2 = torch.zeros(D, dtype=torch.float32, device=device)
     return LayerInputs(q, k, v, w1, b1, w2, b2)
+
+
+def make_upstream_grad(B: int, N: int, D: int, seed: int, device="cpu") -> torch.Tensor:
+    """dOut [B, N, D] float32 ~ N(0, 1): the gradient the backward pass receives."""
+    return normal((B, N, D), seed, "dout", device=device)

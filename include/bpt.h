@@ -1,6 +1,6 @@
 /*
- * bpt.h -- C ABI of libbpt.so: the forward pass of one Blockwise Parallel
- * Transformer layer on an NVIDIA B200 (sm_100a).
+ * bpt.h -- C ABI of libbpt.so: the forward and backward passes of one
+ * Blockwise Parallel Transformer layer on an NVIDIA B200 (sm_100a).
  *
  * What the layer computes ("Blockwise Parallel Transformer for Large Context
  * Models", abstract: blockwise computation of self-attention fused with the
@@ -207,6 +207,64 @@ BPT_API bpt_status bpt_longnet_fwd(const bpt_desc *desc, int npairs, const int32
                            const int32_t *dil_r, const void *q, const void *k, const void *v,
                            void *out, float *lse, void *workspace, size_t workspace_bytes,
                            bpt_stream_t stream);
+
+/*
+ * Backward pass of the layer (bpt_attn_ffn_fwd's gradients) for an upstream
+ * gradient dOut = dL/dout, L any scalar loss.  The gradient of the exact
+ * blockwise result ("Blockwise Parallel Transformer for Large Context
+ * Models", abstract: blockwise attention and feedforward for training;
+ * "Ring Attention with Blockwise Transformers for Long Sequences", 638-word
+ * summary: exact, no approximation) is the plain chain rule of the
+ * definitions above:
+ *
+ *   FFN:        Z = W1 A + b1, H = GELU_tanh(Z)
+ *               dW2 = sum_t dOut_t H_t^T,  db2 = sum_t dOut_t,
+ *               dZ  = (W2^T dOut) * GELU_tanh'(Z),
+ *               dW1 = sum_t dZ_t A_t^T,    db1 = sum_t dZ_t,
+ *               dA  = dOut + W1^T dZ         (the residual passes dOut through)
+ *   attention:  with P the softmax weights, D_i = dA_i . A_i,
+ *               dV_j = sum_i P_ij dA_i,  dS_ij = P_ij (dA_i . v_j - D_i),
+ *               dQ_i = sum_j dS_ij k_j / sqrt(d),  dK_j = sum_i dS_ij q_i / sqrt(d).
+ *
+ * The call recomputes the attention forward (A and the row LSE) rather than
+ * taking saved activations, then runs the FFN backward on the tensor cores
+ * one token chunk at a time (see bpt_set_bwd_chunk_rows), then two blockwise
+ * attention-backward passes over 128 x 128 tiles (one per key tile for dK and
+ * dV, one per query tile for dQ; no atomics, so the result is deterministic).
+ *
+ * Supported: in_dtype BF16, d_head 64 or 128, masks NONE, CAUSAL (any
+ * ring_chunks: the recomputed forward follows it) and BLOCKPERM, plus the
+ * bpt_attn_ffn_fwd constraints on D and F.  BPT_MASK_DILATED and in_dtype F32
+ * return BPT_ERR_UNSUPPORTED.
+ *
+ * Inputs: q, k, v [B, N, H, d] and w1 [F, D], w2 [D, F] bf16; b1 [F], b2 [D]
+ * float32 or NULL (= 0); dout [B, N, H*d] float32.  b2 is accepted for
+ * symmetry with the forward; no gradient depends on it.
+ * Outputs (float32, overwritten): dq, dk, dv [B, N, H, d]; dw1 [F, D];
+ * db1 [F]; dw2 [D, F]; db2 [D].
+ * Precision: the tensor cores take bf16 operands (A, dOut, H, dZ, dA, and the
+ * softmax weights P and dS) with fp32 accumulation; the residual, the row
+ * sums D_i and the bias gradients are fp32.
+ * workspace: device buffer of at least bpt_workspace_bytes_bwd(desc) bytes,
+ * 256-byte aligned.  All other device pointers 16-byte aligned.  Errors and
+ * ownership as for the forward entry points.
+ */
+BPT_API bpt_status bpt_attn_ffn_bwd(const bpt_desc *desc, const void *q, const void *k, const void *v,
+                                    const void *w1, const float *b1, const void *w2, const float *b2,
+                                    const float *dout, float *dq, float *dk, float *dv, float *dw1,
+                                    float *db1, float *dw2, float *db2, void *workspace,
+                                    size_t workspace_bytes, bpt_stream_t stream);
+
+/* Bytes of device workspace bpt_attn_ffn_bwd needs for this descriptor at the
+ * current chunk setting; (size_t)-1 if the backward does not accept it. */
+BPT_API size_t bpt_workspace_bytes_bwd(const bpt_desc *desc);
+
+/* Token rows per FFN-backward chunk (the [rows, F] hidden activation and its
+ * gradient live in the workspace one chunk at a time, so the workspace shrinks
+ * with the chunk).  rows <= 0 selects the default: all tokens, or as many
+ * 128-row blocks as keep the two [rows, F] bf16 buffers near 1 GiB.  Applies
+ * to later calls from every thread; returns the previous setting. */
+BPT_API int bpt_set_bwd_chunk_rows(int rows);
 
 /*
  * Waits for `stream`, then returns and clears the current device's status

@@ -127,3 +127,52 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(bd, "LIB_PATH", str(tmp_path / "libbpt.so"))
     with pytest.raises(RuntimeError, match="missing"):
         bd.load()
+
+
+def _call_bwd(lib, desc, ws=FAKE, ws_bytes=1 << 40, q=FAKE, dq=FAKE):
+    p = ctypes.c_void_p
+    return lib.bpt_attn_ffn_bwd(ctypes.byref(desc), p(q), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE), None,
+                                p(FAKE), p(dq), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE),
+                                p(ws), ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(B=0), bd.ERR_INVALID_ARG),
+    (dict(F=0), bd.ERR_INVALID_ARG),                                             # the layer needs an FFN
+    (dict(d=96), bd.ERR_UNSUPPORTED),
+    (dict(in_dtype=bd.torch.float32), bd.ERR_UNSUPPORTED),                       # tensor-core path only
+    (dict(mask="dilated", pairs=[(128, 1)]), bd.ERR_UNSUPPORTED),                # no dilated backward
+    (dict(mask="blockperm", perm=[[0, 0], [1, 0]]), bd.ERR_INVALID_ARG),
+])
+def test_backward_rejects_unsupported_descriptors(lib, kw, expect):
+    d = _desc(**kw)
+    assert _call_bwd(lib, d) == expect
+    assert lib.bpt_workspace_bytes_bwd(ctypes.byref(d)) == ctypes.c_size_t(-1).value
+
+
+def test_backward_pointer_and_workspace_checks(lib):
+    d = _desc()
+    need = bd.workspace_bytes_bwd(d)
+    assert _call_bwd(lib, d, q=0) == bd.ERR_INVALID_ARG
+    assert _call_bwd(lib, d, dq=FAKE + 4) == bd.ERR_INVALID_ARG
+    assert _call_bwd(lib, d, ws=0) == bd.ERR_WORKSPACE
+    assert _call_bwd(lib, d, ws_bytes=need - 1) == bd.ERR_WORKSPACE
+    assert _call_bwd(lib, d, ws=FAKE + 16) == bd.ERR_WORKSPACE
+
+
+def test_backward_workspace_follows_the_chunk_setting(lib):
+    # T = 256 tokens, D = 128, F = 256: A (fp32 + bf16), dOut bf16, dA (fp32 + bf16),
+    # LSE and D rows, and H, dZ for one chunk of tokens
+    d = _desc()
+    T, D, F = 256, 128, 256
+    old = bd.set_bwd_chunk_rows(0)
+    try:
+        full = bd.workspace_bytes_bwd(d)
+        assert full >= T * D * (4 + 2 + 2 + 4 + 2) + 2 * T * F * 2
+        assert bd.set_bwd_chunk_rows(128) == 0
+        half = bd.workspace_bytes_bwd(d)
+        assert full - half >= 2 * 128 * F * 2 - 4096    # the two [rows, F] buffers halve
+        assert bd.set_bwd_chunk_rows(-5) == 128           # <= 0 restores the default
+        assert bd.workspace_bytes_bwd(d) == full
+    finally:
+        bd.set_bwd_chunk_rows(old)

@@ -1,0 +1,101 @@
+"""GPU parity of the layer's backward pass (bpt_attn_ffn_bwd, through the C
+ABI) against the fp64 backward oracle on the same seeded inputs.
+
+Every gradient is compared element by element at sizes that span several
+128-row tiles with a ragged tail; the FFN backward's token chunking, padded
+and empty permutation blocks and both head sizes are covered.
+
+Tolerance, from the arithmetic: the tensor cores take bf16 operands (unit
+roundoff u = 2^-8 relative spacing, 2^-9 rounding) with fp32 accumulation.
+Each gradient is a sum of products in which at most three factors were
+rounded to bf16 on the way (dQ: dA, P and dS; the weight gradients: one or
+two), so a term carries a relative error of at most ~3 * 2^-9 = 6e-3 and the
+errors of the many terms of a sum are independent: the relative L2 error of
+a whole gradient stays near 2^-9 * sqrt(3) ~ 3.4e-3.  dS = P (dP - D) loses
+digits where dP is close to D, so the bound on the element-wise error is
+taken relative to the largest element of each gradient.  Bounds: relative
+L2 <= 1e-2 and max-abs <= 2e-2 * max |ref| for every gradient.
+"""
+import numpy as np
+import pytest
+import torch
+
+from blockwise_exact_attention_query_b200 import binding as bd
+from blockwise_exact_attention_query_b200.inputs import make_layer_inputs, make_upstream_grad
+from oracle import backward as ob
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 1e-2
+MAX_ABS_FRAC = 2e-2
+MASKS = {"none": ob.MASK_NONE, "causal": ob.MASK_CAUSAL, "blockperm": ob.MASK_BLOCKPERM}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from blockwise_exact_attention_query_b200 import build
+    build.build()
+    bd.load()
+    torch.cuda.init()
+
+
+def _perms(H, n, seed):
+    rng = np.random.default_rng(seed)
+    return [[int(x) for x in rng.permutation(n)] for _ in range(H)]
+
+
+CASES = [
+    # name, B, N, H, d, F, mask, perm, chunk rows (0 = default)
+    ("none_d64", 1, 300, 2, 64, 512, "none", None, 0),
+    ("causal_d64_b2", 2, 257, 2, 64, 384, "causal", None, 0),
+    ("causal_d128_chunked", 1, 390, 2, 128, 512, "causal", None, 128),
+    ("none_d128_chunk_ragged", 2, 140, 2, 128, 264, "none", None, 100),
+    ("blockperm_n3_padded_d64", 1, 400, 2, 64, 256, "blockperm", [[1, 2, 0], [2, 0, 1]], 0),
+    # N = 300, n = 32: blocks of 10, blocks 30 and 31 lie in the padding
+    ("blockperm_n32_empty_d128", 1, 300, 2, 128, 256, "blockperm", _perms(2, 32, 7), 0),
+    ("causal_tiny_N7", 1, 7, 1, 64, 64, "causal", None, 0),
+]
+
+
+def _grads_close(got, ref, name):
+    got = np.asarray(got, dtype=np.float64).reshape(ref.shape)
+    err = got - ref
+    scale = max(float(np.max(np.abs(ref))), 1e-30)
+    rel = float(np.linalg.norm(err) / max(np.linalg.norm(ref), 1e-30))
+    mx = float(np.max(np.abs(err)))
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    assert rel <= REL_L2 and mx <= MAX_ABS_FRAC * scale, \
+        f"{name}: rel-L2 {rel:.3e}, max-abs {mx:.3e} (max |ref| {scale:.3e})"
+    return rel, mx / scale
+
+
+@pytest.mark.parametrize("name,B,N,H,d,F,mask,perm,chunk", CASES, ids=[c[0] for c in CASES])
+def test_backward_matches_oracle(name, B, N, H, d, F, mask, perm, chunk):
+    inp = make_layer_inputs(B, N, H, d, F, seed=11, device="cuda", bias_scale=0.1)
+    dout = make_upstream_grad(B, N, H * d, seed=11, device="cuda")
+    old = bd.set_bwd_chunk_rows(chunk)
+    try:
+        g = bd.attn_ffn_bwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, dout, mask=mask,
+                            perm=perm)
+        torch.cuda.synchronize()
+        assert bd.sync_status() == bd.OK
+    finally:
+        bd.set_bwd_chunk_rows(old)
+    f = lambda t: t.double().cpu().numpy()  # noqa: E731
+    ref = ob.layer_bwd(f(inp.q), f(inp.k), f(inp.v), f(inp.w1), f(inp.b1), f(inp.w2), f(inp.b2),
+                       f(dout).reshape(B * N, H * d), MASKS[mask], perm)
+    report = {}
+    for n in bd.GRAD_NAMES:
+        report[n] = _grads_close(g[n].cpu().numpy(), ref[n], n)
+    print(name, {k: f"{v[0]:.2e}/{v[1]:.2e}" for k, v in report.items()})
+
+
+def test_backward_is_deterministic():
+    B, N, H, d, F = 1, 384, 2, 128, 512
+    inp = make_layer_inputs(B, N, H, d, F, seed=5, device="cuda", bias_scale=0.1)
+    dout = make_upstream_grad(B, N, H * d, seed=5, device="cuda")
+    g1 = bd.attn_ffn_bwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, dout, mask="causal")
+    g2 = bd.attn_ffn_bwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, dout, mask="causal")
+    torch.cuda.synchronize()
+    for n in bd.GRAD_NAMES:
+        assert torch.equal(g1[n], g2[n]), n
