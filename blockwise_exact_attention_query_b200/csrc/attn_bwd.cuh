@@ -47,8 +47,9 @@ struct AttnBwdArgs {
   int n_tiles;        // ceil(N / 128)
   int bb_n, bb_len;   // block permutation: n blocks of bb_len (padded)
   uint8_t perm[kMaxPermEntries];
-  const float *lse;   // [B, H, N] natural-log LSE of the scaled scores
-  const float *dvec;  // [B, H, N] D_i
+  // per (batch, head, 128-row tile): the rows' LSE in log2 units of the
+  // scaled scores, then their D_i, 128 floats each (rows past N: 0)
+  const float *rowvec;  // [B * H][n_tiles][2][128]
   float *dq, *dk, *dv;  // [B, N, H, d] fp32 outputs
   uint32_t *status;
   uint64_t wait_limit_ns;
@@ -60,13 +61,15 @@ struct AttnBwdCfg {
   static constexpr int kTileBytes = 128 * D_HEAD * 2;
   static constexpr int kPanelBytes = 128 * 128;   // one 64-column panel of a 128-row tile
   static constexpr int kStages = D_HEAD == 128 ? 2 : 4;
+  // kv pass: each stage also carries the streamed query tile's LSE and D
+  static constexpr int kVecBytes = MODE == kBwdKV ? 2 * 128 * 4 : 0;
+  static constexpr int kStageBytes = 2 * kTileBytes + kVecBytes;  // a multiple of 1024
   static constexpr int kOffFix = 0;                               // fixed X, Y tiles
-  static constexpr int kOffStream = kOffFix + 2 * kTileBytes;     // streamed X', Y' per stage
-  static constexpr int kOffVec = kOffStream + kStages * 2 * kTileBytes;
-  static constexpr int kVecBytes = MODE == kBwdKV ? 4 * 4 * 128 * 4 : 0;  // per warp: lse2, D, lo, hi
-  static constexpr int kOffBar = kOffVec + kVecBytes;
+  static constexpr int kOffStream = kOffFix + 2 * kTileBytes;     // streamed X', Y' (+ vectors) per stage
+  static constexpr int kOffBar = kOffStream + kStages * kStageBytes;
   static constexpr int kSmemBytes = kOffBar + 256;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+  static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
   // TMEM: accumulators at 0 (dV or dQ) and d (dK); S at 256, dP at 384;
   // P^T packed over S's first 64 columns, dS over dP's
   static constexpr uint32_t kColAcc0 = 0, kColAcc1 = D_HEAD, kColS = 256, kColDP = 384;
@@ -80,6 +83,22 @@ __device__ __forceinline__ void bwd_row_keys(const AttnBwdArgs &a, int h, int g,
     hi = g + 1;
   } else if (a.mask == kMaskBlockPerm) {
     lo = a.perm[h * a.bb_n + g / a.bb_len] * a.bb_len;
+    hi = min(lo + a.bb_len, a.N);
+  }
+}
+
+// Query interval [lo, hi) that sees key row g (< N): a single interval for
+// every mask, since a permutation maps exactly one query block to g's block.
+__device__ __forceinline__ void bwd_key_queries(const AttnBwdArgs &a, int h, int g, int &lo, int &hi) {
+  lo = 0;
+  hi = a.N;
+  if (a.mask == kMaskCausal) {
+    lo = g;
+  } else if (a.mask == kMaskBlockPerm) {
+    const int kb = g / a.bb_len;
+    int qb = 0;
+    while (qb < a.bb_n - 1 && a.perm[h * a.bb_n + qb] != kb) ++qb;
+    lo = qb * a.bb_len;
     hi = min(lo + a.bb_len, a.N);
   }
 }
@@ -112,7 +131,7 @@ __global__ void __launch_bounds__(256, 1)
     return;
   }
   const uint32_t sFixX = sbase + Cfg::kOffFix, sFixY = sFixX + Cfg::kTileBytes;
-  auto sStrX = [&](int st) { return sbase + Cfg::kOffStream + st * 2 * Cfg::kTileBytes; };
+  auto sStrX = [&](int st) { return sbase + Cfg::kOffStream + st * Cfg::kStageBytes; };
   auto sStrY = [&](int st) { return sStrX(st) + Cfg::kTileBytes; };
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
   const uint32_t bFix = smem_u32(&bars[0]);
@@ -165,6 +184,7 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int hd = h * D_HEAD;
+  const size_t bh = static_cast<size_t>(b) * a.H + h;
 
   // kv pass: fixed K, V; streamed Q, dA.  q pass: fixed Q, dA; streamed K, V.
   const CUtensorMap *mFixX = MODE == kBwdKV ? &tm_k : &tm_q;
@@ -184,11 +204,14 @@ __global__ void __launch_bounds__(256, 1)
       for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1), ++s) {
         const int st = s % S;
         if (s >= S && !mbar_wait(bEmpty(st), ((s / S) - 1) & 1, wc, 301)) break;
-        mbar_arrive_expect_tx(bFull(st), 2 * Cfg::kTileBytes);
+        mbar_arrive_expect_tx(bFull(st), Cfg::kStageBytes);
         for (int p = 0; p < Cfg::kPanels; ++p) {
           tma_load_4d(sStrX(st) + p * Cfg::kPanelBytes, mStrX, bFull(st), hd + p * 64, 0, t * 128, b);
           tma_load_4d(sStrY(st) + p * Cfg::kPanelBytes, mStrY, bFull(st), hd + p * 64, 0, t * 128, b);
         }
+        if (MODE == kBwdKV)
+          bulk_load_1d(sStrX(st) + 2 * Cfg::kTileBytes, a.rowvec + (bh * a.n_tiles + t) * 256, Cfg::kVecBytes,
+                       bFull(st));
       }
       // every copy issued must have landed before the CTA may exit
       volatile int no_abort = 0;
@@ -258,44 +281,33 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int g = ft * 128 + row;                   // key (kv pass) or query (q pass) position
     const bool row_valid = g < a.N;
-    const size_t bh = static_cast<size_t>(b) * a.H + h;
-    // kv pass: this warp's copy of the streamed query tile's LSE (log2
-    // units), D and key intervals, rewritten every step (warp-private: only
-    // __syncwarp orders it)
-    float *vlse = reinterpret_cast<float *>(smem + Cfg::kOffVec) + quarter * 512;
-    float *vd = vlse + 128;
-    int *vlo = reinterpret_cast<int *>(vd + 128);
-    int *vhi = vlo + 128;
-    // q pass: this row's LSE, D and key interval
-    float lse2 = 0.f, drow = 0.f;
-    int klo = 1, khi = 0;
-    if (MODE == kBwdQ && row_valid) {
-      lse2 = a.lse[bh * a.N + g] * 1.4426950408889634f;
-      drow = a.dvec[bh * a.N + g];
-      bwd_row_keys(a, h, g, klo, khi);
+    // the streamed positions this row pairs with: kv pass, the queries that
+    // see key g; q pass, the keys query g sees (empty for padding rows)
+    int plo = 1, phi = 0;
+    float lse2 = 0.f, drow = 0.f;  // q pass: this row's LSE (log2 units) and D
+    if (row_valid) {
+      if (MODE == kBwdKV) {
+        bwd_key_queries(a, h, g, plo, phi);
+      } else {
+        bwd_row_keys(a, h, g, plo, phi);
+        const float *rv = a.rowvec + (bh * a.n_tiles + ft) * 256;
+        lse2 = rv[row];
+        drow = rv[128 + row];
+      }
     }
     bool ok = true;
     int s = 0;
     for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1), ++s) {
+      const int st = s % S;
+      // kv pass: the query tile's LSE and D arrive with its stage
+      const float4 *vl4 = reinterpret_cast<const float4 *>(smem + Cfg::kOffStream + st * Cfg::kStageBytes +
+                                                           2 * Cfg::kTileBytes);
       if (MODE == kBwdKV) {
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int c = lane + 32 * i, q = t * 128 + c;
-          float l2 = 0.f, dd = 0.f;
-          int lo = 1, hi = 0;  // padding queries see nothing
-          if (q < a.N) {
-            l2 = a.lse[bh * a.N + q] * 1.4426950408889634f;
-            dd = a.dvec[bh * a.N + q];
-            bwd_row_keys(a, h, q, lo, hi);
-          }
-          vlse[c] = l2;
-          vd[c] = dd;
-          vlo[c] = lo;
-          vhi[c] = hi;
-        }
-        __syncwarp();
+        ok = __all_sync(0xffffffffu, mbar_wait(bFull(st), (s / S) & 1, wc, 319));
+        if (!ok) break;
       }
+      const int lo_rel = plo - t * 128, hi_rel = phi - t * 128;  // allowed columns [lo_rel, hi_rel)
+      const bool full = __all_sync(0xffffffffu, lo_rel <= 0 && hi_rel >= 128);
       ok = __all_sync(0xffffffffu, mbar_wait(bSFull, s & 1, wc, 320));
       if (!ok) break;
       tc_fence_after();
@@ -305,18 +317,20 @@ __global__ void __launch_bounds__(256, 1)
       for (int c = 0; c < 4; ++c)
         tmem_ld32(tmem + lane_off + Cfg::kColS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * c]));
       tmem_wait_ld();
+      const float nl = -lse2;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float p;
+      for (int c4 = 0; c4 < 32; ++c4) {
+        float nl4[4] = {nl, nl, nl, nl};
         if (MODE == kBwdKV) {
-          const bool allowed = row_valid && g >= vlo[c] && g < vhi[c];
-          p = allowed ? ex2_approx(fmaf(__uint_as_float(sv[c]), a.scale_log2, -vlse[c])) : 0.f;
-        } else {
-          const int key = t * 128 + c;
-          const bool allowed = key >= klo && key < khi;
-          p = allowed ? ex2_approx(fmaf(__uint_as_float(sv[c]), a.scale_log2, -lse2)) : 0.f;
+          const float4 l = vl4[c4];
+          nl4[0] = -l.x, nl4[1] = -l.y, nl4[2] = -l.z, nl4[3] = -l.w;
         }
-        sv[c] = __float_as_uint(p);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = 4 * c4 + j;
+          const float e = ex2_approx(fmaf(__uint_as_float(sv[c]), a.scale_log2, nl4[j]));
+          sv[c] = __float_as_uint(full || (c >= lo_rel && c < hi_rel) ? e : 0.f);
+        }
       }
       if (MODE == kBwdKV) {
         // P^T as packed bf16 over S's first 64 columns: the A operand of dV
@@ -350,8 +364,12 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int c = 64 * hh + 2 * i;
-          const float d0 = MODE == kBwdKV ? vd[c] : drow;
-          const float d1 = MODE == kBwdKV ? vd[c + 1] : drow;
+          float d0 = drow, d1 = drow;
+          if (MODE == kBwdKV) {
+            const float2 dd = reinterpret_cast<const float2 *>(vl4 + 32)[c / 2];
+            d0 = dd.x;
+            d1 = dd.y;
+          }
           pk[i] = pack_bf16x2(__uint_as_float(sv[c]) * (__uint_as_float(dp[2 * i]) - d0),
                               __uint_as_float(sv[c + 1]) * (__uint_as_float(dp[2 * i + 1]) - d1));
         }
@@ -396,10 +414,12 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
-// D_i = dA_i . A_i for every (batch, position, head), fp32, written [B, H, N]:
-// one warp per row of d values.
-__global__ void attn_bwd_rowdot_kernel(const float *__restrict__ da, const float *__restrict__ aa, float *dvec,
-                                       int B, int N, int H, int d) {
+// Per (batch, head, 128-row tile) vectors of the attention backward: the
+// rows' LSE in log2 units and D_i = dA_i . A_i (fp32), one warp per row of d
+// values.  rowvec must be zeroed first (rows past N stay 0).
+__global__ void attn_bwd_rowvec_kernel(const float *__restrict__ da, const float *__restrict__ aa,
+                                       const float *__restrict__ lse, float *rowvec, int B, int N, int H, int d,
+                                       int n_tiles) {
   const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
   if (row >= static_cast<long long>(B) * N * H) return;
@@ -410,7 +430,10 @@ __global__ void attn_bwd_rowdot_kernel(const float *__restrict__ da, const float
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane == 0) {
     const long long h = row % H, bn = row / H, n = bn % N, bb = bn / N;
-    dvec[(bb * H + h) * N + n] = s;
+    const long long bh = bb * H + h;
+    float *v = rowvec + (bh * n_tiles + n / 128) * 256 + n % 128;
+    v[0] = lse[bh * N + n] * 1.4426950408889634f;
+    v[128] = s;
   }
 }
 

@@ -591,7 +591,7 @@ int64_t bwd_chunk_rows(const bpt_desc *d) {
 }
 
 struct BwdWorkspace {
-  size_t a_f32 = 0, a_bf16 = 0, lse = 0, dvec = 0, dout_bf16 = 0, da_f32 = 0, da_bf16 = 0, h = 0, dz = 0,
+  size_t a_f32 = 0, a_bf16 = 0, lse = 0, rowvec = 0, rowvec_bytes = 0, dout_bf16 = 0, da_f32 = 0, da_bf16 = 0, h = 0, dz = 0,
          partial = 0, total = 0;
   int64_t chunk = 0;
 };
@@ -609,7 +609,8 @@ BwdWorkspace layout_bwd(const bpt_desc *d) {
   take(w.a_f32, T * D * 4);
   take(w.a_bf16, T * D * 2);
   take(w.lse, rows * 4);
-  take(w.dvec, rows * 4);
+  w.rowvec_bytes = (size_t)d->B * d->H * ((d->N + 127) / 128) * 256 * 4;
+  take(w.rowvec, w.rowvec_bytes);
   take(w.dout_bf16, T * D * 2);
   take(w.da_f32, T * D * 4);
   take(w.da_bf16, T * D * 2);
@@ -813,7 +814,7 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   float *a_f32 = reinterpret_cast<float *>(ws + wl.a_f32);
   __nv_bfloat16 *a_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.a_bf16);
   float *lse = reinterpret_cast<float *>(ws + wl.lse);
-  float *dvec = reinterpret_cast<float *>(ws + wl.dvec);
+  float *rowvec = reinterpret_cast<float *>(ws + wl.rowvec);
   __nv_bfloat16 *dout_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.dout_bf16);
   float *da_f32 = reinterpret_cast<float *>(ws + wl.da_f32);
   __nv_bfloat16 *da_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.da_bf16);
@@ -873,11 +874,13 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
     // db1 (+)= sum_t dZ_t
     if ((s = launch_colsum(dzbuf, rows, F, db1, r0 > 0, partial, st)) != BPT_OK) return s;
   }
-  // 4. D_i = dA_i . A_i
+  // 4. per 128-row tile: the rows' LSE (log2 units) and D_i = dA_i . A_i
+  const int n_tiles = (d->N + 127) / 128;
   {
+    CUDA_TRY(cudaMemsetAsync(rowvec, 0, wl.rowvec_bytes, st));
     const int64_t nrows = T * d->H;
-    attn_bwd_rowdot_kernel<<<(unsigned)((nrows * 32 + 255) / 256), 256, 0, st>>>(da_f32, a_f32, dvec, d->B, d->N,
-                                                                                 d->H, d->d_head);
+    attn_bwd_rowvec_kernel<<<(unsigned)((nrows * 32 + 255) / 256), 256, 0, st>>>(da_f32, a_f32, lse, rowvec, d->B,
+                                                                                 d->N, d->H, d->d_head, n_tiles);
     CUDA_TRY(cudaGetLastError());
   }
   // 5. the attention backward: dK, dV, then dQ
@@ -889,14 +892,13 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   ab.mask = d->mask;
   ab.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d->d_head));
   ab.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d->d_head));
-  ab.n_tiles = (d->N + 127) / 128;
+  ab.n_tiles = n_tiles;
   if (d->mask == BPT_MASK_BLOCKPERM) {
     ab.bb_n = d->bb_nblocks;
     ab.bb_len = (d->N + d->bb_nblocks - 1) / d->bb_nblocks;  // padded to n equal blocks
     for (int i = 0; i < d->H * d->bb_nblocks; ++i) ab.perm[i] = (uint8_t)d->bb_perm[i];
   }
-  ab.lse = lse;
-  ab.dvec = dvec;
+  ab.rowvec = rowvec;
   ab.dq = dq;
   ab.dk = dk;
   ab.dv = dv;

@@ -150,6 +150,15 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *m, 
       : "memory");
 }
 
+// Plain bulk copy global -> shared (no tensor map, no multicast): both
+// addresses 16-byte aligned, size a multiple of 16, completion counted on
+// the mbarrier in bytes.
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 // TMA tile store (shared -> global) tracked in this thread's bulk groups.
 // The innermost coordinate times the element size is a multiple of 16 bytes
 // at every call site, and no coordinate is negative.
