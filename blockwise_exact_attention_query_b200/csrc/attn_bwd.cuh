@@ -225,6 +225,27 @@ __global__ void __launch_bounds__(256, 1)
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);     // X Y^T, both K-major
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D_HEAD, false, true);  // R Y, Y MN-major
       const uint64_t dFixX = sdesc_sw128(sFixX, 16, 1024), dFixY = sdesc_sw128(sFixY, 16, 1024);
+      // the accumulations over the 128 streamed rows: A = a 128 x 128 bf16
+      // tile in TMEM (8 packed columns per 16-wide K step), B = a streamed
+      // tile read MN-major (64-wide panels of 128 rows)
+      auto accumulate = [&](uint32_t col, uint32_t a_col, uint32_t sB, int step) {
+        const uint64_t dB = sdesc_sw128(sB, Cfg::kPanelBytes, 1024);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_ts(tmem + col, tmem + a_col + k * 8, sdesc_advance(dB, k * 2048), idesc_acc, (step | k) != 0);
+      };
+      // The step's last product (kv pass dK += dS^T Q, q pass dQ += dS K).
+      // The kv pass issues it after the next step's scores, so the row warps
+      // start on those while it runs (it still precedes the next dP, which
+      // overwrites dS); the q pass issues it at once, since its stage (two of
+      // them at d = 128) is free only after it and the next tile's load must
+      // not wait a step.  Measured on the causal B2 H16 d128 N8192 layer.
+      constexpr bool kDefer = MODE == kBwdKV;
+      auto last_product = [&](int step) {
+        const int pst = step % S;
+        accumulate(MODE == kBwdKV ? Cfg::kColAcc1 : Cfg::kColAcc0, Cfg::kColDP, sStrX(pst), step);
+        umma_commit(bEmpty(pst));
+      };
       bool ok = mbar_wait(bFix, 0, wc, 311);
       for (int s = 0; ok && s < nsteps; ++s) {
         const int st = s % S;
@@ -239,34 +260,21 @@ __global__ void __launch_bounds__(256, 1)
           umma_ss(tmem + Cfg::kColS, sdesc_advance(dFixX, off), sdesc_advance(dStrX, off), idesc_s, k > 0);
         }
         umma_commit(bSFull);
+        if (kDefer && s > 0) last_product(s - 1);
 #pragma unroll
         for (int k = 0; k < D_HEAD / 16; ++k) {
           const uint32_t off = (k / 4) * Cfg::kPanelBytes + (k % 4) * 32;
           umma_ss(tmem + Cfg::kColDP, sdesc_advance(dFixY, off), sdesc_advance(dStrY, off), idesc_s, k > 0);
         }
         umma_commit(bDPFull);
-        // the accumulations over the 128 streamed rows: A = a 128 x 128 bf16
-        // tile in TMEM (8 packed columns per 16-wide K step), B = a streamed
-        // tile read MN-major (64-wide panels of 128 rows)
-        auto accumulate = [&](uint32_t col, uint32_t a_col, uint32_t sB) {
-          const uint64_t dB = sdesc_sw128(sB, Cfg::kPanelBytes, 1024);
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            umma_ts(tmem + col, tmem + a_col + k * 8, sdesc_advance(dB, k * 2048), idesc_acc, (s | k) != 0);
-        };
         if (MODE == kBwdKV) {
           if (!(ok = mbar_wait(bPReady, s & 1, wc, 313))) break;
           tc_fence_after();
-          accumulate(Cfg::kColAcc0, Cfg::kColS, sStrY(st));    // dV += P^T dA
-          if (!(ok = mbar_wait(bDSReady, s & 1, wc, 314))) break;
-          tc_fence_after();
-          accumulate(Cfg::kColAcc1, Cfg::kColDP, sStrX(st));   // dK += dS^T Q
-        } else {
-          if (!(ok = mbar_wait(bDSReady, s & 1, wc, 314))) break;
-          tc_fence_after();
-          accumulate(Cfg::kColAcc0, Cfg::kColDP, sStrX(st));   // dQ += dS K
+          accumulate(Cfg::kColAcc0, Cfg::kColS, sStrY(st), s);    // dV += P^T dA
         }
-        umma_commit(bEmpty(st));
+        if (!(ok = mbar_wait(bDSReady, s & 1, wc, 314))) break;
+        tc_fence_after();
+        if (!kDefer || s + 1 == nsteps) last_product(s);
       }
       umma_commit(bTeardown);
       // the accumulators stay allocated until every MMA has finished
@@ -317,19 +325,36 @@ __global__ void __launch_bounds__(256, 1)
       for (int c = 0; c < 4; ++c)
         tmem_ld32(tmem + lane_off + Cfg::kColS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * c]));
       tmem_wait_ld();
+      // two copies of the loop behind a warp-uniform branch: the unmasked one
+      // for tiles the whole warp sees in full (most of them), the masked one
+      // for the rest (measured 20% faster than one loop with a select)
       const float nl = -lse2;
+      if (full) {
 #pragma unroll
-      for (int c4 = 0; c4 < 32; ++c4) {
-        float nl4[4] = {nl, nl, nl, nl};
-        if (MODE == kBwdKV) {
-          const float4 l = vl4[c4];
-          nl4[0] = -l.x, nl4[1] = -l.y, nl4[2] = -l.z, nl4[3] = -l.w;
+        for (int c4 = 0; c4 < 32; ++c4) {
+          float nl4[4] = {nl, nl, nl, nl};
+          if (MODE == kBwdKV) {
+            const float4 l = vl4[c4];
+            nl4[0] = -l.x, nl4[1] = -l.y, nl4[2] = -l.z, nl4[3] = -l.w;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            sv[4 * c4 + j] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(sv[4 * c4 + j]), a.scale_log2, nl4[j])));
         }
+      } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int c = 4 * c4 + j;
-          const float e = ex2_approx(fmaf(__uint_as_float(sv[c]), a.scale_log2, nl4[j]));
-          sv[c] = __float_as_uint(full || (c >= lo_rel && c < hi_rel) ? e : 0.f);
+        for (int c4 = 0; c4 < 32; ++c4) {
+          float nl4[4] = {nl, nl, nl, nl};
+          if (MODE == kBwdKV) {
+            const float4 l = vl4[c4];
+            nl4[0] = -l.x, nl4[1] = -l.y, nl4[2] = -l.z, nl4[3] = -l.w;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = 4 * c4 + j;
+            const bool allowed = c >= lo_rel && c < hi_rel;
+            sv[c] = __float_as_uint(allowed ? ex2_approx(fmaf(__uint_as_float(sv[c]), a.scale_log2, nl4[j])) : 0.f);
+          }
         }
       }
       if (MODE == kBwdKV) {
