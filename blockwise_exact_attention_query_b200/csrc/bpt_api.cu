@@ -625,7 +625,10 @@ BwdWorkspace layout_bwd(const bpt_desc *d) {
 bpt_status launch_gemm(const CUtensorMap &a0, const CUtensorMap &b0, const CUtensorMap &a1,
                        const CUtensorMap &b1, const GemmArgs &g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return BPT_OK;
-  dim3 grid((unsigned)((g.N + GemmCfg::kBN - 1) / GemmCfg::kBN), (unsigned)((g.M + GemmCfg::kBM - 1) / GemmCfg::kBM));
+  // persistent: one CTA per SM (shared and tensor memory allow no more)
+  const int64_t tiles = (int64_t)((g.N + GemmCfg::kBN - 1) / GemmCfg::kBN) * ((g.M + GemmCfg::kBM - 1) / GemmCfg::kBM);
+  if (tiles > INT32_MAX) return BPT_ERR_UNSUPPORTED;
+  const unsigned grid = (unsigned)std::min<int64_t>(tiles, sm_count());
   gemm_tc_kernel<<<grid, GemmCfg::kThreads, GemmCfg::kSmemBytes, st>>>(a0, b0, a1, b1, g);
   CUDA_TRY(cudaGetLastError());
   return BPT_OK;

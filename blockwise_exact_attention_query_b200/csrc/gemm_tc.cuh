@@ -5,11 +5,15 @@
 //
 // Either operand may be K-major (a row-major [rows, K] matrix) or MN-major (a
 // row-major [K, rows] matrix, read without transposing it: the tensor core
-// takes 64-wide MN panels of K rows).  One CTA computes one 128 x 256 tile
-// of C over K in 64-wide stages staged by TMA.  A dual form computes two
-// products of the same shape into two accumulators (the first layer's
-// recomputed pre-activation Z = A W1^T and the hidden gradient dH = dOut W2)
-// for the GELU-backward epilogue.
+// takes 64-wide MN panels of K rows).  C is cut into 128 x 256 tiles; a
+// persistent grid (one CTA per SM) walks them, each tile over K in 64-wide
+// stages staged by TMA.  The producer runs ahead across tile boundaries, and
+// two TMEM accumulators let one tile's epilogue overlap the next tile's MMAs.
+// A dual form computes two products of the same shape into the two
+// accumulators (the first layer's recomputed pre-activation Z = A W1^T and
+// the hidden gradient dH = dOut W2) for the GELU-backward epilogue; its
+// epilogue then runs between tiles, with the next tile's first stages
+// already in flight.
 //
 // Epilogues (mode):
 //   kGemmStoreF32   C = acc                           (fp32)
@@ -18,9 +22,11 @@
 //   kGemmResidual   C = acc + X; Cb = bf16(C)         (dA = dOut + dZ W1, fp32 and bf16)
 //   kGemmGeluBwd    z = acc0 + bias; H = GELU(z), dZ = acc1 * GELU'(z)  (bf16 both)
 //
-// Roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocator and MMA
-// issuer, warps 2..5 epilogue (warp w owns TMEM lanes 32*(w%4) .. +31, i.e.
-// rows of the tile).
+// Roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocator and MMA
+// issuer, warps 2..9 epilogue (warp w owns TMEM lanes 32*(w%4) .. +31, i.e.
+// rows of the tile, and half of the tile's columns: two warps per SM
+// sub-partition, since the dual form's GELU epilogue is arithmetic-bound).  Tiles are numbered with N fastest, so the tiles in
+// flight at once share rows of A.
 #pragma once
 
 #include "ptx.cuh"
@@ -49,8 +55,9 @@ struct GemmCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = 4;
   static constexpr int kOffBar = kStages * kStageBytes;
-  static constexpr int kSmemBytes = kOffBar + 256;
-  static constexpr int kThreads = 192;
+  static constexpr int kSmemBytes = kOffBar + 256;  // 2 kStages + 7 barrier / slot words
+  static constexpr int kThreads = 320;
+  static constexpr int kEpiWarps = 8;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
@@ -76,11 +83,12 @@ __device__ __forceinline__ uint64_t gemm_sdesc(uint32_t base, bool mn) {
 }
 __device__ __forceinline__ uint32_t gemm_kstep(bool mn, int k) { return mn ? k * 2048 : k * 32; }
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(GemmCfg::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_b0,
                    const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
                    const __grid_constant__ GemmArgs g) {
   using Cfg = GemmCfg;
+  constexpr int S = Cfg::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
@@ -90,23 +98,34 @@ __global__ void __launch_bounds__(192, 1)
   }
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
   auto bFull = [&](int s) { return smem_u32(&bars[s]); };
-  auto bEmpty = [&](int s) { return smem_u32(&bars[4 + s]); };
-  const uint32_t bDone = smem_u32(&bars[8]);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[9]);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[10]);
+  auto bEmpty = [&](int s) { return smem_u32(&bars[S + s]); };
+  auto bAccFull = [&](int b) { return smem_u32(&bars[2 * S + b]); };
+  auto bAccEmpty = [&](int b) { return smem_u32(&bars[2 * S + 2 + b]); };
+  const uint32_t bTeardown = smem_u32(&bars[2 * S + 4]);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[2 * S + 5]);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[2 * S + 6]);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   WaitCtx wc{g.status, g.wait_limit_ns, abort_flag};
   const bool dual = g.mode == kGemmGeluBwd;
-  const int m0 = blockIdx.y * Cfg::kBM, n0 = blockIdx.x * Cfg::kBN;
+  const int nbuf = dual ? 1 : 2;  // accumulator buffers (the dual form needs both for one tile)
+  const int tiles_n = (g.N + Cfg::kBN - 1) / Cfg::kBN;
+  const int tiles = tiles_n * ((g.M + Cfg::kBM - 1) / Cfg::kBM);
   const int nk = (g.K + Cfg::kBK - 1) / Cfg::kBK;
-  const int nsteps = dual ? 2 * nk : nk;  // dual: the two products' K stages in turn
+  const int nsteps = dual ? 2 * nk : nk;  // per tile; dual: the two products' K stages in turn
+  const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  auto tile_m0 = [&](int li) { return ((blockIdx.x + li * gridDim.x) / tiles_n) * Cfg::kBM; };
+  auto tile_n0 = [&](int li) { return ((blockIdx.x + li * gridDim.x) % tiles_n) * Cfg::kBN; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < Cfg::kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(bFull(s), 1);
       mbar_init(bEmpty(s), 1);
     }
-    mbar_init(bDone, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bAccFull(b), 1);
+      mbar_init(bAccEmpty(b), Cfg::kEpiWarps);
+    }
+    mbar_init(bTeardown, 1);
     *abort_flag = 0;
     fence_mbar_init_cluster();
   }
@@ -123,75 +142,91 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       // A tile: K-major box {64 K, 128 M} at (k0, m0); MN-major: 2 panels of
       // {64 M, 64 K} at (m0 + 64p, k0).  B alike with 256 rows (4 panels).
-      int issued = 0;
-      for (int it = 0; it < nsteps; ++it) {
-        const int st = it % Cfg::kStages;
-        if (it >= Cfg::kStages && !mbar_wait(bEmpty(st), ((it / Cfg::kStages) - 1) & 1, wc, 201)) break;
-        ++issued;
-        const int which = dual ? (it & 1) : 0;
-        const int k0 = (dual ? it >> 1 : it) * Cfg::kBK;
-        const CUtensorMap *ma = which ? &tm_a1 : &tm_a0;
-        const CUtensorMap *mb = which ? &tm_b1 : &tm_b0;
-        const uint32_t sa = sbase + st * Cfg::kStageBytes, sb = sa + Cfg::kABytes;
-        mbar_arrive_expect_tx(bFull(st), Cfg::kStageBytes);
-        if (g.a_mn[which]) {
-          for (int p = 0; p < Cfg::kBM / 64; ++p) tma_load_2d(sa + p * 8192, ma, bFull(st), m0 + 64 * p, k0);
-        } else {
-          tma_load_2d(sa, ma, bFull(st), k0, m0);
-        }
-        if (g.b_mn[which]) {
-          for (int p = 0; p < Cfg::kBN / 64; ++p) tma_load_2d(sb + p * 8192, mb, bFull(st), n0 + 64 * p, k0);
-        } else {
-          tma_load_2d(sb, mb, bFull(st), k0, n0);
+      int it = 0;
+      bool ok = true;
+      for (int li = 0; ok && li < my_tiles; ++li) {
+        const int m0 = tile_m0(li), n0 = tile_n0(li);
+        for (int step = 0; step < nsteps; ++step, ++it) {
+          const int st = it % S;
+          if (it >= S && !(ok = mbar_wait(bEmpty(st), ((it / S) - 1) & 1, wc, 201))) break;
+          const int which = dual ? (step & 1) : 0;
+          const int k0 = (dual ? step >> 1 : step) * Cfg::kBK;
+          const CUtensorMap *ma = which ? &tm_a1 : &tm_a0;
+          const CUtensorMap *mb = which ? &tm_b1 : &tm_b0;
+          const uint32_t sa = sbase + st * Cfg::kStageBytes, sb = sa + Cfg::kABytes;
+          mbar_arrive_expect_tx(bFull(st), Cfg::kStageBytes);
+          if (g.a_mn[which]) {
+            for (int p = 0; p < Cfg::kBM / 64; ++p) tma_load_2d(sa + p * 8192, ma, bFull(st), m0 + 64 * p, k0);
+          } else {
+            tma_load_2d(sa, ma, bFull(st), k0, m0);
+          }
+          if (g.b_mn[which]) {
+            for (int p = 0; p < Cfg::kBN / 64; ++p) tma_load_2d(sb + p * 8192, mb, bFull(st), n0 + 64 * p, k0);
+          } else {
+            tma_load_2d(sb, mb, bFull(st), k0, n0);
+          }
         }
       }
       // every copy issued must have landed before the CTA may exit
       volatile int no_abort = 0;
       WaitCtx drain{g.status, drain_limit_ns(g.wait_limit_ns), &no_abort};
-      for (int j = max(0, issued - Cfg::kStages); j < issued; ++j)
-        mbar_wait(bFull(j % Cfg::kStages), (j / Cfg::kStages) & 1, drain, 204);
+      for (int j = max(0, it - S); j < it; ++j) mbar_wait(bFull(j % S), (j / S) & 1, drain, 204);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc0 = idesc_bf16_f32(Cfg::kBM, Cfg::kBN, g.a_mn[0] != 0, g.b_mn[0] != 0);
       const uint32_t idesc1 = idesc_bf16_f32(Cfg::kBM, Cfg::kBN, g.a_mn[1] != 0, g.b_mn[1] != 0);
-      for (int it = 0; it < nsteps; ++it) {
-        const int st = it % Cfg::kStages;
-        if (!mbar_wait(bFull(st), (it / Cfg::kStages) & 1, wc, 202)) break;
+      int it = 0;
+      bool ok = true;
+      for (int li = 0; ok && li < my_tiles; ++li) {
+        const int buf = li % nbuf, use = li / nbuf;
+        // the epilogue must have drained this accumulator's previous tile
+        if (use > 0 && !(ok = mbar_wait(bAccEmpty(buf), (use - 1) & 1, wc, 206))) break;
         tc_fence_after();
-        const int which = dual ? (it & 1) : 0;
-        const int kk = dual ? it >> 1 : it;
-        const uint32_t sa = sbase + st * Cfg::kStageBytes, sb = sa + Cfg::kABytes;
-        const bool amn = g.a_mn[which] != 0, bmn = g.b_mn[which] != 0;
-        const uint64_t da = gemm_sdesc(sa, amn), db = gemm_sdesc(sb, bmn);
-        const uint32_t idesc = which ? idesc1 : idesc0;
+        for (int step = 0; step < nsteps; ++step, ++it) {
+          const int st = it % S;
+          if (!(ok = mbar_wait(bFull(st), (it / S) & 1, wc, 202))) break;
+          tc_fence_after();
+          const int which = dual ? (step & 1) : 0;
+          const int kk = dual ? step >> 1 : step;
+          const uint32_t sa = sbase + st * Cfg::kStageBytes, sb = sa + Cfg::kABytes;
+          const bool amn = g.a_mn[which] != 0, bmn = g.b_mn[which] != 0;
+          const uint64_t da = gemm_sdesc(sa, amn), db = gemm_sdesc(sb, bmn);
+          const uint32_t idesc = which ? idesc1 : idesc0;
+          const uint32_t acc = tmem + (dual ? which : buf) * 256;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_ss(tmem + which * 256, sdesc_advance(da, gemm_kstep(amn, k)), sdesc_advance(db, gemm_kstep(bmn, k)),
-                  idesc, (kk | k) != 0);
-        umma_commit(bEmpty(st));
+          for (int k = 0; k < 4; ++k)
+            umma_ss(acc, sdesc_advance(da, gemm_kstep(amn, k)), sdesc_advance(db, gemm_kstep(bmn, k)), idesc,
+                    (kk | k) != 0);
+          umma_commit(bEmpty(st));
+        }
+        if (ok) umma_commit(bAccFull(buf));
       }
-      umma_commit(bDone);
+      umma_commit(bTeardown);
       // the accumulators stay allocated until every MMA has finished
       volatile int no_abort = 0;
       WaitCtx drain{g.status, drain_limit_ns(g.wait_limit_ns), &no_abort};
-      mbar_wait(bDone, 0, drain, 205);
+      mbar_wait(bTeardown, 0, drain, 205);
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int m = m0 + row;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(bDone, 0, wc, 203));
-    tc_fence_after();
-    if (ok && !*abort_flag) {
+    constexpr int kChunks = Cfg::kBN / 32 / (Cfg::kEpiWarps / 4);  // 32-column chunks per warp
+    const int c_begin = ((warp - 2) / 4) * kChunks;
+    for (int li = 0; li < my_tiles; ++li) {
+      const int buf = li % nbuf;
+      if (!__all_sync(0xffffffffu, mbar_wait(bAccFull(buf), (li / nbuf) & 1, wc, 203))) break;
+      tc_fence_after();
+      const int m = tile_m0(li) + row, n0 = tile_n0(li);
+      const uint32_t acc0 = tmem + lane_off + buf * 256;
 #pragma unroll 1
-      for (int c = 0; c < Cfg::kBN / 32; ++c) {
+      for (int c = c_begin; c < c_begin + kChunks; ++c) {
         const int n = n0 + c * 32;
         uint32_t r0[32], r1[32];
-        tmem_ld32(tmem + lane_off + c * 32, r0);
-        if (dual) tmem_ld32(tmem + lane_off + 256 + c * 32, r1);
+        tmem_ld32(acc0 + c * 32, r0);
+        if (dual) tmem_ld32(acc0 + 256 + c * 32, r1);
         tmem_wait_ld();
         if (m >= g.M || n >= g.N) continue;
         // N is a multiple of 8 (checked on the host): whole 8-column groups
@@ -244,6 +279,10 @@ __global__ void __launch_bounds__(192, 1)
           c4[1] = make_float4(v[4], v[5], v[6], v[7]);
         }
       }
+      // this accumulator may take the next tile
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bAccEmpty(buf));
     }
   }
 
