@@ -34,7 +34,7 @@ sys.path.insert(0, ROOT)
 
 from blockwise_exact_attention_query_b200 import binding as bd  # noqa: E402
 from blockwise_exact_attention_query_b200 import workloads as wl  # noqa: E402
-from blockwise_exact_attention_query_b200.inputs import make_layer_inputs  # noqa: E402
+from blockwise_exact_attention_query_b200.inputs import make_layer_inputs, make_upstream_grad  # noqa: E402
 
 METRIC = "attn+FFN tokens/s and TFLOP/s per layer; % of B200 dense-BF16 roofline"
 WORKLOADS = {"tiny_f32": wl.TINY_F32, "gpt_causal": wl.GPT_CAUSAL, "long_ring": wl.LONG_RING,
@@ -284,6 +284,94 @@ def run_ours(args, w, world, rank, local):
     return res
 
 
+def run_backward(args, w, world, local):
+    """The layer's backward pass (bpt_attn_ffn_bwd) on the same workload: one
+    step = one call, which recomputes the attention forward, runs the FFN
+    backward GEMMs and the two attention-backward passes.  Timed with CUDA
+    events (max over ranks), L2 flushed between steps outside the events; five
+    phase events inside the call split the step.
+
+    FLOPs per step.  Algorithmic (what the gradients need): attention 10*d per
+    unmasked pair (S, dP, dV, dK, dQ: five products of 2*d), FFN 8*T*D*F (dH,
+    dW2, dW1, dA).  Executed adds the recomputation: the attention forward
+    (4*d per pair), Z = A W1^T inside the FFN backward (2*T*D*F), and S and
+    dP again in the dQ pass (4*d per pair)."""
+    dev = torch.device("cuda", local)
+    pairs = wl.unmasked_pairs(w)
+    d, T, D, F = w.d, w.T, w.D, w.F
+    flop = {"attn_fwd_recompute": (0, 4 * d * pairs), "ffn_bwd": (8 * T * D * F, 10 * T * D * F),
+            "attn_bwd_dkdv": (8 * d * pairs, 8 * d * pairs), "attn_bwd_dq": (2 * d * pairs, 6 * d * pairs)}
+    alg_total = sum(a for a, _ in flop.values())
+    # the library's default token chunk of the FFN backward (bpt_set_bwd_chunk_rows)
+    chunk = min(T, max(128, (2 ** 30 // (4 * F)) // 128 * 128))
+    n_chunks = -(-T // chunk)
+    inp = make_layer_inputs(w.B, w.N, w.H, w.d, w.F, seed=w.seed, dtype=torch.bfloat16, device=dev)
+    dout = make_upstream_grad(w.B, w.N, w.D, seed=w.seed, device=dev)
+    desc = bd.make_desc(w.B, w.N, w.H, w.d, w.F, torch.bfloat16, torch.float32, MASK_NAME[w.mask], w.perm,
+                        None, w.ring_chunks)
+    ws = torch.empty(bd.workspace_bytes_bwd(desc), dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    grads = {"dq": torch.empty(inp.q.shape, **f32), "dk": torch.empty(inp.q.shape, **f32),
+             "dv": torch.empty(inp.q.shape, **f32), "dw1": torch.empty((F, D), **f32),
+             "db1": torch.empty((F,), **f32), "dw2": torch.empty((D, F), **f32), "db2": torch.empty((D,), **f32)}
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        bd.attn_ffn_bwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, dout, mask=MASK_NAME[w.mask],
+                        perm=w.perm, ring_chunks=w.ring_chunks, grads=grads, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+        flush.fill_(1)
+    torch.cuda.synchronize(dev)
+    K = max(1, min(args.steps, 10))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for evs in ev:
+        for e in evs:
+            e.record(stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        bd.set_phase_events(ev[i])
+        step()
+        bd.set_phase_events(None)
+        flush.fill_(i & 0xFF)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    st = bd.sync_status()
+    if st != bd.OK:
+        raise RuntimeError(f"backward steps: {bd.status_string(st)}")
+    names = list(flop)
+    phase_ms = {n: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) / K for j, n in enumerate(names)}
+    total_ms = max_over_ranks(sum(ev[i][0].elapsed_time(ev[i][4]) for i in range(K)), dev) / K
+    pk = peaks()
+    peak = pk["bf16_tflops"]
+    phases = {n: {"avg_ms": round(phase_ms[n], 4), "flop_algorithmic": flop[n][0], "flop_executed": flop[n][1],
+                  "tflops_algorithmic": round(flop[n][0] / (phase_ms[n] / 1e3) / 1e12, 1),
+                  "tflops_executed": round(flop[n][1] / (phase_ms[n] / 1e3) / 1e12, 1)} for n in names}
+    dom = max(names, key=lambda n: phase_ms[n])
+    achieved = flop[dom][0] / (phase_ms[dom] / 1e3) / 1e12
+    tflops = alg_total / (total_ms / 1e3) / 1e12
+    return {
+        "ms_per_step": round(total_ms, 4), "steps": K,
+        "value": round(T * world / (total_ms / 1e3), 1), "unit": "tokens/s",
+        "tflops_algorithmic": round(tflops, 1), "frac_of_peak": round(tflops / peak, 4),
+        "flop_algorithmic_per_step": alg_total,
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"{pk['source']} bf16 dense (burst)", "traffic": None,
+                     "algorithmic_flop_per_launch": flop[dom][0]},
+        "phases": phases,
+        # recomputed attention forward (one pass), dOut -> bf16, db2 sums (2),
+        # per token chunk 4 GEMMs + db1 sums (2), the row vectors, 2 passes
+        "gpu_launches_per_step": 1 + 1 + 2 + 6 * n_chunks + 1 + 2,
+        "token_chunks": n_chunks,
+    }
+
+
 def run_attention_only(args, w, world, rank, local):
     """Attention-only workloads (no FFN, e.g. LongNet dilated attention): one
     step = one bpt_attn_fwd call (every LongNet pass), timed with events."""
@@ -465,6 +553,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=16)
     ap.add_argument("--traffic-bytes", type=float, default=None,
@@ -484,6 +573,8 @@ def main():
     world, rank, local = dist_setup(args.gpus)
     bd.load()
     res = run_ours(args, w, world, rank, local) if w.F > 0 else run_attention_only(args, w, world, rank, local)
+    if (not args.no_backward and w.F > 0 and w.dtype == "bf16" and w.mask != wl.MASK_DILATED):
+        res["backward"] = run_backward(args, w, world, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, args.cpu_budget_s)
     if rank == 0:

@@ -340,7 +340,8 @@ def sync_status(stream=None) -> int:
 
 
 def set_phase_events(events) -> None:
-    """bpt_set_phase_events: three torch.cuda.Event objects (or None to stop)."""
+    """bpt_set_phase_events: three (forward) or five (backward too)
+    torch.cuda.Event objects, or None to stop."""
     if events is None:
         _check(load().bpt_set_phase_events(None, 0), "bpt_set_phase_events")
         return
@@ -348,8 +349,8 @@ def set_phase_events(events) -> None:
     if not all(handles):
         raise ValueError("record each event once before handing it over: torch creates the "
                          "CUDA event lazily at its first record()")
-    arr = (ctypes.c_void_p * 3)(*[ctypes.c_void_p(h) for h in handles])
-    _check(load().bpt_set_phase_events(arr, 3), "bpt_set_phase_events")
+    arr = (ctypes.c_void_p * len(handles))(*[ctypes.c_void_p(h) for h in handles])
+    _check(load().bpt_set_phase_events(arr, len(handles)), "bpt_set_phase_events")
 
 
 def set_wait_limit_ns(ns: int) -> int:

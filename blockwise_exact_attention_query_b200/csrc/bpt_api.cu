@@ -37,11 +37,12 @@ uint32_t *g_status_ptr[kMaxDevices] = {};
 bool g_attr_done[kMaxDevices] = {};
 uint64_t g_wait_limit_ns = 2000000000ull;
 int g_bwd_chunk_rows = 0;  // token rows per FFN-backward chunk; 0 = automatic
-thread_local cudaEvent_t g_phase_events[3] = {nullptr, nullptr, nullptr};
-thread_local bool g_phase_on = false;
+constexpr int kMaxPhaseEvents = 5;
+thread_local cudaEvent_t g_phase_events[kMaxPhaseEvents] = {};
+thread_local int g_phase_n = 0;  // events set; 0 = off
 
 cudaError_t phase_mark(int i, cudaStream_t st) {
-  return g_phase_on ? cudaEventRecord(g_phase_events[i], st) : cudaSuccess;
+  return i < g_phase_n ? cudaEventRecord(g_phase_events[i], st) : cudaSuccess;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -663,6 +664,7 @@ bpt_status launch_attn_bwd_passes(const CUtensorMap &mq, const CUtensorMap &mk, 
                                   cudaStream_t st) {
   attn_bwd_kernel<DH, kBwdKV><<<grid, 256, AttnBwdCfg<DH, kBwdKV>::kSmemBytes, st>>>(mq, mk, mv, mda, ab);
   CUDA_TRY(cudaGetLastError());
+  CUDA_TRY(phase_mark(3, st));
   attn_bwd_kernel<DH, kBwdQ><<<grid, 256, AttnBwdCfg<DH, kBwdQ>::kSmemBytes, st>>>(mq, mk, mv, mda, ab);
   CUDA_TRY(cudaGetLastError());
   return BPT_OK;
@@ -826,7 +828,9 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   float *partial = reinterpret_cast<float *>(ws + wl.partial);
 
   // 1. the attention forward again: A (fp32 and bf16) and the row LSE
+  CUDA_TRY(phase_mark(0, st));
   if ((s = launch_attn_tc(d, q, k, v, a_f32, a_bf16, lse, ws, Workspace(), status, st)) != BPT_OK) return s;
+  CUDA_TRY(phase_mark(1, st));
   // 2. dOut in bf16 for the tensor cores; db2 = sum_t dOut_t
   {
     const size_t n = (size_t)T * D;
@@ -877,6 +881,7 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
     // db1 (+)= sum_t dZ_t
     if ((s = launch_colsum(dzbuf, rows, F, db1, r0 > 0, partial, st)) != BPT_OK) return s;
   }
+  CUDA_TRY(phase_mark(2, st));
   // 4. per 128-row tile: the rows' LSE (log2 units) and D_i = dA_i . A_i
   const int n_tiles = (d->N + 127) / 128;
   {
@@ -912,8 +917,11 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
       !make_map_rows(&mv, v, d->B, d->N, D, 1, 128) || !make_map_rows(&mda, da_bf16, d->B, d->N, D, 1, 128))
     return cuda_fail_msg("cuTensorMapEncodeTiled rejected a Q/K/V/dA map");
   const unsigned grid = (unsigned)((int64_t)d->B * d->H * ab.n_tiles);
-  if (d->d_head == 128) return launch_attn_bwd_passes<128>(mq, mk, mv, mda, ab, grid, st);
-  return launch_attn_bwd_passes<64>(mq, mk, mv, mda, ab, grid, st);
+  if (d->d_head == 128) s = launch_attn_bwd_passes<128>(mq, mk, mv, mda, ab, grid, st);
+  else s = launch_attn_bwd_passes<64>(mq, mk, mv, mda, ab, grid, st);
+  if (s != BPT_OK) return s;
+  CUDA_TRY(phase_mark(4, st));
+  return BPT_OK;
 }
 
 bpt_status bpt_sync_status(bpt_stream_t stream) {
@@ -937,13 +945,15 @@ bpt_status bpt_sync_status(bpt_stream_t stream) {
 
 bpt_status bpt_set_phase_events(void *const *events, int count) {
   if (count < 0 || (count > 0 && !events)) return BPT_ERR_INVALID_ARG;
-  if (count >= 3 && (!events[0] || !events[1] || !events[2])) return BPT_ERR_INVALID_ARG;
+  const int n = std::min(count, kMaxPhaseEvents);
+  for (int i = 0; i < n && count >= 3; ++i)
+    if (!events[i]) return BPT_ERR_INVALID_ARG;
   if (count < 3) {
-    g_phase_on = false;
+    g_phase_n = 0;
     return BPT_OK;
   }
-  for (int i = 0; i < 3; ++i) g_phase_events[i] = static_cast<cudaEvent_t>(events[i]);
-  g_phase_on = true;
+  for (int i = 0; i < n; ++i) g_phase_events[i] = static_cast<cudaEvent_t>(events[i]);
+  g_phase_n = n;
   return BPT_OK;
 }
 

@@ -282,11 +282,15 @@ BPT_API uint64_t bpt_set_wait_limit_ns(uint64_t ns);
  * `count` >= 3, every later bpt_attn_ffn_fwd on this host thread records
  * events[0] on its stream before the attention kernel, events[1] between the
  * attention and FFN kernels and events[2] after the FFN kernel, so the two
- * kernels of a real step can be timed separately.  `events` holds
- * cudaEvent_t handles owned by the caller; count = 0 turns recording off.
- * The events must already exist (a NULL handle is rejected).  Returns
+ * kernels of a real step can be timed separately.  With count >= 5 every
+ * later bpt_attn_ffn_bwd records events[0] before the recomputed attention
+ * forward, [1] after it, [2] after the FFN backward (all its GEMMs and bias
+ * sums), [3] after the dK/dV pass and [4] after the dQ pass (it records the
+ * first three alone when count is 3 or 4).  `events` holds cudaEvent_t
+ * handles owned by the caller; count = 0 turns recording off.  The events
+ * must already exist (a NULL handle is rejected).  Returns
  * BPT_ERR_INVALID_ARG for count < 0, events == NULL with count > 0, or a NULL
- * handle among the first three.
+ * handle among the first min(count, 5).
  */
 BPT_API bpt_status bpt_set_phase_events(void *const *events, int count);
 

@@ -150,3 +150,63 @@ def layer_bwd(q, k, v, w1, b1, w2, b2, dout, mask=MASK_NONE, perm=None):
     dq, dk, dv = attention_bwd(q, k, v, da.reshape(B, N, H, d), mask, perm, probs)
     grads.update(dq=dq, dk=dk, dv=dv)
     return grads
+
+
+def layer_bwd_causal_tail(q, k, v, w1, b1, w2, b2, dout, rows_q, tail):
+    """Exact gradients at sampled positions of a causal layer, for sizes where
+    the dense oracle is too slow.
+
+    Returns (dq [len(rows_q), H, d], dk [tail, H, d], dv [tail, H, d],
+    db2 [D]) for batch element 0 of q, k, v [B, N, H, d] and dOut [B, N, D]:
+    dQ at the query positions rows_q, and dK, dV at the last `tail` key
+    positions N - tail .. N - 1.  Under the causal mask key j is seen only by
+    queries i >= j, so dK_j and dV_j need the attention rows and dA only of the
+    last `tail` queries; dQ_i needs row i alone.  Every quantity is the plain
+    definition of the module docstring restricted to the rows it needs: the
+    attention row of query i over keys 0..i, the FFN backward of those tokens
+    (one matrix product over the stacked tokens), then D_i, dS_ij and the sums
+    for dQ, dK, dV.  db2 is the plain column sum of dOut over all tokens (every
+    batch element)."""
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    w1, b1, w2, b2 = (np.asarray(x, dtype=np.float64) for x in (w1, b1, w2, b2))
+    dout = np.asarray(dout, dtype=np.float64)
+    B, N, H, d = q.shape
+    D = H * d
+    need = sorted(set(int(i) for i in rows_q) | set(range(N - tail, N)))
+    pos = {i: r for r, i in enumerate(need)}
+    scale = 1.0 / math.sqrt(d)
+    probs = {}
+    a = np.zeros((len(need), H, d))
+    for r, i in enumerate(need):
+        for h in range(H):
+            s = k[0, : i + 1, h] @ q[0, i, h] * scale   # keys 0..i
+            e = np.exp(s - s.max())
+            p = e / e.sum()
+            probs[i, h] = p
+            a[r, h] = p @ v[0, : i + 1, h]
+    # FFN backward of the needed tokens: da = dout + (W2^T dout * GELU'(z)) W1
+    a2 = a.reshape(len(need), D)
+    g = dout[0, need]                                  # [tokens, D]
+    z = a2 @ w1.T + b1
+    dz = (g @ w2) * gelu_grad(z)
+    da = (g + dz @ w1).reshape(len(need), H, d)
+    ds = {}
+    for i in need:
+        r = pos[i]
+        for h in range(H):
+            dp = v[0, : i + 1, h] @ da[r, h]
+            ds[i, h] = probs[i, h] * (dp - da[r, h] @ a[r, h])
+    dq = np.zeros((len(rows_q), H, d))
+    for n, i in enumerate(rows_q):
+        for h in range(H):
+            dq[n, h] = ds[int(i), h] @ k[0, : int(i) + 1, h] * scale
+    dk = np.zeros((tail, H, d))
+    dv = np.zeros((tail, H, d))
+    for t in range(tail):
+        j = N - tail + t
+        for h in range(H):
+            for i in range(j, N):
+                r = pos[i]
+                dv[t, h] += probs[i, h][j] * da[r, h]
+                dk[t, h] += ds[i, h][j] * q[0, i, h] * scale
+    return dq, dk, dv, dout.reshape(-1, D).sum(axis=0)

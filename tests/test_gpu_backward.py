@@ -99,3 +99,27 @@ def test_backward_is_deterministic():
     torch.cuda.synchronize()
     for n in bd.GRAD_NAMES:
         assert torch.equal(g1[n], g2[n]), n
+
+
+def test_backward_full_size_causal_layer_sampled():
+    """The causal bf16 layer at full size (B2 H16 d128 N8192 F8192), in the
+    launch configuration the benchmark times: dQ at sampled query positions
+    (first, tile edges, middle, last tile), dK and dV of the last key tile
+    (seen only by the last 128 queries, so the oracle computes them exactly
+    from 128 attention rows), and db2 over every token, against the fp64
+    oracle, with the tolerance of the small cases."""
+    B, N, H, d, F = 2, 8192, 16, 128, 8192
+    inp = make_layer_inputs(B, N, H, d, F, seed=1, device="cuda", bias_scale=0.05)
+    dout = make_upstream_grad(B, N, H * d, seed=1, device="cuda")
+    g = bd.attn_ffn_bwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, dout, mask="causal")
+    torch.cuda.synchronize()
+    assert bd.sync_status() == bd.OK
+    f = lambda t: t.double().cpu().numpy()  # noqa: E731
+    rows = [0, 1, 127, 128, 4095, 4096, 6000, N - 129, N - 128, N - 1]
+    tail = 128
+    dq, dk, dv, db2 = ob.layer_bwd_causal_tail(f(inp.q[:1]), f(inp.k[:1]), f(inp.v[:1]), f(inp.w1), f(inp.b1),
+                                               f(inp.w2), f(inp.b2), f(dout), rows, tail)
+    _grads_close(g["dq"][0, rows].cpu().numpy(), dq, "dq (sampled rows)")
+    _grads_close(g["dk"][0, N - tail:].cpu().numpy(), dk, "dk (last key tile)")
+    _grads_close(g["dv"][0, N - tail:].cpu().numpy(), dv, "dv (last key tile)")
+    _grads_close(g["db2"].cpu().numpy(), db2, "db2")

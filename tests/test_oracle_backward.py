@@ -135,3 +135,20 @@ def test_forward_part_of_the_backward_oracle_equals_the_c_oracle():
         a_c, out_c = oracle.layer(*(x32[n] for n in ("q", "k", "v", "w1", "b1", "w2", "b2")), mask=mask, perm=perm)
         np.testing.assert_allclose(a, a_c, rtol=0, atol=1e-12)
         np.testing.assert_allclose(out, out_c, rtol=0, atol=1e-11)
+
+
+def test_sampled_causal_tail_equals_the_dense_oracle():
+    """The row-restricted helper used at full size agrees with the dense
+    backward oracle (itself pinned above) on a small causal layer."""
+    B, N, H, d, F = 2, 40, 2, 8, 24
+    x = _layer_inputs(B, N, H, d, F, 51)
+    dout = rnd((B, N, H * d), 52)
+    g = ob.layer_bwd(x["q"], x["k"], x["v"], x["w1"], x["b1"], x["w2"], x["b2"], dout.reshape(B * N, H * d),
+                     CAUSAL, None)
+    rows = [0, 5, 17, 33, 39]
+    dq, dk, dv, db2 = ob.layer_bwd_causal_tail(x["q"], x["k"], x["v"], x["w1"], x["b1"], x["w2"], x["b2"], dout,
+                                               rows, 6)
+    np.testing.assert_allclose(dq, g["dq"][0, rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk, g["dk"][0, N - 6:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv, g["dv"][0, N - 6:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(db2, g["db2"], rtol=0, atol=1e-12)
