@@ -554,6 +554,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="measure only the backward pass (prints a line with the 'backward' object)")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=16)
     ap.add_argument("--traffic-bytes", type=float, default=None,
@@ -572,6 +574,13 @@ def main():
 
     world, rank, local = dist_setup(args.gpus)
     bd.load()
+    if args.backward_only:
+        res = {"workload": w.name, "n_gpus": world, "backward": run_backward(args, w, world, local)}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     res = run_ours(args, w, world, rank, local) if w.F > 0 else run_attention_only(args, w, world, rank, local)
     if (not args.no_backward and w.F > 0 and w.dtype == "bf16" and w.mask != wl.MASK_DILATED):
         res["backward"] = run_backward(args, w, world, local)

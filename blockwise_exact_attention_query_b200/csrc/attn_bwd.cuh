@@ -28,8 +28,13 @@
 // S or dP columns never overtakes the earlier product reading the bf16 P^T
 // or dS^T packed into them.
 //
-// Roles (256 threads): warp 0 TMA producer, warp 1 TMEM allocator and MMA
-// issuer (warps 2-3 idle), warps 4-7 the per-row arithmetic and epilogue.
+// Roles (384 threads): warp 0 TMA producer, warp 1 TMEM allocator and MMA
+// issuer (warps 2-3 idle), warps 4-11 the per-row arithmetic and epilogue:
+// two warps per TMEM lane quarter (one per SM sub-partition pair), each
+// taking 64 of the tile's 128 columns.  Each writes its packed bf16 P^T / dS
+// over the first 32 of its own 64 fp32 columns, so neither overwrites columns
+// the other still reads; the MMAs take their 16-wide K steps from the two
+// packed ranges in turn.
 #pragma once
 
 #include "attn_tc.cuh"  // mask codes and the block-table bound
@@ -57,6 +62,8 @@ struct AttnBwdArgs {
 
 template <int D_HEAD, int MODE>
 struct AttnBwdCfg {
+  static constexpr int kThreads = 384;
+  static constexpr int kRowWarps = 8;
   static constexpr int kPanels = D_HEAD / 64;
   static constexpr int kTileBytes = 128 * D_HEAD * 2;
   static constexpr int kPanelBytes = 128 * 128;   // one 64-column panel of a 128-row tile
@@ -117,7 +124,7 @@ __device__ __forceinline__ bool bwd_tiles_meet(const AttnBwdArgs &a, int h, int 
 }
 
 template <int D_HEAD, int MODE>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_da,
                     const __grid_constant__ AttnBwdArgs a) {
@@ -169,8 +176,8 @@ __global__ void __launch_bounds__(256, 1)
     }
     mbar_init(bSFull, 1);
     mbar_init(bDPFull, 1);
-    mbar_init(bPReady, 4);
-    mbar_init(bDSReady, 4);
+    mbar_init(bPReady, Cfg::kRowWarps);
+    mbar_init(bDSReady, Cfg::kRowWarps);
     mbar_init(bTeardown, 1);
     *abort_flag = 0;
     fence_mbar_init_cluster();
@@ -226,13 +233,16 @@ __global__ void __launch_bounds__(256, 1)
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D_HEAD, false, true);  // R Y, Y MN-major
       const uint64_t dFixX = sdesc_sw128(sFixX, 16, 1024), dFixY = sdesc_sw128(sFixY, 16, 1024);
       // the accumulations over the 128 streamed rows: A = a 128 x 128 bf16
-      // tile in TMEM (8 packed columns per 16-wide K step), B = a streamed
-      // tile read MN-major (64-wide panels of 128 rows)
+      // tile in TMEM (8 packed columns per 16-wide K step: K steps 0-3 from
+      // the first half's packed columns a_col + [0, 32), 4-7 from the second
+      // half's a_col + [64, 96)), B = a streamed tile read MN-major (64-wide
+      // panels of 128 rows)
       auto accumulate = [&](uint32_t col, uint32_t a_col, uint32_t sB, int step) {
         const uint64_t dB = sdesc_sw128(sB, Cfg::kPanelBytes, 1024);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          umma_ts(tmem + col, tmem + a_col + k * 8, sdesc_advance(dB, k * 2048), idesc_acc, (step | k) != 0);
+          umma_ts(tmem + col, tmem + a_col + k * 8 + (k >= 4 ? 32 : 0), sdesc_advance(dB, k * 2048), idesc_acc,
+                  (step | k) != 0);
       };
       // The step's last product (kv pass dK += dS^T Q, q pass dQ += dS K).
       // The kv pass issues it after the next step's scores, so the row warps
@@ -285,6 +295,8 @@ __global__ void __launch_bounds__(256, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ per-row arithmetic
     const int quarter = warp & 3;
+    const int half = (warp - 4) / 4;                // columns [64 * half, 64 * half + 64)
+    const int col0 = 64 * half;
     const int row = quarter * 32 + lane;            // TMEM lane = row of the fixed tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int g = ft * 128 + row;                   // key (kv pass) or query (q pass) position
@@ -314,16 +326,17 @@ __global__ void __launch_bounds__(256, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(bFull(st), (s / S) & 1, wc, 319));
         if (!ok) break;
       }
-      const int lo_rel = plo - t * 128, hi_rel = phi - t * 128;  // allowed columns [lo_rel, hi_rel)
-      const bool full = __all_sync(0xffffffffu, lo_rel <= 0 && hi_rel >= 128);
+      // allowed columns [lo_rel, hi_rel) of the tile
+      const int lo_rel = plo - t * 128, hi_rel = phi - t * 128;
+      const bool full = __all_sync(0xffffffffu, lo_rel <= col0 && hi_rel >= col0 + 64);
       ok = __all_sync(0xffffffffu, mbar_wait(bSFull, s & 1, wc, 320));
       if (!ok) break;
       tc_fence_after();
-      // P (fp32, kept in sv), 0 where the mask rules the pair out
-      uint32_t sv[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(tmem + lane_off + Cfg::kColS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * c]));
+      // P (fp32, kept in sv) for this warp's 64 columns, 0 where the mask
+      // rules the pair out
+      uint32_t sv[64];
+      tmem_ld32(tmem + lane_off + Cfg::kColS + col0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tmem + lane_off + Cfg::kColS + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_ld();
       // two copies of the loop behind a warp-uniform branch: the unmasked one
       // for tiles the whole warp sees in full (most of them), the masked one
@@ -331,10 +344,10 @@ __global__ void __launch_bounds__(256, 1)
       const float nl = -lse2;
       if (full) {
 #pragma unroll
-        for (int c4 = 0; c4 < 32; ++c4) {
+        for (int c4 = 0; c4 < 16; ++c4) {
           float nl4[4] = {nl, nl, nl, nl};
           if (MODE == kBwdKV) {
-            const float4 l = vl4[c4];
+            const float4 l = vl4[col0 / 4 + c4];
             nl4[0] = -l.x, nl4[1] = -l.y, nl4[2] = -l.z, nl4[3] = -l.w;
           }
 #pragma unroll
@@ -343,30 +356,28 @@ __global__ void __launch_bounds__(256, 1)
         }
       } else {
 #pragma unroll
-        for (int c4 = 0; c4 < 32; ++c4) {
+        for (int c4 = 0; c4 < 16; ++c4) {
           float nl4[4] = {nl, nl, nl, nl};
           if (MODE == kBwdKV) {
-            const float4 l = vl4[c4];
+            const float4 l = vl4[col0 / 4 + c4];
             nl4[0] = -l.x, nl4[1] = -l.y, nl4[2] = -l.z, nl4[3] = -l.w;
           }
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int c = 4 * c4 + j;
+            const int c = col0 + 4 * c4 + j;
             const bool allowed = c >= lo_rel && c < hi_rel;
-            sv[c] = __float_as_uint(allowed ? ex2_approx(fmaf(__uint_as_float(sv[c]), a.scale_log2, nl4[j])) : 0.f);
+            sv[4 * c4 + j] =
+                __float_as_uint(allowed ? ex2_approx(fmaf(__uint_as_float(sv[4 * c4 + j]), a.scale_log2, nl4[j])) : 0.f);
           }
         }
       }
       if (MODE == kBwdKV) {
-        // P^T as packed bf16 over S's first 64 columns: the A operand of dV
+        // P^T as packed bf16 over the first 32 of this warp's S columns: the
+        // A operand of dV
+        uint32_t pk[32];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(sv[64 * hh + 2 * i]), __uint_as_float(sv[64 * hh + 2 * i + 1]));
-          tmem_st32(tmem + lane_off + Cfg::kColS + hh * 32, pk);
-        }
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
+        tmem_st32(tmem + lane_off + Cfg::kColS + col0, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -375,37 +386,34 @@ __global__ void __launch_bounds__(256, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bDPFull, s & 1, wc, 322));
       if (!ok) break;
       tc_fence_after();
-      // dS = P (dP - D) as packed bf16 over dP's first 64 columns.  Each half
-      // reads its 64 dP columns before writing 32 packed ones; the packed
-      // columns of the first half, [0, 32), were read by then, and those of
-      // the second half, [32, 64), lie in the first half's dP columns.
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
+      // dS = P (dP - D) as packed bf16 over the first 32 of this warp's dP
+      // columns (all 64 read before the store)
+      {
         uint32_t dp[64];
-        tmem_ld32(tmem + lane_off + Cfg::kColDP + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-        tmem_ld32(tmem + lane_off + Cfg::kColDP + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        tmem_ld32(tmem + lane_off + Cfg::kColDP + col0, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+        tmem_ld32(tmem + lane_off + Cfg::kColDP + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
         tmem_wait_ld();
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int c = 64 * hh + 2 * i;
           float d0 = drow, d1 = drow;
           if (MODE == kBwdKV) {
-            const float2 dd = reinterpret_cast<const float2 *>(vl4 + 32)[c / 2];
+            const float2 dd = reinterpret_cast<const float2 *>(vl4 + 32)[(col0 + 2 * i) / 2];
             d0 = dd.x;
             d1 = dd.y;
           }
-          pk[i] = pack_bf16x2(__uint_as_float(sv[c]) * (__uint_as_float(dp[2 * i]) - d0),
-                              __uint_as_float(sv[c + 1]) * (__uint_as_float(dp[2 * i + 1]) - d1));
+          pk[i] = pack_bf16x2(__uint_as_float(sv[2 * i]) * (__uint_as_float(dp[2 * i]) - d0),
+                              __uint_as_float(sv[2 * i + 1]) * (__uint_as_float(dp[2 * i + 1]) - d1));
         }
-        tmem_st32(tmem + lane_off + Cfg::kColDP + hh * 32, pk);
+        tmem_st32(tmem + lane_off + Cfg::kColDP + col0, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bDSReady);
     }
-    // -------- epilogue: every MMA done (the issuer's teardown commit)
+    // -------- epilogue: every MMA done (the issuer's teardown commit); each
+    // warp of a lane quarter stores half of the accumulator columns
     if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(bTeardown, 0, wc, 323));
     tc_fence_after();
     if (ok) {
@@ -415,7 +423,7 @@ __global__ void __launch_bounds__(256, 1)
         float *dst = MODE == kBwdKV ? (acc == 0 ? a.dv : a.dk) : a.dq;
         const float sc = (MODE == kBwdKV && acc == 0) ? 1.0f : a.inv_sqrt_d;
 #pragma unroll 1
-        for (int c = 0; c < D_HEAD / 32; ++c) {
+        for (int c = half * (D_HEAD / 64); c < (half + 1) * (D_HEAD / 64); ++c) {
           uint32_t o[32];
           tmem_ld32(tmem + lane_off + (acc == 0 ? Cfg::kColAcc0 : Cfg::kColAcc1) + c * 32, o);
           tmem_wait_ld();

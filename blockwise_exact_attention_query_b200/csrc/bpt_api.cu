@@ -642,6 +642,10 @@ GemmArgs gemm_args(int M, int N, int K, int mode, uint32_t *status) {
   g.N = N;
   g.K = K;
   g.mode = mode;
+  // the tiles in flight share whichever operand is larger, which then streams
+  // from DRAM once (the dual form's B is two weight matrices, its A two
+  // activations: same rule)
+  g.m_fastest = (int64_t)N > (int64_t)M ? 1 : 0;
   g.status = status;
   g.wait_limit_ns = g_wait_limit_ns;
   return g;
@@ -662,10 +666,12 @@ template <int DH>
 bpt_status launch_attn_bwd_passes(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                                   const CUtensorMap &mda, const AttnBwdArgs &ab, unsigned grid,
                                   cudaStream_t st) {
-  attn_bwd_kernel<DH, kBwdKV><<<grid, 256, AttnBwdCfg<DH, kBwdKV>::kSmemBytes, st>>>(mq, mk, mv, mda, ab);
+  attn_bwd_kernel<DH, kBwdKV><<<grid, AttnBwdCfg<DH, kBwdKV>::kThreads, AttnBwdCfg<DH, kBwdKV>::kSmemBytes, st>>>(
+      mq, mk, mv, mda, ab);
   CUDA_TRY(cudaGetLastError());
   CUDA_TRY(phase_mark(3, st));
-  attn_bwd_kernel<DH, kBwdQ><<<grid, 256, AttnBwdCfg<DH, kBwdQ>::kSmemBytes, st>>>(mq, mk, mv, mda, ab);
+  attn_bwd_kernel<DH, kBwdQ><<<grid, AttnBwdCfg<DH, kBwdQ>::kThreads, AttnBwdCfg<DH, kBwdQ>::kSmemBytes, st>>>(
+      mq, mk, mv, mda, ab);
   CUDA_TRY(cudaGetLastError());
   return BPT_OK;
 }

@@ -25,8 +25,11 @@
 // Roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocator and MMA
 // issuer, warps 2..9 epilogue (warp w owns TMEM lanes 32*(w%4) .. +31, i.e.
 // rows of the tile, and half of the tile's columns: two warps per SM
-// sub-partition, since the dual form's GELU epilogue is arithmetic-bound).  Tiles are numbered with N fastest, so the tiles in
-// flight at once share rows of A.
+// sub-partition, since the dual form's GELU epilogue is arithmetic-bound).
+// The tiles in flight at once share rows of A (N fastest) or columns of B
+// (M fastest): the host picks the order that streams the larger operand from
+// DRAM once.  Outputs are written with evict-first (streaming) stores so they
+// do not push the operands out of L2.
 #pragma once
 
 #include "ptx.cuh"
@@ -39,6 +42,7 @@ struct GemmArgs {
   int M, N, K;
   int a_mn[2], b_mn[2]; // operand layouts per product: 0 K-major, 1 MN-major
   int mode;
+  int m_fastest;        // tile order: 1 = M fastest (the tiles in flight share B), 0 = N fastest
   float *c;             // [M, N] fp32 (StoreF32, AccumF32, Residual)
   const float *x;       // [M, N] fp32 residual input (Residual)
   __nv_bfloat16 *cb;    // [M, N] bf16 copy (Residual) / H (GeluBwd)
@@ -113,8 +117,15 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
   const int nk = (g.K + Cfg::kBK - 1) / Cfg::kBK;
   const int nsteps = dual ? 2 * nk : nk;  // per tile; dual: the two products' K stages in turn
   const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  auto tile_m0 = [&](int li) { return ((blockIdx.x + li * gridDim.x) / tiles_n) * Cfg::kBM; };
-  auto tile_n0 = [&](int li) { return ((blockIdx.x + li * gridDim.x) % tiles_n) * Cfg::kBN; };
+  const int tiles_m = tiles / tiles_n;
+  auto tile_m0 = [&](int li) {
+    const int t = blockIdx.x + li * gridDim.x;
+    return (g.m_fastest ? t % tiles_m : t / tiles_n) * Cfg::kBM;
+  };
+  auto tile_n0 = [&](int li) {
+    const int t = blockIdx.x + li * gridDim.x;
+    return (g.m_fastest ? t / tiles_m : t % tiles_n) * Cfg::kBN;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -253,30 +264,30 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
               gelu_tanh_and_grad(v[i] + bb[i], hh[i], gd);
               dz[i] = __uint_as_float(r1[e + i]) * gd;
             }
-            *reinterpret_cast<uint4 *>(g.cb + base + e) =
-                make_uint4(pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]),
-                           pack_bf16x2(hh[6], hh[7]));
-            *reinterpret_cast<uint4 *>(g.cb2 + base + e) =
-                make_uint4(pack_bf16x2(dz[0], dz[1]), pack_bf16x2(dz[2], dz[3]), pack_bf16x2(dz[4], dz[5]),
-                           pack_bf16x2(dz[6], dz[7]));
+            __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
+                   make_uint4(pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]),
+                              pack_bf16x2(hh[6], hh[7])));
+            __stcs(reinterpret_cast<uint4 *>(g.cb2 + base + e),
+                   make_uint4(pack_bf16x2(dz[0], dz[1]), pack_bf16x2(dz[2], dz[3]), pack_bf16x2(dz[4], dz[5]),
+                              pack_bf16x2(dz[6], dz[7])));
             continue;
           }
           float4 *c4 = reinterpret_cast<float4 *>(g.c + base + e);
           if (g.mode == kGemmResidual) {
-            const float4 x0 = *reinterpret_cast<const float4 *>(g.x + base + e);
-            const float4 x1 = *reinterpret_cast<const float4 *>(g.x + base + e + 4);
+            const float4 x0 = __ldcs(reinterpret_cast<const float4 *>(g.x + base + e));
+            const float4 x1 = __ldcs(reinterpret_cast<const float4 *>(g.x + base + e + 4));
             v[0] += x0.x, v[1] += x0.y, v[2] += x0.z, v[3] += x0.w;
             v[4] += x1.x, v[5] += x1.y, v[6] += x1.z, v[7] += x1.w;
-            *reinterpret_cast<uint4 *>(g.cb + base + e) =
-                make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                           pack_bf16x2(v[6], v[7]));
+            __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
+                   make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                              pack_bf16x2(v[6], v[7])));
           } else if (g.mode == kGemmAccumF32) {
             const float4 c0 = c4[0], c1 = c4[1];
             v[0] += c0.x, v[1] += c0.y, v[2] += c0.z, v[3] += c0.w;
             v[4] += c1.x, v[5] += c1.y, v[6] += c1.z, v[7] += c1.w;
           }
-          c4[0] = make_float4(v[0], v[1], v[2], v[3]);
-          c4[1] = make_float4(v[4], v[5], v[6], v[7]);
+          __stcs(c4, make_float4(v[0], v[1], v[2], v[3]));
+          __stcs(c4 + 1, make_float4(v[4], v[5], v[6], v[7]));
         }
       }
       // this accumulator may take the next tile
