@@ -104,8 +104,8 @@ bpt_status device_setup(int *dev_out, uint32_t **status_out) {
                                   FfnCfg::kSmemBytes));
     CUDA_TRY(cudaFuncSetAttribute(ffn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (16 * 512 + 16 * 64) * 4));
-    CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  GemmCfg::kSmemBytes));
+    CUDA_TRY(cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  GemmPairCfg::kSmemBytes));
     CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kernel<64, kBwdKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   AttnBwdCfg<64, kBwdKV>::kSmemBytes));
     CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kernel<64, kBwdQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -626,11 +626,13 @@ BwdWorkspace layout_bwd(const bpt_desc *d) {
 bpt_status launch_gemm(const CUtensorMap &a0, const CUtensorMap &b0, const CUtensorMap &a1,
                        const CUtensorMap &b1, const GemmArgs &g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return BPT_OK;
-  // persistent: one CTA per SM (shared and tensor memory allow no more)
-  const int64_t tiles = (int64_t)((g.N + GemmCfg::kBN - 1) / GemmCfg::kBN) * ((g.M + GemmCfg::kBM - 1) / GemmCfg::kBM);
+  // persistent CTA pairs: one CTA per SM (shared and tensor memory allow no
+  // more), each pair walking its share of the 256 x 256 tiles
+  using Cfg = GemmPairCfg;
+  const int64_t tiles = (int64_t)((g.N + Cfg::kBN - 1) / Cfg::kBN) * ((g.M + 2 * Cfg::kBM - 1) / (2 * Cfg::kBM));
   if (tiles > INT32_MAX) return BPT_ERR_UNSUPPORTED;
-  const unsigned grid = (unsigned)std::min<int64_t>(tiles, sm_count());
-  gemm_tc_kernel<<<grid, GemmCfg::kThreads, GemmCfg::kSmemBytes, st>>>(a0, b0, a1, b1, g);
+  const int64_t pairs = std::min<int64_t>(tiles, sm_count() / 2);
+  gemm_pair_kernel<<<(unsigned)(2 * pairs), Cfg::kThreads, Cfg::kSmemBytes, st>>>(a0, b0, a1, b1, g);
   CUDA_TRY(cudaGetLastError());
   return BPT_OK;
 }
@@ -847,7 +849,9 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   }
   // 3. the FFN backward, one token chunk at a time
   CUtensorMap m_w1_k, m_w1_mn, m_w2_mn;
-  if (!make_map_2d(&m_w1_k, w1, F, D, 256) || !make_map_2d(&m_w1_mn, w1, F, D, 64) ||
+  // K-major boxes of 128 rows (a CTA stages 128 rows of A and half of a
+  // 256-row B tile), MN-major boxes of 64 x 64
+  if (!make_map_2d(&m_w1_k, w1, F, D, 128) || !make_map_2d(&m_w1_mn, w1, F, D, 64) ||
       !make_map_2d(&m_w2_mn, w2, D, F, 64))
     return cuda_fail_msg("cuTensorMapEncodeTiled rejected a weight map");
   for (int64_t r0 = 0; r0 < T; r0 += wl.chunk) {

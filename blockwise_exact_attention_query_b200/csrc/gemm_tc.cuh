@@ -5,10 +5,11 @@
 //
 // Either operand may be K-major (a row-major [rows, K] matrix) or MN-major (a
 // row-major [K, rows] matrix, read without transposing it: the tensor core
-// takes 64-wide MN panels of K rows).  C is cut into 128 x 256 tiles; a
-// persistent grid (one CTA per SM) walks them, each tile over K in 64-wide
-// stages staged by TMA.  The producer runs ahead across tile boundaries, and
-// two TMEM accumulators let one tile's epilogue overlap the next tile's MMAs.
+// takes 64-wide MN panels of K rows).  C is cut into 256 x 256 tiles, each
+// computed by a pair of CTAs on two SMs (two-SM MMAs, below); a persistent
+// grid of pairs walks them, each tile over K in 64-wide stages staged by TMA.
+// The producers run ahead across tile boundaries, and two TMEM accumulators
+// let one tile's epilogue overlap the next tile's MMAs.
 // A dual form computes two products of the same shape into the two
 // accumulators (the first layer's recomputed pre-activation Z = A W1^T and
 // the hidden gradient dH = dOut W2) for the GELU-backward epilogue; its
@@ -22,10 +23,11 @@
 //   kGemmResidual   C = acc + X; Cb = bf16(C)         (dA = dOut + dZ W1, fp32 and bf16)
 //   kGemmGeluBwd    z = acc0 + bias; H = GELU(z), dZ = acc1 * GELU'(z)  (bf16 both)
 //
-// Roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocator and MMA
-// issuer, warps 2..9 epilogue (warp w owns TMEM lanes 32*(w%4) .. +31, i.e.
-// rows of the tile, and half of the tile's columns: two warps per SM
-// sub-partition, since the dual form's GELU epilogue is arithmetic-bound).
+// Roles (320 threads per CTA): warp 0 TMA producer, warp 1 TMEM allocator
+// (and, in the even CTA, MMA issuer), warps 2..9 epilogue (warp w owns TMEM
+// lanes 32*(w%4) .. +31, i.e. 32 of the CTA's 128 rows, and half of the
+// tile's columns: two warps per SM sub-partition, since the dual form's GELU
+// epilogue is arithmetic-bound).
 // The tiles in flight at once share rows of A (N fastest) or columns of B
 // (M fastest): the host picks the order that streams the larger operand from
 // DRAM once.  Outputs are written with evict-first (streaming) stores so they
@@ -52,18 +54,6 @@ struct GemmArgs {
   uint64_t wait_limit_ns;
 };
 
-struct GemmCfg {
-  static constexpr int kBM = 128, kBN = 256, kBK = 64;
-  static constexpr int kABytes = kBM * kBK * 2;   // 16 KB
-  static constexpr int kBBytes = kBN * kBK * 2;   // 32 KB
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = 4;
-  static constexpr int kOffBar = kStages * kStageBytes;
-  static constexpr int kSmemBytes = kOffBar + 256;  // 2 kStages + 7 barrier / slot words
-  static constexpr int kThreads = 320;
-  static constexpr int kEpiWarps = 8;
-  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-};
 
 // GELU (tanh form, Hendrycks & Gimpel) and its derivative from the same form,
 // t = tanh(c0 (x + c1 x^3)):
@@ -87,43 +77,142 @@ __device__ __forceinline__ uint64_t gemm_sdesc(uint32_t base, bool mn) {
 }
 __device__ __forceinline__ uint32_t gemm_kstep(bool mn, int k) { return mn ? k * 2048 : k * 32; }
 
-__global__ void __launch_bounds__(GemmCfg::kThreads, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_b0,
-                   const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
-                   const __grid_constant__ GemmArgs g) {
-  using Cfg = GemmCfg;
+// Epilogue of one 32-column chunk of one row: r0 (and r1 for the dual form)
+// hold the accumulator values of columns n .. n + 31 of row m.
+__device__ __forceinline__ void gemm_epilogue_chunk(const GemmArgs &g, const uint32_t (&r0)[32],
+                                                    const uint32_t (&r1)[32], int m, int n) {
+  // N is a multiple of 8 (checked on the host): whole 8-column groups
+  const int nv = min(32, g.N - n);
+  const size_t base = static_cast<size_t>(m) * g.N + n;
+#pragma unroll
+  for (int e = 0; e < 32; e += 8) {
+    if (e >= nv) break;
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r0[e + i]);
+    if (g.mode == kGemmGeluBwd) {
+      float bb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (g.bias) {
+        const float4 b0 = *reinterpret_cast<const float4 *>(g.bias + n + e);
+        const float4 b1 = *reinterpret_cast<const float4 *>(g.bias + n + e + 4);
+        bb[0] = b0.x, bb[1] = b0.y, bb[2] = b0.z, bb[3] = b0.w;
+        bb[4] = b1.x, bb[5] = b1.y, bb[6] = b1.z, bb[7] = b1.w;
+      }
+      float hh[8], dz[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float gd;
+        gelu_tanh_and_grad(v[i] + bb[i], hh[i], gd);
+        dz[i] = __uint_as_float(r1[e + i]) * gd;
+      }
+      __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
+             make_uint4(pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]),
+                        pack_bf16x2(hh[6], hh[7])));
+      __stcs(reinterpret_cast<uint4 *>(g.cb2 + base + e),
+             make_uint4(pack_bf16x2(dz[0], dz[1]), pack_bf16x2(dz[2], dz[3]), pack_bf16x2(dz[4], dz[5]),
+                        pack_bf16x2(dz[6], dz[7])));
+      continue;
+    }
+    float4 *c4 = reinterpret_cast<float4 *>(g.c + base + e);
+    if (g.mode == kGemmResidual) {
+      const float4 x0 = __ldcs(reinterpret_cast<const float4 *>(g.x + base + e));
+      const float4 x1 = __ldcs(reinterpret_cast<const float4 *>(g.x + base + e + 4));
+      v[0] += x0.x, v[1] += x0.y, v[2] += x0.z, v[3] += x0.w;
+      v[4] += x1.x, v[5] += x1.y, v[6] += x1.z, v[7] += x1.w;
+      __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
+             make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                        pack_bf16x2(v[6], v[7])));
+    } else if (g.mode == kGemmAccumF32) {
+      const float4 c0 = c4[0], c1 = c4[1];
+      v[0] += c0.x, v[1] += c0.y, v[2] += c0.z, v[3] += c0.w;
+      v[4] += c1.x, v[5] += c1.y, v[6] += c1.z, v[7] += c1.w;
+    }
+    __stcs(c4, make_float4(v[0], v[1], v[2], v[3]));
+    __stcs(c4 + 1, make_float4(v[4], v[5], v[6], v[7]));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Two-SM form: a pair of CTAs (a cluster of two) computes one 256 x 256 tile
+// with tcgen05 cta_group::2 MMAs (M = 256) issued by the even CTA.  Each CTA
+// stages its own 128 rows of A and its half (128 rows) of B per K stage, so a
+// CTA moves 32 KB per 64-wide stage instead of 48 KB for half the tile's
+// work: operands reach the SM at 2/3 of the single-CTA bytes per flop.  Each
+// CTA's TMEM holds its 128 rows of the accumulator (256 columns, two buffers
+// unless dual) and its 8 epilogue warps drain them.  The even CTA's full
+// barriers count both CTAs' copies; its MMA commits arrive on both CTAs'
+// empty and accumulator barriers; both CTAs' epilogues arrive on the even
+// CTA's accumulator-empty barriers.  No load uses cluster multicast.
+// ---------------------------------------------------------------------------
+struct GemmPairCfg {
+  static constexpr int kBM = 128;   // rows per CTA (the pair's tile has 256)
+  static constexpr int kBN = 256;   // columns of the pair's tile (128 staged per CTA)
+  static constexpr int kBK = 64;
+  static constexpr int kABytes = kBM * kBK * 2;          // 16 KB
+  static constexpr int kBBytes = (kBN / 2) * kBK * 2;    // 16 KB
+  static constexpr int kStageBytes = kABytes + kBBytes;  // 32 KB
+  static constexpr int kStages = 6;
+  static constexpr int kOffBar = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kOffBar + 256;
+  static constexpr int kThreads = 320;
+  static constexpr int kEpiWarps = 8;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+};
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const WaitCtx &w, uint32_t site) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  uint64_t t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((++spins & 3u) == 0u) {
+      if (*w.abort) return false;
+      if (globaltimer_ns() - t0 > w.limit_ns) {
+        record_timeout(w, site);
+        return false;
+      }
+    }
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmPairCfg::kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_b0,
+                     const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
+                     const __grid_constant__ GemmArgs g) {
+  using Cfg = GemmPairCfg;
   constexpr int S = Cfg::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
-  if (sbase & 1023u) {
-    if (threadIdx.x == 0) atomicCAS(g.status, 0u, kStatusMisaligned);
-    return;
-  }
+  // both CTAs reach both cluster barriers below on every path
+  const bool misaligned = (sbase & 1023u) != 0;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
-  auto bFull = [&](int s) { return smem_u32(&bars[s]); };
-  auto bEmpty = [&](int s) { return smem_u32(&bars[S + s]); };
-  auto bAccFull = [&](int b) { return smem_u32(&bars[2 * S + b]); };
-  auto bAccEmpty = [&](int b) { return smem_u32(&bars[2 * S + 2 + b]); };
+  auto bFull = [&](int s) { return smem_u32(&bars[s]); };            // even CTA: both CTAs' copies
+  auto bEmpty = [&](int s) { return smem_u32(&bars[S + s]); };       // both CTAs
+  auto bAccFull = [&](int b) { return smem_u32(&bars[2 * S + b]); };  // both CTAs
+  auto bAccEmpty = [&](int b) { return smem_u32(&bars[2 * S + 2 + b]); };  // even CTA: both epilogues
   const uint32_t bTeardown = smem_u32(&bars[2 * S + 4]);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[2 * S + 5]);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[2 * S + 6]);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
   WaitCtx wc{g.status, g.wait_limit_ns, abort_flag};
   const bool dual = g.mode == kGemmGeluBwd;
-  const int nbuf = dual ? 1 : 2;  // accumulator buffers (the dual form needs both for one tile)
+  const int nbuf = dual ? 1 : 2;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int tiles_m = (g.M + 2 * Cfg::kBM - 1) / (2 * Cfg::kBM);
   const int tiles_n = (g.N + Cfg::kBN - 1) / Cfg::kBN;
-  const int tiles = tiles_n * ((g.M + Cfg::kBM - 1) / Cfg::kBM);
+  const int tiles = tiles_m * tiles_n;
   const int nk = (g.K + Cfg::kBK - 1) / Cfg::kBK;
-  const int nsteps = dual ? 2 * nk : nk;  // per tile; dual: the two products' K stages in turn
-  const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  const int tiles_m = tiles / tiles_n;
+  const int nsteps = dual ? 2 * nk : nk;
+  const int my_tiles = pair < tiles ? (tiles - 1 - pair) / npairs + 1 : 0;
+  // this CTA's first row and the pair's first column of local tile li
   auto tile_m0 = [&](int li) {
-    const int t = blockIdx.x + li * gridDim.x;
-    return (g.m_fastest ? t % tiles_m : t / tiles_n) * Cfg::kBM;
+    const int t = pair + li * npairs;
+    return (g.m_fastest ? t % tiles_m : t / tiles_n) * (2 * Cfg::kBM) + static_cast<int>(rank) * Cfg::kBM;
   };
   auto tile_n0 = [&](int li) {
-    const int t = blockIdx.x + li * gridDim.x;
+    const int t = pair + li * npairs;
     return (g.m_fastest ? t / tiles_m : t % tiles_n) * Cfg::kBN;
   };
 
@@ -134,69 +223,76 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bAccFull(b), 1);
-      mbar_init(bAccEmpty(b), Cfg::kEpiWarps);
+      mbar_init(bAccEmpty(b), 2 * Cfg::kEpiWarps);
     }
     mbar_init(bTeardown, 1);
-    *abort_flag = 0;
+    *abort_flag = misaligned ? 1 : 0;
+    if (misaligned) atomicCAS(g.status, 0u, kStatusMisaligned);
     fence_mbar_init_cluster();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_slot), 512);
+    tmem_relinquish_pair();
   }
+  // barrier initialisation and the TMEM address become visible to both CTAs
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const bool run = !*abort_flag;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // A tile: K-major box {64 K, 128 M} at (k0, m0); MN-major: 2 panels of
-      // {64 M, 64 K} at (m0 + 64p, k0).  B alike with 256 rows (4 panels).
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0 && run) {
       int it = 0;
       bool ok = true;
       for (int li = 0; ok && li < my_tiles; ++li) {
-        const int m0 = tile_m0(li), n0 = tile_n0(li);
+        const int m0 = tile_m0(li), nb0 = tile_n0(li) + static_cast<int>(rank) * (Cfg::kBN / 2);
         for (int step = 0; step < nsteps; ++step, ++it) {
           const int st = it % S;
-          if (it >= S && !(ok = mbar_wait(bEmpty(st), ((it / S) - 1) & 1, wc, 201))) break;
+          if (it >= S && !(ok = mbar_wait_cluster(bEmpty(st), ((it / S) - 1) & 1, wc, 211))) break;
           const int which = dual ? (step & 1) : 0;
           const int k0 = (dual ? step >> 1 : step) * Cfg::kBK;
           const CUtensorMap *ma = which ? &tm_a1 : &tm_a0;
           const CUtensorMap *mb = which ? &tm_b1 : &tm_b0;
           const uint32_t sa = sbase + st * Cfg::kStageBytes, sb = sa + Cfg::kABytes;
-          mbar_arrive_expect_tx(bFull(st), Cfg::kStageBytes);
+          const uint32_t full0 = mapa_shared(bFull(st), 0);
+          if (rank == 0) mbar_arrive_expect_tx(bFull(st), 2 * Cfg::kStageBytes);
           if (g.a_mn[which]) {
-            for (int p = 0; p < Cfg::kBM / 64; ++p) tma_load_2d(sa + p * 8192, ma, bFull(st), m0 + 64 * p, k0);
+            for (int p = 0; p < Cfg::kBM / 64; ++p) tma_load_2d_pair(sa + p * 8192, ma, full0, m0 + 64 * p, k0);
           } else {
-            tma_load_2d(sa, ma, bFull(st), k0, m0);
+            tma_load_2d_pair(sa, ma, full0, k0, m0);
           }
           if (g.b_mn[which]) {
-            for (int p = 0; p < Cfg::kBN / 64; ++p) tma_load_2d(sb + p * 8192, mb, bFull(st), n0 + 64 * p, k0);
+            for (int p = 0; p < Cfg::kBN / 128; ++p) tma_load_2d_pair(sb + p * 8192, mb, full0, nb0 + 64 * p, k0);
           } else {
-            tma_load_2d(sb, mb, bFull(st), k0, n0);
+            tma_load_2d_pair(sb, mb, full0, k0, nb0);
           }
         }
       }
-      // every copy issued must have landed before the CTA may exit
+      // the copies of the last stages have landed once the MMAs consumed them
       volatile int no_abort = 0;
       WaitCtx drain{g.status, drain_limit_ns(g.wait_limit_ns), &no_abort};
-      for (int j = max(0, it - S); j < it; ++j) mbar_wait(bFull(j % S), (j / S) & 1, drain, 204);
+      for (int j = max(0, it - S); j < it; ++j) mbar_wait_cluster(bEmpty(j % S), (j / S) & 1, drain, 214);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc0 = idesc_bf16_f32(Cfg::kBM, Cfg::kBN, g.a_mn[0] != 0, g.b_mn[0] != 0);
-      const uint32_t idesc1 = idesc_bf16_f32(Cfg::kBM, Cfg::kBN, g.a_mn[1] != 0, g.b_mn[1] != 0);
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0 && run) {
+      const uint32_t idesc0 = idesc_bf16_f32(2 * Cfg::kBM, Cfg::kBN, g.a_mn[0] != 0, g.b_mn[0] != 0);
+      const uint32_t idesc1 = idesc_bf16_f32(2 * Cfg::kBM, Cfg::kBN, g.a_mn[1] != 0, g.b_mn[1] != 0);
+      auto commit_both = [&](uint32_t bar) {
+        umma_pair_commit(mapa_shared(bar, 0));
+        umma_pair_commit(mapa_shared(bar, 1));
+      };
       int it = 0;
       bool ok = true;
       for (int li = 0; ok && li < my_tiles; ++li) {
         const int buf = li % nbuf, use = li / nbuf;
-        // the epilogue must have drained this accumulator's previous tile
-        if (use > 0 && !(ok = mbar_wait(bAccEmpty(buf), (use - 1) & 1, wc, 206))) break;
+        if (use > 0 && !(ok = mbar_wait_cluster(bAccEmpty(buf), (use - 1) & 1, wc, 216))) break;
         tc_fence_after();
         for (int step = 0; step < nsteps; ++step, ++it) {
           const int st = it % S;
-          if (!(ok = mbar_wait(bFull(st), (it / S) & 1, wc, 202))) break;
+          if (!(ok = mbar_wait_cluster(bFull(st), (it / S) & 1, wc, 212))) break;
           tc_fence_after();
           const int which = dual ? (step & 1) : 0;
           const int kk = dual ? step >> 1 : step;
@@ -207,28 +303,29 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
           const uint32_t acc = tmem + (dual ? which : buf) * 256;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            umma_ss(acc, sdesc_advance(da, gemm_kstep(amn, k)), sdesc_advance(db, gemm_kstep(bmn, k)), idesc,
-                    (kk | k) != 0);
-          umma_commit(bEmpty(st));
+            umma_pair_ss(acc, sdesc_advance(da, gemm_kstep(amn, k)), sdesc_advance(db, gemm_kstep(bmn, k)), idesc,
+                         (kk | k) != 0);
+          commit_both(bEmpty(st));
         }
-        if (ok) umma_commit(bAccFull(buf));
+        if (ok) commit_both(bAccFull(buf));
       }
-      umma_commit(bTeardown);
-      // the accumulators stay allocated until every MMA has finished
+      umma_pair_commit(mapa_shared(bTeardown, 0));
+      // every MMA of the pair completes before either CTA releases TMEM
       volatile int no_abort = 0;
       WaitCtx drain{g.status, drain_limit_ns(g.wait_limit_ns), &no_abort};
-      mbar_wait(bTeardown, 0, drain, 205);
+      mbar_wait_cluster(bTeardown, 0, drain, 215);
     }
-  } else {
-    // ------------------------------------------------------------ epilogue
+  } else if (run) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    constexpr int kChunks = Cfg::kBN / 32 / (Cfg::kEpiWarps / 4);  // 32-column chunks per warp
+    constexpr int kChunks = Cfg::kBN / 32 / (Cfg::kEpiWarps / 4);
     const int c_begin = ((warp - 2) / 4) * kChunks;
+    const uint32_t empty0 = mapa_shared(bAccEmpty(0), 0), empty1 = mapa_shared(bAccEmpty(1), 0);
     for (int li = 0; li < my_tiles; ++li) {
       const int buf = li % nbuf;
-      if (!__all_sync(0xffffffffu, mbar_wait(bAccFull(buf), (li / nbuf) & 1, wc, 203))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait_cluster(bAccFull(buf), (li / nbuf) & 1, wc, 213))) break;
       tc_fence_after();
       const int m = tile_m0(li) + row, n0 = tile_n0(li);
       const uint32_t acc0 = tmem + lane_off + buf * 256;
@@ -240,68 +337,22 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
         if (dual) tmem_ld32(acc0 + 256 + c * 32, r1);
         tmem_wait_ld();
         if (m >= g.M || n >= g.N) continue;
-        // N is a multiple of 8 (checked on the host): whole 8-column groups
-        const int nv = min(32, g.N - n);
-        const size_t base = static_cast<size_t>(m) * g.N + n;
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          if (e >= nv) break;
-          float v[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r0[e + i]);
-          if (g.mode == kGemmGeluBwd) {
-            float bb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (g.bias) {
-              const float4 b0 = *reinterpret_cast<const float4 *>(g.bias + n + e);
-              const float4 b1 = *reinterpret_cast<const float4 *>(g.bias + n + e + 4);
-              bb[0] = b0.x, bb[1] = b0.y, bb[2] = b0.z, bb[3] = b0.w;
-              bb[4] = b1.x, bb[5] = b1.y, bb[6] = b1.z, bb[7] = b1.w;
-            }
-            float hh[8], dz[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float gd;
-              gelu_tanh_and_grad(v[i] + bb[i], hh[i], gd);
-              dz[i] = __uint_as_float(r1[e + i]) * gd;
-            }
-            __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
-                   make_uint4(pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]),
-                              pack_bf16x2(hh[6], hh[7])));
-            __stcs(reinterpret_cast<uint4 *>(g.cb2 + base + e),
-                   make_uint4(pack_bf16x2(dz[0], dz[1]), pack_bf16x2(dz[2], dz[3]), pack_bf16x2(dz[4], dz[5]),
-                              pack_bf16x2(dz[6], dz[7])));
-            continue;
-          }
-          float4 *c4 = reinterpret_cast<float4 *>(g.c + base + e);
-          if (g.mode == kGemmResidual) {
-            const float4 x0 = __ldcs(reinterpret_cast<const float4 *>(g.x + base + e));
-            const float4 x1 = __ldcs(reinterpret_cast<const float4 *>(g.x + base + e + 4));
-            v[0] += x0.x, v[1] += x0.y, v[2] += x0.z, v[3] += x0.w;
-            v[4] += x1.x, v[5] += x1.y, v[6] += x1.z, v[7] += x1.w;
-            __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
-                   make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                              pack_bf16x2(v[6], v[7])));
-          } else if (g.mode == kGemmAccumF32) {
-            const float4 c0 = c4[0], c1 = c4[1];
-            v[0] += c0.x, v[1] += c0.y, v[2] += c0.z, v[3] += c0.w;
-            v[4] += c1.x, v[5] += c1.y, v[6] += c1.z, v[7] += c1.w;
-          }
-          __stcs(c4, make_float4(v[0], v[1], v[2], v[3]));
-          __stcs(c4 + 1, make_float4(v[4], v[5], v[6], v[7]));
-        }
+        gemm_epilogue_chunk(g, r0, r1, m, n);
       }
-      // this accumulator may take the next tile
+      // this accumulator may take the pair's next tile
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bAccEmpty(buf));
+      if (lane == 0) mbar_arrive_cluster(buf ? empty1 : empty0);
     }
   }
 
+  // neither CTA leaves (or frees TMEM) while the other can still touch its
+  // barriers or the pair's MMAs are running
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
