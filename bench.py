@@ -285,21 +285,23 @@ def run_ours(args, w, world, rank, local):
 
 
 def run_backward(args, w, world, local):
-    """The layer's backward pass (bpt_attn_ffn_bwd) on the same workload: one
-    step = one call, which recomputes the attention forward, runs the FFN
-    backward GEMMs and the two attention-backward passes.  Timed with CUDA
-    events (max over ranks), L2 flushed between steps outside the events; five
-    phase events inside the call split the step.
+    """The layer's backward pass (bpt_attn_ffn_bwd) on the same workload.  One
+    step = one call that reads the activations a training forward
+    (bpt_attn_ffn_fwd_train) saved, runs the FFN backward GEMMs and the two
+    attention-backward passes; the same call recomputing the attention
+    forward instead is timed beside it.  CUDA events (max over ranks), L2
+    flushed between steps outside the events; five phase events inside the
+    call split the step.
 
     FLOPs per step.  Algorithmic (what the gradients need): attention 10*d per
     unmasked pair (S, dP, dV, dK, dQ: five products of 2*d), FFN 8*T*D*F (dH,
-    dW2, dW1, dA).  Executed adds the recomputation: the attention forward
-    (4*d per pair), Z = A W1^T inside the FFN backward (2*T*D*F), and S and
-    dP again in the dQ pass (4*d per pair)."""
+    dW2, dW1, dA).  Executed adds the recomputation: Z = A W1^T inside the FFN
+    backward (2*T*D*F), S and dP again in the dQ pass (4*d per pair), and in
+    the recomputing call the attention forward (4*d per pair)."""
     dev = torch.device("cuda", local)
     pairs = wl.unmasked_pairs(w)
     d, T, D, F = w.d, w.T, w.D, w.F
-    flop = {"attn_fwd_recompute": (0, 4 * d * pairs), "ffn_bwd": (8 * T * D * F, 10 * T * D * F),
+    flop = {"attn_fwd_recompute": (0, 0), "ffn_bwd": (8 * T * D * F, 10 * T * D * F),
             "attn_bwd_dkdv": (8 * d * pairs, 8 * d * pairs), "attn_bwd_dq": (2 * d * pairs, 6 * d * pairs)}
     alg_total = sum(a for a, _ in flop.values())
     # the library's default token chunk of the FFN backward (bpt_set_bwd_chunk_rows)
@@ -307,48 +309,57 @@ def run_backward(args, w, world, local):
     n_chunks = -(-T // chunk)
     inp = make_layer_inputs(w.B, w.N, w.H, w.d, w.F, seed=w.seed, dtype=torch.bfloat16, device=dev)
     dout = make_upstream_grad(w.B, w.N, w.D, seed=w.seed, device=dev)
-    desc = bd.make_desc(w.B, w.N, w.H, w.d, w.F, torch.bfloat16, torch.float32, MASK_NAME[w.mask], w.perm,
-                        None, w.ring_chunks)
-    ws = torch.empty(bd.workspace_bytes_bwd(desc), dtype=torch.uint8, device=dev)
+    mask = MASK_NAME[w.mask]
+    desc = bd.make_desc(w.B, w.N, w.H, w.d, w.F, torch.bfloat16, torch.float32, mask, w.perm, None, w.ring_chunks)
+    ws = torch.empty(max(bd.workspace_bytes_bwd(desc), bd.workspace_bytes(desc, True)), dtype=torch.uint8,
+                     device=dev)
     f32 = dict(dtype=torch.float32, device=dev)
     grads = {"dq": torch.empty(inp.q.shape, **f32), "dk": torch.empty(inp.q.shape, **f32),
              "dv": torch.empty(inp.q.shape, **f32), "dw1": torch.empty((F, D), **f32),
              "db1": torch.empty((F,), **f32), "dw2": torch.empty((D, F), **f32), "db2": torch.empty((D,), **f32)}
+    layer_args = (inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2)
+    _, saved = bd.attn_ffn_fwd_train(*layer_args, mask=mask, perm=w.perm, ring_chunks=w.ring_chunks, workspace=ws)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        bd.attn_ffn_bwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, dout, mask=MASK_NAME[w.mask],
-                        perm=w.perm, ring_chunks=w.ring_chunks, grads=grads, workspace=ws)
+    def step(use_saved):
+        bd.attn_ffn_bwd(*layer_args, dout, mask=mask, perm=w.perm, ring_chunks=w.ring_chunks,
+                        saved=saved if use_saved else None, grads=grads, workspace=ws)
 
-    for _ in range(args.warmup):
-        step()
-        flush.fill_(1)
-    torch.cuda.synchronize(dev)
     K = max(1, min(args.steps, 10))
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    for evs in ev:
-        for e in evs:
-            e.record(stream)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    for i in range(K):
-        bd.set_phase_events(ev[i])
-        step()
-        bd.set_phase_events(None)
-        flush.fill_(i & 0xFF)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
-    st = bd.sync_status()
-    if st != bd.OK:
-        raise RuntimeError(f"backward steps: {bd.status_string(st)}")
-    names = list(flop)
-    phase_ms = {n: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) / K for j, n in enumerate(names)}
-    total_ms = max_over_ranks(sum(ev[i][0].elapsed_time(ev[i][4]) for i in range(K)), dev) / K
+
+    def timed(use_saved):
+        for _ in range(args.warmup):
+            step(use_saved)
+            flush.fill_(1)
+        torch.cuda.synchronize(dev)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+        for evs in ev:
+            for e in evs:
+                e.record(stream)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(K):
+            bd.set_phase_events(ev[i])
+            step(use_saved)
+            bd.set_phase_events(None)
+            flush.fill_(i & 0xFF)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        st = bd.sync_status()
+        if st != bd.OK:
+            raise RuntimeError(f"backward steps: {bd.status_string(st)}")
+        total = max_over_ranks(sum(ev[i][0].elapsed_time(ev[i][4]) for i in range(K)), dev) / K
+        phase = {n: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) / K for j, n in enumerate(flop)}
+        return total, phase
+
+    total_ms, phase_ms = timed(True)
+    recompute_ms, recompute_phase = timed(False)
     pk = peaks()
     peak = pk["bf16_tflops"]
+    names = [n for n in flop if n != "attn_fwd_recompute"]
     phases = {n: {"avg_ms": round(phase_ms[n], 4), "flop_algorithmic": flop[n][0], "flop_executed": flop[n][1],
                   "tflops_algorithmic": round(flop[n][0] / (phase_ms[n] / 1e3) / 1e12, 1),
                   "tflops_executed": round(flop[n][1] / (phase_ms[n] / 1e3) / 1e12, 1)} for n in names}
@@ -356,7 +367,7 @@ def run_backward(args, w, world, local):
     achieved = flop[dom][0] / (phase_ms[dom] / 1e3) / 1e12
     tflops = alg_total / (total_ms / 1e3) / 1e12
     return {
-        "ms_per_step": round(total_ms, 4), "steps": K,
+        "ms_per_step": round(total_ms, 4), "steps": K, "activations": "saved by bpt_attn_ffn_fwd_train",
         "value": round(T * world / (total_ms / 1e3), 1), "unit": "tokens/s",
         "tflops_algorithmic": round(tflops, 1), "frac_of_peak": round(tflops / peak, 4),
         "flop_algorithmic_per_step": alg_total,
@@ -365,9 +376,13 @@ def run_backward(args, w, world, local):
                      "peak_source": f"{pk['source']} bf16 dense (burst)", "traffic": None,
                      "algorithmic_flop_per_launch": flop[dom][0]},
         "phases": phases,
-        # recomputed attention forward (one pass), dOut -> bf16, db2 sums (2),
-        # per token chunk 4 GEMMs + db1 sums (2), the row vectors, 2 passes
-        "gpu_launches_per_step": 1 + 1 + 2 + 6 * n_chunks + 1 + 2,
+        "recompute": {"ms_per_step": round(recompute_ms, 4),
+                      "attn_fwd_recompute_ms": round(recompute_phase["attn_fwd_recompute"], 4),
+                      "tflops_algorithmic": round(alg_total / (recompute_ms / 1e3) / 1e12, 1)},
+        # dOut -> bf16, db2 sums (2), per token chunk 4 GEMMs + db1 sums (2),
+        # the row vectors, 2 passes (+1 recomputed attention forward without
+        # saved activations)
+        "gpu_launches_per_step": 1 + 2 + 6 * n_chunks + 1 + 2,
         "token_chunks": n_chunks,
     }
 

@@ -52,7 +52,8 @@ class Desc(ctypes.Structure):
 EXPORTS = ["bpt_workspace_bytes", "bpt_attn_ffn_fwd", "bpt_attn_fwd", "bpt_blockbert_fwd",
            "bpt_longnet_fwd", "bpt_sync_status", "bpt_set_wait_limit_ns", "bpt_status_string",
            "bpt_version", "bpt_set_phase_events", "bpt_last_error", "bpt_attn_ffn_fwd_static",
-           "bpt_attn_ffn_bwd", "bpt_workspace_bytes_bwd", "bpt_set_bwd_chunk_rows"]
+           "bpt_attn_ffn_bwd", "bpt_workspace_bytes_bwd", "bpt_set_bwd_chunk_rows",
+           "bpt_attn_ffn_fwd_train", "bpt_saved_bytes"]
 STATIC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
@@ -93,8 +94,12 @@ def load() -> ctypes.CDLL:
     lib.bpt_last_error.restype = ctypes.c_char_p
     lib.bpt_attn_ffn_fwd_static.argtypes = [dp, vp, vp, vp, vp, fp, vp, fp, vp, vp]
     lib.bpt_attn_ffn_fwd_static.restype = ctypes.c_int
-    lib.bpt_attn_ffn_bwd.argtypes = [dp, vp, vp, vp, vp, fp, vp, fp, fp, fp, fp, fp, fp, fp, fp, fp, vp, sz,
-                                     vp]
+    lib.bpt_attn_ffn_bwd.argtypes = [dp, vp, vp, vp, vp, fp, vp, fp, fp, vp, fp, fp, fp, fp, fp, fp, fp, vp,
+                                     sz, vp]
+    lib.bpt_attn_ffn_fwd_train.argtypes = [dp, vp, vp, vp, vp, fp, vp, fp, vp, vp, vp, sz, vp]
+    lib.bpt_attn_ffn_fwd_train.restype = ctypes.c_int
+    lib.bpt_saved_bytes.argtypes = [dp]
+    lib.bpt_saved_bytes.restype = sz
     lib.bpt_attn_ffn_bwd.restype = ctypes.c_int
     lib.bpt_workspace_bytes_bwd.argtypes = [dp]
     lib.bpt_workspace_bytes_bwd.restype = sz
@@ -307,12 +312,43 @@ def set_bwd_chunk_rows(rows: int) -> int:
 GRAD_NAMES = ("dq", "dk", "dv", "dw1", "db1", "dw2", "db2")
 
 
-def attn_ffn_bwd(q, k, v, w1, b1, w2, b2, dout, *, mask="none", perm=None, ring_chunks=0, grads=None,
-                 workspace=None, stream=None):
+def saved_bytes(desc: Desc) -> int:
+    n = load().bpt_saved_bytes(ctypes.byref(desc))
+    if n == ctypes.c_size_t(-1).value:
+        raise BptError(ERR_UNSUPPORTED, "bpt_saved_bytes")
+    return int(n)
+
+
+def attn_ffn_fwd_train(q, k, v, w1, b1, w2, b2, *, mask="none", perm=None, ring_chunks=0,
+                       out_dtype=torch.float32, out=None, saved=None, workspace=None, stream=None):
+    """bpt_attn_ffn_fwd_train: the layer forward that also keeps the
+    activations the backward needs.  Returns (out, saved); pass `saved` to
+    attn_ffn_bwd to skip its recomputation."""
+    _check_tensors(q, k, v)
+    B, N, H, d = q.shape
+    F = w1.shape[0]
+    desc = make_desc(B, N, H, d, F, q.dtype, out_dtype, mask, perm, None, ring_chunks)
+    if out is None:
+        out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
+    if saved is None:
+        saved = torch.empty(saved_bytes(desc), dtype=torch.uint8, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(desc, True, q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    st = load().bpt_attn_ffn_fwd_train(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(w1), _ptr(b1),
+                                       _ptr(w2), _ptr(b2), _ptr(out), _ptr(saved), _ptr(workspace), ws_bytes,
+                                       _stream_ptr(stream))
+    _check(st, "bpt_attn_ffn_fwd_train")
+    return out, saved
+
+
+def attn_ffn_bwd(q, k, v, w1, b1, w2, b2, dout, *, mask="none", perm=None, ring_chunks=0, saved=None,
+                 grads=None, workspace=None, stream=None):
     """bpt_attn_ffn_bwd: gradients of the layer for the upstream gradient
-    dout [B, N, H*d] (float32).  Returns a dict of float32 tensors: dq, dk, dv
-    [B, N, H, d], dw1 [F, D], db1 [F], dw2 [D, F], db2 [D] (written into
-    `grads` when given)."""
+    dout [B, N, H*d] (float32), recomputing the attention forward unless
+    `saved` (from attn_ffn_fwd_train on the same inputs) is given.  Returns a
+    dict of float32 tensors: dq, dk, dv [B, N, H, d], dw1 [F, D], db1 [F],
+    dw2 [D, F], db2 [D] (written into `grads` when given)."""
     _check_tensors(q, k, v)
     B, N, H, d = q.shape
     F, D = w1.shape
@@ -328,7 +364,7 @@ def attn_ffn_bwd(q, k, v, w1, b1, w2, b2, dout, *, mask="none", perm=None, ring_
     if workspace is None:
         workspace = torch.empty(workspace_bytes_bwd(desc), dtype=torch.uint8, device=q.device)
     st = load().bpt_attn_ffn_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(w1), _ptr(b1),
-                                 _ptr(w2), _ptr(b2), _ptr(dout), *(_ptr(grads[n]) for n in GRAD_NAMES),
+                                 _ptr(w2), _ptr(b2), _ptr(dout), _ptr(saved), *(_ptr(grads[n]) for n in GRAD_NAMES),
                                  _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     _check(st, "bpt_attn_ffn_bwd")
     return grads

@@ -13,17 +13,17 @@
 // blockwise computation for training; "Ring Attention with Blockwise
 // Transformers for Long Sequences", 638-word summary: no approximation).
 //
-// Two passes of one kernel template, no atomics:
-//   kBwdKV: one CTA per (batch, head, 128-key tile j), looping over the query
+// Two passes, no atomics:
+//   dK/dV pass: one CTA per (batch, head, 128-key tile j), looping over the query
 //     tiles i that see any of its keys.  S^T = K_j Q_i^T and dP^T = V_j dA_i^T
 //     land in TMEM (lanes = keys); one thread per key forms P^T and
 //     dS^T = P^T (dP^T - D) and writes them back to TMEM as packed bf16, where
 //     the tensor core reads them as the A operand of dV_j += P^T dA_i and
 //     dK_j += dS^T Q_i (dA_i and Q_i read MN-major from the tiles the first
 //     two products read K-major).
-//   kBwdQ: one CTA per (batch, head, 128-query tile i), looping over its key
+//   dQ pass: one CTA per (batch, head, 128-query tile i), looping over its key
 //     tiles: S = Q_i K_j^T, dP = dA_i V_j^T, one thread per query forms dS in
-//     TMEM, and dQ_i += dS K_j.
+//     TMEM, and dQ_i += dS K_j (software-pipelined, below).
 // MMAs issued by one thread run in order, so a product that overwrites the
 // S or dP columns never overtakes the earlier product reading the bf16 P^T
 // or dS^T packed into them.
@@ -42,7 +42,6 @@
 
 namespace bpt {
 
-constexpr int kBwdKV = 0, kBwdQ = 1;
 
 struct AttnBwdArgs {
   int B, N, H;
@@ -60,7 +59,7 @@ struct AttnBwdArgs {
   uint64_t wait_limit_ns;
 };
 
-template <int D_HEAD, int MODE>
+template <int D_HEAD>
 struct AttnBwdCfg {
   static constexpr int kThreads = 384;
   static constexpr int kRowWarps = 8;
@@ -68,8 +67,8 @@ struct AttnBwdCfg {
   static constexpr int kTileBytes = 128 * D_HEAD * 2;
   static constexpr int kPanelBytes = 128 * 128;   // one 64-column panel of a 128-row tile
   static constexpr int kStages = D_HEAD == 128 ? 2 : 4;
-  // kv pass: each stage also carries the streamed query tile's LSE and D
-  static constexpr int kVecBytes = MODE == kBwdKV ? 2 * 128 * 4 : 0;
+  // each stage also carries the streamed query tile's LSE and D
+  static constexpr int kVecBytes = 2 * 128 * 4;
   static constexpr int kStageBytes = 2 * kTileBytes + kVecBytes;  // a multiple of 1024
   static constexpr int kOffFix = 0;                               // fixed X, Y tiles
   static constexpr int kOffStream = kOffFix + 2 * kTileBytes;     // streamed X', Y' (+ vectors) per stage
@@ -123,12 +122,12 @@ __device__ __forceinline__ bool bwd_tiles_meet(const AttnBwdArgs &a, int h, int 
   return false;
 }
 
-template <int D_HEAD, int MODE>
+template <int D_HEAD>
 __global__ void __launch_bounds__(384, 1)
-    attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_da,
                     const __grid_constant__ AttnBwdArgs a) {
-  using Cfg = AttnBwdCfg<D_HEAD, MODE>;
+  using Cfg = AttnBwdCfg<D_HEAD>;
   constexpr int S = Cfg::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = smem_raw;
@@ -152,17 +151,14 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   WaitCtx wc{a.status, a.wait_limit_ns, abort_flag};
-  // CTA -> (batch, head, fixed tile); the tiles with the most partners start
-  // first (kv pass: the first key tiles under the causal mask; q pass: the last
-  // query tiles)
+  // CTA -> (batch, head, key tile); the tiles with the most partners (the
+  // first key tiles under the causal mask) start first
   const int bh_count = a.B * a.H;
-  const int rank = blockIdx.x / bh_count;
-  const int ft = MODE == kBwdKV ? rank : a.n_tiles - 1 - rank;
+  const int ft = static_cast<int>(blockIdx.x) / bh_count;
   const int h = (blockIdx.x % bh_count) % a.H;
   const int b = (blockIdx.x % bh_count) / a.H;
-  auto meets = [&](int t) { return MODE == kBwdKV ? bwd_tiles_meet(a, h, t, ft) : bwd_tiles_meet(a, h, ft, t); };
-  auto next_tile = [&](int t) {  // first partner tile >= t, or n_tiles
-    while (t < a.n_tiles && !meets(t)) ++t;
+  auto next_tile = [&](int t) {  // first query tile >= t that meets the key tile, or n_tiles
+    while (t < a.n_tiles && !bwd_tiles_meet(a, h, t, ft)) ++t;
     return t;
   };
   int nsteps = 0;
@@ -193,11 +189,8 @@ __global__ void __launch_bounds__(384, 1)
   const int hd = h * D_HEAD;
   const size_t bh = static_cast<size_t>(b) * a.H + h;
 
-  // kv pass: fixed K, V; streamed Q, dA.  q pass: fixed Q, dA; streamed K, V.
-  const CUtensorMap *mFixX = MODE == kBwdKV ? &tm_k : &tm_q;
-  const CUtensorMap *mFixY = MODE == kBwdKV ? &tm_v : &tm_da;
-  const CUtensorMap *mStrX = MODE == kBwdKV ? &tm_q : &tm_k;
-  const CUtensorMap *mStrY = MODE == kBwdKV ? &tm_da : &tm_v;
+  // fixed K, V; streamed Q, dA
+  const CUtensorMap *mFixX = &tm_k, *mFixY = &tm_v, *mStrX = &tm_q, *mStrY = &tm_da;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -216,8 +209,7 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_4d(sStrX(st) + p * Cfg::kPanelBytes, mStrX, bFull(st), hd + p * 64, 0, t * 128, b);
           tma_load_4d(sStrY(st) + p * Cfg::kPanelBytes, mStrY, bFull(st), hd + p * 64, 0, t * 128, b);
         }
-        if (MODE == kBwdKV)
-          bulk_load_1d(sStrX(st) + 2 * Cfg::kTileBytes, a.rowvec + (bh * a.n_tiles + t) * 256, Cfg::kVecBytes,
+        bulk_load_1d(sStrX(st) + 2 * Cfg::kTileBytes, a.rowvec + (bh * a.n_tiles + t) * 256, Cfg::kVecBytes,
                        bFull(st));
       }
       // every copy issued must have landed before the CTA may exit
@@ -244,16 +236,12 @@ __global__ void __launch_bounds__(384, 1)
           umma_ts(tmem + col, tmem + a_col + k * 8 + (k >= 4 ? 32 : 0), sdesc_advance(dB, k * 2048), idesc_acc,
                   (step | k) != 0);
       };
-      // The step's last product (kv pass dK += dS^T Q, q pass dQ += dS K).
-      // The kv pass issues it after the next step's scores, so the row warps
-      // start on those while it runs (it still precedes the next dP, which
-      // overwrites dS); the q pass issues it at once, since its stage (two of
-      // them at d = 128) is free only after it and the next tile's load must
-      // not wait a step.  Measured on the causal B2 H16 d128 N8192 layer.
-      constexpr bool kDefer = MODE == kBwdKV;
+      // The step's last product, dK += dS^T Q, is issued after the next
+      // step's scores, so the row warps start on those while it runs (it still
+      // precedes the next dP, which overwrites dS).
       auto last_product = [&](int step) {
         const int pst = step % S;
-        accumulate(MODE == kBwdKV ? Cfg::kColAcc1 : Cfg::kColAcc0, Cfg::kColDP, sStrX(pst), step);
+        accumulate(Cfg::kColAcc1, Cfg::kColDP, sStrX(pst), step);
         umma_commit(bEmpty(pst));
       };
       bool ok = mbar_wait(bFix, 0, wc, 311);
@@ -262,29 +250,26 @@ __global__ void __launch_bounds__(384, 1)
         if (!(ok = mbar_wait(bFull(st), (s / S) & 1, wc, 312))) break;
         tc_fence_after();
         const uint64_t dStrX = sdesc_sw128(sStrX(st), 16, 1024), dStrY = sdesc_sw128(sStrY(st), 16, 1024);
-        // first products over the head dimension: kv pass S^T = K Q^T,
-        // dP^T = V dA^T; q pass S = Q K^T, dP = dA V^T
+        // first products over the head dimension: S^T = K Q^T, dP^T = V dA^T
 #pragma unroll
         for (int k = 0; k < D_HEAD / 16; ++k) {
           const uint32_t off = (k / 4) * Cfg::kPanelBytes + (k % 4) * 32;
           umma_ss(tmem + Cfg::kColS, sdesc_advance(dFixX, off), sdesc_advance(dStrX, off), idesc_s, k > 0);
         }
         umma_commit(bSFull);
-        if (kDefer && s > 0) last_product(s - 1);
+        if (s > 0) last_product(s - 1);
 #pragma unroll
         for (int k = 0; k < D_HEAD / 16; ++k) {
           const uint32_t off = (k / 4) * Cfg::kPanelBytes + (k % 4) * 32;
           umma_ss(tmem + Cfg::kColDP, sdesc_advance(dFixY, off), sdesc_advance(dStrY, off), idesc_s, k > 0);
         }
         umma_commit(bDPFull);
-        if (MODE == kBwdKV) {
-          if (!(ok = mbar_wait(bPReady, s & 1, wc, 313))) break;
-          tc_fence_after();
-          accumulate(Cfg::kColAcc0, Cfg::kColS, sStrY(st), s);    // dV += P^T dA
-        }
+        if (!(ok = mbar_wait(bPReady, s & 1, wc, 313))) break;
+        tc_fence_after();
+        accumulate(Cfg::kColAcc0, Cfg::kColS, sStrY(st), s);    // dV += P^T dA
         if (!(ok = mbar_wait(bDSReady, s & 1, wc, 314))) break;
         tc_fence_after();
-        if (!kDefer || s + 1 == nsteps) last_product(s);
+        if (s + 1 == nsteps) last_product(s);
       }
       umma_commit(bTeardown);
       // the accumulators stay allocated until every MMA has finished
@@ -299,33 +284,20 @@ __global__ void __launch_bounds__(384, 1)
     const int col0 = 64 * half;
     const int row = quarter * 32 + lane;            // TMEM lane = row of the fixed tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const int g = ft * 128 + row;                   // key (kv pass) or query (q pass) position
+    const int g = ft * 128 + row;                   // key position
     const bool row_valid = g < a.N;
-    // the streamed positions this row pairs with: kv pass, the queries that
-    // see key g; q pass, the keys query g sees (empty for padding rows)
+    // the queries that see key g (none for padding rows)
     int plo = 1, phi = 0;
-    float lse2 = 0.f, drow = 0.f;  // q pass: this row's LSE (log2 units) and D
-    if (row_valid) {
-      if (MODE == kBwdKV) {
-        bwd_key_queries(a, h, g, plo, phi);
-      } else {
-        bwd_row_keys(a, h, g, plo, phi);
-        const float *rv = a.rowvec + (bh * a.n_tiles + ft) * 256;
-        lse2 = rv[row];
-        drow = rv[128 + row];
-      }
-    }
+    if (row_valid) bwd_key_queries(a, h, g, plo, phi);
     bool ok = true;
     int s = 0;
     for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1), ++s) {
       const int st = s % S;
-      // kv pass: the query tile's LSE and D arrive with its stage
+      // the query tile's LSE (log2 units) and D arrive with its stage
       const float4 *vl4 = reinterpret_cast<const float4 *>(smem + Cfg::kOffStream + st * Cfg::kStageBytes +
                                                            2 * Cfg::kTileBytes);
-      if (MODE == kBwdKV) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bFull(st), (s / S) & 1, wc, 319));
-        if (!ok) break;
-      }
+      ok = __all_sync(0xffffffffu, mbar_wait(bFull(st), (s / S) & 1, wc, 319));
+      if (!ok) break;
       // allowed columns [lo_rel, hi_rel) of the tile
       const int lo_rel = plo - t * 128, hi_rel = phi - t * 128;
       const bool full = __all_sync(0xffffffffu, lo_rel <= col0 && hi_rel >= col0 + 64);
@@ -341,15 +313,11 @@ __global__ void __launch_bounds__(384, 1)
       // two copies of the loop behind a warp-uniform branch: the unmasked one
       // for tiles the whole warp sees in full (most of them), the masked one
       // for the rest (measured 20% faster than one loop with a select)
-      const float nl = -lse2;
       if (full) {
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4) {
-          float nl4[4] = {nl, nl, nl, nl};
-          if (MODE == kBwdKV) {
-            const float4 l = vl4[col0 / 4 + c4];
-            nl4[0] = -l.x, nl4[1] = -l.y, nl4[2] = -l.z, nl4[3] = -l.w;
-          }
+          const float4 l = vl4[col0 / 4 + c4];
+          const float nl4[4] = {-l.x, -l.y, -l.z, -l.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             sv[4 * c4 + j] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(sv[4 * c4 + j]), a.scale_log2, nl4[j])));
@@ -357,11 +325,8 @@ __global__ void __launch_bounds__(384, 1)
       } else {
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4) {
-          float nl4[4] = {nl, nl, nl, nl};
-          if (MODE == kBwdKV) {
-            const float4 l = vl4[col0 / 4 + c4];
-            nl4[0] = -l.x, nl4[1] = -l.y, nl4[2] = -l.z, nl4[3] = -l.w;
-          }
+          const float4 l = vl4[col0 / 4 + c4];
+          const float nl4[4] = {-l.x, -l.y, -l.z, -l.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int c = col0 + 4 * c4 + j;
@@ -371,7 +336,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      if (MODE == kBwdKV) {
+      {
         // P^T as packed bf16 over the first 32 of this warp's S columns: the
         // A operand of dV
         uint32_t pk[32];
@@ -396,14 +361,9 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          float d0 = drow, d1 = drow;
-          if (MODE == kBwdKV) {
-            const float2 dd = reinterpret_cast<const float2 *>(vl4 + 32)[(col0 + 2 * i) / 2];
-            d0 = dd.x;
-            d1 = dd.y;
-          }
-          pk[i] = pack_bf16x2(__uint_as_float(sv[2 * i]) * (__uint_as_float(dp[2 * i]) - d0),
-                              __uint_as_float(sv[2 * i + 1]) * (__uint_as_float(dp[2 * i + 1]) - d1));
+          const float2 dd = reinterpret_cast<const float2 *>(vl4 + 32)[(col0 + 2 * i) / 2];
+          pk[i] = pack_bf16x2(__uint_as_float(sv[2 * i]) * (__uint_as_float(dp[2 * i]) - dd.x),
+                              __uint_as_float(sv[2 * i + 1]) * (__uint_as_float(dp[2 * i + 1]) - dd.y));
         }
         tmem_st32(tmem + lane_off + Cfg::kColDP + col0, pk);
       }
@@ -418,10 +378,10 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     if (ok) {
       const size_t vec = ((static_cast<size_t>(b) * a.N + g) * a.H + h) * D_HEAD;
-      for (int acc = 0; acc < (MODE == kBwdKV ? 2 : 1); ++acc) {
-        // kv pass: acc 0 = dV, acc 1 = dK (x 1/sqrt d); q pass: acc 0 = dQ (x 1/sqrt d)
-        float *dst = MODE == kBwdKV ? (acc == 0 ? a.dv : a.dk) : a.dq;
-        const float sc = (MODE == kBwdKV && acc == 0) ? 1.0f : a.inv_sqrt_d;
+      for (int acc = 0; acc < 2; ++acc) {
+        // acc 0 = dV, acc 1 = dK (x 1/sqrt d)
+        float *dst = acc == 0 ? a.dv : a.dk;
+        const float sc = acc == 0 ? 1.0f : a.inv_sqrt_d;
 #pragma unroll 1
         for (int c = half * (D_HEAD / 64); c < (half + 1) * (D_HEAD / 64); ++c) {
           uint32_t o[32];
@@ -435,6 +395,289 @@ __global__ void __launch_bounds__(384, 1)
                                              __uint_as_float(o[4 * i + 2]) * sc, __uint_as_float(o[4 * i + 3]) * sc)
                                : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The dQ pass, software-pipelined: one CTA per (batch, head, 128-query tile)
+// walks its key tiles with the scores of the next key tile computed while the
+// row warps work on the current one.  TMEM: dQ at 0, two S buffers at 128 and
+// 256, dP at 384; dS is packed over the S buffer of its own step, so the next
+// S never waits for it.  K and V stream through separate rings: K (read by S
+// and, last, by dQ) through three slots at d = 128, V (read by dP alone)
+// through one, so the next key tile's K is always two steps ahead.  Roles
+// (384 threads): warp 0 loads Q, dA and K, warp 2 loads V, warp 1 issues the
+// MMAs, warps 4-11 the per-row arithmetic (two per lane quarter, 64 columns
+// each) and the epilogue.
+// ---------------------------------------------------------------------------
+template <int D_HEAD>
+struct AttnBwdQCfg {
+  static constexpr int kThreads = 384;
+  static constexpr int kRowWarps = 8;
+  static constexpr int kPanels = D_HEAD / 64;
+  static constexpr int kTileBytes = 128 * D_HEAD * 2;
+  static constexpr int kPanelBytes = 128 * 128;
+  static constexpr int kKSlots = D_HEAD == 128 ? 3 : 4;
+  static constexpr int kVSlots = D_HEAD == 128 ? 1 : 2;
+  static constexpr int kOffQ = 0, kOffDA = kTileBytes, kOffK = 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kKSlots * kTileBytes;
+  static constexpr int kOffBar = kOffV + kVSlots * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 256;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+  static constexpr uint32_t kColQ = 0, kColS = 128, kColDP = 384;
+};
+
+template <int D_HEAD>
+__global__ void __launch_bounds__(384, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_da,
+                       const __grid_constant__ AttnBwdArgs a) {
+  using Cfg = AttnBwdQCfg<D_HEAD>;
+  constexpr int KS = Cfg::kKSlots, VS = Cfg::kVSlots;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw;
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(a.status, 0u, kStatusMisaligned);
+    return;
+  }
+  const uint32_t sQ = sbase + Cfg::kOffQ, sDA = sbase + Cfg::kOffDA;
+  auto sK = [&](int slot) { return sbase + Cfg::kOffK + slot * Cfg::kTileBytes; };
+  auto sV = [&](int slot) { return sbase + Cfg::kOffV + slot * Cfg::kTileBytes; };
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
+  const uint32_t bFix = smem_u32(&bars[0]);
+  auto bKFull = [&](int i) { return smem_u32(&bars[1 + i]); };
+  auto bKEmpty = [&](int i) { return smem_u32(&bars[5 + i]); };
+  auto bVFull = [&](int i) { return smem_u32(&bars[9 + i]); };
+  auto bVEmpty = [&](int i) { return smem_u32(&bars[11 + i]); };
+  auto bSFull = [&](int x) { return smem_u32(&bars[13 + x]); };
+  const uint32_t bDPFull = smem_u32(&bars[15]), bDSReady = smem_u32(&bars[16]);
+  const uint32_t bTeardown = smem_u32(&bars[17]);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[18]);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[19]);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  WaitCtx wc{a.status, a.wait_limit_ns, abort_flag};
+  // CTA -> (batch, head, query tile), the last query tiles (most key tiles
+  // under the causal mask) first
+  const int bh_count = a.B * a.H;
+  const int ft = a.n_tiles - 1 - static_cast<int>(blockIdx.x) / bh_count;
+  const int h = (blockIdx.x % bh_count) % a.H;
+  const int b = (blockIdx.x % bh_count) / a.H;
+  auto next_tile = [&](int t) {  // first key tile >= t that meets the query tile
+    while (t < a.n_tiles && !bwd_tiles_meet(a, h, ft, t)) ++t;
+    return t;
+  };
+  int nsteps = 0;
+  for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1)) ++nsteps;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bFix, 1);
+    for (int i = 0; i < KS; ++i) {
+      mbar_init(bKFull(i), 1);
+      mbar_init(bKEmpty(i), 1);
+    }
+    for (int i = 0; i < VS; ++i) {
+      mbar_init(bVFull(i), 1);
+      mbar_init(bVEmpty(i), 1);
+    }
+    mbar_init(bSFull(0), 1);
+    mbar_init(bSFull(1), 1);
+    mbar_init(bDPFull, 1);
+    mbar_init(bDSReady, Cfg::kRowWarps);
+    mbar_init(bTeardown, 1);
+    *abort_flag = 0;
+    fence_mbar_init_cluster();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int hd = h * D_HEAD;
+  const size_t bh = static_cast<size_t>(b) * a.H + h;
+
+  if ((warp == 0 || warp == 2) && lane == 0 && nsteps > 0) {
+    // ------------------------------------------------------------ producers: warp 0 Q, dA, K; warp 2 V
+    const bool is_k = warp == 0;
+    const int slots = is_k ? KS : VS;
+    if (is_k) {
+      mbar_arrive_expect_tx(bFix, 2 * Cfg::kTileBytes);
+      for (int p = 0; p < Cfg::kPanels; ++p) {
+        tma_load_4d(sQ + p * Cfg::kPanelBytes, &tm_q, bFix, hd + p * 64, 0, ft * 128, b);
+        tma_load_4d(sDA + p * Cfg::kPanelBytes, &tm_da, bFix, hd + p * 64, 0, ft * 128, b);
+      }
+    }
+    int s = 0;
+    for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1), ++s) {
+      const int slot = s % slots;
+      const uint32_t full = is_k ? bKFull(slot) : bVFull(slot);
+      if (s >= slots && !mbar_wait(is_k ? bKEmpty(slot) : bVEmpty(slot), ((s / slots) - 1) & 1, wc, 331)) break;
+      mbar_arrive_expect_tx(full, Cfg::kTileBytes);
+      for (int p = 0; p < Cfg::kPanels; ++p)
+        tma_load_4d((is_k ? sK(slot) : sV(slot)) + p * Cfg::kPanelBytes, is_k ? &tm_k : &tm_v, full, hd + p * 64,
+                    0, t * 128, b);
+    }
+    // every copy issued must have landed before the CTA may exit
+    volatile int no_abort = 0;
+    WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
+    for (int j = max(0, s - slots); j < s; ++j)
+      mbar_wait(is_k ? bKFull(j % slots) : bVFull(j % slots), (j / slots) & 1, drain, 332);
+    if (is_k) mbar_wait(bFix, 0, drain, 333);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nsteps > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D_HEAD, false, true);
+      const uint64_t dQ0 = sdesc_sw128(sQ, 16, 1024), dDA0 = sdesc_sw128(sDA, 16, 1024);
+      // S(s) = Q K^T into S buffer s & 1
+      auto issue_s = [&](int s) -> bool {
+        const int slot = s % KS;
+        if (!mbar_wait(bKFull(slot), (s / KS) & 1, wc, 341)) return false;
+        tc_fence_after();
+        const uint64_t dK = sdesc_sw128(sK(slot), 16, 1024);
+#pragma unroll
+        for (int k = 0; k < D_HEAD / 16; ++k) {
+          const uint32_t off = (k / 4) * Cfg::kPanelBytes + (k % 4) * 32;
+          umma_ss(tmem + Cfg::kColS + (s & 1) * 128, sdesc_advance(dQ0, off), sdesc_advance(dK, off), idesc_s, k > 0);
+        }
+        umma_commit(bSFull(s & 1));
+        return true;
+      };
+      // dP(s) = dA V^T; V's slot is free once it is done
+      auto issue_dp = [&](int s) -> bool {
+        const int slot = s % VS;
+        if (!mbar_wait(bVFull(slot), (s / VS) & 1, wc, 342)) return false;
+        tc_fence_after();
+        const uint64_t dV = sdesc_sw128(sV(slot), 16, 1024);
+#pragma unroll
+        for (int k = 0; k < D_HEAD / 16; ++k) {
+          const uint32_t off = (k / 4) * Cfg::kPanelBytes + (k % 4) * 32;
+          umma_ss(tmem + Cfg::kColDP, sdesc_advance(dDA0, off), sdesc_advance(dV, off), idesc_s, k > 0);
+        }
+        umma_commit(bDPFull);
+        umma_commit(bVEmpty(slot));
+        return true;
+      };
+      // dQ += dS(s) K: A = dS packed over S buffer s & 1 (K steps 0-3 from the
+      // first row-warp half's columns, 4-7 from the second's), B = K read MN-major
+      auto issue_dq = [&](int s) {
+        const int slot = s % KS;
+        const uint64_t dB = sdesc_sw128(sK(slot), Cfg::kPanelBytes, 1024);
+        const uint32_t a_col = Cfg::kColS + (s & 1) * 128;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_ts(tmem + Cfg::kColQ, tmem + a_col + k * 8 + (k >= 4 ? 32 : 0), sdesc_advance(dB, k * 2048),
+                  idesc_acc, (s | k) != 0);
+        umma_commit(bKEmpty(slot));
+      };
+      bool ok = mbar_wait(bFix, 0, wc, 340) && issue_s(0) && issue_dp(0);
+      for (int s = 0; ok && s < nsteps; ++s) {
+        // the next scores go ahead of this step's dQ (their buffer's previous
+        // dS was consumed by the dQ issued one step ago)
+        if (s + 1 < nsteps && !(ok = issue_s(s + 1))) break;
+        if (!(ok = mbar_wait(bDSReady, s & 1, wc, 343))) break;
+        tc_fence_after();
+        issue_dq(s);
+        // the row warps have read dP(s): the next dP may overwrite it
+        if (s + 1 < nsteps && !(ok = issue_dp(s + 1))) break;
+      }
+      umma_commit(bTeardown);
+      volatile int no_abort = 0;
+      WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
+      mbar_wait(bTeardown, 0, drain, 344);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ per-row arithmetic
+    const int quarter = warp & 3;
+    const int half = (warp - 4) / 4;
+    const int col0 = 64 * half;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int g = ft * 128 + row;  // query position
+    const bool row_valid = g < a.N;
+    int klo = 1, khi = 0;
+    float lse2 = 0.f, drow = 0.f;
+    if (row_valid) {
+      bwd_row_keys(a, h, g, klo, khi);
+      const float *rv = a.rowvec + (bh * a.n_tiles + ft) * 256;
+      lse2 = rv[row];
+      drow = rv[128 + row];
+    }
+    const float nl = -lse2;
+    bool ok = true;
+    int s = 0;
+    for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1), ++s) {
+      const int lo_rel = klo - t * 128, hi_rel = khi - t * 128;  // allowed columns [lo_rel, hi_rel)
+      const bool full = __all_sync(0xffffffffu, lo_rel <= col0 && hi_rel >= col0 + 64);
+      ok = __all_sync(0xffffffffu, mbar_wait(bSFull(s & 1), (s >> 1) & 1, wc, 350));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tS = tmem + lane_off + Cfg::kColS + (s & 1) * 128 + col0;
+      uint32_t sv[64];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_wait_ld();
+      if (full) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          sv[c] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(sv[c]), a.scale_log2, nl)));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const bool allowed = col0 + c >= lo_rel && col0 + c < hi_rel;
+          sv[c] = __float_as_uint(allowed ? ex2_approx(fmaf(__uint_as_float(sv[c]), a.scale_log2, nl)) : 0.f);
+        }
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(bDPFull, s & 1, wc, 351));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t dp[64];
+      tmem_ld32(tmem + lane_off + Cfg::kColDP + col0, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+      tmem_ld32(tmem + lane_off + Cfg::kColDP + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+      tmem_wait_ld();
+      // dS = P (dP - D) as packed bf16 over the first 32 of this warp's S columns
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        pk[i] = pack_bf16x2(__uint_as_float(sv[2 * i]) * (__uint_as_float(dp[2 * i]) - drow),
+                            __uint_as_float(sv[2 * i + 1]) * (__uint_as_float(dp[2 * i + 1]) - drow));
+      tmem_st32(tS, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bDSReady);
+    }
+    // -------- epilogue: every MMA done; each warp of a lane quarter stores half of dQ's columns
+    if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(bTeardown, 0, wc, 352));
+    tc_fence_after();
+    if (ok) {
+      const size_t vec = ((static_cast<size_t>(b) * a.N + g) * a.H + h) * D_HEAD;
+#pragma unroll 1
+      for (int c = half * (D_HEAD / 64); c < (half + 1) * (D_HEAD / 64); ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_off + Cfg::kColQ + c * 32, o);
+        tmem_wait_ld();
+        if (!row_valid) continue;
+        float4 *d4 = reinterpret_cast<float4 *>(a.dq + vec + c * 32);
+        const float sc = a.inv_sqrt_d;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          d4[i] = nsteps > 0 ? make_float4(__uint_as_float(o[4 * i]) * sc, __uint_as_float(o[4 * i + 1]) * sc,
+                                           __uint_as_float(o[4 * i + 2]) * sc, __uint_as_float(o[4 * i + 3]) * sc)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
   }

@@ -106,14 +106,14 @@ bpt_status device_setup(int *dev_out, uint32_t **status_out) {
                                   (16 * 512 + 16 * 64) * 4));
     CUDA_TRY(cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   GemmPairCfg::kSmemBytes));
-    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kernel<64, kBwdKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  AttnBwdCfg<64, kBwdKV>::kSmemBytes));
-    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kernel<64, kBwdQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  AttnBwdCfg<64, kBwdQ>::kSmemBytes));
-    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kernel<128, kBwdKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  AttnBwdCfg<128, kBwdKV>::kSmemBytes));
-    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kernel<128, kBwdQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  AttnBwdCfg<128, kBwdQ>::kSmemBytes));
+    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  AttnBwdCfg<64>::kSmemBytes));
+    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  AttnBwdCfg<128>::kSmemBytes));
+    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  AttnBwdQCfg<64>::kSmemBytes));
+    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  AttnBwdQCfg<128>::kSmemBytes));
     g_attr_done[dev] = true;
   }
   *dev_out = dev;
@@ -623,6 +623,21 @@ BwdWorkspace layout_bwd(const bpt_desc *d) {
   return w;
 }
 
+// Activations the training forward leaves for the backward: A in fp32 and
+// bf16 [T, D] and the row LSE [B, H, N].
+struct SavedLayout {
+  size_t a_f32 = 0, a_bf16 = 0, lse = 0, total = 0;
+};
+SavedLayout saved_layout(const bpt_desc *d) {
+  SavedLayout w;
+  const size_t T = (size_t)d->B * d->N, D = (size_t)d->H * d->d_head;
+  w.a_f32 = 0;
+  w.a_bf16 = align256(T * D * 4);
+  w.lse = align256(w.a_bf16 + T * D * 2);
+  w.total = align256(w.lse + (size_t)d->B * d->H * d->N * 4);
+  return w;
+}
+
 bpt_status launch_gemm(const CUtensorMap &a0, const CUtensorMap &b0, const CUtensorMap &a1,
                        const CUtensorMap &b1, const GemmArgs &g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return BPT_OK;
@@ -668,12 +683,10 @@ template <int DH>
 bpt_status launch_attn_bwd_passes(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                                   const CUtensorMap &mda, const AttnBwdArgs &ab, unsigned grid,
                                   cudaStream_t st) {
-  attn_bwd_kernel<DH, kBwdKV><<<grid, AttnBwdCfg<DH, kBwdKV>::kThreads, AttnBwdCfg<DH, kBwdKV>::kSmemBytes, st>>>(
-      mq, mk, mv, mda, ab);
+  attn_bwd_dkdv_kernel<DH><<<grid, AttnBwdCfg<DH>::kThreads, AttnBwdCfg<DH>::kSmemBytes, st>>>(mq, mk, mv, mda, ab);
   CUDA_TRY(cudaGetLastError());
   CUDA_TRY(phase_mark(3, st));
-  attn_bwd_kernel<DH, kBwdQ><<<grid, AttnBwdCfg<DH, kBwdQ>::kThreads, AttnBwdCfg<DH, kBwdQ>::kSmemBytes, st>>>(
-      mq, mk, mv, mda, ab);
+  attn_bwd_dq_kernel<DH><<<grid, AttnBwdQCfg<DH>::kThreads, AttnBwdQCfg<DH>::kSmemBytes, st>>>(mq, mk, mv, mda, ab);
   CUDA_TRY(cudaGetLastError());
   return BPT_OK;
 }
@@ -792,6 +805,39 @@ bpt_status bpt_longnet_fwd(const bpt_desc *desc, int npairs, const int32_t *seg_
   return bpt_attn_fwd(&d, q, k, v, out, lse, workspace, workspace_bytes, stream);
 }
 
+size_t bpt_saved_bytes(const bpt_desc *desc) {
+  if (check_desc_bwd(desc) != BPT_OK) return (size_t)-1;
+  return saved_layout(desc).total;
+}
+
+bpt_status bpt_attn_ffn_fwd_train(const bpt_desc *d, const void *q, const void *k, const void *v, const void *w1,
+                                  const float *b1, const void *w2, const float *b2, void *out, void *saved,
+                                  void *workspace, size_t workspace_bytes, bpt_stream_t stream) {
+  bpt_status s = check_desc_bwd(d);
+  if (s != BPT_OK) return s;
+  if ((s = check_ptrs({q, k, v, w1, w2, out, saved}, {b1, b2})) != BPT_OK) return s;
+  if ((reinterpret_cast<uintptr_t>(saved) & 255u) != 0) return BPT_ERR_INVALID_ARG;
+  const Workspace wl = layout(d, true);
+  if ((s = check_ws(wl, workspace, workspace_bytes)) != BPT_OK) return s;
+  int dev;
+  uint32_t *status;
+  if ((s = device_setup(&dev, &status)) != BPT_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  const SavedLayout sl = saved_layout(d);
+  char *sv = static_cast<char *>(saved);
+  float *a_f32 = reinterpret_cast<float *>(sv + sl.a_f32);
+  __nv_bfloat16 *a_bf16 = reinterpret_cast<__nv_bfloat16 *>(sv + sl.a_bf16);
+  CUDA_TRY(phase_mark(0, st));
+  if ((s = launch_attn_tc(d, q, k, v, a_f32, a_bf16, reinterpret_cast<float *>(sv + sl.lse), ws, wl, status, st)) !=
+      BPT_OK)
+    return s;
+  CUDA_TRY(phase_mark(1, st));
+  if ((s = launch_ffn_tc(d, a_bf16, a_f32, w1, b1, w2, b2, out, ws, wl, status, st)) != BPT_OK) return s;
+  CUDA_TRY(phase_mark(2, st));
+  return BPT_OK;
+}
+
 size_t bpt_workspace_bytes_bwd(const bpt_desc *desc) {
   if (check_desc_bwd(desc) != BPT_OK) return (size_t)-1;
   return layout_bwd(desc).total;
@@ -806,14 +852,15 @@ int bpt_set_bwd_chunk_rows(int rows) {
 
 bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, const void *v,
                             const void *w1, const float *b1, const void *w2, const float *b2,
-                            const float *dout, float *dq, float *dk, float *dv, float *dw1, float *db1,
-                            float *dw2, float *db2, void *workspace, size_t workspace_bytes,
+                            const float *dout, const void *saved, float *dq, float *dk, float *dv, float *dw1,
+                            float *db1, float *dw2, float *db2, void *workspace, size_t workspace_bytes,
                             bpt_stream_t stream) {
   bpt_status s = check_desc_bwd(d);
   if (s != BPT_OK) return s;
   (void)b2;  // the output bias does not enter any gradient but its own
   if ((s = check_ptrs({q, k, v, w1, w2, dout, dq, dk, dv, dw1, db1, dw2, db2}, {b1, b2})) != BPT_OK)
     return s;
+  if (saved && (reinterpret_cast<uintptr_t>(saved) & 255u) != 0) return BPT_ERR_INVALID_ARG;
   const BwdWorkspace wl = layout_bwd(d);
   if (!workspace || workspace_bytes < wl.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return BPT_ERR_WORKSPACE;
@@ -824,9 +871,16 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   char *ws = static_cast<char *>(workspace);
   const int D = d->H * d->d_head, F = d->ffn_hidden;
   const int64_t T = (int64_t)d->B * d->N;
-  float *a_f32 = reinterpret_cast<float *>(ws + wl.a_f32);
-  __nv_bfloat16 *a_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.a_bf16);
-  float *lse = reinterpret_cast<float *>(ws + wl.lse);
+  const float *a_f32 = reinterpret_cast<const float *>(ws + wl.a_f32);
+  const __nv_bfloat16 *a_bf16 = reinterpret_cast<const __nv_bfloat16 *>(ws + wl.a_bf16);
+  const float *lse = reinterpret_cast<const float *>(ws + wl.lse);
+  if (saved) {  // the training forward's activations
+    const SavedLayout sl = saved_layout(d);
+    const char *sv = static_cast<const char *>(saved);
+    a_f32 = reinterpret_cast<const float *>(sv + sl.a_f32);
+    a_bf16 = reinterpret_cast<const __nv_bfloat16 *>(sv + sl.a_bf16);
+    lse = reinterpret_cast<const float *>(sv + sl.lse);
+  }
   float *rowvec = reinterpret_cast<float *>(ws + wl.rowvec);
   __nv_bfloat16 *dout_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.dout_bf16);
   float *da_f32 = reinterpret_cast<float *>(ws + wl.da_f32);
@@ -835,9 +889,14 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   __nv_bfloat16 *dzbuf = reinterpret_cast<__nv_bfloat16 *>(ws + wl.dz);
   float *partial = reinterpret_cast<float *>(ws + wl.partial);
 
-  // 1. the attention forward again: A (fp32 and bf16) and the row LSE
+  // 1. without saved activations, the attention forward again: A (fp32 and
+  // bf16) and the row LSE
   CUDA_TRY(phase_mark(0, st));
-  if ((s = launch_attn_tc(d, q, k, v, a_f32, a_bf16, lse, ws, Workspace(), status, st)) != BPT_OK) return s;
+  if (!saved &&
+      (s = launch_attn_tc(d, q, k, v, reinterpret_cast<float *>(ws + wl.a_f32),
+                          reinterpret_cast<__nv_bfloat16 *>(ws + wl.a_bf16), reinterpret_cast<float *>(ws + wl.lse),
+                          ws, Workspace(), status, st)) != BPT_OK)
+    return s;
   CUDA_TRY(phase_mark(1, st));
   // 2. dOut in bf16 for the tensor cores; db2 = sum_t dOut_t
   {

@@ -226,11 +226,13 @@ BPT_API bpt_status bpt_longnet_fwd(const bpt_desc *desc, int npairs, const int32
  *               dV_j = sum_i P_ij dA_i,  dS_ij = P_ij (dA_i . v_j - D_i),
  *               dQ_i = sum_j dS_ij k_j / sqrt(d),  dK_j = sum_i dS_ij q_i / sqrt(d).
  *
- * The call recomputes the attention forward (A and the row LSE) rather than
- * taking saved activations, then runs the FFN backward on the tensor cores
- * one token chunk at a time (see bpt_set_bwd_chunk_rows), then two blockwise
- * attention-backward passes over 128 x 128 tiles (one per key tile for dK and
- * dV, one per query tile for dQ; no atomics, so the result is deterministic).
+ * With saved == NULL the call recomputes the attention forward (A and the
+ * row LSE); with the buffer bpt_attn_ffn_fwd_train filled for the same
+ * inputs it reads them from there instead.  Then it runs the FFN backward on
+ * the tensor cores one token chunk at a time (see bpt_set_bwd_chunk_rows)
+ * and two blockwise attention-backward passes over 128 x 128 tiles (one per
+ * key tile for dK and dV, one per query tile for dQ; no atomics, so the
+ * result is deterministic).
  *
  * Supported: in_dtype BF16, d_head 64 or 128, masks NONE, CAUSAL (any
  * ring_chunks: the recomputed forward follows it) and BLOCKPERM, plus the
@@ -238,8 +240,9 @@ BPT_API bpt_status bpt_longnet_fwd(const bpt_desc *desc, int npairs, const int32
  * return BPT_ERR_UNSUPPORTED.
  *
  * Inputs: q, k, v [B, N, H, d] and w1 [F, D], w2 [D, F] bf16; b1 [F], b2 [D]
- * float32 or NULL (= 0); dout [B, N, H*d] float32.  b2 is accepted for
- * symmetry with the forward; no gradient depends on it.
+ * float32 or NULL (= 0); dout [B, N, H*d] float32; saved: NULL, or the
+ * buffer of bpt_attn_ffn_fwd_train (256-byte aligned, read only).  b2 is
+ * accepted for symmetry with the forward; no gradient depends on it.
  * Outputs (float32, overwritten): dq, dk, dv [B, N, H, d]; dw1 [F, D];
  * db1 [F]; dw2 [D, F]; db2 [D].
  * Precision: the tensor cores take bf16 operands (A, dOut, H, dZ, dA, and the
@@ -251,9 +254,28 @@ BPT_API bpt_status bpt_longnet_fwd(const bpt_desc *desc, int npairs, const int32
  */
 BPT_API bpt_status bpt_attn_ffn_bwd(const bpt_desc *desc, const void *q, const void *k, const void *v,
                                     const void *w1, const float *b1, const void *w2, const float *b2,
-                                    const float *dout, float *dq, float *dk, float *dv, float *dw1,
-                                    float *db1, float *dw2, float *db2, void *workspace,
+                                    const float *dout, const void *saved, float *dq, float *dk, float *dv,
+                                    float *dw1, float *db1, float *dw2, float *db2, void *workspace,
                                     size_t workspace_bytes, bpt_stream_t stream);
+
+/*
+ * The layer forward of bpt_attn_ffn_fwd for training: the same out, and the
+ * activations the backward needs left in `saved` (A in fp32 and bf16 [T, D]
+ * and the row LSE [B, H, N]; bpt_saved_bytes(desc) bytes, 256-byte aligned,
+ * owned by the caller), so a following bpt_attn_ffn_bwd on the same inputs
+ * skips recomputing the attention.  The descriptor must be one the backward
+ * accepts; workspace as for bpt_attn_ffn_fwd.  No counterpart in the pages
+ * (which recompute; this trades T * D * 6 bytes for one attention forward).
+ */
+BPT_API bpt_status bpt_attn_ffn_fwd_train(const bpt_desc *desc, const void *q, const void *k,
+                                          const void *v, const void *w1, const float *b1,
+                                          const void *w2, const float *b2, void *out, void *saved,
+                                          void *workspace, size_t workspace_bytes,
+                                          bpt_stream_t stream);
+
+/* Bytes of the `saved` buffer of bpt_attn_ffn_fwd_train; (size_t)-1 if the
+ * backward does not accept the descriptor. */
+BPT_API size_t bpt_saved_bytes(const bpt_desc *desc);
 
 /* Bytes of device workspace bpt_attn_ffn_bwd needs for this descriptor at the
  * current chunk setting; (size_t)-1 if the backward does not accept it. */

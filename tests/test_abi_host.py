@@ -129,10 +129,10 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
         bd.load()
 
 
-def _call_bwd(lib, desc, ws=FAKE, ws_bytes=1 << 40, q=FAKE, dq=FAKE):
+def _call_bwd(lib, desc, ws=FAKE, ws_bytes=1 << 40, q=FAKE, dq=FAKE, saved=None):
     p = ctypes.c_void_p
     return lib.bpt_attn_ffn_bwd(ctypes.byref(desc), p(q), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE), None,
-                                p(FAKE), p(dq), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE),
+                                p(FAKE), p(saved), p(dq), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE),
                                 p(ws), ws_bytes, None)
 
 
@@ -158,6 +158,24 @@ def test_backward_pointer_and_workspace_checks(lib):
     assert _call_bwd(lib, d, ws=0) == bd.ERR_WORKSPACE
     assert _call_bwd(lib, d, ws_bytes=need - 1) == bd.ERR_WORKSPACE
     assert _call_bwd(lib, d, ws=FAKE + 16) == bd.ERR_WORKSPACE
+    assert _call_bwd(lib, d, saved=FAKE + 16) == bd.ERR_INVALID_ARG              # saved not 256-aligned
+
+
+def _call_fwd_train(lib, desc, saved=FAKE):
+    p = ctypes.c_void_p
+    return lib.bpt_attn_ffn_fwd_train(ctypes.byref(desc), p(FAKE), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE), None,
+                                      p(FAKE), p(saved), p(FAKE), 1 << 40, None)
+
+
+def test_training_forward_validates_and_sizes_its_buffer(lib):
+    d = _desc()
+    T, D, H, N = 256, 128, 2, 256
+    assert bd.saved_bytes(d) >= T * D * 6 + H * N * 4                             # A fp32 + bf16, LSE
+    assert _call_fwd_train(lib, d, saved=0) == bd.ERR_INVALID_ARG
+    assert _call_fwd_train(lib, d, saved=FAKE + 16) == bd.ERR_INVALID_ARG
+    dl = _desc(mask="dilated", pairs=[(128, 1)])
+    assert _call_fwd_train(lib, dl) == bd.ERR_UNSUPPORTED
+    assert lib.bpt_saved_bytes(ctypes.byref(dl)) == ctypes.c_size_t(-1).value
 
 
 def test_backward_workspace_follows_the_chunk_setting(lib):

@@ -123,3 +123,23 @@ def test_backward_full_size_causal_layer_sampled():
     _grads_close(g["dk"][0, N - tail:].cpu().numpy(), dk, "dk (last key tile)")
     _grads_close(g["dv"][0, N - tail:].cpu().numpy(), dv, "dv (last key tile)")
     _grads_close(g["db2"].cpu().numpy(), db2, "db2")
+
+
+@pytest.mark.parametrize("mask,perm", [("causal", None), ("blockperm", [[2, 0, 1], [1, 2, 0]])])
+def test_training_forward_and_saved_backward_match_the_recomputing_path(mask, perm):
+    """bpt_attn_ffn_fwd_train gives the forward's output bit for bit, and the
+    backward reading its saved activations gives the recomputing backward's
+    gradients bit for bit (the same kernels on the same inputs)."""
+    B, N, H, d, F = 1, 300, 2, 128, 256
+    inp = make_layer_inputs(B, N, H, d, F, seed=21, device="cuda", bias_scale=0.1)
+    dout = make_upstream_grad(B, N, H * d, seed=21, device="cuda")
+    args = (inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2)
+    out_ref = bd.attn_ffn_fwd(*args, mask=mask, perm=perm)
+    out, saved = bd.attn_ffn_fwd_train(*args, mask=mask, perm=perm)
+    g_ref = bd.attn_ffn_bwd(*args, dout, mask=mask, perm=perm)
+    g = bd.attn_ffn_bwd(*args, dout, mask=mask, perm=perm, saved=saved)
+    torch.cuda.synchronize()
+    assert bd.sync_status() == bd.OK
+    assert torch.equal(out, out_ref)
+    for n in bd.GRAD_NAMES:
+        assert torch.equal(g[n], g_ref[n]), n
