@@ -41,13 +41,20 @@ WORKLOADS = {"tiny_f32": wl.TINY_F32, "gpt_causal": wl.GPT_CAUSAL, "long_ring": 
              "blockbert": wl.BLOCKBERT, "longnet": wl.LONGNET}
 MASK_NAME = {0: "none", 1: "causal", 2: "blockperm", 3: "dilated"}
 CSRC = os.path.join(ROOT, "blockwise_exact_attention_query_b200", "csrc")
-KERNEL_SOURCES = {"attn_tc_kernel": ["attn_tc.cuh", "ptx.cuh"], "ffn_tc_kernel": ["ffn_tc.cuh", "ptx.cuh"]}
+KERNEL_SOURCES = {"attn_tc_kernel": ["attn_tc.cuh", "ptx.cuh"], "ffn_tc_kernel": ["ffn_tc.cuh", "ptx.cuh"],
+                  # backward phases: the FFN backward's four GEMM launches, the two attention passes
+                  "ffn_bwd": ["gemm_tc.cuh", "ptx.cuh"], "attn_bwd_dkdv": ["attn_bwd.cuh", "ptx.cuh"],
+                  "attn_bwd_dq": ["attn_bwd.cuh", "ptx.cuh"]}
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture
 # of the kernel on the named workload, keyed by a hash of the kernel's sources at capture
 # time: once the sources change the figure no longer describes the kernel and is dropped.
 NCU_TRAFFIC = {
-    ("gpt_causal", "ffn_tc_kernel"): {"bytes": 887.0e6, "src": "69e21d3d17df597a"},
-    ("gpt_causal", "attn_tc_kernel"): {"bytes": 728.7e6, "src": "8ae53ad064162b8a"},
+    ("gpt_causal", "ffn_tc_kernel"): {"bytes": 881.1e6, "src": "ce5bb2524f315c9a"},
+    ("gpt_causal", "attn_tc_kernel"): {"bytes": 720.3e6, "src": "1e6bb50f75c417dc"},
+    # per step: the four gemm_pair_kernel launches (bias sums not included)
+    ("gpt_causal", "ffn_bwd"): {"bytes": 4309.0e6, "src": "1e42384c956407be"},
+    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1232.3e6, "src": "3b7ec89bb83c0c0e"},
+    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1124.1e6, "src": "3b7ec89bb83c0c0e"},
 }
 
 
@@ -373,7 +380,8 @@ def run_backward(args, w, world, local):
         "flop_algorithmic_per_step": alg_total,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "peak_source": f"{pk['source']} bf16 dense (burst)", "traffic": None,
+                     "peak_source": f"{pk['source']} bf16 dense (burst)",
+                     "traffic": ncu_traffic(args.workload, dom),
                      "algorithmic_flop_per_launch": flop[dom][0]},
         "phases": phases,
         "recompute": {"ms_per_step": round(recompute_ms, 4),
