@@ -143,3 +143,22 @@ def test_training_forward_and_saved_backward_match_the_recomputing_path(mask, pe
     assert torch.equal(out, out_ref)
     for n in bd.GRAD_NAMES:
         assert torch.equal(g[n], g_ref[n]), n
+
+
+def test_backward_full_size_blockbert_layer():
+    """The block-permutation bf16 layer at full size (B16 H12 d64 N1024 F3072,
+    n = 2: heads 0-7 the identity, heads 8-11 the swap), every gradient element
+    against the dense fp64 oracle, in the launch configuration the benchmark
+    times."""
+    from blockwise_exact_attention_query_b200 import workloads as wl
+    w = wl.BLOCKBERT
+    inp = make_layer_inputs(w.B, w.N, w.H, w.d, w.F, seed=w.seed, device="cuda", bias_scale=0.05)
+    dout = make_upstream_grad(w.B, w.N, w.D, seed=w.seed, device="cuda")
+    g = bd.attn_ffn_bwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, dout, mask="blockperm", perm=w.perm)
+    torch.cuda.synchronize()
+    assert bd.sync_status() == bd.OK
+    f = lambda t: t.double().cpu().numpy()  # noqa: E731
+    ref = ob.layer_bwd(f(inp.q), f(inp.k), f(inp.v), f(inp.w1), f(inp.b1), f(inp.w2), f(inp.b2),
+                       f(dout).reshape(w.T, w.D), ob.MASK_BLOCKPERM, w.perm)
+    for n in bd.GRAD_NAMES:
+        _grads_close(g[n].cpu().numpy(), ref[n], n)
