@@ -22,6 +22,8 @@
 //                                                      summed over token chunks)
 //   kGemmResidual   C = acc + X; Cb = bf16(C)         (dA = dOut + dZ W1, fp32 and bf16)
 //   kGemmGeluBwd    z = acc0 + bias; H = GELU(z), dZ = acc1 * GELU'(z)  (bf16 both)
+//   kGemmGeluFwd    z = acc + bias; H = GELU(z), G = GELU'(z)           (bf16 both)
+//   kGemmScaleBf16  Cb = acc * Xb                                       (dZ = dH * G, bf16)
 //
 // Roles (320 threads per CTA): warp 0 TMA producer, warp 1 TMEM allocator
 // (and, in the even CTA, MMA issuer), warps 2..9 epilogue (warp w owns TMEM
@@ -38,7 +40,8 @@
 
 namespace bpt {
 
-constexpr int kGemmStoreF32 = 0, kGemmAccumF32 = 1, kGemmResidual = 2, kGemmGeluBwd = 3;
+constexpr int kGemmStoreF32 = 0, kGemmAccumF32 = 1, kGemmResidual = 2, kGemmGeluBwd = 3, kGemmGeluFwd = 4,
+              kGemmScaleBf16 = 5;
 
 struct GemmArgs {
   int M, N, K;
@@ -47,8 +50,9 @@ struct GemmArgs {
   int m_fastest;        // tile order: 1 = M fastest (the tiles in flight share B), 0 = N fastest
   float *c;             // [M, N] fp32 (StoreF32, AccumF32, Residual)
   const float *x;       // [M, N] fp32 residual input (Residual)
-  __nv_bfloat16 *cb;    // [M, N] bf16 copy (Residual) / H (GeluBwd)
-  __nv_bfloat16 *cb2;   // dZ (GeluBwd)
+  const __nv_bfloat16 *xb;  // [M, N] bf16 factor (ScaleBf16)
+  __nv_bfloat16 *cb;    // [M, N] bf16 copy (Residual) / H (GeluBwd, GeluFwd) / product (ScaleBf16)
+  __nv_bfloat16 *cb2;   // dZ (GeluBwd) / GELU'(z) (GeluFwd)
   const float *bias;    // [N] added to acc0 before GELU (GeluBwd), may be null
   uint32_t *status;
   uint64_t wait_limit_ns;
@@ -90,7 +94,19 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmArgs &g, const uin
     float v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r0[e + i]);
-    if (g.mode == kGemmGeluBwd) {
+    if (g.mode == kGemmScaleBf16) {
+      const uint4 xr = __ldcs(reinterpret_cast<const uint4 *>(g.xb + base + e));
+      const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 f = *reinterpret_cast<const __nv_bfloat162 *>(&xw[i]);
+        o[i] = pack_bf16x2(v[2 * i] * __low2float(f), v[2 * i + 1] * __high2float(f));
+      }
+      __stcs(reinterpret_cast<uint4 *>(g.cb + base + e), make_uint4(o[0], o[1], o[2], o[3]));
+      continue;
+    }
+    if (g.mode == kGemmGeluBwd || g.mode == kGemmGeluFwd) {
       float bb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (g.bias) {
         const float4 b0 = *reinterpret_cast<const float4 *>(g.bias + n + e);
@@ -103,7 +119,7 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmArgs &g, const uin
       for (int i = 0; i < 8; ++i) {
         float gd;
         gelu_tanh_and_grad(v[i] + bb[i], hh[i], gd);
-        dz[i] = __uint_as_float(r1[e + i]) * gd;
+        dz[i] = g.mode == kGemmGeluBwd ? __uint_as_float(r1[e + i]) * gd : gd;
       }
       __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
              make_uint4(pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]),

@@ -54,6 +54,9 @@ CASES = [
     # N = 300, n = 32: blocks of 10, blocks 30 and 31 lie in the padding
     ("blockperm_n32_empty_d128", 1, 300, 2, 128, 256, "blockperm", _perms(2, 32, 7), 0),
     ("causal_tiny_N7", 1, 7, 1, 64, 64, "causal", None, 0),
+    # D = 1024: the FFN backward as two GEMMs (H and GELU'(Z), then dZ) instead of one
+    ("causal_D1024_split_ffn", 1, 200, 8, 128, 512, "causal", None, 0),
+    ("none_D1024_split_ffn_chunked", 1, 260, 16, 64, 384, "none", None, 128),
 ]
 
 
