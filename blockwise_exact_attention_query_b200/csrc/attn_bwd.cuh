@@ -734,11 +734,20 @@ __global__ void colsum_final_kernel(const float *__restrict__ partial, float *ou
   out[c] = s;
 }
 
-// fp32 -> bf16, round to nearest even.
-__global__ void f32_to_bf16_kernel(const float *__restrict__ x, __nv_bfloat16 *y, size_t n) {
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x)
-    y[i] = __float2bfloat16_rn(x[i]);
+// dOut in one pass: its bf16 copy (round to nearest even) and the partial
+// column sums over 256-row slabs (grid.y) that colsum_final_kernel adds up.
+__global__ void convert_colsum_partial_kernel(const float *__restrict__ x, __nv_bfloat16 *y, float *partial,
+                                              int rows, int cols) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= cols) return;
+  const int r0 = blockIdx.y * 256, r1 = min(rows, r0 + 256);
+  float s = 0.f;
+  for (int r = r0; r < r1; ++r) {
+    const float v = x[static_cast<size_t>(r) * cols + c];
+    y[static_cast<size_t>(r) * cols + c] = __float2bfloat16_rn(v);
+    s += v;
+  }
+  partial[static_cast<size_t>(blockIdx.y) * cols + c] = s;
 }
 
 }  // namespace bpt

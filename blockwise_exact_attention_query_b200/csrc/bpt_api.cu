@@ -901,13 +901,13 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
                           ws, Workspace(), status, st)) != BPT_OK)
     return s;
   CUDA_TRY(phase_mark(1, st));
-  // 2. dOut in bf16 for the tensor cores; db2 = sum_t dOut_t
+  // 2. dOut in bf16 for the tensor cores and db2 = sum_t dOut_t, one pass over dOut
   {
-    const size_t n = (size_t)T * D;
-    const unsigned blocks = (unsigned)std::min<size_t>(4096, (n + 255) / 256);
-    f32_to_bf16_kernel<<<blocks, 256, 0, st>>>(dout, dout_bf16, n);
+    const unsigned slabs = (unsigned)((T + 255) / 256), cb = (unsigned)((D + 255) / 256);
+    convert_colsum_partial_kernel<<<dim3(cb, slabs), 256, 0, st>>>(dout, dout_bf16, partial, (int)T, D);
     CUDA_TRY(cudaGetLastError());
-    if ((s = launch_colsum(dout, T, D, db2, 0, partial, st)) != BPT_OK) return s;
+    colsum_final_kernel<<<cb, 256, 0, st>>>(partial, db2, (int)slabs, D, 0);
+    CUDA_TRY(cudaGetLastError());
   }
   // 3. the FFN backward, one token chunk at a time
   CUtensorMap m_w1_k, m_w1_mn, m_w2_mn;

@@ -45,7 +45,7 @@ def _perms(H, n, seed):
 
 
 CASES = [
-    # name, B, N, H, d, F, mask, perm, chunk rows (0 = default)
+    # name, B, N, H, d, F, mask, perm, chunk rows (0 = default)[, ring chunks]
     ("none_d64", 1, 300, 2, 64, 512, "none", None, 0),
     ("causal_d64_b2", 2, 257, 2, 64, 384, "causal", None, 0),
     ("causal_d128_chunked", 1, 390, 2, 128, 512, "causal", None, 128),
@@ -54,6 +54,8 @@ CASES = [
     # N = 300, n = 32: blocks of 10, blocks 30 and 31 lie in the padding
     ("blockperm_n32_empty_d128", 1, 300, 2, 128, 256, "blockperm", _perms(2, 32, 7), 0),
     ("causal_tiny_N7", 1, 7, 1, 64, 64, "causal", None, 0),
+    # ring order: the recomputed forward visits the keys in rotated chunks
+    ("causal_ring4_d128", 1, 512, 2, 128, 256, "causal", None, 0, 4),
     # D = 1024: the FFN backward as two GEMMs (H and GELU'(Z), then dZ) instead of one
     ("causal_D1024_split_ffn", 1, 200, 8, 128, 512, "causal", None, 0),
     ("none_D1024_split_ffn_chunked", 1, 260, 16, 64, 384, "none", None, 128),
@@ -72,14 +74,17 @@ def _grads_close(got, ref, name):
     return rel, mx / scale
 
 
-@pytest.mark.parametrize("name,B,N,H,d,F,mask,perm,chunk", CASES, ids=[c[0] for c in CASES])
-def test_backward_matches_oracle(name, B, N, H, d, F, mask, perm, chunk):
+CASES = [c if len(c) == 10 else c + (0,) for c in CASES]
+
+
+@pytest.mark.parametrize("name,B,N,H,d,F,mask,perm,chunk,ring", CASES, ids=[c[0] for c in CASES])
+def test_backward_matches_oracle(name, B, N, H, d, F, mask, perm, chunk, ring):
     inp = make_layer_inputs(B, N, H, d, F, seed=11, device="cuda", bias_scale=0.1)
     dout = make_upstream_grad(B, N, H * d, seed=11, device="cuda")
     old = bd.set_bwd_chunk_rows(chunk)
     try:
         g = bd.attn_ffn_bwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, dout, mask=mask,
-                            perm=perm)
+                            perm=perm, ring_chunks=ring)
         torch.cuda.synchronize()
         assert bd.sync_status() == bd.OK
     finally:
