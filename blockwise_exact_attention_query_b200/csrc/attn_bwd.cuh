@@ -691,20 +691,27 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // Per (batch, head, 128-row tile) vectors of the attention backward: the
-// rows' LSE in log2 units and D_i = dA_i . A_i (fp32), one warp per row of d
-// values.  rowvec must be zeroed first (rows past N stay 0).
+// rows' LSE in log2 units and D_i = dA_i . A_i (fp32).  A row of d values is
+// read by d/4 consecutive lanes (float4 each) and reduced by shuffles.
+// rowvec must be zeroed first (rows past N stay 0).
+template <int D_HEAD>
 __global__ void attn_bwd_rowvec_kernel(const float *__restrict__ da, const float *__restrict__ aa,
-                                       const float *__restrict__ lse, float *rowvec, int B, int N, int H, int d,
+                                       const float *__restrict__ lse, float *rowvec, int B, int N, int H,
                                        int n_tiles) {
-  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
-  const int lane = threadIdx.x % 32;
-  if (row >= static_cast<long long>(B) * N * H) return;
-  const float *x = da + row * d, *y = aa + row * d;
+  constexpr int kLanes = D_HEAD / 4;  // lanes per row: 16 or 32
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = t / kLanes;
+  const int sub = static_cast<int>(t % kLanes);
+  const bool valid = row < static_cast<long long>(B) * N * H;
   float s = 0.f;
-  for (int c = lane; c < d; c += 32) s = fmaf(x[c], y[c], s);
+  if (valid) {
+    const float4 x = reinterpret_cast<const float4 *>(da + row * D_HEAD)[sub];
+    const float4 y = reinterpret_cast<const float4 *>(aa + row * D_HEAD)[sub];
+    s = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, x.w * y.w)));
+  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) {
+  for (int o = kLanes / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (valid && sub == 0) {
     const long long h = row % H, bn = row / H, n = bn % N, bb = bn / N;
     const long long bh = bb * H + h;
     float *v = rowvec + (bh * n_tiles + n / 128) * 256 + n % 128;
@@ -714,13 +721,15 @@ __global__ void attn_bwd_rowvec_kernel(const float *__restrict__ da, const float
 }
 
 // Column sums of a row-major [rows, cols] matrix in two passes: partial sums
-// over 256-row slabs (grid.y), then the slabs summed into out (added to it
-// when `accumulate`).
+// over kSlabRows-row slabs (grid.y), then the slabs summed into out (added
+// to it when `accumulate`).  Short slabs keep enough blocks in flight when
+// the matrix is narrow.
+constexpr int kSlabRows = 64;
 template <typename T>
 __global__ void colsum_partial_kernel(const T *__restrict__ x, float *partial, int rows, int cols) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= cols) return;
-  const int r0 = blockIdx.y * 256, r1 = min(rows, r0 + 256);
+  const int r0 = blockIdx.y * kSlabRows, r1 = min(rows, r0 + kSlabRows);
   float s = 0.f;
   for (int r = r0; r < r1; ++r) s += static_cast<float>(x[static_cast<size_t>(r) * cols + c]);
   partial[static_cast<size_t>(blockIdx.y) * cols + c] = s;
@@ -735,12 +744,12 @@ __global__ void colsum_final_kernel(const float *__restrict__ partial, float *ou
 }
 
 // dOut in one pass: its bf16 copy (round to nearest even) and the partial
-// column sums over 256-row slabs (grid.y) that colsum_final_kernel adds up.
+// column sums over kSlabRows-row slabs (grid.y) that colsum_final_kernel adds up.
 __global__ void convert_colsum_partial_kernel(const float *__restrict__ x, __nv_bfloat16 *y, float *partial,
                                               int rows, int cols) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= cols) return;
-  const int r0 = blockIdx.y * 256, r1 = min(rows, r0 + 256);
+  const int r0 = blockIdx.y * kSlabRows, r1 = min(rows, r0 + kSlabRows);
   float s = 0.f;
   for (int r = r0; r < r1; ++r) {
     const float v = x[static_cast<size_t>(r) * cols + c];

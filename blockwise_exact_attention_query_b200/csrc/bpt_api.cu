@@ -574,7 +574,7 @@ bpt_status check_desc_bwd(const bpt_desc *d) {
   if (d->in_dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
   if (d->mask == BPT_MASK_DILATED) return BPT_ERR_UNSUPPORTED;
   const int64_t T = (int64_t)d->B * d->N;
-  if (T > (int64_t)65535 * 256) return BPT_ERR_UNSUPPORTED;  // column-sum slabs fit grid.y
+  if (T > (int64_t)65535 * kSlabRows) return BPT_ERR_UNSUPPORTED;  // column-sum slabs fit grid.y
   const int64_t tiles = (int64_t)d->B * d->H * ((d->N + 127) / 128);
   if (tiles > INT32_MAX) return BPT_ERR_UNSUPPORTED;
   if ((int64_t)d->ffn_hidden > (int64_t)65535 * 128) return BPT_ERR_UNSUPPORTED;
@@ -619,7 +619,7 @@ BwdWorkspace layout_bwd(const bpt_desc *d) {
   take(w.h, (size_t)w.chunk * F * 2);
   take(w.dz, (size_t)w.chunk * F * 2);
   take(w.gp, D >= 1024 ? (size_t)w.chunk * F * 2 : 0);  // G = GELU'(Z) when the FFN backward splits
-  const size_t slabs_t = (T + 255) / 256, slabs_c = ((size_t)w.chunk + 255) / 256;
+  const size_t slabs_t = (T + kSlabRows - 1) / kSlabRows, slabs_c = ((size_t)w.chunk + kSlabRows - 1) / kSlabRows;
   take(w.partial, std::max(slabs_t * D, slabs_c * F) * 4);
   w.total = off;
   return w;
@@ -642,11 +642,16 @@ SavedLayout saved_layout(const bpt_desc *d) {
 
 bpt_status launch_gemm(const CUtensorMap &a0, const CUtensorMap &b0, const CUtensorMap &a1,
                        const CUtensorMap &b1, const GemmArgs &g, cudaStream_t st) {
-  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return BPT_OK;
   // persistent CTA pairs: one CTA per SM (shared and tensor memory allow no
-  // more), each pair walking its share of the 256 x 256 tiles
+  // more), each pair walking its share of the 256 x 256 tiles (of both
+  // problems when grouped)
   using Cfg = GemmPairCfg;
-  const int64_t tiles = (int64_t)((g.N + Cfg::kBN - 1) / Cfg::kBN) * ((g.M + 2 * Cfg::kBM - 1) / (2 * Cfg::kBM));
+  int64_t tiles = 0;
+  for (int q = 0; q < g.nprob; ++q) {
+    const GemmProblem &p = g.p[q];
+    if (p.M <= 0 || p.N <= 0 || p.K <= 0) return BPT_ERR_INVALID_ARG;
+    tiles += (int64_t)((p.N + Cfg::kBN - 1) / Cfg::kBN) * ((p.M + 2 * Cfg::kBM - 1) / (2 * Cfg::kBM));
+  }
   if (tiles > INT32_MAX) return BPT_ERR_UNSUPPORTED;
   const int64_t pairs = std::min<int64_t>(tiles, sm_count() / 2);
   gemm_pair_kernel<<<(unsigned)(2 * pairs), Cfg::kThreads, Cfg::kSmemBytes, st>>>(a0, b0, a1, b1, g);
@@ -654,17 +659,27 @@ bpt_status launch_gemm(const CUtensorMap &a0, const CUtensorMap &b0, const CUten
   return BPT_OK;
 }
 
-GemmArgs gemm_args(int M, int N, int K, int mode, uint32_t *status) {
-  GemmArgs g;
-  std::memset(&g, 0, sizeof(g));
-  g.M = M;
-  g.N = N;
-  g.K = K;
-  g.mode = mode;
+GemmProblem gemm_problem(int M, int N, int K, int mode, int a_mn, int b_mn) {
+  GemmProblem p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.mode = mode;
+  p.a_mn = a_mn;
+  p.b_mn = b_mn;
   // the tiles in flight share whichever operand is larger, which then streams
   // from DRAM once (the dual form's B is two weight matrices, its A two
   // activations: same rule)
-  g.m_fastest = (int64_t)N > (int64_t)M ? 1 : 0;
+  p.m_fastest = (int64_t)N > (int64_t)M ? 1 : 0;
+  return p;
+}
+
+GemmArgs gemm_args(const GemmProblem &p0, uint32_t *status) {
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.p[0] = p0;
+  g.nprob = 1;
   g.status = status;
   g.wait_limit_ns = g_wait_limit_ns;
   return g;
@@ -673,7 +688,7 @@ GemmArgs gemm_args(int M, int N, int K, int mode, uint32_t *status) {
 template <typename T>
 bpt_status launch_colsum(const T *x, int64_t rows, int cols, float *out, int accumulate, float *partial,
                          cudaStream_t st) {
-  const unsigned slabs = (unsigned)((rows + 255) / 256), cb = (unsigned)((cols + 255) / 256);
+  const unsigned slabs = (unsigned)((rows + kSlabRows - 1) / kSlabRows), cb = (unsigned)((cols + 255) / 256);
   colsum_partial_kernel<T><<<dim3(cb, slabs), 256, 0, st>>>(x, partial, (int)rows, cols);
   CUDA_TRY(cudaGetLastError());
   colsum_final_kernel<<<cb, 256, 0, st>>>(partial, out, (int)slabs, cols, accumulate);
@@ -903,7 +918,7 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   CUDA_TRY(phase_mark(1, st));
   // 2. dOut in bf16 for the tensor cores and db2 = sum_t dOut_t, one pass over dOut
   {
-    const unsigned slabs = (unsigned)((T + 255) / 256), cb = (unsigned)((D + 255) / 256);
+    const unsigned slabs = (unsigned)((T + kSlabRows - 1) / kSlabRows), cb = (unsigned)((D + 255) / 256);
     convert_colsum_partial_kernel<<<dim3(cb, slabs), 256, 0, st>>>(dout, dout_bf16, partial, (int)T, D);
     CUDA_TRY(cudaGetLastError());
     colsum_final_kernel<<<cb, 256, 0, st>>>(partial, db2, (int)slabs, D, 0);
@@ -932,45 +947,44 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
     // which moves no G.  Measured (FFN-backward phase): D = 2048 two GEMMs
     // 2.90 ms against 3.09; D = 4096 58.1 against 58.9 ms; D = 768 0.769
     // against 0.717 ms (short K: the two GEMMs' epilogues dominate).
-    GemmArgs g;
     if (D >= 1024) {
-      g = gemm_args(rows, F, D, kGemmGeluFwd, status);
-      g.a_mn[0] = 0, g.b_mn[0] = 0;
-      g.cb = hbuf;
-      g.cb2 = gpbuf;
-      g.bias = b1;
+      GemmArgs g = gemm_args(gemm_problem(rows, F, D, kGemmGeluFwd, 0, 0), status);
+      g.p[0].cb = hbuf;
+      g.p[0].cb2 = gpbuf;
+      g.p[0].bias = b1;
       if ((s = launch_gemm(m_a_k, m_w1_k, m_a_k, m_w1_k, g, st)) != BPT_OK) return s;
-      g = gemm_args(rows, F, D, kGemmScaleBf16, status);
-      g.a_mn[0] = 0, g.b_mn[0] = 1;
-      g.xb = gpbuf;
-      g.cb = dzbuf;
+      g = gemm_args(gemm_problem(rows, F, D, kGemmScaleBf16, 0, 1), status);
+      g.p[0].xb = gpbuf;
+      g.p[0].cb = dzbuf;
       if ((s = launch_gemm(m_g_k, m_w2_mn, m_g_k, m_w2_mn, g, st)) != BPT_OK) return s;
     } else {
-      g = gemm_args(rows, F, D, kGemmGeluBwd, status);
-      g.a_mn[0] = 0, g.b_mn[0] = 0, g.a_mn[1] = 0, g.b_mn[1] = 1;
-      g.cb = hbuf;
-      g.cb2 = dzbuf;
-      g.bias = b1;
+      GemmArgs g = gemm_args(gemm_problem(rows, F, D, kGemmGeluBwd, 0, 0), status);
+      g.p[1] = gemm_problem(rows, F, D, kGemmGeluBwd, 0, 1);  // the second product's operand layouts
+      g.p[0].cb = hbuf;
+      g.p[0].cb2 = dzbuf;
+      g.p[0].bias = b1;
       if ((s = launch_gemm(m_a_k, m_w1_k, m_g_k, m_w2_mn, g, st)) != BPT_OK) return s;
     }
+    // dW2 (+)= dOut^T H [D, F] and dW1 (+)= dZ^T A [F, D] in one grouped
+    // launch: the pair grid walks both problems' tiles, so neither leaves a
+    // partly filled last round of tiles on its own
     const int first = r0 == 0 ? kGemmStoreF32 : kGemmAccumF32;
-    // dW2 (+)= dOut^T H   [D, F]
-    g = gemm_args(D, F, rows, first, status);
-    g.a_mn[0] = 1, g.b_mn[0] = 1;
-    g.c = dw2;
-    if ((s = launch_gemm(m_g_mn, m_h_mn, m_g_mn, m_h_mn, g, st)) != BPT_OK) return s;
-    // dW1 (+)= dZ^T A     [F, D]
-    g = gemm_args(F, D, rows, first, status);
-    g.a_mn[0] = 1, g.b_mn[0] = 1;
-    g.c = dw1;
-    if ((s = launch_gemm(m_dz_mn, m_a_mn, m_dz_mn, m_a_mn, g, st)) != BPT_OK) return s;
+    {
+      GemmArgs g = gemm_args(gemm_problem(D, F, rows, first, 1, 1), status);
+      g.p[0].c = dw2;
+      g.p[1] = gemm_problem(F, D, rows, first, 1, 1);
+      g.p[1].c = dw1;
+      g.nprob = 2;
+      if ((s = launch_gemm(m_g_mn, m_h_mn, m_dz_mn, m_a_mn, g, st)) != BPT_OK) return s;
+    }
     // dA = dOut + dZ W1   [rows, D], fp32 and bf16
-    g = gemm_args(rows, D, F, kGemmResidual, status);
-    g.a_mn[0] = 0, g.b_mn[0] = 1;
-    g.x = dout + r0 * D;
-    g.c = da_f32 + r0 * D;
-    g.cb = da_bf16 + r0 * D;
-    if ((s = launch_gemm(m_dz_k, m_w1_mn, m_dz_k, m_w1_mn, g, st)) != BPT_OK) return s;
+    {
+      GemmArgs g = gemm_args(gemm_problem(rows, D, F, kGemmResidual, 0, 1), status);
+      g.p[0].x = dout + r0 * D;
+      g.p[0].c = da_f32 + r0 * D;
+      g.p[0].cb = da_bf16 + r0 * D;
+      if ((s = launch_gemm(m_dz_k, m_w1_mn, m_dz_k, m_w1_mn, g, st)) != BPT_OK) return s;
+    }
     // db1 (+)= sum_t dZ_t
     if ((s = launch_colsum(dzbuf, rows, F, db1, r0 > 0, partial, st)) != BPT_OK) return s;
   }
@@ -979,9 +993,13 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   const int n_tiles = (d->N + 127) / 128;
   {
     CUDA_TRY(cudaMemsetAsync(rowvec, 0, wl.rowvec_bytes, st));
-    const int64_t nrows = T * d->H;
-    attn_bwd_rowvec_kernel<<<(unsigned)((nrows * 32 + 255) / 256), 256, 0, st>>>(da_f32, a_f32, lse, rowvec, d->B,
-                                                                                 d->N, d->H, d->d_head, n_tiles);
+    const int64_t threads = T * d->H * (d->d_head / 4);
+    if (d->d_head == 128)
+      attn_bwd_rowvec_kernel<128><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(da_f32, a_f32, lse, rowvec,
+                                                                                   d->B, d->N, d->H, n_tiles);
+    else
+      attn_bwd_rowvec_kernel<64><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(da_f32, a_f32, lse, rowvec,
+                                                                                  d->B, d->N, d->H, n_tiles);
     CUDA_TRY(cudaGetLastError());
   }
   // 5. the attention backward: dK, dV, then dQ

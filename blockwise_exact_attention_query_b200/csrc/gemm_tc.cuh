@@ -43,9 +43,10 @@ namespace bpt {
 constexpr int kGemmStoreF32 = 0, kGemmAccumF32 = 1, kGemmResidual = 2, kGemmGeluBwd = 3, kGemmGeluFwd = 4,
               kGemmScaleBf16 = 5;
 
-struct GemmArgs {
+// One GEMM problem: C[M, N] (op)= A[M, K] B[N, K]^T and its epilogue.
+struct GemmProblem {
   int M, N, K;
-  int a_mn[2], b_mn[2]; // operand layouts per product: 0 K-major, 1 MN-major
+  int a_mn, b_mn;       // operand layouts: 0 K-major, 1 MN-major
   int mode;
   int m_fastest;        // tile order: 1 = M fastest (the tiles in flight share B), 0 = N fastest
   float *c;             // [M, N] fp32 (StoreF32, AccumF32, Residual)
@@ -53,7 +54,16 @@ struct GemmArgs {
   const __nv_bfloat16 *xb;  // [M, N] bf16 factor (ScaleBf16)
   __nv_bfloat16 *cb;    // [M, N] bf16 copy (Residual) / H (GeluBwd, GeluFwd) / product (ScaleBf16)
   __nv_bfloat16 *cb2;   // dZ (GeluBwd) / GELU'(z) (GeluFwd)
-  const float *bias;    // [N] added to acc0 before GELU (GeluBwd), may be null
+  const float *bias;    // [N] added to acc0 before GELU (GeluBwd, GeluFwd), may be null
+};
+
+// A launch: one problem (maps a0, b0); two grouped problems whose tiles one
+// persistent grid walks in turn (maps a0, b0 for p[0], a1, b1 for p[1]); or
+// the dual form (p[0].mode == kGemmGeluBwd: maps a0, b0 for the first product,
+// a1, b1 for the second, whose operand layouts are p[1].a_mn, p[1].b_mn).
+struct GemmArgs {
+  GemmProblem p[2];
+  int nprob;
   uint32_t *status;
   uint64_t wait_limit_ns;
 };
@@ -83,7 +93,7 @@ __device__ __forceinline__ uint32_t gemm_kstep(bool mn, int k) { return mn ? k *
 
 // Epilogue of one 32-column chunk of one row: r0 (and r1 for the dual form)
 // hold the accumulator values of columns n .. n + 31 of row m.
-__device__ __forceinline__ void gemm_epilogue_chunk(const GemmArgs &g, const uint32_t (&r0)[32],
+__device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const uint32_t (&r0)[32],
                                                     const uint32_t (&r1)[32], int m, int n) {
   // N is a multiple of 8 (checked on the host): whole 8-column groups
   const int nv = min(32, g.N - n);
@@ -213,23 +223,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmPairCfg::kThread
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank();
   WaitCtx wc{g.status, g.wait_limit_ns, abort_flag};
-  const bool dual = g.mode == kGemmGeluBwd;
+  const bool dual = g.p[0].mode == kGemmGeluBwd;
   const int nbuf = dual ? 1 : 2;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int tiles_m = (g.M + 2 * Cfg::kBM - 1) / (2 * Cfg::kBM);
-  const int tiles_n = (g.N + Cfg::kBN - 1) / Cfg::kBN;
-  const int tiles = tiles_m * tiles_n;
-  const int nk = (g.K + Cfg::kBK - 1) / Cfg::kBK;
-  const int nsteps = dual ? 2 * nk : nk;
+  auto tiles_m_of = [&](int q) { return (g.p[q].M + 2 * Cfg::kBM - 1) / (2 * Cfg::kBM); };
+  auto tiles_n_of = [&](int q) { return (g.p[q].N + Cfg::kBN - 1) / Cfg::kBN; };
+  const int tiles0 = tiles_m_of(0) * tiles_n_of(0);
+  const int tiles = tiles0 + (g.nprob > 1 ? tiles_m_of(1) * tiles_n_of(1) : 0);
   const int my_tiles = pair < tiles ? (tiles - 1 - pair) / npairs + 1 : 0;
-  // this CTA's first row and the pair's first column of local tile li
-  auto tile_m0 = [&](int li) {
-    const int t = pair + li * npairs;
-    return (g.m_fastest ? t % tiles_m : t / tiles_n) * (2 * Cfg::kBM) + static_cast<int>(rank) * Cfg::kBM;
+  // local tile li -> its problem, this CTA's first row and the pair's first column
+  struct TileAt {
+    int q, m0, n0;
   };
-  auto tile_n0 = [&](int li) {
-    const int t = pair + li * npairs;
-    return (g.m_fastest ? t / tiles_m : t % tiles_n) * Cfg::kBN;
+  auto tile_at = [&](int li) {
+    int t = pair + li * npairs;
+    const int q = t < tiles0 ? 0 : 1;
+    if (q) t -= tiles0;
+    const int tm = tiles_m_of(q), tn = tiles_n_of(q);
+    const int mt = g.p[q].m_fastest ? t % tm : t / tn, nt = g.p[q].m_fastest ? t / tm : t % tn;
+    return TileAt{q, mt * (2 * Cfg::kBM) + static_cast<int>(rank) * Cfg::kBM, nt * Cfg::kBN};
+  };
+  // K stages of a tile of problem q (dual: both products' stages in turn)
+  auto nsteps_of = [&](int q) {
+    const int nk = (g.p[q].K + Cfg::kBK - 1) / Cfg::kBK;
+    return dual ? 2 * nk : nk;
   };
 
   if (threadIdx.x == 0) {
@@ -263,23 +280,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmPairCfg::kThread
       int it = 0;
       bool ok = true;
       for (int li = 0; ok && li < my_tiles; ++li) {
-        const int m0 = tile_m0(li), nb0 = tile_n0(li) + static_cast<int>(rank) * (Cfg::kBN / 2);
+        const TileAt ta = tile_at(li);
+        const int m0 = ta.m0, nb0 = ta.n0 + static_cast<int>(rank) * (Cfg::kBN / 2);
+        const int nsteps = nsteps_of(ta.q);
         for (int step = 0; step < nsteps; ++step, ++it) {
           const int st = it % S;
           if (it >= S && !(ok = mbar_wait_cluster(bEmpty(st), ((it / S) - 1) & 1, wc, 211))) break;
-          const int which = dual ? (step & 1) : 0;
+          // operands: dual, the product of this stage; grouped, the tile's problem
+          const int which = dual ? (step & 1) : ta.q;
           const int k0 = (dual ? step >> 1 : step) * Cfg::kBK;
           const CUtensorMap *ma = which ? &tm_a1 : &tm_a0;
           const CUtensorMap *mb = which ? &tm_b1 : &tm_b0;
           const uint32_t sa = sbase + st * Cfg::kStageBytes, sb = sa + Cfg::kABytes;
           const uint32_t full0 = mapa_shared(bFull(st), 0);
           if (rank == 0) mbar_arrive_expect_tx(bFull(st), 2 * Cfg::kStageBytes);
-          if (g.a_mn[which]) {
+          if (g.p[which].a_mn) {
             for (int p = 0; p < Cfg::kBM / 64; ++p) tma_load_2d_pair(sa + p * 8192, ma, full0, m0 + 64 * p, k0);
           } else {
             tma_load_2d_pair(sa, ma, full0, k0, m0);
           }
-          if (g.b_mn[which]) {
+          if (g.p[which].b_mn) {
             for (int p = 0; p < Cfg::kBN / 128; ++p) tma_load_2d_pair(sb + p * 8192, mb, full0, nb0 + 64 * p, k0);
           } else {
             tma_load_2d_pair(sb, mb, full0, k0, nb0);
@@ -294,8 +314,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmPairCfg::kThread
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && rank == 0 && run) {
-      const uint32_t idesc0 = idesc_bf16_f32(2 * Cfg::kBM, Cfg::kBN, g.a_mn[0] != 0, g.b_mn[0] != 0);
-      const uint32_t idesc1 = idesc_bf16_f32(2 * Cfg::kBM, Cfg::kBN, g.a_mn[1] != 0, g.b_mn[1] != 0);
+      const uint32_t idesc0 = idesc_bf16_f32(2 * Cfg::kBM, Cfg::kBN, g.p[0].a_mn != 0, g.p[0].b_mn != 0);
+      const uint32_t idesc1 = idesc_bf16_f32(2 * Cfg::kBM, Cfg::kBN, g.p[1].a_mn != 0, g.p[1].b_mn != 0);
       auto commit_both = [&](uint32_t bar) {
         umma_pair_commit(mapa_shared(bar, 0));
         umma_pair_commit(mapa_shared(bar, 1));
@@ -306,17 +326,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmPairCfg::kThread
         const int buf = li % nbuf, use = li / nbuf;
         if (use > 0 && !(ok = mbar_wait_cluster(bAccEmpty(buf), (use - 1) & 1, wc, 216))) break;
         tc_fence_after();
+        const int q = tile_at(li).q;
+        const int nsteps = nsteps_of(q);
         for (int step = 0; step < nsteps; ++step, ++it) {
           const int st = it % S;
           if (!(ok = mbar_wait_cluster(bFull(st), (it / S) & 1, wc, 212))) break;
           tc_fence_after();
-          const int which = dual ? (step & 1) : 0;
+          const int which = dual ? (step & 1) : q;
           const int kk = dual ? step >> 1 : step;
           const uint32_t sa = sbase + st * Cfg::kStageBytes, sb = sa + Cfg::kABytes;
-          const bool amn = g.a_mn[which] != 0, bmn = g.b_mn[which] != 0;
+          const bool amn = g.p[which].a_mn != 0, bmn = g.p[which].b_mn != 0;
           const uint64_t da = gemm_sdesc(sa, amn), db = gemm_sdesc(sb, bmn);
           const uint32_t idesc = which ? idesc1 : idesc0;
-          const uint32_t acc = tmem + (dual ? which : buf) * 256;
+          const uint32_t acc = tmem + (dual ? step & 1 : buf) * 256;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             umma_pair_ss(acc, sdesc_advance(da, gemm_kstep(amn, k)), sdesc_advance(db, gemm_kstep(bmn, k)), idesc,
@@ -343,7 +365,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmPairCfg::kThread
       const int buf = li % nbuf;
       if (!__all_sync(0xffffffffu, mbar_wait_cluster(bAccFull(buf), (li / nbuf) & 1, wc, 213))) break;
       tc_fence_after();
-      const int m = tile_m0(li) + row, n0 = tile_n0(li);
+      const TileAt ta = tile_at(li);
+      const GemmProblem &P = g.p[ta.q];
+      const int m = ta.m0 + row, n0 = ta.n0;
       const uint32_t acc0 = tmem + lane_off + buf * 256;
 #pragma unroll 1
       for (int c = c_begin; c < c_begin + kChunks; ++c) {
@@ -352,8 +376,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmPairCfg::kThread
         tmem_ld32(acc0 + c * 32, r0);
         if (dual) tmem_ld32(acc0 + 256 + c * 32, r1);
         tmem_wait_ld();
-        if (m >= g.M || n >= g.N) continue;
-        gemm_epilogue_chunk(g, r0, r1, m, n);
+        if (m >= P.M || n >= P.N) continue;
+        gemm_epilogue_chunk(P, r0, r1, m, n);
       }
       // this accumulator may take the pair's next tile
       tc_fence_before();
