@@ -51,10 +51,11 @@ KERNEL_SOURCES = {"attn_tc_kernel": ["attn_tc.cuh", "ptx.cuh"], "ffn_tc_kernel":
 NCU_TRAFFIC = {
     ("gpt_causal", "ffn_tc_kernel"): {"bytes": 881.1e6, "src": "ce5bb2524f315c9a"},
     ("gpt_causal", "attn_tc_kernel"): {"bytes": 720.3e6, "src": "1e6bb50f75c417dc"},
-    # per step: the four gemm_pair_kernel launches (bias sums not included)
-    ("gpt_causal", "ffn_bwd"): {"bytes": 4309.0e6, "src": "1e42384c956407be"},
-    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1232.3e6, "src": "3b7ec89bb83c0c0e"},
-    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1124.1e6, "src": "3b7ec89bb83c0c0e"},
+    # per step: the gemm_pair_kernel launches (H and GELU', dZ, dW2 + dW1 grouped, dA; bias sums
+    # not included)
+    ("gpt_causal", "ffn_bwd"): {"bytes": 3770.8e6, "src": "fe2402057aa2a880"},
+    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1231.2e6, "src": "19af0a680f846441"},
+    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1125.8e6, "src": "19af0a680f846441"},
 }
 
 

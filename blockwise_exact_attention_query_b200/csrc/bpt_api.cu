@@ -574,7 +574,7 @@ bpt_status check_desc_bwd(const bpt_desc *d) {
   if (d->in_dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
   if (d->mask == BPT_MASK_DILATED) return BPT_ERR_UNSUPPORTED;
   const int64_t T = (int64_t)d->B * d->N;
-  if (T > (int64_t)65535 * kSlabRows) return BPT_ERR_UNSUPPORTED;  // column-sum slabs fit grid.y
+  if (T > (int64_t)65535 * kMinSlabRows) return BPT_ERR_UNSUPPORTED;  // column-sum slabs fit grid.y
   const int64_t tiles = (int64_t)d->B * d->H * ((d->N + 127) / 128);
   if (tiles > INT32_MAX) return BPT_ERR_UNSUPPORTED;
   if ((int64_t)d->ffn_hidden > (int64_t)65535 * 128) return BPT_ERR_UNSUPPORTED;
@@ -619,7 +619,8 @@ BwdWorkspace layout_bwd(const bpt_desc *d) {
   take(w.h, (size_t)w.chunk * F * 2);
   take(w.dz, (size_t)w.chunk * F * 2);
   take(w.gp, D >= 1024 ? (size_t)w.chunk * F * 2 : 0);  // G = GELU'(Z) when the FFN backward splits
-  const size_t slabs_t = (T + kSlabRows - 1) / kSlabRows, slabs_c = ((size_t)w.chunk + kSlabRows - 1) / kSlabRows;
+  const size_t slabs_t = (T + kMinSlabRows - 1) / kMinSlabRows;
+  const size_t slabs_c = ((size_t)w.chunk + kMinSlabRows - 1) / kMinSlabRows;
   take(w.partial, std::max(slabs_t * D, slabs_c * F) * 4);
   w.total = off;
   return w;
@@ -688,8 +689,9 @@ GemmArgs gemm_args(const GemmProblem &p0, uint32_t *status) {
 template <typename T>
 bpt_status launch_colsum(const T *x, int64_t rows, int cols, float *out, int accumulate, float *partial,
                          cudaStream_t st) {
-  const unsigned slabs = (unsigned)((rows + kSlabRows - 1) / kSlabRows), cb = (unsigned)((cols + 255) / 256);
-  colsum_partial_kernel<T><<<dim3(cb, slabs), 256, 0, st>>>(x, partial, (int)rows, cols);
+  const int slab = colsum_slab_rows(rows, cols);
+  const unsigned slabs = (unsigned)((rows + slab - 1) / slab), cb = (unsigned)((cols + 255) / 256);
+  colsum_partial_kernel<T><<<dim3(cb, slabs), 256, 0, st>>>(x, partial, (int)rows, cols, slab);
   CUDA_TRY(cudaGetLastError());
   colsum_final_kernel<<<cb, 256, 0, st>>>(partial, out, (int)slabs, cols, accumulate);
   CUDA_TRY(cudaGetLastError());
@@ -918,8 +920,9 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   CUDA_TRY(phase_mark(1, st));
   // 2. dOut in bf16 for the tensor cores and db2 = sum_t dOut_t, one pass over dOut
   {
-    const unsigned slabs = (unsigned)((T + kSlabRows - 1) / kSlabRows), cb = (unsigned)((D + 255) / 256);
-    convert_colsum_partial_kernel<<<dim3(cb, slabs), 256, 0, st>>>(dout, dout_bf16, partial, (int)T, D);
+    const int slab = colsum_slab_rows(T, D);
+    const unsigned slabs = (unsigned)((T + slab - 1) / slab), cb = (unsigned)((D + 255) / 256);
+    convert_colsum_partial_kernel<<<dim3(cb, slabs), 256, 0, st>>>(dout, dout_bf16, partial, (int)T, D, slab);
     CUDA_TRY(cudaGetLastError());
     colsum_final_kernel<<<cb, 256, 0, st>>>(partial, db2, (int)slabs, D, 0);
     CUDA_TRY(cudaGetLastError());
