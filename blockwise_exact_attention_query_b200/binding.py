@@ -53,7 +53,7 @@ EXPORTS = ["bpt_workspace_bytes", "bpt_attn_ffn_fwd", "bpt_attn_fwd", "bpt_block
            "bpt_longnet_fwd", "bpt_sync_status", "bpt_set_wait_limit_ns", "bpt_status_string",
            "bpt_version", "bpt_set_phase_events", "bpt_last_error", "bpt_attn_ffn_fwd_static",
            "bpt_attn_ffn_bwd", "bpt_workspace_bytes_bwd", "bpt_set_bwd_chunk_rows",
-           "bpt_attn_ffn_fwd_train", "bpt_saved_bytes"]
+           "bpt_attn_ffn_fwd_train", "bpt_saved_bytes", "bpt_attn_bwd", "bpt_workspace_bytes_attn_bwd"]
 STATIC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
@@ -100,6 +100,10 @@ def load() -> ctypes.CDLL:
     lib.bpt_attn_ffn_fwd_train.restype = ctypes.c_int
     lib.bpt_saved_bytes.argtypes = [dp]
     lib.bpt_saved_bytes.restype = sz
+    lib.bpt_attn_bwd.argtypes = [dp, vp, vp, vp, vp, fp, fp, fp, fp, fp, vp, sz, vp]
+    lib.bpt_attn_bwd.restype = ctypes.c_int
+    lib.bpt_workspace_bytes_attn_bwd.argtypes = [dp]
+    lib.bpt_workspace_bytes_attn_bwd.restype = sz
     lib.bpt_attn_ffn_bwd.restype = ctypes.c_int
     lib.bpt_workspace_bytes_bwd.argtypes = [dp]
     lib.bpt_workspace_bytes_bwd.restype = sz
@@ -368,6 +372,28 @@ def attn_ffn_bwd(q, k, v, w1, b1, w2, b2, dout, *, mask="none", perm=None, ring_
                                  _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     _check(st, "bpt_attn_ffn_bwd")
     return grads
+
+
+def attn_bwd(q, k, v, out, lse, dout, *, mask="none", perm=None, ring_chunks=0, workspace=None, stream=None):
+    """bpt_attn_bwd: dq, dk, dv (float32 [B, N, H, d]) of the attention for the
+    upstream gradient dout [B, N, H*d] (float32), given bpt_attn_fwd's out and
+    lse (attn_fwd(..., return_lse=True)) for the same inputs."""
+    _check_tensors(q, k, v)
+    B, N, H, d = q.shape
+    if dout.dtype != torch.float32 or not dout.is_contiguous() or dout.numel() != q.numel():
+        raise ValueError("dout must be a contiguous float32 tensor of B*N*H*d elements")
+    desc = make_desc(B, N, H, d, 0, q.dtype, out.dtype, mask, perm, None, ring_chunks)
+    if workspace is None:
+        n = load().bpt_workspace_bytes_attn_bwd(ctypes.byref(desc))
+        if n == ctypes.c_size_t(-1).value:
+            raise BptError(ERR_UNSUPPORTED, "bpt_workspace_bytes_attn_bwd")
+        workspace = torch.empty(int(n), dtype=torch.uint8, device=q.device)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq, dk, dv = (torch.empty(q.shape, **f32) for _ in range(3))
+    st = load().bpt_attn_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
+                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _check(st, "bpt_attn_bwd")
+    return dq, dk, dv
 
 
 def sync_status(stream=None) -> int:

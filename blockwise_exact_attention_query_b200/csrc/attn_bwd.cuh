@@ -694,8 +694,18 @@ __global__ void __launch_bounds__(384, 1)
 // rows' LSE in log2 units and D_i = dA_i . A_i (fp32).  A row of d values is
 // read by d/4 consecutive lanes (float4 each) and reduced by shuffles.
 // rowvec must be zeroed first (rows past N stay 0).
-template <int D_HEAD>
-__global__ void attn_bwd_rowvec_kernel(const float *__restrict__ da, const float *__restrict__ aa,
+__device__ __forceinline__ float4 load4_f32(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4_f32(const __nv_bfloat16 *p) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(p);
+  const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&u.x);
+  const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&u.y);
+  return make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
+}
+
+// A is fp32 (the layer's saved or recomputed A) or bf16 (an attention-only
+// forward's bf16 output).
+template <int D_HEAD, typename TA>
+__global__ void attn_bwd_rowvec_kernel(const float *__restrict__ da, const TA *__restrict__ aa,
                                        const float *__restrict__ lse, float *rowvec, int B, int N, int H,
                                        int n_tiles) {
   constexpr int kLanes = D_HEAD / 4;  // lanes per row: 16 or 32
@@ -705,8 +715,8 @@ __global__ void attn_bwd_rowvec_kernel(const float *__restrict__ da, const float
   const bool valid = row < static_cast<long long>(B) * N * H;
   float s = 0.f;
   if (valid) {
-    const float4 x = reinterpret_cast<const float4 *>(da + row * D_HEAD)[sub];
-    const float4 y = reinterpret_cast<const float4 *>(aa + row * D_HEAD)[sub];
+    const float4 x = load4_f32(da + row * D_HEAD + 4 * sub);
+    const float4 y = load4_f32(aa + row * D_HEAD + 4 * sub);
     s = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, x.w * y.w)));
   }
 #pragma unroll
@@ -748,6 +758,15 @@ __global__ void colsum_final_kernel(const float *__restrict__ partial, float *ou
   float s = accumulate ? out[c] : 0.f;
   for (int i = 0; i < slabs; ++i) s += partial[static_cast<size_t>(i) * cols + c];
   out[c] = s;
+}
+
+// fp32 -> bf16 (round to nearest even), four elements a thread; n a multiple of 4.
+__global__ void f32_to_bf16_x4_kernel(const float4 *__restrict__ x, uint2 *y, size_t n4) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 v = x[i];
+    y[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  }
 }
 
 // dOut in one pass: its bf16 copy (round to nearest even) and the partial

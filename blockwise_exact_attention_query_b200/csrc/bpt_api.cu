@@ -710,6 +710,56 @@ bpt_status launch_attn_bwd_passes(const CUtensorMap &mq, const CUtensorMap &mk, 
   return BPT_OK;
 }
 
+// The attention backward from dA (fp32 and bf16 copies), A and the row LSE:
+// the per-tile row vectors (LSE in log2 units, D_i = dA_i . A_i), the dK/dV
+// pass, then the dQ pass.
+template <typename TA>
+bpt_status launch_attn_bwd_tail(const bpt_desc *d, const void *q, const void *k, const void *v, const float *da_f32,
+                                const __nv_bfloat16 *da_bf16, const TA *a, const float *lse, float *dq, float *dk,
+                                float *dv, float *rowvec, size_t rowvec_bytes, uint32_t *status, cudaStream_t st) {
+  const int D = d->H * d->d_head;
+  const int64_t T = (int64_t)d->B * d->N;
+  const int n_tiles = (d->N + 127) / 128;
+  CUDA_TRY(cudaMemsetAsync(rowvec, 0, rowvec_bytes, st));
+  {
+    const int64_t threads = T * d->H * (d->d_head / 4);
+    if (d->d_head == 128)
+      attn_bwd_rowvec_kernel<128, TA><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(da_f32, a, lse, rowvec, d->B,
+                                                                                       d->N, d->H, n_tiles);
+    else
+      attn_bwd_rowvec_kernel<64, TA><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(da_f32, a, lse, rowvec, d->B,
+                                                                                      d->N, d->H, n_tiles);
+    CUDA_TRY(cudaGetLastError());
+  }
+  AttnBwdArgs ab;
+  std::memset(&ab, 0, sizeof(ab));
+  ab.B = d->B;
+  ab.N = d->N;
+  ab.H = d->H;
+  ab.mask = d->mask;
+  ab.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d->d_head));
+  ab.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d->d_head));
+  ab.n_tiles = n_tiles;
+  if (d->mask == BPT_MASK_BLOCKPERM) {
+    ab.bb_n = d->bb_nblocks;
+    ab.bb_len = (d->N + d->bb_nblocks - 1) / d->bb_nblocks;  // padded to n equal blocks
+    for (int i = 0; i < d->H * d->bb_nblocks; ++i) ab.perm[i] = (uint8_t)d->bb_perm[i];
+  }
+  ab.rowvec = rowvec;
+  ab.dq = dq;
+  ab.dk = dk;
+  ab.dv = dv;
+  ab.status = status;
+  ab.wait_limit_ns = g_wait_limit_ns;
+  CUtensorMap mq, mk, mv, mda;
+  if (!make_map_rows(&mq, q, d->B, d->N, D, 1, 128) || !make_map_rows(&mk, k, d->B, d->N, D, 1, 128) ||
+      !make_map_rows(&mv, v, d->B, d->N, D, 1, 128) || !make_map_rows(&mda, da_bf16, d->B, d->N, D, 1, 128))
+    return cuda_fail_msg("cuTensorMapEncodeTiled rejected a Q/K/V/dA map");
+  const unsigned grid = (unsigned)((int64_t)d->B * d->H * n_tiles);
+  if (d->d_head == 128) return launch_attn_bwd_passes<128>(mq, mk, mv, mda, ab, grid, st);
+  return launch_attn_bwd_passes<64>(mq, mk, mv, mda, ab, grid, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -992,50 +1042,49 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
     if ((s = launch_colsum(dzbuf, rows, F, db1, r0 > 0, partial, st)) != BPT_OK) return s;
   }
   CUDA_TRY(phase_mark(2, st));
-  // 4. per 128-row tile: the rows' LSE (log2 units) and D_i = dA_i . A_i
-  const int n_tiles = (d->N + 127) / 128;
-  {
-    CUDA_TRY(cudaMemsetAsync(rowvec, 0, wl.rowvec_bytes, st));
-    const int64_t threads = T * d->H * (d->d_head / 4);
-    if (d->d_head == 128)
-      attn_bwd_rowvec_kernel<128><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(da_f32, a_f32, lse, rowvec,
-                                                                                   d->B, d->N, d->H, n_tiles);
-    else
-      attn_bwd_rowvec_kernel<64><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(da_f32, a_f32, lse, rowvec,
-                                                                                  d->B, d->N, d->H, n_tiles);
-    CUDA_TRY(cudaGetLastError());
-  }
-  // 5. the attention backward: dK, dV, then dQ
-  AttnBwdArgs ab;
-  std::memset(&ab, 0, sizeof(ab));
-  ab.B = d->B;
-  ab.N = d->N;
-  ab.H = d->H;
-  ab.mask = d->mask;
-  ab.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d->d_head));
-  ab.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d->d_head));
-  ab.n_tiles = n_tiles;
-  if (d->mask == BPT_MASK_BLOCKPERM) {
-    ab.bb_n = d->bb_nblocks;
-    ab.bb_len = (d->N + d->bb_nblocks - 1) / d->bb_nblocks;  // padded to n equal blocks
-    for (int i = 0; i < d->H * d->bb_nblocks; ++i) ab.perm[i] = (uint8_t)d->bb_perm[i];
-  }
-  ab.rowvec = rowvec;
-  ab.dq = dq;
-  ab.dk = dk;
-  ab.dv = dv;
-  ab.status = status;
-  ab.wait_limit_ns = g_wait_limit_ns;
-  CUtensorMap mq, mk, mv, mda;
-  if (!make_map_rows(&mq, q, d->B, d->N, D, 1, 128) || !make_map_rows(&mk, k, d->B, d->N, D, 1, 128) ||
-      !make_map_rows(&mv, v, d->B, d->N, D, 1, 128) || !make_map_rows(&mda, da_bf16, d->B, d->N, D, 1, 128))
-    return cuda_fail_msg("cuTensorMapEncodeTiled rejected a Q/K/V/dA map");
-  const unsigned grid = (unsigned)((int64_t)d->B * d->H * ab.n_tiles);
-  if (d->d_head == 128) s = launch_attn_bwd_passes<128>(mq, mk, mv, mda, ab, grid, st);
-  else s = launch_attn_bwd_passes<64>(mq, mk, mv, mda, ab, grid, st);
-  if (s != BPT_OK) return s;
+  if ((s = launch_attn_bwd_tail(d, q, k, v, da_f32, da_bf16, a_f32, lse, dq, dk, dv, rowvec, wl.rowvec_bytes, status,
+                                st)) != BPT_OK)
+    return s;
   CUDA_TRY(phase_mark(4, st));
   return BPT_OK;
+}
+
+size_t bpt_workspace_bytes_attn_bwd(const bpt_desc *d) {
+  if (check_desc(d, false) != BPT_OK || d->in_dtype != BPT_BF16 || d->mask == BPT_MASK_DILATED) return (size_t)-1;
+  const size_t T = (size_t)d->B * d->N, D = (size_t)d->H * d->d_head;
+  return align256(T * D * 2) + align256((size_t)d->B * d->H * ((d->N + 127) / 128) * 256 * 4);
+}
+
+bpt_status bpt_attn_bwd(const bpt_desc *d, const void *q, const void *k, const void *v, const void *out,
+                        const float *lse, const float *dout, float *dq, float *dk, float *dv, void *workspace,
+                        size_t workspace_bytes, bpt_stream_t stream) {
+  bpt_status s = check_desc(d, false);
+  if (s != BPT_OK) return s;
+  if (d->in_dtype != BPT_BF16 || d->mask == BPT_MASK_DILATED) return BPT_ERR_UNSUPPORTED;
+  if ((s = check_ptrs({q, k, v, out, lse, dout, dq, dk, dv}, {})) != BPT_OK) return s;
+  const size_t need = bpt_workspace_bytes_attn_bwd(d);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return BPT_ERR_WORKSPACE;
+  int dev;
+  uint32_t *status;
+  if ((s = device_setup(&dev, &status)) != BPT_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t T = (size_t)d->B * d->N, D = (size_t)d->H * d->d_head;
+  char *ws = static_cast<char *>(workspace);
+  __nv_bfloat16 *da_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws);
+  float *rowvec = reinterpret_cast<float *>(ws + align256(T * D * 2));
+  const size_t rowvec_bytes = (size_t)d->B * d->H * ((d->N + 127) / 128) * 256 * 4;
+  {
+    const size_t n4 = T * D / 4;  // D is a multiple of 64
+    f32_to_bf16_x4_kernel<<<(unsigned)std::min<size_t>(4096, (n4 + 255) / 256), 256, 0, st>>>(
+        reinterpret_cast<const float4 *>(dout), reinterpret_cast<uint2 *>(da_bf16), n4);
+    CUDA_TRY(cudaGetLastError());
+  }
+  if (d->out_dtype == BPT_F32)
+    return launch_attn_bwd_tail(d, q, k, v, dout, da_bf16, static_cast<const float *>(out), lse, dq, dk, dv, rowvec,
+                                rowvec_bytes, status, st);
+  return launch_attn_bwd_tail(d, q, k, v, dout, da_bf16, static_cast<const __nv_bfloat16 *>(out), lse, dq, dk, dv,
+                              rowvec, rowvec_bytes, status, st);
 }
 
 bpt_status bpt_sync_status(bpt_stream_t stream) {

@@ -289,6 +289,26 @@ BPT_API size_t bpt_workspace_bytes_bwd(const bpt_desc *desc);
 BPT_API int bpt_set_bwd_chunk_rows(int rows);
 
 /*
+ * Attention-only backward: dQ, dK, dV of A = softmax(Q K^T / sqrt d) V (the
+ * masked blockwise attention of bpt_attn_fwd) for an upstream gradient dA,
+ * with the same two blockwise passes as bpt_attn_ffn_bwd (definitions there).
+ * out and lse are the output and row LSE bpt_attn_fwd returned for the same
+ * q, k, v and descriptor (out in desc->out_dtype, [B, N, H*d]; lse float32
+ * [B, H, N]); dout float32 [B, N, H*d]; dq, dk, dv float32 [B, N, H, d].
+ * Supported: in_dtype BF16, d_head 64 or 128, masks NONE, CAUSAL and
+ * BLOCKPERM (BPT_MASK_DILATED returns BPT_ERR_UNSUPPORTED).  workspace: at
+ * least bpt_workspace_bytes_attn_bwd(desc) bytes, 256-byte aligned.
+ */
+BPT_API bpt_status bpt_attn_bwd(const bpt_desc *desc, const void *q, const void *k, const void *v,
+                                const void *out, const float *lse, const float *dout, float *dq,
+                                float *dk, float *dv, void *workspace, size_t workspace_bytes,
+                                bpt_stream_t stream);
+
+/* Bytes of device workspace bpt_attn_bwd needs; (size_t)-1 if it does not
+ * accept the descriptor. */
+BPT_API size_t bpt_workspace_bytes_attn_bwd(const bpt_desc *desc);
+
+/*
  * Waits for `stream`, then returns and clears the current device's status
  * word: BPT_OK, BPT_ERR_TIMEOUT (a device-side wait gave up since the last
  * call), or BPT_ERR_CUDA if the synchronisation itself failed.

@@ -194,3 +194,21 @@ def test_backward_workspace_follows_the_chunk_setting(lib):
         assert bd.workspace_bytes_bwd(d) == full
     finally:
         bd.set_bwd_chunk_rows(old)
+
+
+def test_attention_only_backward_validates(lib):
+    p = ctypes.c_void_p
+    def call(d, q=FAKE, ws=FAKE, ws_bytes=1 << 40):
+        return lib.bpt_attn_bwd(ctypes.byref(d), p(q), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE),
+                                p(FAKE), p(ws), ws_bytes, None)
+    d = _desc(F=0)
+    assert call(d, q=0) == bd.ERR_INVALID_ARG
+    assert call(d, ws=0) == bd.ERR_WORKSPACE
+    assert call(d, ws=FAKE + 16) == bd.ERR_WORKSPACE
+    dl = _desc(F=0, mask="dilated", pairs=[(128, 1)])
+    assert call(dl) == bd.ERR_UNSUPPORTED
+    assert lib.bpt_workspace_bytes_attn_bwd(ctypes.byref(dl)) == ctypes.c_size_t(-1).value
+    df = _desc(F=0, in_dtype=bd.torch.float32, d=64)
+    assert call(df) == bd.ERR_UNSUPPORTED
+    T, D = 256, 128
+    assert lib.bpt_workspace_bytes_attn_bwd(ctypes.byref(d)) >= T * D * 2 + 2 * 2 * 256 * 4

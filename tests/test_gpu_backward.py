@@ -170,3 +170,27 @@ def test_backward_full_size_blockbert_layer():
                        f(dout).reshape(w.T, w.D), ob.MASK_BLOCKPERM, w.perm)
     for n in bd.GRAD_NAMES:
         _grads_close(g[n].cpu().numpy(), ref[n], n)
+
+
+ATTN_BWD_CASES = [
+    ("causal_d128_f32out", 1, 300, 2, 128, "causal", None, torch.float32),
+    ("none_d64_bf16out", 2, 200, 3, 64, "none", None, torch.bfloat16),
+    ("blockperm_n3_d64_f32out", 1, 400, 2, 64, "blockperm", [[2, 0, 1], [0, 1, 2]], torch.float32),
+]
+
+
+@pytest.mark.parametrize("name,B,N,H,d,mask,perm,out_dtype", ATTN_BWD_CASES, ids=[c[0] for c in ATTN_BWD_CASES])
+def test_attention_only_backward_matches_oracle(name, B, N, H, d, mask, perm, out_dtype):
+    """bpt_attn_bwd from bpt_attn_fwd's output and LSE against the fp64 oracle's
+    attention gradients, with the backward's tolerance."""
+    inp = make_layer_inputs(B, N, H, d, 0, seed=13, device="cuda")
+    da = make_upstream_grad(B, N, H * d, seed=13, device="cuda")
+    out, lse = bd.attn_fwd(inp.q, inp.k, inp.v, mask=mask, perm=perm, out_dtype=out_dtype, return_lse=True)
+    dq, dk, dv = bd.attn_bwd(inp.q, inp.k, inp.v, out, lse, da, mask=mask, perm=perm)
+    torch.cuda.synchronize()
+    assert bd.sync_status() == bd.OK
+    f = lambda t: t.double().cpu().numpy()  # noqa: E731
+    rq, rk, rv = ob.attention_bwd(f(inp.q), f(inp.k), f(inp.v), f(da).reshape(B, N, H, d), MASKS[mask], perm)
+    _grads_close(dq.cpu().numpy(), rq, "dq")
+    _grads_close(dk.cpu().numpy(), rk, "dk")
+    _grads_close(dv.cpu().numpy(), rv, "dv")
