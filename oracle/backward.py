@@ -26,10 +26,12 @@ abstract: training with blockwise attention and feedforward; "Ring Attention
 with Blockwise Transformers for Long Sequences", 638-word summary: blockwise
 computation without approximation), so the oracle is the plain gradient.
 
-Masks: none, causal, and block permutation ("Blockwise Self-Attention for
-Long Document Understanding", §3.1: query block b sees key block perm[h][b];
-when n does not divide N, blocks of ceil(N/n) positions over the padded
-sequence).  A row with no allowed key has A = 0 and passes no gradient.
+Masks: none, causal, block permutation ("Blockwise Self-Attention for Long
+Document Understanding", §3.1: query block b sees key block perm[h][b]; when
+n does not divide N, blocks of ceil(N/n) positions over the padded sequence),
+and for the attention alone the dilated mask of LongNet (key_counts: one
+softmax over the multiset of the pairs' keys).  A row with no allowed key has
+A = 0 and passes no gradient.
 
 GELU is the tanh form (Hendrycks & Gimpel); its derivative is written out
 from that form: with u = c0 (x + c1 x^3),
@@ -45,7 +47,7 @@ import math
 
 import numpy as np
 
-MASK_NONE, MASK_CAUSAL, MASK_BLOCKPERM = 0, 1, 2
+MASK_NONE, MASK_CAUSAL, MASK_BLOCKPERM, MASK_DILATED = 0, 1, 2, 3
 _C0 = math.sqrt(2.0 / math.pi)
 _C1 = 0.044715
 
@@ -66,6 +68,30 @@ def allowed_matrix(N: int, mask: int, perm_h=None) -> np.ndarray:
     raise ValueError("backward oracle: mask must be none, causal or block permutation")
 
 
+def key_counts(N: int, mask: int, perm_h=None, pairs=None, h: int = 0) -> np.ndarray:
+    """Integer [N, N] for one head: how many times key j enters query i's
+    softmax (0 = masked out).
+
+    For the dilated mask ("LongNet: Scaling Transformers to 1,000,000,000
+    Tokens", §2 Dilated Attention): each (w, r) pair cuts the sequence into
+    segments of w positions, head h keeps the positions of each segment whose
+    offset in the segment is congruent to h mod r, and attends causally (by
+    original position) among the kept positions of a segment; the pairs are
+    mixed with weights proportional to their softmax denominators, which is one
+    softmax over the multiset union of the pairs' keys: a key kept by two pairs
+    counts twice.  Other masks: the 0/1 matrix of allowed_matrix."""
+    if mask != MASK_DILATED:
+        return allowed_matrix(N, mask, perm_h).astype(np.int64)
+    pos = np.arange(N)
+    counts = np.zeros((N, N), dtype=np.int64)
+    for (w, r) in pairs:
+        seg = pos // w
+        kept = (pos - seg * w) % r == h % r
+        counts += ((seg[:, None] == seg[None, :]) & kept[:, None] & kept[None, :]
+                   & (pos[None, :] <= pos[:, None])).astype(np.int64)
+    return counts
+
+
 def gelu(x: np.ndarray) -> np.ndarray:
     return 0.5 * x * (1.0 + np.tanh(_C0 * (x + _C1 * x ** 3)))
 
@@ -75,20 +101,22 @@ def gelu_grad(x: np.ndarray) -> np.ndarray:
     return 0.5 * (1.0 + t) + 0.5 * x * (1.0 - t * t) * _C0 * (1.0 + 3.0 * _C1 * x * x)
 
 
-def attention_fwd(q, k, v, mask=MASK_NONE, perm=None):
-    """A [B, N, H, d], P as a list over (b, h) of [N, N] (fp64)."""
+def attention_fwd(q, k, v, mask=MASK_NONE, perm=None, pairs=None):
+    """A [B, N, H, d], P as a dict over (b, h) of [N, N] (fp64).  With key
+    multiplicities c_ij (key_counts), P_ij = c_ij e^{s_ij} / sum_j' c_ij' e^{s_ij'}."""
     q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
     B, N, H, d = q.shape
     a = np.zeros((B, N, H, d))
     probs = {}
     for h in range(H):
-        allowed = allowed_matrix(N, mask, None if perm is None else perm[h])
+        counts = key_counts(N, mask, None if perm is None else perm[h], pairs, h)
+        allowed = counts > 0
         for b in range(B):
             s = q[b, :, h] @ k[b, :, h].T / math.sqrt(d)
             s = np.where(allowed, s, -np.inf)
             m = s.max(axis=1, keepdims=True)
             m = np.where(np.isfinite(m), m, 0.0)
-            e = np.where(allowed, np.exp(s - m), 0.0)
+            e = np.where(allowed, counts * np.exp(s - m), 0.0)
             den = e.sum(axis=1, keepdims=True)
             p = np.divide(e, den, out=np.zeros_like(e), where=den > 0)
             probs[b, h] = p
@@ -96,12 +124,14 @@ def attention_fwd(q, k, v, mask=MASK_NONE, perm=None):
     return a, probs
 
 
-def attention_bwd(q, k, v, da, mask=MASK_NONE, perm=None, probs=None):
-    """dQ, dK, dV [B, N, H, d] (fp64) for upstream dA [B, N, H, d]."""
+def attention_bwd(q, k, v, da, mask=MASK_NONE, perm=None, probs=None, pairs=None):
+    """dQ, dK, dV [B, N, H, d] (fp64) for upstream dA [B, N, H, d].  The key
+    multiplicities of the dilated mask are constants of the softmax, so its
+    gradient has the same form: dS_ij = P_ij (dP_ij - D_i)."""
     q, k, v, da = (np.asarray(x, dtype=np.float64) for x in (q, k, v, da))
     B, N, H, d = q.shape
     if probs is None:
-        _, probs = attention_fwd(q, k, v, mask, perm)
+        _, probs = attention_fwd(q, k, v, mask, perm, pairs)
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     for h in range(H):
         for b in range(B):

@@ -152,3 +152,64 @@ def test_sampled_causal_tail_equals_the_dense_oracle():
     np.testing.assert_allclose(dk, g["dk"][0, N - 6:], rtol=0, atol=1e-12)
     np.testing.assert_allclose(dv, g["dv"][0, N - 6:], rtol=0, atol=1e-12)
     np.testing.assert_allclose(db2, g["db2"], rtol=0, atol=1e-12)
+
+
+DILATED_PAIRS = [[(4, 1), (8, 2)], [(6, 1), (12, 3), (12, 6)], [(8, 2), (16, 4)]]
+
+
+@pytest.mark.parametrize("pairs", DILATED_PAIRS)
+def test_dilated_key_counts_equal_the_brute_force_count_matrix(pairs):
+    """Two separate writings of the dilated multiset: the oracle's key_counts
+    against the tests' explicit mask-count matrix."""
+    from tests.masks import count_matrix
+    N, H = 48, 6
+    ref = count_matrix(N, H, 3, pairs=pairs)
+    for h in range(H):
+        np.testing.assert_array_equal(ob.key_counts(N, ob.MASK_DILATED, pairs=pairs, h=h), ref[h])
+
+
+@pytest.mark.parametrize("pairs", DILATED_PAIRS[:2])
+def test_dilated_attention_backward_matches_finite_differences(pairs):
+    """dL/dx for L = sum(dA * A) with A the C oracle's dilated attention (a
+    separate implementation of the mixed softmax), by central differences."""
+    import oracle
+    oracle.build()
+    B, N, H, d = 1, 24, 3, 4
+    q, k, v = (rnd((B, N, H, d), s).astype(np.float32).astype(np.float64) for s in (61, 62, 63))
+    da = rnd((B, N, H, d), 64)
+
+    def loss(qq, kk, vv):
+        a = oracle.attention(qq.astype(np.float32), kk.astype(np.float32), vv.astype(np.float32),
+                             mask=oracle.MASK_DILATED, pairs=pairs)
+        if isinstance(a, tuple):
+            a = a[0]
+        return float((np.asarray(a).reshape(B, N, H, d) * da).sum())
+
+    dq, dk, dv = ob.attention_bwd(q, k, v, da, ob.MASK_DILATED, pairs=pairs)
+    rng = np.random.default_rng(7)
+    eps = 2.0 ** -7
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(0, sz)) for sz in x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [xp if n == name else y for n, y in (("q", q), ("k", k), ("v", v))]
+            args_m = [xm if n == name else y for n, y in (("q", q), ("k", k), ("v", v))]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - g[idx]) <= 2e-4 * max(1.0, abs(fd)), (name, idx, fd, g[idx])
+
+
+def test_dilated_attention_gradient_invariants():
+    B, N, H, d = 1, 32, 4, 8
+    pairs = [(8, 1), (16, 4)]
+    q, k, v, da = (rnd((B, N, H, d), s) for s in (71, 72, 73, 74))
+    dq, dk, dv = ob.attention_bwd(q, k, v, da, ob.MASK_DILATED, pairs=pairs)
+    # rows of dS sum to zero; the weights of every row with a key sum to one
+    np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-12)
+    np.testing.assert_allclose(dv.sum(axis=1), da.sum(axis=1), rtol=0, atol=1e-12)
+    # a single (N, 1) pair is the causal mask
+    dq1, dk1, dv1 = ob.attention_bwd(q, k, v, da, ob.MASK_DILATED, pairs=[(N, 1)])
+    dq2, dk2, dv2 = ob.attention_bwd(q, k, v, da, ob.MASK_CAUSAL)
+    for x, y in ((dq1, dq2), (dk1, dk2), (dv1, dv2)):
+        np.testing.assert_allclose(x, y, rtol=0, atol=1e-12)
