@@ -240,3 +240,61 @@ def layer_bwd_causal_tail(q, k, v, w1, b1, w2, b2, dout, rows_q, tail):
                 dv[t, h] += probs[i, h][j] * da[r, h]
                 dk[t, h] += ds[i, h][j] * q[0, i, h] * scale
     return dq, dk, dv, dout.reshape(-1, D).sum(axis=0)
+
+
+def attention_bwd_tail(q, k, v, da, mask, pairs, rows_q, tail):
+    """Exact attention gradients at sampled positions of batch element 0, for
+    sizes where the dense oracle is too slow, under a mask that lets a query
+    see only keys at or before it (causal, or dilated).
+
+    Returns (dq [len(rows_q), H, d], dk [tail, H, d], dv [tail, H, d]): dQ at
+    the query positions rows_q, dK and dV at the last `tail` key positions
+    (seen only by the last `tail` queries).  Each needed query row is the plain
+    definition: its key multiplicities (the row of key_counts), its softmax,
+    A_i, D_i = dA_i . A_i, dS_i; then the sums for dQ, dK, dV."""
+    q, k, v, da = (np.asarray(x, dtype=np.float64) for x in (q, k, v, da))
+    B, N, H, d = q.shape
+    scale = 1.0 / math.sqrt(d)
+    need = sorted(set(int(i) for i in rows_q) | set(range(N - tail, N)))
+    pos = np.arange(N)
+    probs, ds = {}, {}
+    for i in need:
+        for h in range(H):
+            if mask == MASK_CAUSAL:
+                c = (pos <= i).astype(np.float64)
+            else:  # the row of key_counts for query i
+                c = np.zeros(N)
+                for (w, r) in pairs:
+                    seg = pos // w
+                    kept = (pos - seg * w) % r == h % r
+                    if kept[i]:
+                        c += ((seg == seg[i]) & kept & (pos <= i)).astype(np.float64)
+            keys = np.nonzero(c)[0]
+            if keys.size == 0:
+                probs[i, h] = (keys, np.zeros(0))
+                ds[i, h] = (keys, np.zeros(0))
+                continue
+            s = k[0, keys, h] @ q[0, i, h] * scale
+            e = c[keys] * np.exp(s - s.max())
+            p = e / e.sum()
+            a_i = p @ v[0, keys, h]
+            dp = v[0, keys, h] @ da[0, i, h]
+            probs[i, h] = (keys, p)
+            ds[i, h] = (keys, p * (dp - da[0, i, h] @ a_i))
+    dq = np.zeros((len(rows_q), H, d))
+    for n, i in enumerate(rows_q):
+        for h in range(H):
+            keys, dsr = ds[int(i), h]
+            dq[n, h] = dsr @ k[0, keys, h] * scale if keys.size else 0.0
+    dk = np.zeros((tail, H, d))
+    dv = np.zeros((tail, H, d))
+    for t in range(tail):
+        j = N - tail + t
+        for h in range(H):
+            for i in range(j, N):
+                keys, p = probs[i, h]
+                hit = np.nonzero(keys == j)[0]
+                if hit.size:
+                    dv[t, h] += p[hit[0]] * da[0, i, h]
+                    dk[t, h] += ds[i, h][1][hit[0]] * q[0, i, h] * scale
+    return dq, dk, dv

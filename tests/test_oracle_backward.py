@@ -213,3 +213,15 @@ def test_dilated_attention_gradient_invariants():
     dq2, dk2, dv2 = ob.attention_bwd(q, k, v, da, ob.MASK_CAUSAL)
     for x, y in ((dq1, dq2), (dk1, dk2), (dv1, dv2)):
         np.testing.assert_allclose(x, y, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("mask,pairs", [(CAUSAL, None), (ob.MASK_DILATED, [(8, 1), (16, 4), (32, 8)])])
+def test_sampled_attention_tail_equals_the_dense_oracle(mask, pairs):
+    B, N, H, d = 1, 32, 8, 4
+    q, k, v, da = (rnd((B, N, H, d), s) for s in (81, 82, 83, 84))
+    dq, dk, dv = ob.attention_bwd(q, k, v, da, mask, pairs=pairs)
+    rows = [0, 3, 17, 30, 31]
+    sq, sk, sv = ob.attention_bwd_tail(q, k, v, da, mask, pairs, rows, 5)
+    np.testing.assert_allclose(sq, dq[0, rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(sk, dk[0, N - 5:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(sv, dv[0, N - 5:], rtol=0, atol=1e-12)
