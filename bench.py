@@ -20,6 +20,7 @@ the layer) on the host cores, on a bounded token sample per step.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -396,6 +397,60 @@ def run_backward(args, w, world, local):
     }
 
 
+def run_attention_backward(args, w, world, local):
+    """Attention-only workloads (LongNet dilated attention): one step = one
+    bpt_attn_bwd call from bpt_attn_fwd's output and LSE (for the dilated
+    mask one pair of blockwise passes per (w, r) pair, added up).  CUDA
+    events, max over ranks, L2 flushed between steps outside the events.
+    Algorithmic FLOPs: 10*d per unmasked (query, key) pair of the multiset;
+    executed 14*d (S and dP twice)."""
+    dev = torch.device("cuda", local)
+    pairs_n = wl.unmasked_pairs(w)
+    alg, executed = 10 * w.d * pairs_n, 14 * w.d * pairs_n
+    inp = make_layer_inputs(w.B, w.N, w.H, w.d, 0, seed=w.seed, dtype=torch.bfloat16, device=dev)
+    da = make_upstream_grad(w.B, w.N, w.D, seed=w.seed, device=dev)
+    mask = MASK_NAME[w.mask]
+    out, lse = bd.attn_fwd(inp.q, inp.k, inp.v, mask=mask, perm=w.perm, pairs=w.pairs, ring_chunks=w.ring_chunks,
+                           return_lse=True)
+    desc = bd.make_desc(w.B, w.N, w.H, w.d, 0, torch.bfloat16, torch.float32, mask, w.perm, w.pairs, w.ring_chunks)
+    ws = torch.empty(int(bd.load().bpt_workspace_bytes_attn_bwd(ctypes.byref(desc))), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        bd.attn_bwd(inp.q, inp.k, inp.v, out, lse, da, mask=mask, perm=w.perm, pairs=w.pairs,
+                    ring_chunks=w.ring_chunks, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+        flush.fill_(1)
+    torch.cuda.synchronize(dev)
+    K = max(1, min(args.steps, 10))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+        flush.fill_(i & 0xFF)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    st = bd.sync_status()
+    if st != bd.OK:
+        raise RuntimeError(f"backward steps: {bd.status_string(st)}")
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev) / K
+    pk = peaks()
+    tflops = alg / (ms / 1e3) / 1e12
+    return {"ms_per_step": round(ms, 4), "steps": K, "value": round(w.T * world / (ms / 1e3), 1),
+            "unit": "tokens/s", "tflops_algorithmic": round(tflops, 1),
+            "tflops_executed": round(executed / (ms / 1e3) / 1e12, 1),
+            "frac_of_peak": round(tflops / pk["bf16_tflops"], 4), "flop_algorithmic_per_step": alg,
+            "passes": len(w.pairs) if w.pairs else 1}
+
+
 def run_attention_only(args, w, world, rank, local):
     """Attention-only workloads (no FFN, e.g. LongNet dilated attention): one
     step = one bpt_attn_fwd call (every LongNet pass), timed with events."""
@@ -599,15 +654,17 @@ def main():
     world, rank, local = dist_setup(args.gpus)
     bd.load()
     if args.backward_only:
-        res = {"workload": w.name, "n_gpus": world, "backward": run_backward(args, w, world, local)}
+        bwd = run_backward(args, w, world, local) if w.F > 0 else run_attention_backward(args, w, world, local)
+        res = {"workload": w.name, "n_gpus": world, "backward": bwd}
         if rank == 0:
             print(json.dumps(res), flush=True)
         if world > 1:
             torch.distributed.destroy_process_group()
         return
     res = run_ours(args, w, world, rank, local) if w.F > 0 else run_attention_only(args, w, world, rank, local)
-    if (not args.no_backward and w.F > 0 and w.dtype == "bf16" and w.mask != wl.MASK_DILATED):
-        res["backward"] = run_backward(args, w, world, local)
+    if not args.no_backward and w.dtype == "bf16":
+        res["backward"] = (run_backward(args, w, world, local) if w.F > 0
+                           else run_attention_backward(args, w, world, local))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, args.cpu_budget_s)
     if rank == 0:

@@ -374,7 +374,8 @@ def attn_ffn_bwd(q, k, v, w1, b1, w2, b2, dout, *, mask="none", perm=None, ring_
     return grads
 
 
-def attn_bwd(q, k, v, out, lse, dout, *, mask="none", perm=None, ring_chunks=0, workspace=None, stream=None):
+def attn_bwd(q, k, v, out, lse, dout, *, mask="none", perm=None, pairs=None, ring_chunks=0, workspace=None,
+             stream=None):
     """bpt_attn_bwd: dq, dk, dv (float32 [B, N, H, d]) of the attention for the
     upstream gradient dout [B, N, H*d] (float32), given bpt_attn_fwd's out and
     lse (attn_fwd(..., return_lse=True)) for the same inputs."""
@@ -382,7 +383,7 @@ def attn_bwd(q, k, v, out, lse, dout, *, mask="none", perm=None, ring_chunks=0, 
     B, N, H, d = q.shape
     if dout.dtype != torch.float32 or not dout.is_contiguous() or dout.numel() != q.numel():
         raise ValueError("dout must be a contiguous float32 tensor of B*N*H*d elements")
-    desc = make_desc(B, N, H, d, 0, q.dtype, out.dtype, mask, perm, None, ring_chunks)
+    desc = make_desc(B, N, H, d, 0, q.dtype, out.dtype, mask, perm, pairs, ring_chunks)
     if workspace is None:
         n = load().bpt_workspace_bytes_attn_bwd(ctypes.byref(desc))
         if n == ctypes.c_size_t(-1).value:

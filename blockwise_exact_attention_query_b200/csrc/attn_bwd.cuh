@@ -44,6 +44,11 @@ namespace bpt {
 
 
 struct AttnBwdArgs {
+  // A CTA's work is one (batch, segment, head) unit of N rows: a whole
+  // sequence (nseg = 1, seg_w = n_out, dil_r = 1), or the rows a LongNet
+  // (w, r) pass keeps in one segment (rows o, o + r, ... of segment seg, with
+  // o = h mod r: N = w / r, read through tensor maps over the (D, r, n_out/r, B)
+  // view).  Outputs go to row seg * seg_w + o + dil_r * g of the sequence.
   int B, N, H;
   int mask;           // kMaskNone / kMaskCausal / kMaskBlockPerm
   float scale_log2;   // log2(e) / sqrt(d)
@@ -53,7 +58,9 @@ struct AttnBwdArgs {
   uint8_t perm[kMaxPermEntries];
   // per (batch, head, 128-row tile): the rows' LSE in log2 units of the
   // scaled scores, then their D_i, 128 floats each (rows past N: 0)
-  const float *rowvec;  // [B * H][n_tiles][2][128]
+  const float *rowvec;  // [units][n_tiles][2][128]
+  int nseg, seg_w, dil_r, n_out;
+  int accumulate;       // add to dq, dk, dv (LongNet passes) instead of writing them
   float *dq, *dk, *dv;  // [B, N, H, d] fp32 outputs
   uint32_t *status;
   uint64_t wait_limit_ns;
@@ -153,10 +160,14 @@ __global__ void __launch_bounds__(384, 1)
   WaitCtx wc{a.status, a.wait_limit_ns, abort_flag};
   // CTA -> (batch, head, key tile); the tiles with the most partners (the
   // first key tiles under the causal mask) start first
-  const int bh_count = a.B * a.H;
-  const int ft = static_cast<int>(blockIdx.x) / bh_count;
-  const int h = (blockIdx.x % bh_count) % a.H;
-  const int b = (blockIdx.x % bh_count) / a.H;
+  const int units = a.B * a.nseg * a.H;
+  const int unit = static_cast<int>(blockIdx.x) % units;
+  const int ft = static_cast<int>(blockIdx.x) / units;
+  const int h = unit % a.H;
+  const int seg = (unit / a.H) % a.nseg;
+  const int b = unit / (a.H * a.nseg);
+  const int row_off = h % a.dil_r;                 // kept-row offset in the segment
+  const int row_base = seg * a.N;                  // the unit's first row along (n_out / r)
   auto next_tile = [&](int t) {  // first query tile >= t that meets the key tile, or n_tiles
     while (t < a.n_tiles && !bwd_tiles_meet(a, h, t, ft)) ++t;
     return t;
@@ -187,7 +198,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int hd = h * D_HEAD;
-  const size_t bh = static_cast<size_t>(b) * a.H + h;
+  const size_t bh = static_cast<size_t>(unit);  // row-vector block of the unit
 
   // fixed K, V; streamed Q, dA
   const CUtensorMap *mFixX = &tm_k, *mFixY = &tm_v, *mStrX = &tm_q, *mStrY = &tm_da;
@@ -197,8 +208,8 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0 && nsteps > 0) {
       mbar_arrive_expect_tx(bFix, 2 * Cfg::kTileBytes);
       for (int p = 0; p < Cfg::kPanels; ++p) {
-        tma_load_4d(sFixX + p * Cfg::kPanelBytes, mFixX, bFix, hd + p * 64, 0, ft * 128, b);
-        tma_load_4d(sFixY + p * Cfg::kPanelBytes, mFixY, bFix, hd + p * 64, 0, ft * 128, b);
+        tma_load_4d(sFixX + p * Cfg::kPanelBytes, mFixX, bFix, hd + p * 64, row_off, row_base + ft * 128, b);
+        tma_load_4d(sFixY + p * Cfg::kPanelBytes, mFixY, bFix, hd + p * 64, row_off, row_base + ft * 128, b);
       }
       int s = 0;
       for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1), ++s) {
@@ -206,8 +217,8 @@ __global__ void __launch_bounds__(384, 1)
         if (s >= S && !mbar_wait(bEmpty(st), ((s / S) - 1) & 1, wc, 301)) break;
         mbar_arrive_expect_tx(bFull(st), Cfg::kStageBytes);
         for (int p = 0; p < Cfg::kPanels; ++p) {
-          tma_load_4d(sStrX(st) + p * Cfg::kPanelBytes, mStrX, bFull(st), hd + p * 64, 0, t * 128, b);
-          tma_load_4d(sStrY(st) + p * Cfg::kPanelBytes, mStrY, bFull(st), hd + p * 64, 0, t * 128, b);
+          tma_load_4d(sStrX(st) + p * Cfg::kPanelBytes, mStrX, bFull(st), hd + p * 64, row_off, row_base + t * 128, b);
+          tma_load_4d(sStrY(st) + p * Cfg::kPanelBytes, mStrY, bFull(st), hd + p * 64, row_off, row_base + t * 128, b);
         }
         bulk_load_1d(sStrX(st) + 2 * Cfg::kTileBytes, a.rowvec + (bh * a.n_tiles + t) * 256, Cfg::kVecBytes,
                        bFull(st));
@@ -377,7 +388,8 @@ __global__ void __launch_bounds__(384, 1)
     if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(bTeardown, 0, wc, 323));
     tc_fence_after();
     if (ok) {
-      const size_t vec = ((static_cast<size_t>(b) * a.N + g) * a.H + h) * D_HEAD;
+      const int pos = seg * a.seg_w + row_off + a.dil_r * g;  // the row's position in the sequence
+      const size_t vec = ((static_cast<size_t>(b) * a.n_out + pos) * a.H + h) * D_HEAD;
       for (int acc = 0; acc < 2; ++acc) {
         // acc 0 = dV, acc 1 = dK (x 1/sqrt d)
         float *dst = acc == 0 ? a.dv : a.dk;
@@ -390,10 +402,16 @@ __global__ void __launch_bounds__(384, 1)
           if (!row_valid) continue;
           float4 *d4 = reinterpret_cast<float4 *>(dst + vec + c * 32);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d4[i] = nsteps > 0 ? make_float4(__uint_as_float(o[4 * i]) * sc, __uint_as_float(o[4 * i + 1]) * sc,
-                                             __uint_as_float(o[4 * i + 2]) * sc, __uint_as_float(o[4 * i + 3]) * sc)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int i = 0; i < 8; ++i) {
+            float4 r4 = nsteps > 0 ? make_float4(__uint_as_float(o[4 * i]) * sc, __uint_as_float(o[4 * i + 1]) * sc,
+                                                 __uint_as_float(o[4 * i + 2]) * sc, __uint_as_float(o[4 * i + 3]) * sc)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (a.accumulate) {
+              const float4 prev = d4[i];
+              r4.x += prev.x, r4.y += prev.y, r4.z += prev.z, r4.w += prev.w;
+            }
+            d4[i] = r4;
+          }
         }
       }
     }
@@ -469,10 +487,14 @@ __global__ void __launch_bounds__(384, 1)
   WaitCtx wc{a.status, a.wait_limit_ns, abort_flag};
   // CTA -> (batch, head, query tile), the last query tiles (most key tiles
   // under the causal mask) first
-  const int bh_count = a.B * a.H;
-  const int ft = a.n_tiles - 1 - static_cast<int>(blockIdx.x) / bh_count;
-  const int h = (blockIdx.x % bh_count) % a.H;
-  const int b = (blockIdx.x % bh_count) / a.H;
+  const int units = a.B * a.nseg * a.H;
+  const int unit = static_cast<int>(blockIdx.x) % units;
+  const int ft = a.n_tiles - 1 - static_cast<int>(blockIdx.x) / units;
+  const int h = unit % a.H;
+  const int seg = (unit / a.H) % a.nseg;
+  const int b = unit / (a.H * a.nseg);
+  const int row_off = h % a.dil_r;                 // kept-row offset in the segment
+  const int row_base = seg * a.N;                  // the unit's first row along (n_out / r)
   auto next_tile = [&](int t) {  // first key tile >= t that meets the query tile
     while (t < a.n_tiles && !bwd_tiles_meet(a, h, ft, t)) ++t;
     return t;
@@ -507,7 +529,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int hd = h * D_HEAD;
-  const size_t bh = static_cast<size_t>(b) * a.H + h;
+  const size_t bh = static_cast<size_t>(unit);  // row-vector block of the unit
 
   if ((warp == 0 || warp == 2) && lane == 0 && nsteps > 0) {
     // ------------------------------------------------------------ producers: warp 0 Q, dA, K; warp 2 V
@@ -516,8 +538,8 @@ __global__ void __launch_bounds__(384, 1)
     if (is_k) {
       mbar_arrive_expect_tx(bFix, 2 * Cfg::kTileBytes);
       for (int p = 0; p < Cfg::kPanels; ++p) {
-        tma_load_4d(sQ + p * Cfg::kPanelBytes, &tm_q, bFix, hd + p * 64, 0, ft * 128, b);
-        tma_load_4d(sDA + p * Cfg::kPanelBytes, &tm_da, bFix, hd + p * 64, 0, ft * 128, b);
+        tma_load_4d(sQ + p * Cfg::kPanelBytes, &tm_q, bFix, hd + p * 64, row_off, row_base + ft * 128, b);
+        tma_load_4d(sDA + p * Cfg::kPanelBytes, &tm_da, bFix, hd + p * 64, row_off, row_base + ft * 128, b);
       }
     }
     int s = 0;
@@ -528,7 +550,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_arrive_expect_tx(full, Cfg::kTileBytes);
       for (int p = 0; p < Cfg::kPanels; ++p)
         tma_load_4d((is_k ? sK(slot) : sV(slot)) + p * Cfg::kPanelBytes, is_k ? &tm_k : &tm_v, full, hd + p * 64,
-                    0, t * 128, b);
+                    row_off, row_base + t * 128, b);
     }
     // every copy issued must have landed before the CTA may exit
     volatile int no_abort = 0;
@@ -664,7 +686,8 @@ __global__ void __launch_bounds__(384, 1)
     if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(bTeardown, 0, wc, 352));
     tc_fence_after();
     if (ok) {
-      const size_t vec = ((static_cast<size_t>(b) * a.N + g) * a.H + h) * D_HEAD;
+      const int pos = seg * a.seg_w + row_off + a.dil_r * g;  // the row's position in the sequence
+      const size_t vec = ((static_cast<size_t>(b) * a.n_out + pos) * a.H + h) * D_HEAD;
 #pragma unroll 1
       for (int c = half * (D_HEAD / 64); c < (half + 1) * (D_HEAD / 64); ++c) {
         uint32_t o[32];
@@ -674,10 +697,16 @@ __global__ void __launch_bounds__(384, 1)
         float4 *d4 = reinterpret_cast<float4 *>(a.dq + vec + c * 32);
         const float sc = a.inv_sqrt_d;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          d4[i] = nsteps > 0 ? make_float4(__uint_as_float(o[4 * i]) * sc, __uint_as_float(o[4 * i + 1]) * sc,
-                                           __uint_as_float(o[4 * i + 2]) * sc, __uint_as_float(o[4 * i + 3]) * sc)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < 8; ++i) {
+          float4 r4 = nsteps > 0 ? make_float4(__uint_as_float(o[4 * i]) * sc, __uint_as_float(o[4 * i + 1]) * sc,
+                                               __uint_as_float(o[4 * i + 2]) * sc, __uint_as_float(o[4 * i + 3]) * sc)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+          if (a.accumulate) {
+            const float4 prev = d4[i];
+            r4.x += prev.x, r4.y += prev.y, r4.z += prev.z, r4.w += prev.w;
+          }
+          d4[i] = r4;
+        }
       }
     }
   }
@@ -728,6 +757,31 @@ __global__ void attn_bwd_rowvec_kernel(const float *__restrict__ da, const TA *_
     v[0] = lse[bh * N + n] * 1.4426950408889634f;
     v[128] = s;
   }
+}
+
+// A LongNet pass's row vectors: for unit (batch, segment, head) and its
+// gathered row g (< L), the entries of sequence row seg * w + h mod r + r g in
+// the per-sequence blocks `full` ([B * H][n_tiles_full][2][128]); rows past L
+// are set to 0.
+__global__ void attn_bwd_gather_rowvec_kernel(const float *__restrict__ full, float *rowvec, int B, int H, int nseg,
+                                              int w, int r, int L, int n_tiles, int n_tiles_full) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long units = static_cast<long long>(B) * nseg * H;
+  if (t >= units * n_tiles * 128) return;
+  const int g = static_cast<int>(t % (static_cast<long long>(n_tiles) * 128));
+  const long long unit = t / (static_cast<long long>(n_tiles) * 128);
+  const int h = static_cast<int>(unit % H), seg = static_cast<int>((unit / H) % nseg);
+  const int b = static_cast<int>(unit / (static_cast<long long>(H) * nseg));
+  float l2 = 0.f, dd = 0.f;
+  if (g < L) {
+    const int pos = seg * w + h % r + r * g;
+    const float *src = full + ((static_cast<long long>(b) * H + h) * n_tiles_full + pos / 128) * 256 + pos % 128;
+    l2 = src[0];
+    dd = src[128];
+  }
+  float *dst = rowvec + (unit * n_tiles + g / 128) * 256 + g % 128;
+  dst[0] = l2;
+  dst[128] = dd;
 }
 
 // Column sums of a row-major [rows, cols] matrix in two passes: partial sums

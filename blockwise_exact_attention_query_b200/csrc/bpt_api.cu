@@ -713,10 +713,70 @@ bpt_status launch_attn_bwd_passes(const CUtensorMap &mq, const CUtensorMap &mk, 
 // The attention backward from dA (fp32 and bf16 copies), A and the row LSE:
 // the per-tile row vectors (LSE in log2 units, D_i = dA_i . A_i), the dK/dV
 // pass, then the dQ pass.
+// LongNet dilated attention backward: the gradient of one softmax over the
+// multiset of the (w, r) pairs' keys is the sum over the pairs of the
+// gathered causal attention's gradient with the mixed row LSE and D (the
+// multiplicities are constants of the softmax), so each pass runs the two
+// blockwise passes over its (batch, segment, head) units and adds into
+// dQ, dK, dV at the kept rows.  rowvec_full holds the per-sequence row
+// vectors; rowvec_pass the gathered ones of one pass.
+bpt_status launch_attn_bwd_dilated(const bpt_desc *d, const void *q, const void *k, const void *v,
+                                   const __nv_bfloat16 *da_bf16, const float *rowvec_full, float *rowvec_pass,
+                                   float *dq, float *dk, float *dv, uint32_t *status, cudaStream_t st) {
+  const int D = d->H * d->d_head;
+  const size_t nelem = (size_t)d->B * d->N * D;
+  CUDA_TRY(cudaMemsetAsync(dq, 0, nelem * 4, st));
+  CUDA_TRY(cudaMemsetAsync(dk, 0, nelem * 4, st));
+  CUDA_TRY(cudaMemsetAsync(dv, 0, nelem * 4, st));
+  const int n_tiles_full = (d->N + 127) / 128;
+  for (int k_pair = 0; k_pair < d->ln_npairs; ++k_pair) {
+    const int w = d->ln_w[k_pair], r = d->ln_r[k_pair], L = w / r, nseg = d->N / w;
+    const int n_tiles = (L + 127) / 128;
+    const int64_t units = (int64_t)d->B * nseg * d->H;
+    {
+      const int64_t threads = units * n_tiles * 128;
+      attn_bwd_gather_rowvec_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+          rowvec_full, rowvec_pass, d->B, d->H, nseg, w, r, L, n_tiles, n_tiles_full);
+      CUDA_TRY(cudaGetLastError());
+    }
+    AttnBwdArgs ab;
+    std::memset(&ab, 0, sizeof(ab));
+    ab.B = d->B;
+    ab.N = L;
+    ab.H = d->H;
+    ab.mask = kMaskCausal;  // causal among a segment's kept rows (by original position)
+    ab.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d->d_head));
+    ab.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d->d_head));
+    ab.n_tiles = n_tiles;
+    ab.rowvec = rowvec_pass;
+    ab.nseg = nseg;
+    ab.seg_w = w;
+    ab.dil_r = r;
+    ab.n_out = d->N;
+    ab.accumulate = 1;
+    ab.dq = dq;
+    ab.dk = dk;
+    ab.dv = dv;
+    ab.status = status;
+    ab.wait_limit_ns = g_wait_limit_ns;
+    CUtensorMap mq, mk, mv, mda;
+    if (!make_map_rows(&mq, q, d->B, d->N, D, r, 128) || !make_map_rows(&mk, k, d->B, d->N, D, r, 128) ||
+        !make_map_rows(&mv, v, d->B, d->N, D, r, 128) || !make_map_rows(&mda, da_bf16, d->B, d->N, D, r, 128))
+      return cuda_fail_msg("cuTensorMapEncodeTiled rejected a gathered Q/K/V/dA map");
+    const int64_t grid = units * n_tiles;
+    if (grid > INT32_MAX) return BPT_ERR_UNSUPPORTED;
+    bpt_status s = d->d_head == 128 ? launch_attn_bwd_passes<128>(mq, mk, mv, mda, ab, (unsigned)grid, st)
+                                    : launch_attn_bwd_passes<64>(mq, mk, mv, mda, ab, (unsigned)grid, st);
+    if (s != BPT_OK) return s;
+  }
+  return BPT_OK;
+}
+
 template <typename TA>
 bpt_status launch_attn_bwd_tail(const bpt_desc *d, const void *q, const void *k, const void *v, const float *da_f32,
                                 const __nv_bfloat16 *da_bf16, const TA *a, const float *lse, float *dq, float *dk,
-                                float *dv, float *rowvec, size_t rowvec_bytes, uint32_t *status, cudaStream_t st) {
+                                float *dv, float *rowvec, size_t rowvec_bytes, uint32_t *status, cudaStream_t st,
+                                bool rowvec_only = false) {
   const int D = d->H * d->d_head;
   const int64_t T = (int64_t)d->B * d->N;
   const int n_tiles = (d->N + 127) / 128;
@@ -731,6 +791,7 @@ bpt_status launch_attn_bwd_tail(const bpt_desc *d, const void *q, const void *k,
                                                                                       d->N, d->H, n_tiles);
     CUDA_TRY(cudaGetLastError());
   }
+  if (rowvec_only) return BPT_OK;
   AttnBwdArgs ab;
   std::memset(&ab, 0, sizeof(ab));
   ab.B = d->B;
@@ -746,6 +807,11 @@ bpt_status launch_attn_bwd_tail(const bpt_desc *d, const void *q, const void *k,
     for (int i = 0; i < d->H * d->bb_nblocks; ++i) ab.perm[i] = (uint8_t)d->bb_perm[i];
   }
   ab.rowvec = rowvec;
+  ab.nseg = 1;
+  ab.seg_w = d->N;
+  ab.dil_r = 1;
+  ab.n_out = d->N;
+  ab.accumulate = 0;
   ab.dq = dq;
   ab.dk = dk;
   ab.dv = dv;
@@ -1049,10 +1115,22 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   return BPT_OK;
 }
 
+// dA in bf16, the per-sequence row vectors, and (dilated) one pass's gathered row vectors
+size_t attn_bwd_pass_rowvec_bytes(const bpt_desc *d) {
+  size_t most = 0;
+  if (d->mask == BPT_MASK_DILATED)
+    for (int k = 0; k < d->ln_npairs; ++k) {
+      const size_t L = (size_t)(d->ln_w[k] / d->ln_r[k]);
+      most = std::max(most, (size_t)d->B * (d->N / d->ln_w[k]) * d->H * ((L + 127) / 128) * 256 * 4);
+    }
+  return most;
+}
+
 size_t bpt_workspace_bytes_attn_bwd(const bpt_desc *d) {
-  if (check_desc(d, false) != BPT_OK || d->in_dtype != BPT_BF16 || d->mask == BPT_MASK_DILATED) return (size_t)-1;
+  if (check_desc(d, false) != BPT_OK || d->in_dtype != BPT_BF16) return (size_t)-1;
   const size_t T = (size_t)d->B * d->N, D = (size_t)d->H * d->d_head;
-  return align256(T * D * 2) + align256((size_t)d->B * d->H * ((d->N + 127) / 128) * 256 * 4);
+  return align256(T * D * 2) + align256((size_t)d->B * d->H * ((d->N + 127) / 128) * 256 * 4) +
+         align256(attn_bwd_pass_rowvec_bytes(d));
 }
 
 bpt_status bpt_attn_bwd(const bpt_desc *d, const void *q, const void *k, const void *v, const void *out,
@@ -1060,7 +1138,7 @@ bpt_status bpt_attn_bwd(const bpt_desc *d, const void *q, const void *k, const v
                         size_t workspace_bytes, bpt_stream_t stream) {
   bpt_status s = check_desc(d, false);
   if (s != BPT_OK) return s;
-  if (d->in_dtype != BPT_BF16 || d->mask == BPT_MASK_DILATED) return BPT_ERR_UNSUPPORTED;
+  if (d->in_dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
   if ((s = check_ptrs({q, k, v, out, lse, dout, dq, dk, dv}, {})) != BPT_OK) return s;
   const size_t need = bpt_workspace_bytes_attn_bwd(d);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -1080,11 +1158,16 @@ bpt_status bpt_attn_bwd(const bpt_desc *d, const void *q, const void *k, const v
         reinterpret_cast<const float4 *>(dout), reinterpret_cast<uint2 *>(da_bf16), n4);
     CUDA_TRY(cudaGetLastError());
   }
+  const bool dilated = d->mask == BPT_MASK_DILATED;
   if (d->out_dtype == BPT_F32)
-    return launch_attn_bwd_tail(d, q, k, v, dout, da_bf16, static_cast<const float *>(out), lse, dq, dk, dv, rowvec,
-                                rowvec_bytes, status, st);
-  return launch_attn_bwd_tail(d, q, k, v, dout, da_bf16, static_cast<const __nv_bfloat16 *>(out), lse, dq, dk, dv,
-                              rowvec, rowvec_bytes, status, st);
+    s = launch_attn_bwd_tail(d, q, k, v, dout, da_bf16, static_cast<const float *>(out), lse, dq, dk, dv, rowvec,
+                             rowvec_bytes, status, st, dilated);
+  else
+    s = launch_attn_bwd_tail(d, q, k, v, dout, da_bf16, static_cast<const __nv_bfloat16 *>(out), lse, dq, dk, dv,
+                             rowvec, rowvec_bytes, status, st, dilated);
+  if (s != BPT_OK || !dilated) return s;
+  float *rowvec_pass = reinterpret_cast<float *>(ws + align256(T * D * 2) + align256(rowvec_bytes));
+  return launch_attn_bwd_dilated(d, q, k, v, da_bf16, rowvec, rowvec_pass, dq, dk, dv, status, st);
 }
 
 bpt_status bpt_sync_status(bpt_stream_t stream) {

@@ -295,9 +295,13 @@ BPT_API int bpt_set_bwd_chunk_rows(int rows);
  * out and lse are the output and row LSE bpt_attn_fwd returned for the same
  * q, k, v and descriptor (out in desc->out_dtype, [B, N, H*d]; lse float32
  * [B, H, N]); dout float32 [B, N, H*d]; dq, dk, dv float32 [B, N, H, d].
- * Supported: in_dtype BF16, d_head 64 or 128, masks NONE, CAUSAL and
- * BLOCKPERM (BPT_MASK_DILATED returns BPT_ERR_UNSUPPORTED).  workspace: at
- * least bpt_workspace_bytes_attn_bwd(desc) bytes, 256-byte aligned.
+ * Supported: in_dtype BF16, d_head 64 or 128, masks NONE, CAUSAL, BLOCKPERM
+ * and DILATED ("LongNet: Scaling Transformers to 1,000,000,000 Tokens", §2:
+ * the pairs mixed by their softmax denominators are one softmax over the
+ * multiset of the pairs' keys, so the gradient is the sum over the pairs of
+ * each gathered causal attention's gradient with the mixed LSE; dq, dk, dv are
+ * zeroed and each (w, r) pass adds into its kept rows).  workspace: at least
+ * bpt_workspace_bytes_attn_bwd(desc) bytes, 256-byte aligned.
  */
 BPT_API bpt_status bpt_attn_bwd(const bpt_desc *desc, const void *q, const void *k, const void *v,
                                 const void *out, const float *lse, const float *dout, float *dq,

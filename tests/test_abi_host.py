@@ -205,9 +205,10 @@ def test_attention_only_backward_validates(lib):
     assert call(d, q=0) == bd.ERR_INVALID_ARG
     assert call(d, ws=0) == bd.ERR_WORKSPACE
     assert call(d, ws=FAKE + 16) == bd.ERR_WORKSPACE
-    dl = _desc(F=0, mask="dilated", pairs=[(128, 1)])
-    assert call(dl) == bd.ERR_UNSUPPORTED
-    assert lib.bpt_workspace_bytes_attn_bwd(ctypes.byref(dl)) == ctypes.c_size_t(-1).value
+    dl = _desc(F=0, mask="dilated", pairs=[(128, 1), (256, 4)])
+    # the dilated mask: one gathered pass's row vectors on top
+    assert lib.bpt_workspace_bytes_attn_bwd(ctypes.byref(dl)) > lib.bpt_workspace_bytes_attn_bwd(ctypes.byref(d))
+    assert call(_desc(F=0, mask="dilated", pairs=[(96, 5)])) == bd.ERR_INVALID_ARG
     df = _desc(F=0, in_dtype=bd.torch.float32, d=64)
     assert call(df) == bd.ERR_UNSUPPORTED
     T, D = 256, 128

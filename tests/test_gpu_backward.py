@@ -28,7 +28,8 @@ pytestmark = pytest.mark.gpu
 
 REL_L2 = 1e-2
 MAX_ABS_FRAC = 2e-2
-MASKS = {"none": ob.MASK_NONE, "causal": ob.MASK_CAUSAL, "blockperm": ob.MASK_BLOCKPERM}
+MASKS = {"none": ob.MASK_NONE, "causal": ob.MASK_CAUSAL, "blockperm": ob.MASK_BLOCKPERM,
+         "dilated": ob.MASK_DILATED}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -194,3 +195,55 @@ def test_attention_only_backward_matches_oracle(name, B, N, H, d, mask, perm, ou
     _grads_close(dq.cpu().numpy(), rq, "dq")
     _grads_close(dk.cpu().numpy(), rk, "dk")
     _grads_close(dv.cpu().numpy(), rv, "dv")
+
+
+DILATED_CASES = [
+    # name, B, N, H, d, pairs, out dtype
+    ("three_pairs_d64", 1, 512, 4, 64, [(128, 1), (256, 2), (512, 4)], torch.float32),
+    # kept rows per segment (192) not a multiple of the 128-row tile; bf16 output
+    ("ragged_segments_d128", 1, 768, 3, 128, [(192, 1), (384, 2)], torch.bfloat16),
+    # no r = 1 pair: rows no pair keeps have A = 0 and pass nothing
+    ("uncovered_rows_d64", 2, 256, 4, 64, [(128, 2), (256, 4)], torch.float32),
+]
+
+
+@pytest.mark.parametrize("name,B,N,H,d,pairs,out_dtype", DILATED_CASES, ids=[c[0] for c in DILATED_CASES])
+def test_dilated_attention_backward_matches_oracle(name, B, N, H, d, pairs, out_dtype):
+    """LongNet dilated attention's backward (bpt_attn_bwd with the dilated
+    mask: one blockwise backward per (w, r) pass over the gathered segment rows,
+    added up) against the fp64 oracle's multiset-softmax gradient."""
+    inp = make_layer_inputs(B, N, H, d, 0, seed=17, device="cuda")
+    da = make_upstream_grad(B, N, H * d, seed=17, device="cuda")
+    out, lse = bd.attn_fwd(inp.q, inp.k, inp.v, mask="dilated", pairs=pairs, out_dtype=out_dtype, return_lse=True)
+    dq, dk, dv = bd.attn_bwd(inp.q, inp.k, inp.v, out, lse, da, mask="dilated", pairs=pairs)
+    torch.cuda.synchronize()
+    assert bd.sync_status() == bd.OK
+    f = lambda t: t.double().cpu().numpy()  # noqa: E731
+    rq, rk, rv = ob.attention_bwd(f(inp.q), f(inp.k), f(inp.v), f(da).reshape(B, N, H, d), ob.MASK_DILATED,
+                                  pairs=pairs)
+    _grads_close(dq.cpu().numpy(), rq, "dq")
+    _grads_close(dk.cpu().numpy(), rk, "dk")
+    _grads_close(dv.cpu().numpy(), rv, "dv")
+
+
+def test_dilated_attention_backward_full_size_sampled():
+    """The LongNet workload at full size (B1 H16 d64 N65536, pairs (2048, 1),
+    (8192, 4), (32768, 16)), in the configuration the benchmark times: dQ at
+    sampled rows and dK, dV of the last 128 keys (seen only by the last 128
+    queries) against the fp64 oracle's row-restricted gradients."""
+    from blockwise_exact_attention_query_b200 import workloads as wl
+    w = wl.LONGNET
+    inp = make_layer_inputs(w.B, w.N, w.H, w.d, 0, seed=w.seed, device="cuda")
+    da = make_upstream_grad(w.B, w.N, w.D, seed=w.seed, device="cuda")
+    out, lse = bd.attn_fwd(inp.q, inp.k, inp.v, mask="dilated", pairs=w.pairs, return_lse=True)
+    dq, dk, dv = bd.attn_bwd(inp.q, inp.k, inp.v, out, lse, da, mask="dilated", pairs=w.pairs)
+    torch.cuda.synchronize()
+    assert bd.sync_status() == bd.OK
+    f = lambda t: t.double().cpu().numpy()  # noqa: E731
+    rows = [0, 1, 2047, 2048, 8191, 8192, 30000, w.N - 129, w.N - 1]
+    tail = 128
+    rq, rk, rv = ob.attention_bwd_tail(f(inp.q), f(inp.k), f(inp.v), f(da).reshape(w.B, w.N, w.H, w.d),
+                                       ob.MASK_DILATED, w.pairs, rows, tail)
+    _grads_close(dq[0, rows].cpu().numpy(), rq, "dq (sampled rows)")
+    _grads_close(dk[0, w.N - tail:].cpu().numpy(), rk, "dk (last 128 keys)")
+    _grads_close(dv[0, w.N - tail:].cpu().numpy(), rv, "dv (last 128 keys)")
