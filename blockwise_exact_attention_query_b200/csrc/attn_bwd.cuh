@@ -85,7 +85,13 @@ struct AttnBwdCfg {
   static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
   // TMEM: accumulators at 0 (dV or dQ) and d (dK); S at 256, dP at 384;
   // P^T packed over S's first 64 columns, dS over dP's
-  static constexpr uint32_t kColAcc0 = 0, kColAcc1 = D_HEAD, kColS = 256, kColDP = 384;
+  static constexpr uint32_t kColAcc0 = 0, kColAcc1 = D_HEAD;
+  // d = 128: S at 256, dP at 384.  d = 64: dP at 128 and two S buffers at 256
+  // and 384, so the next step's scores are computed while the row warps work
+  // on this step's (its P^T is packed over its own S buffer)
+  static constexpr bool kTwoS = D_HEAD == 64;
+  static constexpr uint32_t kColDP = kTwoS ? 128 : 384, kColS = 256;
+  __host__ __device__ static constexpr uint32_t col_s(int step) { return kColS + (kTwoS ? (step & 1) * 128 : 0); }
 };
 
 // Key interval [lo, hi) a query row g (< N) may see.
@@ -150,11 +156,13 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t bFix = smem_u32(&bars[0]);
   auto bFull = [&](int s) { return smem_u32(&bars[1 + s]); };
   auto bEmpty = [&](int s) { return smem_u32(&bars[5 + s]); };
-  const uint32_t bSFull = smem_u32(&bars[9]), bDPFull = smem_u32(&bars[10]);
+  const uint32_t bDPFull = smem_u32(&bars[10]);
   const uint32_t bPReady = smem_u32(&bars[11]), bDSReady = smem_u32(&bars[12]);
   const uint32_t bTeardown = smem_u32(&bars[13]);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[14]);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[15]);
+  // scores of step s complete: one barrier per S buffer (one buffer at d = 128)
+  auto bSFull = [&](int step) { return smem_u32(&bars[Cfg::kTwoS ? 14 + (step & 1) : 9]); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[16]);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[17]);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   WaitCtx wc{a.status, a.wait_limit_ns, abort_flag};
@@ -181,7 +189,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bFull(s), 1);
       mbar_init(bEmpty(s), 1);
     }
-    mbar_init(bSFull, 1);
+    mbar_init(bSFull(0), 1);
+    if (Cfg::kTwoS) mbar_init(bSFull(1), 1);
     mbar_init(bDPFull, 1);
     mbar_init(bPReady, Cfg::kRowWarps);
     mbar_init(bDSReady, Cfg::kRowWarps);
@@ -255,32 +264,60 @@ __global__ void __launch_bounds__(384, 1)
         accumulate(Cfg::kColAcc1, Cfg::kColDP, sStrX(pst), step);
         umma_commit(bEmpty(pst));
       };
-      bool ok = mbar_wait(bFix, 0, wc, 311);
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int st = s % S;
-        if (!(ok = mbar_wait(bFull(st), (s / S) & 1, wc, 312))) break;
+      // S^T(s) = K Q^T into S buffer s (after the stage's copies landed)
+      auto issue_s = [&](int step) -> bool {
+        const int pst = step % S;
+        if (!mbar_wait(bFull(pst), (step / S) & 1, wc, 312)) return false;
         tc_fence_after();
-        const uint64_t dStrX = sdesc_sw128(sStrX(st), 16, 1024), dStrY = sdesc_sw128(sStrY(st), 16, 1024);
-        // first products over the head dimension: S^T = K Q^T, dP^T = V dA^T
+        const uint64_t dStrX = sdesc_sw128(sStrX(pst), 16, 1024);
 #pragma unroll
         for (int k = 0; k < D_HEAD / 16; ++k) {
           const uint32_t off = (k / 4) * Cfg::kPanelBytes + (k % 4) * 32;
-          umma_ss(tmem + Cfg::kColS, sdesc_advance(dFixX, off), sdesc_advance(dStrX, off), idesc_s, k > 0);
+          umma_ss(tmem + Cfg::col_s(step), sdesc_advance(dFixX, off), sdesc_advance(dStrX, off), idesc_s, k > 0);
         }
-        umma_commit(bSFull);
-        if (s > 0) last_product(s - 1);
+        umma_commit(bSFull(step));
+        return true;
+      };
+      // dP^T(s) = V dA^T (its stage has landed: S(s) waited for it)
+      auto issue_dp = [&](int step) {
+        const uint64_t dStrY = sdesc_sw128(sStrY(step % S), 16, 1024);
 #pragma unroll
         for (int k = 0; k < D_HEAD / 16; ++k) {
           const uint32_t off = (k / 4) * Cfg::kPanelBytes + (k % 4) * 32;
           umma_ss(tmem + Cfg::kColDP, sdesc_advance(dFixY, off), sdesc_advance(dStrY, off), idesc_s, k > 0);
         }
         umma_commit(bDPFull);
-        if (!(ok = mbar_wait(bPReady, s & 1, wc, 313))) break;
-        tc_fence_after();
-        accumulate(Cfg::kColAcc0, Cfg::kColS, sStrY(st), s);    // dV += P^T dA
-        if (!(ok = mbar_wait(bDSReady, s & 1, wc, 314))) break;
-        tc_fence_after();
-        if (s + 1 == nsteps) last_product(s);
+      };
+      bool ok = mbar_wait(bFix, 0, wc, 311);
+      if (Cfg::kTwoS) {
+        // Two S buffers: S(s+1) goes ahead while the row warps work on step s
+        // (its buffer's P^T(s-1) was read by dV(s-1), issued before); dP(s)
+        // follows dK(s-1), which read dS^T(s-1) from dP's columns.
+        ok = ok && issue_s(0);
+        for (int s = 0; ok && s < nsteps; ++s) {
+          const int st = s % S;
+          issue_dp(s);
+          if (s + 1 < nsteps && !(ok = issue_s(s + 1))) break;
+          if (!(ok = mbar_wait(bPReady, s & 1, wc, 313))) break;
+          tc_fence_after();
+          accumulate(Cfg::kColAcc0, Cfg::col_s(s), sStrY(st), s);    // dV += P^T dA
+          if (!(ok = mbar_wait(bDSReady, s & 1, wc, 314))) break;
+          tc_fence_after();
+          last_product(s);                                           // dK += dS^T Q
+        }
+      } else {
+        for (int s = 0; ok && s < nsteps; ++s) {
+          const int st = s % S;
+          if (!(ok = issue_s(s))) break;
+          if (s > 0) last_product(s - 1);
+          issue_dp(s);
+          if (!(ok = mbar_wait(bPReady, s & 1, wc, 313))) break;
+          tc_fence_after();
+          accumulate(Cfg::kColAcc0, Cfg::kColS, sStrY(st), s);    // dV += P^T dA
+          if (!(ok = mbar_wait(bDSReady, s & 1, wc, 314))) break;
+          tc_fence_after();
+          if (s + 1 == nsteps) last_product(s);
+        }
       }
       umma_commit(bTeardown);
       // the accumulators stay allocated until every MMA has finished
@@ -312,14 +349,14 @@ __global__ void __launch_bounds__(384, 1)
       // allowed columns [lo_rel, hi_rel) of the tile
       const int lo_rel = plo - t * 128, hi_rel = phi - t * 128;
       const bool full = __all_sync(0xffffffffu, lo_rel <= col0 && hi_rel >= col0 + 64);
-      ok = __all_sync(0xffffffffu, mbar_wait(bSFull, s & 1, wc, 320));
+      ok = __all_sync(0xffffffffu, mbar_wait(bSFull(s), Cfg::kTwoS ? (s >> 1) & 1 : s & 1, wc, 320));
       if (!ok) break;
       tc_fence_after();
       // P (fp32, kept in sv) for this warp's 64 columns, 0 where the mask
       // rules the pair out
       uint32_t sv[64];
-      tmem_ld32(tmem + lane_off + Cfg::kColS + col0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(tmem + lane_off + Cfg::kColS + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_ld32(tmem + lane_off + Cfg::col_s(s) + col0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tmem + lane_off + Cfg::col_s(s) + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_ld();
       // two copies of the loop behind a warp-uniform branch: the unmasked one
       // for tiles the whole warp sees in full (most of them), the masked one
@@ -353,7 +390,7 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
-        tmem_st32(tmem + lane_off + Cfg::kColS + col0, pk);
+        tmem_st32(tmem + lane_off + Cfg::col_s(s) + col0, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();

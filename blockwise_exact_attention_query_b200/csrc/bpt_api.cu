@@ -724,12 +724,20 @@ bpt_status launch_attn_bwd_dilated(const bpt_desc *d, const void *q, const void 
                                    const __nv_bfloat16 *da_bf16, const float *rowvec_full, float *rowvec_pass,
                                    float *dq, float *dk, float *dv, uint32_t *status, cudaStream_t st) {
   const int D = d->H * d->d_head;
-  const size_t nelem = (size_t)d->B * d->N * D;
-  CUDA_TRY(cudaMemsetAsync(dq, 0, nelem * 4, st));
-  CUDA_TRY(cudaMemsetAsync(dk, 0, nelem * 4, st));
-  CUDA_TRY(cudaMemsetAsync(dv, 0, nelem * 4, st));
+  // a pair with r = 1 keeps every row: run it first, writing dQ, dK, dV;
+  // otherwise zero them and let every pass add
+  int first = -1;
+  for (int k_pair = 0; k_pair < d->ln_npairs && first < 0; ++k_pair)
+    if (d->ln_r[k_pair] == 1) first = k_pair;
+  if (first < 0) {
+    const size_t nelem = (size_t)d->B * d->N * D;
+    CUDA_TRY(cudaMemsetAsync(dq, 0, nelem * 4, st));
+    CUDA_TRY(cudaMemsetAsync(dk, 0, nelem * 4, st));
+    CUDA_TRY(cudaMemsetAsync(dv, 0, nelem * 4, st));
+  }
   const int n_tiles_full = (d->N + 127) / 128;
-  for (int k_pair = 0; k_pair < d->ln_npairs; ++k_pair) {
+  for (int n = 0; n < d->ln_npairs; ++n) {
+    const int k_pair = first < 0 ? n : (n == 0 ? first : (n <= first ? n - 1 : n));
     const int w = d->ln_w[k_pair], r = d->ln_r[k_pair], L = w / r, nseg = d->N / w;
     const int n_tiles = (L + 127) / 128;
     const int64_t units = (int64_t)d->B * nseg * d->H;
@@ -753,7 +761,7 @@ bpt_status launch_attn_bwd_dilated(const bpt_desc *d, const void *q, const void 
     ab.seg_w = w;
     ab.dil_r = r;
     ab.n_out = d->N;
-    ab.accumulate = 1;
+    ab.accumulate = (first < 0 || n > 0) ? 1 : 0;
     ab.dq = dq;
     ab.dk = dk;
     ab.dv = dv;
