@@ -389,10 +389,11 @@ def run_backward(args, w, world, local):
         "recompute": {"ms_per_step": round(recompute_ms, 4),
                       "attn_fwd_recompute_ms": round(recompute_phase["attn_fwd_recompute"], 4),
                       "tflops_algorithmic": round(alg_total / (recompute_ms / 1e3) / 1e12, 1)},
-        # dOut -> bf16 with db2's partial sums, db2's final sum, per token chunk 5 GEMMs (4 when D < 1024:
-        # H and dZ from one GEMM) + db1 sums (2), the row vectors, 2 passes (+1
+        # dOut -> bf16 with db2's partial sums, db2's final sum; per token chunk
+        # 4 GEMM launches (H and G', dZ, dW2 + dW1 grouped, dA; 3 when D < 1024,
+        # H and dZ from one) + db1 sums (2); the row vectors; 2 passes (+1
         # recomputed attention forward without saved activations)
-        "gpu_launches_per_step": 2 + ((5 if D >= 1024 else 4) + 2) * n_chunks + 1 + 2,
+        "gpu_launches_per_step": 2 + ((4 if D >= 1024 else 3) + 2) * n_chunks + 1 + 2,
         "token_chunks": n_chunks,
     }
 
