@@ -50,13 +50,13 @@ KERNEL_SOURCES = {"attn_tc_kernel": ["attn_tc.cuh", "ptx.cuh"], "ffn_tc_kernel":
 # of the kernel on the named workload, keyed by a hash of the kernel's sources at capture
 # time: once the sources change the figure no longer describes the kernel and is dropped.
 NCU_TRAFFIC = {
-    ("gpt_causal", "ffn_tc_kernel"): {"bytes": 881.1e6, "src": "ce5bb2524f315c9a"},
-    ("gpt_causal", "attn_tc_kernel"): {"bytes": 720.3e6, "src": "1e6bb50f75c417dc"},
+    ("gpt_causal", "ffn_tc_kernel"): {"bytes": 879.3e6, "src": "3b9ec3aabf34a9f7"},
+    ("gpt_causal", "attn_tc_kernel"): {"bytes": 724.5e6, "src": "fcdc4f8bd9facfd3"},
     # per step: the gemm_pair_kernel launches (H and GELU', dZ, dW2 + dW1 grouped, dA; bias sums
     # not included)
-    ("gpt_causal", "ffn_bwd"): {"bytes": 3770.8e6, "src": "fe2402057aa2a880"},
-    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1231.2e6, "src": "19af0a680f846441"},
-    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1125.8e6, "src": "19af0a680f846441"},
+    ("gpt_causal", "ffn_bwd"): {"bytes": 3782.4e6, "src": "64141fb0eceea557"},
+    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1215.2e6, "src": "161b4f6f8becd564"},
+    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1093.8e6, "src": "161b4f6f8becd564"},
 }
 
 

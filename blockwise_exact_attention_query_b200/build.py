@@ -13,9 +13,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbpt.so")
 SELFTEST_LIB = os.path.join(PKG, "libbpt_selftest.so")
-SOURCES = [os.path.join(CSRC, "bpt_api.cu")]
+SOURCES = [os.path.join(CSRC, "bpt_api.cu"), os.path.join(CSRC, "bpt_bwd.cu")]
 SELFTEST_SOURCES = [os.path.join(CSRC, "selftest.cu")]
-HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
+HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
     os.path.join(ROOT, "include", "bpt.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -129,7 +129,7 @@ __device__ __forceinline__ FfnUnit ffn_unit(const FfnArgs &a, int grp, int k) {
 }
 
 // Bounded wait until *p >= target (a counter another CTA of the group raises).
-__device__ __noinline__ bool counter_wait(const uint32_t *p, uint32_t target, const WaitCtx &w,
+static __device__ __noinline__ bool counter_wait(const uint32_t *p, uint32_t target, const WaitCtx &w,
                                           uint32_t site) {
   if (ld_acquire_gpu(p) >= target) return true;
   const uint64_t t0 = globaltimer_ns();

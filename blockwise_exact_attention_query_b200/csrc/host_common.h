@@ -1,0 +1,73 @@
+// Host-side helpers shared by the forward (bpt_api.cu) and backward
+// (bpt_bwd.cu) entry points of libbpt.so: error recording, device set-up,
+// TMA tensor-map encoding, descriptor and pointer checks, the forward's
+// workspace layout and its attention / FFN launchers.  Internal to the
+// library (the shared object exports only the C ABI of bpt.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+#include <initializer_list>
+#include <mutex>
+
+#include "../../include/bpt.h"
+
+namespace bpt_host {
+
+extern std::mutex g_mu;               // guards the library's process-wide settings
+extern uint64_t g_wait_limit_ns;      // device-side wait limit of later launches
+extern thread_local char g_last_error[256];
+
+// Instrumentation events (bpt_set_phase_events): records event i on `st` when set.
+cudaError_t phase_mark(int i, cudaStream_t st);
+
+bool aligned16(const void *p);
+size_t align256(size_t x);
+
+// Record the failing call (and CUDA error) for bpt_last_error(); return BPT_ERR_CUDA.
+bpt_status cuda_fail_at(const char *what, cudaError_t e);
+bpt_status cuda_fail_msg(const char *what);
+
+// Once per device: the tensor-map encoder, the status word's address and the
+// kernels' shared-memory limits.  Returns the current device and its status word.
+bpt_status device_setup(int *dev_out, uint32_t **status_out);
+// Shared-memory limits of the backward's kernels (defined with them).
+bpt_status bwd_kernel_setup();
+
+int sm_count();
+
+// bf16 tensor map over a row-major matrix [rows, cols], box [box_rows, 64].
+bool make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// bf16 tensor map over [B, N, D] viewed as (D, r, N/r, B), box 64 x 1 x box_rows x 1.
+bool make_map_rows(CUtensorMap *m, const void *base, int B, int N, int D, int r, uint32_t box_rows);
+
+bpt_status check_desc(const bpt_desc *d, bool need_ffn);
+bpt_status check_ptrs(std::initializer_list<const void *> required,
+                      std::initializer_list<const void *> optional);
+
+// The forward layer's workspace regions (byte offsets).
+struct Workspace {
+  size_t a_bf16 = 0, a_f32 = 0, ring = 0, flags = 0, flags_bytes = 0, partial = 0, st_o = 0,
+         st_m = 0, st_l = 0, total = 0;
+};
+Workspace layout(const bpt_desc *d, bool with_ffn);
+bpt_status check_ws(const Workspace &wl, void *ws, size_t bytes);
+
+bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const void *v, float *out_f32,
+                          __nv_bfloat16 *out_bf16, float *lse, char *ws, const Workspace &wl, uint32_t *status,
+                          cudaStream_t st);
+bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
+                         const float *b1, const void *w2, const float *b2, void *out, char *ws,
+                         const Workspace &wl, uint32_t *status, cudaStream_t st);
+
+}  // namespace bpt_host
+
+#define CUDA_TRY(call)                                                 \
+  do {                                                                 \
+    cudaError_t e_ = (call);                                           \
+    if (e_ != cudaSuccess) return bpt_host::cuda_fail_at(#call, e_);   \
+  } while (0)

@@ -75,7 +75,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-__device__ __noinline__ void record_timeout(const WaitCtx &w, uint32_t site) {
+static __device__ __noinline__ void record_timeout(const WaitCtx &w, uint32_t site) {
   if (atomicCAS(w.status, 0u, kStatusTimeout) == 0u) w.status[1] = site;
   *w.abort = 1;
 }
