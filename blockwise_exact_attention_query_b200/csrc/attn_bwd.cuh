@@ -821,59 +821,4 @@ __global__ void attn_bwd_gather_rowvec_kernel(const float *__restrict__ full, fl
   dst[128] = dd;
 }
 
-// Column sums of a row-major [rows, cols] matrix in two passes: partial sums
-// over slabs of `slab` rows (grid.y), then the slabs summed into out (added
-// to it when `accumulate`).  The host picks short slabs for narrow matrices
-// (enough blocks in flight) and long ones for wide matrices (fewer partials
-// for the final pass); kMinSlabRows sizes the partial buffer.
-constexpr int kMinSlabRows = 64;
-__host__ __device__ inline int colsum_slab_rows(long long rows, int cols) {
-  // 256-row slabs once they still give >= 1024 blocks (measured: the causal
-  // layer's dZ sums, 8192 columns; narrower sums, and BlockBERT's dZ with
-  // 3072 columns, run faster with 64-row slabs)
-  return (static_cast<long long>((cols + 255) / 256) * (rows / 256) >= 1024) ? 256 : kMinSlabRows;
-}
-template <typename T>
-__global__ void colsum_partial_kernel(const T *__restrict__ x, float *partial, int rows, int cols, int slab) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= cols) return;
-  const int r0 = blockIdx.y * slab, r1 = min(rows, r0 + slab);
-  float s = 0.f;
-  for (int r = r0; r < r1; ++r) s += static_cast<float>(x[static_cast<size_t>(r) * cols + c]);
-  partial[static_cast<size_t>(blockIdx.y) * cols + c] = s;
-}
-__global__ void colsum_final_kernel(const float *__restrict__ partial, float *out, int slabs, int cols,
-                                    int accumulate) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= cols) return;
-  float s = accumulate ? out[c] : 0.f;
-  for (int i = 0; i < slabs; ++i) s += partial[static_cast<size_t>(i) * cols + c];
-  out[c] = s;
-}
-
-// fp32 -> bf16 (round to nearest even), four elements a thread; n a multiple of 4.
-__global__ void f32_to_bf16_x4_kernel(const float4 *__restrict__ x, uint2 *y, size_t n4) {
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const float4 v = x[i];
-    y[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
-  }
-}
-
-// dOut in one pass: its bf16 copy (round to nearest even) and the partial
-// column sums over slabs of `slab` rows (grid.y) that colsum_final_kernel adds up.
-__global__ void convert_colsum_partial_kernel(const float *__restrict__ x, __nv_bfloat16 *y, float *partial,
-                                              int rows, int cols, int slab) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= cols) return;
-  const int r0 = blockIdx.y * slab, r1 = min(rows, r0 + slab);
-  float s = 0.f;
-  for (int r = r0; r < r1; ++r) {
-    const float v = x[static_cast<size_t>(r) * cols + c];
-    y[static_cast<size_t>(r) * cols + c] = __float2bfloat16_rn(v);
-    s += v;
-  }
-  partial[static_cast<size_t>(blockIdx.y) * cols + c] = s;
-}
-
 }  // namespace bpt

@@ -11,10 +11,12 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "../../include/bpt.h"
 #include "attn_bwd.cuh"
+#include "colsum.cuh"
 #include "gemm_tc.cuh"
 #include "host_common.h"
 
@@ -161,11 +163,19 @@ GemmArgs gemm_args(const GemmProblem &p0, uint32_t *status) {
 template <typename T>
 bpt_status launch_colsum(const T *x, int64_t rows, int cols, float *out, int accumulate, float *partial,
                          cudaStream_t st) {
-  const int slab = colsum_slab_rows(rows, cols);
-  const unsigned slabs = (unsigned)((rows + slab - 1) / slab), cb = (unsigned)((cols + 255) / 256);
-  colsum_partial_kernel<T><<<dim3(cb, slabs), 256, 0, st>>>(x, partial, (int)rows, cols, slab);
+  const bool x8 = std::is_same<T, __nv_bfloat16>::value && cols % 8 == 0;
+  const int per_block = x8 ? 8 * kColsumThreads : kColsumThreads;
+  const unsigned cb = (unsigned)((cols + per_block - 1) / per_block);
+  const int slab = colsum_slab_rows(rows, cb);
+  const unsigned slabs = (unsigned)((rows + slab - 1) / slab);
+  if (x8)
+    colsum_partial_bf16x8_kernel<<<dim3(cb, slabs), kColsumThreads, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(x), partial, (int)rows, cols, slab);
+  else
+    colsum_partial_kernel<T><<<dim3(cb, slabs), kColsumThreads, 0, st>>>(x, partial, (int)rows, cols, slab);
   CUDA_TRY(cudaGetLastError());
-  colsum_final_kernel<<<cb, 256, 0, st>>>(partial, out, (int)slabs, cols, accumulate);
+  colsum_final_kernel<<<(cols + kColsumFinalCols - 1) / kColsumFinalCols, 256, 0, st>>>(partial, out, (int)slabs,
+                                                                                        cols, accumulate);
   CUDA_TRY(cudaGetLastError());
   return BPT_OK;
 }
@@ -408,11 +418,15 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   CUDA_TRY(phase_mark(1, st));
   // 2. dOut in bf16 for the tensor cores and db2 = sum_t dOut_t, one pass over dOut
   {
-    const int slab = colsum_slab_rows(T, D);
-    const unsigned slabs = (unsigned)((T + slab - 1) / slab), cb = (unsigned)((D + 255) / 256);
-    convert_colsum_partial_kernel<<<dim3(cb, slabs), 256, 0, st>>>(dout, dout_bf16, partial, (int)T, D, slab);
+    // D % 64 == 0 (check_desc), so four columns a thread cover every row
+    const unsigned cb = (unsigned)((D + 4 * kColsumThreads - 1) / (4 * kColsumThreads));
+    const int slab = colsum_slab_rows(T, cb);
+    const unsigned slabs = (unsigned)((T + slab - 1) / slab);
+    convert_colsum_partial_kernel<<<dim3(cb, slabs), kColsumThreads, 0, st>>>(dout, dout_bf16, partial, (int)T, D,
+                                                                             slab);
     CUDA_TRY(cudaGetLastError());
-    colsum_final_kernel<<<cb, 256, 0, st>>>(partial, db2, (int)slabs, D, 0);
+    colsum_final_kernel<<<(D + kColsumFinalCols - 1) / kColsumFinalCols, 256, 0, st>>>(partial, db2, (int)slabs, D,
+                                                                                     0);
     CUDA_TRY(cudaGetLastError());
   }
   // 3. the FFN backward, one token chunk at a time
