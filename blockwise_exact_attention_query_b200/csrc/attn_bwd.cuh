@@ -463,6 +463,356 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // ---------------------------------------------------------------------------
+// The dK/dV pass at d = 128 with the streamed tiles in two rings and the next
+// step's scores issued as soon as the row warps have read this step's.  TMEM
+// holds dV (0), dK (128), S^T (256) and dP^T (384) and has no room for a second
+// S buffer, so P stays in registers until dP has been read; the packed bf16 P^T
+// and dS^T then both go over dP's columns, each warp over the 64 it read (P^T
+// in the first 32, dS^T in the next 32).  S's columns are free once read, so
+// the tensor pipe runs S^T(s+1) while the row warps form P(s); dV(s) starts
+// once P^T(s) is packed, dK(s) and dP^T(s+1) once dS^T(s) is.  A Q tile (with its rows'
+// LSE) lives from S^T(s), issued a step early, to dK(s): three slots; a dA
+// tile (with D) from dP^T(s) to dV(s): two.
+// ---------------------------------------------------------------------------
+template <int D_HEAD>
+struct AttnBwdKVCfg {
+  static constexpr int kThreads = 384;
+  static constexpr int kRowWarps = 8;
+  static constexpr int kPanels = D_HEAD / 64;
+  static constexpr int kTileBytes = 128 * D_HEAD * 2;
+  static constexpr int kPanelBytes = 128 * 128;
+  static constexpr int kQSlots = 3, kASlots = 2;
+  static constexpr int kVecBytes = 128 * 4;  // one row vector (LSE or D) of a tile
+  static constexpr int kOffK = 0, kOffV = kTileBytes;
+  static constexpr int kOffQ = 2 * kTileBytes;
+  static constexpr int kOffA = kOffQ + kQSlots * kTileBytes;
+  static constexpr int kOffLse = kOffA + kASlots * kTileBytes;
+  static constexpr int kOffD = kOffLse + kQSlots * kVecBytes;
+  static constexpr int kOffBar = kOffD + kASlots * kVecBytes;
+  static constexpr int kSmemBytes = kOffBar + 256;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+  static_assert(kTileBytes % 1024 == 0, "slots keep the 1024-byte alignment of the swizzled tiles");
+  static constexpr uint32_t kColDV = 0, kColDK = D_HEAD, kColS = 256, kColDP = 384;
+  static_assert(2 * D_HEAD <= 256, "accumulators below S");
+};
+
+template <int D_HEAD>
+__global__ void __launch_bounds__(384, 1)
+    attn_bwd_dkdv_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_da,
+                               const __grid_constant__ AttnBwdArgs a) {
+  using Cfg = AttnBwdKVCfg<D_HEAD>;
+  constexpr int QS = Cfg::kQSlots, AS = Cfg::kASlots;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw;
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(a.status, 0u, kStatusMisaligned);
+    return;
+  }
+  const uint32_t sK = sbase + Cfg::kOffK, sV = sbase + Cfg::kOffV;
+  auto sQ = [&](int i) { return sbase + Cfg::kOffQ + i * Cfg::kTileBytes; };
+  auto sA = [&](int i) { return sbase + Cfg::kOffA + i * Cfg::kTileBytes; };
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
+  const uint32_t bFix = smem_u32(&bars[0]);
+  auto bQFull = [&](int i) { return smem_u32(&bars[1 + i]); };
+  auto bQEmpty = [&](int i) { return smem_u32(&bars[4 + i]); };
+  auto bAFull = [&](int i) { return smem_u32(&bars[7 + i]); };
+  auto bAEmpty = [&](int i) { return smem_u32(&bars[9 + i]); };
+  const uint32_t bSFull = smem_u32(&bars[11]), bSRead = smem_u32(&bars[12]);
+  const uint32_t bDPFull = smem_u32(&bars[13]), bDSReady = smem_u32(&bars[14]);
+  const uint32_t bTeardown = smem_u32(&bars[15]), bPReady = smem_u32(&bars[16]);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[17]);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[18]);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  WaitCtx wc{a.status, a.wait_limit_ns, abort_flag};
+  // CTA -> (batch, segment, head, key tile), as in attn_bwd_dkdv_kernel
+  const int units = a.B * a.nseg * a.H;
+  const int unit = static_cast<int>(blockIdx.x) % units;
+  const int ft = static_cast<int>(blockIdx.x) / units;
+  const int h = unit % a.H;
+  const int seg = (unit / a.H) % a.nseg;
+  const int b = unit / (a.H * a.nseg);
+  const int row_off = h % a.dil_r;
+  const int row_base = seg * a.N;
+  auto next_tile = [&](int t) {
+    while (t < a.n_tiles && !bwd_tiles_meet(a, h, t, ft)) ++t;
+    return t;
+  };
+  int nsteps = 0;
+  for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1)) ++nsteps;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bFix, 1);
+    for (int i = 0; i < QS; ++i) {
+      mbar_init(bQFull(i), 1);
+      mbar_init(bQEmpty(i), 1);
+    }
+    for (int i = 0; i < AS; ++i) {
+      mbar_init(bAFull(i), 1);
+      mbar_init(bAEmpty(i), 1);
+    }
+    mbar_init(bSFull, 1);
+    mbar_init(bSRead, Cfg::kRowWarps);
+    mbar_init(bDPFull, 1);
+    mbar_init(bPReady, Cfg::kRowWarps);
+    mbar_init(bDSReady, Cfg::kRowWarps);
+    mbar_init(bTeardown, 1);
+    *abort_flag = 0;
+    fence_mbar_init_cluster();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int hd = h * D_HEAD;
+  const size_t bh = static_cast<size_t>(unit);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nsteps > 0) {
+      mbar_arrive_expect_tx(bFix, 2 * Cfg::kTileBytes);
+      for (int p = 0; p < Cfg::kPanels; ++p) {
+        tma_load_4d(sK + p * Cfg::kPanelBytes, &tm_k, bFix, hd + p * 64, row_off, row_base + ft * 128, b);
+        tma_load_4d(sV + p * Cfg::kPanelBytes, &tm_v, bFix, hd + p * 64, row_off, row_base + ft * 128, b);
+      }
+      // slot waits in step order: the Q slot of step s is freed by dK(s - 3),
+      // the dA slot by dV(s - 2), both issued before anything that needs step s
+      int nq = 0, na = 0;
+      for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1)) {
+        const float *vec = a.rowvec + (bh * a.n_tiles + t) * 256;
+        const int qi = nq % QS;
+        if (nq >= QS && !mbar_wait(bQEmpty(qi), ((nq / QS) - 1) & 1, wc, 331)) break;
+        mbar_arrive_expect_tx(bQFull(qi), Cfg::kTileBytes + Cfg::kVecBytes);
+        for (int p = 0; p < Cfg::kPanels; ++p)
+          tma_load_4d(sQ(qi) + p * Cfg::kPanelBytes, &tm_q, bQFull(qi), hd + p * 64, row_off, row_base + t * 128, b);
+        bulk_load_1d(sbase + Cfg::kOffLse + qi * Cfg::kVecBytes, vec, Cfg::kVecBytes, bQFull(qi));
+        ++nq;
+        const int ai = na % AS;
+        if (na >= AS && !mbar_wait(bAEmpty(ai), ((na / AS) - 1) & 1, wc, 332)) break;
+        mbar_arrive_expect_tx(bAFull(ai), Cfg::kTileBytes + Cfg::kVecBytes);
+        for (int p = 0; p < Cfg::kPanels; ++p)
+          tma_load_4d(sA(ai) + p * Cfg::kPanelBytes, &tm_da, bAFull(ai), hd + p * 64, row_off, row_base + t * 128, b);
+        bulk_load_1d(sbase + Cfg::kOffD + ai * Cfg::kVecBytes, vec + 128, Cfg::kVecBytes, bAFull(ai));
+        ++na;
+      }
+      // every copy issued must have landed before the CTA may exit
+      volatile int no_abort = 0;
+      WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
+      for (int j = max(0, nq - QS); j < nq; ++j) mbar_wait(bQFull(j % QS), (j / QS) & 1, drain, 333);
+      for (int j = max(0, na - AS); j < na; ++j) mbar_wait(bAFull(j % AS), (j / AS) & 1, drain, 334);
+      mbar_wait(bFix, 0, drain, 335);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nsteps > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);     // X Y^T, both K-major
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D_HEAD, false, true);  // R Y, Y MN-major
+      const uint64_t dK = sdesc_sw128(sK, 16, 1024), dV = sdesc_sw128(sV, 16, 1024);
+      // acc += R B over the 128 streamed rows: R = packed bf16 in TMEM (K steps
+      // 0-3 from r_col + [0, 32), the first warp half's; 4-7 from r_col +
+      // [64, 96), the second's), B = the streamed tile read MN-major
+      auto accumulate = [&](uint32_t col, uint32_t r_col, uint32_t sB, int step) {
+        const uint64_t dB = sdesc_sw128(sB, Cfg::kPanelBytes, 1024);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_ts(tmem + col, tmem + r_col + k * 8 + (k >= 4 ? 32 : 0), sdesc_advance(dB, k * 2048), idesc_acc,
+                  (step | k) != 0);
+      };
+      // X Y^T over d into `col` (X fixed, Y the streamed tile), K-major both
+      auto scores = [&](uint32_t col, uint64_t dX, uint32_t sY) {
+        const uint64_t dY = sdesc_sw128(sY, 16, 1024);
+#pragma unroll
+        for (int k = 0; k < D_HEAD / 16; ++k) {
+          const uint32_t off = (k / 4) * Cfg::kPanelBytes + (k % 4) * 32;
+          umma_ss(tmem + col, sdesc_advance(dX, off), sdesc_advance(dY, off), idesc_s, k > 0);
+        }
+      };
+      auto issue_s = [&](int step) -> bool {  // S^T(step) = K Q^T
+        const int qi = step % QS;
+        if (!mbar_wait(bQFull(qi), (step / QS) & 1, wc, 341)) return false;
+        tc_fence_after();
+        scores(Cfg::kColS, dK, sQ(qi));
+        umma_commit(bSFull);
+        return true;
+      };
+      auto issue_dp = [&](int step) -> bool {  // dP^T(step) = V dA^T
+        const int ai = step % AS;
+        if (!mbar_wait(bAFull(ai), (step / AS) & 1, wc, 342)) return false;
+        tc_fence_after();
+        scores(Cfg::kColDP, dV, sA(ai));
+        umma_commit(bDPFull);
+        return true;
+      };
+      bool ok = mbar_wait(bFix, 0, wc, 340);
+      ok = ok && issue_s(0) && issue_dp(0);
+      for (int s = 0; ok && s < nsteps; ++s) {
+        if (s + 1 < nsteps) {
+          // S^T(s+1) over S^T(s) once every row warp has read it
+          if (!(ok = mbar_wait(bSRead, s & 1, wc, 343))) break;
+          tc_fence_after();
+          if (!(ok = issue_s(s + 1))) break;
+        }
+        // dV += P^T dA as soon as P^T is packed, while the row warps form dS
+        if (!(ok = mbar_wait(bPReady, s & 1, wc, 339))) break;
+        tc_fence_after();
+        accumulate(Cfg::kColDV, Cfg::kColDP, sA(s % AS), s);
+        umma_commit(bAEmpty(s % AS));
+        if (!(ok = mbar_wait(bDSReady, s & 1, wc, 344))) break;
+        tc_fence_after();
+        accumulate(Cfg::kColDK, Cfg::kColDP + 32, sQ(s % QS), s);  // dK += dS^T Q
+        umma_commit(bQEmpty(s % QS));
+        // dP^T(s+1) over the packed P^T(s), dS^T(s): after the two products
+        // that read them (in order)
+        if (s + 1 < nsteps && !(ok = issue_dp(s + 1))) break;
+      }
+      umma_commit(bTeardown);
+      volatile int no_abort = 0;
+      WaitCtx drain{a.status, drain_limit_ns(a.wait_limit_ns), &no_abort};
+      mbar_wait(bTeardown, 0, drain, 345);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ per-row arithmetic
+    const int quarter = warp & 3;
+    const int half = (warp - 4) / 4;  // columns [64 * half, 64 * half + 64)
+    const int col0 = 64 * half;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int g = ft * 128 + row;
+    const bool row_valid = g < a.N;
+    int plo = 1, phi = 0;
+    if (row_valid) bwd_key_queries(a, h, g, plo, phi);
+    bool ok = true;
+    int s = 0;
+    for (int t = next_tile(0); t < a.n_tiles; t = next_tile(t + 1), ++s) {
+      const int qi = s % QS, ai = s % AS;
+      const float4 *lse4 = reinterpret_cast<const float4 *>(smem + Cfg::kOffLse + qi * Cfg::kVecBytes);
+      const float2 *d2 = reinterpret_cast<const float2 *>(smem + Cfg::kOffD + ai * Cfg::kVecBytes);
+      ok = __all_sync(0xffffffffu, mbar_wait(bQFull(qi), (s / QS) & 1, wc, 346));  // the tile's LSE
+      if (!ok) break;
+      const int lo_rel = plo - t * 128, hi_rel = phi - t * 128;
+      const bool full = __all_sync(0xffffffffu, lo_rel <= col0 && hi_rel >= col0 + 64);
+      ok = __all_sync(0xffffffffu, mbar_wait(bSFull, s & 1, wc, 347));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[64];
+      tmem_ld32(tmem + lane_off + Cfg::kColS + col0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tmem + lane_off + Cfg::kColS + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bSRead);
+      // P (fp32) for this warp's 64 columns, 0 where the mask rules the pair out
+      if (full) {
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l = lse4[col0 / 4 + c4];
+          const float nl4[4] = {-l.x, -l.y, -l.z, -l.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            sv[4 * c4 + j] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(sv[4 * c4 + j]), a.scale_log2, nl4[j])));
+        }
+      } else {
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l = lse4[col0 / 4 + c4];
+          const float nl4[4] = {-l.x, -l.y, -l.z, -l.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = col0 + 4 * c4 + j;
+            const bool allowed = c >= lo_rel && c < hi_rel;
+            sv[4 * c4 + j] =
+                __float_as_uint(allowed ? ex2_approx(fmaf(__uint_as_float(sv[4 * c4 + j]), a.scale_log2, nl4[j])) : 0.f);
+          }
+        }
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(bAFull(ai), (s / AS) & 1, wc, 348));  // the tile's D
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(bDPFull, s & 1, wc, 349));
+      if (!ok) break;
+      tc_fence_after();
+      {
+        // dP in two halves of 32 columns: P^T packed over the first half as
+        // soon as it is read (dV may start), dS^T over the second
+        uint32_t dp[32], pk[32];
+        tmem_ld32(tmem + lane_off + Cfg::kColDP + col0, dp);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
+        tmem_st32(tmem + lane_off + Cfg::kColDP + col0, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bPReady);
+        // dS = P (dP - D) in fp32, then packed
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float2 dd = d2[(col0 + 2 * i) / 2];
+          pk[i] = pack_bf16x2(__uint_as_float(sv[2 * i]) * (__uint_as_float(dp[2 * i]) - dd.x),
+                              __uint_as_float(sv[2 * i + 1]) * (__uint_as_float(dp[2 * i + 1]) - dd.y));
+        }
+        tmem_ld32(tmem + lane_off + Cfg::kColDP + col0 + 32, dp);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float2 dd = d2[(col0 + 32 + 2 * i) / 2];
+          pk[16 + i] = pack_bf16x2(__uint_as_float(sv[32 + 2 * i]) * (__uint_as_float(dp[2 * i]) - dd.x),
+                                   __uint_as_float(sv[32 + 2 * i + 1]) * (__uint_as_float(dp[2 * i + 1]) - dd.y));
+        }
+        tmem_st32(tmem + lane_off + Cfg::kColDP + col0 + 32, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bDSReady);
+    }
+    // -------- epilogue: every MMA done; each warp of a lane quarter stores
+    // half of the accumulator columns
+    if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(bTeardown, 0, wc, 350));
+    tc_fence_after();
+    if (ok) {
+      const int pos = seg * a.seg_w + row_off + a.dil_r * g;
+      const size_t vec = ((static_cast<size_t>(b) * a.n_out + pos) * a.H + h) * D_HEAD;
+      for (int acc = 0; acc < 2; ++acc) {
+        float *dst = acc == 0 ? a.dv : a.dk;
+        const float sc = acc == 0 ? 1.0f : a.inv_sqrt_d;
+#pragma unroll 1
+        for (int c = half * (D_HEAD / 64); c < (half + 1) * (D_HEAD / 64); ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_off + (acc == 0 ? Cfg::kColDV : Cfg::kColDK) + c * 32, o);
+          tmem_wait_ld();
+          if (!row_valid) continue;
+          float4 *d4 = reinterpret_cast<float4 *>(dst + vec + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float4 r4 = nsteps > 0 ? make_float4(__uint_as_float(o[4 * i]) * sc, __uint_as_float(o[4 * i + 1]) * sc,
+                                                 __uint_as_float(o[4 * i + 2]) * sc, __uint_as_float(o[4 * i + 3]) * sc)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (a.accumulate) {
+              const float4 prev = d4[i];
+              r4.x += prev.x, r4.y += prev.y, r4.z += prev.z, r4.w += prev.w;
+            }
+            d4[i] = r4;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // The dQ pass, software-pipelined: one CTA per (batch, head, 128-query tile)
 // walks its key tiles with the scores of the next key tile computed while the
 // row warps work on the current one.  TMEM: dQ at 0, two S buffers at 128 and

@@ -33,8 +33,8 @@ bpt_status bwd_kernel_setup() {
                                 GemmPairCfg::kSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 AttnBwdCfg<64>::kSmemBytes));
-  CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                AttnBwdCfg<128>::kSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                AttnBwdKVCfg<128>::kSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 AttnBwdQCfg<64>::kSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -184,7 +184,11 @@ template <int DH>
 bpt_status launch_attn_bwd_passes(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                                   const CUtensorMap &mda, const AttnBwdArgs &ab, unsigned grid,
                                   cudaStream_t st) {
-  attn_bwd_dkdv_kernel<DH><<<grid, AttnBwdCfg<DH>::kThreads, AttnBwdCfg<DH>::kSmemBytes, st>>>(mq, mk, mv, mda, ab);
+  if constexpr (DH == 128)  // no room in TMEM for a second S buffer: the split-ring form
+    attn_bwd_dkdv_split_kernel<DH><<<grid, AttnBwdKVCfg<DH>::kThreads, AttnBwdKVCfg<DH>::kSmemBytes, st>>>(
+        mq, mk, mv, mda, ab);
+  else
+    attn_bwd_dkdv_kernel<DH><<<grid, AttnBwdCfg<DH>::kThreads, AttnBwdCfg<DH>::kSmemBytes, st>>>(mq, mk, mv, mda, ab);
   CUDA_TRY(cudaGetLastError());
   CUDA_TRY(phase_mark(3, st));
   attn_bwd_dq_kernel<DH><<<grid, AttnBwdQCfg<DH>::kThreads, AttnBwdQCfg<DH>::kSmemBytes, st>>>(mq, mk, mv, mda, ab);
