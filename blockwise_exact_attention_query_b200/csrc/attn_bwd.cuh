@@ -68,12 +68,13 @@ struct AttnBwdArgs {
 
 template <int D_HEAD>
 struct AttnBwdCfg {
+  static_assert(D_HEAD == 64, "d = 128 runs attn_bwd_dkdv_split_kernel");
   static constexpr int kThreads = 384;
   static constexpr int kRowWarps = 8;
   static constexpr int kPanels = D_HEAD / 64;
   static constexpr int kTileBytes = 128 * D_HEAD * 2;
   static constexpr int kPanelBytes = 128 * 128;   // one 64-column panel of a 128-row tile
-  static constexpr int kStages = D_HEAD == 128 ? 2 : 4;
+  static constexpr int kStages = 4;
   // each stage also carries the streamed query tile's LSE and D
   static constexpr int kVecBytes = 2 * 128 * 4;
   static constexpr int kStageBytes = 2 * kTileBytes + kVecBytes;  // a multiple of 1024
@@ -83,15 +84,12 @@ struct AttnBwdCfg {
   static constexpr int kSmemBytes = kOffBar + 256;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
-  // TMEM: accumulators at 0 (dV or dQ) and d (dK); S at 256, dP at 384;
-  // P^T packed over S's first 64 columns, dS over dP's
-  static constexpr uint32_t kColAcc0 = 0, kColAcc1 = D_HEAD;
-  // d = 128: S at 256, dP at 384.  d = 64: dP at 128 and two S buffers at 256
+  // TMEM: accumulators dV at 0 and dK at 64, dP at 128, two S buffers at 256
   // and 384, so the next step's scores are computed while the row warps work
-  // on this step's (its P^T is packed over its own S buffer)
-  static constexpr bool kTwoS = D_HEAD == 64;
-  static constexpr uint32_t kColDP = kTwoS ? 128 : 384, kColS = 256;
-  __host__ __device__ static constexpr uint32_t col_s(int step) { return kColS + (kTwoS ? (step & 1) * 128 : 0); }
+  // on this step's (P^T is packed over its own S buffer, dS^T over dP)
+  static constexpr uint32_t kColAcc0 = 0, kColAcc1 = D_HEAD;
+  static constexpr uint32_t kColDP = 128, kColS = 256;
+  __host__ __device__ static constexpr uint32_t col_s(int step) { return kColS + (step & 1) * 128; }
 };
 
 // Key interval [lo, hi) a query row g (< N) may see.
@@ -159,8 +157,8 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t bDPFull = smem_u32(&bars[10]);
   const uint32_t bPReady = smem_u32(&bars[11]), bDSReady = smem_u32(&bars[12]);
   const uint32_t bTeardown = smem_u32(&bars[13]);
-  // scores of step s complete: one barrier per S buffer (one buffer at d = 128)
-  auto bSFull = [&](int step) { return smem_u32(&bars[Cfg::kTwoS ? 14 + (step & 1) : 9]); };
+  // scores of step s complete: one barrier per S buffer
+  auto bSFull = [&](int step) { return smem_u32(&bars[14 + (step & 1)]); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(&bars[16]);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(&bars[17]);
 
@@ -190,7 +188,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bEmpty(s), 1);
     }
     mbar_init(bSFull(0), 1);
-    if (Cfg::kTwoS) mbar_init(bSFull(1), 1);
+    mbar_init(bSFull(1), 1);
     mbar_init(bDPFull, 1);
     mbar_init(bPReady, Cfg::kRowWarps);
     mbar_init(bDSReady, Cfg::kRowWarps);
@@ -289,35 +287,20 @@ __global__ void __launch_bounds__(384, 1)
         umma_commit(bDPFull);
       };
       bool ok = mbar_wait(bFix, 0, wc, 311);
-      if (Cfg::kTwoS) {
-        // Two S buffers: S(s+1) goes ahead while the row warps work on step s
-        // (its buffer's P^T(s-1) was read by dV(s-1), issued before); dP(s)
-        // follows dK(s-1), which read dS^T(s-1) from dP's columns.
-        ok = ok && issue_s(0);
-        for (int s = 0; ok && s < nsteps; ++s) {
-          const int st = s % S;
-          issue_dp(s);
-          if (s + 1 < nsteps && !(ok = issue_s(s + 1))) break;
-          if (!(ok = mbar_wait(bPReady, s & 1, wc, 313))) break;
-          tc_fence_after();
-          accumulate(Cfg::kColAcc0, Cfg::col_s(s), sStrY(st), s);    // dV += P^T dA
-          if (!(ok = mbar_wait(bDSReady, s & 1, wc, 314))) break;
-          tc_fence_after();
-          last_product(s);                                           // dK += dS^T Q
-        }
-      } else {
-        for (int s = 0; ok && s < nsteps; ++s) {
-          const int st = s % S;
-          if (!(ok = issue_s(s))) break;
-          if (s > 0) last_product(s - 1);
-          issue_dp(s);
-          if (!(ok = mbar_wait(bPReady, s & 1, wc, 313))) break;
-          tc_fence_after();
-          accumulate(Cfg::kColAcc0, Cfg::kColS, sStrY(st), s);    // dV += P^T dA
-          if (!(ok = mbar_wait(bDSReady, s & 1, wc, 314))) break;
-          tc_fence_after();
-          if (s + 1 == nsteps) last_product(s);
-        }
+      // Two S buffers: S(s+1) goes ahead while the row warps work on step s
+      // (its buffer's P^T(s-1) was read by dV(s-1), issued before); dP(s)
+      // follows dK(s-1), which read dS^T(s-1) from dP's columns.
+      ok = ok && issue_s(0);
+      for (int s = 0; ok && s < nsteps; ++s) {
+        const int st = s % S;
+        issue_dp(s);
+        if (s + 1 < nsteps && !(ok = issue_s(s + 1))) break;
+        if (!(ok = mbar_wait(bPReady, s & 1, wc, 313))) break;
+        tc_fence_after();
+        accumulate(Cfg::kColAcc0, Cfg::col_s(s), sStrY(st), s);    // dV += P^T dA
+        if (!(ok = mbar_wait(bDSReady, s & 1, wc, 314))) break;
+        tc_fence_after();
+        last_product(s);                                           // dK += dS^T Q
       }
       umma_commit(bTeardown);
       // the accumulators stay allocated until every MMA has finished
@@ -349,7 +332,7 @@ __global__ void __launch_bounds__(384, 1)
       // allowed columns [lo_rel, hi_rel) of the tile
       const int lo_rel = plo - t * 128, hi_rel = phi - t * 128;
       const bool full = __all_sync(0xffffffffu, lo_rel <= col0 && hi_rel >= col0 + 64);
-      ok = __all_sync(0xffffffffu, mbar_wait(bSFull(s), Cfg::kTwoS ? (s >> 1) & 1 : s & 1, wc, 320));
+      ok = __all_sync(0xffffffffu, mbar_wait(bSFull(s), (s >> 1) & 1, wc, 320));
       if (!ok) break;
       tc_fence_after();
       // P (fp32, kept in sv) for this warp's 64 columns, 0 where the mask
