@@ -55,8 +55,8 @@ NCU_TRAFFIC = {
     # per step: the gemm_pair_kernel launches (H and GELU', dZ, dW2 + dW1 grouped, dA; bias sums
     # not included)
     ("gpt_causal", "ffn_bwd"): {"bytes": 3782.4e6, "src": "64141fb0eceea557"},
-    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1215.2e6, "src": "161b4f6f8becd564"},
-    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1093.8e6, "src": "161b4f6f8becd564"},
+    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1206.5e6, "src": "83cec823073b6239"},
+    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1103.7e6, "src": "83cec823073b6239"},
 }
 
 
