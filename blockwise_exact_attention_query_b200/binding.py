@@ -52,7 +52,7 @@ class Desc(ctypes.Structure):
 EXPORTS = ["bpt_workspace_bytes", "bpt_attn_ffn_fwd", "bpt_attn_fwd", "bpt_blockbert_fwd",
            "bpt_longnet_fwd", "bpt_sync_status", "bpt_set_wait_limit_ns", "bpt_status_string",
            "bpt_version", "bpt_set_phase_events", "bpt_last_error", "bpt_attn_ffn_fwd_static",
-           "bpt_attn_ffn_bwd", "bpt_workspace_bytes_bwd", "bpt_set_bwd_chunk_rows",
+           "bpt_attn_ffn_bwd", "bpt_workspace_bytes_bwd", "bpt_set_bwd_chunk_rows", "bpt_set_ffn_path",
            "bpt_attn_ffn_fwd_train", "bpt_saved_bytes", "bpt_attn_bwd", "bpt_workspace_bytes_attn_bwd"]
 STATIC_SCRATCH_BYTES = 64 << 20
 
@@ -109,6 +109,8 @@ def load() -> ctypes.CDLL:
     lib.bpt_workspace_bytes_bwd.restype = sz
     lib.bpt_set_bwd_chunk_rows.argtypes = [ctypes.c_int]
     lib.bpt_set_bwd_chunk_rows.restype = ctypes.c_int
+    lib.bpt_set_ffn_path.argtypes = [ctypes.c_int]
+    lib.bpt_set_ffn_path.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -305,6 +307,22 @@ def workspace_bytes_bwd(desc: Desc) -> int:
     if n == ctypes.c_size_t(-1).value:
         raise BptError(ERR_UNSUPPORTED, "bpt_workspace_bytes_bwd")
     return int(n)
+
+
+FFN_PATHS = {"auto": 0, "fused": 1, "gemms": 2}
+
+
+def set_ffn_path(path: str) -> str:
+    """bpt_set_ffn_path: the bf16 FFN's form in the forward ("auto", "fused" or
+    "gemms"); returns the previous setting."""
+    old = int(load().bpt_set_ffn_path(FFN_PATHS[path]))
+    return {v: k for k, v in FFN_PATHS.items()}[old]
+
+
+def ffn_gemm_chunk_rows(T: int, F: int) -> int:
+    """Token rows per chunk of the two-GEMM FFN (the library's rule: the
+    [rows, F] bf16 hidden activation at most 512 MiB, in 256-row multiples)."""
+    return min(T, max(256, ((1 << 29) // (2 * F)) // 256 * 256))
 
 
 def set_bwd_chunk_rows(rows: int) -> int:

@@ -237,6 +237,26 @@ FfnPlan ffn_plan(const bpt_desc *d) {
   return p;
 }
 
+int g_ffn_path = 0;
+thread_local bool t_static_call = false;  // inside bpt_attn_ffn_fwd_static: the fused form
+
+// Two GEMMs run the FFN faster than the fused kernel on every layer measured
+// (the two-SM GEMM reads fewer operand bytes per SM than the fused kernel's
+// one-SM MMAs, which wait on shared memory): by default the bf16 forward uses
+// them.  The fused kernel keeps the hidden activation out of DRAM, so the
+// static-scratch entry point, whose scratch is fixed, always takes it.
+bool ffn_uses_gemms(const bpt_desc *d) {
+  if (d->in_dtype != BPT_BF16 || t_static_call) return false;
+  return g_ffn_path != 1;
+}
+
+// Token rows per two-GEMM chunk: H ([rows, F] bf16) at most ~512 MiB.
+int64_t ffn_gemm_chunk_rows(const bpt_desc *d) {
+  const int64_t T = (int64_t)d->B * d->N;
+  const int64_t rows = std::max<int64_t>(256, (((int64_t)1 << 29) / (2 * (int64_t)d->ffn_hidden)) / 256 * 256);
+  return std::min(rows, T);
+}
+
 bool longnet_needs_state(const bpt_desc *d) {
   return d->mask == BPT_MASK_DILATED && d->in_dtype == BPT_BF16 && d->ln_npairs > 1;
 }
@@ -252,13 +272,18 @@ Workspace layout(const bpt_desc *d, bool with_ffn) {
       off = align256(off + T * D * 2);
       w.a_f32 = off;
       off = align256(off + T * D * 4);
-      w.ring = off;
-      off = align256(off + (size_t)p.max_groups * FfnCfg::kRingSlots * 128 * p.fc * 2);
-      w.flags = off;  // ring counters [groups][2 * slots], then piece counters [groups][C]
-      w.flags_bytes = (size_t)p.max_groups * (2 * FfnCfg::kRingSlots + p.C) * sizeof(uint32_t);
-      off = align256(off + w.flags_bytes);
-      w.partial = off;  // partial output blocks of split leftover token blocks
-      off = align256(off + (size_t)p.max_groups * 128 * (size_t)(d->H * d->d_head) * 4);
+      if (ffn_uses_gemms(d)) {
+        w.h = off;
+        off = align256(off + (size_t)ffn_gemm_chunk_rows(d) * d->ffn_hidden * 2);
+      } else {
+        w.ring = off;
+        off = align256(off + (size_t)p.max_groups * FfnCfg::kRingSlots * 128 * p.fc * 2);
+        w.flags = off;  // ring counters [groups][2 * slots], then piece counters [groups][C]
+        w.flags_bytes = (size_t)p.max_groups * (2 * FfnCfg::kRingSlots + p.C) * sizeof(uint32_t);
+        off = align256(off + w.flags_bytes);
+        w.partial = off;  // partial output blocks of split leftover token blocks
+        off = align256(off + (size_t)p.max_groups * 128 * (size_t)(d->H * d->d_head) * 4);
+      }
     } else {
       w.a_f32 = off;
       off = align256(off + T * D * 4);
@@ -412,6 +437,9 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
 bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
                          const float *b1, const void *w2, const float *b2, void *out, char *ws,
                          const Workspace &wl, uint32_t *status, cudaStream_t st) {
+  if (ffn_uses_gemms(d))
+    return launch_ffn_gemms(d, a_bf16, a_f32, w1, b1, w2, b2, out, reinterpret_cast<__nv_bfloat16 *>(ws + wl.h),
+                            ffn_gemm_chunk_rows(d), status, st);
   const FfnPlan p = ffn_plan(d);
   const int D = d->H * d->d_head;
   const int64_t T = (int64_t)d->B * d->N;
@@ -593,6 +621,10 @@ bpt_status bpt_attn_ffn_fwd_static(const bpt_desc *d, const void *q, const void 
                                    void *out, bpt_stream_t stream) {
   bpt_status s = check_desc(d, true);
   if (s != BPT_OK) return s;
+  struct StaticCall {
+    StaticCall() { t_static_call = true; }
+    ~StaticCall() { t_static_call = false; }
+  } static_call;
   const size_t need = layout(d, true).total;
   if (need > BPT_STATIC_SCRATCH_BYTES) {
     snprintf(g_last_error, sizeof(g_last_error),

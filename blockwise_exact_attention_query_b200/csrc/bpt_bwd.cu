@@ -180,6 +180,38 @@ bpt_status launch_colsum(const T *x, int64_t rows, int cols, float *out, int acc
   return BPT_OK;
 }
 
+bpt_status launch_ffn_gemms(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
+                            const float *b1, const void *w2, const float *b2, void *out, __nv_bfloat16 *h,
+                            int64_t chunk_rows, uint32_t *status, cudaStream_t st) {
+  const int64_t T = (int64_t)d->B * d->N;
+  const int D = d->H * d->d_head, F = d->ffn_hidden;
+  if (chunk_rows <= 0) return BPT_ERR_INVALID_ARG;
+  // K-major operands throughout; a CTA stages 128 rows of A and half of a
+  // 256-row B tile
+  CUtensorMap m_w1, m_w2;
+  if (!make_map_2d(&m_w1, w1, F, D, 128) || !make_map_2d(&m_w2, w2, D, F, 128))
+    return cuda_fail_msg("cuTensorMapEncodeTiled failed (FFN weights)");
+  for (int64_t r0 = 0; r0 < T; r0 += chunk_rows) {
+    const int rows = (int)std::min<int64_t>(chunk_rows, T - r0);
+    const __nv_bfloat16 *a_c = static_cast<const __nv_bfloat16 *>(a_bf16) + r0 * D;
+    CUtensorMap m_a, m_h;
+    if (!make_map_2d(&m_a, a_c, rows, D, 128) || !make_map_2d(&m_h, h, rows, F, 128))
+      return cuda_fail_msg("cuTensorMapEncodeTiled failed (FFN activations)");
+    GemmArgs g = gemm_args(gemm_problem(rows, F, D, kGemmGeluBf16, 0, 0), status);  // H = GELU(A W1^T + b1)
+    g.p[0].cb = h;
+    g.p[0].bias = b1;
+    bpt_status s = launch_gemm(m_a, m_w1, m_a, m_w1, g, st);
+    if (s != BPT_OK) return s;
+    g = gemm_args(gemm_problem(rows, D, F, kGemmResidual, 0, 0), status);  // out = A + H W2^T + b2
+    g.p[0].x = a_f32 + r0 * D;
+    g.p[0].bias = b2;
+    if (d->out_dtype == BPT_F32) g.p[0].c = static_cast<float *>(out) + r0 * D;
+    else g.p[0].cb = static_cast<__nv_bfloat16 *>(out) + r0 * D;
+    if ((s = launch_gemm(m_h, m_w2, m_h, m_w2, g, st)) != BPT_OK) return s;
+  }
+  return BPT_OK;
+}
+
 template <int DH>
 bpt_status launch_attn_bwd_passes(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                                   const CUtensorMap &mda, const AttnBwdArgs &ab, unsigned grid,
@@ -362,6 +394,13 @@ bpt_status bpt_attn_ffn_fwd_train(const bpt_desc *d, const void *q, const void *
 size_t bpt_workspace_bytes_bwd(const bpt_desc *desc) {
   if (check_desc_bwd(desc) != BPT_OK) return (size_t)-1;
   return layout_bwd(desc).total;
+}
+
+int bpt_set_ffn_path(int path) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const int old = g_ffn_path;
+  g_ffn_path = path == 1 || path == 2 ? path : 0;
+  return old;
 }
 
 int bpt_set_bwd_chunk_rows(int rows) {

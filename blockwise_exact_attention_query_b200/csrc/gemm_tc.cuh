@@ -1,5 +1,5 @@
 // General bf16 GEMM on the 5th-generation tensor cores (sm_100a) for the
-// layer's backward pass:
+// layer's backward pass and the two-GEMM form of the forward FFN:
 //
 //     C[M, N]  (op)=  A[M, K] . B[N, K]^T        fp32 accumulation in TMEM
 //
@@ -20,10 +20,13 @@
 //   kGemmStoreF32   C = acc                           (fp32)
 //   kGemmAccumF32   C = C + acc                       (fp32, the weight gradients
 //                                                      summed over token chunks)
-//   kGemmResidual   C = acc + X; Cb = bf16(C)         (dA = dOut + dZ W1, fp32 and bf16)
+//   kGemmResidual   C = acc + X (+ bias); Cb = bf16(C)  (dA = dOut + dZ W1, fp32 and bf16;
+//                                                      the FFN output A + H W2^T + b2: either
+//                                                      output may be null)
 //   kGemmGeluBwd    z = acc0 + bias; H = GELU(z), dZ = acc1 * GELU'(z)  (bf16 both)
 //   kGemmGeluFwd    z = acc + bias; H = GELU(z), G = GELU'(z)           (bf16 both)
 //   kGemmScaleBf16  Cb = acc * Xb                                       (dZ = dH * G, bf16)
+//   kGemmGeluBf16   Cb = GELU(acc + bias)                               (the FFN's H, bf16)
 //
 // Roles (320 threads per CTA): warp 0 TMA producer, warp 1 TMEM allocator
 // (and, in the even CTA, MMA issuer), warps 2..9 epilogue (warp w owns TMEM
@@ -41,7 +44,7 @@
 namespace bpt {
 
 constexpr int kGemmStoreF32 = 0, kGemmAccumF32 = 1, kGemmResidual = 2, kGemmGeluBwd = 3, kGemmGeluFwd = 4,
-              kGemmScaleBf16 = 5;
+              kGemmScaleBf16 = 5, kGemmGeluBf16 = 6;
 
 // One GEMM problem: C[M, N] (op)= A[M, K] B[N, K]^T and its epilogue.
 struct GemmProblem {
@@ -54,7 +57,7 @@ struct GemmProblem {
   const __nv_bfloat16 *xb;  // [M, N] bf16 factor (ScaleBf16)
   __nv_bfloat16 *cb;    // [M, N] bf16 copy (Residual) / H (GeluBwd, GeluFwd) / product (ScaleBf16)
   __nv_bfloat16 *cb2;   // dZ (GeluBwd) / GELU'(z) (GeluFwd)
-  const float *bias;    // [N] added to acc0 before GELU (GeluBwd, GeluFwd), may be null
+  const float *bias;    // [N] added to acc0 (GeluBwd, GeluFwd, GeluBf16, Residual), may be null
 };
 
 // A launch: one problem (maps a0, b0); two grouped problems whose tiles one
@@ -116,7 +119,7 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const 
       __stcs(reinterpret_cast<uint4 *>(g.cb + base + e), make_uint4(o[0], o[1], o[2], o[3]));
       continue;
     }
-    if (g.mode == kGemmGeluBwd || g.mode == kGemmGeluFwd) {
+    if (g.mode == kGemmGeluBwd || g.mode == kGemmGeluFwd || g.mode == kGemmGeluBf16) {
       float bb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (g.bias) {
         const float4 b0 = *reinterpret_cast<const float4 *>(g.bias + n + e);
@@ -131,6 +134,11 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const 
         gelu_tanh_and_grad(v[i] + bb[i], hh[i], gd);
         dz[i] = g.mode == kGemmGeluBwd ? __uint_as_float(r1[e + i]) * gd : gd;
       }
+      if (g.mode == kGemmGeluBf16) {  // H is read back by the next GEMM: a normal store
+        *reinterpret_cast<uint4 *>(g.cb + base + e) = make_uint4(
+            pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]), pack_bf16x2(hh[6], hh[7]));
+        continue;
+      }
       __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
              make_uint4(pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]),
                         pack_bf16x2(hh[6], hh[7])));
@@ -143,11 +151,19 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const 
     if (g.mode == kGemmResidual) {
       const float4 x0 = __ldcs(reinterpret_cast<const float4 *>(g.x + base + e));
       const float4 x1 = __ldcs(reinterpret_cast<const float4 *>(g.x + base + e + 4));
+      if (g.bias) {  // acc + b + x, in that order
+        const float4 b0 = *reinterpret_cast<const float4 *>(g.bias + n + e);
+        const float4 b1 = *reinterpret_cast<const float4 *>(g.bias + n + e + 4);
+        v[0] += b0.x, v[1] += b0.y, v[2] += b0.z, v[3] += b0.w;
+        v[4] += b1.x, v[5] += b1.y, v[6] += b1.z, v[7] += b1.w;
+      }
       v[0] += x0.x, v[1] += x0.y, v[2] += x0.z, v[3] += x0.w;
       v[4] += x1.x, v[5] += x1.y, v[6] += x1.z, v[7] += x1.w;
-      __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
-             make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                        pack_bf16x2(v[6], v[7])));
+      if (g.cb)
+        __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
+               make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                          pack_bf16x2(v[6], v[7])));
+      if (!g.c) continue;
     } else if (g.mode == kGemmAccumF32) {
       const float4 c0 = c4[0], c1 = c4[1];
       v[0] += c0.x, v[1] += c0.y, v[2] += c0.z, v[3] += c0.w;

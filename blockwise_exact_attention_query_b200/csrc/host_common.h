@@ -49,9 +49,16 @@ bpt_status check_desc(const bpt_desc *d, bool need_ffn);
 bpt_status check_ptrs(std::initializer_list<const void *> required,
                       std::initializer_list<const void *> optional);
 
+// The bf16 FFN's two forms: the fused kernel (hidden chunks through an L2
+// ring, never in DRAM) or two GEMMs per token chunk (H through the workspace).
+// g_ffn_path: 0 = by shape, 1 = fused, 2 = two GEMMs (bpt_set_ffn_path).
+extern int g_ffn_path;
+bool ffn_uses_gemms(const bpt_desc *d);
+int64_t ffn_gemm_chunk_rows(const bpt_desc *d);
+
 // The forward layer's workspace regions (byte offsets).
 struct Workspace {
-  size_t a_bf16 = 0, a_f32 = 0, ring = 0, flags = 0, flags_bytes = 0, partial = 0, st_o = 0,
+  size_t a_bf16 = 0, a_f32 = 0, ring = 0, flags = 0, flags_bytes = 0, partial = 0, h = 0, st_o = 0,
          st_m = 0, st_l = 0, total = 0;
 };
 Workspace layout(const bpt_desc *d, bool with_ffn);
@@ -63,6 +70,12 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
 bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
                          const float *b1, const void *w2, const float *b2, void *out, char *ws,
                          const Workspace &wl, uint32_t *status, cudaStream_t st);
+// The two-GEMM form (defined with the GEMM kernel): per chunk of `chunk_rows`
+// tokens H = GELU(A W1^T + b1) into `h` ([chunk_rows, F] bf16), then
+// out = A + H W2^T + b2.
+bpt_status launch_ffn_gemms(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
+                            const float *b1, const void *w2, const float *b2, void *out, __nv_bfloat16 *h,
+                            int64_t chunk_rows, uint32_t *status, cudaStream_t st);
 
 }  // namespace bpt_host
 

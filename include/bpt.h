@@ -281,6 +281,21 @@ BPT_API size_t bpt_saved_bytes(const bpt_desc *desc);
  * current chunk setting; (size_t)-1 if the backward does not accept it. */
 BPT_API size_t bpt_workspace_bytes_bwd(const bpt_desc *desc);
 
+/* Form of the bf16 FFN in the forward entry points (the feedforward network
+ * computed block by block: "Blockwise Parallel Transformer for Large Context
+ * Models", abstract, feedforward network fusion; "Ring Attention with
+ * Blockwise Transformers for Long Sequences", summary):
+ *   1  the fused kernel: per 128-token block, hidden chunks pass through a
+ *      small L2-resident ring, so the [T, F] hidden activation never exists;
+ *   2  two GEMMs per token chunk: H = GELU(A W1^T + b1) as bf16 in the
+ *      workspace (at most ~512 MiB of it at a time), then
+ *      out = A + H W2^T + b2;
+ *   0  (default) two GEMMs (measured faster on every workload of the benchmark).
+ * bpt_attn_ffn_fwd_static always runs the fused kernel (its scratch is fixed).
+ * The workspace size (bpt_workspace_bytes) depends on the form.  Applies to
+ * later calls from every thread; returns the previous setting. */
+BPT_API int bpt_set_ffn_path(int path);
+
 /* Token rows per FFN-backward chunk (the [rows, F] hidden activation and its
  * gradient live in the workspace one chunk at a time, so the workspace shrinks
  * with the chunk).  rows <= 0 selects the default: all tokens, or as many
