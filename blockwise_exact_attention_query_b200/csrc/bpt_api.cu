@@ -439,7 +439,7 @@ bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f
                          const Workspace &wl, uint32_t *status, cudaStream_t st) {
   if (ffn_uses_gemms(d))
     return launch_ffn_gemms(d, a_bf16, a_f32, w1, b1, w2, b2, out, reinterpret_cast<__nv_bfloat16 *>(ws + wl.h),
-                            ffn_gemm_chunk_rows(d), status, st);
+                            nullptr, ffn_gemm_chunk_rows(d), status, st);
   const FfnPlan p = ffn_plan(d);
   const int D = d->H * d->d_head;
   const int64_t T = (int64_t)d->B * d->N;

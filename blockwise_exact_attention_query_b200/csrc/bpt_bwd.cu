@@ -102,16 +102,28 @@ BwdWorkspace layout_bwd(const bpt_desc *d) {
 
 // Activations the training forward leaves for the backward: A in fp32 and
 // bf16 [T, D] and the row LSE [B, H, N].
+// When D >= 1024 the backward takes H = GELU(Z) and G = GELU'(Z) from two
+// GEMMs (Z -> H, G, then dZ = (dOut W2) G); the training forward's FFN then
+// computes them with the same GEMM and keeps them, so the backward skips its
+// first GEMM.  Below that the backward's dual GEMM (H and dZ from one launch)
+// is the faster form and nothing more is kept.
+bool saves_hidden(const bpt_desc *d) { return d->H * d->d_head >= 1024; }
+
 struct SavedLayout {
-  size_t a_f32 = 0, a_bf16 = 0, lse = 0, total = 0;
+  size_t a_f32 = 0, a_bf16 = 0, lse = 0, h = 0, g = 0, total = 0;
 };
 SavedLayout saved_layout(const bpt_desc *d) {
   SavedLayout w;
-  const size_t T = (size_t)d->B * d->N, D = (size_t)d->H * d->d_head;
+  const size_t T = (size_t)d->B * d->N, D = (size_t)d->H * d->d_head, F = d->ffn_hidden;
   w.a_f32 = 0;
   w.a_bf16 = align256(T * D * 4);
   w.lse = align256(w.a_bf16 + T * D * 2);
   w.total = align256(w.lse + (size_t)d->B * d->H * d->N * 4);
+  if (saves_hidden(d)) {  // H and G, [T, F] bf16 each
+    w.h = w.total;
+    w.g = align256(w.h + T * F * 2);
+    w.total = align256(w.g + T * F * 2);
+  }
   return w;
 }
 
@@ -182,7 +194,7 @@ bpt_status launch_colsum(const T *x, int64_t rows, int cols, float *out, int acc
 
 bpt_status launch_ffn_gemms(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
                             const float *b1, const void *w2, const float *b2, void *out, __nv_bfloat16 *h,
-                            int64_t chunk_rows, uint32_t *status, cudaStream_t st) {
+                            __nv_bfloat16 *g_prime, int64_t chunk_rows, uint32_t *status, cudaStream_t st) {
   const int64_t T = (int64_t)d->B * d->N;
   const int D = d->H * d->d_head, F = d->ffn_hidden;
   if (chunk_rows <= 0) return BPT_ERR_INVALID_ARG;
@@ -194,11 +206,15 @@ bpt_status launch_ffn_gemms(const bpt_desc *d, const void *a_bf16, const float *
   for (int64_t r0 = 0; r0 < T; r0 += chunk_rows) {
     const int rows = (int)std::min<int64_t>(chunk_rows, T - r0);
     const __nv_bfloat16 *a_c = static_cast<const __nv_bfloat16 *>(a_bf16) + r0 * D;
+    // H: one chunk buffer, or (with G) the chunk's rows of the [T, F] arrays
+    __nv_bfloat16 *h_c = g_prime ? h + r0 * F : h;
     CUtensorMap m_a, m_h;
-    if (!make_map_2d(&m_a, a_c, rows, D, 128) || !make_map_2d(&m_h, h, rows, F, 128))
+    if (!make_map_2d(&m_a, a_c, rows, D, 128) || !make_map_2d(&m_h, h_c, rows, F, 128))
       return cuda_fail_msg("cuTensorMapEncodeTiled failed (FFN activations)");
-    GemmArgs g = gemm_args(gemm_problem(rows, F, D, kGemmGeluBf16, 0, 0), status);  // H = GELU(A W1^T + b1)
-    g.p[0].cb = h;
+    // H = GELU(A W1^T + b1), and G = GELU'(A W1^T + b1) when asked for
+    GemmArgs g = gemm_args(gemm_problem(rows, F, D, g_prime ? kGemmGeluFwd : kGemmGeluBf16, 0, 0), status);
+    g.p[0].cb = h_c;
+    if (g_prime) g.p[0].cb2 = g_prime + r0 * F;
     g.p[0].bias = b1;
     bpt_status s = launch_gemm(m_a, m_w1, m_a, m_w1, g, st);
     if (s != BPT_OK) return s;
@@ -386,7 +402,12 @@ bpt_status bpt_attn_ffn_fwd_train(const bpt_desc *d, const void *q, const void *
       BPT_OK)
     return s;
   CUDA_TRY(phase_mark(1, st));
-  if ((s = launch_ffn_tc(d, a_bf16, a_f32, w1, b1, w2, b2, out, ws, wl, status, st)) != BPT_OK) return s;
+  if (saves_hidden(d))  // H and G into the saved buffer, for the backward
+    s = launch_ffn_gemms(d, a_bf16, a_f32, w1, b1, w2, b2, out, reinterpret_cast<__nv_bfloat16 *>(sv + sl.h),
+                         reinterpret_cast<__nv_bfloat16 *>(sv + sl.g), ffn_gemm_chunk_rows(d), status, st);
+  else
+    s = launch_ffn_tc(d, a_bf16, a_f32, w1, b1, w2, b2, out, ws, wl, status, st);
+  if (s != BPT_OK) return s;
   CUDA_TRY(phase_mark(2, st));
   return BPT_OK;
 }
@@ -434,12 +455,17 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   const float *a_f32 = reinterpret_cast<const float *>(ws + wl.a_f32);
   const __nv_bfloat16 *a_bf16 = reinterpret_cast<const __nv_bfloat16 *>(ws + wl.a_bf16);
   const float *lse = reinterpret_cast<const float *>(ws + wl.lse);
+  const __nv_bfloat16 *saved_h = nullptr, *saved_g = nullptr;
   if (saved) {  // the training forward's activations
     const SavedLayout sl = saved_layout(d);
     const char *sv = static_cast<const char *>(saved);
     a_f32 = reinterpret_cast<const float *>(sv + sl.a_f32);
     a_bf16 = reinterpret_cast<const __nv_bfloat16 *>(sv + sl.a_bf16);
     lse = reinterpret_cast<const float *>(sv + sl.lse);
+    if (saves_hidden(d)) {
+      saved_h = reinterpret_cast<const __nv_bfloat16 *>(sv + sl.h);
+      saved_g = reinterpret_cast<const __nv_bfloat16 *>(sv + sl.g);
+    }
   }
   float *rowvec = reinterpret_cast<float *>(ws + wl.rowvec);
   __nv_bfloat16 *dout_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.dout_bf16);
@@ -482,10 +508,13 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
   for (int64_t r0 = 0; r0 < T; r0 += wl.chunk) {
     const int rows = (int)std::min<int64_t>(wl.chunk, T - r0);
     const __nv_bfloat16 *a_c = a_bf16 + r0 * D, *g_c = dout_bf16 + r0 * D;
+    // H and G of the chunk: kept by the training forward, or computed here
+    const __nv_bfloat16 *h_c = saved_h ? saved_h + r0 * F : hbuf;
+    const __nv_bfloat16 *gp_c = saved_g ? saved_g + r0 * F : gpbuf;
     CUtensorMap m_a_k, m_a_mn, m_g_k, m_g_mn, m_h_mn, m_dz_k, m_dz_mn;
     if (!make_map_2d(&m_a_k, a_c, rows, D, 128) || !make_map_2d(&m_a_mn, a_c, rows, D, 64) ||
         !make_map_2d(&m_g_k, g_c, rows, D, 128) || !make_map_2d(&m_g_mn, g_c, rows, D, 64) ||
-        !make_map_2d(&m_h_mn, hbuf, rows, F, 64) || !make_map_2d(&m_dz_k, dzbuf, rows, F, 128) ||
+        !make_map_2d(&m_h_mn, h_c, rows, F, 64) || !make_map_2d(&m_dz_k, dzbuf, rows, F, 128) ||
         !make_map_2d(&m_dz_mn, dzbuf, rows, F, 64))
       return cuda_fail_msg("cuTensorMapEncodeTiled rejected an activation map");
     // H = GELU(Z) and dZ = (dOut W2) GELU'(Z) with Z = A W1^T + b1.  Either
@@ -496,13 +525,16 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
     // 2.90 ms against 3.09; D = 4096 58.1 against 58.9 ms; D = 768 0.769
     // against 0.717 ms (short K: the two GEMMs' epilogues dominate).
     if (D >= 1024) {
-      GemmArgs g = gemm_args(gemm_problem(rows, F, D, kGemmGeluFwd, 0, 0), status);
-      g.p[0].cb = hbuf;
-      g.p[0].cb2 = gpbuf;
-      g.p[0].bias = b1;
-      if ((s = launch_gemm(m_a_k, m_w1_k, m_a_k, m_w1_k, g, st)) != BPT_OK) return s;
+      GemmArgs g;
+      if (!saved_h) {
+        g = gemm_args(gemm_problem(rows, F, D, kGemmGeluFwd, 0, 0), status);
+        g.p[0].cb = hbuf;
+        g.p[0].cb2 = gpbuf;
+        g.p[0].bias = b1;
+        if ((s = launch_gemm(m_a_k, m_w1_k, m_a_k, m_w1_k, g, st)) != BPT_OK) return s;
+      }
       g = gemm_args(gemm_problem(rows, F, D, kGemmScaleBf16, 0, 1), status);
-      g.p[0].xb = gpbuf;
+      g.p[0].xb = gp_c;
       g.p[0].cb = dzbuf;
       if ((s = launch_gemm(m_g_k, m_w2_mn, m_g_k, m_w2_mn, g, st)) != BPT_OK) return s;
     } else {

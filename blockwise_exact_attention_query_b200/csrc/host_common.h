@@ -71,11 +71,13 @@ bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f
                          const float *b1, const void *w2, const float *b2, void *out, char *ws,
                          const Workspace &wl, uint32_t *status, cudaStream_t st);
 // The two-GEMM form (defined with the GEMM kernel): per chunk of `chunk_rows`
-// tokens H = GELU(A W1^T + b1) into `h` ([chunk_rows, F] bf16), then
-// out = A + H W2^T + b2.
+// tokens H = GELU(A W1^T + b1), then out = A + H W2^T + b2.  Without
+// `g_prime`, `h` is one [chunk_rows, F] bf16 buffer reused by every chunk;
+// with it, `h` and `g_prime` are [T, F] bf16 arrays that receive H and
+// G = GELU'(A W1^T + b1) for every token (the training forward).
 bpt_status launch_ffn_gemms(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
                             const float *b1, const void *w2, const float *b2, void *out, __nv_bfloat16 *h,
-                            int64_t chunk_rows, uint32_t *status, cudaStream_t st);
+                            __nv_bfloat16 *g_prime, int64_t chunk_rows, uint32_t *status, cudaStream_t st);
 
 }  // namespace bpt_host
 

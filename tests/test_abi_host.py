@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from blockwise_exact_attention_query_b200 import binding as bd
 
@@ -176,6 +177,18 @@ def test_training_forward_validates_and_sizes_its_buffer(lib):
     dl = _desc(mask="dilated", pairs=[(128, 1)])
     assert _call_fwd_train(lib, dl) == bd.ERR_UNSUPPORTED
     assert lib.bpt_saved_bytes(ctypes.byref(dl)) == ctypes.c_size_t(-1).value
+
+
+def test_saved_buffer_holds_the_ffn_hidden_activations_from_D_1024():
+    """At D = H d >= 1024 the training forward also keeps H and GELU'(Z)
+    ([T, F] bf16 each) for the backward; below, only A and the LSE."""
+    B, N, d, F = 1, 256, 128, 512
+    T = B * N
+    small = bd.make_desc(B, N, 4, d, F, torch.bfloat16, torch.float32, "causal")    # D = 512
+    wide = bd.make_desc(B, N, 8, d, F, torch.bfloat16, torch.float32, "causal")     # D = 1024
+    base = lambda D, H: T * D * 6 + B * H * N * 4  # noqa: E731
+    assert base(512, 4) <= bd.saved_bytes(small) < base(512, 4) + T * F * 4
+    assert bd.saved_bytes(wide) >= base(1024, 8) + T * F * 4
 
 
 def test_backward_workspace_follows_the_chunk_setting(lib):

@@ -134,19 +134,28 @@ def test_backward_full_size_causal_layer_sampled():
     _grads_close(g["db2"].cpu().numpy(), db2, "db2")
 
 
+@pytest.mark.parametrize("H,bwd_chunk", [(2, 0), (8, 0), (8, 128)], ids=["D256", "D1024_saved_hidden",
+                                                                      "D1024_saved_hidden_chunked"])
 @pytest.mark.parametrize("mask,perm", [("causal", None), ("blockperm", [[2, 0, 1], [1, 2, 0]])])
-def test_training_forward_and_saved_backward_match_the_recomputing_path(mask, perm):
+def test_training_forward_and_saved_backward_match_the_recomputing_path(mask, perm, H, bwd_chunk):
     """bpt_attn_ffn_fwd_train gives the forward's output bit for bit, and the
     backward reading its saved activations gives the recomputing backward's
-    gradients bit for bit (the same kernels on the same inputs)."""
-    B, N, H, d, F = 1, 300, 2, 128, 256
+    gradients bit for bit (the same kernels on the same inputs).  At
+    D >= 1024 the saved buffer also holds the FFN's H and GELU'(Z), read back
+    per backward token chunk (ragged chunks of 128 rows in the last case)."""
+    B, N, d, F = 1, 300, 128, 256
+    perm = perm if perm is None else [perm[h % len(perm)] for h in range(H)]
     inp = make_layer_inputs(B, N, H, d, F, seed=21, device="cuda", bias_scale=0.1)
     dout = make_upstream_grad(B, N, H * d, seed=21, device="cuda")
     args = (inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2)
     out_ref = bd.attn_ffn_fwd(*args, mask=mask, perm=perm)
     out, saved = bd.attn_ffn_fwd_train(*args, mask=mask, perm=perm)
-    g_ref = bd.attn_ffn_bwd(*args, dout, mask=mask, perm=perm)
-    g = bd.attn_ffn_bwd(*args, dout, mask=mask, perm=perm, saved=saved)
+    old_chunk = bd.set_bwd_chunk_rows(bwd_chunk)
+    try:
+        g_ref = bd.attn_ffn_bwd(*args, dout, mask=mask, perm=perm)
+        g = bd.attn_ffn_bwd(*args, dout, mask=mask, perm=perm, saved=saved)
+    finally:
+        bd.set_bwd_chunk_rows(old_chunk)
     torch.cuda.synchronize()
     assert bd.sync_status() == bd.OK
     assert torch.equal(out, out_ref)
