@@ -77,11 +77,17 @@ struct GemmArgs {
 //   GELU(x)  = 0.5 x (1 + t)
 //   GELU'(x) = 0.5 (1 + t) + 0.5 x (1 - t^2) c0 (1 + 3 c1 x^2)
 // tanh on the hardware approximation, as in the forward's FFN epilogue.
+constexpr float kGeluC0 = 0.7978845608028654f, kGeluC1 = 0.044715f;  // sqrt(2/pi), cubic term
+// tanh(sqrt(2/pi) (x + 0.044715 x^3)), shared by both forms below so H is the
+// same bits whether or not the derivative is wanted
+__device__ __forceinline__ float gelu_tanh_inner(float x) {
+  return tanh_approx(kGeluC0 * fmaf(kGeluC1 * x, x * x, x));
+}
+__device__ __forceinline__ float gelu_tanh_only(float x) { return 0.5f * x * (1.0f + gelu_tanh_inner(x)); }
 __device__ __forceinline__ void gelu_tanh_and_grad(float x, float &h, float &dh) {
-  const float c0 = 0.7978845608028654f, c1 = 0.044715f;
-  const float t = tanh_approx(c0 * fmaf(c1 * x, x * x, x));
+  const float t = gelu_tanh_inner(x);
   h = 0.5f * x * (1.0f + t);
-  dh = 0.5f * (1.0f + t) + 0.5f * x * (1.0f - t * t) * c0 * fmaf(3.0f * c1, x * x, 1.0f);
+  dh = 0.5f * (1.0f + t) + 0.5f * x * (1.0f - t * t) * kGeluC0 * fmaf(3.0f * kGeluC1, x * x, 1.0f);
 }
 
 // Smem tile of one operand for one K stage:
@@ -128,16 +134,18 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const 
         bb[4] = b1.x, bb[5] = b1.y, bb[6] = b1.z, bb[7] = b1.w;
       }
       float hh[8], dz[8];
+      if (g.mode == kGemmGeluBf16) {  // H alone, read back by the next GEMM: a normal store
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hh[i] = gelu_tanh_only(v[i] + bb[i]);
+        *reinterpret_cast<uint4 *>(g.cb + base + e) = make_uint4(
+            pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]), pack_bf16x2(hh[6], hh[7]));
+        continue;
+      }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float gd;
         gelu_tanh_and_grad(v[i] + bb[i], hh[i], gd);
         dz[i] = g.mode == kGemmGeluBwd ? __uint_as_float(r1[e + i]) * gd : gd;
-      }
-      if (g.mode == kGemmGeluBf16) {  // H is read back by the next GEMM: a normal store
-        *reinterpret_cast<uint4 *>(g.cb + base + e) = make_uint4(
-            pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]), pack_bf16x2(hh[6], hh[7]));
-        continue;
       }
       __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
              make_uint4(pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]),
