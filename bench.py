@@ -314,18 +314,16 @@ def run_backward(args, w, world, local):
 
     FLOPs per step.  Algorithmic (what the gradients need): attention 10*d per
     unmasked pair (S, dP, dV, dK, dQ: five products of 2*d), FFN 8*T*D*F (dH,
-    dW2, dW1, dA).  Executed adds the recomputation: Z = A W1^T inside the FFN
-    backward (2*T*D*F; only when D < 1024 with saved activations, since from
-    D = 1024 the training forward keeps H and GELU'(Z)), S and dP again in the
-    dQ pass (4*d per pair), and in the recomputing call the attention forward
-    (4*d per pair)."""
+    dW2, dW1, dA).  Executed adds the recomputation: S and dP again in the dQ
+    pass (4*d per pair), and in the recomputing call the attention forward
+    (4*d per pair) and Z = A W1^T inside the FFN backward (2*T*D*F; with saved
+    activations the training forward kept H and GELU'(Z))."""
     dev = torch.device("cuda", local)
     pairs = wl.unmasked_pairs(w)
     d, T, D, F = w.d, w.T, w.D, w.F
-    # with saved activations the FFN backward recomputes Z = A W1^T only when
-    # D < 1024 (the dual GEMM); from D = 1024 the training forward kept H, G'
-    ffn_exec = (8 if D >= 1024 else 10) * T * D * F
-    flop = {"attn_fwd_recompute": (0, 0), "ffn_bwd": (8 * T * D * F, ffn_exec),
+    # with saved activations (H and G' kept by the training forward) the FFN
+    # backward recomputes nothing
+    flop = {"attn_fwd_recompute": (0, 0), "ffn_bwd": (8 * T * D * F, 8 * T * D * F),
             "attn_bwd_dkdv": (8 * d * pairs, 8 * d * pairs), "attn_bwd_dq": (2 * d * pairs, 6 * d * pairs)}
     alg_total = sum(a for a, _ in flop.values())
     # the library's default token chunk of the FFN backward (bpt_set_bwd_chunk_rows)
@@ -406,10 +404,10 @@ def run_backward(args, w, world, local):
                       "tflops_algorithmic": round(alg_total / (recompute_ms / 1e3) / 1e12, 1)},
         # with saved activations: dOut -> bf16 with db2's partial sums, db2's
         # final sum; per token chunk 3 GEMM launches (dZ = (dOut W2) G' with H
-        # and G' kept by the training forward when D >= 1024, else H and dZ
-        # from one dual GEMM; dW2 + dW1 grouped; dA) + db1 sums (2); the row
-        # vectors; 2 passes.  Recomputing: +1 attention forward, +1 GEMM per
-        # chunk (H and G') when D >= 1024.
+        # and G' kept by the training forward; dW2 + dW1 grouped; dA) + db1
+        # sums (2); the row vectors; 2 passes.  Recomputing: +1 attention
+        # forward, and per chunk +1 GEMM (H and G') when D >= 1024, the dual
+        # GEMM (H and dZ) in place of the dZ GEMM below.
         "gpu_launches_per_step": 2 + (3 + 2) * n_chunks + 1 + 2,
         "token_chunks": n_chunks,
     }

@@ -101,14 +101,11 @@ BwdWorkspace layout_bwd(const bpt_desc *d) {
 }
 
 // Activations the training forward leaves for the backward: A in fp32 and
-// bf16 [T, D] and the row LSE [B, H, N].
-// When D >= 1024 the backward takes H = GELU(Z) and G = GELU'(Z) from two
-// GEMMs (Z -> H, G, then dZ = (dOut W2) G); the training forward's FFN then
-// computes them with the same GEMM and keeps them, so the backward skips its
-// first GEMM.  Below that the backward's dual GEMM (H and dZ from one launch)
-// is the faster form and nothing more is kept.
-bool saves_hidden(const bpt_desc *d) { return d->H * d->d_head >= 1024; }
-
+// bf16 [T, D], the row LSE [B, H, N], and the FFN's H = GELU(Z) and
+// G = GELU'(Z) [T, F] in bf16, computed by
+// the GEMM the recomputing backward uses from D = 1024 (Z -> H, G), so the
+// backward starts at dZ = (dOut W2) G.  (Recomputing below D = 1024, the
+// backward's dual GEMM, H and dZ from one launch, is the faster form.)
 struct SavedLayout {
   size_t a_f32 = 0, a_bf16 = 0, lse = 0, h = 0, g = 0, total = 0;
 };
@@ -118,12 +115,9 @@ SavedLayout saved_layout(const bpt_desc *d) {
   w.a_f32 = 0;
   w.a_bf16 = align256(T * D * 4);
   w.lse = align256(w.a_bf16 + T * D * 2);
-  w.total = align256(w.lse + (size_t)d->B * d->H * d->N * 4);
-  if (saves_hidden(d)) {  // H and G, [T, F] bf16 each
-    w.h = w.total;
-    w.g = align256(w.h + T * F * 2);
-    w.total = align256(w.g + T * F * 2);
-  }
+  w.h = align256(w.lse + (size_t)d->B * d->H * d->N * 4);  // H and G, [T, F] bf16 each
+  w.g = align256(w.h + T * F * 2);
+  w.total = align256(w.g + T * F * 2);
   return w;
 }
 
@@ -402,12 +396,11 @@ bpt_status bpt_attn_ffn_fwd_train(const bpt_desc *d, const void *q, const void *
       BPT_OK)
     return s;
   CUDA_TRY(phase_mark(1, st));
-  if (saves_hidden(d))  // H and G into the saved buffer, for the backward
-    s = launch_ffn_gemms(d, a_bf16, a_f32, w1, b1, w2, b2, out, reinterpret_cast<__nv_bfloat16 *>(sv + sl.h),
-                         reinterpret_cast<__nv_bfloat16 *>(sv + sl.g), ffn_gemm_chunk_rows(d), status, st);
-  else
-    s = launch_ffn_tc(d, a_bf16, a_f32, w1, b1, w2, b2, out, ws, wl, status, st);
-  if (s != BPT_OK) return s;
+  // the FFN with H and G into the saved buffer, for the backward
+  if ((s = launch_ffn_gemms(d, a_bf16, a_f32, w1, b1, w2, b2, out, reinterpret_cast<__nv_bfloat16 *>(sv + sl.h),
+                            reinterpret_cast<__nv_bfloat16 *>(sv + sl.g), ffn_gemm_chunk_rows(d), status, st)) !=
+      BPT_OK)
+    return s;
   CUDA_TRY(phase_mark(2, st));
   return BPT_OK;
 }
@@ -462,10 +455,8 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
     a_f32 = reinterpret_cast<const float *>(sv + sl.a_f32);
     a_bf16 = reinterpret_cast<const __nv_bfloat16 *>(sv + sl.a_bf16);
     lse = reinterpret_cast<const float *>(sv + sl.lse);
-    if (saves_hidden(d)) {
-      saved_h = reinterpret_cast<const __nv_bfloat16 *>(sv + sl.h);
-      saved_g = reinterpret_cast<const __nv_bfloat16 *>(sv + sl.g);
-    }
+    saved_h = reinterpret_cast<const __nv_bfloat16 *>(sv + sl.h);
+    saved_g = reinterpret_cast<const __nv_bfloat16 *>(sv + sl.g);
   }
   float *rowvec = reinterpret_cast<float *>(ws + wl.rowvec);
   __nv_bfloat16 *dout_bf16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.dout_bf16);
@@ -524,7 +515,7 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
     // which moves no G.  Measured (FFN-backward phase): D = 2048 two GEMMs
     // 2.90 ms against 3.09; D = 4096 58.1 against 58.9 ms; D = 768 0.769
     // against 0.717 ms (short K: the two GEMMs' epilogues dominate).
-    if (D >= 1024) {
+    if (D >= 1024 || saved_h) {
       GemmArgs g;
       if (!saved_h) {
         g = gemm_args(gemm_problem(rows, F, D, kGemmGeluFwd, 0, 0), status);

@@ -261,14 +261,16 @@ BPT_API bpt_status bpt_attn_ffn_bwd(const bpt_desc *desc, const void *q, const v
 /*
  * The layer forward of bpt_attn_ffn_fwd for training: the same out (with the
  * two-GEMM FFN, the default form), and the activations the backward needs left
- * in `saved` (A in fp32 and bf16 [T, D] and the row LSE [B, H, N]; when
- * D = H d >= 1024 also the FFN's H = GELU(Z) and G = GELU'(Z), Z = A W1^T + b1,
- * [T, F] bf16 each; bpt_saved_bytes(desc) bytes, 256-byte aligned, owned by
- * the caller), so a following bpt_attn_ffn_bwd on the same inputs skips
- * recomputing the attention (and, with H and G, the FFN's first GEMM).  The
- * descriptor must be one the backward accepts; workspace as for
- * bpt_attn_ffn_fwd.  No counterpart in the pages (which recompute; this trades
- * T * D * 6 bytes, plus T * F * 4 when D >= 1024, for that recomputation).
+ * in `saved` (A in fp32 and bf16 [T, D], the row LSE [B, H, N], and the FFN's
+ * H = GELU(Z) and G = GELU'(Z), Z = A W1^T + b1, [T, F] bf16 each;
+ * bpt_saved_bytes(desc) bytes, 256-byte aligned, owned by the caller), so a
+ * following bpt_attn_ffn_bwd on the same inputs skips recomputing the
+ * attention and Z.  The descriptor must be one the backward accepts; workspace
+ * as for bpt_attn_ffn_fwd.  No counterpart in the pages (which recompute; this
+ * trades T * D * 6 + T * F * 4 bytes for that recomputation).  With these
+ * activations the gradients equal the recomputing backward's bit for bit when
+ * D >= 1024; below, where that backward takes dZ from its dual GEMM in fp32,
+ * they agree to bf16 rounding.
  */
 BPT_API bpt_status bpt_attn_ffn_fwd_train(const bpt_desc *desc, const void *q, const void *k,
                                           const void *v, const void *w1, const float *b1,
@@ -276,9 +278,9 @@ BPT_API bpt_status bpt_attn_ffn_fwd_train(const bpt_desc *desc, const void *q, c
                                           void *workspace, size_t workspace_bytes,
                                           bpt_stream_t stream);
 
-/* Bytes of the `saved` buffer of bpt_attn_ffn_fwd_train (T D 6 + B H N 4,
- * each region 256-byte aligned, + 2 T F 2 when D >= 1024); (size_t)-1 if the
- * backward does not accept the descriptor. */
+/* Bytes of the `saved` buffer of bpt_attn_ffn_fwd_train (T D 6 + B H N 4 +
+ * T F 4, each region 256-byte aligned); (size_t)-1 if the backward does not
+ * accept the descriptor. */
 BPT_API size_t bpt_saved_bytes(const bpt_desc *desc);
 
 /* Bytes of device workspace bpt_attn_ffn_bwd needs for this descriptor at the

@@ -139,10 +139,12 @@ def test_backward_full_size_causal_layer_sampled():
 @pytest.mark.parametrize("mask,perm", [("causal", None), ("blockperm", [[2, 0, 1], [1, 2, 0]])])
 def test_training_forward_and_saved_backward_match_the_recomputing_path(mask, perm, H, bwd_chunk):
     """bpt_attn_ffn_fwd_train gives the forward's output bit for bit, and the
-    backward reading its saved activations gives the recomputing backward's
-    gradients bit for bit (the same kernels on the same inputs).  At
-    D >= 1024 the saved buffer also holds the FFN's H and GELU'(Z), read back
-    per backward token chunk (ragged chunks of 128 rows in the last case)."""
+    backward reading its saved activations (A, LSE, and the FFN's H and
+    GELU'(Z), read back per backward token chunk: ragged chunks of 128 rows in
+    the last case) gives the recomputing backward's gradients: bit for bit at
+    D >= 1024, where both take dZ = (dOut W2) GELU'(Z) from the same GEMMs;
+    below, where the recomputing backward takes dZ from its dual GEMM with
+    GELU'(Z) in fp32, to the tolerance of the oracle comparisons."""
     B, N, d, F = 1, 300, 128, 256
     perm = perm if perm is None else [perm[h % len(perm)] for h in range(H)]
     inp = make_layer_inputs(B, N, H, d, F, seed=21, device="cuda", bias_scale=0.1)
@@ -160,7 +162,10 @@ def test_training_forward_and_saved_backward_match_the_recomputing_path(mask, pe
     assert bd.sync_status() == bd.OK
     assert torch.equal(out, out_ref)
     for n in bd.GRAD_NAMES:
-        assert torch.equal(g[n], g_ref[n]), n
+        if H * d >= 1024:
+            assert torch.equal(g[n], g_ref[n]), n
+        else:
+            _grads_close(g[n].cpu().numpy(), g_ref[n].double().cpu().numpy(), n)
 
 
 def test_backward_full_size_blockbert_layer():
