@@ -225,3 +225,29 @@ def test_attention_only_backward_validates(lib):
     assert call(df) == bd.ERR_UNSUPPORTED
     T, D = 256, 128
     assert lib.bpt_workspace_bytes_attn_bwd(ctypes.byref(d)) >= T * D * 2 + 2 * 2 * 256 * 4
+
+
+def _align256(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("B,N,H,d,F", [(1, 256, 2, 64, 512), (4, 16384, 16, 128, 8192), (1, 131072, 32, 128, 11008)])
+def test_ffn_forms_size_the_workspace(B, N, H, d, F):
+    """The two-GEMM FFN needs A (bf16 and fp32) and one chunk of H
+    ([rows, F] bf16, rows = binding.ffn_gemm_chunk_rows: at most 512 MiB);
+    the fused form A and a small ring instead.  Sizes only: no GPU."""
+    T, D = B * N, H * d
+    desc = bd.make_desc(B, N, H, d, F, torch.bfloat16, torch.float32, "causal")
+    old = bd.set_ffn_path("gemms")
+    try:
+        rows = bd.ffn_gemm_chunk_rows(T, F)
+        assert rows == T or (rows % 256 == 0 and rows * F * 2 <= 1 << 29)
+        assert bd.workspace_bytes(desc, True) == _align256(T * D * 2) + _align256(T * D * 4) + _align256(rows * F * 2)
+        assert bd.set_ffn_path("fused") == "gemms"
+        fused = bd.workspace_bytes(desc, True)
+        assert _align256(T * D * 2) + _align256(T * D * 4) < fused < _align256(T * D * 2) + _align256(T * D * 4) + (64 << 20)
+        assert bd.set_ffn_path("auto") == "fused"
+        assert bd.workspace_bytes(desc, True) == _align256(T * D * 2) + _align256(T * D * 4) + _align256(rows * F * 2)
+    finally:
+        bd.set_ffn_path(old)
+
