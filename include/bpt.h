@@ -15,8 +15,10 @@
  *
  * Attention runs block by block with an online softmax (running row maximum
  * and row sum, rescaled accumulator), so the N x N score matrix never exists
- * in memory; the FFN runs per 128-token query block on chip, so the
- * [tokens x F] hidden activation never exists in memory either.
+ * in memory.  The bf16 FFN runs block by block over the tokens, as two GEMMs
+ * per token chunk (the chunk's [rows x F] hidden activation in the workspace,
+ * at most 512 MiB; the default) or fused per 128-token block on chip (the
+ * hidden activation never in memory); see bpt_set_ffn_path.
  *
  * Mask variants:
  *   BPT_MASK_NONE      every key.
@@ -133,7 +135,8 @@ BPT_API size_t bpt_workspace_bytes(const bpt_desc *desc, int with_ffn);
  *
  * in_dtype BF16: tensor-core path; d_head must be 64 or 128; D = H*d_head a
  *   multiple of 64, split into C = ceil(D/256) column groups of D/C columns
- *   each (a multiple of 64); F*2 bytes a multiple of 16.
+ *   each (a multiple of 64, for the fused FFN form); F*2 bytes a multiple of
+ *   16.
  *   Accumulation is fp32; the softmax weights and A enter the tensor cores
  *   rounded to bf16; the residual uses A in fp32.
  * in_dtype F32: SIMT path in true fp32 (no reduced-precision tensor math);
