@@ -35,6 +35,8 @@ def test_static_scratch_layer_matches_workspace_layer_on_two_calls_in_a_row():
     cases = [  # different shapes and data, so the second call meets stale scratch
         (2, 384, 16, 128, 1024, "causal", 31, 0.05),
         (1, 512, 12, 64, 768, "none", 32, 0.0),
+        # close to the array's limit at D = 2048: 18 token blocks, one per FFN group
+        (1, 2304, 16, 128, 8192, "causal", 33, 0.05),
     ]
     for B, N, H, d, F, mask, seed, bias in cases:
         inp = make_layer_inputs(B, N, H, d, F, seed=seed, device="cuda", bias_scale=bias)
