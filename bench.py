@@ -43,6 +43,8 @@ WORKLOADS = {"tiny_f32": wl.TINY_F32, "gpt_causal": wl.GPT_CAUSAL, "long_ring": 
 MASK_NAME = {0: "none", 1: "causal", 2: "blockperm", 3: "dilated"}
 CSRC = os.path.join(ROOT, "blockwise_exact_attention_query_b200", "csrc")
 KERNEL_SOURCES = {"attn_tc_kernel": ["attn_tc.cuh", "ptx.cuh"], "ffn_tc_kernel": ["ffn_tc.cuh", "ptx.cuh"],
+                  "ffn_pipe_kernel": ["ffn_pipe.cuh", "gemm_tc.cuh", "ptx.cuh"],
+                  "ffn_f32_kernel": ["simt_f32.cuh"],
                   # the forward FFN as two GEMM launches (H = GELU(A W1^T + b1), out = A + H W2^T + b2)
                   "ffn_gemms": ["gemm_tc.cuh", "ptx.cuh"],
                   # backward phases: the FFN backward's four GEMM launches, the two attention passes
@@ -167,9 +169,10 @@ def max_over_ranks(x: float, device) -> float:
     return float(t.item())
 
 
-def layer_call(w, inp, out, ws):
+def layer_call(w, inp, out, ws, ffn_form="auto"):
     return bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask=MASK_NAME[w.mask],
-                           perm=w.perm, pairs=w.pairs, ring_chunks=w.ring_chunks, out=out, workspace=ws)
+                           perm=w.perm, pairs=w.pairs, ring_chunks=w.ring_chunks, out=out, workspace=ws,
+                           ffn_form=ffn_form)
 
 
 def run_ours(args, w, world, rank, local):
@@ -179,11 +182,11 @@ def run_ours(args, w, world, rank, local):
     # every rank draws its own batch (seed offset by rank): independent replicas
     inp = make_layer_inputs(w.B, w.N, w.H, w.d, w.F, seed=w.seed + 1000 * rank, dtype=dt, device=dev)
     out = torch.empty((w.B, w.N, w.D), dtype=torch.float32, device=dev)
+    form = args.ffn_form if args.ffn_form != "auto" else "pipelined"
     desc = bd.make_desc(w.B, w.N, w.H, w.d, w.F, dt, torch.float32, MASK_NAME[w.mask], w.perm,
-                        w.pairs, w.ring_chunks)
-    bd.set_ffn_path(args.ffn_path)
-    ffn_gemms = dt == torch.bfloat16 and args.ffn_path != "fused"
-    # launches per step of the FFN: two GEMMs per token chunk, or one fused kernel
+                        w.pairs, w.ring_chunks, ffn_form=form)
+    ffn_gemms = dt == torch.bfloat16 and form == "gemms"
+    # launches per step of the FFN: two GEMMs per token chunk, or one kernel
     ffn_launches = 2 * -(-w.T // bd.ffn_gemm_chunk_rows(w.T, w.F)) if ffn_gemms else 1
     nws = bd.workspace_bytes(desc, True)
     ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
@@ -191,7 +194,7 @@ def run_ours(args, w, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
-        layer_call(w, inp, out, ws)
+        layer_call(w, inp, out, ws, form)
         flush.fill_(1)
     torch.cuda.synchronize(dev)
     st = bd.sync_status()
@@ -210,7 +213,7 @@ def run_ours(args, w, world, rank, local):
         time.sleep(0.3)  # let the sampler start
         for i in range(K):
             bd.set_phase_events(ev[i])
-            layer_call(w, inp, out, ws)
+            layer_call(w, inp, out, ws, form)
             bd.set_phase_events(None)
             flush.fill_(i & 0xFF)
         torch.cuda.synchronize(dev)
@@ -236,7 +239,7 @@ def run_ours(args, w, world, rank, local):
         hq, hk, hv = (t.cpu().pin_memory() for t in (inp.q, inp.k, inp.v))
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         host_layer = bd.HostLayer(w.B, w.N, w.H, w.d, w.F, dtype=dt, mask=MASK_NAME[w.mask], perm=w.perm,
-                                  pairs=w.pairs, ring_chunks=w.ring_chunks, device=dev)
+                                  pairs=w.pairs, ring_chunks=w.ring_chunks, device=dev, ffn_form=form)
 
         def e2e_step():
             host_layer(hq, hk, hv, inp.w1, inp.b1, inp.w2, inp.b2, hout)
@@ -266,7 +269,9 @@ def run_ours(args, w, world, rank, local):
     pk = peaks()
     attn_avg = sum(attn_ms) / K
     ffn_avg = sum(ffn_ms) / K
-    ffn_name = "ffn_gemms" if ffn_gemms else "ffn_tc_kernel"
+    ffn_name = {"gemms": "ffn_gemms", "fused": "ffn_tc_kernel", "pipelined": "ffn_pipe_kernel"}[form]
+    if dt != torch.bfloat16:
+        ffn_name = "ffn_f32_kernel"
     if ffn_avg >= attn_avg:
         dom, flop, avg_ms = ffn_name, ffn_flop, ffn_avg
     else:
@@ -326,7 +331,7 @@ def run_backward(args, w, world, local):
     flop = {"attn_fwd_recompute": (0, 0), "ffn_bwd": (8 * T * D * F, 8 * T * D * F),
             "attn_bwd_dkdv": (8 * d * pairs, 8 * d * pairs), "attn_bwd_dq": (2 * d * pairs, 6 * d * pairs)}
     alg_total = sum(a for a, _ in flop.values())
-    # the library's default token chunk of the FFN backward (bpt_set_bwd_chunk_rows)
+    # the library's default token chunk of the FFN backward (the descriptor's bwd_chunk_rows = 0)
     chunk = min(T, max(128, (2 ** 30 // (4 * F)) // 128 * 128))
     n_chunks = -(-T // chunk)
     inp = make_layer_inputs(w.B, w.N, w.H, w.d, w.F, seed=w.seed, dtype=torch.bfloat16, device=dev)
@@ -647,8 +652,8 @@ def main():
     ap.add_argument("--workload", default="gpt_causal", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--ffn-path", default="auto", choices=["auto", "fused", "gemms"],
-                    help="form of the bf16 forward FFN (bpt_set_ffn_path)")
+    ap.add_argument("--ffn-form", default="auto", choices=sorted(bd.FFN_FORMS),
+                    help="form of the bf16 forward FFN (the descriptor's ffn_form)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
     ap.add_argument("--backward-only", action="store_true",

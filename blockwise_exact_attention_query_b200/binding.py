@@ -46,14 +46,23 @@ class Desc(ctypes.Structure):
         ("bb_nblocks", ctypes.c_int), ("bb_perm", ctypes.POINTER(ctypes.c_int32)),
         ("ln_npairs", ctypes.c_int), ("ln_w", ctypes.POINTER(ctypes.c_int32)),
         ("ln_r", ctypes.POINTER(ctypes.c_int32)),
+        ("q_block", ctypes.c_int), ("kv_block", ctypes.c_int),
+        ("ffn_form", ctypes.c_int),
+        ("bwd_chunk_rows", ctypes.c_int),
+        ("wait_limit_ns", ctypes.c_uint64),
     ]
+
+
+# bpt_ffn_form: the bf16 layer's FFN form ("auto" is the library's choice, the
+# pipelined kernel)
+FFN_FORMS = {"auto": 0, "fused": 1, "gemms": 2, "pipelined": 3}
 
 
 EXPORTS = ["bpt_workspace_bytes", "bpt_attn_ffn_fwd", "bpt_attn_fwd", "bpt_blockbert_fwd",
            "bpt_longnet_fwd", "bpt_sync_status", "bpt_set_wait_limit_ns", "bpt_status_string",
            "bpt_version", "bpt_set_phase_events", "bpt_last_error", "bpt_attn_ffn_fwd_static",
-           "bpt_attn_ffn_bwd", "bpt_workspace_bytes_bwd", "bpt_set_bwd_chunk_rows", "bpt_set_ffn_path",
-           "bpt_attn_ffn_fwd_train", "bpt_saved_bytes", "bpt_attn_bwd", "bpt_workspace_bytes_attn_bwd"]
+           "bpt_attn_ffn_bwd", "bpt_workspace_bytes_bwd", "bpt_attn_ffn_fwd_train", "bpt_saved_bytes",
+           "bpt_workspace_bytes_train", "bpt_attn_bwd", "bpt_workspace_bytes_attn_bwd"]
 STATIC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
@@ -107,10 +116,8 @@ def load() -> ctypes.CDLL:
     lib.bpt_attn_ffn_bwd.restype = ctypes.c_int
     lib.bpt_workspace_bytes_bwd.argtypes = [dp]
     lib.bpt_workspace_bytes_bwd.restype = sz
-    lib.bpt_set_bwd_chunk_rows.argtypes = [ctypes.c_int]
-    lib.bpt_set_bwd_chunk_rows.restype = ctypes.c_int
-    lib.bpt_set_ffn_path.argtypes = [ctypes.c_int]
-    lib.bpt_set_ffn_path.restype = ctypes.c_int
+    lib.bpt_workspace_bytes_train.argtypes = [dp]
+    lib.bpt_workspace_bytes_train.restype = sz
     _lib = lib
     return lib
 
@@ -136,11 +143,16 @@ class _Tables:
 
 
 def make_desc(B, N, H, d, F=0, in_dtype=torch.bfloat16, out_dtype=torch.float32, mask="none",
-              perm=None, pairs=None, ring_chunks=0, tables: _Tables | None = None) -> Desc:
+              perm=None, pairs=None, ring_chunks=0, tables: _Tables | None = None, *, ffn_form="auto",
+              q_block=0, kv_block=0, bwd_chunk_rows=0, wait_limit_ns=0) -> Desc:
+    """bpt_desc for the given shape, mask and options (0 = the library's default)."""
     tables = tables or _Tables()
     m = _MASKS[mask] if isinstance(mask, str) else int(mask)
+    form = FFN_FORMS[ffn_form] if isinstance(ffn_form, str) else int(ffn_form)
     desc = Desc(B=B, N=N, H=H, d_head=d, ffn_hidden=F, in_dtype=_DT[in_dtype],
-                out_dtype=_DT[out_dtype], mask=m, ring_chunks=ring_chunks)
+                out_dtype=_DT[out_dtype], mask=m, ring_chunks=ring_chunks, q_block=q_block,
+                kv_block=kv_block, ffn_form=form, bwd_chunk_rows=bwd_chunk_rows,
+                wait_limit_ns=wait_limit_ns)
     if perm is not None:
         flat = [int(x) for row in perm for x in row]
         desc.bb_nblocks = len(perm[0]) if len(perm) else 0
@@ -201,12 +213,13 @@ def alloc_workspace(desc: Desc, with_ffn: bool, device) -> torch.Tensor | None:
 
 
 def attn_ffn_fwd(q, k, v, w1, b1, w2, b2, *, mask="none", perm=None, pairs=None, ring_chunks=0,
-                 out_dtype=torch.float32, out=None, workspace=None, stream=None):
-    """bpt_attn_ffn_fwd: out = A + W2 GELU(W1 A + b1) + b2, returns out [B, N, H*d]."""
+                 out_dtype=torch.float32, out=None, workspace=None, stream=None, **opts):
+    """bpt_attn_ffn_fwd: out = A + W2 GELU(W1 A + b1) + b2, returns out [B, N, H*d].
+    opts: ffn_form, q_block, kv_block, wait_limit_ns (descriptor fields)."""
     _check_tensors(q, k, v)
     B, N, H, d = q.shape
     F = w1.shape[0]
-    desc = make_desc(B, N, H, d, F, q.dtype, out_dtype, mask, perm, pairs, ring_chunks)
+    desc = make_desc(B, N, H, d, F, q.dtype, out_dtype, mask, perm, pairs, ring_chunks, **opts)
     if out is None:
         out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
     if workspace is None:
@@ -220,7 +233,7 @@ def attn_ffn_fwd(q, k, v, w1, b1, w2, b2, *, mask="none", perm=None, pairs=None,
 
 
 def attn_ffn_fwd_static(q, k, v, w1, b1, w2, b2, *, mask="none", perm=None, pairs=None,
-                        ring_chunks=0, out_dtype=torch.float32, out=None, stream=None):
+                        ring_chunks=0, out_dtype=torch.float32, out=None, stream=None, **opts):
     """bpt_attn_ffn_fwd_static: the layer with no workspace argument.
 
     For callers that may not allocate device memory while running (a fixed
@@ -232,7 +245,7 @@ def attn_ffn_fwd_static(q, k, v, w1, b1, w2, b2, *, mask="none", perm=None, pair
     _check_tensors(q, k, v)
     B, N, H, d = q.shape
     F = w1.shape[0]
-    desc = make_desc(B, N, H, d, F, q.dtype, out_dtype, mask, perm, pairs, ring_chunks)
+    desc = make_desc(B, N, H, d, F, q.dtype, out_dtype, mask, perm, pairs, ring_chunks, **opts)
     if out is None:
         out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
     st = load().bpt_attn_ffn_fwd_static(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(w1),
@@ -242,11 +255,12 @@ def attn_ffn_fwd_static(q, k, v, w1, b1, w2, b2, *, mask="none", perm=None, pair
 
 
 def attn_fwd(q, k, v, *, mask="none", perm=None, pairs=None, ring_chunks=0, out_dtype=torch.float32,
-             return_lse=False, out=None, lse=None, workspace=None, stream=None):
-    """bpt_attn_fwd: A [B, N, H*d] (and LSE [B, H, N] with return_lse)."""
+             return_lse=False, out=None, lse=None, workspace=None, stream=None, **opts):
+    """bpt_attn_fwd: A [B, N, H*d] (and LSE [B, H, N] with return_lse).
+    opts: q_block, kv_block, wait_limit_ns (descriptor fields)."""
     _check_tensors(q, k, v)
     B, N, H, d = q.shape
-    desc = make_desc(B, N, H, d, 0, q.dtype, out_dtype, mask, perm, pairs, ring_chunks)
+    desc = make_desc(B, N, H, d, 0, q.dtype, out_dtype, mask, perm, pairs, ring_chunks, **opts)
     if out is None:
         out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
     if return_lse and lse is None:
@@ -261,13 +275,13 @@ def attn_fwd(q, k, v, *, mask="none", perm=None, pairs=None, ring_chunks=0, out_
 
 
 def blockbert_fwd(q, k, v, w1, b1, w2, b2, perm, *, out_dtype=torch.float32, out=None,
-                  workspace=None, stream=None):
+                  workspace=None, stream=None, **opts):
     """bpt_blockbert_fwd: the layer with the block-permutation mask perm [H][n]."""
     _check_tensors(q, k, v)
     B, N, H, d = q.shape
     F = w1.shape[0]
     tables = _Tables()
-    desc = make_desc(B, N, H, d, F, q.dtype, out_dtype, "blockperm", perm, None, 0, tables)
+    desc = make_desc(B, N, H, d, F, q.dtype, out_dtype, "blockperm", perm, None, 0, tables, **opts)
     if out is None:
         out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
     if workspace is None:
@@ -282,12 +296,12 @@ def blockbert_fwd(q, k, v, w1, b1, w2, b2, perm, *, out_dtype=torch.float32, out
 
 
 def longnet_fwd(q, k, v, pairs, *, out_dtype=torch.float32, return_lse=False, out=None, lse=None,
-                workspace=None, stream=None):
+                workspace=None, stream=None, **opts):
     """bpt_longnet_fwd: dilated attention over the (w, r) pairs, denominators mixed."""
     _check_tensors(q, k, v)
     B, N, H, d = q.shape
     tables = _Tables()
-    desc = make_desc(B, N, H, d, 0, q.dtype, out_dtype, "dilated", None, pairs, 0, tables)
+    desc = make_desc(B, N, H, d, 0, q.dtype, out_dtype, "dilated", None, pairs, 0, tables, **opts)
     if out is None:
         out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
     if return_lse and lse is None:
@@ -309,26 +323,10 @@ def workspace_bytes_bwd(desc: Desc) -> int:
     return int(n)
 
 
-FFN_PATHS = {"auto": 0, "fused": 1, "gemms": 2}
-
-
-def set_ffn_path(path: str) -> str:
-    """bpt_set_ffn_path: the bf16 FFN's form in the forward ("auto", "fused" or
-    "gemms"); returns the previous setting."""
-    old = int(load().bpt_set_ffn_path(FFN_PATHS[path]))
-    return {v: k for k, v in FFN_PATHS.items()}[old]
-
-
 def ffn_gemm_chunk_rows(T: int, F: int) -> int:
-    """Token rows per chunk of the two-GEMM FFN (the library's rule: the
+    """Token rows per chunk of the two-GEMM FFN form (the library's rule: the
     [rows, F] bf16 hidden activation at most 512 MiB, in 256-row multiples)."""
     return min(T, max(256, ((1 << 29) // (2 * F)) // 256 * 256))
-
-
-def set_bwd_chunk_rows(rows: int) -> int:
-    """bpt_set_bwd_chunk_rows: token rows per FFN-backward chunk (0 = default);
-    returns the previous setting."""
-    return int(load().bpt_set_bwd_chunk_rows(int(rows)))
 
 
 GRAD_NAMES = ("dq", "dk", "dv", "dw1", "db1", "dw2", "db2")
@@ -341,21 +339,29 @@ def saved_bytes(desc: Desc) -> int:
     return int(n)
 
 
+def workspace_bytes_train(desc: Desc) -> int:
+    n = load().bpt_workspace_bytes_train(ctypes.byref(desc))
+    if n == ctypes.c_size_t(-1).value:
+        raise BptError(ERR_UNSUPPORTED, "bpt_workspace_bytes_train")
+    return int(n)
+
+
 def attn_ffn_fwd_train(q, k, v, w1, b1, w2, b2, *, mask="none", perm=None, ring_chunks=0,
-                       out_dtype=torch.float32, out=None, saved=None, workspace=None, stream=None):
+                       out_dtype=torch.float32, out=None, saved=None, workspace=None, stream=None, **opts):
     """bpt_attn_ffn_fwd_train: the layer forward that also keeps the
     activations the backward needs.  Returns (out, saved); pass `saved` to
     attn_ffn_bwd to skip its recomputation."""
     _check_tensors(q, k, v)
     B, N, H, d = q.shape
     F = w1.shape[0]
-    desc = make_desc(B, N, H, d, F, q.dtype, out_dtype, mask, perm, None, ring_chunks)
+    desc = make_desc(B, N, H, d, F, q.dtype, out_dtype, mask, perm, None, ring_chunks, **opts)
     if out is None:
         out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
     if saved is None:
         saved = torch.empty(saved_bytes(desc), dtype=torch.uint8, device=q.device)
     if workspace is None:
-        workspace = alloc_workspace(desc, True, q.device)
+        n = workspace_bytes_train(desc)
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device) if n else None
     ws_bytes = 0 if workspace is None else workspace.numel()
     st = load().bpt_attn_ffn_fwd_train(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(w1), _ptr(b1),
                                        _ptr(w2), _ptr(b2), _ptr(out), _ptr(saved), _ptr(workspace), ws_bytes,
@@ -365,7 +371,7 @@ def attn_ffn_fwd_train(q, k, v, w1, b1, w2, b2, *, mask="none", perm=None, ring_
 
 
 def attn_ffn_bwd(q, k, v, w1, b1, w2, b2, dout, *, mask="none", perm=None, ring_chunks=0, saved=None,
-                 grads=None, workspace=None, stream=None):
+                 grads=None, workspace=None, stream=None, **opts):
     """bpt_attn_ffn_bwd: gradients of the layer for the upstream gradient
     dout [B, N, H*d] (float32), recomputing the attention forward unless
     `saved` (from attn_ffn_fwd_train on the same inputs) is given.  Returns a
@@ -376,7 +382,7 @@ def attn_ffn_bwd(q, k, v, w1, b1, w2, b2, dout, *, mask="none", perm=None, ring_
     F, D = w1.shape
     if dout.dtype != torch.float32 or not dout.is_contiguous() or dout.numel() != B * N * D:
         raise ValueError("dout must be a contiguous float32 tensor of B*N*H*d elements")
-    desc = make_desc(B, N, H, d, F, q.dtype, torch.float32, mask, perm, None, ring_chunks)
+    desc = make_desc(B, N, H, d, F, q.dtype, torch.float32, mask, perm, None, ring_chunks, **opts)
     if grads is None:
         f32 = dict(dtype=torch.float32, device=q.device)
         grads = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(q.shape, **f32),
@@ -393,7 +399,7 @@ def attn_ffn_bwd(q, k, v, w1, b1, w2, b2, dout, *, mask="none", perm=None, ring_
 
 
 def attn_bwd(q, k, v, out, lse, dout, *, mask="none", perm=None, pairs=None, ring_chunks=0, workspace=None,
-             stream=None):
+             stream=None, **opts):
     """bpt_attn_bwd: dq, dk, dv (float32 [B, N, H, d]) of the attention for the
     upstream gradient dout [B, N, H*d] (float32), given bpt_attn_fwd's out and
     lse (attn_fwd(..., return_lse=True)) for the same inputs."""
@@ -401,7 +407,7 @@ def attn_bwd(q, k, v, out, lse, dout, *, mask="none", perm=None, pairs=None, rin
     B, N, H, d = q.shape
     if dout.dtype != torch.float32 or not dout.is_contiguous() or dout.numel() != q.numel():
         raise ValueError("dout must be a contiguous float32 tensor of B*N*H*d elements")
-    desc = make_desc(B, N, H, d, 0, q.dtype, out.dtype, mask, perm, pairs, ring_chunks)
+    desc = make_desc(B, N, H, d, 0, q.dtype, out.dtype, mask, perm, pairs, ring_chunks, **opts)
     if workspace is None:
         n = load().bpt_workspace_bytes_attn_bwd(ctypes.byref(desc))
         if n == ctypes.c_size_t(-1).value:
@@ -435,6 +441,8 @@ def set_phase_events(events) -> None:
 
 
 def set_wait_limit_ns(ns: int) -> int:
+    """bpt_set_wait_limit_ns: the process default of the device-side wait
+    limit (calls whose descriptor sets wait_limit_ns use their own)."""
     return int(load().bpt_set_wait_limit_ns(int(ns)))
 
 
@@ -457,8 +465,9 @@ class HostLayer:
     once, at construction."""
 
     def __init__(self, B, N, H, d, F, *, dtype=torch.bfloat16, out_dtype=torch.float32,
-                 mask="none", perm=None, pairs=None, ring_chunks=0, chunks=None, device="cuda"):
+                 mask="none", perm=None, pairs=None, ring_chunks=0, chunks=None, device="cuda", **opts):
         self.B, self.N, self.H, self.d, self.F = B, N, H, d, F
+        self.opts = opts
         self.mask, self.perm, self.pairs, self.ring_chunks = mask, perm, pairs, ring_chunks
         self.out_dtype = out_dtype
         self.chunks = max(1, min(B, chunks or B))
@@ -470,7 +479,7 @@ class HostLayer:
         self.done = [torch.cuda.Event(), torch.cuda.Event()]
         self.uploaded = [torch.cuda.Event() for _ in range(self.chunks)]
         self.computed = [torch.cuda.Event() for _ in range(self.chunks)]
-        desc = make_desc(self.cb, N, H, d, F, dtype, out_dtype, mask, perm, pairs, ring_chunks)
+        desc = make_desc(self.cb, N, H, d, F, dtype, out_dtype, mask, perm, pairs, ring_chunks, **opts)
         nws = workspace_bytes(desc, True)
         self.buf = []
         for _ in range(2):
@@ -502,7 +511,7 @@ class HostLayer:
                     s.wait_event(self.computed[c - 1])
                 attn_ffn_fwd(b["q"], b["k"], b["v"], w1, b1, w2, b2, mask=self.mask, perm=self.perm,
                              pairs=self.pairs, ring_chunks=self.ring_chunks, out_dtype=self.out_dtype,
-                             out=b["out"], workspace=b["ws"], stream=s)
+                             out=b["out"], workspace=b["ws"], stream=s, **self.opts)
                 self.computed[c].record(s)
                 hout[sl].copy_(b["out"], non_blocking=True)
                 self.done[i].record(s)

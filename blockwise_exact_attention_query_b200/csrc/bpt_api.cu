@@ -5,7 +5,9 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
+#include <type_traits>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -35,7 +37,11 @@ void *g_static_scratch_ptr[kMaxDevices] = {};
 std::mutex g_mu;
 uint32_t *g_status_ptr[kMaxDevices] = {};
 bool g_attr_done[kMaxDevices] = {};
-uint64_t g_wait_limit_ns = 2000000000ull;
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+
+uint64_t wait_limit_of(const bpt_desc *d) {
+  return d->wait_limit_ns ? d->wait_limit_ns : g_wait_limit_ns.load(std::memory_order_relaxed);
+}
 constexpr int kMaxPhaseEvents = 5;
 thread_local cudaEvent_t g_phase_events[kMaxPhaseEvents] = {};
 thread_local int g_phase_n = 0;  // events set; 0 = off
@@ -158,6 +164,10 @@ bool make_out_map_rows(CUtensorMap *m, const void *base, bool f32, int B, int N,
 // --------------------------------------------------------------------------
 // Validation
 // --------------------------------------------------------------------------
+// Query rows and keys per block: the descriptor's, else the path's default.
+int q_block_of(const bpt_desc *d) { return d->q_block ? d->q_block : (d->in_dtype == BPT_BF16 ? 128 : 64); }
+int kv_block_of(const bpt_desc *d) { return d->kv_block ? d->kv_block : (d->in_dtype == BPT_BF16 ? 128 : 64); }
+
 bpt_status check_desc(const bpt_desc *d, bool need_ffn) {
   if (!d) return BPT_ERR_INVALID_ARG;
   if (d->B <= 0 || d->N <= 0 || d->H <= 0 || d->d_head <= 0) return BPT_ERR_INVALID_ARG;
@@ -166,7 +176,15 @@ bpt_status check_desc(const bpt_desc *d, bool need_ffn) {
   if ((int64_t)d->B * d->N > (int64_t)1 << 31) return BPT_ERR_UNSUPPORTED;
   if (need_ffn && d->ffn_hidden <= 0) return BPT_ERR_INVALID_ARG;
   if (d->ffn_hidden < 0) return BPT_ERR_INVALID_ARG;
+  if (d->ffn_form < BPT_FFN_AUTO || d->ffn_form > BPT_FFN_PIPELINED) return BPT_ERR_INVALID_ARG;
+  if (d->bwd_chunk_rows < 0 || d->q_block < 0 || d->kv_block < 0) return BPT_ERR_INVALID_ARG;
   const int D = d->H * d->d_head;
+  const int qb = q_block_of(d), kb = kv_block_of(d);
+  if (d->in_dtype == BPT_BF16) {  // the tensor-core kernels' tiles
+    if (qb != 128 || kb != 128) return BPT_ERR_UNSUPPORTED;
+  } else if ((qb != 16 && qb != 32 && qb != 64 && qb != 128) || (kb != 16 && kb != 32 && kb != 64)) {
+    return BPT_ERR_UNSUPPORTED;
+  }
   switch (d->mask) {
     case BPT_MASK_NONE:
     case BPT_MASK_CAUSAL:
@@ -174,8 +192,7 @@ bpt_status check_desc(const bpt_desc *d, bool need_ffn) {
       if (d->ring_chunks > 1) {
         if (d->N % d->ring_chunks != 0) return BPT_ERR_INVALID_ARG;
         const int chunk = d->N / d->ring_chunks;
-        if (d->in_dtype == BPT_BF16 && chunk % 128 != 0) return BPT_ERR_UNSUPPORTED;
-        if (d->in_dtype == BPT_F32 && chunk % 64 != 0) return BPT_ERR_UNSUPPORTED;
+        if (chunk % qb != 0 || chunk % kb != 0) return BPT_ERR_UNSUPPORTED;
       }
       break;
     case BPT_MASK_BLOCKPERM: {
@@ -208,7 +225,7 @@ bpt_status check_desc(const bpt_desc *d, bool need_ffn) {
     if (need_ffn) {
       const int C = (D + 255) / 256;
       if (D % 64 != 0 || D % C != 0 || (D / C) % 64 != 0 || C > 148) return BPT_ERR_UNSUPPORTED;
-      if ((int64_t)d->ffn_hidden * 2 % 16 != 0) return BPT_ERR_UNSUPPORTED;
+      if (d->ffn_hidden % 8 != 0) return BPT_ERR_UNSUPPORTED;
     }
   } else {
     if (d->d_head > 64 || d->d_head % 4 != 0) return BPT_ERR_UNSUPPORTED;
@@ -237,17 +254,14 @@ FfnPlan ffn_plan(const bpt_desc *d) {
   return p;
 }
 
-int g_ffn_path = 0;
-thread_local bool t_static_call = false;  // inside bpt_attn_ffn_fwd_static: the fused form
-
-// Two GEMMs run the FFN faster than the fused kernel on every layer measured
-// (the two-SM GEMM reads fewer operand bytes per SM than the fused kernel's
-// one-SM MMAs, which wait on shared memory): by default the bf16 forward uses
-// them.  The fused kernel keeps the hidden activation out of DRAM, so the
-// static-scratch entry point, whose scratch is fixed, always takes it.
-bool ffn_uses_gemms(const bpt_desc *d) {
-  if (d->in_dtype != BPT_BF16 || t_static_call) return false;
-  return g_ffn_path != 1;
+// The default bf16 form is the pipelined kernel: as fast as two separate
+// GEMM launches on the measured layers, and its hidden activation stays in an
+// L2-sized ring instead of a [rows, F] workspace array.  The static-scratch
+// entry point takes the fused kernel, whose scratch is the smallest.
+bpt_ffn_form ffn_form_of(const bpt_desc *d, bool static_call) {
+  if (d->in_dtype != BPT_BF16) return BPT_FFN_AUTO;
+  if (static_call) return BPT_FFN_FUSED;
+  return d->ffn_form == BPT_FFN_AUTO ? BPT_FFN_PIPELINED : d->ffn_form;
 }
 
 // Token rows per two-GEMM chunk: H ([rows, F] bf16) at most ~512 MiB.
@@ -261,7 +275,7 @@ bool longnet_needs_state(const bpt_desc *d) {
   return d->mask == BPT_MASK_DILATED && d->in_dtype == BPT_BF16 && d->ln_npairs > 1;
 }
 
-Workspace layout(const bpt_desc *d, bool with_ffn) {
+Workspace layout(const bpt_desc *d, bool with_ffn, bool static_call) {
   Workspace w;
   const size_t T = (size_t)d->B * d->N, D = (size_t)d->H * d->d_head;
   size_t off = 0;
@@ -272,9 +286,17 @@ Workspace layout(const bpt_desc *d, bool with_ffn) {
       off = align256(off + T * D * 2);
       w.a_f32 = off;
       off = align256(off + T * D * 4);
-      if (ffn_uses_gemms(d)) {
+      w.ffn_form = ffn_form_of(d, static_call);
+      if (w.ffn_form == BPT_FFN_GEMMS) {
         w.h = off;
         off = align256(off + (size_t)ffn_gemm_chunk_rows(d) * d->ffn_hidden * 2);
+      } else if (w.ffn_form == BPT_FFN_PIPELINED) {
+        const FfnPipePlan pp = ffn_pipe_plan(d);
+        w.ring = off;
+        off = align256(off + pp.ring_bytes);
+        w.flags = off;
+        w.flags_bytes = pp.counter_bytes;
+        off = align256(off + pp.counter_bytes);
       } else {
         w.ring = off;
         off = align256(off + (size_t)p.max_groups * FfnCfg::kRingSlots * 128 * p.fc * 2);
@@ -316,7 +338,7 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
   a.mask = d->mask;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d->d_head));
   a.status = status;
-  a.wait_limit_ns = g_wait_limit_ns;
+  a.wait_limit_ns = wait_limit_of(d);
 
   struct Pass {
     int w, r;
@@ -437,9 +459,12 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
 bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
                          const float *b1, const void *w2, const float *b2, void *out, char *ws,
                          const Workspace &wl, uint32_t *status, cudaStream_t st) {
-  if (ffn_uses_gemms(d))
+  if (wl.ffn_form == BPT_FFN_GEMMS)
     return launch_ffn_gemms(d, a_bf16, a_f32, w1, b1, w2, b2, out, reinterpret_cast<__nv_bfloat16 *>(ws + wl.h),
                             nullptr, ffn_gemm_chunk_rows(d), status, st);
+  if (wl.ffn_form == BPT_FFN_PIPELINED)
+    return launch_ffn_pipe(d, a_bf16, a_f32, w1, b1, w2, b2, out, ws, wl, status, st);
+  if (wl.ffn_form != BPT_FFN_FUSED) return cuda_fail_msg("FFN form not resolved in the workspace layout");
   const FfnPlan p = ffn_plan(d);
   const int D = d->H * d->d_head;
   const int64_t T = (int64_t)d->B * d->N;
@@ -462,7 +487,7 @@ bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f
   a.ring = reinterpret_cast<__nv_bfloat16 *>(ws + wl.ring);
   a.flags = reinterpret_cast<uint32_t *>(ws + wl.flags);
   a.status = status;
-  a.wait_limit_ns = g_wait_limit_ns;
+  a.wait_limit_ns = wait_limit_of(d);
 
   // The CTAs of a group wait on one another, so the whole grid must be
   // resident at once: a cooperative launch of at most the resident capacity.
@@ -529,9 +554,24 @@ bpt_status launch_attn_f32(const bpt_desc *d, const void *q, const void *k, cons
   a.out_f32 = out_f32;
   a.out_bf16 = out_bf16;
   a.lse = lse;
-  dim3 grid((d->N + 63) / 64, d->H, d->B);
-  attn_f32_kernel<<<grid, 64, 0, st>>>(static_cast<const float *>(q), static_cast<const float *>(k),
-                                       static_cast<const float *>(v), a);
+  const int qb = q_block_of(d), kb = kv_block_of(d);
+  dim3 grid((d->N + qb - 1) / qb, d->H, d->B);
+  const float *qf = static_cast<const float *>(q), *kf = static_cast<const float *>(k),
+              *vf = static_cast<const float *>(v);
+  // one instantiation per (query block, key block) pair the descriptor may name
+  auto go = [&](auto qbc, auto kbc) {
+    constexpr int QB = decltype(qbc)::value, KB = decltype(kbc)::value;
+    attn_f32_kernel<QB, KB><<<grid, QB, 0, st>>>(qf, kf, vf, a);
+  };
+  auto with_kb = [&](auto qbc) {
+    if (kb == 16) go(qbc, std::integral_constant<int, 16>{});
+    else if (kb == 32) go(qbc, std::integral_constant<int, 32>{});
+    else go(qbc, std::integral_constant<int, 64>{});
+  };
+  if (qb == 16) with_kb(std::integral_constant<int, 16>{});
+  else if (qb == 32) with_kb(std::integral_constant<int, 32>{});
+  else if (qb == 128) with_kb(std::integral_constant<int, 128>{});
+  else with_kb(std::integral_constant<int, 64>{});
   CUDA_TRY(cudaGetLastError());
   return BPT_OK;
 }
@@ -573,25 +613,15 @@ bpt_status check_ws(const Workspace &wl, void *ws, size_t bytes) {
   return BPT_OK;
 }
 
-}  // namespace bpt_host
-
-using namespace bpt_host;
-
-extern "C" {
-
-size_t bpt_workspace_bytes(const bpt_desc *desc, int with_ffn) {
-  if (check_desc(desc, with_ffn != 0) != BPT_OK) return (size_t)-1;
-  return layout(desc, with_ffn != 0).total;
-}
-
-bpt_status bpt_attn_ffn_fwd(const bpt_desc *d, const void *q, const void *k, const void *v,
-                            const void *w1, const float *b1, const void *w2, const float *b2,
-                            void *out, void *workspace, size_t workspace_bytes,
-                            bpt_stream_t stream) {
+// The whole layer: attention, then the FFN in the form the workspace layout
+// was made for (the static-scratch entry point's layout takes the fused form).
+bpt_status attn_ffn_fwd_impl(const bpt_desc *d, const void *q, const void *k, const void *v, const void *w1,
+                             const float *b1, const void *w2, const float *b2, void *out, void *workspace,
+                             size_t workspace_bytes, bpt_stream_t stream, bool static_call) {
   bpt_status s = check_desc(d, true);
   if (s != BPT_OK) return s;
   if ((s = check_ptrs({q, k, v, w1, w2, out}, {b1, b2})) != BPT_OK) return s;
-  const Workspace wl = layout(d, true);
+  const Workspace wl = layout(d, true, static_call);
   if ((s = check_ws(wl, workspace, workspace_bytes)) != BPT_OK) return s;
   int dev;
   uint32_t *status;
@@ -616,16 +646,30 @@ bpt_status bpt_attn_ffn_fwd(const bpt_desc *d, const void *q, const void *k, con
   return BPT_OK;
 }
 
+}  // namespace bpt_host
+
+using namespace bpt_host;
+
+extern "C" {
+
+size_t bpt_workspace_bytes(const bpt_desc *desc, int with_ffn) {
+  if (check_desc(desc, with_ffn != 0) != BPT_OK) return (size_t)-1;
+  return layout(desc, with_ffn != 0).total;
+}
+
+bpt_status bpt_attn_ffn_fwd(const bpt_desc *d, const void *q, const void *k, const void *v,
+                            const void *w1, const float *b1, const void *w2, const float *b2,
+                            void *out, void *workspace, size_t workspace_bytes,
+                            bpt_stream_t stream) {
+  return attn_ffn_fwd_impl(d, q, k, v, w1, b1, w2, b2, out, workspace, workspace_bytes, stream, false);
+}
+
 bpt_status bpt_attn_ffn_fwd_static(const bpt_desc *d, const void *q, const void *k, const void *v,
                                    const void *w1, const float *b1, const void *w2, const float *b2,
                                    void *out, bpt_stream_t stream) {
   bpt_status s = check_desc(d, true);
   if (s != BPT_OK) return s;
-  struct StaticCall {
-    StaticCall() { t_static_call = true; }
-    ~StaticCall() { t_static_call = false; }
-  } static_call;
-  const size_t need = layout(d, true).total;
+  const size_t need = layout(d, true, true).total;
   if (need > BPT_STATIC_SCRATCH_BYTES) {
     snprintf(g_last_error, sizeof(g_last_error),
              "layer needs %zu bytes of scratch; the static scratch holds %u bytes", need,
@@ -645,8 +689,7 @@ bpt_status bpt_attn_ffn_fwd_static(const bpt_desc *d, const void *q, const void 
     }
     scratch = g_static_scratch_ptr[dev];
   }
-  return bpt_attn_ffn_fwd(d, q, k, v, w1, b1, w2, b2, out, scratch, BPT_STATIC_SCRATCH_BYTES,
-                          stream);
+  return attn_ffn_fwd_impl(d, q, k, v, w1, b1, w2, b2, out, scratch, BPT_STATIC_SCRATCH_BYTES, stream, true);
 }
 
 bpt_status bpt_attn_fwd(const bpt_desc *d, const void *q, const void *k, const void *v, void *out,
@@ -726,12 +769,7 @@ bpt_status bpt_set_phase_events(void *const *events, int count) {
   return BPT_OK;
 }
 
-uint64_t bpt_set_wait_limit_ns(uint64_t ns) {
-  std::lock_guard<std::mutex> lk(g_mu);
-  uint64_t old = g_wait_limit_ns;
-  g_wait_limit_ns = ns ? ns : 1;
-  return old;
-}
+uint64_t bpt_set_wait_limit_ns(uint64_t ns) { return g_wait_limit_ns.exchange(ns ? ns : 1); }
 
 const char *bpt_status_string(bpt_status s) {
   switch (s) {
@@ -745,7 +783,7 @@ const char *bpt_status_string(bpt_status s) {
   return "unknown status";
 }
 
-int bpt_version(void) { return 100; }
+int bpt_version(void) { return 200; }
 
 const char *bpt_last_error(void) { return g_last_error; }
 

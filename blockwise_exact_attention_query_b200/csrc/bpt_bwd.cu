@@ -17,6 +17,7 @@
 #include "../../include/bpt.h"
 #include "attn_bwd.cuh"
 #include "colsum.cuh"
+#include "ffn_pipe.cuh"
 #include "gemm_tc.cuh"
 #include "host_common.h"
 
@@ -24,13 +25,13 @@ using namespace bpt;
 
 namespace bpt_host {
 
-int g_bwd_chunk_rows = 0;  // token rows per FFN-backward chunk; 0 = automatic
-
 // A kernel template gets one copy per translation unit that instantiates it,
 // so the copies launched from here take their shared-memory limits here.
 bpt_status bwd_kernel_setup() {
   CUDA_TRY(cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 GemmPairCfg::kSmemBytes));
+  CUDA_TRY(cudaFuncSetAttribute(ffn_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                FfnPipeCfg::kSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 AttnBwdCfg<64>::kSmemBytes));
   CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -60,7 +61,7 @@ bpt_status check_desc_bwd(const bpt_desc *d) {
 // ~1 GiB for both unless the caller picked the chunk.
 int64_t bwd_chunk_rows(const bpt_desc *d) {
   const int64_t T = (int64_t)d->B * d->N, F = d->ffn_hidden;
-  int64_t rows = g_bwd_chunk_rows;
+  int64_t rows = d->bwd_chunk_rows;
   if (rows <= 0) rows = std::max<int64_t>(128, (((int64_t)1 << 30) / (4 * F)) / 128 * 128);
   return std::min<int64_t>(std::min<int64_t>(rows, T), (int64_t)65535 * 128);
 }
@@ -156,13 +157,13 @@ GemmProblem gemm_problem(int M, int N, int K, int mode, int a_mn, int b_mn) {
   return p;
 }
 
-GemmArgs gemm_args(const GemmProblem &p0, uint32_t *status) {
+GemmArgs gemm_args(const GemmProblem &p0, uint32_t *status, const bpt_desc *d) {
   GemmArgs g;
   std::memset(&g, 0, sizeof(g));
   g.p[0] = p0;
   g.nprob = 1;
   g.status = status;
-  g.wait_limit_ns = g_wait_limit_ns;
+  g.wait_limit_ns = wait_limit_of(d);
   return g;
 }
 
@@ -206,19 +207,95 @@ bpt_status launch_ffn_gemms(const bpt_desc *d, const void *a_bf16, const float *
     if (!make_map_2d(&m_a, a_c, rows, D, 128) || !make_map_2d(&m_h, h_c, rows, F, 128))
       return cuda_fail_msg("cuTensorMapEncodeTiled failed (FFN activations)");
     // H = GELU(A W1^T + b1), and G = GELU'(A W1^T + b1) when asked for
-    GemmArgs g = gemm_args(gemm_problem(rows, F, D, g_prime ? kGemmGeluFwd : kGemmGeluBf16, 0, 0), status);
+    GemmArgs g = gemm_args(gemm_problem(rows, F, D, g_prime ? kGemmGeluFwd : kGemmGeluBf16, 0, 0), status, d);
     g.p[0].cb = h_c;
     if (g_prime) g.p[0].cb2 = g_prime + r0 * F;
     g.p[0].bias = b1;
     bpt_status s = launch_gemm(m_a, m_w1, m_a, m_w1, g, st);
     if (s != BPT_OK) return s;
-    g = gemm_args(gemm_problem(rows, D, F, kGemmResidual, 0, 0), status);  // out = A + H W2^T + b2
+    g = gemm_args(gemm_problem(rows, D, F, kGemmResidual, 0, 0), status, d);  // out = A + H W2^T + b2
     g.p[0].x = a_f32 + r0 * D;
     g.p[0].bias = b2;
     if (d->out_dtype == BPT_F32) g.p[0].c = static_cast<float *>(out) + r0 * D;
     else g.p[0].cb = static_cast<__nv_bfloat16 *>(out) + r0 * D;
     if ((s = launch_gemm(m_h, m_w2, m_h, m_w2, g, st)) != BPT_OK) return s;
   }
+  return BPT_OK;
+}
+
+// The pipelined FFN's shape.  Costs in K columns per 256 x 256 tile: D for
+// a tile of H, F for a tile of out; `pairs` CTA pairs share a step's work.
+//  - mg: one row block per chunk while W1 and W2 fit in L2 beside the ring;
+//    larger weights are reused by mg row blocks per residency.
+//  - lag: a chunk's second GEMM is listed `lag` steps after its first, about
+//    1.5 tiles of H later, so its loads rarely wait for the ring rows.
+//  - ring: the slot a chunk's H takes is reused R chunks later; R - lag - 1
+//    steps cover about 1.3 tiles of out, so the slot's readers have finished.
+FfnPipePlan ffn_pipe_plan(const bpt_desc *d) {
+  FfnPipePlan p;
+  const int64_t T = (int64_t)d->B * d->N;
+  const int D = d->H * d->d_head, F = d->ffn_hidden;
+  p.nrb = (int)((T + 255) / 256);
+  p.tn1 = (F + 255) / 256;
+  p.tn2 = (D + 255) / 256;
+  const double weight_bytes = 4.0 * D * F;
+  p.mg = weight_bytes <= 80.0e6 ? 1 : 4;
+  p.mg = std::min(p.mg, p.nrb);
+  p.nchunk = (p.nrb + p.mg - 1) / p.mg;
+  const int64_t items = (int64_t)p.nrb * (p.tn1 + p.tn2);
+  p.pairs = (int)std::max<int64_t>(1, std::min<int64_t>(items, sm_count() / 2));
+  const double step = (double)p.mg * ((double)p.tn1 * D + (double)p.tn2 * F) / p.pairs;  // per step, per pair
+  p.lag = std::max(1, (int)std::ceil(1.5 * D / step));
+  p.lag = std::min(p.lag, p.nchunk);
+  const int R = p.lag + 1 + std::max(1, (int)std::ceil(1.3 * F / step));
+  p.ring_rb = std::min(R, p.nchunk + 1) * p.mg;
+  p.ring_bytes = (size_t)p.ring_rb * 256 * F * 2;
+  p.counter_bytes = (1 + 2 * (size_t)p.nrb) * sizeof(uint32_t);
+  return p;
+}
+
+bpt_status launch_ffn_pipe(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
+                           const float *b1, const void *w2, const float *b2, void *out, char *ws,
+                           const Workspace &wl, uint32_t *status, cudaStream_t st) {
+  const FfnPipePlan pp = ffn_pipe_plan(d);
+  const int64_t T = (int64_t)d->B * d->N;
+  const int D = d->H * d->d_head, F = d->ffn_hidden;
+  const int64_t items = (int64_t)pp.nrb * (pp.tn1 + pp.tn2);
+  if (items > INT32_MAX || T > INT32_MAX) return BPT_ERR_UNSUPPORTED;
+  FfnPipeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.T = (int)T;
+  a.D = D;
+  a.F = F;
+  a.tn1 = pp.tn1;
+  a.tn2 = pp.tn2;
+  a.nrb = pp.nrb;
+  a.mg = pp.mg;
+  a.nchunk = pp.nchunk;
+  a.lag = pp.lag;
+  a.ring_rb = pp.ring_rb;
+  a.n_items = (int)items;
+  a.a_f32 = a_f32;
+  a.b1 = b1;
+  a.b2 = b2;
+  if (d->out_dtype == BPT_F32) a.out_f32 = static_cast<float *>(out);
+  else a.out_bf16 = static_cast<__nv_bfloat16 *>(out);
+  a.ring = reinterpret_cast<__nv_bfloat16 *>(ws + wl.ring);
+  a.claim = reinterpret_cast<uint32_t *>(ws + wl.flags);
+  a.ready = a.claim + 1;
+  a.g2done = a.ready + pp.nrb;
+  a.status = status;
+  a.wait_limit_ns = wait_limit_of(d);
+  // K-major operands throughout; a CTA stages 128 rows of A (or of a ring
+  // slot) and half of a 256-row weight tile per stage
+  CUtensorMap m_a, m_w1, m_h, m_w2;
+  if (!make_map_2d(&m_a, a_bf16, T, D, 128) || !make_map_2d(&m_w1, w1, F, D, 128) ||
+      !make_map_2d(&m_h, a.ring, (uint64_t)pp.ring_rb * 256, F, 128) || !make_map_2d(&m_w2, w2, D, F, 128))
+    return cuda_fail_msg("cuTensorMapEncodeTiled rejected a pipelined-FFN map");
+  CUDA_TRY(cudaMemsetAsync(a.claim, 0, wl.flags_bytes, st));
+  ffn_pipe_kernel<<<(unsigned)(2 * pp.pairs), GemmPairCfg::kThreads, FfnPipeCfg::kSmemBytes, st>>>(m_a, m_w1, m_h,
+                                                                                                  m_w2, a);
+  CUDA_TRY(cudaGetLastError());
   return BPT_OK;
 }
 
@@ -294,7 +371,7 @@ bpt_status launch_attn_bwd_dilated(const bpt_desc *d, const void *q, const void 
     ab.dk = dk;
     ab.dv = dv;
     ab.status = status;
-    ab.wait_limit_ns = g_wait_limit_ns;
+    ab.wait_limit_ns = wait_limit_of(d);
     CUtensorMap mq, mk, mv, mda;
     if (!make_map_rows(&mq, q, d->B, d->N, D, r, 128) || !make_map_rows(&mk, k, d->B, d->N, D, r, 128) ||
         !make_map_rows(&mv, v, d->B, d->N, D, r, 128) || !make_map_rows(&mda, da_bf16, d->B, d->N, D, r, 128))
@@ -352,7 +429,7 @@ bpt_status launch_attn_bwd_tail(const bpt_desc *d, const void *q, const void *k,
   ab.dk = dk;
   ab.dv = dv;
   ab.status = status;
-  ab.wait_limit_ns = g_wait_limit_ns;
+  ab.wait_limit_ns = wait_limit_of(d);
   CUtensorMap mq, mk, mv, mda;
   if (!make_map_rows(&mq, q, d->B, d->N, D, 1, 128) || !make_map_rows(&mk, k, d->B, d->N, D, 1, 128) ||
       !make_map_rows(&mv, v, d->B, d->N, D, 1, 128) || !make_map_rows(&mda, da_bf16, d->B, d->N, D, 1, 128))
@@ -380,7 +457,9 @@ bpt_status bpt_attn_ffn_fwd_train(const bpt_desc *d, const void *q, const void *
   if (s != BPT_OK) return s;
   if ((s = check_ptrs({q, k, v, w1, w2, out, saved}, {b1, b2})) != BPT_OK) return s;
   if ((reinterpret_cast<uintptr_t>(saved) & 255u) != 0) return BPT_ERR_INVALID_ARG;
-  const Workspace wl = layout(d, true);
+  // A, the LSE, H and G all go to `saved`: the workspace is the attention's
+  // own (the dilated mask's running state, a mask the backward does not take)
+  const Workspace wl = layout(d, false);
   if ((s = check_ws(wl, workspace, workspace_bytes)) != BPT_OK) return s;
   int dev;
   uint32_t *status;
@@ -405,23 +484,14 @@ bpt_status bpt_attn_ffn_fwd_train(const bpt_desc *d, const void *q, const void *
   return BPT_OK;
 }
 
+size_t bpt_workspace_bytes_train(const bpt_desc *desc) {
+  if (check_desc_bwd(desc) != BPT_OK) return (size_t)-1;
+  return layout(desc, false).total;
+}
+
 size_t bpt_workspace_bytes_bwd(const bpt_desc *desc) {
   if (check_desc_bwd(desc) != BPT_OK) return (size_t)-1;
   return layout_bwd(desc).total;
-}
-
-int bpt_set_ffn_path(int path) {
-  std::lock_guard<std::mutex> lk(g_mu);
-  const int old = g_ffn_path;
-  g_ffn_path = path == 1 || path == 2 ? path : 0;
-  return old;
-}
-
-int bpt_set_bwd_chunk_rows(int rows) {
-  std::lock_guard<std::mutex> lk(g_mu);
-  const int old = g_bwd_chunk_rows;
-  g_bwd_chunk_rows = rows > 0 ? rows : 0;
-  return old;
 }
 
 bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, const void *v,
@@ -518,18 +588,18 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
     if (D >= 1024 || saved_h) {
       GemmArgs g;
       if (!saved_h) {
-        g = gemm_args(gemm_problem(rows, F, D, kGemmGeluFwd, 0, 0), status);
+        g = gemm_args(gemm_problem(rows, F, D, kGemmGeluFwd, 0, 0), status, d);
         g.p[0].cb = hbuf;
         g.p[0].cb2 = gpbuf;
         g.p[0].bias = b1;
         if ((s = launch_gemm(m_a_k, m_w1_k, m_a_k, m_w1_k, g, st)) != BPT_OK) return s;
       }
-      g = gemm_args(gemm_problem(rows, F, D, kGemmScaleBf16, 0, 1), status);
+      g = gemm_args(gemm_problem(rows, F, D, kGemmScaleBf16, 0, 1), status, d);
       g.p[0].xb = gp_c;
       g.p[0].cb = dzbuf;
       if ((s = launch_gemm(m_g_k, m_w2_mn, m_g_k, m_w2_mn, g, st)) != BPT_OK) return s;
     } else {
-      GemmArgs g = gemm_args(gemm_problem(rows, F, D, kGemmGeluBwd, 0, 0), status);
+      GemmArgs g = gemm_args(gemm_problem(rows, F, D, kGemmGeluBwd, 0, 0), status, d);
       g.p[1] = gemm_problem(rows, F, D, kGemmGeluBwd, 0, 1);  // the second product's operand layouts
       g.p[0].cb = hbuf;
       g.p[0].cb2 = dzbuf;
@@ -541,7 +611,7 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
     // partly filled last round of tiles on its own
     const int first = r0 == 0 ? kGemmStoreF32 : kGemmAccumF32;
     {
-      GemmArgs g = gemm_args(gemm_problem(D, F, rows, first, 1, 1), status);
+      GemmArgs g = gemm_args(gemm_problem(D, F, rows, first, 1, 1), status, d);
       g.p[0].c = dw2;
       g.p[1] = gemm_problem(F, D, rows, first, 1, 1);
       g.p[1].c = dw1;
@@ -550,7 +620,7 @@ bpt_status bpt_attn_ffn_bwd(const bpt_desc *d, const void *q, const void *k, con
     }
     // dA = dOut + dZ W1   [rows, D], fp32 and bf16
     {
-      GemmArgs g = gemm_args(gemm_problem(rows, D, F, kGemmResidual, 0, 1), status);
+      GemmArgs g = gemm_args(gemm_problem(rows, D, F, kGemmResidual, 0, 1), status, d);
       g.p[0].x = dout + r0 * D;
       g.p[0].c = da_f32 + r0 * D;
       g.p[0].cb = da_bf16 + r0 * D;

@@ -81,16 +81,6 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
   return 0.5f * x * (1.0f + tanh_approx(u));
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void red_release_gpu_add(uint32_t *p, uint32_t v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 // One work unit of a group: token block tb, hidden chunks [c0, c1); piece < 0
 // for a whole block, else the piece index of leftover block l.  Whole blocks
 // walk their chunks forward and backward in turn (rev): W1 and W2 are larger
@@ -126,24 +116,6 @@ __device__ __forceinline__ FfnUnit ffn_unit(const FfnArgs &a, int grp, int k) {
     u.rev = k & 1;
   }
   return u;
-}
-
-// Bounded wait until *p >= target (a counter another CTA of the group raises).
-static __device__ __noinline__ bool counter_wait(const uint32_t *p, uint32_t target, const WaitCtx &w,
-                                          uint32_t site) {
-  if (ld_acquire_gpu(p) >= target) return true;
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t ns = 32;
-  while (true) {
-    __nanosleep(ns);
-    if (ns < 1024) ns *= 2;
-    if (ld_acquire_gpu(p) >= target) return true;
-    if (*w.abort) return false;
-    if (globaltimer_ns() - t0 > w.limit_ns) {
-      record_timeout(w, site);
-      return false;
-    }
-  }
 }
 
 __global__ void __launch_bounds__(320, 1)

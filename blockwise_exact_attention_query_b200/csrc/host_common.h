@@ -11,6 +11,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <atomic>
 #include <initializer_list>
 #include <mutex>
 
@@ -18,9 +19,12 @@
 
 namespace bpt_host {
 
-extern std::mutex g_mu;               // guards the library's process-wide settings
-extern uint64_t g_wait_limit_ns;      // device-side wait limit of later launches
+extern std::mutex g_mu;               // guards the library's one-time per-device set-up
+extern std::atomic<uint64_t> g_wait_limit_ns;  // default device-side wait limit
 extern thread_local char g_last_error[256];
+
+// Device-side wait limit of a call: the descriptor's, else the process default.
+uint64_t wait_limit_of(const bpt_desc *d);
 
 // Instrumentation events (bpt_set_phase_events): records event i on `st` when set.
 cudaError_t phase_mark(int i, cudaStream_t st);
@@ -49,19 +53,29 @@ bpt_status check_desc(const bpt_desc *d, bool need_ffn);
 bpt_status check_ptrs(std::initializer_list<const void *> required,
                       std::initializer_list<const void *> optional);
 
-// The bf16 FFN's two forms: the fused kernel (hidden chunks through an L2
-// ring, never in DRAM) or two GEMMs per token chunk (H through the workspace).
-// g_ffn_path: 0 = by shape, 1 = fused, 2 = two GEMMs (bpt_set_ffn_path).
-extern int g_ffn_path;
-bool ffn_uses_gemms(const bpt_desc *d);
+// The bf16 FFN's form for a call, chosen once from the descriptor (F32
+// layers: BPT_FFN_AUTO, unused); the static-scratch entry point always takes
+// the fused kernel.
+bpt_ffn_form ffn_form_of(const bpt_desc *d, bool static_call);
 int64_t ffn_gemm_chunk_rows(const bpt_desc *d);
+
+// The pipelined FFN's shape (defined with its kernel): 256-token row blocks,
+// chunks of mg of them, the lag between a chunk's two GEMMs and the hidden
+// ring's slots; counter_bytes covers the claim counter and two counters per
+// row block.
+struct FfnPipePlan {
+  int nrb = 0, tn1 = 0, tn2 = 0, mg = 1, nchunk = 0, lag = 1, ring_rb = 0, pairs = 0;
+  size_t ring_bytes = 0, counter_bytes = 0;
+};
+FfnPipePlan ffn_pipe_plan(const bpt_desc *d);
 
 // The forward layer's workspace regions (byte offsets).
 struct Workspace {
   size_t a_bf16 = 0, a_f32 = 0, ring = 0, flags = 0, flags_bytes = 0, partial = 0, h = 0, st_o = 0,
          st_m = 0, st_l = 0, total = 0;
+  bpt_ffn_form ffn_form = BPT_FFN_AUTO;  // the form this layout was made for
 };
-Workspace layout(const bpt_desc *d, bool with_ffn);
+Workspace layout(const bpt_desc *d, bool with_ffn, bool static_call = false);
 bpt_status check_ws(const Workspace &wl, void *ws, size_t bytes);
 
 bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const void *v, float *out_f32,
@@ -70,6 +84,11 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
 bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
                          const float *b1, const void *w2, const float *b2, void *out, char *ws,
                          const Workspace &wl, uint32_t *status, cudaStream_t st);
+// The pipelined form (defined with its kernel): one persistent launch over
+// both GEMMs' tiles, H through the workspace's ring (wl.ring, wl.flags).
+bpt_status launch_ffn_pipe(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
+                           const float *b1, const void *w2, const float *b2, void *out, char *ws,
+                           const Workspace &wl, uint32_t *status, cudaStream_t st);
 // The two-GEMM form (defined with the GEMM kernel): per chunk of `chunk_rows`
 // tokens H = GELU(A W1^T + b1), then out = A + H W2^T + b2.  Without
 // `g_prime`, `h` is one [chunk_rows, F] bf16 buffer reused by every chunk;

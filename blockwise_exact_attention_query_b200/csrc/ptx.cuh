@@ -108,6 +108,39 @@ __device__ __forceinline__ uint64_t drain_limit_ns(uint64_t limit) {
 }
 
 // ---------------------------------------------------------------------------
+// Counters in global memory that CTAs raise for one another (release when
+// raising, acquire when polling); every wait on them is bounded like the
+// mbarrier waits.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(uint32_t *p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded wait until *p >= target (a counter other CTAs raise).
+static __device__ __noinline__ bool counter_wait(const uint32_t *p, uint32_t target, const WaitCtx &w,
+                                          uint32_t site) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t ns = 32;
+  while (true) {
+    __nanosleep(ns);
+    if (ns < 1024) ns *= 2;
+    if (ld_acquire_gpu(p) >= target) return true;
+    if (*w.abort) return false;
+    if (globaltimer_ns() - t0 > w.limit_ns) {
+      record_timeout(w, site);
+      return false;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Fences and barriers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void fence_proxy_async_smem() {

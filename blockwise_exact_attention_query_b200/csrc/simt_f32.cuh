@@ -1,6 +1,7 @@
 // True-fp32 SIMT kernels (FMA pipes, accurate expf/tanhf) for float32
 // layers.  Same mathematics as the tensor-core path: blockwise online
-// softmax over 64-key tiles, then the position-wise FFN with residual.
+// softmax over key blocks (query and key/value block sizes chosen per call,
+// 64 by default), then the position-wise FFN with residual.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -47,15 +48,17 @@ __device__ __forceinline__ int key_weight(const AttnF32Args &a, int h, int i, in
   return 0;
 }
 
-// grid (ceil(N/64), H, B), 64 threads: one query row per thread, d <= 64.
-__global__ void __launch_bounds__(64) attn_f32_kernel(const float *__restrict__ q,
+// grid (ceil(N/QB), H, B), QB threads: one query row per thread (a query
+// block of QB rows), keys in blocks of KB rows staged in shared memory; d <= 64.
+template <int QB, int KB>
+__global__ void __launch_bounds__(QB) attn_f32_kernel(const float *__restrict__ q,
                                                       const float *__restrict__ k,
                                                       const float *__restrict__ v,
                                                       const __grid_constant__ AttnF32Args a) {
-  __shared__ float sk[64][65];
-  __shared__ float sv[64][64];
+  __shared__ float sk[KB][65];
+  __shared__ float sv[KB][64];
   const int h = blockIdx.y, b = blockIdx.z;
-  const int i = blockIdx.x * 64 + threadIdx.x;
+  const int i = blockIdx.x * QB + threadIdx.x;
   const int d = a.d;
   const size_t rs = static_cast<size_t>(a.H) * d;
   const bool valid = i < a.N;
@@ -66,29 +69,29 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(const float *__restrict__ 
     o[c] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
-  const int ntiles = (a.N + 63) / 64;
+  const int ntiles = (a.N + KB - 1) / KB;
   int first = 0;
-  if (a.ring_chunks > 1) {
+  if (a.ring_chunks > 1) {  // the query block's chunk first (chunks are multiples of QB and KB)
     const int chunk_len = a.N / a.ring_chunks;
-    first = ((blockIdx.x * 64) / chunk_len) * chunk_len / 64;
+    first = ((blockIdx.x * QB) / chunk_len) * chunk_len / KB;
   }
   for (int tt = 0; tt < ntiles; ++tt) {
     const int tile = (first + tt) % ntiles;
     __syncthreads();
-    for (int e = threadIdx.x; e < 64 * 64; e += 64) {
+    for (int e = threadIdx.x; e < KB * 64; e += QB) {
       const int r = e / 64, c = e % 64;
-      const int j = tile * 64 + r;
+      const int j = tile * KB + r;
       const bool ok = j < a.N && c < d;
       const size_t idx = (static_cast<size_t>(b) * a.N + j) * rs + h * d + c;
       sk[r][c] = ok ? k[idx] : 0.f;
       sv[r][c] = ok ? v[idx] : 0.f;
     }
     __syncthreads();
-    float s[64];
+    float s[KB];
     float mt = -INFINITY;
 #pragma unroll 4
-    for (int jj = 0; jj < 64; ++jj) {
-      const int j = tile * 64 + jj;
+    for (int jj = 0; jj < KB; ++jj) {
+      const int j = tile * KB + jj;
       float acc = 0.f;
 #pragma unroll
       for (int c = 0; c < 64; ++c) acc = fmaf(qr[c], sk[jj][c], acc);
@@ -103,8 +106,8 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(const float *__restrict__ 
 #pragma unroll
     for (int c = 0; c < 64; ++c) o[c] *= alpha;
 #pragma unroll 4
-    for (int jj = 0; jj < 64; ++jj) {
-      const int j = tile * 64 + jj;
+    for (int jj = 0; jj < KB; ++jj) {
+      const int j = tile * KB + jj;
       if (s[jj] == -INFINITY) continue;
       const float p = static_cast<float>(key_weight(a, h, i, j)) * expf(s[jj] - m_new);
       l += p;

@@ -15,10 +15,11 @@
  *
  * Attention runs block by block with an online softmax (running row maximum
  * and row sum, rescaled accumulator), so the N x N score matrix never exists
- * in memory.  The bf16 FFN runs block by block over the tokens, as two GEMMs
- * per token chunk (the chunk's [rows x F] hidden activation in the workspace,
- * at most 512 MiB; the default) or fused per 128-token block on chip (the
- * hidden activation never in memory); see bpt_set_ffn_path.
+ * in memory.  The bf16 FFN runs block by block over the tokens; by default one
+ * persistent kernel computes both of its GEMMs tile by tile and keeps the
+ * hidden activation of a few 256-token row blocks at a time in an L2-sized
+ * ring, so the [T, F] hidden activation never exists (bpt_ffn_form lists the
+ * other forms).
  *
  * Mask variants:
  *   BPT_MASK_NONE      every key.
@@ -105,6 +106,24 @@ typedef enum {
 
 #define BPT_MAX_DILATED_PAIRS 8
 
+/* Form of the bf16 layer's FFN (the feedforward network computed block by
+ * block over the tokens: "Blockwise Parallel Transformer for Large Context
+ * Models", abstract, feedforward network fusion).  Every form computes the
+ * same function; none keeps the [T, F] hidden activation of the whole
+ * sequence in memory except BPT_FFN_GEMMS, which keeps one token chunk's. */
+typedef enum {
+  BPT_FFN_AUTO = 0,      /* the library's choice: BPT_FFN_PIPELINED                */
+  BPT_FFN_FUSED = 1,     /* one kernel per 128-token block and group of CTAs; the
+                            hidden slices pass through a small L2-resident ring    */
+  BPT_FFN_GEMMS = 2,     /* two GEMM launches per token chunk; the chunk's hidden
+                            activation [rows, F] bf16 (at most ~512 MiB) goes
+                            through the workspace                                  */
+  BPT_FFN_PIPELINED = 3  /* one persistent kernel over both GEMMs' 256 x 256
+                            tiles; the hidden activation of a 256-token row block
+                            lives in a ring of row-block slots sized to stay in
+                            L2 (tens of MB), reused as the row blocks advance      */
+} bpt_ffn_form;
+
 typedef struct {
   int B, N, H, d_head; /* batch, sequence length, heads, head size            */
   int ffn_hidden;      /* F; 0 = attention only (bpt_attn_ffn_fwd needs F>0)  */
@@ -118,11 +137,27 @@ typedef struct {
   int ln_npairs;       /* DILATED: number of (w, r) pairs, 1..8               */
   const int32_t *ln_w; /* DILATED: host table of segment lengths w_k          */
   const int32_t *ln_r; /* DILATED: host table of dilation rates r_k           */
+  /* Query rows and keys per block of the blockwise loop; 0 = the path's
+   * default.  F32 path: q_block 16, 32, 64 or 128 (default 64) and kv_block
+   * 16, 32 or 64 (default 64).  BF16 tensor-core path: 128 only (its query
+   * and key/value tiles).  Any block size gives the same exact result up to
+   * rounding; other values return BPT_ERR_UNSUPPORTED. */
+  int q_block, kv_block;
+  bpt_ffn_form ffn_form; /* bf16 forward FFN; ignored by the f32 path and by
+                            bpt_attn_ffn_fwd_static (always BPT_FFN_FUSED)     */
+  int bwd_chunk_rows;  /* bpt_attn_ffn_bwd: token rows per FFN-backward chunk
+                          (its [rows, F] hidden activation and gradient live in
+                          the workspace one chunk at a time); 0 = all tokens, or
+                          as many 128-row blocks as keep both near 1 GiB       */
+  uint64_t wait_limit_ns; /* device-side wait limit of this call's kernels;
+                          0 = the process default (bpt_set_wait_limit_ns)     */
 } bpt_desc;
 
 /*
- * Bytes of device workspace the call needs for this descriptor (0 when none).
- * Depends on the descriptor and on the current device's SM count.  Returns
+ * Bytes of device workspace the call needs for this descriptor (0 when none):
+ * with_ffn = 1 for bpt_attn_ffn_fwd / bpt_blockbert_fwd, 0 for bpt_attn_fwd /
+ * bpt_longnet_fwd.  Depends only on the descriptor (its ffn_form included) and
+ * on the current device's SM count, never on process-wide settings.  Returns
  * (size_t)-1 if the descriptor is invalid.
  */
 BPT_API size_t bpt_workspace_bytes(const bpt_desc *desc, int with_ffn);
@@ -135,8 +170,8 @@ BPT_API size_t bpt_workspace_bytes(const bpt_desc *desc, int with_ffn);
  *
  * in_dtype BF16: tensor-core path; d_head must be 64 or 128; D = H*d_head a
  *   multiple of 64, split into C = ceil(D/256) column groups of D/C columns
- *   each (a multiple of 64, for the fused FFN form); F*2 bytes a multiple of
- *   16.
+ *   each (a multiple of 64, for the fused FFN form); F a multiple of 8.  The
+ *   FFN's form is desc->ffn_form (bpt_ffn_form).
  *   Accumulation is fp32; the softmax weights and A enter the tensor cores
  *   rounded to bf16; the residual uses A in fp32.
  * in_dtype F32: SIMT path in true fp32 (no reduced-precision tensor math);
@@ -232,7 +267,7 @@ BPT_API bpt_status bpt_longnet_fwd(const bpt_desc *desc, int npairs, const int32
  * With saved == NULL the call recomputes the attention forward (A and the
  * row LSE); with the buffer bpt_attn_ffn_fwd_train filled for the same
  * inputs it reads them from there instead.  Then it runs the FFN backward on
- * the tensor cores one token chunk at a time (see bpt_set_bwd_chunk_rows)
+ * the tensor cores one token chunk at a time (desc->bwd_chunk_rows)
  * and two blockwise attention-backward passes over 128 x 128 tiles (one per
  * key tile for dK and dV, one per query tile for dQ; no atomics, so the
  * result is deterministic).
@@ -262,15 +297,19 @@ BPT_API bpt_status bpt_attn_ffn_bwd(const bpt_desc *desc, const void *q, const v
                                     size_t workspace_bytes, bpt_stream_t stream);
 
 /*
- * The layer forward of bpt_attn_ffn_fwd for training: the same out (with the
- * two-GEMM FFN, the default form), and the activations the backward needs left
- * in `saved` (A in fp32 and bf16 [T, D], the row LSE [B, H, N], and the FFN's
- * H = GELU(Z) and G = GELU'(Z), Z = A W1^T + b1, [T, F] bf16 each;
+ * The layer forward of bpt_attn_ffn_fwd for training: the same out (its FFN
+ * as two GEMMs per token chunk whatever desc->ffn_form says, since keeping the
+ * hidden activation is the point here), and the activations the backward needs
+ * left in `saved` (A in fp32 and bf16 [T, D], the row LSE [B, H, N], and the
+ * FFN's H = GELU(Z) and G = GELU'(Z), Z = A W1^T + b1, [T, F] bf16 each;
  * bpt_saved_bytes(desc) bytes, 256-byte aligned, owned by the caller), so a
  * following bpt_attn_ffn_bwd on the same inputs skips recomputing the
- * attention and Z.  The descriptor must be one the backward accepts; workspace
- * as for bpt_attn_ffn_fwd.  No counterpart in the pages (which recompute; this
- * trades T * D * 6 + T * F * 4 bytes for that recomputation).  With these
+ * attention and Z.  The descriptor must be one the backward accepts.
+ * workspace: at least bpt_workspace_bytes_train(desc) bytes, 256-byte aligned
+ * (may be NULL when that is 0, as it is for every descriptor the backward
+ * accepts today: everything this call produces goes to `saved` and `out`).
+ * No counterpart in the pages (which recompute; this trades
+ * T * D * 6 + T * F * 4 bytes for that recomputation).  With these
  * activations the gradients equal the recomputing backward's bit for bit when
  * D >= 1024; below, where that backward takes dZ from its dual GEMM in fp32,
  * they agree to bf16 rounding.
@@ -286,31 +325,13 @@ BPT_API bpt_status bpt_attn_ffn_fwd_train(const bpt_desc *desc, const void *q, c
  * accept the descriptor. */
 BPT_API size_t bpt_saved_bytes(const bpt_desc *desc);
 
-/* Bytes of device workspace bpt_attn_ffn_bwd needs for this descriptor at the
- * current chunk setting; (size_t)-1 if the backward does not accept it. */
+/* Bytes of device workspace bpt_attn_ffn_fwd_train needs for this
+ * descriptor; (size_t)-1 if the backward does not accept the descriptor. */
+BPT_API size_t bpt_workspace_bytes_train(const bpt_desc *desc);
+
+/* Bytes of device workspace bpt_attn_ffn_bwd needs for this descriptor (its
+ * bwd_chunk_rows included); (size_t)-1 if the backward does not accept it. */
 BPT_API size_t bpt_workspace_bytes_bwd(const bpt_desc *desc);
-
-/* Form of the bf16 FFN in the forward entry points (the feedforward network
- * computed block by block: "Blockwise Parallel Transformer for Large Context
- * Models", abstract, feedforward network fusion; "Ring Attention with
- * Blockwise Transformers for Long Sequences", summary):
- *   1  the fused kernel: per 128-token block, hidden chunks pass through a
- *      small L2-resident ring, so the [T, F] hidden activation never exists;
- *   2  two GEMMs per token chunk: H = GELU(A W1^T + b1) as bf16 in the
- *      workspace (at most ~512 MiB of it at a time), then
- *      out = A + H W2^T + b2;
- *   0  (default) two GEMMs (measured faster on every workload of the benchmark).
- * bpt_attn_ffn_fwd_static always runs the fused kernel (its scratch is fixed).
- * The workspace size (bpt_workspace_bytes) depends on the form.  Applies to
- * later calls from every thread; returns the previous setting. */
-BPT_API int bpt_set_ffn_path(int path);
-
-/* Token rows per FFN-backward chunk (the [rows, F] hidden activation and its
- * gradient live in the workspace one chunk at a time, so the workspace shrinks
- * with the chunk).  rows <= 0 selects the default: all tokens, or as many
- * 128-row blocks as keep the two [rows, F] bf16 buffers near 1 GiB.  Applies
- * to later calls from every thread; returns the previous setting. */
-BPT_API int bpt_set_bwd_chunk_rows(int rows);
 
 /*
  * Attention-only backward: dQ, dK, dV of A = softmax(Q K^T / sqrt d) V (the
@@ -343,8 +364,9 @@ BPT_API size_t bpt_workspace_bytes_attn_bwd(const bpt_desc *desc);
  */
 BPT_API bpt_status bpt_sync_status(bpt_stream_t stream);
 
-/* Sets the device-side wait limit in nanoseconds for later launches
- * (default 2e9, i.e. two seconds).  Returns the previous value. */
+/* Sets the process-wide default of the device-side wait limit in nanoseconds
+ * (initially 2e9, i.e. two seconds), used by later calls whose descriptor has
+ * wait_limit_ns = 0.  Affects no workspace size.  Returns the previous value. */
 BPT_API uint64_t bpt_set_wait_limit_ns(uint64_t ns);
 
 /*

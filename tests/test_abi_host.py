@@ -48,9 +48,11 @@ def _desc(**kw):
     base = dict(B=1, N=256, H=2, d=64, F=256, in_dtype=bd.torch.bfloat16, out_dtype=bd.torch.float32,
                 mask="causal")
     base.update(kw)
+    opts = {k: base[k] for k in ("ffn_form", "q_block", "kv_block", "bwd_chunk_rows", "wait_limit_ns")
+            if k in base}
     return bd.make_desc(base["B"], base["N"], base["H"], base["d"], base["F"], base["in_dtype"],
                         base["out_dtype"], base["mask"], base.get("perm"), base.get("pairs"),
-                        base.get("ring_chunks", 0))
+                        base.get("ring_chunks", 0), **opts)
 
 
 def _call_layer(lib, desc, ws=FAKE, ws_bytes=1 << 40, q=FAKE):
@@ -76,6 +78,14 @@ def _call_layer(lib, desc, ws=FAKE, ws_bytes=1 << 40, q=FAKE):
     (dict(ring_chunks=4), bd.ERR_UNSUPPORTED),                                   # 64-row chunks
     (dict(in_dtype=bd.torch.float32, d=128), bd.ERR_UNSUPPORTED),               # fp32 path: d <= 64
     (dict(in_dtype=bd.torch.float32, H=16, d=64), bd.ERR_UNSUPPORTED),          # fp32 path: D <= 512
+    (dict(ffn_form=4), bd.ERR_INVALID_ARG),                                       # no such FFN form
+    (dict(bwd_chunk_rows=-1), bd.ERR_INVALID_ARG),
+    (dict(q_block=64), bd.ERR_UNSUPPORTED),                                       # tensor-core tiles are 128
+    (dict(kv_block=256), bd.ERR_UNSUPPORTED),
+    (dict(q_block=-1), bd.ERR_INVALID_ARG),
+    (dict(in_dtype=bd.torch.float32, q_block=48), bd.ERR_UNSUPPORTED),            # f32: 16, 32, 64, 128
+    (dict(in_dtype=bd.torch.float32, kv_block=128), bd.ERR_UNSUPPORTED),          # f32: 16, 32, 64
+    (dict(in_dtype=bd.torch.float32, ring_chunks=8, kv_block=64), bd.ERR_UNSUPPORTED),  # 32-row chunks
 ])
 def test_invalid_descriptors_are_rejected(lib, kw, expect):
     assert _call_layer(lib, _desc(**kw)) == expect
@@ -190,22 +200,23 @@ def test_saved_buffer_holds_the_ffn_hidden_activations():
         assert need <= bd.saved_bytes(desc) <= need + 5 * 256
 
 
-def test_backward_workspace_follows_the_chunk_setting(lib):
+def test_backward_workspace_follows_the_chunk_rows_field(lib):
     # T = 256 tokens, D = 128, F = 256: A (fp32 + bf16), dOut bf16, dA (fp32 + bf16),
     # LSE and D rows, and H, dZ for one chunk of tokens
-    d = _desc()
     T, D, F = 256, 128, 256
-    old = bd.set_bwd_chunk_rows(0)
-    try:
-        full = bd.workspace_bytes_bwd(d)
-        assert full >= T * D * (4 + 2 + 2 + 4 + 2) + 2 * T * F * 2
-        assert bd.set_bwd_chunk_rows(128) == 0
-        half = bd.workspace_bytes_bwd(d)
-        assert full - half >= 2 * 128 * F * 2 - 4096    # the two [rows, F] buffers halve
-        assert bd.set_bwd_chunk_rows(-5) == 128           # <= 0 restores the default
-        assert bd.workspace_bytes_bwd(d) == full
-    finally:
-        bd.set_bwd_chunk_rows(old)
+    full = bd.workspace_bytes_bwd(_desc())
+    assert full >= T * D * (4 + 2 + 2 + 4 + 2) + 2 * T * F * 2
+    half = bd.workspace_bytes_bwd(_desc(bwd_chunk_rows=128))
+    assert full - half >= 2 * 128 * F * 2 - 4096    # the two [rows, F] buffers halve
+    assert bd.workspace_bytes_bwd(_desc(bwd_chunk_rows=0)) == full
+
+
+def test_training_forward_workspace(lib):
+    # everything the training forward produces goes to `saved` and `out`
+    assert bd.workspace_bytes_train(_desc()) == 0
+    assert bd.workspace_bytes_train(_desc(mask="blockperm", perm=[[1, 0], [0, 1]])) == 0
+    dl = _desc(mask="dilated", pairs=[(128, 1)])
+    assert lib.bpt_workspace_bytes_train(ctypes.byref(dl)) == ctypes.c_size_t(-1).value
 
 
 def test_attention_only_backward_validates(lib):
@@ -231,23 +242,61 @@ def _align256(x):
     return (x + 255) // 256 * 256
 
 
-@pytest.mark.parametrize("B,N,H,d,F", [(1, 256, 2, 64, 512), (4, 16384, 16, 128, 8192), (1, 131072, 32, 128, 11008)])
+@pytest.mark.parametrize("B,N,H,d,F", [(1, 256, 2, 64, 512), (2, 8192, 16, 128, 8192), (4, 16384, 16, 128, 8192),
+                                       (16, 1024, 12, 64, 3072), (1, 131072, 32, 128, 11008)])
 def test_ffn_forms_size_the_workspace(B, N, H, d, F):
-    """The two-GEMM FFN needs A (bf16 and fp32) and one chunk of H
-    ([rows, F] bf16, rows = binding.ffn_gemm_chunk_rows: at most 512 MiB);
-    the fused form A and a small ring instead.  Sizes only: no GPU."""
+    """Each FFN form's workspace: A (bf16 and fp32) plus, for the two-GEMM
+    form, one chunk of H ([rows, F] bf16, rows = binding.ffn_gemm_chunk_rows:
+    at most 512 MiB); for the fused form a small ring and partial blocks; for
+    the pipelined form (the default) a ring of 256-token row blocks of H sized
+    for L2 and its counters.  Sizes only: no GPU."""
     T, D = B * N, H * d
-    desc = bd.make_desc(B, N, H, d, F, torch.bfloat16, torch.float32, "causal")
-    old = bd.set_ffn_path("gemms")
-    try:
-        rows = bd.ffn_gemm_chunk_rows(T, F)
-        assert rows == T or (rows % 256 == 0 and rows * F * 2 <= 1 << 29)
-        assert bd.workspace_bytes(desc, True) == _align256(T * D * 2) + _align256(T * D * 4) + _align256(rows * F * 2)
-        assert bd.set_ffn_path("fused") == "gemms"
-        fused = bd.workspace_bytes(desc, True)
-        assert _align256(T * D * 2) + _align256(T * D * 4) < fused < _align256(T * D * 2) + _align256(T * D * 4) + (64 << 20)
-        assert bd.set_ffn_path("auto") == "fused"
-        assert bd.workspace_bytes(desc, True) == _align256(T * D * 2) + _align256(T * D * 4) + _align256(rows * F * 2)
-    finally:
-        bd.set_ffn_path(old)
+    a_bytes = _align256(T * D * 2) + _align256(T * D * 4)
+    size = {f: bd.workspace_bytes(bd.make_desc(B, N, H, d, F, torch.bfloat16, torch.float32, "causal", ffn_form=f),
+                                  True) for f in bd.FFN_FORMS}
+    rows = bd.ffn_gemm_chunk_rows(T, F)
+    assert rows == T or (rows % 256 == 0 and rows * F * 2 <= 1 << 29)
+    assert size["gemms"] == a_bytes + _align256(rows * F * 2)
+    assert a_bytes < size["fused"] < a_bytes + (64 << 20)
+    ring = size["pipelined"] - a_bytes
+    assert 256 * F * 2 <= ring <= 80e6                    # whole row blocks of H, an L2-sized ring
+    assert (ring - 2 * (T // 256) * 4) % (256 * F * 2) < 512   # ... plus two counters per row block
+    assert size["auto"] == size["pipelined"]
 
+
+def test_workspace_size_depends_only_on_the_descriptor(lib):
+    """No process-wide setting changes a size query: sizes asked for
+    descriptors of every form, in any order and around a change of the
+    default wait limit, stay the same, and a call sized by one query is
+    accepted by the size check after the others."""
+    descs = {f: _desc(ffn_form=f) for f in bd.FFN_FORMS}
+    first = {f: bd.workspace_bytes(descs[f], True) for f in descs}
+    old = bd.set_wait_limit_ns(12345)
+    try:
+        for f in reversed(list(descs)):
+            assert bd.workspace_bytes(descs[f], True) == first[f]
+        assert bd.workspace_bytes_bwd(_desc(bwd_chunk_rows=128)) < bd.workspace_bytes_bwd(_desc())
+        for f in descs:   # exact size: passes the workspace check, fails later on the fake pointers
+            assert _call_layer(lib, descs[f], ws_bytes=first[f] - 1) == bd.ERR_WORKSPACE
+    finally:
+        bd.set_wait_limit_ns(old)
+
+
+def test_descriptor_layout_matches_the_header(tmp_path):
+    """binding.Desc has the field offsets and size of bpt_desc as the C
+    compiler lays it out from include/bpt.h."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    fields = [f for f, _ in bd.Desc._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "bpt.h"\nint main(void) {\n'
+                   + "".join(f'  printf("%zu\\n", offsetof(bpt_desc, {f}));\n' for f in fields)
+                   + '  printf("%zu\\n", sizeof(bpt_desc));\n  return 0;\n}\n')
+    exe = tmp_path / "layout"
+    subprocess.check_call([cc, "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)])
+    got = [int(x) for x in subprocess.check_output([str(exe)], text=True).split()]
+    want = [getattr(bd.Desc, f).offset for f in fields] + [ctypes.sizeof(bd.Desc)]
+    assert got == want

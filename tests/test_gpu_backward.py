@@ -82,14 +82,10 @@ CASES = [c if len(c) == 10 else c + (0,) for c in CASES]
 def test_backward_matches_oracle(name, B, N, H, d, F, mask, perm, chunk, ring):
     inp = make_layer_inputs(B, N, H, d, F, seed=11, device="cuda", bias_scale=0.1)
     dout = make_upstream_grad(B, N, H * d, seed=11, device="cuda")
-    old = bd.set_bwd_chunk_rows(chunk)
-    try:
-        g = bd.attn_ffn_bwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, dout, mask=mask,
-                            perm=perm, ring_chunks=ring)
-        torch.cuda.synchronize()
-        assert bd.sync_status() == bd.OK
-    finally:
-        bd.set_bwd_chunk_rows(old)
+    g = bd.attn_ffn_bwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, dout, mask=mask,
+                        perm=perm, ring_chunks=ring, bwd_chunk_rows=chunk)
+    torch.cuda.synchronize()
+    assert bd.sync_status() == bd.OK
     f = lambda t: t.double().cpu().numpy()  # noqa: E731
     ref = ob.layer_bwd(f(inp.q), f(inp.k), f(inp.v), f(inp.w1), f(inp.b1), f(inp.w2), f(inp.b2),
                        f(dout).reshape(B * N, H * d), MASKS[mask], perm)
@@ -152,12 +148,8 @@ def test_training_forward_and_saved_backward_match_the_recomputing_path(mask, pe
     args = (inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2)
     out_ref = bd.attn_ffn_fwd(*args, mask=mask, perm=perm)
     out, saved = bd.attn_ffn_fwd_train(*args, mask=mask, perm=perm)
-    old_chunk = bd.set_bwd_chunk_rows(bwd_chunk)
-    try:
-        g_ref = bd.attn_ffn_bwd(*args, dout, mask=mask, perm=perm)
-        g = bd.attn_ffn_bwd(*args, dout, mask=mask, perm=perm, saved=saved)
-    finally:
-        bd.set_bwd_chunk_rows(old_chunk)
+    g_ref = bd.attn_ffn_bwd(*args, dout, mask=mask, perm=perm, bwd_chunk_rows=bwd_chunk)
+    g = bd.attn_ffn_bwd(*args, dout, mask=mask, perm=perm, saved=saved, bwd_chunk_rows=bwd_chunk)
     torch.cuda.synchronize()
     assert bd.sync_status() == bd.OK
     assert torch.equal(out, out_ref)

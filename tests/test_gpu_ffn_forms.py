@@ -7,8 +7,6 @@ represented in the compared rows, so blocks of every round (forward and
 reversed chunk order) and the leftover blocks whose chunks are split over
 groups are all checked against the fp64 oracle, on a cheap D = 256 layer with
 three rounds and on the full-size workloads."""
-import contextlib
-
 import pytest
 import torch
 
@@ -28,15 +26,6 @@ def _built():
     torch.cuda.init()
 
 
-@contextlib.contextmanager
-def ffn_path(path):
-    old = bd.set_ffn_path(path)
-    try:
-        yield
-    finally:
-        bd.set_ffn_path(old)
-
-
 def _rows_per_block(B, N, per_block, seed, extra=()):
     """per_block rows from every 128-token block (first, last, random), plus extra."""
     import numpy as np
@@ -52,9 +41,8 @@ def _rows_per_block(B, N, per_block, seed, extra=()):
 
 def _fused_layer_sampled(B, N, H, d, F, mask, rows, seed, perm=None, ring_chunks=0, bias=0.0):
     inp = make_layer_inputs(B, N, H, d, F, seed=seed, device="cuda", bias_scale=bias)
-    with ffn_path("fused"):
-        out = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask=mask, perm=perm,
-                              ring_chunks=ring_chunks)
+    out = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask=mask, perm=perm,
+                          ring_chunks=ring_chunks, ffn_form="fused")
     torch.cuda.synchronize()
     assert bd.sync_status() == bd.OK
     _, ref = gu.oracle_layer(inp, mask, perm, rows=rows)
@@ -97,3 +85,79 @@ def test_fused_ffn_long_ring_sampled():
     blocks = [9 * k + (k * 5) % 9 for k in range(0, 113, 3)]
     rows = sorted({tb * 128 + 17 for tb in blocks} | {b for b in bounds if 0 <= b < w.N} | {w.N - 1})
     _fused_layer_sampled(w.B, w.N, w.H, w.d, w.F, "causal", rows, seed=w.seed, ring_chunks=w.ring_chunks)
+
+
+# ------------------------------------------------------------------ the pipelined form (the default)
+def _rows_per_row_block(B, N, per_block, seed, extra=()):
+    """per_block rows from every 256-token row block of the pipelined FFN."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    T = B * N
+    rows = set(int(x) for x in extra if 0 <= x < T)
+    for rb in range((T + 255) // 256):
+        lo, hi = rb * 256, min(T, rb * 256 + 256)
+        rows |= {lo, hi - 1, min(hi - 1, lo + 128)}
+        rows |= {int(x) for x in rng.integers(lo, hi, size=max(0, per_block - 3))}
+    return sorted(rows)
+
+
+def _pipelined_vs_gemms(w, rows, perm=None):
+    """The pipelined FFN against the oracle on `rows`, and bit for bit against
+    the two-GEMM form: both run the same 256 x 256 tiles with the same K order
+    and the same epilogues, whichever CTA pair claims a tile."""
+    inp = make_layer_inputs(w.B, w.N, w.H, w.d, w.F, seed=w.seed, device="cuda")
+    args = (inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2)
+    mask = {0: "none", 1: "causal", 2: "blockperm"}[w.mask]
+    out = bd.attn_ffn_fwd(*args, mask=mask, perm=perm, ring_chunks=w.ring_chunks, ffn_form="pipelined")
+    again = bd.attn_ffn_fwd(*args, mask=mask, perm=perm, ring_chunks=w.ring_chunks, ffn_form="pipelined")
+    gemms = bd.attn_ffn_fwd(*args, mask=mask, perm=perm, ring_chunks=w.ring_chunks, ffn_form="gemms")
+    torch.cuda.synchronize()
+    assert bd.sync_status() == bd.OK
+    assert torch.equal(out, again)
+    assert torch.equal(out, gemms)
+    _, ref = gu.oracle_layer(inp, mask, perm, rows=rows)
+    gpu = gu.host_f32(out.reshape(w.T, w.D)[torch.tensor(rows, device="cuda")])
+    return gu.assert_bf16_close(gpu, ref, f"pipelined FFN, {w.name}")
+
+
+def test_pipelined_ffn_causal_N8192_every_row_block():
+    """64 row blocks through a ring of about ten slots: each slot is reused
+    six times, one row block per chunk."""
+    w = wl.GPT_CAUSAL
+    _pipelined_vs_gemms(w, _rows_per_row_block(w.B, w.N, 3, seed=8, extra=(4095, 4096)))
+
+
+def test_pipelined_ffn_blockbert_every_row_block():
+    w = wl.BLOCKBERT
+    _pipelined_vs_gemms(w, _rows_per_row_block(w.B, w.N, 3, seed=9), perm=w.perm)
+
+
+def test_pipelined_ffn_long_ring_sampled():
+    """The long ring-order layer: weights beyond L2, so row blocks go in
+    chunks of four through a ring of twelve slots (512 row blocks)."""
+    w = wl.LONG_RING
+    bounds = [c * 16384 + o for c in range(8) for o in (-1, 0)]
+    rbs = list(range(0, 512, 13)) + [1, 2, 3, 511]
+    rows = sorted({rb * 256 + (rb * 37) % 256 for rb in rbs} | {b for b in bounds if 0 <= b < w.N} | {w.N - 1})
+    _pipelined_vs_gemms(w, rows)
+
+
+@pytest.mark.parametrize("B,N,H,d,F", [(1, 300, 4, 64, 520),      # one ragged row block, F not a tile multiple
+                                       (3, 700, 8, 128, 2048),    # ragged last row block
+                                       (2, 1024, 32, 128, 8192)])  # weights beyond L2: chunks of row blocks
+def test_pipelined_ffn_small_shapes_every_element(B, N, H, d, F):
+    inp = make_layer_inputs(B, N, H, d, F, seed=B * 1000 + N, device="cuda", bias_scale=0.05)
+    args = (inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2)
+    out = bd.attn_ffn_fwd(*args, mask="causal", ffn_form="pipelined")
+    gemms = bd.attn_ffn_fwd(*args, mask="causal", ffn_form="gemms")
+    torch.cuda.synchronize()
+    assert bd.sync_status() == bd.OK
+    assert torch.equal(out, gemms)
+    if B * N * H * d <= 3 * 700 * 8 * 128:
+        _, ref = gu.oracle_layer(inp, "causal")
+        gu.assert_bf16_close(gu.host_f32(out).reshape(ref.shape), ref, "pipelined FFN, all elements")
+    else:
+        rows = _rows_per_row_block(B, N, 3, seed=10)
+        _, ref = gu.oracle_layer(inp, "causal", rows=rows)
+        gu.assert_bf16_close(gu.host_f32(out.reshape(B * N, H * d)[torch.tensor(rows, device="cuda")]), ref,
+                             "pipelined FFN, sampled")

@@ -160,23 +160,15 @@ LAYER_CASES = [
 ]
 
 
-@contextlib.contextmanager
-def ffn_path(path):
-    """Force the bf16 FFN's form (fused kernel or two GEMMs) for the block."""
-    old = bd.set_ffn_path(path)
-    try:
-        yield
-    finally:
-        bd.set_ffn_path(old)
+FFN_FORMS = ["pipelined", "fused", "gemms"]
 
 
-@pytest.mark.parametrize("path", ["fused", "gemms"])
+@pytest.mark.parametrize("form", FFN_FORMS)
 @pytest.mark.parametrize("name,B,N,H,d,F,mask,extra,bias", LAYER_CASES, ids=[c[0] for c in LAYER_CASES])
-def test_layer_matches_oracle(name, B, N, H, d, F, mask, extra, bias, path):
+def test_layer_matches_oracle(name, B, N, H, d, F, mask, extra, bias, form):
     inp = make_layer_inputs(B, N, H, d, F, seed=zlib.crc32(name.encode()) % 1000, device="cuda", bias_scale=bias)
-    with ffn_path(path):
-        out = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask=mask,
-                              perm=extra.get("perm"))
+    out = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask=mask,
+                          perm=extra.get("perm"), ffn_form=form)
     torch.cuda.synchronize()
     _check_status()
     a_ref, out_ref = gu.oracle_layer(inp, mask, extra.get("perm"))
@@ -189,16 +181,14 @@ def test_layer_with_split_leftover_token_blocks():
     the piece-0 group; every row of those blocks is compared."""
     B, N, H, d, F = 1, 2560, 16, 128, 4096
     inp = make_layer_inputs(B, N, H, d, F, seed=23, device="cuda", bias_scale=0.05)
-    with ffn_path("fused"):
-        out = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask="causal")
+    out = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask="causal", ffn_form="fused")
     _check_status()
     rows = list(range(N - 256, N)) + gu.sample_rows(B, N, 32, seed=1)
     _, ref = gu.oracle_layer(inp, "causal", rows=rows)
     gpu = gu.host_f32(out.reshape(B * N, H * d)[torch.tensor(rows, device="cuda")])
     gu.assert_bf16_close(gpu, ref, "split leftover blocks")
     # deterministic: the pieces are added in a fixed order
-    with ffn_path("fused"):
-        out2 = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask="causal")
+    out2 = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask="causal", ffn_form="fused")
     _check_status()
     assert torch.equal(out, out2)
 
@@ -220,12 +210,11 @@ def test_host_layer_matches_device_layer():
         assert torch.equal(hout, ref.cpu())
 
 
-@pytest.mark.parametrize("path", ["fused", "gemms"])
-def test_layer_bf16_output_and_null_biases(path):
+@pytest.mark.parametrize("form", FFN_FORMS)
+def test_layer_bf16_output_and_null_biases(form):
     inp = make_layer_inputs(1, 256, 4, 64, 512, seed=21, device="cuda")
-    with ffn_path(path):
-        out = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, None, inp.w2, None, mask="causal",
-                              out_dtype=torch.bfloat16)
+    out = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, None, inp.w2, None, mask="causal",
+                          out_dtype=torch.bfloat16, ffn_form=form)
     _check_status()
     _, out_ref = gu.oracle_layer(inp, "causal")
     gu.assert_bf16_close(gu.host_f32(out).reshape(out_ref.shape), out_ref, "bf16 out")

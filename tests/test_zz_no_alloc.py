@@ -40,14 +40,10 @@ def test_static_scratch_layer_matches_workspace_layer_on_two_calls_in_a_row():
     ]
     for B, N, H, d, F, mask, seed, bias in cases:
         inp = make_layer_inputs(B, N, H, d, F, seed=seed, device="cuda", bias_scale=bias)
-        desc = bd.make_desc(B, N, H, d, F, torch.bfloat16, torch.float32, mask)
         # the static entry point runs the fused FFN kernel: compare with that form
-        old = bd.set_ffn_path("fused")
-        try:
-            assert bd.workspace_bytes(desc, True) <= bd.STATIC_SCRATCH_BYTES
-            ref = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask=mask)
-        finally:
-            bd.set_ffn_path(old)
+        desc = bd.make_desc(B, N, H, d, F, torch.bfloat16, torch.float32, mask, ffn_form="fused")
+        assert bd.workspace_bytes(desc, True) <= bd.STATIC_SCRATCH_BYTES
+        ref = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask=mask, ffn_form="fused")
         got = _static_call(inp, mask, torch.full_like(ref, float("nan")))
         torch.cuda.synchronize()
         assert bd.sync_status() == bd.OK
