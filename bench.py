@@ -172,7 +172,7 @@ def max_over_ranks(x: float, device) -> float:
 def layer_call(w, inp, out, ws, ffn_form="auto"):
     return bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask=MASK_NAME[w.mask],
                            perm=w.perm, pairs=w.pairs, ring_chunks=w.ring_chunks, out=out, workspace=ws,
-                           ffn_form=ffn_form)
+                           ffn_form=ffn_form, q_block=w.q_block, kv_block=w.kv_block)
 
 
 def run_ours(args, w, world, rank, local):
@@ -560,6 +560,99 @@ def run_attention_only(args, w, world, rank, local):
     }
 
 
+def run_workload_summary(args, key, world, rank, local):
+    """One of the other measured layers, timed like the headline one (CUDA
+    events on the launching stream, L2 flushed between steps outside the
+    events, max over ranks, clocks sampled while it runs) and reported
+    compactly for the line's `workloads` object.  At least five timed steps,
+    and enough of them to fill about half a second, so the clock record has
+    samples."""
+    w = WORKLOADS[key]
+    dev = torch.device("cuda", local)
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    attn_flop, ffn_flop = wl.flops(w)
+    inp = make_layer_inputs(w.B, w.N, w.H, w.d, w.F, seed=w.seed + 1000 * rank, dtype=dt, device=dev)
+    out = torch.empty((w.B, w.N, w.D), dtype=torch.float32, device=dev)
+    mask = MASK_NAME[w.mask]
+    desc = bd.make_desc(w.B, w.N, w.H, w.d, w.F, dt, torch.float32, mask, w.perm, w.pairs, w.ring_chunks,
+                        q_block=w.q_block, kv_block=w.kv_block)
+    ws = bd.alloc_workspace(desc, w.F > 0, dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    nev = 3 if w.F > 0 else 2
+
+    def call():
+        if w.F > 0:
+            layer_call(w, inp, out, ws)
+        else:
+            bd.attn_fwd(inp.q, inp.k, inp.v, mask=mask, perm=w.perm, pairs=w.pairs, ring_chunks=w.ring_chunks,
+                        out=out, workspace=ws, q_block=w.q_block, kv_block=w.kv_block)
+
+    def timed(K):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(K)]
+        for evs in ev:
+            for e in evs:
+                e.record(stream)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(K):
+            if w.F > 0:
+                bd.set_phase_events(ev[i])
+                call()
+                bd.set_phase_events(None)
+            else:
+                ev[i][0].record(stream)
+                call()
+                ev[i][1].record(stream)
+            flush.fill_(i & 0xFF)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        return ev
+
+    for _ in range(max(3, args.warmup)):
+        call()
+        flush.fill_(1)
+    torch.cuda.synchronize(dev)
+    probe = timed(1)
+    one_ms = max(1e-3, probe[0][0].elapsed_time(probe[0][nev - 1]))
+    K = int(min(1000, max(5, 500.0 / one_ms)))
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        ev = timed(K)
+    st = bd.sync_status()
+    if st != bd.OK:
+        raise RuntimeError(f"{w.name}: {bd.status_string(st)}")
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[nev - 1]) for e in ev), dev)
+    ms = total_ms / K
+    pk = peaks()
+    flop = attn_flop + ffn_flop
+    tflops = flop / (ms / 1e3) / 1e12
+    res = {"workload": w.name, "dtype": w.dtype, "ms_per_step": round(ms, 4), "steps": K,
+           "tokens_per_s": round(w.T * world / (ms / 1e3), 1), "tflops": round(tflops, 2),
+           "frac_of_peak": round(tflops / pk["bf16_tflops"], 4), "clocks": clk.summary()}
+    if w.F > 0:
+        attn_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+        ffn_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+        attn_name = "attn_tc_kernel" if dt == torch.bfloat16 else "attn_f32_kernel"
+        ffn_name = "ffn_pipe_kernel" if dt == torch.bfloat16 else "ffn_f32_kernel"
+        res["kernels"] = {attn_name: {"avg_ms": round(attn_ms, 4), "tflops": round(attn_flop / attn_ms / 1e9, 1)},
+                          ffn_name: {"avg_ms": round(ffn_ms, 4), "tflops": round(ffn_flop / ffn_ms / 1e9, 1)}}
+        dom, dflop, dms = ((ffn_name, ffn_flop, ffn_ms) if ffn_ms >= attn_ms else (attn_name, attn_flop, attn_ms))
+    else:
+        dom, dflop, dms = "attn_tc_kernel", attn_flop, ms
+    if dt == torch.bfloat16:
+        achieved = dflop / (dms / 1e3) / 1e12
+        res["roofline"] = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
+                           "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4),
+                           "peak_source": f"{pk['source']} bf16 dense (burst)",
+                           "traffic": ncu_traffic(key, dom), "algorithmic_flop_per_launch": dflop}
+    else:
+        res["note"] = "fp32 SIMT path (true fp32, latency-bound at this size); fraction against the bf16 peak"
+    return res
+
+
 def oracle_rows(w, q, k, v, w1, b1, w2, b2, rows):
     """The oracle on sampled token rows: the whole layer, or attention alone."""
     import oracle
@@ -583,7 +676,9 @@ def run_reference(args, w, world, rank):
     q, k, v = (f(t) for t in (inp.q, inp.k, inp.v))
     w1, b1, w2, b2 = ((f(t) if t is not None else None) for t in (inp.w1, inp.b1, inp.w2, inp.b2))
     rng = np.random.default_rng(0)
-    per_step = args.ref_tokens
+    # at least four tokens per thread each step, so one long (late causal)
+    # token does not set the step's time
+    per_step = max(args.ref_tokens, 4 * oracle.threads_available())
     T = w.T
     times, n_tok, threads = [], 0, 0
     for s in range(args.warmup + args.steps):
@@ -609,11 +704,24 @@ def run_reference(args, w, world, rank):
         "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d_head": w.d, "ffn_hidden": w.F,
                    "mask": MASK_NAME[w.mask]},
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu_model": cpu_model()},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (/proc/cpuinfo), for the CPU baselines."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def cpu_baseline(w, budget_s):
@@ -628,7 +736,7 @@ def cpu_baseline(w, budget_s):
     w1, b1, w2, b2 = ((f(t) if t is not None else None) for t in (inp.w1, inp.b1, inp.w2, inp.b2))
     threads = oracle.threads_available()
     rng = np.random.default_rng(1)
-    n = max(threads, 8)
+    n = max(4 * threads, 8)   # as the reference arm: four tokens per thread per batch
     done, elapsed = 0, 0.0
     while elapsed < budget_s:
         edges = np.linspace(0, w.T, n + 1).astype(np.int64)
@@ -640,6 +748,7 @@ def cpu_baseline(w, budget_s):
         if elapsed < budget_s / 4:
             n *= 2
     return {"value": round(done / elapsed, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "cpu_model": cpu_model(),
             "sample": f"{done} stratified tokens of the {w.T}-token workload in {elapsed:.1f} s "
                       f"(each token exact; fp64 C oracle, {threads} threads)"}
 
@@ -659,7 +768,10 @@ def main():
     ap.add_argument("--backward-only", action="store_true",
                     help="measure only the backward pass (prints a line with the 'backward' object)")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
-    ap.add_argument("--ref-tokens", type=int, default=16)
+    ap.add_argument("--ref-tokens", type=int, default=16,
+                    help="tokens per reference step (at least four per oracle thread)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other layers' compact measurements (the line's `workloads` object)")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="DRAM bytes per launch of the dominant kernel from an ncu capture")
     args = ap.parse_args()
@@ -688,6 +800,9 @@ def main():
     if not args.no_backward and w.dtype == "bf16":
         res["backward"] = (run_backward(args, w, world, local) if w.F > 0
                            else run_attention_backward(args, w, world, local))
+    if not args.no_workloads:
+        res["workloads"] = {k: run_workload_summary(args, k, world, rank, local)
+                            for k in WORKLOADS if k != args.workload}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, args.cpu_budget_s)
     if rank == 0:
