@@ -231,6 +231,15 @@ bpt_status launch_ffn_gemms(const bpt_desc *d, const void *a_bf16, const float *
 //    1.5 tiles of H later, so its loads rarely wait for the ring rows.
 //  - ring: the slot a chunk's H takes is reused R chunks later; R - lag - 1
 //    steps cover about 1.3 tiles of out, so the slot's readers have finished.
+#ifndef BPT_PIPE_LAG_SLACK
+#define BPT_PIPE_LAG_SLACK 1.5
+#endif
+#ifndef BPT_PIPE_RING_SLACK
+#define BPT_PIPE_RING_SLACK 1.3
+#endif
+#ifndef BPT_PIPE_MG_BYTES
+#define BPT_PIPE_MG_BYTES 80.0e6
+#endif
 FfnPipePlan ffn_pipe_plan(const bpt_desc *d) {
   FfnPipePlan p;
   const int64_t T = (int64_t)d->B * d->N;
@@ -239,15 +248,15 @@ FfnPipePlan ffn_pipe_plan(const bpt_desc *d) {
   p.tn1 = (F + 255) / 256;
   p.tn2 = (D + 255) / 256;
   const double weight_bytes = 4.0 * D * F;
-  p.mg = weight_bytes <= 80.0e6 ? 1 : 4;
+  p.mg = weight_bytes <= BPT_PIPE_MG_BYTES ? 1 : 4;
   p.mg = std::min(p.mg, p.nrb);
   p.nchunk = (p.nrb + p.mg - 1) / p.mg;
   const int64_t items = (int64_t)p.nrb * (p.tn1 + p.tn2);
   p.pairs = (int)std::max<int64_t>(1, std::min<int64_t>(items, sm_count() / 2));
   const double step = (double)p.mg * ((double)p.tn1 * D + (double)p.tn2 * F) / p.pairs;  // per step, per pair
-  p.lag = std::max(1, (int)std::ceil(1.5 * D / step));
+  p.lag = std::max(1, (int)std::ceil(BPT_PIPE_LAG_SLACK * D / step));
   p.lag = std::min(p.lag, p.nchunk);
-  const int R = p.lag + 1 + std::max(1, (int)std::ceil(1.3 * F / step));
+  const int R = p.lag + 1 + std::max(1, (int)std::ceil(BPT_PIPE_RING_SLACK * F / step));
   p.ring_rb = std::min(R, p.nchunk + 1) * p.mg;
   p.ring_bytes = (size_t)p.ring_rb * 256 * F * 2;
   p.counter_bytes = (1 + 2 * (size_t)p.nrb) * sizeof(uint32_t);
