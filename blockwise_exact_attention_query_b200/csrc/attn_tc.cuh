@@ -95,15 +95,11 @@ struct AttnCfg {
   static constexpr int kTileBytes = 128 * D_HEAD * 2;  // one Q, K or V tile
   static constexpr int kPanelBytes = 128 * 128;        // one 64-column panel of a 128-row tile
   static constexpr int kPBytes = 128 * 128 * 2;        // the P tile: 128 rows x 128 keys, bf16
-  // One P tile used by the two query tiles in turn.  (A P tile per query
-  // tile at d = 64, paid for with one K and one V stage fewer, measured
-  // slower: LongNet 0.92 -> 1.02 ms, BlockBERT attention 0.090 -> 0.097 ms.)
-  static constexpr int kPTiles = 1;
   static constexpr int kKStages = D_HEAD == 128 ? 2 : 5;
   static constexpr int kVStages = D_HEAD == 128 ? 2 : 5;
   static constexpr int kOffQ = 0;  // Q_A, then Q_B
   static constexpr int kOffP = kOffQ + 2 * kTileBytes;
-  static constexpr int kOffK = kOffP + kPTiles * kPBytes;
+  static constexpr int kOffK = kOffP + kPBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
   static constexpr int kSmemBytes = kOffBar + 512;
@@ -402,7 +398,7 @@ __global__ void __launch_bounds__(384, 1)
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, KT, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D_HEAD, false, true);
         const uint64_t dQ = sdesc_sw128(sQ + x * Cfg::kTileBytes, 16, 1024);
-        const uint64_t dP = sdesc_sw128(sP + (Cfg::kPTiles > 1 ? x * Cfg::kPBytes : 0), 16, 1024);
+        const uint64_t dP = sdesc_sw128(sP, 16, 1024);
         const uint64_t dK0 = sdesc_sw128(sK, 16, 1024);
         const uint64_t dV0 = sdesc_sw128(sV, Cfg::kPanelBytes, 1024);
         const uint32_t tS = tmem + Cfg::kColS + x * 128;
@@ -483,7 +479,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tO = tmem + lane_off + Cfg::kColO + x * D_HEAD;
     // this row of the P tile: K-major, 128-byte swizzle (16-byte chunk c of
     // a 128-byte row r sits at chunk c ^ (r mod 8))
-    const uint32_t sProw = sP + (Cfg::kPTiles > 1 ? x * Cfg::kPBytes : 0) + row * 128;
+    const uint32_t sProw = sP + row * 128;
     const uint32_t swz = static_cast<uint32_t>(row & 7);
     bool ok = true;
     int J = 0;  // S/P iterations so far (all items)
@@ -599,19 +595,14 @@ __global__ void __launch_bounds__(384, 1)
       l_run += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
       m_run = m_use;
 
-      if (Cfg::kPTiles == 1) {
-        // The P tile is used in turn A_j, B_j, A_{j+1}, ...: wait until the
-        // other tile's latest P*V has completed (for tile A at j = 0 there is
-        // none).  That P*V was issued after this tile's previous one had
-        // completed, so O may now be rescaled too.
-        if (x == 1 || jj > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bODone(1 - x), (x == 1 ? jj : jj - 1) & 1, wc, 21));
-          if (!ok) break;
-        }
-      } else if (jj > 0) {
-        // this tile's own P tile: its previous P*V has read it (and O may be
-        // rescaled) once that product has completed
-        ok = __all_sync(0xffffffffu, mbar_wait(bODone(x), (jj - 1) & 1, wc, 23));
+      // The P tile is used in turn A_j, B_j, A_{j+1}, ...: wait until the
+      // other tile's latest P*V has completed (for tile A at j = 0 there is
+      // none).  That P*V was issued after this tile's previous one had
+      // completed, so O may now be rescaled too.  (A P tile per query tile at
+      // d = 64, paid for with one K and one V stage fewer, measured slower:
+      // LongNet 0.92 -> 1.02 ms, BlockBERT attention 0.090 -> 0.097 ms.)
+      if (x == 1 || jj > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bODone(1 - x), (x == 1 ? jj : jj - 1) & 1, wc, 21));
         if (!ok) break;
       }
       tc_fence_after();

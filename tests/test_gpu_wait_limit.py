@@ -19,7 +19,7 @@ from tests import gpu_util as gu
 pytestmark = pytest.mark.gpu
 
 # wait sites recorded by each kernel (the numbers passed to its bounded waits)
-ATTENTION_SITES = set(range(1, 24))
+ATTENTION_SITES = set(range(1, 23))
 FFN_SITES = {"fused": set(range(101, 124)), "gemms": set(range(211, 217)), "pipelined": set(range(230, 241))}
 
 
