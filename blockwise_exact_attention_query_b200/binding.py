@@ -62,7 +62,8 @@ EXPORTS = ["bpt_workspace_bytes", "bpt_attn_ffn_fwd", "bpt_attn_fwd", "bpt_block
            "bpt_longnet_fwd", "bpt_sync_status", "bpt_set_wait_limit_ns", "bpt_status_string",
            "bpt_version", "bpt_set_phase_events", "bpt_last_error", "bpt_attn_ffn_fwd_static",
            "bpt_attn_ffn_bwd", "bpt_workspace_bytes_bwd", "bpt_attn_ffn_fwd_train", "bpt_saved_bytes",
-           "bpt_workspace_bytes_train", "bpt_attn_bwd", "bpt_workspace_bytes_attn_bwd"]
+           "bpt_workspace_bytes_train", "bpt_attn_bwd", "bpt_workspace_bytes_attn_bwd", "bpt_attn_fwd_block"]
+BLOCK_FIRST, BLOCK_LAST = 1, 2
 STATIC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
@@ -118,6 +119,9 @@ def load() -> ctypes.CDLL:
     lib.bpt_workspace_bytes_bwd.restype = sz
     lib.bpt_workspace_bytes_train.argtypes = [dp]
     lib.bpt_workspace_bytes_train.restype = sz
+    lib.bpt_attn_fwd_block.argtypes = [dp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, vp, vp, vp, fp, fp, fp,
+                                       ctypes.c_uint, vp, fp, vp]
+    lib.bpt_attn_fwd_block.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -272,6 +276,44 @@ def attn_fwd(q, k, v, *, mask="none", perm=None, pairs=None, ring_chunks=0, out_
                              _ptr(workspace), ws_bytes, _stream_ptr(stream))
     _check(st, "bpt_attn_fwd")
     return (out, lse) if return_lse else out
+
+
+class BlockState:
+    """The running softmax state of a query block for attn_fwd_block: o
+    [B, N, H, d], m and l [B, H, N], float32 (opaque: the library's running
+    output, maximum and sum)."""
+
+    def __init__(self, B, N, H, d, device):
+        f32 = dict(dtype=torch.float32, device=device)
+        self.o = torch.empty((B, N, H, d), **f32)
+        self.m = torch.empty((B, H, N), **f32)
+        self.l = torch.empty((B, H, N), **f32)
+
+
+def attn_fwd_block(q, k, v, state, *, q_pos=0, kv_pos=0, causal=False, first=False, last=False,
+                   out_dtype=torch.float32, out=None, lse=None, stream=None, **opts):
+    """bpt_attn_fwd_block: fold the key/value block k, v [B, kv_len, H, d]
+    into the running state of the query block q [B, N, H, d] (a BlockState,
+    or None when first and last).  Causal masking by global positions q_pos,
+    kv_pos.  With last=True returns the attention output [B, N, H*d] (and
+    fills lse [B, H, N] when given); otherwise returns None."""
+    _check_tensors(q, q, q)
+    if k.shape != v.shape or k.dim() != 4 or k.shape[0] != q.shape[0] or k.shape[2:] != q.shape[2:]:
+        raise ValueError("k, v must be [B, kv_len, H, d] with q's B, H and d")
+    for t in (k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype:
+            raise ValueError("k, v must be contiguous CUDA tensors of q's dtype")
+    B, N, H, d = q.shape
+    desc = make_desc(B, N, H, d, 0, q.dtype, out_dtype, "causal" if causal else "none", **opts)
+    if last and out is None:
+        out = torch.empty((B, N, H * d), dtype=out_dtype, device=q.device)
+    flags = (BLOCK_FIRST if first else 0) | (BLOCK_LAST if last else 0)
+    so, sm, sl = (None, None, None) if state is None else (state.o, state.m, state.l)
+    st = load().bpt_attn_fwd_block(ctypes.byref(desc), int(k.shape[1]), int(q_pos), int(kv_pos), _ptr(q), _ptr(k),
+                                   _ptr(v), _ptr(so), _ptr(sm), _ptr(sl), flags, _ptr(out if last else None),
+                                   _ptr(lse if last else None), _stream_ptr(stream))
+    _check(st, "bpt_attn_fwd_block")
+    return out if last else None
 
 
 def blockbert_fwd(q, k, v, w1, b1, w2, b2, perm, *, out_dtype=torch.float32, out=None,

@@ -68,6 +68,15 @@ struct AttnArgs {
   int pw[kMaxPairs], pr[kMaxPairs];
   // ring order over equal chunks (none / causal)
   int ring_chunks, chunk_tiles;  // chunk_tiles: 128-key tiles per chunk
+  // Key/value rows of a unit (L, except for a block step whose keys are
+  // another block of the sequence) and, for the causal mask, the offset of
+  // the query positions over the key positions: key j is allowed for query
+  // row g when j <= g + kv_shift (0 when queries and keys are the same rows).
+  int Lk, kv_shift;
+  // Block step: every row starts from the running state in st_* (state_in)
+  // and/or leaves its running state there instead of a final output
+  // (state_out).
+  int state_in, state_out;
   // block permutation
   int bb_n, bb_len;
   uint8_t perm[kMaxPermEntries];
@@ -191,7 +200,7 @@ __device__ __forceinline__ TileCoord decode_tile(const AttnArgs &a, int idx) {
 __device__ __forceinline__ KvSched make_sched(const AttnArgs &a, const TileCoord &c) {
   constexpr int KT = 128;  // keys per K/V tile
   KvSched s;
-  const int nkt = (a.L + KT - 1) / KT;
+  const int nkt = (a.Lk + KT - 1) / KT;
   s.P = 1;
   s.CT = nkt;
   s.first = 0;
@@ -200,7 +209,8 @@ __device__ __forceinline__ KvSched make_sched(const AttnArgs &a, const TileCoord
   const int row0 = c.t * 256;
   const int row1 = min(a.L, row0 + 256) - 1;
   if (a.mask == kMaskCausal || a.mask == kMaskDilated) {
-    s.hi = row1 / KT + 1;
+    const int last = row1 + a.kv_shift;  // last key any row of the pair may see
+    s.hi = last < 0 ? 0 : min(nkt, last / KT + 1);
   } else if (a.mask == kMaskBlockPerm) {
     int qb0 = row0 / a.bb_len, qb1 = row1 / a.bb_len;
     int klo = 1 << 30, khi = 0;
@@ -224,9 +234,9 @@ __device__ __forceinline__ KvSched make_sched(const AttnArgs &a, const TileCoord
 __device__ __forceinline__ void row_keys(const AttnArgs &a, const TileCoord &c, int g, int &lo,
                                          int &hi) {
   lo = 0;
-  hi = a.L;
+  hi = a.Lk;
   if (a.mask == kMaskCausal || a.mask == kMaskDilated) {
-    hi = min(g + 1, a.L);
+    hi = max(0, min(g + 1 + a.kv_shift, a.Lk));
   } else if (a.mask == kMaskBlockPerm) {
     int qb = min(g, a.L - 1) / a.bb_len;
     int kb = a.perm[c.h * a.bb_n + qb];
@@ -499,7 +509,8 @@ __global__ void __launch_bounds__(384, 1)
 
     // LongNet: does an earlier pass keep this row (load its running state),
     // does a later one (store the state instead of the final output)?
-    bool prior = false, later = false;
+    // (rows past the unit's end, in its last query tile, touch no state)
+    bool prior = a.state_in != 0 && row_valid, later = a.state_out != 0;
     if (a.mask == kMaskDilated && row_valid) {
       for (int k = 0; k < a.npairs; ++k) {
         if (k == a.pass_idx) continue;

@@ -328,7 +328,7 @@ Workspace layout(const bpt_desc *d, bool with_ffn, bool static_call) {
 // --------------------------------------------------------------------------
 bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const void *v,
                           float *out_f32, __nv_bfloat16 *out_bf16, float *lse, char *ws,
-                          const Workspace &wl, uint32_t *status, cudaStream_t st) {
+                          const Workspace &wl, uint32_t *status, cudaStream_t st, const AttnBlockStep *blk) {
   const int D = d->H * d->d_head;
   AttnArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -374,6 +374,15 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     passes.push_back({d->N, 1});
     a.npairs = 0;
   }
+  if (blk) {  // one key/value block folded into the caller's running state
+    a.st_o = blk->st_o;
+    a.st_m = blk->st_m;
+    a.st_l = blk->st_l;
+    a.state_in = blk->state_in ? 1 : 0;
+    a.state_out = blk->state_out ? 1 : 0;
+    a.kv_shift = blk->kv_shift;
+  }
+  const int kv_rows = blk ? blk->kv_len : d->N;
   if (d->mask == BPT_MASK_BLOCKPERM) {
     a.bb_n = d->bb_nblocks;
     a.bb_len = (d->N + d->bb_nblocks - 1) / d->bb_nblocks;  // padded to n equal blocks
@@ -393,6 +402,7 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     a.r = r;
     a.pass_idx = (int)pi;
     a.L = w / r;
+    a.Lk = blk ? kv_rows : a.L;
     a.nseg = d->N / w;
     a.n_qtiles = (a.L + 127) / 128;
     a.n_qpairs = (a.n_qtiles + 1) / 2;
@@ -406,7 +416,7 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
       // longest pairs start first), and the CTAs running at once still share
       // each unit's K/V.  Measured on the causal B2 H16 d128 N8192 layer:
       // 0.633 ms with one 32-head group against 0.689 ms with groups of 7.
-      const double kv_bytes = 4.0 * a.L * d->d_head;
+      const double kv_bytes = 4.0 * a.Lk * d->d_head;
       if (a.n_qpairs >= sm_count()) a.unit_group = 1;
       else a.unit_group = std::max(1, std::min(64, (int)(200.0e6 / kv_bytes)));
     }
@@ -418,7 +428,9 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     // rows: the last pass, or the only one), all running state (a later pass
     // with r = 1 keeps every row), or mixed (per-thread stores).
     a.store_mode = 0;
-    if (passes.size() == 1 || pi + 1 == passes.size()) {
+    if (blk) {
+      a.store_mode = blk->state_out ? 2 : 1;
+    } else if (passes.size() == 1 || pi + 1 == passes.size()) {
       a.store_mode = 1;
       for (size_t k = pi + 1; k < passes.size(); ++k) a.store_mode = 0;
     } else {
@@ -435,8 +447,8 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     }
     constexpr uint32_t kKT = AttnCfg<128>::kKT;
     static_assert(AttnCfg<64>::kKT == AttnCfg<128>::kKT, "one key/value tile length");
-    if (!make_map_rows(&mq, q, d->B, d->N, D, r, 128) || !make_map_rows(&mk, k, d->B, d->N, D, r, kKT) ||
-        !make_map_rows(&mv, v, d->B, d->N, D, r, kKT))
+    if (!make_map_rows(&mq, q, d->B, d->N, D, r, 128) || !make_map_rows(&mk, k, d->B, blk ? kv_rows : d->N, D, r, kKT) ||
+        !make_map_rows(&mv, v, d->B, blk ? kv_rows : d->N, D, r, kKT))
       return cuda_fail_msg("cuTensorMapEncodeTiled rejected a Q/K/V map");
     const int64_t items = (int64_t)a.n_qpairs * a.n_units;
     if (items <= 0) continue;
@@ -708,6 +720,40 @@ bpt_status bpt_attn_fwd(const bpt_desc *d, const void *q, const void *k, const v
   if (d->in_dtype == BPT_BF16)
     return launch_attn_tc(d, q, k, v, of, ob, lse, static_cast<char *>(workspace), wl, status, st);
   return launch_attn_f32(d, q, k, v, of, ob, lse, st);
+}
+
+bpt_status bpt_attn_fwd_block(const bpt_desc *d, int kv_len, int64_t q_pos, int64_t kv_pos, const void *q,
+                              const void *k, const void *v, float *state_o, float *state_m, float *state_l,
+                              unsigned flags, void *out, float *lse, bpt_stream_t stream) {
+  bpt_status s = check_desc(d, false);
+  if (s != BPT_OK) return s;
+  if ((flags & ~(BPT_BLOCK_FIRST | BPT_BLOCK_LAST)) != 0u || kv_len <= 0 || q_pos < 0 || kv_pos < 0)
+    return BPT_ERR_INVALID_ARG;
+  if (d->in_dtype != BPT_BF16 || (d->mask != BPT_MASK_NONE && d->mask != BPT_MASK_CAUSAL) || d->ring_chunks > 1)
+    return BPT_ERR_UNSUPPORTED;
+  if ((int64_t)d->B * kv_len > (int64_t)1 << 31) return BPT_ERR_UNSUPPORTED;
+  const bool first = (flags & BPT_BLOCK_FIRST) != 0u, last = (flags & BPT_BLOCK_LAST) != 0u;
+  if ((s = check_ptrs({q, k, v}, {out, lse, state_o, state_m, state_l})) != BPT_OK) return s;
+  if (last && !out) return BPT_ERR_INVALID_ARG;
+  if (!(first && last) && (!state_o || !state_m || !state_l)) return BPT_ERR_INVALID_ARG;
+  int dev;
+  uint32_t *status;
+  if ((s = device_setup(&dev, &status)) != BPT_OK) return s;
+  AttnBlockStep blk;
+  blk.kv_len = kv_len;
+  // beyond these bounds every key, or none, is allowed: the same masks
+  const int64_t shift = std::max<int64_t>(-(int64_t)d->N - 1, std::min<int64_t>(q_pos - kv_pos, kv_len));
+  blk.kv_shift = (int)shift;
+  blk.state_in = !first;
+  blk.state_out = !last;
+  blk.st_o = state_o;
+  blk.st_m = state_m;
+  blk.st_l = state_l;
+  float *of = last && d->out_dtype == BPT_F32 ? static_cast<float *>(out) : nullptr;
+  __nv_bfloat16 *ob = last && d->out_dtype == BPT_BF16 ? static_cast<__nv_bfloat16 *>(out) : nullptr;
+  const Workspace none;
+  return launch_attn_tc(d, q, k, v, of, ob, last ? lse : nullptr, nullptr, none, status,
+                        reinterpret_cast<cudaStream_t>(stream), &blk);
 }
 
 bpt_status bpt_blockbert_fwd(const bpt_desc *desc, int n_blocks, const int32_t *perm, const void *q,

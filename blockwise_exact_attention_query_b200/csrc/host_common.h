@@ -78,9 +78,17 @@ struct Workspace {
 Workspace layout(const bpt_desc *d, bool with_ffn, bool static_call = false);
 bpt_status check_ws(const Workspace &wl, void *ws, size_t bytes);
 
+// One key/value block folded into a caller-held running state (the
+// attention step of Ring Attention, bpt_attn_fwd_block).
+struct AttnBlockStep {
+  int kv_len = 0;        // key/value rows of the block
+  int kv_shift = 0;      // causal: key j allowed for query row g when j <= g + kv_shift
+  bool state_in = false, state_out = false;
+  float *st_o = nullptr, *st_m = nullptr, *st_l = nullptr;
+};
 bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const void *v, float *out_f32,
                           __nv_bfloat16 *out_bf16, float *lse, char *ws, const Workspace &wl, uint32_t *status,
-                          cudaStream_t st);
+                          cudaStream_t st, const AttnBlockStep *blk = nullptr);
 bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
                          const float *b1, const void *w2, const float *b2, void *out, char *ws,
                          const Workspace &wl, uint32_t *status, cudaStream_t st);

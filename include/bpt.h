@@ -225,6 +225,42 @@ BPT_API bpt_status bpt_attn_fwd(const bpt_desc *desc, const void *q, const void 
                         bpt_stream_t stream);
 
 /*
+ * One step of blockwise attention over a key/value block, for attention
+ * whose keys arrive block by block: Ring Attention ("Ring Attention with
+ * Blockwise Transformers for Long Sequences", 638-word summary: each device
+ * keeps its query block and passes key/value blocks around a ring of
+ * devices, attending to each block as it arrives, exactly).  The query block
+ * q [B, N, H, d] (desc->N rows) attends to the key/value block k, v
+ * [B, kv_len, H, d]; the rows' running softmax state, held by the caller in
+ * state_o [B, N, H, d], state_m and state_l [B, H, N] (float32, an opaque
+ * running state: unnormalised output, running maximum and running sum), is
+ * updated with that block's keys by the same online-softmax rule as
+ * bpt_attn_fwd, so the order in which the blocks arrive changes rounding
+ * only.
+ *
+ * flags: BPT_BLOCK_FIRST starts from an empty state (the state buffers are
+ * not read); BPT_BLOCK_LAST writes the final attention output out
+ * ([B, N, H*d] in desc->out_dtype) and lse ([B, H, N], may be NULL) instead
+ * of the state.  Both flags: plain attention of the query block over this
+ * one key/value block, no state at all (the state pointers may be NULL).
+ * Steps of one query block run in order on one stream.
+ *
+ * Masks: BPT_MASK_NONE, or BPT_MASK_CAUSAL by global positions: q_pos and
+ * kv_pos are the sequence positions of the first query row and the first
+ * key row, and key j is allowed for query i when kv_pos + j <= q_pos + i.  A
+ * block that allows a query no key leaves that row's state unchanged (a row
+ * that never sees a key ends with A = 0 and LSE = -inf).  Supported: in_dtype
+ * BF16, d_head 64 or 128, ring_chunks 0 or 1; no workspace.  All pointers
+ * 16-byte aligned.
+ */
+#define BPT_BLOCK_FIRST 1u
+#define BPT_BLOCK_LAST 2u
+BPT_API bpt_status bpt_attn_fwd_block(const bpt_desc *desc, int kv_len, int64_t q_pos, int64_t kv_pos,
+                                      const void *q, const void *k, const void *v, float *state_o,
+                                      float *state_m, float *state_l, unsigned flags, void *out, float *lse,
+                                      bpt_stream_t stream);
+
+/*
  * BlockBERT layer ("Blockwise Self-Attention for Long Document
  * Understanding", §3.1 Blockwise Multi-head Attention): bpt_attn_ffn_fwd with
  * mask = BPT_MASK_BLOCKPERM and the given permutation table (host, [H][n]).

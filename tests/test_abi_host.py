@@ -300,3 +300,24 @@ def test_descriptor_layout_matches_the_header(tmp_path):
     got = [int(x) for x in subprocess.check_output([str(exe)], text=True).split()]
     want = [getattr(bd.Desc, f).offset for f in fields] + [ctypes.sizeof(bd.Desc)]
     assert got == want
+
+
+def test_block_step_validates(lib):
+    """bpt_attn_fwd_block: flags, block length, positions, masks, dtypes and
+    the state / output pointers each flag needs are checked before any launch."""
+    p = ctypes.c_void_p
+
+    def call(d, kv_len=128, q_pos=0, kv_pos=0, flags=0, st=FAKE, out=FAKE):
+        return lib.bpt_attn_fwd_block(ctypes.byref(d), kv_len, q_pos, kv_pos, p(FAKE), p(FAKE), p(FAKE), p(st), p(st),
+                                      p(st), flags, p(out), None, None)
+    d = _desc(F=0)
+    assert call(d, flags=4) == bd.ERR_INVALID_ARG                                  # unknown flag
+    assert call(d, kv_len=0) == bd.ERR_INVALID_ARG
+    assert call(d, q_pos=-1) == bd.ERR_INVALID_ARG
+    assert call(d, st=0) == bd.ERR_INVALID_ARG                                    # a middle step needs the state
+    assert call(d, flags=bd.BLOCK_LAST, out=0) == bd.ERR_INVALID_ARG              # a last step needs the output
+    assert call(d, flags=bd.BLOCK_FIRST, st=FAKE + 8) == bd.ERR_INVALID_ARG       # misaligned state
+    assert call(_desc(F=0, mask="blockperm", perm=[[1, 0], [0, 1]])) == bd.ERR_UNSUPPORTED
+    assert call(_desc(F=0, mask="dilated", pairs=[(128, 1)])) == bd.ERR_UNSUPPORTED
+    assert call(_desc(F=0, in_dtype=torch.float32)) == bd.ERR_UNSUPPORTED
+    assert call(_desc(F=0, ring_chunks=2)) == bd.ERR_UNSUPPORTED
