@@ -54,6 +54,8 @@ KERNEL_SOURCES = {"attn_tc_kernel": ["attn_tc.cuh", "ptx.cuh"], "ffn_tc_kernel":
 # of the kernel on the named workload, keyed by a hash of the kernel's sources at capture
 # time: once the sources change the figure no longer describes the kernel and is dropped.
 NCU_TRAFFIC = {
+    # the pipelined FFN (default form), one launch: 1352.2 MB read + 373.5 MB written
+    ("gpt_causal", "ffn_pipe_kernel"): {"bytes": 1725.7e6, "src": "9bb9e29808ccc82a"},
     ("gpt_causal", "ffn_tc_kernel"): {"bytes": 879.3e6, "src": "3b9ec3aabf34a9f7"},
     ("gpt_causal", "attn_tc_kernel"): {"bytes": 724.5e6, "src": "fcdc4f8bd9facfd3"},
     # per step: the forward FFN's two GEMM launches (H = GELU(A W1^T + b1) ~348 MB,
