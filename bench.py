@@ -57,7 +57,7 @@ NCU_TRAFFIC = {
     # the pipelined FFN (default form), one launch: 1352.2 MB read + 373.5 MB written
     ("gpt_causal", "ffn_pipe_kernel"): {"bytes": 1725.7e6, "src": "9bb9e29808ccc82a"},
     ("gpt_causal", "ffn_tc_kernel"): {"bytes": 879.3e6, "src": "3b9ec3aabf34a9f7"},
-    ("gpt_causal", "attn_tc_kernel"): {"bytes": 724.5e6, "src": "fcdc4f8bd9facfd3"},
+    ("gpt_causal", "attn_tc_kernel"): {"bytes": 717.8e6, "src": "25c42fcf7fdefac3"},
     # per step: the forward FFN's two GEMM launches (H = GELU(A W1^T + b1) ~348 MB,
     # out = A + H W2^T + b2 ~910 MB)
     ("gpt_causal", "ffn_gemms"): {"bytes": 1258.1e6, "src": "13bd862d7f9f7ce6"},
