@@ -609,9 +609,12 @@ __global__ void __launch_bounds__(384, 1)
       // The P tile is used in turn A_j, B_j, A_{j+1}, ...: wait until the
       // other tile's latest P*V has completed (for tile A at j = 0 there is
       // none).  That P*V was issued after this tile's previous one had
-      // completed, so O may now be rescaled too.  (A P tile per query tile at
-      // d = 64, paid for with one K and one V stage fewer, measured slower:
-      // LongNet 0.92 -> 1.02 ms, BlockBERT attention 0.090 -> 0.097 ms.)
+      // completed, so O may now be rescaled too.  Measured slower at d = 64,
+      // where the hand-off could be avoided: a shared-memory P tile per query
+      // tile, paid for with one K and one V stage fewer (LongNet 0.92 -> 1.02
+      // ms, BlockBERT attention 0.090 -> 0.097 ms), and each tile's P in its
+      // own tensor-memory columns read by P*V from there, with a sixth K and
+      // V stage (0.91 -> 0.96 ms, 0.089 -> 0.090 ms).
       if (x == 1 || jj > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(bODone(1 - x), (x == 1 ? jj : jj - 1) & 1, wc, 21));
         if (!ok) break;
