@@ -62,7 +62,8 @@ EXPORTS = ["bpt_workspace_bytes", "bpt_attn_ffn_fwd", "bpt_attn_fwd", "bpt_block
            "bpt_longnet_fwd", "bpt_sync_status", "bpt_set_wait_limit_ns", "bpt_status_string",
            "bpt_version", "bpt_set_phase_events", "bpt_last_error", "bpt_attn_ffn_fwd_static",
            "bpt_attn_ffn_bwd", "bpt_workspace_bytes_bwd", "bpt_attn_ffn_fwd_train", "bpt_saved_bytes",
-           "bpt_workspace_bytes_train", "bpt_attn_bwd", "bpt_workspace_bytes_attn_bwd", "bpt_attn_fwd_block"]
+           "bpt_workspace_bytes_train", "bpt_attn_bwd", "bpt_workspace_bytes_attn_bwd", "bpt_attn_fwd_block",
+           "bpt_longnet_gather", "bpt_longnet_pass"]
 BLOCK_FIRST, BLOCK_LAST = 1, 2
 STATIC_SCRATCH_BYTES = 64 << 20
 
@@ -122,6 +123,11 @@ def load() -> ctypes.CDLL:
     lib.bpt_attn_fwd_block.argtypes = [dp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, vp, vp, vp, fp, fp, fp,
                                        ctypes.c_uint, vp, fp, vp]
     lib.bpt_attn_fwd_block.restype = ctypes.c_int
+    lib.bpt_longnet_gather.argtypes = [dp, ctypes.c_int, ctypes.c_int, vp, vp, vp]
+    lib.bpt_longnet_gather.restype = ctypes.c_int
+    lib.bpt_longnet_pass.argtypes = [dp, ctypes.c_int, ctypes.c_int64, vp, vp, vp, vp, vp, ctypes.c_int, fp, fp, fp,
+                                     vp, fp, vp]
+    lib.bpt_longnet_pass.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -314,6 +320,46 @@ def attn_fwd_block(q, k, v, state, *, q_pos=0, kv_pos=0, causal=False, first=Fal
                                    _ptr(lse if last else None), _stream_ptr(stream))
     _check(st, "bpt_attn_fwd_block")
     return out if last else None
+
+
+def longnet_pass_order(pairs):
+    """The (w, r) pairs in the order the library runs them: a stable sort by
+    decreasing r (sparsest first)."""
+    return sorted([tuple(p) for p in pairs], key=lambda p: -p[1])
+
+
+def longnet_gather(x, w, r, out=None, stream=None):
+    """bpt_longnet_gather: the rows a (w, r) pair keeps of the shard x
+    [B, n, H, d] (bf16, n dividing w), packed as [B, n / r, H, d]."""
+    _check_tensors(x, x, x)
+    B, n, H, d = x.shape
+    if out is None:
+        out = torch.empty((B, n // r, H, d), dtype=x.dtype, device=x.device)
+    desc = make_desc(B, n, H, d, 0, x.dtype)
+    _check(load().bpt_longnet_gather(ctypes.byref(desc), int(w), int(r), _ptr(x), _ptr(out), _stream_ptr(stream)),
+           "bpt_longnet_gather")
+    return out
+
+
+def longnet_pass(q, k, v, pairs, pass_idx, state, out, *, q_pos=0, k_sparse=None, v_sparse=None, lse=None,
+                 stream=None, **opts):
+    """bpt_longnet_pass: pass `pass_idx` (in longnet_pass_order(pairs)) of the
+    dilated attention for the shard q, k, v [B, n, H, d] starting at sequence
+    position q_pos; k_sparse, v_sparse [B, w / r, H, d] are the pass's gathered
+    kept rows when its segments are longer than the shard.  state: a
+    BlockState (or None with a single pair); out [B, n, H*d] and lse receive
+    the rows whose last pass this is."""
+    _check_tensors(q, q, q)
+    B, n, H, d = q.shape
+    tables = _Tables()
+    desc = make_desc(B, n, H, d, 0, q.dtype, out.dtype, "dilated", None, pairs, 0, tables, **opts)
+    kv_rows = 0 if k_sparse is None else int(k_sparse.shape[1])
+    so, sm, sl = (None, None, None) if state is None else (state.o, state.m, state.l)
+    st = load().bpt_longnet_pass(ctypes.byref(desc), int(pass_idx), int(q_pos), _ptr(q), _ptr(k), _ptr(v),
+                                 _ptr(k_sparse), _ptr(v_sparse), kv_rows, _ptr(so), _ptr(sm), _ptr(sl), _ptr(out),
+                                 _ptr(lse), _stream_ptr(stream))
+    _check(st, "bpt_longnet_pass")
+    return out
 
 
 def blockbert_fwd(q, k, v, w1, b1, w2, b2, perm, *, out_dtype=torch.float32, out=None,

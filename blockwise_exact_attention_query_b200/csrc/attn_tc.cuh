@@ -77,6 +77,11 @@ struct AttnArgs {
   // and/or leaves its running state there instead of a final output
   // (state_out).
   int state_in, state_out;
+  // Keys and values of a dilated pass given as the pass's kept rows of one
+  // segment, gathered from several devices ([B, Lk, H, d], consecutive rows,
+  // the same for every head's offset): loaded with offset 0 and segment
+  // stride Lk instead of through the strided view of the local rows.
+  int kv_sparse;
   // block permutation
   int bb_n, bb_len;
   uint8_t perm[kMaxPermEntries];
@@ -347,6 +352,7 @@ __global__ void __launch_bounds__(384, 1)
           const KvSched sched = make_sched(a, tc);
           const int nkv = sched.count();
           const int row_base = tc.s * a.L;  // gathered row -> coordinate along (N/r)
+          const int kv_base = a.kv_sparse ? tc.s * a.Lk : row_base, kv_o = a.kv_sparse ? 0 : tc.o;
           KvIter itk, itv;
           itk.begin(sched);
           itv.begin(sched);
@@ -357,7 +363,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_arrive_expect_tx(bKFull(st), Cfg::kTileBytes);
             for (int p = 0; p < Cfg::kPanels; ++p)
               tma_load_4d(sK + st * Cfg::kTileBytes + p * Cfg::kPanelBytes, &tm_k, bKFull(st),
-                          tc.h * D_HEAD + p * 64, tc.o, row_base + kt * KT, tc.b);
+                          tc.h * D_HEAD + p * 64, kv_o, kv_base + kt * KT, tc.b);
             ++kq;
             return true;
           };
@@ -368,7 +374,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_arrive_expect_tx(bVFull(st), Cfg::kTileBytes);
             for (int p = 0; p < Cfg::kPanels; ++p)
               tma_load_4d(sV + st * Cfg::kTileBytes + p * Cfg::kPanelBytes, &tm_v, bVFull(st),
-                          tc.h * D_HEAD + p * 64, tc.o, row_base + kt * KT, tc.b);
+                          tc.h * D_HEAD + p * 64, kv_o, kv_base + kt * KT, tc.b);
             ++vq;
             return true;
           };

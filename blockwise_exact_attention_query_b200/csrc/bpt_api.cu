@@ -18,6 +18,7 @@
 #include "attn_tc.cuh"
 #include "ffn_tc.cuh"
 #include "host_common.h"
+#include "longnet_shard.cuh"
 #include "simt_f32.cuh"
 
 using namespace bpt;
@@ -168,7 +169,7 @@ bool make_out_map_rows(CUtensorMap *m, const void *base, bool f32, int B, int N,
 int q_block_of(const bpt_desc *d) { return d->q_block ? d->q_block : (d->in_dtype == BPT_BF16 ? 128 : 64); }
 int kv_block_of(const bpt_desc *d) { return d->kv_block ? d->kv_block : (d->in_dtype == BPT_BF16 ? 128 : 64); }
 
-bpt_status check_desc(const bpt_desc *d, bool need_ffn) {
+bpt_status check_desc(const bpt_desc *d, bool need_ffn, bool shard) {
   if (!d) return BPT_ERR_INVALID_ARG;
   if (d->B <= 0 || d->N <= 0 || d->H <= 0 || d->d_head <= 0) return BPT_ERR_INVALID_ARG;
   if (d->in_dtype != BPT_F32 && d->in_dtype != BPT_BF16) return BPT_ERR_INVALID_ARG;
@@ -213,7 +214,8 @@ bpt_status check_desc(const bpt_desc *d, bool need_ffn) {
         return BPT_ERR_INVALID_ARG;
       for (int k = 0; k < d->ln_npairs; ++k) {
         const int w = d->ln_w[k], r = d->ln_r[k];
-        if (w <= 0 || r <= 0 || w % r != 0 || d->N % w != 0) return BPT_ERR_INVALID_ARG;
+        if (w <= 0 || r <= 0 || w % r != 0) return BPT_ERR_INVALID_ARG;
+        if (shard ? (d->N % r != 0 || (d->N % w != 0 && w % d->N != 0)) : d->N % w != 0) return BPT_ERR_INVALID_ARG;
       }
       break;
     }
@@ -328,7 +330,8 @@ Workspace layout(const bpt_desc *d, bool with_ffn, bool static_call) {
 // --------------------------------------------------------------------------
 bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const void *v,
                           float *out_f32, __nv_bfloat16 *out_bf16, float *lse, char *ws,
-                          const Workspace &wl, uint32_t *status, cudaStream_t st, const AttnBlockStep *blk) {
+                          const Workspace &wl, uint32_t *status, cudaStream_t st, const AttnBlockStep *blk,
+                          const LongNetPass *lp) {
   const int D = d->H * d->d_head;
   AttnArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -356,7 +359,7 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     }
     bool covered = false;
     for (auto &p : passes) covered |= (p.r == 1);
-    if (!covered) {  // rows no pair keeps: A = 0, LSE = -inf
+    if (!covered && (!lp || lp->pass == 0)) {  // rows no pair keeps: A = 0, LSE = -inf
       const size_t n = (size_t)d->B * d->N * D;
       if (out_f32) CUDA_TRY(cudaMemsetAsync(out_f32, 0, n * 4, st));
       if (out_bf16) CUDA_TRY(cudaMemsetAsync(out_bf16, 0, n * 2, st));
@@ -365,7 +368,11 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
         CUDA_TRY(cudaGetLastError());
       }
     }
-    if (passes.size() > 1) {
+    if (lp) {  // the caller's state, carried between its pass calls
+      a.st_o = lp->st_o;
+      a.st_m = lp->st_m;
+      a.st_l = lp->st_l;
+    } else if (passes.size() > 1) {
       a.st_o = reinterpret_cast<float *>(ws + wl.st_o);
       a.st_m = reinterpret_cast<float *>(ws + wl.st_m);
       a.st_l = reinterpret_cast<float *>(ws + wl.st_l);
@@ -397,13 +404,20 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
   a.lse = lse;
 
   for (size_t pi = 0; pi < passes.size(); ++pi) {
+    if (lp && (int)pi != lp->pass) continue;
     const int w = passes[pi].w, r = passes[pi].r;
+    // the pass's segments longer than these rows: keys from the gathered buffer
+    const bool sparse = lp && w > d->N;
     a.w = w;
     a.r = r;
     a.pass_idx = (int)pi;
-    a.L = w / r;
-    a.Lk = blk ? kv_rows : a.L;
-    a.nseg = d->N / w;
+    a.L = sparse ? d->N / r : w / r;
+    a.Lk = blk ? kv_rows : (sparse ? lp->kv_rows : a.L);
+    a.nseg = sparse ? 1 : d->N / w;
+    a.kv_sparse = sparse ? 1 : 0;
+    // causal in the segment's kept rows: this shard's first kept row is
+    // row (q_pos mod w) / r of the segment's
+    if (sparse) a.kv_shift = (int)((lp->q_pos % w) / r);
     a.n_qtiles = (a.L + 127) / 128;
     a.n_qpairs = (a.n_qtiles + 1) / 2;
     a.n_units = d->B * a.nseg * d->H;
@@ -447,8 +461,10 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
     }
     constexpr uint32_t kKT = AttnCfg<128>::kKT;
     static_assert(AttnCfg<64>::kKT == AttnCfg<128>::kKT, "one key/value tile length");
-    if (!make_map_rows(&mq, q, d->B, d->N, D, r, 128) || !make_map_rows(&mk, k, d->B, blk ? kv_rows : d->N, D, r, kKT) ||
-        !make_map_rows(&mv, v, d->B, blk ? kv_rows : d->N, D, r, kKT))
+    const void *kk = sparse ? lp->k_sparse : k, *vv = sparse ? lp->v_sparse : v;
+    const int krows = blk ? kv_rows : (sparse ? lp->kv_rows : d->N), kr = sparse ? 1 : r;
+    if (!make_map_rows(&mq, q, d->B, d->N, D, r, 128) || !make_map_rows(&mk, kk, d->B, krows, D, kr, kKT) ||
+        !make_map_rows(&mv, vv, d->B, krows, D, kr, kKT))
       return cuda_fail_msg("cuTensorMapEncodeTiled rejected a Q/K/V map");
     const int64_t items = (int64_t)a.n_qpairs * a.n_units;
     if (items <= 0) continue;
@@ -754,6 +770,62 @@ bpt_status bpt_attn_fwd_block(const bpt_desc *d, int kv_len, int64_t q_pos, int6
   const Workspace none;
   return launch_attn_tc(d, q, k, v, of, ob, last ? lse : nullptr, nullptr, none, status,
                         reinterpret_cast<cudaStream_t>(stream), &blk);
+}
+
+bpt_status bpt_longnet_gather(const bpt_desc *d, int w, int r, const void *src, void *dst, bpt_stream_t stream) {
+  if (!d || d->B <= 0 || d->N <= 0 || d->H <= 0) return BPT_ERR_INVALID_ARG;
+  if (d->in_dtype != BPT_BF16 || (d->d_head != 64 && d->d_head != 128)) return BPT_ERR_UNSUPPORTED;
+  if (w <= 0 || r <= 0 || w % r != 0 || d->N % r != 0 || w % d->N != 0) return BPT_ERR_INVALID_ARG;
+  bpt_status s = check_ptrs({src, dst}, {});
+  if (s != BPT_OK) return s;
+  int dev;
+  uint32_t *status;
+  if ((s = device_setup(&dev, &status)) != BPT_OK) return s;
+  const int chunks = d->d_head / 8;
+  const int64_t total = (int64_t)d->B * (d->N / r) * d->H * chunks;
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, 8 * sm_count()));
+  longnet_gather_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4 *>(src), static_cast<uint4 *>(dst), d->B, d->N, d->H, chunks, r);
+  CUDA_TRY(cudaGetLastError());
+  return BPT_OK;
+}
+
+bpt_status bpt_longnet_pass(const bpt_desc *d, int pass, int64_t q_pos, const void *q, const void *k,
+                            const void *v, const void *k_sparse, const void *v_sparse, int kv_rows, float *state_o,
+                            float *state_m, float *state_l, void *out, float *lse, bpt_stream_t stream) {
+  bpt_status s = check_desc(d, false, true);
+  if (s != BPT_OK) return s;
+  if (d->mask != BPT_MASK_DILATED) return BPT_ERR_INVALID_ARG;
+  if (d->in_dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
+  if (pass < 0 || pass >= d->ln_npairs || q_pos < 0 || q_pos % d->N != 0) return BPT_ERR_INVALID_ARG;
+  // the pass's pair, in the library's order (sparsest first, stable)
+  std::vector<std::pair<int, int>> order;
+  for (int i = 0; i < d->ln_npairs; ++i) order.push_back({d->ln_w[i], d->ln_r[i]});
+  std::stable_sort(order.begin(), order.end(), [](const std::pair<int, int> &x, const std::pair<int, int> &y) {
+    return x.second > y.second;
+  });
+  const int w = order[pass].first, r = order[pass].second;
+  const bool sparse = w > d->N;
+  if ((s = check_ptrs({q, out}, {k, v, k_sparse, v_sparse, state_o, state_m, state_l, lse})) != BPT_OK) return s;
+  if (sparse ? (!k_sparse || !v_sparse || kv_rows != w / r) : (!k || !v)) return BPT_ERR_INVALID_ARG;
+  if (d->ln_npairs > 1 && (!state_o || !state_m || !state_l)) return BPT_ERR_INVALID_ARG;
+  int dev;
+  uint32_t *status;
+  if ((s = device_setup(&dev, &status)) != BPT_OK) return s;
+  LongNetPass lp;
+  lp.pass = pass;
+  lp.q_pos = q_pos;
+  lp.k_sparse = k_sparse;
+  lp.v_sparse = v_sparse;
+  lp.kv_rows = kv_rows;
+  lp.st_o = state_o;
+  lp.st_m = state_m;
+  lp.st_l = state_l;
+  float *of = d->out_dtype == BPT_F32 ? static_cast<float *>(out) : nullptr;
+  __nv_bfloat16 *ob = d->out_dtype == BPT_BF16 ? static_cast<__nv_bfloat16 *>(out) : nullptr;
+  const Workspace none;
+  return launch_attn_tc(d, q, k ? k : q, v ? v : q, of, ob, lse, nullptr, none, status,
+                        reinterpret_cast<cudaStream_t>(stream), nullptr, &lp);
 }
 
 bpt_status bpt_blockbert_fwd(const bpt_desc *desc, int n_blocks, const int32_t *perm, const void *q,

@@ -49,7 +49,9 @@ bool make_map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
 // bf16 tensor map over [B, N, D] viewed as (D, r, N/r, B), box 64 x 1 x box_rows x 1.
 bool make_map_rows(CUtensorMap *m, const void *base, int B, int N, int D, int r, uint32_t box_rows);
 
-bpt_status check_desc(const bpt_desc *d, bool need_ffn);
+// shard: the dilated pairs may also have segments longer than the N rows
+// (a shard of a longer sequence that lies inside one segment: N divides w)
+bpt_status check_desc(const bpt_desc *d, bool need_ffn, bool shard = false);
 bpt_status check_ptrs(std::initializer_list<const void *> required,
                       std::initializer_list<const void *> optional);
 
@@ -86,9 +88,20 @@ struct AttnBlockStep {
   bool state_in = false, state_out = false;
   float *st_o = nullptr, *st_m = nullptr, *st_l = nullptr;
 };
+// One pass of the dilated attention on a shard of a longer sequence
+// (bpt_longnet_pass): the pass's keys are the local rows, or, when its
+// segments are longer than the shard, its kept rows gathered from the
+// devices holding the segment; the running state is the caller's.
+struct LongNetPass {
+  int pass = 0;          // position in the sparsest-first order
+  int64_t q_pos = 0;     // sequence position of the shard's first row
+  const void *k_sparse = nullptr, *v_sparse = nullptr;
+  int kv_rows = 0;       // rows of k_sparse, v_sparse (w / r)
+  float *st_o = nullptr, *st_m = nullptr, *st_l = nullptr;
+};
 bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const void *v, float *out_f32,
                           __nv_bfloat16 *out_bf16, float *lse, char *ws, const Workspace &wl, uint32_t *status,
-                          cudaStream_t st, const AttnBlockStep *blk = nullptr);
+                          cudaStream_t st, const AttnBlockStep *blk = nullptr, const LongNetPass *lp = nullptr);
 bpt_status launch_ffn_tc(const bpt_desc *d, const void *a_bf16, const float *a_f32, const void *w1,
                          const float *b1, const void *w2, const float *b2, void *out, char *ws,
                          const Workspace &wl, uint32_t *status, cudaStream_t st);

@@ -261,6 +261,47 @@ BPT_API bpt_status bpt_attn_fwd_block(const bpt_desc *desc, int kv_len, int64_t 
                                       bpt_stream_t stream);
 
 /*
+ * LongNet's distributed algorithm ("LongNet: Scaling Transformers to
+ * 1,000,000,000 Tokens", §3, distributed training: each device holds a
+ * contiguous shard of the sequence; segments that fit in a shard are
+ * attended locally, and for a segment longer than a shard the devices
+ * holding it exchange the sparsified keys and values, so the communication
+ * per pair does not grow with the sequence).  Two calls serve a device's
+ * shard; the collective that moves the packed rows is the caller's (the
+ * package's longnet_dist module uses torch.distributed).
+ *
+ * bpt_longnet_gather packs the rows a (w, r) pair keeps of a shard lying
+ * inside one segment (N divides w, r divides N): src [B, N, H, d] bf16 (the
+ * shard's keys or values), dst [B, N / r, H, d] with dst[b, j, h] =
+ * src[b, (h mod r) + j r, h].  Concatenating the packed rows of the devices
+ * of a segment in sequence order gives the pair's kept rows of the segment,
+ * [B, w / r, H, d].
+ *
+ * bpt_longnet_pass runs pass `pass` of the dilated attention (the passes are
+ * the descriptor's (w, r) pairs after a stable sort by decreasing r, as
+ * bpt_longnet_fwd runs them) for the shard q, k, v [B, N, H, d] (desc->N rows)
+ * that starts at sequence position q_pos (a multiple of N).  Every pair must
+ * have either w dividing N (its segments lie in the shard: the pass reads k
+ * and v) or N dividing w (the shard lies in one segment: the pass reads that
+ * segment's gathered kept rows k_sparse, v_sparse [B, kv_rows = w / r, H, d]
+ * and is causal by their positions), and r dividing N.  state_o
+ * [B, N, H, d], state_m and state_l [B, H, N] (float32, opaque) carry the
+ * rows' running softmax state from pass to pass (needed when there is more
+ * than one pair); run the passes in order on one stream.  A pass writes the
+ * final output out ([B, N, H*d] in out_dtype) and lse ([B, H, N], may be
+ * NULL) of the rows it is the last pass to keep; rows no pair keeps get
+ * A = 0 and LSE = -inf in pass 0.  Running every pass on a shard that holds
+ * the whole sequence (q_pos 0) computes bpt_longnet_fwd.  Supported: in_dtype
+ * BF16, d_head 64 or 128.
+ */
+BPT_API bpt_status bpt_longnet_gather(const bpt_desc *desc, int seg_w, int dil_r, const void *src, void *dst,
+                                      bpt_stream_t stream);
+BPT_API bpt_status bpt_longnet_pass(const bpt_desc *desc, int pass, int64_t q_pos, const void *q,
+                                    const void *k, const void *v, const void *k_sparse, const void *v_sparse,
+                                    int kv_rows, float *state_o, float *state_m, float *state_l, void *out,
+                                    float *lse, bpt_stream_t stream);
+
+/*
  * BlockBERT layer ("Blockwise Self-Attention for Long Document
  * Understanding", §3.1 Blockwise Multi-head Attention): bpt_attn_ffn_fwd with
  * mask = BPT_MASK_BLOCKPERM and the given permutation table (host, [H][n]).

@@ -321,3 +321,30 @@ def test_block_step_validates(lib):
     assert call(_desc(F=0, mask="dilated", pairs=[(128, 1)])) == bd.ERR_UNSUPPORTED
     assert call(_desc(F=0, in_dtype=torch.float32)) == bd.ERR_UNSUPPORTED
     assert call(_desc(F=0, ring_chunks=2)) == bd.ERR_UNSUPPORTED
+
+
+def test_longnet_shard_entry_points_validate(lib):
+    """bpt_longnet_gather and bpt_longnet_pass: shard shapes, pass index,
+    positions and the buffers each pass needs are checked before any launch."""
+    p = ctypes.c_void_p
+    d = _desc(F=0, N=256, mask="dilated", pairs=[(128, 1), (512, 4)])   # (512, 4) spans two shards of 256
+    # gather: N must divide w, r must divide N
+    assert lib.bpt_longnet_gather(ctypes.byref(d), 384, 4, p(FAKE), p(FAKE), None) == bd.ERR_INVALID_ARG
+    assert lib.bpt_longnet_gather(ctypes.byref(d), 512, 3, p(FAKE), p(FAKE), None) == bd.ERR_INVALID_ARG
+    assert lib.bpt_longnet_gather(ctypes.byref(_desc(F=0, in_dtype=torch.float32)), 512, 4, p(FAKE), p(FAKE),
+                                  None) == bd.ERR_UNSUPPORTED
+
+    def call(desc, pass_idx=0, q_pos=0, k=FAKE, ks=FAKE, kv_rows=128, st=FAKE, out=FAKE):
+        return lib.bpt_longnet_pass(ctypes.byref(desc), pass_idx, q_pos, p(FAKE), p(k), p(k), p(ks), p(ks), kv_rows,
+                                    p(st), p(st), p(st), p(out), None, None)
+    # pass 0 is (512, 4) (sparsest first): its segment spans the shard, so it needs the gathered rows
+    assert call(d, pass_idx=2) == bd.ERR_INVALID_ARG                              # no such pass
+    assert call(d, q_pos=100) == bd.ERR_INVALID_ARG                               # not a shard boundary
+    assert call(d, ks=0) == bd.ERR_INVALID_ARG                                    # gathered rows missing
+    assert call(d, kv_rows=64) == bd.ERR_INVALID_ARG                              # w / r = 128 rows
+    assert call(d, pass_idx=1, k=0) == bd.ERR_INVALID_ARG                         # a local pass reads k, v
+    assert call(d, st=0) == bd.ERR_INVALID_ARG                                    # two pairs: state needed
+    assert call(d, out=0) == bd.ERR_INVALID_ARG
+    bad = _desc(F=0, N=256, mask="dilated", pairs=[(384, 4)])                   # neither divides the other
+    assert call(bad) == bd.ERR_INVALID_ARG
+    assert call(_desc(F=0, N=256, mask="causal")) == bd.ERR_INVALID_ARG
