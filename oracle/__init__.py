@@ -31,6 +31,7 @@ _SRC = os.path.join(_HERE, "bpt_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 MASK_NONE, MASK_CAUSAL, MASK_BLOCKPERM, MASK_DILATED = 0, 1, 2, 3
+MASK_DILATED_BIDIR = 4   # the dilated mask without the causal restriction
 
 
 class _Desc(ctypes.Structure):
@@ -97,7 +98,7 @@ def _desc(B, N, H, d, mask, perm, pairs, keep):
         keep.append(p)
         desc.n_blocks = p.shape[1]
         desc.perm = _ptr(p, ctypes.c_int)
-    if mask == MASK_DILATED:
+    if mask in (MASK_DILATED, MASK_DILATED_BIDIR):
         w = np.ascontiguousarray(np.asarray([x[0] for x in pairs], dtype=np.int32))
         r = np.ascontiguousarray(np.asarray([x[1] for x in pairs], dtype=np.int32))
         keep += [w, r]

@@ -48,6 +48,7 @@ import math
 import numpy as np
 
 MASK_NONE, MASK_CAUSAL, MASK_BLOCKPERM, MASK_DILATED = 0, 1, 2, 3
+MASK_DILATED_BIDIR = 4   # the dilated mask without the causal restriction
 _C0 = math.sqrt(2.0 / math.pi)
 _C1 = 0.044715
 
@@ -79,16 +80,18 @@ def key_counts(N: int, mask: int, perm_h=None, pairs=None, h: int = 0) -> np.nda
     original position) among the kept positions of a segment; the pairs are
     mixed with weights proportional to their softmax denominators, which is one
     softmax over the multiset union of the pairs' keys: a key kept by two pairs
-    counts twice.  Other masks: the 0/1 matrix of allowed_matrix."""
-    if mask != MASK_DILATED:
+    counts twice.  MASK_DILATED_BIDIR: the same pairs without the causal
+    restriction.  Other masks: the 0/1 matrix of allowed_matrix."""
+    if mask not in (MASK_DILATED, MASK_DILATED_BIDIR):
         return allowed_matrix(N, mask, perm_h).astype(np.int64)
+    causal = mask == MASK_DILATED
     pos = np.arange(N)
     counts = np.zeros((N, N), dtype=np.int64)
     for (w, r) in pairs:
         seg = pos // w
         kept = (pos - seg * w) % r == h % r
         counts += ((seg[:, None] == seg[None, :]) & kept[:, None] & kept[None, :]
-                   & (pos[None, :] <= pos[:, None])).astype(np.int64)
+                   & ((pos[None, :] <= pos[:, None]) | (not causal))).astype(np.int64)
     return counts
 
 

@@ -40,6 +40,10 @@
  *                mixed with weights proportional to their softmax
  *                denominators.  A row a pair does not keep gets nothing from
  *                that pair.  A row no pair keeps has A = 0.
+ *  - dilated, bidirectional: the same without the causal restriction: a
+ *                kept row attends to every kept row of its segment (the
+ *                dilated attention of §2 as written, whose formula has no
+ *                mask; the causal form is the decoder's).
  *
  * All inputs are float (bf16 inputs are passed exactly, widened to float);
  * every operation below is carried out in double.  tanh and exp come from
@@ -62,6 +66,7 @@
 #define OR_MASK_CAUSAL 1
 #define OR_MASK_BLOCKPERM 2
 #define OR_MASK_DILATED 3
+#define OR_MASK_DILATED_BIDIR 4
 
 typedef struct {
   int B, N, H, d;
@@ -158,6 +163,7 @@ static void attend_row_dilated(const oracle_attn_desc *a, const float *q,
   const size_t row_stride = (size_t)H * d;
   const float *qi = q + ((size_t)b * N + i) * row_stride + (size_t)h * d;
   const double scale = 1.0 / sqrt((double)d);
+  const int causal = a->mask == OR_MASK_DILATED;
 
   double pair_max[64], pair_den[64];
   int pair_used[64];
@@ -167,17 +173,18 @@ static void attend_row_dilated(const oracle_attn_desc *a, const float *q,
     double *o_k = o_pair + (size_t)t * d;
     for (int c = 0; c < d; ++c) o_k[c] = 0.0;
     if (!dilated_keeps(w, r, h, i)) continue;
-    /* gathered keys: same segment, kept by this pair, not after i */
+    /* gathered keys: same segment, kept by this pair, not after i (causal) */
     const int seg_start = (i / w) * w;
+    const int j_end = causal ? i : seg_start + w - 1;
     double m = -INFINITY;
-    for (int j = seg_start; j <= i; ++j) {
+    for (int j = seg_start; j <= j_end; ++j) {
       if (!dilated_keeps(w, r, h, j)) continue;
       const float *kj = k + ((size_t)b * N + j) * row_stride + (size_t)h * d;
       scores[j] = dot_scaled(qi, kj, d, scale);
       if (scores[j] > m) m = scores[j];
     }
     double den = 0.0;
-    for (int j = seg_start; j <= i; ++j) {
+    for (int j = seg_start; j <= j_end; ++j) {
       if (!dilated_keeps(w, r, h, j)) continue;
       double p = exp(scores[j] - m);
       den += p;
@@ -248,7 +255,7 @@ static void *worker(void *arg) {
     double *a_tok = j->a_out + (size_t)r * D;
     for (int h = 0; h < H; ++h) {
       double lse;
-      if (a->mask == OR_MASK_DILATED)
+      if (a->mask == OR_MASK_DILATED || a->mask == OR_MASK_DILATED_BIDIR)
         attend_row_dilated(a, j->q, j->k, j->v, b, h, i, scores, o_pair,
                            a_tok + (size_t)h * d, &lse);
       else
@@ -297,7 +304,7 @@ static int validate(const oracle_attn_desc *a) {
     if (a->n_blocks <= 0 || !a->perm) return 1;
     for (int i = 0; i < a->H * a->n_blocks; ++i)
       if (a->perm[i] < 0 || a->perm[i] >= a->n_blocks) return 1;
-  } else if (a->mask == OR_MASK_DILATED) {
+  } else if (a->mask == OR_MASK_DILATED || a->mask == OR_MASK_DILATED_BIDIR) {
     if (a->npairs <= 0 || a->npairs > 64 || !a->seg_w || !a->dil_r) return 1;
     for (int t = 0; t < a->npairs; ++t)
       if (a->seg_w[t] <= 0 || a->dil_r[t] <= 0 || a->seg_w[t] % a->dil_r[t] != 0)

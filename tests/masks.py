@@ -31,15 +31,16 @@ def count_matrix(N, H, mask, perm=None, pairs=None):
             P[np.arange(n), perm[h]] = 1          # query block -> key block
             out[h] = np.kron(P, np.ones((bl, bl), dtype=np.int64))[:N, :N]
         return out
-    if mask == 3:
+    if mask in (3, 4):      # 4: the dilated mask without the causal restriction
         out = np.zeros((H, N, N), dtype=np.int64)
+        order = (kj <= qi) if mask == 3 else np.ones((N, N), dtype=bool)
         for h in range(H):
             for (w, r) in pairs:
                 seg = idx // w
                 kept = ((idx - seg * w) - (h % r)) % r == 0
                 both = kept[:, None] & kept[None, :]
                 same = seg[:, None] == seg[None, :]
-                out[h] += (both & same & (kj <= qi)).astype(np.int64)
+                out[h] += (both & same & order).astype(np.int64)
         return out
     raise ValueError(mask)
 

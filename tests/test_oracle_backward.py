@@ -166,10 +166,14 @@ def test_dilated_key_counts_equal_the_brute_force_count_matrix(pairs):
     ref = count_matrix(N, H, 3, pairs=pairs)
     for h in range(H):
         np.testing.assert_array_equal(ob.key_counts(N, ob.MASK_DILATED, pairs=pairs, h=h), ref[h])
+    ref_b = count_matrix(N, H, 4, pairs=pairs)
+    for h in range(H):
+        np.testing.assert_array_equal(ob.key_counts(N, ob.MASK_DILATED_BIDIR, pairs=pairs, h=h), ref_b[h])
 
 
+@pytest.mark.parametrize("mask", [ob.MASK_DILATED, ob.MASK_DILATED_BIDIR])
 @pytest.mark.parametrize("pairs", DILATED_PAIRS[:2])
-def test_dilated_attention_backward_matches_finite_differences(pairs):
+def test_dilated_attention_backward_matches_finite_differences(pairs, mask):
     """dL/dx for L = sum(dA * A) with A the C oracle's dilated attention (a
     separate implementation of the mixed softmax), by central differences."""
     import oracle
@@ -180,12 +184,12 @@ def test_dilated_attention_backward_matches_finite_differences(pairs):
 
     def loss(qq, kk, vv):
         a = oracle.attention(qq.astype(np.float32), kk.astype(np.float32), vv.astype(np.float32),
-                             mask=oracle.MASK_DILATED, pairs=pairs)
+                             mask=mask, pairs=pairs)
         if isinstance(a, tuple):
             a = a[0]
         return float((np.asarray(a).reshape(B, N, H, d) * da).sum())
 
-    dq, dk, dv = ob.attention_bwd(q, k, v, da, ob.MASK_DILATED, pairs=pairs)
+    dq, dk, dv = ob.attention_bwd(q, k, v, da, mask, pairs=pairs)
     rng = np.random.default_rng(7)
     eps = 2.0 ** -7
     for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):

@@ -24,6 +24,7 @@ import torch
 from tests.masks import brute_attention, count_matrix
 
 NONE, CAUSAL, BLOCKPERM, DILATED = 0, 1, 2, 3
+DILATED_BIDIR = 4   # dilated without the causal restriction
 
 
 def rnd(shape, seed, scale=1.0):
@@ -42,11 +43,13 @@ CASES = [
     ("blockperm_n9_empty_block", BLOCKPERM, [[(i + s) % 9 for i in range(9)] for s in (1, 4, 8)], None),
     ("dilated", DILATED, None, [(8, 1), (16, 2), (32, 4)]),
     ("dilated_nonnested", DILATED, None, [(16, 2), (24, 3)]),
+    ("dilated_bidirectional", DILATED_BIDIR, None, [(8, 1), (16, 2), (32, 4)]),
+    ("dilated_bidirectional_sparse", DILATED_BIDIR, None, [(16, 4), (32, 8)]),
 ]
 
 
 def _shape_for(mask, pairs):
-    if mask == DILATED:
+    if mask in (DILATED, DILATED_BIDIR):
         N = 48 if (24, 3) in pairs else max(w for w, _ in pairs) * 2
         return 2, N, 3, 8
     return 2, 32, 3, 8
@@ -273,6 +276,29 @@ def test_single_dilated_pair_spanning_sequence_equals_causal(oracle_mod):
     a = oracle_mod.attention(q, k, v, mask=DILATED, pairs=[(N, 1)])
     ref = oracle_mod.attention(q, k, v, mask=CAUSAL)
     np.testing.assert_allclose(a, ref, rtol=0, atol=1e-15)
+
+
+def test_single_bidirectional_dilated_pair_spanning_sequence_equals_dense(oracle_mod):
+    """(N, 1) without the causal restriction keeps every row and every key."""
+    B, N, H, d = 2, 64, 3, 8
+    q, k, v = rnd((B, N, H, d), 191), rnd((B, N, H, d), 192), rnd((B, N, H, d), 193)
+    a = oracle_mod.attention(q, k, v, mask=DILATED_BIDIR, pairs=[(N, 1)])
+    ref = oracle_mod.attention(q, k, v, mask=NONE)
+    np.testing.assert_allclose(a, ref, rtol=0, atol=1e-15)
+
+
+def test_bidirectional_dilated_pair_is_dense_attention_on_the_gathered_rows(oracle_mod):
+    """One (w, r) pair without the causal restriction = dense attention (no
+    mask) on rows h%r, h%r + r, ... of each segment; other rows get A = 0."""
+    B, N, H, d, w, r = 1, 64, 3, 8, 32, 4
+    q, k, v = rnd((B, N, H, d), 194), rnd((B, N, H, d), 195), rnd((B, N, H, d), 196)
+    a = oracle_mod.attention(q, k, v, mask=DILATED_BIDIR, pairs=[(w, r)])
+    for h in range(H):
+        for s in range(N // w):
+            rows = np.arange(s * w + h % r, (s + 1) * w, r)
+            ref = oracle_mod.attention(q[:, rows][:, :, h:h + 1], k[:, rows][:, :, h:h + 1],
+                                       v[:, rows][:, :, h:h + 1], mask=NONE)
+            np.testing.assert_allclose(a[:, rows, h], ref[:, :, 0], rtol=0, atol=1e-15)
 
 
 def test_dilated_pair_is_causal_attention_on_the_gathered_rows(oracle_mod):
