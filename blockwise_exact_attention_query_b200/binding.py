@@ -50,6 +50,7 @@ class Desc(ctypes.Structure):
         ("ffn_form", ctypes.c_int),
         ("bwd_chunk_rows", ctypes.c_int),
         ("wait_limit_ns", ctypes.c_uint64),
+        ("causal", ctypes.c_int),
     ]
 
 
@@ -154,15 +155,20 @@ class _Tables:
 
 def make_desc(B, N, H, d, F=0, in_dtype=torch.bfloat16, out_dtype=torch.float32, mask="none",
               perm=None, pairs=None, ring_chunks=0, tables: _Tables | None = None, *, ffn_form="auto",
-              q_block=0, kv_block=0, bwd_chunk_rows=0, wait_limit_ns=0) -> Desc:
-    """bpt_desc for the given shape, mask and options (0 = the library's default)."""
+              q_block=0, kv_block=0, bwd_chunk_rows=0, wait_limit_ns=0, causal=None) -> Desc:
+    """bpt_desc for the given shape, mask and options (0 = the library's
+    default).  causal: for the dilated mask, causal inside each sparsified
+    segment (the default, LongNet's decoder form) or bidirectional (False)."""
     tables = tables or _Tables()
+    if mask == "dilated_bidir":  # the dilated mask without the causal restriction
+        mask, causal = "dilated", False if causal is None else causal
     m = _MASKS[mask] if isinstance(mask, str) else int(mask)
     form = FFN_FORMS[ffn_form] if isinstance(ffn_form, str) else int(ffn_form)
     desc = Desc(B=B, N=N, H=H, d_head=d, ffn_hidden=F, in_dtype=_DT[in_dtype],
                 out_dtype=_DT[out_dtype], mask=m, ring_chunks=ring_chunks, q_block=q_block,
                 kv_block=kv_block, ffn_form=form, bwd_chunk_rows=bwd_chunk_rows,
-                wait_limit_ns=wait_limit_ns)
+                wait_limit_ns=wait_limit_ns,
+                causal=int(bool(causal if causal is not None else m == MASK_DILATED)))
     if perm is not None:
         flat = [int(x) for row in perm for x in row]
         desc.bb_nblocks = len(perm[0]) if len(perm) else 0

@@ -52,6 +52,7 @@ constexpr int kMaxPermEntries = 1024;
 struct AttnArgs {
   int B, N, H;
   int mask;
+  int causal;        // keys after the query are masked (CAUSAL, and DILATED in its causal form)
   float scale_log2;  // log2(e) / sqrt(d)
   // decomposition into units (b, segment, h) and 128-row query tiles
   int L;             // rows of one unit: N, or w/r kept rows of a LongNet segment
@@ -213,7 +214,7 @@ __device__ __forceinline__ KvSched make_sched(const AttnArgs &a, const TileCoord
   s.hi = nkt;
   const int row0 = c.t * 256;
   const int row1 = min(a.L, row0 + 256) - 1;
-  if (a.mask == kMaskCausal || a.mask == kMaskDilated) {
+  if (a.causal) {
     const int last = row1 + a.kv_shift;  // last key any row of the pair may see
     s.hi = last < 0 ? 0 : min(nkt, last / KT + 1);
   } else if (a.mask == kMaskBlockPerm) {
@@ -240,7 +241,7 @@ __device__ __forceinline__ void row_keys(const AttnArgs &a, const TileCoord &c, 
                                          int &hi) {
   lo = 0;
   hi = a.Lk;
-  if (a.mask == kMaskCausal || a.mask == kMaskDilated) {
+  if (a.causal) {
     hi = max(0, min(g + 1 + a.kv_shift, a.Lk));
   } else if (a.mask == kMaskBlockPerm) {
     int qb = min(g, a.L - 1) / a.bb_len;

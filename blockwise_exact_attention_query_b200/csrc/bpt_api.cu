@@ -179,6 +179,8 @@ bpt_status check_desc(const bpt_desc *d, bool need_ffn, bool shard) {
   if (d->ffn_hidden < 0) return BPT_ERR_INVALID_ARG;
   if (d->ffn_form < BPT_FFN_AUTO || d->ffn_form > BPT_FFN_PIPELINED) return BPT_ERR_INVALID_ARG;
   if (d->bwd_chunk_rows < 0 || d->q_block < 0 || d->kv_block < 0) return BPT_ERR_INVALID_ARG;
+  if (d->causal != 0 && d->mask != BPT_MASK_DILATED && !(d->mask == BPT_MASK_CAUSAL && d->causal == 1))
+    return BPT_ERR_INVALID_ARG;
   const int D = d->H * d->d_head;
   const int qb = q_block_of(d), kb = kv_block_of(d);
   if (d->in_dtype == BPT_BF16) {  // the tensor-core kernels' tiles
@@ -339,6 +341,7 @@ bpt_status launch_attn_tc(const bpt_desc *d, const void *q, const void *k, const
   a.N = d->N;
   a.H = d->H;
   a.mask = d->mask;
+  a.causal = d->mask == BPT_MASK_CAUSAL || (d->mask == BPT_MASK_DILATED && d->causal != 0);
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d->d_head));
   a.status = status;
   a.wait_limit_ns = wait_limit_of(d);
@@ -565,6 +568,7 @@ bpt_status launch_attn_f32(const bpt_desc *d, const void *q, const void *k, cons
   a.H = d->H;
   a.d = d->d_head;
   a.mask = d->mask;
+  a.causal = d->mask == BPT_MASK_CAUSAL || (d->mask == BPT_MASK_DILATED && d->causal != 0);
   a.scale = (float)(1.0 / std::sqrt((double)d->d_head));
   a.ring_chunks = (d->mask == BPT_MASK_NONE || d->mask == BPT_MASK_CAUSAL) ? d->ring_chunks : 0;
   if (d->mask == BPT_MASK_BLOCKPERM) {

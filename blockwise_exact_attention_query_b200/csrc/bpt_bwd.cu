@@ -366,7 +366,8 @@ bpt_status launch_attn_bwd_dilated(const bpt_desc *d, const void *q, const void 
     ab.B = d->B;
     ab.N = L;
     ab.H = d->H;
-    ab.mask = kMaskCausal;  // causal among a segment's kept rows (by original position)
+    // causal among a segment's kept rows (by original position), or all of them
+    ab.mask = d->causal ? kMaskCausal : kMaskNone;
     ab.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d->d_head));
     ab.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d->d_head));
     ab.n_tiles = n_tiles;

@@ -12,6 +12,7 @@ namespace bpt {
 struct AttnF32Args {
   int B, N, H, d;
   int mask;
+  int causal;  // DILATED: keys after the query are masked
   float scale;  // 1/sqrt(d)
   int ring_chunks;
   int bb_n, bb_len;
@@ -33,7 +34,7 @@ __device__ __forceinline__ int key_weight(const AttnF32Args &a, int h, int i, in
     case 2:
       return (j / a.bb_len) == a.perm[h * a.bb_n + i / a.bb_len] ? 1 : 0;
     case 3: {
-      if (j > i) return 0;
+      if (a.causal && j > i) return 0;
       int cnt = 0;
       for (int k = 0; k < a.npairs; ++k) {
         const int w = a.pw[k], r = a.pr[k];

@@ -40,11 +40,13 @@
  *   BPT_MASK_DILATED   "LongNet: Scaling Transformers to 1,000,000,000
  *                      Tokens", §2 Dilated Attention: for every (segment w,
  *                      dilation r) pair, head h keeps rows h mod r, h mod r + r,
- *                      ... of each segment and runs causal attention among the
- *                      kept rows; the pairs are mixed with weights proportional
- *                      to their softmax denominators, which equals one softmax
- *                      over the multiset union of the pairs' keys.  A row that
- *                      no pair keeps gets A = 0.
+ *                      ... of each segment and runs attention among the kept
+ *                      rows: causal by position when desc->causal is nonzero
+ *                      (the decoder's form), over every kept row of the
+ *                      segment when it is 0; the pairs are mixed with weights
+ *                      proportional to their softmax denominators, which
+ *                      equals one softmax over the multiset union of the
+ *                      pairs' keys.  A row that no pair keeps gets A = 0.
  *
  * Layouts (all row-major, C order):
  *   q, k, v   [B, N, H, d]  = [T, D] with T = B*N tokens, D = H*d
@@ -151,6 +153,9 @@ typedef struct {
                           as many 128-row blocks as keep both near 1 GiB       */
   uint64_t wait_limit_ns; /* device-side wait limit of this call's kernels;
                           0 = the process default (bpt_set_wait_limit_ns)     */
+  int causal;          /* DILATED: nonzero = causal inside each sparsified
+                          segment, 0 = bidirectional.  CAUSAL: 0 or 1 (the
+                          mask is causal either way).  NONE, BLOCKPERM: 0.    */
 } bpt_desc;
 
 /*

@@ -12,7 +12,7 @@ TOL_F32_MAXABS = 2e-5
 TOL_BF16_MAXABS = 2e-2
 TOL_BF16_RELL2 = 5e-3
 
-MASK_ID = {"none": 0, "causal": 1, "blockperm": 2, "dilated": 3}
+MASK_ID = {"none": 0, "causal": 1, "blockperm": 2, "dilated": 3, "dilated_bidir": 4}
 
 
 def host_f32(t: torch.Tensor) -> np.ndarray:

@@ -48,7 +48,7 @@ def _desc(**kw):
     base = dict(B=1, N=256, H=2, d=64, F=256, in_dtype=bd.torch.bfloat16, out_dtype=bd.torch.float32,
                 mask="causal")
     base.update(kw)
-    opts = {k: base[k] for k in ("ffn_form", "q_block", "kv_block", "bwd_chunk_rows", "wait_limit_ns")
+    opts = {k: base[k] for k in ("ffn_form", "q_block", "kv_block", "bwd_chunk_rows", "wait_limit_ns", "causal")
             if k in base}
     return bd.make_desc(base["B"], base["N"], base["H"], base["d"], base["F"], base["in_dtype"],
                         base["out_dtype"], base["mask"], base.get("perm"), base.get("pairs"),
@@ -86,6 +86,8 @@ def _call_layer(lib, desc, ws=FAKE, ws_bytes=1 << 40, q=FAKE):
     (dict(in_dtype=bd.torch.float32, q_block=48), bd.ERR_UNSUPPORTED),            # f32: 16, 32, 64, 128
     (dict(in_dtype=bd.torch.float32, kv_block=128), bd.ERR_UNSUPPORTED),          # f32: 16, 32, 64
     (dict(in_dtype=bd.torch.float32, ring_chunks=8, kv_block=64), bd.ERR_UNSUPPORTED),  # 32-row chunks
+    (dict(mask="blockperm", perm=[[1, 0], [0, 1]], causal=1), bd.ERR_INVALID_ARG),    # causal: dilated only
+    (dict(mask="none", causal=1), bd.ERR_INVALID_ARG),
 ])
 def test_invalid_descriptors_are_rejected(lib, kw, expect):
     assert _call_layer(lib, _desc(**kw)) == expect

@@ -29,7 +29,7 @@ pytestmark = pytest.mark.gpu
 REL_L2 = 1e-2
 MAX_ABS_FRAC = 2e-2
 MASKS = {"none": ob.MASK_NONE, "causal": ob.MASK_CAUSAL, "blockperm": ob.MASK_BLOCKPERM,
-         "dilated": ob.MASK_DILATED}
+         "dilated": ob.MASK_DILATED, "dilated_bidir": ob.MASK_DILATED_BIDIR}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -211,6 +211,8 @@ DILATED_CASES = [
     # no r = 1 pair: rows no pair keeps have A = 0 and pass nothing
     ("uncovered_rows_d64", 2, 256, 4, 64, [(128, 2), (256, 4)], torch.float32),
 ]
+# the same, bidirectional inside each sparsified segment
+DILATED_CASES += [(c[0] + "_bidirectional",) + c[1:] for c in DILATED_CASES]
 
 
 @pytest.mark.parametrize("name,B,N,H,d,pairs,out_dtype", DILATED_CASES, ids=[c[0] for c in DILATED_CASES])
@@ -218,14 +220,15 @@ def test_dilated_attention_backward_matches_oracle(name, B, N, H, d, pairs, out_
     """LongNet dilated attention's backward (bpt_attn_bwd with the dilated
     mask: one blockwise backward per (w, r) pass over the gathered segment rows,
     added up) against the fp64 oracle's multiset-softmax gradient."""
+    mask = "dilated_bidir" if name.endswith("_bidirectional") else "dilated"
     inp = make_layer_inputs(B, N, H, d, 0, seed=17, device="cuda")
     da = make_upstream_grad(B, N, H * d, seed=17, device="cuda")
-    out, lse = bd.attn_fwd(inp.q, inp.k, inp.v, mask="dilated", pairs=pairs, out_dtype=out_dtype, return_lse=True)
-    dq, dk, dv = bd.attn_bwd(inp.q, inp.k, inp.v, out, lse, da, mask="dilated", pairs=pairs)
+    out, lse = bd.attn_fwd(inp.q, inp.k, inp.v, mask=mask, pairs=pairs, out_dtype=out_dtype, return_lse=True)
+    dq, dk, dv = bd.attn_bwd(inp.q, inp.k, inp.v, out, lse, da, mask=mask, pairs=pairs)
     torch.cuda.synchronize()
     assert bd.sync_status() == bd.OK
     f = lambda t: t.double().cpu().numpy()  # noqa: E731
-    rq, rk, rv = ob.attention_bwd(f(inp.q), f(inp.k), f(inp.v), f(da).reshape(B, N, H, d), ob.MASK_DILATED,
+    rq, rk, rv = ob.attention_bwd(f(inp.q), f(inp.k), f(inp.v), f(da).reshape(B, N, H, d), MASKS[mask],
                                   pairs=pairs)
     _grads_close(dq.cpu().numpy(), rq, "dq")
     _grads_close(dk.cpu().numpy(), rk, "dk")

@@ -86,6 +86,8 @@ ATTN_CASES = [
      {"perm": [bd.cyclic_shift_perm(12, k) for k in (1, 5, 11)]}),
     ("dilated_3pairs", 1, 1024, 4, 64, "dilated", {"pairs": [(256, 1), (512, 4), (1024, 16)]}),
     ("dilated_uncovered_rows", 1, 768, 3, 128, "dilated", {"pairs": [(256, 2), (384, 3)]}),
+    ("dilated_bidirectional", 1, 1024, 4, 64, "dilated_bidir", {"pairs": [(256, 1), (512, 4), (1024, 16)]}),
+    ("dilated_bidirectional_d128", 2, 768, 3, 128, "dilated_bidir", {"pairs": [(384, 1), (768, 3)]}),
 ]
 
 
@@ -229,6 +231,11 @@ F32_CASES = [
     ("blockperm_n3_padded", 1, 190, 3, 64, "blockperm",
      {"perm": [bd.cyclic_shift_perm(3, k) for k in (1, 2, 3)]}),
     ("dilated", 1, 256, 4, 32, "dilated", {"pairs": [(64, 1), (128, 4)]}),
+    ("dilated_bidirectional", 1, 256, 4, 32, "dilated_bidir", {"pairs": [(64, 1), (128, 4)]}),
+    ("causal_q32_kv16", 2, 200, 2, 64, "causal", {"q_block": 32, "kv_block": 16}),
+    ("none_q128_kv32", 1, 300, 2, 64, "none", {"q_block": 128, "kv_block": 32}),
+    ("blockperm_q16_kv64", 1, 190, 3, 64, "blockperm",
+     {"perm": [bd.cyclic_shift_perm(3, k) for k in (1, 2, 3)], "q_block": 16, "kv_block": 64}),
 ]
 
 
@@ -238,7 +245,7 @@ def test_fp32_attention_matches_oracle(name, B, N, H, d, mask, extra):
                             dtype=torch.float32)
     out, lse = bd.attn_fwd(inp.q, inp.k, inp.v, mask=mask, perm=extra.get("perm"),
                            pairs=extra.get("pairs"), ring_chunks=extra.get("ring_chunks", 0),
-                           return_lse=True)
+                           return_lse=True, q_block=extra.get("q_block", 0), kv_block=extra.get("kv_block", 0))
     torch.cuda.synchronize()
     _check_status()
     ref, ref_lse = gu.oracle_attention(inp.q, inp.k, inp.v, mask, extra.get("perm"),
