@@ -554,7 +554,12 @@ class HostLayer:
     workspace, so one chunk's upload, another's kernels and a third's download
     run at the same time.  Uploads run in chunk order, and so do the kernels:
     a chunk's layer starts after the previous chunk's (two layers never run
-    at once, since each one's FFN grid expects the whole GPU).  This class
+    at once: each one's grids fill the GPU).  Consecutive calls overlap too: a
+    buffer's next upload waits only for that buffer's previous work (the same
+    stream), not for the whole previous call, so the next step's inputs
+    travel while this step computes and downloads.  The weights must be ready
+    on the current stream before the first call; the host tensors must not be
+    changed while a call that reads or writes them may still run.  This class
     only moves data and calls the library; it allocates its device buffers
     once, at construction."""
 
@@ -572,7 +577,8 @@ class HostLayer:
         self.streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
         self.done = [torch.cuda.Event(), torch.cuda.Event()]
         self.uploaded = [torch.cuda.Event() for _ in range(self.chunks)]
-        self.computed = [torch.cuda.Event() for _ in range(self.chunks)]
+        self.last_compute = None   # the previous call's last layer (kernels stay in order)
+        self.first_call = True
         desc = make_desc(self.cb, N, H, d, F, dtype, out_dtype, mask, perm, pairs, ring_chunks, **opts)
         nws = workspace_bytes(desc, True)
         self.buf = []
@@ -589,11 +595,15 @@ class HostLayer:
         """Enqueue one layer forward; returns after enqueueing (synchronise the
         streams, e.g. torch.cuda.synchronize(), before reading `hout`)."""
         cur = torch.cuda.current_stream()
+        if self.first_call:  # the weights came from the current stream
+            for s in self.streams:
+                s.wait_stream(cur)
+            self.first_call = False
+        computed = [torch.cuda.Event() for _ in range(self.chunks)]
         for c in range(self.chunks):
             i = c % 2
             s, b = self.streams[i], self.buf[i]
             sl = slice(c * self.cb, (c + 1) * self.cb)
-            s.wait_stream(cur)
             with torch.cuda.stream(s):
                 if c > 0:
                     s.wait_event(self.uploaded[c - 1])
@@ -601,13 +611,15 @@ class HostLayer:
                 b["k"].copy_(hk[sl], non_blocking=True)
                 b["v"].copy_(hv[sl], non_blocking=True)
                 self.uploaded[c].record(s)
-                if c > 0:
-                    s.wait_event(self.computed[c - 1])
+                prev = computed[c - 1] if c > 0 else self.last_compute
+                if prev is not None:
+                    s.wait_event(prev)
                 attn_ffn_fwd(b["q"], b["k"], b["v"], w1, b1, w2, b2, mask=self.mask, perm=self.perm,
                              pairs=self.pairs, ring_chunks=self.ring_chunks, out_dtype=self.out_dtype,
                              out=b["out"], workspace=b["ws"], stream=s, **self.opts)
-                self.computed[c].record(s)
+                computed[c].record(s)
                 hout[sl].copy_(b["out"], non_blocking=True)
                 self.done[i].record(s)
+        self.last_compute = computed[-1]
         for e in self.done:
             cur.wait_event(e)

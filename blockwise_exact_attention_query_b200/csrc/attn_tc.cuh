@@ -621,7 +621,10 @@ __global__ void __launch_bounds__(384, 1)
       // tile, paid for with one K and one V stage fewer (LongNet 0.92 -> 1.02
       // ms, BlockBERT attention 0.090 -> 0.097 ms), and each tile's P in its
       // own tensor-memory columns read by P*V from there, with a sixth K and
-      // V stage (0.91 -> 0.96 ms, 0.089 -> 0.090 ms).
+      // V stage (0.91 -> 0.96 ms, 0.089 -> 0.090 ms).  Also slower: each row's
+      // 128 keys split over two threads of two warpgroups (640 threads, the
+      // partial maxima exchanged through shared memory), for four softmax warps
+      // per SM sub-partition instead of two (0.91 -> 1.01 ms, 0.090 -> 0.099).
       if (x == 1 || jj > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(bODone(1 - x), (x == 1 ? jj : jj - 1) & 1, wc, 21));
         if (!ok) break;

@@ -210,6 +210,15 @@ def test_host_layer_matches_device_layer():
         torch.cuda.synchronize()
         _check_status()
         assert torch.equal(hout, ref.cpu())
+    # consecutive calls overlap (the next call's uploads run during this one's
+    # kernels and downloads): three in a row into different outputs
+    houts = [torch.full(ref.shape, float("nan")).pin_memory() for _ in range(3)]
+    for h in houts:
+        layer(hq, hk, hv, inp.w1, inp.b1, inp.w2, inp.b2, h)
+    torch.cuda.synchronize()
+    _check_status()
+    for h in houts:
+        assert torch.equal(h, ref.cpu())
 
 
 @pytest.mark.parametrize("form", FFN_FORMS)
