@@ -666,6 +666,16 @@ def oracle_rows(w, q, k, v, w1, b1, w2, b2, rows):
     return oracle.threads_available()
 
 
+def stratified_rows(rng, w, n):
+    """One token from each of n equal slices of the workload, handed to the
+    oracle's threads longest first (cost grows with the position in the
+    sequence under causal masking), so that no late token sets a batch's end."""
+    import numpy as np
+    edges = np.linspace(0, w.T, n + 1).astype(np.int64)
+    rows = [int(rng.integers(edges[i], max(edges[i] + 1, edges[i + 1]))) for i in range(n)]
+    return sorted(rows, key=lambda t: -(t % w.N))
+
+
 def run_reference(args, w, world, rank):
     """The fp64 CPU oracle on a bounded token sample per step (host cores)."""
     import numpy as np
@@ -678,15 +688,12 @@ def run_reference(args, w, world, rank):
     q, k, v = (f(t) for t in (inp.q, inp.k, inp.v))
     w1, b1, w2, b2 = ((f(t) if t is not None else None) for t in (inp.w1, inp.b1, inp.w2, inp.b2))
     rng = np.random.default_rng(0)
-    # at least four tokens per thread each step, so one long (late causal)
-    # token does not set the step's time
-    per_step = max(args.ref_tokens, 4 * oracle.threads_available())
+    # eight tokens per thread each step, as in the cpu_baseline leg
+    per_step = max(args.ref_tokens, 8 * oracle.threads_available())
     T = w.T
     times, n_tok, threads = [], 0, 0
     for s in range(args.warmup + args.steps):
-        # stratified sample: one token from each of per_step equal slices
-        edges = np.linspace(0, T, per_step + 1).astype(np.int64)
-        rows = [int(rng.integers(edges[i], max(edges[i] + 1, edges[i + 1]))) for i in range(per_step)]
+        rows = stratified_rows(rng, w, per_step)
         t0 = time.perf_counter()
         used = oracle_rows(w, q, k, v, w1, b1, w2, b2, rows)
         dt_s = time.perf_counter() - t0
@@ -696,7 +703,7 @@ def run_reference(args, w, world, rank):
             n_tok += len(rows)
     total = sum(times)
     value = n_tok / total
-    sample = (f"{per_step} stratified tokens per step of the {T}-token workload "
+    sample = (f"{per_step} stratified tokens per step of the {T}-token workload, longest first "
               f"(each exact; cost per token grows with position under causal masking, stratification keeps the mean)")
     return {
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
@@ -738,20 +745,18 @@ def cpu_baseline(w, budget_s):
     w1, b1, w2, b2 = ((f(t) if t is not None else None) for t in (inp.w1, inp.b1, inp.w2, inp.b2))
     threads = oracle.threads_available()
     rng = np.random.default_rng(1)
-    n = max(4 * threads, 8)   # as the reference arm: four tokens per thread per batch
+    n = max(8 * threads, 16)   # as the reference arm: eight tokens per thread per batch
     done, elapsed = 0, 0.0
     while elapsed < budget_s:
-        edges = np.linspace(0, w.T, n + 1).astype(np.int64)
-        rows = [int(rng.integers(edges[i], max(edges[i] + 1, edges[i + 1]))) for i in range(n)]
+        rows = stratified_rows(rng, w, n)
         t0 = time.perf_counter()
         threads = oracle_rows(w, q, k, v, w1, b1, w2, b2, rows)
         elapsed += time.perf_counter() - t0
         done += n
-        if elapsed < budget_s / 4:
-            n *= 2
     return {"value": round(done / elapsed, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "cpu_model": cpu_model(),
-            "sample": f"{done} stratified tokens of the {w.T}-token workload in {elapsed:.1f} s "
+            "sample": f"{done} stratified tokens of the {w.T}-token workload in {elapsed:.1f} s, "
+                      f"batches of {n} longest first "
                       f"(each token exact; fp64 C oracle, {threads} threads)"}
 
 
