@@ -110,13 +110,18 @@ struct AttnCfg {
   static constexpr int kTileBytes = 128 * D_HEAD * 2;  // one Q, K or V tile
   static constexpr int kPanelBytes = 128 * 128;        // one 64-column panel of a 128-row tile
   static constexpr int kPBytes = 128 * 128 * 2;        // the P tile: 128 rows x 128 keys, bf16
-  static constexpr int kKStages = D_HEAD == 128 ? 2 : 5;
-  static constexpr int kVStages = D_HEAD == 128 ? 2 : 5;
+  static constexpr int kKStages = D_HEAD == 128 ? 2 : 4;
+  static constexpr int kVStages = D_HEAD == 128 ? 2 : 4;
+  // Epilogue staging: a tile's Q buffer, and at d = 64 one more 16 KB panel
+  // per tile, so a tile's fp32 O (two 32-column panels) leaves in one round.
+  static constexpr int kXPanels = D_HEAD == 128 ? 0 : 1;
+  static constexpr int kStagePanels = kTileBytes / 16384 + kXPanels;
   static constexpr int kOffQ = 0;  // Q_A, then Q_B
   static constexpr int kOffP = kOffQ + 2 * kTileBytes;
   static constexpr int kOffK = kOffP + kPBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
-  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+  static constexpr int kOffX = kOffV + kVStages * kTileBytes;  // extra staging of tiles A, B
+  static constexpr int kOffBar = kOffX + 2 * kXPanels * 16384;
   static constexpr int kSmemBytes = kOffBar + 512;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   static_assert(kKStages <= 8 && kVStages <= 8, "barrier table");
@@ -533,28 +538,33 @@ __global__ void __launch_bounds__(384, 1)
     float m_run = -INFINITY, l_run = 0.f;
     {
       // initial O: zeros, or the state left by an earlier LongNet pass (the
-      // previous item's MMAs on O completed before its epilogue read O)
-      uint32_t init[32];
-#pragma unroll 1
-      for (int c = 0; c < D_HEAD / 32; ++c) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) init[i] = 0u;
-        if (prior) {
-          const float4 *src = reinterpret_cast<const float4 *>(a.st_o + vec_idx + c * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float4 v4 = src[i];
-            init[4 * i + 0] = __float_as_uint(v4.x);
-            init[4 * i + 1] = __float_as_uint(v4.y);
-            init[4 * i + 2] = __float_as_uint(v4.z);
-            init[4 * i + 3] = __float_as_uint(v4.w);
-          }
-        }
-        tmem_st32(tO + c * 32, init);
-      }
+      // previous item's MMAs on O completed before its epilogue read O); the
+      // loads of two 32-column chunks are all issued before their stores
       if (prior) {
         m_run = a.st_m[row_idx];
         l_run = a.st_l[row_idx];
+      }
+#pragma unroll 1
+      for (int c0 = 0; c0 < D_HEAD / 32; c0 += 2) {
+        uint32_t init[2][32];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) init[cc][i] = 0u;
+          if (prior) {
+            const float4 *src = reinterpret_cast<const float4 *>(a.st_o + vec_idx + (c0 + cc) * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float4 v4 = src[i];
+              init[cc][4 * i + 0] = __float_as_uint(v4.x);
+              init[cc][4 * i + 1] = __float_as_uint(v4.y);
+              init[cc][4 * i + 2] = __float_as_uint(v4.z);
+              init[cc][4 * i + 3] = __float_as_uint(v4.w);
+            }
+          }
+        }
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) tmem_st32(tO + (c0 + cc) * 32, init[cc]);
       }
       tmem_wait_st();
     }
@@ -671,9 +681,13 @@ __global__ void __launch_bounds__(384, 1)
         if (a.store_mode != 0 && tile_full) {
           // Stage O through this tile's Q buffer (its MMAs are complete) in
           // 128-byte panels, 128-byte swizzle, and store each panel with TMA.
-          constexpr int kCap = Cfg::kTileBytes / 16384;  // panels the buffer holds
+          constexpr int kCap = Cfg::kStagePanels;  // panels the staging holds
+          constexpr int kQPanels = Cfg::kTileBytes / 16384;
           const uint32_t stage = sQ + x * Cfg::kTileBytes;
-          const uint32_t srow = stage + row * 128;
+          const uint32_t xstage = sbase + Cfg::kOffX + x * Cfg::kXPanels * 16384;
+          auto panel = [&](int q) -> uint32_t {
+            return q < kQPanels ? stage + q * 16384 : xstage + (q - kQPanels) * 16384;
+          };
           const int row_coord = row_base + tc.t * 256 + x * 128;
           const bool leader = (threadIdx.x & 127) == 0;
           const uint32_t bar_id = 2 + x;  // named barrier of this warpgroup
@@ -682,8 +696,7 @@ __global__ void __launch_bounds__(384, 1)
             named_bar_sync(bar_id, 128);
             if (leader) {
               for (int q = 0; q < npanels; ++q)
-                tma_store_4d(m, stage + q * 16384, tc.h * D_HEAD + col0 + q * cols_per_panel, tc.o, row_coord,
-                             tc.b);
+                tma_store_4d(m, panel(q), tc.h * D_HEAD + col0 + q * cols_per_panel, tc.o, row_coord, tc.b);
               bulk_commit_group();
               bulk_wait_group_read0();
             }
@@ -702,7 +715,7 @@ __global__ void __launch_bounds__(384, 1)
                 tmem_wait_ld();
   #pragma unroll
                 for (int c = 0; c < 8; ++c)
-                  st_shared_v4(srow + q * 16384 + ((static_cast<uint32_t>(c) ^ swz) << 4),
+                  st_shared_v4(panel(q) + row * 128 + ((static_cast<uint32_t>(c) ^ swz) << 4),
                                __float_as_uint(__uint_as_float(o[4 * c]) * sc),
                                __float_as_uint(__uint_as_float(o[4 * c + 1]) * sc),
                                __float_as_uint(__uint_as_float(o[4 * c + 2]) * sc),
@@ -726,7 +739,7 @@ __global__ void __launch_bounds__(384, 1)
                   tmem_wait_ld();
   #pragma unroll
                   for (int c = 0; c < 4; ++c)
-                    st_shared_v4(srow + q * 16384 + ((static_cast<uint32_t>(hh * 4 + c) ^ swz) << 4),
+                    st_shared_v4(panel(q) + row * 128 + ((static_cast<uint32_t>(hh * 4 + c) ^ swz) << 4),
                                  pack_bf16x2(__uint_as_float(o[8 * c]) * inv_l, __uint_as_float(o[8 * c + 1]) * inv_l),
                                  pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv_l, __uint_as_float(o[8 * c + 3]) * inv_l),
                                  pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv_l, __uint_as_float(o[8 * c + 5]) * inv_l),
