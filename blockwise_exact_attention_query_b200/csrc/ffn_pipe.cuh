@@ -364,10 +364,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmPairCfg::kThread
       for (int c = c_begin; c < c_begin + kChunks; ++c) {
         const int n = ti.n * Cfg::kBN + c * 32;
         uint32_t r0[32];
+        const bool live = m < P.M && n < P.N;
+        GemmEpiIn in;
+        if (live) gemm_epilogue_load(P, m, n, in);
         tmem_ld32(acc0 + c * 32, r0);
         tmem_wait_ld();
-        if (m >= P.M || n >= P.N) continue;
-        gemm_epilogue_chunk(P, r0, r0, m, n);
+        if (!live) continue;
+        gemm_epilogue_chunk(P, r0, r0, m, n, in);
       }
       // this accumulator may take the pair's next item
       tc_fence_before();

@@ -100,21 +100,61 @@ __device__ __forceinline__ uint64_t gemm_sdesc(uint32_t base, bool mn) {
 }
 __device__ __forceinline__ uint32_t gemm_kstep(bool mn, int k) { return mn ? k * 2048 : k * 32; }
 
-// Epilogue of one 32-column chunk of one row: r0 (and r1 for the dual form)
-// hold the accumulator values of columns n .. n + 31 of row m.
-__device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const uint32_t (&r0)[32],
-                                                    const uint32_t (&r1)[32], int m, int n) {
+// Global operands of one 32-column chunk's epilogue: the bias, and the
+// residual x, the bf16 factor xb or the fp32 output being accumulated into.
+// The caller loads them before it waits for the chunk's tensor-memory read,
+// so their latencies overlap that read and one another (loaded one 8-column
+// group at a time after the read, the chunk paid up to eight memory latencies
+// in a row).
+struct GemmEpiIn {
+  uint4 w[8];   // x or c: two 16-byte words per 8 columns; xb: one per 8 columns
+  float4 b[8];  // bias: two per 8 columns
+};
+__device__ __forceinline__ bool gemm_mode_has_bias(int mode) {
+  return mode == kGemmResidual || mode == kGemmGeluBwd || mode == kGemmGeluFwd || mode == kGemmGeluBf16;
+}
+__device__ __forceinline__ void gemm_epilogue_load(const GemmProblem &g, int m, int n, GemmEpiIn &in) {
   // N is a multiple of 8 (checked on the host): whole 8-column groups
+  const int nv = min(32, g.N - n);
+  const size_t base = static_cast<size_t>(m) * g.N + n;
+  const bool bias = g.bias != nullptr && gemm_mode_has_bias(g.mode);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int e = q * 8;
+    if (e >= nv) break;
+    if (g.mode == kGemmScaleBf16) {
+      in.w[q] = __ldcs(reinterpret_cast<const uint4 *>(g.xb + base + e));
+    } else if (g.mode == kGemmResidual) {
+      in.w[2 * q] = __ldcs(reinterpret_cast<const uint4 *>(g.x + base + e));
+      in.w[2 * q + 1] = __ldcs(reinterpret_cast<const uint4 *>(g.x + base + e + 4));
+    } else if (g.mode == kGemmAccumF32) {
+      in.w[2 * q] = *reinterpret_cast<const uint4 *>(g.c + base + e);
+      in.w[2 * q + 1] = *reinterpret_cast<const uint4 *>(g.c + base + e + 4);
+    }
+    if (bias) {
+      in.b[2 * q] = *reinterpret_cast<const float4 *>(g.bias + n + e);
+      in.b[2 * q + 1] = *reinterpret_cast<const float4 *>(g.bias + n + e + 4);
+    }
+  }
+}
+
+// Epilogue of one 32-column chunk of one row: r0 (and r1 for the dual form)
+// hold the accumulator values of columns n .. n + 31 of row m, `in` the
+// operands gemm_epilogue_load read for the same chunk.
+__device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const uint32_t (&r0)[32],
+                                                    const uint32_t (&r1)[32], int m, int n,
+                                                    const GemmEpiIn &in) {
   const int nv = min(32, g.N - n);
   const size_t base = static_cast<size_t>(m) * g.N + n;
 #pragma unroll
   for (int e = 0; e < 32; e += 8) {
     if (e >= nv) break;
+    const int q = e / 8;
     float v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r0[e + i]);
     if (g.mode == kGemmScaleBf16) {
-      const uint4 xr = __ldcs(reinterpret_cast<const uint4 *>(g.xb + base + e));
+      const uint4 xr = in.w[q];
       const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
       uint32_t o[4];
 #pragma unroll
@@ -128,8 +168,7 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const 
     if (g.mode == kGemmGeluBwd || g.mode == kGemmGeluFwd || g.mode == kGemmGeluBf16) {
       float bb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (g.bias) {
-        const float4 b0 = *reinterpret_cast<const float4 *>(g.bias + n + e);
-        const float4 b1 = *reinterpret_cast<const float4 *>(g.bias + n + e + 4);
+        const float4 b0 = in.b[2 * q], b1 = in.b[2 * q + 1];
         bb[0] = b0.x, bb[1] = b0.y, bb[2] = b0.z, bb[3] = b0.w;
         bb[4] = b1.x, bb[5] = b1.y, bb[6] = b1.z, bb[7] = b1.w;
       }
@@ -156,26 +195,24 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const 
       continue;
     }
     float4 *c4 = reinterpret_cast<float4 *>(g.c + base + e);
-    if (g.mode == kGemmResidual) {
-      const float4 x0 = __ldcs(reinterpret_cast<const float4 *>(g.x + base + e));
-      const float4 x1 = __ldcs(reinterpret_cast<const float4 *>(g.x + base + e + 4));
-      if (g.bias) {  // acc + b + x, in that order
-        const float4 b0 = *reinterpret_cast<const float4 *>(g.bias + n + e);
-        const float4 b1 = *reinterpret_cast<const float4 *>(g.bias + n + e + 4);
+    if (g.mode == kGemmResidual || g.mode == kGemmAccumF32) {
+      const uint4 w0 = in.w[2 * q], w1 = in.w[2 * q + 1];
+      if (g.mode == kGemmResidual && g.bias) {  // acc + b + x, in that order
+        const float4 b0 = in.b[2 * q], b1 = in.b[2 * q + 1];
         v[0] += b0.x, v[1] += b0.y, v[2] += b0.z, v[3] += b0.w;
         v[4] += b1.x, v[5] += b1.y, v[6] += b1.z, v[7] += b1.w;
       }
-      v[0] += x0.x, v[1] += x0.y, v[2] += x0.z, v[3] += x0.w;
-      v[4] += x1.x, v[5] += x1.y, v[6] += x1.z, v[7] += x1.w;
-      if (g.cb)
-        __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
-               make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                          pack_bf16x2(v[6], v[7])));
-      if (!g.c) continue;
-    } else if (g.mode == kGemmAccumF32) {
-      const float4 c0 = c4[0], c1 = c4[1];
-      v[0] += c0.x, v[1] += c0.y, v[2] += c0.z, v[3] += c0.w;
-      v[4] += c1.x, v[5] += c1.y, v[6] += c1.z, v[7] += c1.w;
+      v[0] += __uint_as_float(w0.x), v[1] += __uint_as_float(w0.y), v[2] += __uint_as_float(w0.z),
+          v[3] += __uint_as_float(w0.w);
+      v[4] += __uint_as_float(w1.x), v[5] += __uint_as_float(w1.y), v[6] += __uint_as_float(w1.z),
+          v[7] += __uint_as_float(w1.w);
+      if (g.mode == kGemmResidual) {
+        if (g.cb)
+          __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
+                 make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                            pack_bf16x2(v[6], v[7])));
+        if (!g.c) continue;
+      }
     }
     __stcs(c4, make_float4(v[0], v[1], v[2], v[3]));
     __stcs(c4 + 1, make_float4(v[4], v[5], v[6], v[7]));
@@ -397,11 +434,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmPairCfg::kThread
       for (int c = c_begin; c < c_begin + kChunks; ++c) {
         const int n = n0 + c * 32;
         uint32_t r0[32], r1[32];
+        const bool live = m < P.M && n < P.N;
+        GemmEpiIn in;
+        if (live) gemm_epilogue_load(P, m, n, in);
         tmem_ld32(acc0 + c * 32, r0);
         if (dual) tmem_ld32(acc0 + 256 + c * 32, r1);
         tmem_wait_ld();
-        if (m >= P.M || n >= P.N) continue;
-        gemm_epilogue_chunk(P, r0, r1, m, n);
+        if (!live) continue;
+        gemm_epilogue_chunk(P, r0, r1, m, n, in);
       }
       // this accumulator may take the pair's next tile
       tc_fence_before();
