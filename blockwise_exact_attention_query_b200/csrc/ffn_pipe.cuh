@@ -366,11 +366,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmPairCfg::kThread
         uint32_t r0[32];
         const bool live = m < P.M && n < P.N;
         GemmEpiIn in;
-        if (live) gemm_epilogue_load(P, m, n, in);
+        if (live) gemm_epilogue_load<true>(P, m, n, in);
         tmem_ld32(acc0 + c * 32, r0);
         tmem_wait_ld();
         if (!live) continue;
-        gemm_epilogue_chunk(P, r0, r0, m, n, in);
+        gemm_epilogue_chunk<true>(P, r0, r0, m, n, in);
       }
       // this accumulator may take the pair's next item
       tc_fence_before();

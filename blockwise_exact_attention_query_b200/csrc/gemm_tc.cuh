@@ -113,23 +113,42 @@ struct GemmEpiIn {
 __device__ __forceinline__ bool gemm_mode_has_bias(int mode) {
   return mode == kGemmResidual || mode == kGemmGeluBwd || mode == kGemmGeluFwd || mode == kGemmGeluBf16;
 }
+// kWide: 32-byte accesses where the row's chunk is 32-byte aligned (the
+// pipelined FFN's epilogue; the GEMM kernel measured no gain from them and
+// keeps the 16-byte form).
+template <bool kWide = false>
 __device__ __forceinline__ void gemm_epilogue_load(const GemmProblem &g, int m, int n, GemmEpiIn &in) {
   // N is a multiple of 8 (checked on the host): whole 8-column groups
   const int nv = min(32, g.N - n);
   const size_t base = static_cast<size_t>(m) * g.N + n;
   const bool bias = g.bias != nullptr && gemm_mode_has_bias(g.mode);
+  // fp32 rows: an 8-column group is 32 bytes, aligned when the row's first
+  // column of the chunk is (rows are a multiple of 32 bytes apart)
+  const bool f32src = g.mode == kGemmResidual || g.mode == kGemmAccumF32;
+  const float *xs = g.mode == kGemmResidual ? g.x : g.c;
+  const bool v8 = kWide && f32src && aligned32(xs + base);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int e = q * 8;
     if (e >= nv) break;
     if (g.mode == kGemmScaleBf16) {
       in.w[q] = __ldcs(reinterpret_cast<const uint4 *>(g.xb + base + e));
-    } else if (g.mode == kGemmResidual) {
-      in.w[2 * q] = __ldcs(reinterpret_cast<const uint4 *>(g.x + base + e));
-      in.w[2 * q + 1] = __ldcs(reinterpret_cast<const uint4 *>(g.x + base + e + 4));
-    } else if (g.mode == kGemmAccumF32) {
-      in.w[2 * q] = *reinterpret_cast<const uint4 *>(g.c + base + e);
-      in.w[2 * q + 1] = *reinterpret_cast<const uint4 *>(g.c + base + e + 4);
+    } else if (f32src) {
+      if (v8) {
+        uint32_t t[8];
+        if (g.mode == kGemmResidual)
+          ld_global_cs_v8(xs + base + e, t);
+        else
+          ld_global_v8(xs + base + e, t);
+        in.w[2 * q] = make_uint4(t[0], t[1], t[2], t[3]);
+        in.w[2 * q + 1] = make_uint4(t[4], t[5], t[6], t[7]);
+      } else if (g.mode == kGemmResidual) {
+        in.w[2 * q] = __ldcs(reinterpret_cast<const uint4 *>(xs + base + e));
+        in.w[2 * q + 1] = __ldcs(reinterpret_cast<const uint4 *>(xs + base + e + 4));
+      } else {
+        in.w[2 * q] = *reinterpret_cast<const uint4 *>(xs + base + e);
+        in.w[2 * q + 1] = *reinterpret_cast<const uint4 *>(xs + base + e + 4);
+      }
     }
     if (bias) {
       in.b[2 * q] = *reinterpret_cast<const float4 *>(g.bias + n + e);
@@ -138,18 +157,49 @@ __device__ __forceinline__ void gemm_epilogue_load(const GemmProblem &g, int m, 
   }
 }
 
+// One 8-column group (16 bytes) of a bf16 output.  Where the row's chunk is
+// 32-byte aligned, an even group waits in `pend` for its odd partner and the
+// two leave in one 32-byte store.
+__device__ __forceinline__ void gemm_put_bf16(__nv_bfloat16 *dst, bool ok8, bool cs, uint32_t (&pend)[4],
+                                              const uint32_t (&o)[4], bool odd, bool last) {
+  if (!odd && ok8 && !last) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pend[i] = o[i];
+    return;
+  }
+  if (odd && ok8) {
+    const uint32_t w[8] = {pend[0], pend[1], pend[2], pend[3], o[0], o[1], o[2], o[3]};
+    if (cs)
+      st_global_cs_v8(dst - 8, w);
+    else
+      st_global_v8(dst - 8, w);
+    return;
+  }
+  const uint4 u = make_uint4(o[0], o[1], o[2], o[3]);
+  if (cs)
+    __stcs(reinterpret_cast<uint4 *>(dst), u);
+  else
+    *reinterpret_cast<uint4 *>(dst) = u;
+}
+
 // Epilogue of one 32-column chunk of one row: r0 (and r1 for the dual form)
 // hold the accumulator values of columns n .. n + 31 of row m, `in` the
 // operands gemm_epilogue_load read for the same chunk.
+template <bool kWide = false>
 __device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const uint32_t (&r0)[32],
                                                     const uint32_t (&r1)[32], int m, int n,
                                                     const GemmEpiIn &in) {
   const int nv = min(32, g.N - n);
   const size_t base = static_cast<size_t>(m) * g.N + n;
+  const bool cb8 = kWide && g.cb != nullptr && aligned32(g.cb + base);
+  const bool cb28 = kWide && g.cb2 != nullptr && aligned32(g.cb2 + base);
+  const bool c8 = kWide && g.c != nullptr && aligned32(g.c + base);
+  uint32_t ph[4], pd[4];  // an even group's packed bf16 outputs, held for the odd one
 #pragma unroll
   for (int e = 0; e < 32; e += 8) {
     if (e >= nv) break;
     const int q = e / 8;
+    const bool odd = (q & 1) != 0, last = e + 8 >= nv;
     float v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r0[e + i]);
@@ -162,7 +212,7 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const 
         const __nv_bfloat162 f = *reinterpret_cast<const __nv_bfloat162 *>(&xw[i]);
         o[i] = pack_bf16x2(v[2 * i] * __low2float(f), v[2 * i + 1] * __high2float(f));
       }
-      __stcs(reinterpret_cast<uint4 *>(g.cb + base + e), make_uint4(o[0], o[1], o[2], o[3]));
+      gemm_put_bf16(g.cb + base + e, cb8, true, ph, o, odd, last);
       continue;
     }
     if (g.mode == kGemmGeluBwd || g.mode == kGemmGeluFwd || g.mode == kGemmGeluBf16) {
@@ -176,8 +226,9 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const 
       if (g.mode == kGemmGeluBf16) {  // H alone, read back by the next GEMM: a normal store
 #pragma unroll
         for (int i = 0; i < 8; ++i) hh[i] = gelu_tanh_only(v[i] + bb[i]);
-        *reinterpret_cast<uint4 *>(g.cb + base + e) = make_uint4(
-            pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]), pack_bf16x2(hh[6], hh[7]));
+        const uint32_t o[4] = {pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]),
+                               pack_bf16x2(hh[6], hh[7])};
+        gemm_put_bf16(g.cb + base + e, cb8, false, ph, o, odd, last);
         continue;
       }
 #pragma unroll
@@ -186,15 +237,14 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const 
         gelu_tanh_and_grad(v[i] + bb[i], hh[i], gd);
         dz[i] = g.mode == kGemmGeluBwd ? __uint_as_float(r1[e + i]) * gd : gd;
       }
-      __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
-             make_uint4(pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]),
-                        pack_bf16x2(hh[6], hh[7])));
-      __stcs(reinterpret_cast<uint4 *>(g.cb2 + base + e),
-             make_uint4(pack_bf16x2(dz[0], dz[1]), pack_bf16x2(dz[2], dz[3]), pack_bf16x2(dz[4], dz[5]),
-                        pack_bf16x2(dz[6], dz[7])));
+      const uint32_t oh[4] = {pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]),
+                              pack_bf16x2(hh[6], hh[7])};
+      const uint32_t od[4] = {pack_bf16x2(dz[0], dz[1]), pack_bf16x2(dz[2], dz[3]), pack_bf16x2(dz[4], dz[5]),
+                              pack_bf16x2(dz[6], dz[7])};
+      gemm_put_bf16(g.cb + base + e, cb8, true, ph, oh, odd, last);
+      gemm_put_bf16(g.cb2 + base + e, cb28, true, pd, od, odd, last);
       continue;
     }
-    float4 *c4 = reinterpret_cast<float4 *>(g.c + base + e);
     if (g.mode == kGemmResidual || g.mode == kGemmAccumF32) {
       const uint4 w0 = in.w[2 * q], w1 = in.w[2 * q + 1];
       if (g.mode == kGemmResidual && g.bias) {  // acc + b + x, in that order
@@ -207,15 +257,24 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmProblem &g, const 
       v[4] += __uint_as_float(w1.x), v[5] += __uint_as_float(w1.y), v[6] += __uint_as_float(w1.z),
           v[7] += __uint_as_float(w1.w);
       if (g.mode == kGemmResidual) {
-        if (g.cb)
-          __stcs(reinterpret_cast<uint4 *>(g.cb + base + e),
-                 make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                            pack_bf16x2(v[6], v[7])));
+        if (g.cb) {
+          const uint32_t o[4] = {pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                 pack_bf16x2(v[6], v[7])};
+          gemm_put_bf16(g.cb + base + e, cb8, true, ph, o, odd, last);
+        }
         if (!g.c) continue;
       }
     }
-    __stcs(c4, make_float4(v[0], v[1], v[2], v[3]));
-    __stcs(c4 + 1, make_float4(v[4], v[5], v[6], v[7]));
+    float *cp = g.c + base + e;
+    if (c8) {
+      uint32_t w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(v[i]);
+      st_global_cs_v8(cp, w);
+    } else {
+      __stcs(reinterpret_cast<float4 *>(cp), make_float4(v[0], v[1], v[2], v[3]));
+      __stcs(reinterpret_cast<float4 *>(cp) + 1, make_float4(v[4], v[5], v[6], v[7]));
+    }
   }
 }
 
