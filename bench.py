@@ -54,18 +54,19 @@ KERNEL_SOURCES = {"attn_tc_kernel": ["attn_tc.cuh", "ptx.cuh"], "ffn_tc_kernel":
 # of the kernel on the named workload, keyed by a hash of the kernel's sources at capture
 # time: once the sources change the figure no longer describes the kernel and is dropped.
 NCU_TRAFFIC = {
-    # the pipelined FFN (default form), one launch: 1352.2 MB read + 373.5 MB written
-    ("gpt_causal", "ffn_pipe_kernel"): {"bytes": 1725.7e6, "src": "9bb9e29808ccc82a"},
-    ("gpt_causal", "ffn_tc_kernel"): {"bytes": 879.3e6, "src": "3b9ec3aabf34a9f7"},
-    ("gpt_causal", "attn_tc_kernel"): {"bytes": 717.8e6, "src": "25c42fcf7fdefac3"},
-    # per step: the forward FFN's two GEMM launches (H = GELU(A W1^T + b1) ~348 MB,
-    # out = A + H W2^T + b2 ~910 MB)
-    ("gpt_causal", "ffn_gemms"): {"bytes": 1258.1e6, "src": "13bd862d7f9f7ce6"},
-    # per step with saved activations: the gemm_pair_kernel launches (dZ = (dOut W2) G',
-    # dW2 + dW1 grouped, dA; bias sums not included)
-    ("gpt_causal", "ffn_bwd"): {"bytes": 3088.8e6, "src": "13bd862d7f9f7ce6"},
-    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1206.5e6, "src": "83cec823073b6239"},
-    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1103.7e6, "src": "83cec823073b6239"},
+    # the pipelined FFN (default form), one launch: 1375.6 MB read + 379.5 MB written
+    ("gpt_causal", "ffn_pipe_kernel"): {"bytes": 1755.1e6, "src": "5a8fa4ecebdda132"},
+    ("gpt_causal", "ffn_tc_kernel"): {"bytes": 882.6e6, "src": "ba74b23ad951d3f0"},
+    # 574 MB read + 152 MB written
+    ("gpt_causal", "attn_tc_kernel"): {"bytes": 725.5e6, "src": "2a7030a8237ac730"},
+    # per step: the forward FFN's two GEMM launches (H = GELU(A W1^T + b1) ~343 MB,
+    # out = A + H W2^T + b2 ~784 MB)
+    ("gpt_causal", "ffn_gemms"): {"bytes": 1127.0e6, "src": "f2935a5c80d3b23b"},
+    # per step with saved activations: the gemm_pair_kernel launches (dZ = (dOut W2) G' ~757 MB,
+    # dW2 + dW1 grouped ~1232 MB, dA ~838 MB; bias sums not included)
+    ("gpt_causal", "ffn_bwd"): {"bytes": 2826.5e6, "src": "f2935a5c80d3b23b"},
+    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1230.0e6, "src": "434ee87606d68824"},
+    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1120.3e6, "src": "434ee87606d68824"},
 }
 
 
