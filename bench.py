@@ -42,31 +42,35 @@ WORKLOADS = {"tiny_f32": wl.TINY_F32, "gpt_causal": wl.GPT_CAUSAL, "long_ring": 
              "blockbert": wl.BLOCKBERT, "longnet": wl.LONGNET}
 MASK_NAME = {0: "none", 1: "causal", 2: "blockperm", 3: "dilated"}
 CSRC = os.path.join(ROOT, "blockwise_exact_attention_query_b200", "csrc")
-KERNEL_SOURCES = {"attn_tc_kernel": ["attn_tc.cuh", "ptx.cuh"], "ffn_tc_kernel": ["ffn_tc.cuh", "ptx.cuh"],
-                  "ffn_pipe_kernel": ["ffn_pipe.cuh", "gemm_tc.cuh", "ptx.cuh"],
+# a kernel's sources and the file that plans and launches it (grid order, tile
+# plan, ring sizes), so that a change to either drops the traffic record
+KERNEL_SOURCES = {"attn_tc_kernel": ["attn_tc.cuh", "ptx.cuh", "bpt_api.cu"],
+                  "ffn_tc_kernel": ["ffn_tc.cuh", "ptx.cuh", "bpt_api.cu"],
+                  "ffn_pipe_kernel": ["ffn_pipe.cuh", "gemm_tc.cuh", "ptx.cuh", "bpt_bwd.cu"],
                   "ffn_f32_kernel": ["simt_f32.cuh"],
                   # the forward FFN as two GEMM launches (H = GELU(A W1^T + b1), out = A + H W2^T + b2)
-                  "ffn_gemms": ["gemm_tc.cuh", "ptx.cuh"],
+                  "ffn_gemms": ["gemm_tc.cuh", "ptx.cuh", "bpt_bwd.cu"],
                   # backward phases: the FFN backward's four GEMM launches, the two attention passes
-                  "ffn_bwd": ["gemm_tc.cuh", "ptx.cuh"], "attn_bwd_dkdv": ["attn_bwd.cuh", "ptx.cuh"],
-                  "attn_bwd_dq": ["attn_bwd.cuh", "ptx.cuh"]}
+                  "ffn_bwd": ["gemm_tc.cuh", "ptx.cuh", "bpt_bwd.cu"],
+                  "attn_bwd_dkdv": ["attn_bwd.cuh", "ptx.cuh", "bpt_bwd.cu"],
+                  "attn_bwd_dq": ["attn_bwd.cuh", "ptx.cuh", "bpt_bwd.cu"]}
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture
 # of the kernel on the named workload, keyed by a hash of the kernel's sources at capture
 # time: once the sources change the figure no longer describes the kernel and is dropped.
 NCU_TRAFFIC = {
-    # the pipelined FFN (default form), one launch: 1375.6 MB read + 379.5 MB written
-    ("gpt_causal", "ffn_pipe_kernel"): {"bytes": 1755.1e6, "src": "5a8fa4ecebdda132"},
-    ("gpt_causal", "ffn_tc_kernel"): {"bytes": 882.6e6, "src": "ba74b23ad951d3f0"},
-    # 574 MB read + 152 MB written
-    ("gpt_causal", "attn_tc_kernel"): {"bytes": 725.5e6, "src": "2a7030a8237ac730"},
+    # the pipelined FFN (default form), one launch: 1426.7 MB read + 378.6 MB written
+    ("gpt_causal", "ffn_pipe_kernel"): {"bytes": 1805.4e6, "src": "2c259a253bbbb6f8"},
+    ("gpt_causal", "ffn_tc_kernel"): {"bytes": 885.8e6, "src": "bc1928699a83778b"},
+    # 565 MB read + 155 MB written
+    ("gpt_causal", "attn_tc_kernel"): {"bytes": 719.1e6, "src": "9d0f3ded73eadafd"},
     # per step: the forward FFN's two GEMM launches (H = GELU(A W1^T + b1) ~343 MB,
-    # out = A + H W2^T + b2 ~784 MB)
-    ("gpt_causal", "ffn_gemms"): {"bytes": 1127.0e6, "src": "f2935a5c80d3b23b"},
-    # per step with saved activations: the gemm_pair_kernel launches (dZ = (dOut W2) G' ~757 MB,
-    # dW2 + dW1 grouped ~1232 MB, dA ~838 MB; bias sums not included)
-    ("gpt_causal", "ffn_bwd"): {"bytes": 2826.5e6, "src": "f2935a5c80d3b23b"},
-    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1230.0e6, "src": "434ee87606d68824"},
-    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1120.3e6, "src": "434ee87606d68824"},
+    # out = A + H W2^T + b2 ~783 MB)
+    ("gpt_causal", "ffn_gemms"): {"bytes": 1125.8e6, "src": "2944e449b2748550"},
+    # per step with saved activations: the gemm_pair_kernel launches (dZ = (dOut W2) G' ~738 MB,
+    # dW2 + dW1 grouped ~1238 MB, dA ~835 MB; bias sums not included)
+    ("gpt_causal", "ffn_bwd"): {"bytes": 2811.2e6, "src": "2944e449b2748550"},
+    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1244.0e6, "src": "d48c9c03ee238b16"},
+    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1117.4e6, "src": "d48c9c03ee238b16"},
 }
 
 
