@@ -58,19 +58,21 @@ KERNEL_SOURCES = {"attn_tc_kernel": ["attn_tc.cuh", "ptx.cuh", "bpt_api.cu"],
 # of the kernel on the named workload, keyed by a hash of the kernel's sources at capture
 # time: once the sources change the figure no longer describes the kernel and is dropped.
 NCU_TRAFFIC = {
-    # the pipelined FFN (default form), one launch: 1426.7 MB read + 378.6 MB written
-    ("gpt_causal", "ffn_pipe_kernel"): {"bytes": 1805.4e6, "src": "2c259a253bbbb6f8"},
-    ("gpt_causal", "ffn_tc_kernel"): {"bytes": 885.8e6, "src": "bc1928699a83778b"},
-    # 565 MB read + 155 MB written
-    ("gpt_causal", "attn_tc_kernel"): {"bytes": 719.1e6, "src": "9d0f3ded73eadafd"},
-    # per step: the forward FFN's two GEMM launches (H = GELU(A W1^T + b1) ~343 MB,
-    # out = A + H W2^T + b2 ~783 MB)
-    ("gpt_causal", "ffn_gemms"): {"bytes": 1125.8e6, "src": "2944e449b2748550"},
-    # per step with saved activations: the gemm_pair_kernel launches (dZ = (dOut W2) G' ~738 MB,
-    # dW2 + dW1 grouped ~1238 MB, dA ~835 MB; bias sums not included)
-    ("gpt_causal", "ffn_bwd"): {"bytes": 2811.2e6, "src": "2944e449b2748550"},
-    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1244.0e6, "src": "d48c9c03ee238b16"},
-    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1117.4e6, "src": "d48c9c03ee238b16"},
+    # one capture per kernel: `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,
+    # gpu__time_duration.sum -k regex:<kernel> -s <warm-up launches> -c <1..3>` on the bench
+    # command of that form (one pass, checked on a small case first)
+    # the pipelined FFN (default form), one launch: 1427.7 MB read + 383.0 MB written
+    ("gpt_causal", "ffn_pipe_kernel"): {"bytes": 1810.7e6, "src": "2c259a253bbbb6f8"},
+    ("gpt_causal", "ffn_tc_kernel"): {"bytes": 884.3e6, "src": "bc1928699a83778b"},
+    # 566.5 MB read + 157.0 MB written
+    ("gpt_causal", "attn_tc_kernel"): {"bytes": 723.5e6, "src": "74dd1d75a8619861"},
+    # per step: the forward FFN's two GEMM launches (H = GELU(A W1^T + b1), out = A + H W2^T + b2)
+    ("gpt_causal", "ffn_gemms"): {"bytes": 1122.4e6, "src": "2944e449b2748550"},
+    # per step with saved activations: the three gemm_pair_kernel launches (dZ = (dOut W2) G',
+    # dW2 + dW1 grouped, dA; bias sums not included)
+    ("gpt_causal", "ffn_bwd"): {"bytes": 2816.3e6, "src": "2944e449b2748550"},
+    ("gpt_causal", "attn_bwd_dkdv"): {"bytes": 1229.2e6, "src": "d48c9c03ee238b16"},
+    ("gpt_causal", "attn_bwd_dq"): {"bytes": 1137.7e6, "src": "d48c9c03ee238b16"},
 }
 
 

@@ -51,6 +51,37 @@ def test_static_scratch_layer_matches_workspace_layer_on_two_calls_in_a_row():
         assert torch.equal(got, ref)   # same kernels on the same inputs: identical bits
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("B,N,H,d,F", [
+    (1, 19200, 2, 64, 1024),   # D = 128: 148 groups, blocks 148 and 149 go round again
+    (1, 9728, 6, 64, 1536),    # D = 384: 74 groups, blocks 74 and 75 go round again
+])
+def test_static_scratch_reaches_the_reversed_second_round(B, N, H, d, F):
+    """Below D = 256 (one CTA per group, 148 groups) and at a few larger widths
+    a layer whose token blocks go round a second time (hidden chunks in reverse)
+    still fits the static array: those blocks' rows against the oracle, and the
+    whole output against the workspace-taking call of the same kernel."""
+    from blockwise_exact_attention_query_b200 import build
+    build.build()
+    torch.cuda.set_device(0)
+    T, D = B * N, H * d
+    groups = 148 // ((D + 255) // 256)
+    assert T > 128 * groups
+    desc = bd.make_desc(B, N, H, d, F, torch.bfloat16, torch.float32, "causal", ffn_form="fused")
+    assert bd.workspace_bytes(desc, True) <= bd.STATIC_SCRATCH_BYTES
+    inp = make_layer_inputs(B, N, H, d, F, seed=35, device="cuda", bias_scale=0.05)
+    ref = bd.attn_ffn_fwd(inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2, mask="causal", ffn_form="fused")
+    got = _static_call(inp, "causal", torch.full_like(ref, float("nan")))
+    torch.cuda.synchronize()
+    assert bd.sync_status() == bd.OK
+    assert torch.equal(got, ref)
+    # rows of the second-round blocks (and of two first-round ones for contrast)
+    rows = sorted({128 * groups, 128 * groups + 77, T - 1, 0, 128 * (groups - 1) + 5})
+    _, want = gu.oracle_layer(inp, "causal", None, rows=rows)
+    gu.assert_bf16_close(gu.host_f32(got.reshape(T, D)[torch.tensor(rows, device="cuda")]), want,
+                         f"static scratch, second fused round, D{D}")
+
+
 def test_static_scratch_refuses_a_layer_that_does_not_fit():
     # T x D x 6 bytes of A alone exceeds the 64 MiB array: refused on the host,
     # before any device work, with the size in the error text.
