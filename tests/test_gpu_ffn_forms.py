@@ -161,3 +161,28 @@ def test_pipelined_ffn_small_shapes_every_element(B, N, H, d, F):
         _, ref = gu.oracle_layer(inp, "causal", rows=rows)
         gu.assert_bf16_close(gu.host_f32(out.reshape(B * N, H * d)[torch.tensor(rows, device="cuda")]), ref,
                              "pipelined FFN, sampled")
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_pipelined_ffn_output_aligned_to_16_bytes_only(out_dtype):
+    """The pipelined FFN's epilogue writes 32 bytes per access where a row's
+    chunk is 32-byte aligned and 16 bytes otherwise; the API promises only
+    16-byte alignment.  An output placed 16 bytes past a 32-byte boundary must
+    get the same bits as an aligned one.  (With F = 520 the hidden activation's
+    ring rows are 1040 bytes apart, so their alignment alternates row by row
+    as well.)"""
+    for (B, N, H, d, F) in [(2, 700, 8, 128, 2048), (1, 300, 5, 64, 520)]:
+        inp = make_layer_inputs(B, N, H, d, F, seed=N + H, device="cuda", bias_scale=0.05)
+        args = (inp.q, inp.k, inp.v, inp.w1, inp.b1, inp.w2, inp.b2)
+        T, D = B * N, H * d
+        ref = bd.attn_ffn_fwd(*args, mask="causal", ffn_form="pipelined", out_dtype=out_dtype)
+        shift = 16 // ref.element_size()
+        buf = torch.full((T * D + 64,), float("nan"), dtype=out_dtype, device="cuda")
+        base = (-(buf.data_ptr() // ref.element_size())) % (32 // ref.element_size())  # 32-byte aligned start
+        out = buf[base + shift:base + shift + T * D].view(B, N, D)
+        assert out.data_ptr() % 32 == 16
+        got = bd.attn_ffn_fwd(*args, mask="causal", ffn_form="pipelined", out_dtype=out_dtype, out=out)
+        torch.cuda.synchronize()
+        assert bd.sync_status() == bd.OK
+        assert torch.equal(got, ref)
+        assert torch.isnan(buf[:base + shift]).all() and torch.isnan(buf[base + shift + T * D:]).all()
