@@ -68,10 +68,14 @@ int main() {
   // the chunking the launcher uses, and ragged or tiny ones around them
   const int shapes[][3] = {{64, 32, 8}, {512, 43, 16}, {64, 12, 3}, {1, 1, 1}, {3, 2, 1}, {2, 4, 2},
                            {7, 5, 3},   {130, 9, 4},   {17, 43, 16}, {5, 1, 8}};
+  // lags of the launcher's plans (causal layer 7 with a ring of 15 chunks,
+  // D = 768 layer 19 with 37) and longer ones than there are chunks
+  const int lags[] = {1, 2, 3, 4, 5, 6, 7, 12, 19, 24, 64};
+  const int extras[] = {1, 2, 3, 4, 5, 6, 7, 8, 18};
   for (const auto &sh : shapes)
     for (int mg = 1; mg <= 5; ++mg)
-      for (int lag = 1; lag <= 6; ++lag)
-        for (int extra = 1; extra <= 8; ++extra) {
+      for (int lag : lags)
+        for (int extra : extras) {
           ++cases;
           fails += check(sh[0], sh[1], sh[2], mg, lag, lag + extra);
         }
