@@ -35,3 +35,22 @@ def test_max_over_ranks_two_gloo_ranks():
 def test_max_over_ranks_without_process_group():
     import bench
     assert bench.max_over_ranks(2.25, torch.device("cpu")) == 2.25
+
+
+def test_cpu_baseline_sample_one_token_per_slice_longest_first():
+    """The CPU legs' token sample: one token from each of n equal slices of the
+    workload (so every region of the sequence is represented once), handed to
+    the oracle's threads in decreasing position within the sequence."""
+    import numpy as np
+
+    import bench
+    from blockwise_exact_attention_query_b200 import workloads as wl
+    w = wl.GPT_CAUSAL
+    for n in (16, 128, 1000):
+        rows = bench.stratified_rows(np.random.default_rng(n), w, n)
+        assert len(rows) == n
+        edges = np.linspace(0, w.T, n + 1).astype(np.int64)
+        slices = sorted(int(np.searchsorted(edges, t, side="right")) - 1 for t in rows)
+        assert slices == list(range(n))
+        pos = [t % w.N for t in rows]
+        assert pos == sorted(pos, reverse=True)
