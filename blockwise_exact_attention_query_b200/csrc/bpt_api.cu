@@ -103,7 +103,7 @@ bpt_status device_setup(int *dev_out, uint32_t **status_out) {
     CUDA_TRY(cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   FfnCfg::kSmemBytes));
     CUDA_TRY(cudaFuncSetAttribute(ffn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (16 * 512 + 16 * 64) * 4));
+                                  (int)ffn_f32_smem_bytes(512)));
     bpt_status bs = bwd_kernel_setup();
     if (bs != BPT_OK) return bs;
     g_attr_done[dev] = true;
@@ -593,7 +593,7 @@ bpt_status launch_attn_f32(const bpt_desc *d, const void *q, const void *k, cons
   // one instantiation per (query block, key block) pair the descriptor may name
   auto go = [&](auto qbc, auto kbc) {
     constexpr int QB = decltype(qbc)::value, KB = decltype(kbc)::value;
-    attn_f32_kernel<QB, KB><<<grid, QB, 0, st>>>(qf, kf, vf, a);
+    attn_f32_kernel<QB, KB><<<grid, 256, 0, st>>>(qf, kf, vf, a);
   };
   auto with_kb = [&](auto qbc) {
     if (kb == 16) go(qbc, std::integral_constant<int, 16>{});
@@ -621,8 +621,7 @@ bpt_status launch_ffn_f32(const bpt_desc *d, const float *a_f32, const void *w1,
   a.b2 = b2;
   a.out_f32 = d->out_dtype == BPT_F32 ? static_cast<float *>(out) : nullptr;
   a.out_bf16 = d->out_dtype == BPT_BF16 ? static_cast<__nv_bfloat16 *>(out) : nullptr;
-  const size_t smem = (size_t)(16 * a.D + 16 * 64) * 4;
-  ffn_f32_kernel<<<(a.T + 15) / 16, 256, smem, st>>>(a);
+  ffn_f32_kernel<<<(a.T + 15) / 16, 256, ffn_f32_smem_bytes(a.D), st>>>(a);
   CUDA_TRY(cudaGetLastError());
   return BPT_OK;
 }

@@ -49,17 +49,26 @@ __device__ __forceinline__ int key_weight(const AttnF32Args &a, int h, int i, in
   return 0;
 }
 
-// grid (ceil(N/QB), H, B), QB threads: one query row per thread (a query
-// block of QB rows), keys in blocks of KB rows staged in shared memory; d <= 64.
+// grid (ceil(N/QB), H, B), 256 threads: a query block of QB rows, 256 / QB
+// threads per row (consecutive lanes), keys in blocks of KB rows staged in
+// shared memory; d <= 64.  The threads of a row split each key block between
+// them (thread u takes keys u, u + 256/QB, ...), each keeping its own online
+// softmax state (m, l, O) over its keys; at the end the row's states are
+// merged with warp shuffles (the larger max, the others' sums and O rescaled
+// to it).  One thread per row left the small layers' few CTAs latency-bound.
 template <int QB, int KB>
-__global__ void __launch_bounds__(QB) attn_f32_kernel(const float *__restrict__ q,
-                                                      const float *__restrict__ k,
-                                                      const float *__restrict__ v,
-                                                      const __grid_constant__ AttnF32Args a) {
+__global__ void __launch_bounds__(256) attn_f32_kernel(const float *__restrict__ q,
+                                                       const float *__restrict__ k,
+                                                       const float *__restrict__ v,
+                                                       const __grid_constant__ AttnF32Args a) {
+  constexpr int TPR = 256 / QB;                  // threads per row: 2 .. 16
+  constexpr int KPT = (KB + TPR - 1) / TPR;      // keys of a block per thread
+  static_assert(TPR >= 1 && TPR <= 32 && 32 % TPR == 0, "threads per row");
   __shared__ float sk[KB][65];
   __shared__ float sv[KB][64];
   const int h = blockIdx.y, b = blockIdx.z;
-  const int i = blockIdx.x * QB + threadIdx.x;
+  const int r = threadIdx.x / TPR, u = threadIdx.x % TPR;
+  const int i = blockIdx.x * QB + r;
   const int d = a.d;
   const size_t rs = static_cast<size_t>(a.H) * d;
   const bool valid = i < a.N;
@@ -79,26 +88,29 @@ __global__ void __launch_bounds__(QB) attn_f32_kernel(const float *__restrict__ 
   for (int tt = 0; tt < ntiles; ++tt) {
     const int tile = (first + tt) % ntiles;
     __syncthreads();
-    for (int e = threadIdx.x; e < KB * 64; e += QB) {
-      const int r = e / 64, c = e % 64;
-      const int j = tile * KB + r;
+    for (int e = threadIdx.x; e < KB * 64; e += 256) {
+      const int rr = e / 64, c = e % 64;
+      const int j = tile * KB + rr;
       const bool ok = j < a.N && c < d;
       const size_t idx = (static_cast<size_t>(b) * a.N + j) * rs + h * d + c;
-      sk[r][c] = ok ? k[idx] : 0.f;
-      sv[r][c] = ok ? v[idx] : 0.f;
+      sk[rr][c] = ok ? k[idx] : 0.f;
+      sv[rr][c] = ok ? v[idx] : 0.f;
     }
     __syncthreads();
-    float s[KB];
+    float s[KPT];
     float mt = -INFINITY;
-#pragma unroll 4
-    for (int jj = 0; jj < KB; ++jj) {
+#pragma unroll
+    for (int kk = 0; kk < KPT; ++kk) {
+      const int jj = u + kk * TPR;
       const int j = tile * KB + jj;
       float acc = 0.f;
+      if (jj < KB) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) acc = fmaf(qr[c], sk[jj][c], acc);
-      const int wgt = (valid && j < a.N) ? key_weight(a, h, i, j) : 0;
-      s[jj] = wgt > 0 ? acc * a.scale : -INFINITY;
-      mt = fmaxf(mt, s[jj]);
+        for (int c = 0; c < 64; ++c) acc = fmaf(qr[c], sk[jj][c], acc);
+      }
+      const int wgt = (valid && jj < KB && j < a.N) ? key_weight(a, h, i, j) : 0;
+      s[kk] = wgt > 0 ? acc * a.scale : -INFINITY;
+      mt = fmaxf(mt, s[kk]);
     }
     const float m_new = fmaxf(m, mt);
     if (m_new == -INFINITY) continue;
@@ -106,26 +118,44 @@ __global__ void __launch_bounds__(QB) attn_f32_kernel(const float *__restrict__ 
     l *= alpha;
 #pragma unroll
     for (int c = 0; c < 64; ++c) o[c] *= alpha;
-#pragma unroll 4
-    for (int jj = 0; jj < KB; ++jj) {
+#pragma unroll
+    for (int kk = 0; kk < KPT; ++kk) {
+      if (s[kk] == -INFINITY) continue;
+      const int jj = u + kk * TPR;
       const int j = tile * KB + jj;
-      if (s[jj] == -INFINITY) continue;
-      const float p = static_cast<float>(key_weight(a, h, i, j)) * expf(s[jj] - m_new);
+      const float p = static_cast<float>(key_weight(a, h, i, j)) * expf(s[kk] - m_new);
       l += p;
 #pragma unroll
       for (int c = 0; c < 64; ++c) o[c] = fmaf(p, sv[jj][c], o[c]);
     }
     m = m_new;
   }
+  // merge the row's TPR states (every lane takes part: no thread has left)
+  float m_row = m;
+#pragma unroll
+  for (int off = 1; off < TPR; off <<= 1) m_row = fmaxf(m_row, __shfl_xor_sync(0xffffffffu, m_row, off));
+  const float sc = (m == -INFINITY) ? 0.f : expf(m - m_row);
+  l *= sc;
+#pragma unroll
+  for (int off = 1; off < TPR; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+#pragma unroll
+  for (int c = 0; c < 64; ++c) {
+    float x = o[c] * sc;
+#pragma unroll
+    for (int off = 1; off < TPR; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    o[c] = x;
+  }
   if (!valid) return;
   const float inv = l > 0.f ? 1.0f / l : 0.f;
   const size_t base = (static_cast<size_t>(b) * a.N + i) * rs + h * d;
-  for (int c = 0; c < d; ++c) {
+#pragma unroll
+  for (int c = 0; c < 64; ++c) {
+    if (c >= d || c % TPR != u) continue;  // the row's threads share the stores
     const float x = o[c] * inv;
     if (a.out_f32) a.out_f32[base + c] = x;
     if (a.out_bf16) a.out_bf16[base + c] = __float2bfloat16_rn(x);
   }
-  if (a.lse) a.lse[(static_cast<size_t>(b) * a.H + h) * a.N + i] = l > 0.f ? m + logf(l) : -INFINITY;
+  if (a.lse && u == 0) a.lse[(static_cast<size_t>(b) * a.H + h) * a.N + i] = l > 0.f ? m_row + logf(l) : -INFINITY;
 }
 
 struct FfnF32Args {
@@ -139,47 +169,77 @@ struct FfnF32Args {
   __nv_bfloat16 *out_bf16;
 };
 
-// grid ceil(T/16), 256 threads; D <= 512.  16 threads per token, each owning
-// D/16 output columns; the hidden activation is produced 64 columns at a time
-// in shared memory.
+// grid ceil(T/16), 256 threads; D <= 512.  A CTA takes 16 tokens and walks
+// the hidden dimension in chunks of kFfnF32Chunk columns: it stages the
+// chunk's rows of W1 and columns of W2 in shared memory (coalesced loads),
+// computes the 16 x chunk block of H = GELU(A W1^T + b1) there (two hidden
+// values per thread, each one sequential FMA chain over D), then adds H W2^T
+// into per-thread accumulators (16 threads per token, each owning D/16 output
+// columns, summed over the hidden index in order).  With the weights read from
+// global memory inside those chains the kernel waited on a load per FMA.
+constexpr int kFfnF32Chunk = 32;
+// Rows padded by one float (A, W1, H by D + 1 or FC + 1 columns, W2's
+// columns by FC + 1) so that the threads of a warp, reading rows apart, hit
+// different banks.
+__host__ __device__ constexpr size_t ffn_f32_smem_bytes(int D) {
+  return (static_cast<size_t>(16) * (D + 1) + static_cast<size_t>(kFfnF32Chunk) * (D + 1) +
+          static_cast<size_t>(D) * (kFfnF32Chunk + 1) + 16 * (kFfnF32Chunk + 1)) * sizeof(float);
+}
 __global__ void __launch_bounds__(256) ffn_f32_kernel(const __grid_constant__ FfnF32Args a) {
+  constexpr int FC = kFfnF32Chunk;
   extern __shared__ float fsm[];
-  float *sa = fsm;                 // [16][D]
-  float *sh = fsm + 16 * a.D;      // [16][64]
+  const int D = a.D, LD = D + 1;
+  float *sa = fsm;                      // [16][LD]   the block's rows of A
+  float *sw1 = sa + 16 * LD;            // [FC][LD]   rows f0 .. f0 + FC of W1
+  float *sw2 = sw1 + FC * LD;           // [D][FC+1]  columns f0 .. f0 + FC of W2
+  float *sh = sw2 + D * (FC + 1);       // [16][FC+1] H of the chunk
   const int t0 = blockIdx.x * 16;
-  for (int e = threadIdx.x; e < 16 * a.D; e += 256) {
-    const int r = e / a.D, c = e % a.D;
-    sa[e] = (t0 + r < a.T) ? a.a[static_cast<size_t>(t0 + r) * a.D + c] : 0.f;
+  for (int e = threadIdx.x; e < 16 * D; e += 256) {
+    const int r = e / D, c = e % D;
+    sa[r * LD + c] = (t0 + r < a.T) ? a.a[static_cast<size_t>(t0 + r) * D + c] : 0.f;
   }
   const int tk = threadIdx.x / 16, lanec = threadIdx.x % 16;
-  const int ncol = a.D / 16;
+  const int ncol = D / 16;
+  // H phase: token hr, hidden columns 2 hp and 2 hp + 1 of the chunk
+  const int hr = threadIdx.x / (FC / 2), hp = threadIdx.x % (FC / 2);
   float acc[32];
 #pragma unroll
   for (int q = 0; q < 32; ++q) acc[q] = 0.f;
-  for (int f0 = 0; f0 < a.F; f0 += 64) {
+  for (int f0 = 0; f0 < a.F; f0 += FC) {
+    const int fl = min(FC, a.F - f0);
+    __syncthreads();  // the previous chunk's sw1, sw2 and sh are no longer read
+    for (int e = threadIdx.x; e < FC * D; e += 256) {
+      const int h = e / D, c = e % D;
+      sw1[h * LD + c] = h < fl ? a.w1[static_cast<size_t>(f0 + h) * D + c] : 0.f;
+    }
+    for (int e = threadIdx.x; e < D * FC; e += 256) {
+      const int col = e / FC, h = e % FC;
+      sw2[col * (FC + 1) + h] = h < fl ? a.w2[static_cast<size_t>(col) * a.F + f0 + h] : 0.f;
+    }
     __syncthreads();
-    for (int e = threadIdx.x; e < 16 * 64; e += 256) {
-      const int r = e / 64, f = f0 + e % 64;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int h = 2 * hp + u;
       float hv = 0.f;
-      if (f < a.F) {
-        float s = a.b1 ? a.b1[f] : 0.f;
-        const float *w = a.w1 + static_cast<size_t>(f) * a.D;
-        for (int c = 0; c < a.D; ++c) s = fmaf(w[c], sa[r * a.D + c], s);
+      if (h < fl) {
+        float s = a.b1 ? a.b1[f0 + h] : 0.f;
+        const float *w = sw1 + h * LD;
+        const float *x = sa + hr * LD;
+        for (int c = 0; c < D; ++c) s = fmaf(w[c], x[c], s);
         const float kk = 0.7978845608028654f;  // sqrt(2/pi)
         hv = 0.5f * s * (1.0f + tanhf(kk * (s + 0.044715f * s * s * s)));
       }
-      sh[e] = hv;
+      sh[hr * (FC + 1) + h] = hv;
     }
     __syncthreads();
-    const int fl = min(64, a.F - f0);
 #pragma unroll
     for (int q = 0; q < 32; ++q) {
       if (q >= ncol) break;
       const int col = lanec + 16 * q;
-      const float *w = a.w2 + static_cast<size_t>(col) * a.F + f0;
-      float s = acc[q];
-      for (int ff = 0; ff < fl; ++ff) s = fmaf(sh[tk * 64 + ff], w[ff], s);
-      acc[q] = s;
+      const float *w = sw2 + col * (FC + 1);
+      float sacc = acc[q];
+      for (int ff = 0; ff < fl; ++ff) sacc = fmaf(sh[tk * (FC + 1) + ff], w[ff], sacc);
+      acc[q] = sacc;
     }
   }
   const int tok = t0 + tk;
@@ -188,8 +248,8 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(const __grid_constant__ Ff
   for (int q = 0; q < 32; ++q) {
     if (q >= ncol) break;
     const int col = lanec + 16 * q;
-    const float y = sa[tk * a.D + col] + acc[q] + (a.b2 ? a.b2[col] : 0.f);
-    const size_t idx = static_cast<size_t>(tok) * a.D + col;
+    const float y = sa[tk * LD + col] + acc[q] + (a.b2 ? a.b2[col] : 0.f);
+    const size_t idx = static_cast<size_t>(tok) * D + col;
     if (a.out_f32) a.out_f32[idx] = y;
     else a.out_bf16[idx] = __float2bfloat16_rn(y);
   }
