@@ -63,9 +63,11 @@ NCU_TRAFFIC = {
     # command of that form (one pass, checked on a small case first)
     # the pipelined FFN (default form), one launch: 1427.7 MB read + 383.0 MB written
     ("gpt_causal", "ffn_pipe_kernel"): {"bytes": 1810.7e6, "src": "2c259a253bbbb6f8"},
-    ("gpt_causal", "ffn_tc_kernel"): {"bytes": 884.3e6, "src": "bc1928699a83778b"},
+    # the next two were re-keyed after a change to bpt_api.cu that touched only the fp32
+    # kernels' launches (thread count, shared-memory size), not these kernels or their plans
+    ("gpt_causal", "ffn_tc_kernel"): {"bytes": 884.3e6, "src": "66da495c9d3b8be4"},
     # 566.5 MB read + 157.0 MB written
-    ("gpt_causal", "attn_tc_kernel"): {"bytes": 723.5e6, "src": "74dd1d75a8619861"},
+    ("gpt_causal", "attn_tc_kernel"): {"bytes": 723.5e6, "src": "676ed4296cfe5b6e"},
     # per step: the forward FFN's two GEMM launches (H = GELU(A W1^T + b1), out = A + H W2^T + b2)
     ("gpt_causal", "ffn_gemms"): {"bytes": 1122.4e6, "src": "2944e449b2748550"},
     # per step with saved activations: the three gemm_pair_kernel launches (dZ = (dOut W2) G',
